@@ -1,0 +1,333 @@
+"""fp64 CPU oracle for one forward + backward training step of the GPT.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check in
+``__graft_entry__`` and the ``cpu_baseline`` / reference arm of ``bench.py``
+may import this module.  The CUDA library never calls it, and it never calls
+the CUDA library: the two share no code.  Inputs come from ``synth`` (seeded
+generators, no model arithmetic).
+
+What is computed, and where it comes from
+-----------------------------------------
+"ChatGPT'nizi 50 Dolara Nasil Egitirsiniz?" (dev.to), section "1. GPT Modeli
+(nanochat/gpt.py)", lists the model's ingredients: rotary embeddings, QK
+normalisation, untied embedding and output weights, the ReLU^2 activation
+(plus GQA, sliding windows and Flash Attention 3, which change nothing in
+exact arithmetic for the full-causal, n_kv = n_head shapes used here).
+Section "3. Hassasiyet Yonetimi (nanochat/common.py)" shows every linear layer
+as ``F.linear(x, W)`` with W stored [out, in] and no bias.  Section "5. Flash
+Dikkat Mekanizmasi Birlesimi" calls the attention with ``causal=True``.  The
+norm is parameter-free RMSNorm and the loss is the mean next-token
+cross-entropy in fp32 or better.
+
+Where the pages are silent the plainest reading is taken:
+
+* pre-norm blocks (norm before attention and before the MLP), one final norm
+  before lm_head, no norm directly after the embedding;
+* RMSNorm y = x / sqrt(mean(x^2) + eps), eps = 1e-6, no weight;
+* RoPE on q and k with half-split pairs (i, i + hd/2), angle t * base^(-2i/hd),
+  (a, b) -> (a cos - b sin, a sin + b cos), positions 0..T-1 per sequence;
+* QK norm = the same parameter-free RMSNorm over each head's hd entries,
+  applied after RoPE (a rotation keeps the norm, so the order does not change
+  the result in exact arithmetic);
+* attention scale 1/sqrt(hd), no dropout, no soft-capping;
+* MLP u = h W_up^T, a = max(u, 0)^2, y = a W_down^T (not gated);
+* loss = mean over all B*T positions of logsumexp(z) - z[target].
+
+Layout conventions shared with the library's documented ABI (not its code):
+W_qkv is [3d, d] with the q rows first, then k, then v; inside each block head
+h owns rows [h*hd, (h+1)*hd).
+
+The backward pass is derived by hand from the forward above; each step names
+the forward step it inverts.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Dict, Optional, Sequence
+
+import numpy as np
+
+__all__ = [
+    "OracleConfig",
+    "from_workload",
+    "rms_norm",
+    "rms_norm_backward",
+    "rope_tables",
+    "rope",
+    "rope_backward",
+    "causal_attention",
+    "causal_attention_backward",
+    "cross_entropy",
+    "sequence_forward",
+    "sequence_backward",
+    "step",
+    "StepResult",
+]
+
+
+@dataclasses.dataclass(frozen=True)
+class OracleConfig:
+    n_layer: int
+    d_model: int
+    n_head: int
+    head_dim: int
+    d_ff: int
+    vocab: int
+    seq_len: int
+    batch: int
+    norm_eps: float = 1e-6
+    rope_base: float = 10000.0
+    qk_norm: bool = True
+
+
+def from_workload(w) -> OracleConfig:
+    return OracleConfig(
+        n_layer=w.n_layer, d_model=w.d_model, n_head=w.n_head, head_dim=w.head_dim,
+        d_ff=w.d_ff, vocab=w.vocab, seq_len=w.seq_len, batch=w.batch,
+        norm_eps=w.norm_eps, rope_base=w.rope_base, qk_norm=w.qk_norm)
+
+
+# ---------------------------------------------------------------------------
+# building blocks
+# ---------------------------------------------------------------------------
+
+def rms_norm(x: np.ndarray, eps: float):
+    """Parameter-free RMSNorm over the last axis.
+
+    Returns (y, r) with r = 1/sqrt(mean(x^2) + eps) (one per row) and y = x*r.
+    """
+    r = 1.0 / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    return x * r, r
+
+
+def rms_norm_backward(dy: np.ndarray, y: np.ndarray, r: np.ndarray) -> np.ndarray:
+    """Inverse of ``rms_norm``: dx = r * (dy - y * mean(dy * y)).
+
+    From y_i = x_i r with dr/dx_j = -r^3 x_j / n.
+    """
+    return r * (dy - y * np.mean(dy * y, axis=-1, keepdims=True))
+
+
+def rope_tables(seq_len: int, head_dim: int, base: float):
+    """cos/sin of t * base^(-2i/hd) for t < seq_len, i < hd/2, shape [T, hd/2]."""
+    half = head_dim // 2
+    i = np.arange(half, dtype=np.float64)
+    theta = base ** (-2.0 * i / head_dim)
+    ang = np.arange(seq_len, dtype=np.float64)[:, None] * theta[None, :]
+    return np.cos(ang), np.sin(ang)
+
+
+def rope(x: np.ndarray, cos: np.ndarray, sin: np.ndarray) -> np.ndarray:
+    """Rotate each (x[i], x[i+hd/2]) pair of x [T, H, hd] by the position's angle."""
+    half = x.shape[-1] // 2
+    a, b = x[..., :half], x[..., half:]
+    c, s = cos[:, None, :], sin[:, None, :]
+    return np.concatenate([a * c - b * s, a * s + b * c], axis=-1)
+
+
+def rope_backward(dy: np.ndarray, cos: np.ndarray, sin: np.ndarray) -> np.ndarray:
+    """Transpose of the rotation in ``rope`` (rotation by the negative angle)."""
+    half = dy.shape[-1] // 2
+    da, db = dy[..., :half], dy[..., half:]
+    c, s = cos[:, None, :], sin[:, None, :]
+    return np.concatenate([da * c + db * s, -da * s + db * c], axis=-1)
+
+
+def _heads_first(x: np.ndarray) -> np.ndarray:
+    """[T, H, hd] -> [H, T, hd]"""
+    return np.ascontiguousarray(x.transpose(1, 0, 2))
+
+
+def _causal_probs(q: np.ndarray, k: np.ndarray):
+    """Scores and probabilities for q, k [T, H, hd]; returns P [H, T, T] and lse [H, T]."""
+    T, H, hd = q.shape
+    s = (_heads_first(q) @ _heads_first(k).transpose(0, 2, 1)) / math.sqrt(hd)
+    future = np.triu(np.ones((T, T), dtype=bool), k=1)
+    s = np.where(future[None, :, :], -np.inf, s)
+    m = np.max(s, axis=-1, keepdims=True)
+    e = np.exp(s - m)
+    tot = np.sum(e, axis=-1, keepdims=True)
+    return e / tot, (m + np.log(tot))[..., 0]
+
+
+def causal_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray):
+    """softmax(q k^T / sqrt(hd) with j > i masked) v, per head.
+
+    q, k, v: [T, H, hd].  Returns o [T, H, hd], the probabilities P [H, T, T]
+    and the row log-sum-exp [H, T] of the scaled, masked scores.
+    """
+    p, lse = _causal_probs(q, k)
+    o = (p @ _heads_first(v)).transpose(1, 0, 2)
+    return o, p, lse
+
+
+def causal_attention_backward(do, q, k, v, p):
+    """Gradients of ``causal_attention`` w.r.t. q, k, v given dO and P.
+
+    dV = P^T dO;  dP = dO V^T;  dS = P * (dP - rowsum(dP * P));
+    dQ = dS K / sqrt(hd);  dK = dS^T Q / sqrt(hd).
+    """
+    hd = q.shape[-1]
+    do_h, q_h, k_h, v_h = (_heads_first(t) for t in (do, q, k, v))
+    dv = p.transpose(0, 2, 1) @ do_h
+    dp = do_h @ v_h.transpose(0, 2, 1)
+    ds = p * (dp - np.sum(dp * p, axis=-1, keepdims=True))
+    dq = (ds @ k_h) / math.sqrt(hd)
+    dk = (ds.transpose(0, 2, 1) @ q_h) / math.sqrt(hd)
+    back = lambda t: t.transpose(1, 0, 2)
+    return back(dq), back(dk), back(dv)
+
+
+def cross_entropy(z: np.ndarray, y: np.ndarray):
+    """Per-position loss logsumexp(z) - z[y] (max-shifted), plus lse and softmax."""
+    m = np.max(z, axis=-1, keepdims=True)
+    e = np.exp(z - m)
+    tot = np.sum(e, axis=-1, keepdims=True)
+    lse = (m + np.log(tot))[:, 0]
+    loss = lse - z[np.arange(z.shape[0]), y]
+    return loss, lse, e / tot
+
+
+# ---------------------------------------------------------------------------
+# one sequence
+# ---------------------------------------------------------------------------
+
+def _layer_params(params, l):
+    return (params[f"layers.{l}.wqkv"], params[f"layers.{l}.wo"],
+            params[f"layers.{l}.wup"], params[f"layers.{l}.wdown"])
+
+
+def sequence_forward(cfg: OracleConfig, params: Dict[str, np.ndarray],
+                     tok: np.ndarray, tgt: np.ndarray) -> dict:
+    """Forward pass of one sequence (tok, tgt: int [T]); returns a cache dict.
+
+    The cache holds what the backward needs plus the per-position loss
+    (``token_loss``), the final logits' lse, and per-layer intermediates.
+    """
+    T = tok.shape[0]
+    d, H, hd = cfg.d_model, cfg.n_head, cfg.head_dim
+    eps = cfg.norm_eps
+    cos, sin = rope_tables(T, hd, cfg.rope_base)
+
+    x = params["wte"][tok].astype(np.float64)           # token embedding gather
+    layers = []
+    for l in range(cfg.n_layer):
+        wqkv, wo, wup, wdown = _layer_params(params, l)
+        c = {"x_in": x}
+        h, r1 = rms_norm(x, eps)                         # pre-attention norm
+        qkv = h @ wqkv.T                                 # F.linear, no bias
+        q = qkv[:, :d].reshape(T, H, hd)
+        k = qkv[:, d:2 * d].reshape(T, H, hd)
+        v = qkv[:, 2 * d:].reshape(T, H, hd)
+        q = rope(q, cos, sin)
+        k = rope(k, cos, sin)
+        if cfg.qk_norm:
+            qn, rq = rms_norm(q, eps)
+            kn, rk = rms_norm(k, eps)
+        else:
+            qn, rq, kn, rk = q, None, k, None
+        o, p, lse = causal_attention(qn, kn, v)
+        o2 = o.reshape(T, d)
+        x = x + o2 @ wo.T                                # attention residual
+        h2, r2 = rms_norm(x, eps)                        # pre-MLP norm
+        u = h2 @ wup.T
+        a = np.maximum(u, 0.0) ** 2                      # ReLU^2
+        x = x + a @ wdown.T                              # MLP residual
+        c.update(h=h, r1=r1, q=q, k=k, qn=qn, kn=kn, rq=rq, rk=rk, v=v, o=o2,
+                 lse=lse, x_mid=x - a @ wdown.T, h2=h2, r2=r2, u=u, a=a)
+        layers.append(c)
+
+    hf, rf = rms_norm(x, eps)                            # final norm
+    z = hf @ params["lm_head"].T                         # untied lm_head
+    loss_t, lse_z, probs = cross_entropy(z, tgt)
+    return {"tok": tok, "tgt": tgt, "layers": layers, "x_out": x, "hf": hf,
+            "rf": rf, "z": z, "probs": probs, "lse_z": lse_z, "token_loss": loss_t,
+            "cos": cos, "sin": sin}
+
+
+def sequence_backward(cfg: OracleConfig, params: Dict[str, np.ndarray], cache: dict,
+                      scale: float, grads: Dict[str, np.ndarray]) -> None:
+    """Accumulate d(scale * sum_t loss_t)/d(params) into ``grads``."""
+    tok, tgt = cache["tok"], cache["tgt"]
+    T = tok.shape[0]
+    d, H, hd = cfg.d_model, cfg.n_head, cfg.head_dim
+    cos, sin = cache["cos"], cache["sin"]
+
+    g = cache["probs"].copy()                            # d loss / d z
+    g[np.arange(T), tgt] -= 1.0
+    g *= scale
+    grads["lm_head"] += g.T @ cache["hf"]
+    dhf = g @ params["lm_head"]
+    dx = rms_norm_backward(dhf, cache["hf"], cache["rf"])
+
+    for l in reversed(range(cfg.n_layer)):
+        wqkv, wo, wup, wdown = _layer_params(params, l)
+        c = cache["layers"][l]
+        # x_out = x_mid + a W_down^T
+        grads[f"layers.{l}.wdown"] += dx.T @ c["a"]
+        da = dx @ wdown
+        du = da * 2.0 * np.maximum(c["u"], 0.0)
+        grads[f"layers.{l}.wup"] += du.T @ c["h2"]
+        dh2 = du @ wup
+        dx = dx + rms_norm_backward(dh2, c["h2"], c["r2"])
+        # x_mid = x_in + o W_o^T
+        grads[f"layers.{l}.wo"] += dx.T @ c["o"]
+        do = (dx @ wo).reshape(T, H, hd)
+        _, p, _ = causal_attention(c["qn"], c["kn"], c["v"])
+        dqn, dkn, dv = causal_attention_backward(do, c["qn"], c["kn"], c["v"], p)
+        if cfg.qk_norm:
+            dq = rms_norm_backward(dqn, c["qn"], c["rq"])
+            dk = rms_norm_backward(dkn, c["kn"], c["rk"])
+        else:
+            dq, dk = dqn, dkn
+        dq = rope_backward(dq, cos, sin)
+        dk = rope_backward(dk, cos, sin)
+        dqkv = np.concatenate([dq.reshape(T, d), dk.reshape(T, d), dv.reshape(T, d)], axis=1)
+        grads[f"layers.{l}.wqkv"] += dqkv.T @ c["h"]
+        dh = dqkv @ wqkv
+        dx = dx + rms_norm_backward(dh, c["h"], c["r1"])
+
+    np.add.at(grads["wte"], tok, dx)                     # embedding scatter-add
+
+
+# ---------------------------------------------------------------------------
+# the whole step
+# ---------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class StepResult:
+    loss: float
+    token_loss: np.ndarray                 # [B, T] (only the rows that were run)
+    grads: Optional[Dict[str, np.ndarray]]
+    caches: Optional[list] = None
+
+
+def step(cfg: OracleConfig, params: Dict[str, np.ndarray], tokens: np.ndarray,
+         targets: np.ndarray, *, backward: bool = True, keep_caches: bool = False,
+         rows: Optional[Sequence[int]] = None, loss_denominator: Optional[int] = None
+         ) -> StepResult:
+    """Loss = mean over all B*T positions; gradients of that loss.
+
+    Sequences are independent, so they are run one at a time and their
+    gradient contributions summed.  ``rows`` restricts the run to some
+    sequences (their token losses, and their share of the gradient with the
+    full batch's 1/(B*T) factor); ``loss_denominator`` overrides B*T.
+    """
+    B, T = tokens.shape
+    denom = loss_denominator if loss_denominator is not None else B * T
+    rows = list(range(B)) if rows is None else list(rows)
+    grads = None
+    if backward:
+        grads = {name: np.zeros_like(p, dtype=np.float64) for name, p in params.items()}
+    token_loss = np.zeros((len(rows), T))
+    caches = [] if keep_caches else None
+    for i, b in enumerate(rows):
+        cache = sequence_forward(cfg, params, tokens[b], targets[b])
+        token_loss[i] = cache["token_loss"]
+        if backward:
+            sequence_backward(cfg, params, cache, 1.0 / denom, grads)
+        if keep_caches:
+            caches.append(cache)
+    loss = float(np.sum(token_loss) / denom)
+    return StepResult(loss=loss, token_loss=token_loss, grads=grads, caches=caches)
