@@ -1,0 +1,469 @@
+// libgpt C ABI: configuration, parameter / workspace layout and the step
+// orchestration (which kernel runs when, on which buffers).  Every numeric
+// step runs in the CUDA kernels of this directory; this file only enqueues.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+
+#include "gpt_internal.h"
+
+namespace gpt {
+namespace {
+
+constexpr uint64_t kAlign = 256;
+
+uint64_t align_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
+
+struct Bump {
+  uint64_t off = 0;
+  uint64_t take(uint64_t bytes) {
+    off = align_up(off, kAlign);
+    uint64_t o = off;
+    off += bytes;
+    return o;
+  }
+};
+
+int64_t param_elems_aligned(int64_t n) { return (n + 127) / 128 * 128; }
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int cuda_rc(cudaError_t e) { return e == cudaSuccess ? GPT_OK : GPT_ECUDA; }
+
+#define GPT_TRY(expr)                           \
+  do {                                          \
+    int rc_ = (expr);                           \
+    if (rc_ != 0) return rc_ > 0 ? GPT_ECUDA : rc_; \
+  } while (0)
+
+}  // namespace
+
+bool make_layout(const gpt_config& c, Layout* L) {
+  const int64_t N = int64_t(c.batch) * c.seq_len;
+  const int64_t d = c.d_model, F = c.d_ff, V = c.vocab, H = c.n_head, T = c.seq_len,
+                B = c.batch, hd = c.head_dim;
+  const int esz = c.dtype == GPT_BF16 ? 2 : 4;
+  L->N = N;
+  L->esz = esz;
+  L->vpad = (V + 255) / 256 * 256;
+  Bump b;
+  L->status = b.take(sizeof(gpt_device_status) < 256 ? 256 : sizeof(gpt_device_status));
+  L->tok_stage = b.take(N * 4);
+  L->tgt_stage = b.take(N * 4);
+  L->rope_cos = b.take(T * (hd / 2) * 4);
+  L->rope_sin = b.take(T * (hd / 2) * 4);
+  L->x = b.take(N * d * 4);
+  L->dxs = b.take(N * d * esz);
+  // one layer's saved activations
+  Bump lb;
+  L->lo.h1 = lb.take(N * d * esz);
+  L->lo.r1 = lb.take(N * 4);
+  L->lo.q = lb.take(N * d * esz);
+  L->lo.k = lb.take(N * d * esz);
+  L->lo.v = lb.take(N * d * esz);
+  L->lo.rq = lb.take(B * H * T * 4);
+  L->lo.rk = lb.take(B * H * T * 4);
+  L->lo.o = lb.take(N * d * esz);
+  L->lo.lse = lb.take(B * H * T * 4);
+  L->lo.h2 = lb.take(N * d * esz);
+  L->lo.r2 = lb.take(N * 4);
+  L->lo.a = lb.take(N * F * esz);
+  L->layer_stride = align_up(lb.off, kAlign);
+  L->layer_base = b.take(L->layer_stride * uint64_t(c.n_layer));
+  L->hf = b.take(N * d * esz);
+  L->rf = b.take(N * 4);
+  L->qkv_raw = b.take(N * 3 * d * esz);
+  // cross-entropy partials: the narrowest GEMM tile used for the logits is 64 columns
+  L->n_part_max = (V + 63) / 64;
+  L->part_max = b.take(N * L->n_part_max * 4);
+  L->part_sum = b.take(N * L->n_part_max * 4);
+  L->tgt_logit = b.take(N * 4);
+  L->lse_z = b.take(N * 4);
+  L->tok_loss = b.take(N * 4);
+  L->loss_acc = b.take(256);
+  L->G = b.take(N * L->vpad * esz);
+  L->dh = b.take(N * d * esz);
+  L->du = b.take(N * F * esz);
+  L->dO = b.take(N * d * esz);
+  L->dqkv = b.take(N * 3 * d * esz);
+  L->Dattn = b.take(B * H * T * 4);
+  // deterministic embedding scatter
+  L->sort_tiles = (N + 1023) / 1024;
+  L->sort_perm = b.take(N * 4);
+  L->sort_offs = b.take((V + 1) * 4);
+  L->sort_count = b.take((V + 1) * 4);
+  L->sort_tilehist = b.take(L->sort_tiles * V * 4);
+  L->scat_max_items = N / 64 + V + 1;
+  L->scat_items = b.take(L->scat_max_items * 8);
+  L->scat_item_offs = b.take((V + 1) * 8);
+  L->scat_partial = b.take((N / 64 + 1) * d * 4 * 2);
+  L->total = align_up(b.off, kAlign);
+  return true;
+}
+
+}  // namespace gpt
+
+using namespace gpt;
+
+extern "C" {
+
+const char* gpt_version(void) { return "libgpt 0.1 (sm_100a)"; }
+
+const char* gpt_strerror(int code) {
+  switch (code) {
+    case GPT_OK: return "ok";
+    case GPT_EINVAL: return "invalid argument (null, misaligned or inconsistent)";
+    case GPT_EUNSUPPORTED: return "unsupported shape or dtype";
+    case GPT_ECUDA: return "CUDA call failed";
+    case GPT_EDATA: return "token or target id outside [0, vocab)";
+    case GPT_ETIMEOUT: return "bounded device wait expired";
+    case GPT_ENONFINITE: return "loss is not finite";
+    default: return "unknown error code";
+  }
+}
+
+int gpt_config_init(gpt_config* c) {
+  if (!c) return GPT_EINVAL;
+  if (c->rope_base == 0.f) c->rope_base = 10000.f;
+  if (c->norm_eps == 0.f) c->norm_eps = 1e-6f;
+  if (c->n_layer < 0 || c->d_model <= 0 || c->n_head <= 0 || c->head_dim <= 0 ||
+      c->d_ff <= 0 || c->vocab < 2 || c->seq_len <= 0 || c->batch <= 0)
+    return GPT_EINVAL;
+  if (int64_t(c->n_head) * c->head_dim != c->d_model) return GPT_EINVAL;
+  if (!(c->rope_base > 1.f) || !(c->norm_eps > 0.f) || !std::isfinite(c->rope_base) ||
+      !std::isfinite(c->norm_eps))
+    return GPT_EINVAL;
+  if (c->qk_norm != 0 && c->qk_norm != 1) return GPT_EINVAL;
+  if (c->dtype == GPT_BF16) {
+    if (c->d_model % 64 || c->d_ff % 64) return GPT_EUNSUPPORTED;
+    if (c->head_dim != 64 && c->head_dim != 128) return GPT_EUNSUPPORTED;
+  } else if (c->dtype == GPT_F32) {
+    if (c->head_dim % 2 || c->head_dim > 128) return GPT_EUNSUPPORTED;
+    if (c->seq_len > 4096) return GPT_EUNSUPPORTED;
+  } else {
+    return GPT_EINVAL;
+  }
+  const int64_t N = int64_t(c->batch) * c->seq_len;
+  if (N > (int64_t(1) << 31) / 4 || int64_t(c->vocab) > (int64_t(1) << 24)) return GPT_EUNSUPPORTED;
+  const int64_t d = c->d_model, F = c->d_ff, V = c->vocab;
+  int64_t n = 2 * V * d + int64_t(c->n_layer) * (3 * d * d + d * d + 2 * F * d);
+  c->n_params = n;
+  int64_t elems = 2 * param_elems_aligned(V * d) +
+                  int64_t(c->n_layer) * (param_elems_aligned(3 * d * d) + param_elems_aligned(d * d) +
+                                         2 * param_elems_aligned(F * d));
+  c->param_bytes = uint64_t(elems) * (c->dtype == GPT_BF16 ? 2 : 4);
+  Layout L;
+  make_layout(*c, &L);
+  c->workspace_bytes = L.total;
+  return GPT_OK;
+}
+
+int gpt_config_from_depth(gpt_config* c, int depth, int seq_len, int batch, int vocab) {
+  if (!c || depth < 2 || depth % 2) return GPT_EINVAL;
+  std::memset(c, 0, sizeof(*c));
+  c->n_layer = depth;
+  c->d_model = 64 * depth;
+  c->head_dim = 128;
+  c->n_head = c->d_model / 128;
+  c->d_ff = 4 * c->d_model;
+  c->vocab = vocab;
+  c->seq_len = seq_len;
+  c->batch = batch;
+  c->dtype = GPT_BF16;
+  c->qk_norm = 1;
+  c->rope_base = 10000.f;
+  c->norm_eps = 1e-6f;
+  return gpt_config_init(c);
+}
+
+int gpt_param_offset(const gpt_config* c, int tensor, int layer, int64_t* off, int64_t* rows,
+                     int64_t* cols) {
+  if (!c || !off || !rows || !cols) return GPT_EINVAL;
+  const int64_t d = c->d_model, F = c->d_ff, V = c->vocab;
+  const bool per_layer = tensor >= GPT_T_WQKV && tensor <= GPT_T_WDOWN;
+  if (tensor < GPT_T_WTE || tensor > GPT_T_LM_HEAD) return GPT_EINVAL;
+  if (per_layer && (layer < 0 || layer >= c->n_layer)) return GPT_EINVAL;
+  const int64_t lsz = param_elems_aligned(3 * d * d) + param_elems_aligned(d * d) +
+                      2 * param_elems_aligned(F * d);
+  const int64_t base = param_elems_aligned(V * d);
+  switch (tensor) {
+    case GPT_T_WTE: *off = 0; *rows = V; *cols = d; break;
+    case GPT_T_WQKV: *off = base + layer * lsz; *rows = 3 * d; *cols = d; break;
+    case GPT_T_WO:
+      *off = base + layer * lsz + param_elems_aligned(3 * d * d); *rows = d; *cols = d; break;
+    case GPT_T_WUP:
+      *off = base + layer * lsz + param_elems_aligned(3 * d * d) + param_elems_aligned(d * d);
+      *rows = F; *cols = d; break;
+    case GPT_T_WDOWN:
+      *off = base + layer * lsz + param_elems_aligned(3 * d * d) + param_elems_aligned(d * d) +
+             param_elems_aligned(F * d);
+      *rows = d; *cols = F; break;
+    case GPT_T_LM_HEAD: *off = base + int64_t(c->n_layer) * lsz; *rows = V; *cols = d; break;
+  }
+  return GPT_OK;
+}
+
+int gpt_workspace_region(const gpt_config* c, int region, int layer, uint64_t* off,
+                         uint64_t* bytes) {
+  if (!c || !off || !bytes) return GPT_EINVAL;
+  Layout L;
+  make_layout(*c, &L);
+  const uint64_t N = L.N, d = c->d_model, V = c->vocab;
+  switch (region) {
+    case GPT_W_STATUS: *off = L.status; *bytes = sizeof(gpt_device_status); break;
+    case GPT_W_RESID: *off = L.x; *bytes = N * d * 4; break;
+    case GPT_W_LSE: *off = L.lse_z; *bytes = N * 4; break;
+    case GPT_W_SORT_PERM: *off = L.sort_perm; *bytes = N * 4; break;
+    case GPT_W_SORT_OFFS: *off = L.sort_offs; *bytes = (V + 1) * 4; break;
+    case GPT_W_ATTN_LSE:
+      if (layer < 0 || layer >= c->n_layer) return GPT_EINVAL;
+      *off = L.layer_base + L.layer_stride * layer + L.lo.lse;
+      *bytes = uint64_t(c->batch) * c->n_head * c->seq_len * 4;
+      break;
+    default: return GPT_EINVAL;
+  }
+  return GPT_OK;
+}
+
+static int check_common(const gpt_config* c, const int32_t* tok, const int32_t* tgt,
+                        const void* params, void* ws) {
+  if (!c || !tok || !tgt || !params || !ws) return GPT_EINVAL;
+  gpt_config chk = *c;
+  int rc = gpt_config_init(&chk);
+  if (rc != GPT_OK) return rc;
+  if (chk.param_bytes != c->param_bytes || chk.workspace_bytes != c->workspace_bytes)
+    return GPT_EINVAL;  // derived fields stale: call gpt_config_init again
+  if (!aligned(tok, 16) || !aligned(tgt, 16) || !aligned(params, 256) || !aligned(ws, 256))
+    return GPT_EINVAL;
+  return GPT_OK;
+}
+
+struct Bufs {
+  char* ws;
+  const char* p;
+  Layout L;
+  int esz;
+  const gpt_config* c;
+  char* layer(int l) const { return ws + L.layer_base + L.layer_stride * uint64_t(l); }
+  const void* param(int t, int l) const {
+    int64_t off, r, cc;
+    gpt_param_offset(c, t, l, &off, &r, &cc);
+    return p + off * esz;
+  }
+};
+
+static GemmArgs gemm_kk(const void* A, int64_t lda, const void* B, int64_t ldb, int M, int N,
+                        int K, Epilogue epi, void* out, int64_t ldo) {
+  GemmArgs g{};
+  g.A = A; g.B = B; g.lda = lda; g.ldb = ldb;
+  g.a_mn_major = false; g.b_mn_major = false;
+  g.M = M; g.N = N; g.K = K; g.epi = epi; g.out = out; g.ldo = ldo;
+  return g;
+}
+
+int gpt_forward_loss(const gpt_config* c, const int32_t* tok, const int32_t* tgt,
+                     const void* params, void* workspace, float* loss, float* token_loss,
+                     void* stream) {
+  int rc = check_common(c, tok, tgt, params, workspace);
+  if (rc) return rc;
+  if (!loss || !aligned(loss, 4) || (token_loss && !aligned(token_loss, 4))) return GPT_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Bufs b{static_cast<char*>(workspace), static_cast<const char*>(params), {}, 0, c};
+  make_layout(*c, &b.L);
+  b.esz = b.L.esz;
+  const Layout& L = b.L;
+  const int N = int(L.N), d = c->d_model, F = c->d_ff, V = c->vocab;
+  char* ws = b.ws;
+  int32_t* status = reinterpret_cast<int32_t*>(ws + L.status);
+  float* cos_t = reinterpret_cast<float*>(ws + L.rope_cos);
+  float* sin_t = reinterpret_cast<float*>(ws + L.rope_sin);
+  float* x = reinterpret_cast<float*>(ws + L.x);
+
+  GPT_TRY(cuda_rc(cudaMemsetAsync(ws + L.status, 0, 256, st)));
+  GPT_TRY(launch_rope_table(*c, cos_t, sin_t, st));
+  {
+    void* h0 = c->n_layer > 0 ? (void*)(b.layer(0) + L.lo.h1) : (void*)(ws + L.hf);
+    float* r0 = reinterpret_cast<float*>(c->n_layer > 0 ? b.layer(0) + L.lo.r1 : ws + L.rf);
+    GPT_TRY(launch_embed_norm(*c, tok, b.param(GPT_T_WTE, 0), x, h0, r0, status, st));
+  }
+  for (int l = 0; l < c->n_layer; ++l) {
+    char* Lb = b.layer(l);
+    GemmArgs g = gemm_kk(Lb + L.lo.h1, d, b.param(GPT_T_WQKV, l), d, N, 3 * d, d, EPI_STORE,
+                         ws + L.qkv_raw, 3 * d);
+    g.status = status;
+    GPT_TRY(launch_gemm(*c, g, st));
+    GPT_TRY(launch_qkv_post(*c, ws + L.qkv_raw, cos_t, sin_t, Lb + L.lo.q, Lb + L.lo.k,
+                            Lb + L.lo.v, reinterpret_cast<float*>(Lb + L.lo.rq),
+                            reinterpret_cast<float*>(Lb + L.lo.rk), st));
+    GPT_TRY(launch_attn_fwd(*c, Lb + L.lo.q, Lb + L.lo.k, Lb + L.lo.v, Lb + L.lo.o,
+                            reinterpret_cast<float*>(Lb + L.lo.lse), st));
+    g = gemm_kk(Lb + L.lo.o, d, b.param(GPT_T_WO, l), d, N, d, d, EPI_RESID_F32, x, d);
+    g.status = status;
+    GPT_TRY(launch_gemm(*c, g, st));
+    GPT_TRY(launch_rms_fwd(*c, x, Lb + L.lo.h2, reinterpret_cast<float*>(Lb + L.lo.r2), st));
+    g = gemm_kk(Lb + L.lo.h2, d, b.param(GPT_T_WUP, l), d, N, F, d, EPI_RELU2, Lb + L.lo.a, F);
+    g.status = status;
+    GPT_TRY(launch_gemm(*c, g, st));
+    g = gemm_kk(Lb + L.lo.a, F, b.param(GPT_T_WDOWN, l), F, N, d, F, EPI_RESID_F32, x, d);
+    g.status = status;
+    GPT_TRY(launch_gemm(*c, g, st));
+    const bool last = l + 1 == c->n_layer;
+    void* hn = last ? (void*)(ws + L.hf) : (void*)(b.layer(l + 1) + L.lo.h1);
+    float* rn = reinterpret_cast<float*>(last ? ws + L.rf : b.layer(l + 1) + L.lo.r1);
+    GPT_TRY(launch_rms_fwd(*c, x, hn, rn, st));
+  }
+  // lm_head GEMM with the cross-entropy statistics in its epilogue
+  GemmArgs g = gemm_kk(ws + L.hf, d, b.param(GPT_T_LM_HEAD, 0), d, N, V, d, EPI_CE_FWD,
+                       nullptr, 0);
+  g.targets = tgt;
+  g.part_max = reinterpret_cast<float*>(ws + L.part_max);
+  g.part_sum = reinterpret_cast<float*>(ws + L.part_sum);
+  g.tgt_logit = reinterpret_cast<float*>(ws + L.tgt_logit);
+  g.n_valid = V;
+  g.status = status;
+  GPT_TRY(launch_gemm(*c, g, st));
+  const int tile_n = gemm_ce_tile_n(*c);
+  GPT_TRY(launch_ce_merge(*c, reinterpret_cast<float*>(ws + L.part_max),
+                          reinterpret_cast<float*>(ws + L.part_sum), (V + tile_n - 1) / tile_n,
+                          reinterpret_cast<float*>(ws + L.tgt_logit), tgt,
+                          reinterpret_cast<float*>(ws + L.lse_z),
+                          reinterpret_cast<float*>(ws + L.tok_loss), status, st));
+  GPT_TRY(launch_loss_mean(*c, reinterpret_cast<float*>(ws + L.tok_loss), loss, token_loss,
+                           status, st));
+  return GPT_OK;
+}
+
+int gpt_backward(const gpt_config* c, const int32_t* tok, const int32_t* tgt,
+                 const void* params, void* workspace, void* grads, int accumulate,
+                 void* stream) {
+  int rc = check_common(c, tok, tgt, params, workspace);
+  if (rc) return rc;
+  if (!grads || !aligned(grads, 256) || (accumulate != 0 && accumulate != 1)) return GPT_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Bufs b{static_cast<char*>(workspace), static_cast<const char*>(params), {}, 0, c};
+  make_layout(*c, &b.L);
+  b.esz = b.L.esz;
+  const Layout& L = b.L;
+  const int N = int(L.N), d = c->d_model, F = c->d_ff, V = c->vocab;
+  const int esz = L.esz;
+  char* ws = b.ws;
+  int32_t* status = reinterpret_cast<int32_t*>(ws + L.status);
+  float* cos_t = reinterpret_cast<float*>(ws + L.rope_cos);
+  float* sin_t = reinterpret_cast<float*>(ws + L.rope_sin);
+  float* dx = reinterpret_cast<float*>(ws + L.x);
+  char* gr = static_cast<char*>(grads);
+  auto grad = [&](int t, int l) -> void* {
+    int64_t off, r, cc;
+    gpt_param_offset(c, t, l, &off, &r, &cc);
+    return gr + off * esz;
+  };
+
+  GPT_TRY(launch_sort_tokens(*c, L, tok, ws, st));
+
+  // logits gradient G = (softmax(z) - onehot(target)) / N, recomputed from the saved lse
+  GemmArgs g = gemm_kk(ws + L.hf, d, b.param(GPT_T_LM_HEAD, 0), d, N, int(L.vpad), d,
+                       EPI_CE_BWD, ws + L.G, L.vpad);
+  g.targets = tgt;
+  g.lse = reinterpret_cast<float*>(ws + L.lse_z);
+  g.inv_n = 1.0f / float(N);
+  g.n_valid = V;
+  g.status = status;
+  GPT_TRY(launch_gemm(*c, g, st));
+  // dhf = G Wlm
+  g = gemm_kk(ws + L.G, L.vpad, b.param(GPT_T_LM_HEAD, 0), d, N, d, V, EPI_STORE, ws + L.dh, d);
+  g.b_mn_major = true;
+  g.status = status;
+  GPT_TRY(launch_gemm(*c, g, st));
+  // dWlm = G^T hf
+  g = gemm_kk(ws + L.G, L.vpad, ws + L.hf, d, V, d, N, EPI_STORE, grad(GPT_T_LM_HEAD, 0), d);
+  g.a_mn_major = true; g.b_mn_major = true; g.beta = accumulate;
+  g.status = status;
+  GPT_TRY(launch_gemm(*c, g, st));
+  GPT_TRY(launch_rms_bwd(*c, ws + L.dh, ws + L.hf, reinterpret_cast<float*>(ws + L.rf), dx,
+                         ws + L.dxs, 0, st));
+
+  for (int l = c->n_layer - 1; l >= 0; --l) {
+    char* Lb = b.layer(l);
+    // MLP down: da = dx Wdown, du = da * 2 relu(u) (from the stored a = relu(u)^2)
+    g = gemm_kk(ws + L.dxs, d, b.param(GPT_T_WDOWN, l), F, N, F, d, EPI_DRELU2, ws + L.du, F);
+    g.b_mn_major = true; g.aux = Lb + L.lo.a; g.status = status;
+    GPT_TRY(launch_gemm(*c, g, st));
+    g = gemm_kk(ws + L.dxs, d, Lb + L.lo.a, F, d, F, N, EPI_STORE, grad(GPT_T_WDOWN, l), F);
+    g.a_mn_major = true; g.b_mn_major = true; g.beta = accumulate; g.status = status;
+    GPT_TRY(launch_gemm(*c, g, st));
+    // MLP up
+    g = gemm_kk(ws + L.du, F, b.param(GPT_T_WUP, l), d, N, d, F, EPI_STORE, ws + L.dh, d);
+    g.b_mn_major = true; g.status = status;
+    GPT_TRY(launch_gemm(*c, g, st));
+    g = gemm_kk(ws + L.du, F, Lb + L.lo.h2, d, F, d, N, EPI_STORE, grad(GPT_T_WUP, l), d);
+    g.a_mn_major = true; g.b_mn_major = true; g.beta = accumulate; g.status = status;
+    GPT_TRY(launch_gemm(*c, g, st));
+    GPT_TRY(launch_rms_bwd(*c, ws + L.dh, Lb + L.lo.h2, reinterpret_cast<float*>(Lb + L.lo.r2),
+                           dx, ws + L.dxs, 1, st));
+    // attention out-projection
+    g = gemm_kk(ws + L.dxs, d, b.param(GPT_T_WO, l), d, N, d, d, EPI_STORE, ws + L.dO, d);
+    g.b_mn_major = true; g.status = status;
+    GPT_TRY(launch_gemm(*c, g, st));
+    g = gemm_kk(ws + L.dxs, d, Lb + L.lo.o, d, d, d, N, EPI_STORE, grad(GPT_T_WO, l), d);
+    g.a_mn_major = true; g.b_mn_major = true; g.beta = accumulate; g.status = status;
+    GPT_TRY(launch_gemm(*c, g, st));
+    // attention, then QK-norm and RoPE backward, into dqkv [N, 3d]
+    GPT_TRY(launch_attn_bwd(*c, Lb + L.lo.q, Lb + L.lo.k, Lb + L.lo.v, Lb + L.lo.o, ws + L.dO,
+                            reinterpret_cast<float*>(Lb + L.lo.lse),
+                            reinterpret_cast<float*>(Lb + L.lo.rq),
+                            reinterpret_cast<float*>(Lb + L.lo.rk), cos_t, sin_t,
+                            reinterpret_cast<float*>(ws + L.Dattn), ws + L.dqkv, st));
+    g = gemm_kk(ws + L.dqkv, 3 * d, b.param(GPT_T_WQKV, l), d, N, d, 3 * d, EPI_STORE,
+                ws + L.dh, d);
+    g.b_mn_major = true; g.status = status;
+    GPT_TRY(launch_gemm(*c, g, st));
+    g = gemm_kk(ws + L.dqkv, 3 * d, Lb + L.lo.h1, d, 3 * d, d, N, EPI_STORE,
+                grad(GPT_T_WQKV, l), d);
+    g.a_mn_major = true; g.b_mn_major = true; g.beta = accumulate; g.status = status;
+    GPT_TRY(launch_gemm(*c, g, st));
+    GPT_TRY(launch_rms_bwd(*c, ws + L.dh, Lb + L.lo.h1, reinterpret_cast<float*>(Lb + L.lo.r1),
+                           dx, ws + L.dxs, 1, st));
+  }
+  GPT_TRY(launch_embed_scatter(*c, L, dx, ws, grad(GPT_T_WTE, 0), accumulate, st));
+  return GPT_OK;
+}
+
+int gpt_train_step_host(const gpt_config* c, const int32_t* host_tokens,
+                        const int32_t* host_targets, const void* params, void* workspace,
+                        void* grads, int accumulate, float* host_loss, void* stream) {
+  if (!c || !host_tokens || !host_targets || !workspace || !host_loss) return GPT_EINVAL;
+  if (!aligned(workspace, 256)) return GPT_EINVAL;
+  Layout L;
+  make_layout(*c, &L);
+  char* ws = static_cast<char*>(workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t* dtok = reinterpret_cast<int32_t*>(ws + L.tok_stage);
+  int32_t* dtgt = reinterpret_cast<int32_t*>(ws + L.tgt_stage);
+  float* dloss = reinterpret_cast<float*>(ws + L.loss_acc);
+  const size_t nb = size_t(L.N) * 4;
+  if (cudaMemcpyAsync(dtok, host_tokens, nb, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return GPT_ECUDA;
+  if (cudaMemcpyAsync(dtgt, host_targets, nb, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return GPT_ECUDA;
+  int rc = gpt_forward_loss(c, dtok, dtgt, params, workspace, dloss, nullptr, stream);
+  if (rc) return rc;
+  rc = gpt_backward(c, dtok, dtgt, params, workspace, grads, accumulate, stream);
+  if (rc) return rc;
+  if (cudaMemcpyAsync(host_loss, dloss, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return GPT_ECUDA;
+  return GPT_OK;
+}
+
+int gpt_status(const void* workspace, void* stream) {
+  if (!workspace) return GPT_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return GPT_ECUDA;
+  gpt_device_status s;
+  if (cudaMemcpy(&s, workspace, sizeof(s), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return GPT_ECUDA;
+  return s.code;
+}
+
+}  // extern "C"

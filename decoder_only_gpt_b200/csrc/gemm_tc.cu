@@ -1,0 +1,442 @@
+// bf16 GEMM on the sm_100a tensor cores: C[m,n] = sum_k A(m,k) B(n,k), fp32
+// accumulation in tensor memory, with the fused epilogues of the step.
+//
+// Design (one CTA per SM, persistent over output tiles):
+//   tile 128 x 256, K-block 64 (one 128-byte swizzle atom), 4-stage smem ring;
+//   warp 0      TMA producer: A and B tiles -> smem, mbarrier complete_tx;
+//   warp 1      one thread issues tcgen05.mma (M=128, N=256, K=16) into one of
+//               two 256-column fp32 accumulators in TMEM (512 columns), and
+//               tcgen05.commit frees smem stages / hands accumulators over;
+//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time (thread = row),
+//               apply the epilogue, store to global.  Double-buffered TMEM
+//               lets the epilogue of tile i overlap the MMAs of tile i+1.
+// Either operand may be K-major (forward: X W^T) or MN-major (dgrad reads W
+// as stored, wgrad reads dY and X as stored), selected per operand through
+// the TMA box shape, the smem descriptor and the instruction descriptor.
+// Every wait is bounded (GPT_ETIMEOUT recorded in the status word).
+#include <cudaTypedefs.h>
+
+#include "epilogue.cuh"
+#include "tc_ptx.cuh"
+
+namespace gpt {
+
+namespace {
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int kThreads = 192;
+constexpr uint32_t A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2;
+constexpr uint32_t TMEM_COLS = 2 * BN;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+struct __align__(8) SmemTail {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tmem_full[2];
+  uint64_t tmem_empty[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort;
+};
+constexpr size_t kSmemBytes = 1024 /*align slack*/ + STAGES * (A_BYTES + B_BYTES) + sizeof(SmemTail);
+}  // namespace
+
+__device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
+  __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&u);
+  return __bfloat1622float2(h);
+}
+
+// Epilogue of 32 consecutive columns [col0, col0+32) of one row.
+__device__ __forceinline__ void epi_chunk(const GemmArgs& g, int row, int col0, float (&v)[32],
+                                          float& ce_max, float& ce_sum, float& ce_tgt,
+                                          int tgt, float lse_row) {
+  const bool full = col0 + 32 <= g.N;
+  const int64_t base = int64_t(row) * g.ldo + col0;
+  switch (g.epi) {
+    case EPI_CE_FWD: {
+      const int nv = min(32, g.n_valid - col0);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (j < nv) mx = fmaxf(mx, v[j]);
+      if (nv > 0) {
+        float nm = fmaxf(ce_max, mx);
+        float s = 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (j < nv) s += __expf(v[j] - nm);
+        ce_sum = ce_sum * __expf(ce_max - nm) + s;
+        ce_max = nm;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (col0 + j == tgt && j < nv) ce_tgt = v[j];
+      }
+      return;
+    }
+    case EPI_RESID_F32: {
+      float* o = static_cast<float*>(g.out) + base;
+      if (full) {
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+          float4 x = *reinterpret_cast<float4*>(o + j);
+          x.x += v[j]; x.y += v[j + 1]; x.z += v[j + 2]; x.w += v[j + 3];
+          *reinterpret_cast<float4*>(o + j) = x;
+        }
+      } else {
+        for (int j = 0; j < 32 && col0 + j < g.N; ++j) o[j] += v[j];
+      }
+      return;
+    }
+    case EPI_STORE_F32: {
+      float* o = static_cast<float*>(g.out) + base;
+      for (int j = 0; j < 32 && col0 + j < g.N; ++j) o[j] = v[j];
+      return;
+    }
+    default:
+      break;
+  }
+  // bf16 outputs
+  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(g.out) + base;
+  float r[32];
+  switch (g.epi) {
+    case EPI_STORE:
+      if (g.beta) {
+        if (full) {
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            uint4 u = *reinterpret_cast<const uint4*>(o + j);
+            float2 a = unpack_bf16(u.x), b = unpack_bf16(u.y), c = unpack_bf16(u.z),
+                   d = unpack_bf16(u.w);
+            r[j] = v[j] + a.x; r[j + 1] = v[j + 1] + a.y; r[j + 2] = v[j + 2] + b.x;
+            r[j + 3] = v[j + 3] + b.y; r[j + 4] = v[j + 4] + c.x; r[j + 5] = v[j + 5] + c.y;
+            r[j + 6] = v[j + 6] + d.x; r[j + 7] = v[j + 7] + d.y;
+          }
+        } else {
+          for (int j = 0; j < 32; ++j) r[j] = v[j] + (col0 + j < g.N ? __bfloat162float(o[j]) : 0.f);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) r[j] = v[j];
+      }
+      break;
+    case EPI_RELU2:
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        float t = fmaxf(v[j], 0.f);
+        r[j] = t * t;
+      }
+      break;
+    case EPI_DRELU2: {
+      const __nv_bfloat16* a = static_cast<const __nv_bfloat16*>(g.aux) + base;
+      if (full) {
+#pragma unroll
+        for (int j = 0; j < 32; j += 8) {
+          uint4 u = *reinterpret_cast<const uint4*>(a + j);
+          float2 p0 = unpack_bf16(u.x), p1 = unpack_bf16(u.y), p2 = unpack_bf16(u.z),
+                 p3 = unpack_bf16(u.w);
+          r[j] = v[j] * 2.f * sqrtf(p0.x); r[j + 1] = v[j + 1] * 2.f * sqrtf(p0.y);
+          r[j + 2] = v[j + 2] * 2.f * sqrtf(p1.x); r[j + 3] = v[j + 3] * 2.f * sqrtf(p1.y);
+          r[j + 4] = v[j + 4] * 2.f * sqrtf(p2.x); r[j + 5] = v[j + 5] * 2.f * sqrtf(p2.y);
+          r[j + 6] = v[j + 6] * 2.f * sqrtf(p3.x); r[j + 7] = v[j + 7] * 2.f * sqrtf(p3.y);
+        }
+      } else {
+        for (int j = 0; j < 32; ++j)
+          r[j] = col0 + j < g.N ? v[j] * 2.f * sqrtf(__bfloat162float(a[j])) : 0.f;
+      }
+      break;
+    }
+    case EPI_CE_BWD:
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int n = col0 + j;
+        float p = __expf(v[j] - lse_row);
+        r[j] = n < g.n_valid ? (p - (n == tgt ? 1.f : 0.f)) * g.inv_n : 0.f;
+      }
+      break;
+    default:
+#pragma unroll
+      for (int j = 0; j < 32; ++j) r[j] = v[j];
+      break;
+  }
+  if (full) {
+#pragma unroll
+    for (int j = 0; j < 32; j += 8) {
+      uint4 u;
+      u.x = pack_bf16(r[j], r[j + 1]);
+      u.y = pack_bf16(r[j + 2], r[j + 3]);
+      u.z = pack_bf16(r[j + 4], r[j + 5]);
+      u.w = pack_bf16(r[j + 6], r[j + 7]);
+      *reinterpret_cast<uint4*>(o + j) = u;
+    }
+  } else {
+    for (int j = 0; j < 32 && col0 + j < g.N; ++j) o[j] = __float2bfloat16_rn(r[j]);
+  }
+}
+
+template <bool AMN, bool BMN>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a,
+                   const __grid_constant__ CUtensorMap map_b, const __grid_constant__ GemmArgs g) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* smA = smem;
+  uint8_t* smB = smem + STAGES * A_BYTES;
+  SmemTail* tail = reinterpret_cast<SmemTail*>(smem + STAGES * (A_BYTES + B_BYTES));
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+  const int m_tiles = (g.M + BM - 1) / BM, n_tiles = (g.N + BN - 1) / BN;
+  const int num_tiles = m_tiles * n_tiles;
+  const int num_kb = (g.K + BK - 1) / BK;
+  constexpr uint32_t idesc = tc::idesc_bf16_f32(BM, BN, AMN, BMN);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      tc::mbar_init(&tail->full[s], 1);
+      tc::mbar_init(&tail->empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      tc::mbar_init(&tail->tmem_full[a], 1);
+      tc::mbar_init(&tail->tmem_empty[a], 128);
+    }
+    tc::mbar_init(&tail->mma_done, 1);
+    tail->abort = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&tail->tmem_base, TMEM_COLS);
+    tc::tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tc::tma_prefetch_desc(&map_a);
+    tc::tma_prefetch_desc(&map_b);
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem_base = tail->tmem_base;
+  volatile int* abort = &tail->abort;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, last_parity = 0;
+      for (int tile = blockIdx.x; tile < num_tiles && !*abort; tile += gridDim.x) {
+        const int mb = tile / n_tiles, nb = tile % n_tiles;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!tc::mbar_wait_bounded(&tail->empty[stage], phase ^ 1, abort, kWaitLimitNs)) {
+            record_status(g.status, GPT_ETIMEOUT, K_GEMM_TC, 1);
+            *abort = 1;
+            break;
+          }
+          tc::mbar_arrive_expect_tx(&tail->full[stage], A_BYTES + B_BYTES);
+          uint8_t* a_dst = smA + stage * A_BYTES;
+          uint8_t* b_dst = smB + stage * B_BYTES;
+          if (AMN) {
+            tc::tma_load_2d(a_dst, &map_a, &tail->full[stage], mb * BM, kb * BK);
+            tc::tma_load_2d(a_dst + 8192, &map_a, &tail->full[stage], mb * BM + 64, kb * BK);
+          } else {
+            tc::tma_load_2d(a_dst, &map_a, &tail->full[stage], kb * BK, mb * BM);
+          }
+          if (BMN) {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j)
+              tc::tma_load_2d(b_dst + j * 8192, &map_b, &tail->full[stage], nb * BN + 64 * j,
+                              kb * BK);
+          } else {
+            tc::tma_load_2d(b_dst, &map_b, &tail->full[stage], kb * BK, nb * BN);
+          }
+          issued_mask |= 1u << stage;
+          last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (*abort) {
+        // let every copy this thread started land before the CTA exits
+        for (int s = 0; s < STAGES; ++s)
+          if (issued_mask >> s & 1)
+            tc::mbar_wait_bounded(&tail->full[s], (last_parity >> s) & 1, nullptr, kWaitLimitNs);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool issued_any = false;
+      for (int tile = blockIdx.x; tile < num_tiles && !*abort; tile += gridDim.x, ++local) {
+        const int acc = local & 1;
+        const uint32_t acc_phase = (local >> 1) & 1;
+        if (!tc::mbar_wait_bounded(&tail->tmem_empty[acc], acc_phase ^ 1, abort, kWaitLimitNs)) {
+          record_status(g.status, GPT_ETIMEOUT, K_GEMM_TC, 2);
+          *abort = 1;
+          break;
+        }
+        tc::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!tc::mbar_wait_bounded(&tail->full[stage], phase, abort, kWaitLimitNs)) {
+            record_status(g.status, GPT_ETIMEOUT, K_GEMM_TC, 3);
+            *abort = 1;
+            break;
+          }
+          tc::tc_fence_after();
+          const uint32_t a_addr = tc::smem_u32(smA + stage * A_BYTES);
+          const uint32_t b_addr = tc::smem_u32(smB + stage * B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t da = AMN ? tc::smem_desc_sw128(a_addr + k * 2048, 8192)
+                                    : tc::smem_desc_sw128(a_addr + k * 32, 16);
+            const uint64_t db = BMN ? tc::smem_desc_sw128(b_addr + k * 2048, 8192)
+                                    : tc::smem_desc_sw128(b_addr + k * 32, 16);
+            tc::mma_bf16_ss(d_tmem, da, db, idesc, (kb | k) != 0);
+          }
+          issued_any = true;
+          tc::mma_commit(&tail->empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (*abort) break;
+        tc::mma_commit(&tail->tmem_full[acc]);
+      }
+      // all MMAs of this CTA complete before TMEM is released
+      if (issued_any) {
+        tc::mma_commit(&tail->mma_done);
+        tc::mbar_wait_bounded(&tail->mma_done, 0, nullptr, kWaitLimitNs);
+      }
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int quarter = warp & 3;  // TMEM lanes accessible to this warp
+    int local = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      const bool ok = tc::mbar_wait_bounded(&tail->tmem_full[acc], acc_phase, abort, kWaitLimitNs);
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) record_status(g.status, GPT_ETIMEOUT, K_GEMM_TC, 4);
+        *abort = 1;
+        break;
+      }
+      tc::tc_fence_after();
+      const int mb = tile / n_tiles, nb = tile % n_tiles;
+      const int row = mb * BM + quarter * 32 + lane;
+      const bool row_ok = row < g.M;
+      int tgt = -1;
+      float lse_row = 0.f;
+      if (row_ok && (g.epi == EPI_CE_FWD || g.epi == EPI_CE_BWD)) {
+        tgt = g.targets[row];
+        if (g.epi == EPI_CE_BWD) lse_row = g.lse[row];
+      }
+      float ce_max = -INFINITY, ce_sum = 0.f, ce_tgt = 0.f;
+      const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + acc * BN;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t u[32];
+        tc::tmem_ld_32x32b_x32(taddr + c * 32, u);
+        tc::tmem_wait_ld();
+        const int col0 = nb * BN + c * 32;
+        if (row_ok && col0 < g.N) {
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = u2f(u[j]);
+          epi_chunk(g, row, col0, v, ce_max, ce_sum, ce_tgt, tgt, lse_row);
+        }
+      }
+      if (row_ok && g.epi == EPI_CE_FWD) {
+        g.part_max[int64_t(row) * g.n_part + nb] = ce_max;
+        g.part_sum[int64_t(row) * g.n_part + nb] = ce_sum;
+        if (tgt >= nb * BN && tgt < nb * BN + BN && tgt < g.n_valid) g.tgt_logit[row] = ce_tgt;
+      }
+      tc::tc_fence_before();
+      tc::mbar_arrive(&tail->tmem_empty[acc]);
+    }
+  }
+
+  __syncwarp();
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;  // resolved once per process
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor [outer, inner] (inner contiguous, row pitch ld elements),
+// box [box_outer, box_inner], 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t ld,
+              uint32_t box_inner, uint32_t box_outer) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <bool AMN, bool BMN>
+int launch_tc(const GemmArgs& g, int grid, cudaStream_t st) {
+  CUtensorMap ma, mb;
+  bool ok = AMN ? make_map(&ma, g.A, g.M, g.K, g.lda, 64, 64)
+                : make_map(&ma, g.A, g.K, g.M, g.lda, 64, BM);
+  ok = ok && (BMN ? make_map(&mb, g.B, g.N, g.K, g.ldb, 64, 64)
+                  : make_map(&mb, g.B, g.K, g.N, g.ldb, 64, BN));
+  if (!ok) return 1;
+  auto kern = gemm_tc_kernel<AMN, BMN>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes)) !=
+      cudaSuccess)
+    return 1;
+  kern<<<grid, kThreads, kSmemBytes, st>>>(ma, mb, g);
+  return last_launch_rc();
+}
+
+}  // namespace
+
+int launch_gemm_tc(const GemmArgs& g_in, void* stream) {
+  GemmArgs g = g_in;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (g.M <= 0 || g.N <= 0 || g.K <= 0) return 0;
+  const int tiles = ((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN);
+  if (g.epi == EPI_CE_FWD) g.n_part = (g.N + BN - 1) / BN;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = tiles < sms ? tiles : sms;
+  if (!g.a_mn_major && !g.b_mn_major) return launch_tc<false, false>(g, grid, st);
+  if (!g.a_mn_major && g.b_mn_major) return launch_tc<false, true>(g, grid, st);
+  if (g.a_mn_major && g.b_mn_major) return launch_tc<true, true>(g, grid, st);
+  return launch_tc<true, false>(g, grid, st);
+}
+
+int gemm_tc_tile_n() { return BN; }
+
+}  // namespace gpt

@@ -1,0 +1,113 @@
+// Internal declarations of libgpt: workspace layout and kernel launchers.
+// Host-only C++ (no CUDA headers needed to include it).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include "gpt.h"
+
+namespace gpt {
+
+// Kernel ids recorded in gpt_device_status::where.
+enum KernelId : int32_t {
+  K_EMBED = 1,
+  K_CE_MERGE = 2,
+  K_GEMM_TC = 3,
+  K_ATTN = 4,
+  K_LOSS = 5,
+};
+
+// Epilogues of the GEMM C[m,n] = sum_k A(m,k) B(n,k).
+enum Epilogue : int32_t {
+  EPI_STORE = 0,    // out_t[m*ldo+n] = acc (+ out_t if beta)
+  EPI_STORE_F32,    // out_f32[m*ldo+n] = acc
+  EPI_RESID_F32,    // out_f32[m*ldo+n] += acc        (residual stream update)
+  EPI_RELU2,        // out_t = max(acc,0)^2           (MLP activation)
+  EPI_DRELU2,       // out_t = acc * 2*sqrt(aux_t)    (ReLU^2' from the stored activation)
+  EPI_CE_FWD,       // per-row partial (max, sum exp) over the tile's columns + target logit
+  EPI_CE_BWD,       // out_t = (exp(acc - lse[m]) - [n == tgt[m]]) * inv_n; 0 for n >= n_valid
+};
+
+struct GemmArgs {
+  // operands; element (m,k) of A is A[m*lda+k] if !a_mn_major else A[k*lda+m]
+  const void* A;
+  const void* B;
+  int64_t lda, ldb;
+  bool a_mn_major, b_mn_major;
+  int M, N, K;
+  // epilogue
+  Epilogue epi;
+  void* out;
+  int64_t ldo;
+  int beta;                 // EPI_STORE: 1 = accumulate into out
+  const void* aux;          // EPI_DRELU2: stored activation a, leading dim ldo
+  // cross-entropy epilogues
+  const int32_t* targets;   // [M]
+  float* part_max;          // [M, n_part]
+  float* part_sum;          // [M, n_part]
+  float* tgt_logit;         // [M]
+  const float* lse;         // [M]
+  int n_part;               // partial columns per row = ceil(N / tile_n)
+  float inv_n;
+  int n_valid;              // columns >= n_valid are padding (EPI_CE_BWD writes 0)
+  int32_t* status;          // device status word
+};
+
+struct LayerOffsets {
+  uint64_t h1, r1, q, k, v, rq, rk, o, lse, h2, r2, a;
+};
+
+// Byte offsets of every workspace region.  Computed from the config only.
+struct Layout {
+  int64_t N;               // batch * seq_len
+  int64_t vpad;            // vocab rounded up to 256 (row stride of the logit-gradient buffer)
+  int esz;                 // bytes per stored activation element (2 bf16, 4 f32)
+  uint64_t status, tok_stage, tgt_stage, rope_cos, rope_sin;
+  uint64_t x, dxs;
+  uint64_t layer_base, layer_stride;
+  LayerOffsets lo;         // offsets relative to the layer's base
+  uint64_t hf, rf;
+  uint64_t qkv_raw;
+  uint64_t part_max, part_sum, tgt_logit, lse_z, tok_loss, loss_acc;
+  uint64_t G, dh, du, dO, dqkv, Dattn;
+  uint64_t sort_perm, sort_offs, sort_count, sort_tilehist, scat_items, scat_item_offs,
+      scat_partial;
+  int64_t n_part_max;      // partial-stat columns reserved per row
+  int64_t sort_tiles;      // N / 1024 rounded up
+  int64_t scat_max_items;  // upper bound of (row, chunk) work items of the scatter
+  uint64_t total;
+};
+
+bool make_layout(const gpt_config& c, Layout* L);
+
+// ---- launchers (all enqueue on `stream`, return cudaError_t as int) ------
+int launch_rope_table(const gpt_config& c, float* cos_t, float* sin_t, void* stream);
+int launch_embed_norm(const gpt_config& c, const int32_t* tok, const void* wte, float* x,
+                      void* h, float* r, int32_t* status, void* stream);
+int launch_rms_fwd(const gpt_config& c, const float* x, void* h, float* r, void* stream);
+int launch_rms_bwd(const gpt_config& c, const void* dh, const void* h, const float* r,
+                   float* dx, void* dxs, int accumulate, void* stream);
+int launch_qkv_post(const gpt_config& c, const void* qkv_raw, const float* cos_t,
+                    const float* sin_t, void* q, void* k, void* v, float* rq, float* rk,
+                    void* stream);
+int launch_ce_merge(const gpt_config& c, const float* part_max, const float* part_sum,
+                    int n_part, const float* tgt_logit, const int32_t* targets, float* lse,
+                    float* tok_loss, int32_t* status, void* stream);
+int launch_loss_mean(const gpt_config& c, const float* tok_loss, float* loss,
+                     float* user_tok_loss, int32_t* status, void* stream);
+int launch_attn_fwd(const gpt_config& c, const void* q, const void* k, const void* v, void* o,
+                    float* lse, void* stream);
+int launch_attn_bwd(const gpt_config& c, const void* q, const void* k, const void* v,
+                    const void* o, const void* dO, const float* lse, const float* rq,
+                    const float* rk, const float* cos_t, const float* sin_t, float* Dbuf,
+                    void* dqkv, void* stream);
+int launch_sort_tokens(const gpt_config& c, const Layout& L, const int32_t* tok, char* ws,
+                       void* stream);
+int launch_embed_scatter(const gpt_config& c, const Layout& L, const float* dx0, char* ws,
+                         void* dwte, int accumulate, void* stream);
+int launch_gemm(const gpt_config& c, const GemmArgs& g, void* stream);
+// Column width of the GEMM tile that produces the logits (partial-statistics granularity).
+int gemm_ce_tile_n(const gpt_config& c);
+
+}  // namespace gpt

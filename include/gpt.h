@@ -1,0 +1,178 @@
+/*
+ * gpt.h -- C ABI of libgpt: one forward + backward training step of a
+ * pre-norm decoder-only GPT on one NVIDIA B200 (sm_100a).
+ *
+ * The model is the one sketched in "ChatGPT'nizi 50 Dolara Nasil
+ * Egitirsiniz?" (dev.to), section "1. GPT Modeli (nanochat/gpt.py)": rotary
+ * position embeddings, QK normalisation, untied token embedding and lm_head,
+ * ReLU^2 MLP, causal attention (section "5. Flash Dikkat Mekanizmasi
+ * Birlesimi", causal=True), bias-free linear layers (section "3. Hassasiyet
+ * Yonetimi", F.linear(x, W) with W stored [out, in]).  Width, heads and MLP
+ * size follow the depth dial of section "Felsefe: Her Seyi Kontrol Eden Tek
+ * Bir Kadran" (d_model = 64 * depth, head_dim 128, d_ff = 4 * d_model).
+ *
+ * Step, per sequence of T tokens (all norms parameter-free RMSNorm,
+ * y = x / sqrt(mean(x^2) + eps)):
+ *   x = wte[tokens]
+ *   per layer:  h = rms(x); [q|k|v] = h Wqkv^T; q,k <- rms_head(RoPE(q,k))
+ *               x += causal_softmax(q k^T / sqrt(hd)) v  Wo^T
+ *               h = rms(x); x += relu(h Wup^T)^2 Wdown^T
+ *   z = rms(x) Wlm^T;  loss = mean_t (logsumexp(z_t) - z_t[target_t])
+ * and the exact gradient of that loss w.r.t. every parameter.
+ *
+ * Conventions for every call below:
+ *  - All device buffers are owned by the caller; the library allocates no
+ *    device memory and keeps no global mutable state.  Pointers marked
+ *    "device" must be device memory of the current CUDA device.
+ *  - Device pointers must be 16-byte aligned (TMA); params/grads/workspace
+ *    256-byte aligned.  A violation returns GPT_EINVAL before any launch.
+ *  - Work is enqueued asynchronously on `stream` (a cudaStream_t, NULL = the
+ *    legacy default stream).  Results are deterministic: bit-identical
+ *    across runs for identical inputs (no floating-point atomics).
+ *  - Return value 0 on success, a negative GPT_E* code otherwise.  Errors
+ *    found on the device (bad token ids, an expired bounded wait, a
+ *    non-finite loss) are recorded in the workspace and read by gpt_status().
+ */
+#ifndef GPT_B200_H
+#define GPT_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- error codes ------------------------------------------------------ */
+#define GPT_OK 0
+#define GPT_EINVAL (-1)       /* null / misaligned pointer, inconsistent config */
+#define GPT_EUNSUPPORTED (-2) /* shape or dtype outside what the kernels cover  */
+#define GPT_ECUDA (-3)        /* a CUDA runtime / driver call failed            */
+#define GPT_EDATA (-4)        /* a token or target id outside [0, vocab)        */
+#define GPT_ETIMEOUT (-5)     /* a bounded device-side wait expired             */
+#define GPT_ENONFINITE (-6)   /* the loss came out NaN or Inf                   */
+
+/* ---- storage types ---------------------------------------------------- */
+#define GPT_BF16 0 /* bf16 params/activations/grads, fp32 accumulate (tensor cores) */
+#define GPT_F32 1  /* fp32 everywhere (small models; SIMT kernels)                  */
+
+/* ---- parameter tensors (for gpt_param_offset) -------------------------- */
+#define GPT_T_WTE 0     /* [vocab, d_model]          token embedding          */
+#define GPT_T_WQKV 1    /* [3*d_model, d_model]      q rows, then k, then v;  */
+                        /*   inside each block head h owns rows h*hd..h*hd+hd-1 */
+#define GPT_T_WO 2      /* [d_model, d_model]        attention out-projection */
+#define GPT_T_WUP 3     /* [d_ff, d_model]           MLP up                   */
+#define GPT_T_WDOWN 4   /* [d_model, d_ff]           MLP down                 */
+#define GPT_T_LM_HEAD 5 /* [vocab, d_model]          untied output head       */
+
+/* ---- workspace regions (for gpt_workspace_region, diagnostics/tests) ---- */
+#define GPT_W_STATUS 0     /* gpt_device_status struct                                 */
+#define GPT_W_RESID 1      /* fp32 [N, d]: residual stream.  After gpt_forward_loss it */
+                           /*   holds the last layer's output (x0 = wte[tokens], exact, */
+                           /*   when n_layer == 0); after gpt_backward, d loss / d x0   */
+#define GPT_W_LSE 2        /* fp32 [N]: logsumexp of each position's logits           */
+#define GPT_W_SORT_PERM 3  /* int32 [N]: positions stably sorted by token id          */
+#define GPT_W_SORT_OFFS 4  /* int32 [vocab+1]: segment starts in SORT_PERM            */
+#define GPT_W_ATTN_LSE 5   /* fp32 [B, H, T] of layer `layer`: row logsumexp of the    */
+                           /*   scaled attention scores                                */
+
+/* Device-side status, at the start of the workspace. */
+typedef struct gpt_device_status {
+  int32_t code;      /* 0 or the first GPT_E* recorded              */
+  int32_t where;     /* kernel id that recorded it (diagnostic)      */
+  int64_t index;     /* offending token position / wait site         */
+  int32_t reserved[12];
+} gpt_device_status;
+
+typedef struct gpt_config {
+  /* model and batch shape (set by the caller) */
+  int32_t n_layer;  /* >= 0                                             */
+  int32_t d_model;  /* = n_head * head_dim                               */
+  int32_t n_head;
+  int32_t head_dim; /* bf16: 64 or 128; f32: even, <= 128               */
+  int32_t d_ff;     /* bf16: multiple of 64; f32: any >= 1              */
+  int32_t vocab;    /* >= 2                                              */
+  int32_t seq_len;  /* T >= 1                                            */
+  int32_t batch;    /* B >= 1                                            */
+  int32_t dtype;    /* GPT_BF16 or GPT_F32                               */
+  int32_t qk_norm;  /* 1: RMSNorm q and k per head after RoPE (default)  */
+  float rope_base;  /* 10000 by default                                  */
+  float norm_eps;   /* 1e-6 by default                                   */
+  /* derived by gpt_config_init */
+  int64_t n_params;        /* parameter count                               */
+  uint64_t param_bytes;    /* bytes of the flat parameter (and grad) buffer */
+  uint64_t workspace_bytes;/* bytes of the workspace                        */
+} gpt_config;
+
+/* Validate `cfg` and fill its derived fields.  Host only, no CUDA call.
+ * Zero-valued rope_base / norm_eps are replaced by the defaults.
+ * GPT_EINVAL for a NULL or inconsistent config (d_model != n_head*head_dim,
+ * non-positive sizes), GPT_EUNSUPPORTED for shapes the kernels do not cover
+ * (bf16: d_model % 64, d_ff % 64, head_dim not 64/128; f32: odd head_dim or
+ * head_dim > 128). */
+int gpt_config_init(gpt_config* cfg);
+
+/* The depth dial: d_model = 64*depth, head_dim = 128, n_head = depth/2,
+ * d_ff = 4*d_model, n_layer = depth, bf16, qk_norm on, defaults for eps and
+ * RoPE base; then gpt_config_init.  depth must be even and >= 2. */
+int gpt_config_from_depth(gpt_config* cfg, int depth, int seq_len, int batch, int vocab);
+
+/* Element offset and [rows, cols] of one parameter tensor inside the flat
+ * parameter buffer (the grad buffer has the same layout).  Tensors are
+ * row-major [out, in].  `layer` is ignored for GPT_T_WTE / GPT_T_LM_HEAD.
+ * Order in the buffer: wte, then per layer wqkv, wo, wup, wdown, then lm_head;
+ * every tensor starts on a 128-element boundary. */
+int gpt_param_offset(const gpt_config* cfg, int tensor, int layer, int64_t* elem_offset,
+                     int64_t* rows, int64_t* cols);
+
+/* Byte offset and size of a workspace region (GPT_W_*); `layer` is used by
+ * per-layer regions only. */
+int gpt_workspace_region(const gpt_config* cfg, int region, int layer, uint64_t* byte_offset,
+                         uint64_t* bytes);
+
+/* Forward pass and loss.
+ *   tokens, targets: device int32 [batch, seq_len], row-major.
+ *   params:          device, flat buffer of cfg->param_bytes (layout above).
+ *   workspace:       device, cfg->workspace_bytes; receives every activation
+ *                    the backward needs, and the status word (reset here).
+ *   loss:            device fp32 scalar = mean per-position loss.
+ *   token_loss:      device fp32 [batch*seq_len] or NULL.
+ * Token/target ids outside [0, vocab) record GPT_EDATA (read it with
+ * gpt_status); their rows are computed from id 0 and their loss is 0. */
+int gpt_forward_loss(const gpt_config* cfg, const int32_t* tokens, const int32_t* targets,
+                     const void* params, void* workspace, float* loss, float* token_loss,
+                     void* stream);
+
+/* Backward pass of the loss computed by the last gpt_forward_loss on the same
+ * workspace and stream, with the same tokens/targets/params.
+ *   grads:      device, same layout and dtype as params.
+ *   accumulate: 0 = overwrite grads, 1 = grads += this step's gradient.
+ * The gradient is that of the mean loss over all batch*seq_len positions. */
+int gpt_backward(const gpt_config* cfg, const int32_t* tokens, const int32_t* targets,
+                 const void* params, void* workspace, void* grads, int accumulate,
+                 void* stream);
+
+/* One whole training step from HOST token/target arrays (pinned memory gives
+ * asynchronous copies): copies tokens/targets into the workspace's staging
+ * area, runs gpt_forward_loss and gpt_backward, and copies the loss back to
+ * *host_loss.  Returns after enqueueing; *host_loss is valid once `stream`
+ * has been synchronised. */
+int gpt_train_step_host(const gpt_config* cfg, const int32_t* host_tokens,
+                        const int32_t* host_targets, const void* params, void* workspace,
+                        void* grads, int accumulate, float* host_loss, void* stream);
+
+/* Synchronise `stream`, then return the device status recorded in
+ * `workspace` (GPT_OK or the first GPT_E* a kernel recorded), or GPT_ECUDA
+ * if the synchronisation itself failed. */
+int gpt_status(const void* workspace, void* stream);
+
+/* Static string for a GPT_E* code. */
+const char* gpt_strerror(int code);
+
+/* Library version string. */
+const char* gpt_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GPT_B200_H */

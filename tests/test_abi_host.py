@@ -1,0 +1,158 @@
+"""Host-side tests of the C ABI (no GPU needed, no kernel launched).
+
+The library is built if missing; every function declared in include/gpt.h
+must be exported; configuration validation, the parameter layout and the
+workspace regions are checked against the workload shapes; invalid arguments
+are rejected before any CUDA call.
+"""
+import ctypes
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def B():
+    from decoder_only_gpt_b200 import build
+    build.build()
+    from decoder_only_gpt_b200 import binding
+    return binding
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "gpt.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gpt_[a-z_]+)\s*\(", src)))
+
+
+def test_every_declared_function_is_exported(B):
+    names = header_functions()
+    assert "gpt_forward_loss" in names and "gpt_backward" in names and "gpt_config_init" in names
+    lib = ctypes.CDLL(B.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_header_constants_match_binding(B):
+    src = open(os.path.join(ROOT, "include", "gpt.h")).read()
+    consts = dict(re.findall(r"#define (GPT_[A-Z0-9_]+) \(?(-?\d+)\)?", src))
+    for k, v in consts.items():
+        if hasattr(B, k):
+            assert getattr(B, k) == int(v), k
+
+
+@pytest.mark.parametrize("name", list(synth.WORKLOADS))
+def test_config_derived_fields(B, name):
+    w = synth.workload(name)
+    c = B.config_from_workload(w)
+    d, F, V, L = w.d_model, w.d_ff, w.vocab, w.n_layer
+    assert c.n_params == 2 * V * d + L * (4 * d * d + 2 * F * d)
+    esz = 2 if w.dtype == "bf16" else 4
+    assert c.param_bytes >= c.n_params * esz
+    assert c.param_bytes - c.n_params * esz < (2 + 4 * L) * 128 * esz
+    assert c.workspace_bytes > 0 and c.workspace_bytes % 256 == 0
+
+
+def test_depth_dial(B):
+    for depth, d, H in [(4, 256, 2), (12, 768, 6), (24, 1536, 12)]:
+        c = B.config_from_depth(depth, 2048, 16, 32768)
+        assert (c.n_layer, c.d_model, c.n_head, c.head_dim, c.d_ff) == (depth, d, H, 128, 4 * d)
+        assert c.dtype == B.GPT_BF16 and c.qk_norm == 1
+    assert B.lib().gpt_config_from_depth(ctypes.byref(B.GptConfig()), 3, 64, 1, 100) == B.GPT_EINVAL
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d_model=100), "EINVAL"),              # != n_head * head_dim
+    (dict(head_dim=32, d_model=128, n_head=4), "EUNSUPPORTED"),
+    (dict(d_ff=100), "EUNSUPPORTED"),
+    (dict(vocab=1), "EINVAL"),
+    (dict(seq_len=0), "EINVAL"),
+    (dict(batch=-1), "EINVAL"),
+])
+def test_config_rejects(B, kw, code):
+    base = dict(n_layer=2, d_model=256, n_head=2, head_dim=128, d_ff=1024, vocab=4096,
+                seq_len=64, batch=2)
+    base.update(kw)
+    c = B.make_config(**base, check=False)
+    rc = B.lib().gpt_config_init(ctypes.byref(c))
+    assert rc == getattr(B, "GPT_" + code)
+
+
+def test_f32_config_rules(B):
+    ok = B.make_config(2, 64, 4, 16, 256, 256, 64, 4, dtype="f32")
+    assert ok.param_bytes % 4 == 0
+    bad = B.make_config(2, 66, 2, 33, 256, 256, 64, 4, dtype="f32", check=False)
+    assert B.lib().gpt_config_init(ctypes.byref(bad)) == B.GPT_EUNSUPPORTED
+
+
+@pytest.mark.parametrize("name", ["tiny", "story", "d24"])
+def test_param_layout(B, name):
+    w = synth.workload(name)
+    c = B.config_from_workload(w)
+    esz = 2 if w.dtype == "bf16" else 4
+    shapes = dict(synth.param_shapes(w))
+    prev_end = 0
+    for pname, tid, layer in B.tensor_slots(c):
+        off, r, cc = B.param_offset(c, tid, layer)
+        assert (r, cc) == shapes[pname]
+        assert off % 128 == 0 and off >= prev_end
+        prev_end = off + r * cc
+    assert prev_end * esz <= c.param_bytes
+
+
+def test_param_offset_rejects(B):
+    c = B.config_from_workload(synth.workload("tiny"))
+    o = ctypes.c_int64()
+    assert B.lib().gpt_param_offset(ctypes.byref(c), 9, 0, ctypes.byref(o), ctypes.byref(o),
+                                    ctypes.byref(o)) == B.GPT_EINVAL
+    assert B.lib().gpt_param_offset(ctypes.byref(c), B.GPT_T_WO, 5, ctypes.byref(o),
+                                    ctypes.byref(o), ctypes.byref(o)) == B.GPT_EINVAL
+
+
+def test_workspace_regions_in_bounds(B):
+    w = synth.workload("story")
+    c = B.config_from_workload(w)
+    for reg, layer in [(B.GPT_W_STATUS, 0), (B.GPT_W_RESID, 0), (B.GPT_W_LSE, 0),
+                       (B.GPT_W_SORT_PERM, 0), (B.GPT_W_SORT_OFFS, 0), (B.GPT_W_ATTN_LSE, 2)]:
+        off, nb = B.workspace_region(c, reg, layer)
+        assert off % 256 == 0 and off + nb <= c.workspace_bytes
+    N = w.batch * w.seq_len
+    assert B.workspace_region(c, B.GPT_W_RESID)[1] == N * w.d_model * 4
+    assert B.workspace_region(c, B.GPT_W_SORT_OFFS)[1] == (w.vocab + 1) * 4
+
+
+def test_invalid_pointers_rejected_before_any_launch(B):
+    c = B.config_from_workload(synth.workload("tiny"))
+    a = 1 << 20  # fake, never dereferenced: validation fails first
+    assert B.raw_forward_loss(c, None, a, a, a, a) == B.GPT_EINVAL
+    assert B.raw_forward_loss(c, a + 4, a, a, a, a) == B.GPT_EINVAL      # misaligned tokens
+    assert B.raw_forward_loss(c, a, a, a + 16, a, a) == B.GPT_EINVAL     # params not 256-aligned
+    assert B.raw_backward(c, a, a, a, a, None) == B.GPT_EINVAL
+    assert B.raw_backward(c, a, a, a, a, a, accumulate=2) == B.GPT_EINVAL
+    stale = B.make_config(2, 64, 4, 16, 256, 256, 64, 4, dtype="f32")
+    stale.batch = 8  # derived fields no longer match
+    assert B.raw_forward_loss(stale, a, a, a, a, a) == B.GPT_EINVAL
+
+
+def test_strerror(B):
+    for code in range(0, -7, -1):
+        assert B.strerror(code) and "unknown" not in B.strerror(code)
+    assert "unknown" in B.strerror(-99)
+    assert B.lib().gpt_version().startswith(b"libgpt")
+
+
+def test_pack_unpack_roundtrip(B):
+    w = synth.workload("tiny")
+    c = B.config_from_workload(w)
+    p = synth.make_params(w, as_bits=True)
+    flat = B.pack_params(c, p)
+    back = B.unpack_flat(c, flat)
+    for k in p:
+        assert np.array_equal(back[k], p[k])

@@ -1,0 +1,272 @@
+"""Parity of the CUDA training step with the fp64 CPU oracle (needs a B200).
+
+Tolerances:
+* bf16 storage: loss within 1e-3 relative; every gradient tensor with cosine
+  similarity >= 0.999 and max|g - r| / max|r| <= 3e-2; per-position losses
+  within 2e-2 relative (each one is a difference of two O(10) numbers formed
+  from bf16 activations, so its error is about ten bf16 half-ulps of the
+  logits, ~1e-2 relative at most, while the mean averages that down).
+* fp32 storage (tiny model): loss 1e-5 relative, cosine >= 0.99999,
+  max-rel <= 1e-3 (fp32 accumulation over at most a few thousand terms).
+* index work (gather, stable sort of positions by token id): bit-exact.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+TOL = {
+    "bf16": dict(loss=1e-3, cos=0.999, maxrel=3e-2, tok=2e-2),
+    "f32": dict(loss=1e-5, cos=0.99999, maxrel=1e-3, tok=1e-4),
+}
+
+# (name, base workload, overrides): full-size small workloads plus ragged shapes
+CASES = {
+    "tiny": ("tiny", {}),
+    "story": ("story", {}),
+    "d4": ("d4", {}),
+    # ragged: 300 tokens (3 row tiles, last partial), vocab 1000 (last column tile partial),
+    # seq 100 (attention tail), hd 64
+    "ragged": ("story", dict(n_layer=2, d_model=128, n_head=2, head_dim=64, d_ff=320, vocab=1000,
+                             seq_len=100, batch=3)),
+    # head_dim 128 with two heads, odd batch
+    "hd128": ("d4", dict(n_layer=1, d_model=256, n_head=2, head_dim=128, d_ff=512, vocab=2048,
+                         seq_len=192, batch=3)),
+    # fp32 ragged
+    "tiny_ragged": ("tiny", dict(seq_len=37, batch=3, vocab=100, d_ff=96)),
+}
+
+
+@pytest.fixture(scope="module")
+def B():
+    from decoder_only_gpt_b200 import build
+    build.build()
+    from decoder_only_gpt_b200 import binding
+    return binding
+
+
+@pytest.fixture(scope="module")
+def R():
+    from decoder_only_gpt_b200 import runtime
+    return runtime
+
+
+def workload_of(case):
+    base, kw = CASES[case]
+    return synth.workload(base, **kw)
+
+
+_oracle_cache = {}
+
+
+def oracle_result(case):
+    if case not in _oracle_cache:
+        w = workload_of(case)
+        tok, tgt = synth.make_tokens(w)
+        res = oracle.step(oracle.from_workload(w), synth.make_params(w), tok, tgt)
+        _oracle_cache[case] = res
+    return _oracle_cache[case]
+
+
+def run_gpu(B, R, w, tokens=None, targets=None, forward_only=False):
+    cfg = B.config_from_workload(w)
+    st = R.TrainStep(cfg)
+    st.load_params(synth.make_params(w, as_bits=True))
+    tok, tgt = synth.make_tokens(w)
+    if tokens is not None:
+        tok = tokens
+    if targets is not None:
+        tgt = targets
+    st.set_batch(tok, tgt)
+    if forward_only:
+        st.forward()
+    else:
+        st.step()
+    code = st.status()
+    return st, code
+
+
+def grad_metrics(g, r):
+    g = g.ravel()
+    r = r.ravel()
+    cos = float(np.dot(g, r) / (np.linalg.norm(g) * np.linalg.norm(r) + 1e-300))
+    maxrel = float(np.max(np.abs(g - r)) / (np.max(np.abs(r)) + 1e-300))
+    return cos, maxrel
+
+
+def check_against_oracle(st, w, res):
+    tol = TOL[w.dtype]
+    loss = float(st.loss.cpu().numpy()[0])
+    assert abs(loss - res.loss) / abs(res.loss) <= tol["loss"], (loss, res.loss)
+    tl = st.token_loss.cpu().numpy().astype(np.float64).reshape(w.batch, w.seq_len)
+    rel = np.abs(tl - res.token_loss) / np.maximum(np.abs(res.token_loss), 1.0)
+    assert rel.max() <= tol["tok"], rel.max()
+    grads = st.grads_f64()
+    worst = {}
+    for name, ref in res.grads.items():
+        cos, mr = grad_metrics(grads[name], ref)
+        worst[name] = (cos, mr)
+    bad = {k: v for k, v in worst.items() if v[0] < tol["cos"] or v[1] > tol["maxrel"]}
+    assert not bad, bad
+
+
+@pytest.mark.parametrize("case", list(CASES))
+def test_step_matches_oracle(B, R, case):
+    w = workload_of(case)
+    st, code = run_gpu(B, R, w)
+    assert code == B.GPT_OK, B.strerror(code)
+    check_against_oracle(st, w, oracle_result(case))
+
+
+@pytest.mark.parametrize("case", ["story", "tiny"])
+def test_bitwise_deterministic(B, R, case):
+    w = workload_of(case)
+    a, _ = run_gpu(B, R, w)
+    b, _ = run_gpu(B, R, w)
+    assert np.array_equal(a.loss.cpu().numpy().view(np.uint32), b.loss.cpu().numpy().view(np.uint32))
+    assert np.array_equal(a.token_loss.cpu().numpy().view(np.uint32),
+                          b.token_loss.cpu().numpy().view(np.uint32))
+    assert np.array_equal(a.grads_raw(), b.grads_raw())
+    # same workspace, second step: still identical
+    a.step()
+    assert np.array_equal(a.grads_raw(), b.grads_raw())
+
+
+@pytest.mark.parametrize("shape", ["ragged", "full_d24"])
+def test_gather_bit_exact(B, R, shape):
+    # n_layer = 0: after the forward the residual buffer holds x0 = wte[tokens]
+    if shape == "ragged":
+        w = workload_of("ragged").replace(n_layer=0)
+    else:
+        w = synth.workload("d24", n_layer=0)
+    st, code = run_gpu(B, R, w, forward_only=True)
+    assert code == B.GPT_OK
+    x0 = st.region(B.GPT_W_RESID).view(np.float32).reshape(-1, w.d_model)
+    tok, _ = synth.make_tokens(w)
+    wte = synth.make_params(w, as_bits=True)["wte"]
+    want = (wte[tok.ravel()].astype(np.uint32) << 16).view(np.float32)
+    assert np.array_equal(x0.view(np.uint32), want.view(np.uint32))
+
+
+@pytest.mark.parametrize("shape", ["ragged", "full_d24"])
+def test_token_sort_bit_exact(B, R, shape):
+    w = workload_of("ragged") if shape == "ragged" else synth.workload("d24", n_layer=0)
+    st, code = run_gpu(B, R, w)
+    assert code == B.GPT_OK
+    tok, _ = synth.make_tokens(w)
+    perm = st.region(B.GPT_W_SORT_PERM).view(np.int32)
+    offs = st.region(B.GPT_W_SORT_OFFS).view(np.int32)
+    want_perm = np.argsort(tok.ravel(), kind="stable").astype(np.int32)
+    want_offs = np.concatenate([[0], np.cumsum(np.bincount(tok.ravel(), minlength=w.vocab))])
+    assert np.array_equal(perm, want_perm)
+    assert np.array_equal(offs, want_offs.astype(np.int32))
+
+
+def test_untouched_embedding_rows_are_zero(B, R):
+    w = workload_of("story")
+    st, _ = run_gpu(B, R, w)
+    tok, _ = synth.make_tokens(w)
+    g = st.grads_f64()["wte"]
+    miss = np.setdiff1d(np.arange(w.vocab), np.unique(tok))
+    assert miss.size > 0 and np.all(g[miss] == 0.0)
+
+
+def test_causality_on_gpu(B, R):
+    w = workload_of("story")
+    tok, tgt = synth.make_tokens(w)
+    a, _ = run_gpu(B, R, w)
+    tok2 = tok.copy()
+    b, t = 5, 100
+    tok2[b, t + 1:] = (tok2[b, t + 1:] + 7) % w.vocab
+    c, _ = run_gpu(B, R, w, tokens=tok2)
+    la = a.token_loss.cpu().numpy().reshape(w.batch, w.seq_len)
+    lc = c.token_loss.cpu().numpy().reshape(w.batch, w.seq_len)
+    assert np.array_equal(la[b, : t + 1].view(np.uint32), lc[b, : t + 1].view(np.uint32))
+    assert not np.array_equal(la[b, t + 1:], lc[b, t + 1:])
+
+
+def test_accumulate_doubles_gradient(B, R):
+    w = workload_of("ragged")
+    st, _ = run_gpu(B, R, w)
+    st.backward(accumulate=True)
+    grads = st.grads_f64()
+    res = oracle_result("ragged")
+    for name, ref in res.grads.items():
+        cos, mr = grad_metrics(grads[name], 2 * ref)
+        assert cos >= 0.999 and mr <= 3e-2, (name, cos, mr)
+
+
+def test_bad_ids_reported(B, R):
+    w = workload_of("ragged")
+    tok, tgt = synth.make_tokens(w)
+    bad_tok = tok.copy()
+    bad_tok[1, 3] = w.vocab
+    _, code = run_gpu(B, R, w, tokens=bad_tok)
+    assert code == B.GPT_EDATA
+    bad_tgt = tgt.copy()
+    bad_tgt[0, 0] = -1
+    st, code = run_gpu(B, R, w, targets=bad_tgt)
+    assert code == B.GPT_EDATA
+    # the next clean forward resets the status
+    st.set_batch(tok, tgt)
+    st.step()
+    assert st.status() == B.GPT_OK
+
+
+def test_train_step_host_matches_device_path(B, R):
+    import torch
+    w = workload_of("ragged")
+    st, _ = run_gpu(B, R, w)
+    want = st.grads_raw()
+    tok, tgt = synth.make_tokens(w)
+    ht = torch.from_numpy(tok.ravel().copy()).pin_memory()
+    hy = torch.from_numpy(tgt.ravel().copy()).pin_memory()
+    hl = torch.zeros(1, dtype=torch.float32).pin_memory()
+    st.grads.zero_()
+    B.train_step_host(st.cfg, ht, hy, st.params, st.workspace, st.grads, hl, stream=st.stream)
+    torch.cuda.synchronize()
+    assert float(hl[0]) == float(st.loss.cpu()[0])
+    assert np.array_equal(st.grads_raw(), want)
+
+
+def _samples(name):
+    path = os.path.join(GOLDEN, f"oracle_samples_{name}.npz")
+    if not os.path.exists(path):
+        pytest.skip(f"{path} not generated")
+    return np.load(path)
+
+
+@pytest.mark.parametrize("name", ["d12", "d24"])
+def test_full_size_against_oracle_samples(B, R, name):
+    """Full-size workloads in the benchmark's launch configuration: the loss, every
+    per-position loss, and gradient entries at the oracle's seeded coordinates."""
+    s = _samples(name)
+    w = synth.workload(name)
+    st, code = run_gpu(B, R, w)
+    assert code == B.GPT_OK
+    tol = TOL["bf16"]
+    loss = float(st.loss.cpu()[0])
+    assert abs(loss - float(s["loss"])) / float(s["loss"]) <= tol["loss"]
+    tl = st.token_loss.cpu().numpy().astype(np.float64).reshape(w.batch, w.seq_len)
+    rel = np.abs(tl - s["token_loss"]) / np.maximum(np.abs(s["token_loss"]), 1.0)
+    assert rel.max() <= tol["tok"], rel.max()
+    grads = st.grads_f64()
+    bad = {}
+    for pname, _ in synth.param_shapes(w):
+        r, c = s[f"{pname}/rows"], s[f"{pname}/cols"]
+        ref = s[f"{pname}/values"]
+        got = grads[pname][r, c]
+        cos = float(np.dot(got, ref) / (np.linalg.norm(got) * np.linalg.norm(ref) + 1e-300))
+        mr = float(np.max(np.abs(got - ref)) / float(s[f"{pname}/absmax"]))
+        fro = float(np.linalg.norm(grads[pname]))
+        if cos < tol["cos"] or mr > tol["maxrel"] or abs(fro / float(s[f"{pname}/fro"]) - 1) > 0.02:
+            bad[pname] = (cos, mr, fro / float(s[f"{pname}/fro"]))
+    assert not bad, bad
