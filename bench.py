@@ -1,0 +1,386 @@
+#!/usr/bin/env python
+"""Training-step throughput of the depth-24 GPT on B200 (tokens/s and MFU).
+
+One step = gpt_forward_loss + gpt_backward (every gradient written, no
+optimizer) on one synthetic batch of 16 x 2048 tokens (Zipf(1.1) ids, seeded
+N(0, 0.02) bf16 weights).  Inputs are resident in HBM when the timed region
+starts; the step touches tens of GB, far more than the 126 MB L2, so no L2
+flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU runs (under torchrun) are replicas: every rank runs the whole step
+on its own batch; ranks meet only at the timing barriers, and the reported
+time is the maximum over ranks.  Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle (the only reference there is) on
+the host cores, on a bounded sample of the same workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+WORKLOAD = "d24"
+METRIC = "train tokens/sec (fwd+bwd) on 1 B200 for depth-12/24 GPT; MFU vs bf16 peak"
+
+
+def flops_per_token(w) -> float:
+    """Algorithmic FLOPs per token, fwd+bwd = 3x fwd: 6*(12 L d^2 + V d) + 6 L T d (causal)."""
+    L, d, V, T = w.n_layer, w.d_model, w.vocab, w.seq_len
+    return 6.0 * (12 * L * d * d + V * d) + 6.0 * L * T * d
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=p["hbm_gbs"], bf16_tflops=p["bf16_tflops"],
+                    bf16_tflops_sustained=p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def workload_desc(w):
+    return (f"{w.name}: {w.n_layer} layers, d_model {w.d_model}, {w.n_head}x{w.head_dim} heads, "
+            f"d_ff {w.d_ff}, vocab {w.vocab}, seq {w.seq_len}, batch {w.batch}")
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id: str | None):
+        self.bus = bus_id
+        self.proc = None
+        self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.tmp.flush()
+        self.tmp.seek(0)
+        rows = [r.split(", ") for r in self.tmp.read().strip().splitlines() if r.strip()]
+        os.unlink(self.tmp.name)
+        if self.bus:
+            key = self.bus.lower()[-7:]
+            rows = [r for r in rows if r and r[0].lower().endswith(key)] or rows
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample_setup(w, bits=None, target_s=10.0):
+    """The oracle on the first n positions of one sequence of workload w, with n
+    (a multiple of 32, at most seq_len) sized from a 32-position probe so that
+    one sample takes about target_s seconds on this host."""
+    import oracle
+    if bits is None:
+        bits = synth.make_params(w, as_bits=True)
+    params = {k: synth.bf16_bits_to_f64(v) for k, v in bits.items()}
+    tok, tgt = synth.make_tokens(w)
+
+    def setup(n):
+        ws = w.replace(seq_len=n, batch=1)
+        return oracle, oracle.from_workload(ws), params, tok[:1, :n], tgt[:1, :n]
+
+    probe = setup(min(32, w.seq_len))
+    time_oracle(probe)                       # untimed: BLAS start-up, page-in
+    per_tok = time_oracle(probe) / probe[3].shape[1]
+    n = int(max(32, min(w.seq_len, round(target_s / per_tok / 32) * 32)))
+    return setup(min(n, w.seq_len))
+
+
+def time_oracle(setup, steps=1):
+    oracle, cfg, params, tok, tgt = setup
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        oracle.step(cfg, params, tok, tgt)
+    return time.perf_counter() - t0
+
+
+def sample_tokens(setup):
+    return int(setup[3].shape[1])
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from decoder_only_gpt_b200 import binding as B
+    from decoder_only_gpt_b200 import runtime as R
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    w = synth.workload(args.workload)
+    if args.batch:
+        w = w.replace(batch=args.batch)
+    wr = w.replace(seed=w.seed + 100 * rank)  # each replica its own batch
+    cfg = B.config_from_workload(w)
+    st = R.TrainStep(cfg, device=f"cuda:{local_rank}")
+    bits = synth.make_params(w, as_bits=True)
+    st.load_params(bits)
+    tok, tgt = synth.make_tokens(wr)
+    st.set_batch(tok, tgt)
+    N = w.batch * w.seq_len
+    stream = torch.cuda.current_stream(dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        st.step()
+    torch.cuda.synchronize()
+    code = st.status()
+    if code != B.GPT_OK:
+        raise SystemExit(f"device status after warm-up: {B.strerror(code)}")
+
+    per_step = 600
+    trace = B.Trace(capacity=per_step * args.steps + 16)
+    bus = None
+    try:
+        bus = torch.cuda.get_device_properties(dev).pci_bus_id
+    except Exception:
+        bus = None
+    clocks = ClockSampler(bus if isinstance(bus, str) else None)
+
+    # ---- timed region (device time, CUDA events on the launching stream) ----
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    trace.attach()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        st.step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    B.Trace.detach()
+    barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    code = st.status()
+    if code != B.GPT_OK:
+        raise SystemExit(f"device status after timed steps: {B.strerror(code)}")
+    stats, dropped = trace.summary()
+    trace.close()
+
+    # ---- end to end through the public host-buffer call ----
+    ht = torch.from_numpy(tok.ravel().copy()).pin_memory()
+    hy = torch.from_numpy(tgt.ravel().copy()).pin_memory()
+    hl = torch.zeros(1, dtype=torch.float32).pin_memory()
+    B.train_step_host(cfg, ht, hy, st.params, st.workspace, st.grads, hl, stream=stream.cuda_stream)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        B.train_step_host(cfg, ht, hy, st.params, st.workspace, st.grads, hl,
+                          stream=stream.cuda_stream)
+        stream.synchronize()  # the loss is read on the host every step
+        assert math.isfinite(float(hl[0]))
+    f1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = f0.elapsed_time(f1)
+
+    if world > 1:
+        t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, e2e_ms = float(t[0]), float(t[1])
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks = load_peaks()
+    tok_s = world * N * args.steps / (ms / 1e3)
+    fpt = flops_per_token(w)
+    g = stats["gemm"]
+    gemm_tf = g["flops"] / (g["ms"] / 1e3) / 1e12 if g["ms"] > 0 else 0.0
+    peak_tf = peaks["bf16_tflops_sustained"]
+    kernels = sum(s["kernels"] for s in stats.values())
+    breakdown = {k: {"ms_per_step": round(v["ms"] / args.steps, 3),
+                     "launches_per_step": v["launches"] // max(args.steps, 1),
+                     **({"tflops": round(v["flops"] / (v["ms"] / 1e3) / 1e12, 1)} if v["flops"] and v["ms"] else {}),
+                     **({"gbs": round(v["bytes"] / (v["ms"] / 1e3) / 1e9, 1)} if not v["flops"] and v["ms"] else {})}
+                 for k, v in stats.items() if v["launches"]}
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only) ----
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        setup = oracle_sample_setup(w, bits)
+        n = sample_tokens(setup)
+        secs = time_oracle(setup)
+        cpu = {"value": round(n / secs, 3), "unit": "tokens/s",
+               "cores": cpu_cores(), "kind": "oracle",
+               "sample": f"fp64 NumPy oracle fwd+bwd of the {w.name} model on the first "
+                         f"{n} positions of one sequence ({secs:.1f} s)"}
+
+    line = {
+        "metric": METRIC,
+        "value": round(tok_s, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms / args.steps, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (Zipf(1.1) token ids, seeded N(0,0.02) bf16 weights)",
+        "config": {"workload": workload_desc(w), "global_batch": w.batch * world,
+                   "seq_len": w.seq_len, "tokens_per_step": N * world,
+                   "parallelism": f"replicas only x{world}" if world > 1 else "single GPU",
+                   "l2": "no flush: every step moves tens of GB, far above the 126 MB L2"},
+        "mfu": round(tok_s / world * fpt / (peak_tf * 1e12), 4),
+        "mfu_vs_nominal_2250tf": round(tok_s / world * fpt / 2.25e15, 4),
+        "flops_per_token": fpt,
+        "roofline": {"bound": "tensor", "kernel": "gemm_tc_kernel (tcgen05 GEMM, all launches)",
+                     "achieved": round(gemm_tf, 1), "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": round(gemm_tf / peak_tf, 4),
+                     "peak_source": f"{peaks['source']} bf16_tflops_sustained",
+                     "traffic": None},
+        "kernel_breakdown": breakdown,
+        "gpu_launches": kernels,
+        "trace_dropped": dropped,
+        "e2e": {"value": round(world * N * args.steps / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": 2 * N * 4, "d2h_bytes_per_step": 4},
+        "clocks": clk,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle
+# ---------------------------------------------------------------------------
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    w = synth.workload(args.workload)
+    setup = oracle_sample_setup(w, target_s=8.0)
+    n = sample_tokens(setup)
+    if args.warmup > 0:
+        time_oracle(setup)  # one untimed sample
+    secs = time_oracle(setup, steps=args.steps)
+    value = n * args.steps / secs
+    sample = (f"fp64 NumPy oracle fwd+bwd of the {w.name} model on the first {n} "
+              f"positions of one sequence per step")
+    line = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": "tokens/s",
+        "n_gpus": args.gpus,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(secs / args.steps * 1e3, 1),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (Zipf(1.1) token ids, seeded N(0,0.02) bf16 weights)",
+        "config": {"workload": workload_desc(w), "global_batch": w.batch, "seq_len": w.seq_len,
+                   "tokens_per_step": n, "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cpu_cores(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WORKLOAD, choices=list(synth.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip timing the CPU oracle sample")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (profiling captures on a smaller "
+                         "case; the line then reports that batch)")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+    else:
+        run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

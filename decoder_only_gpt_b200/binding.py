@@ -198,3 +198,50 @@ def raw_forward_loss(cfg, tokens, targets, params, workspace, loss, token_loss=N
 def raw_backward(cfg, tokens, targets, params, workspace, grads, accumulate=0, stream=None):
     return lib().gpt_backward(ctypes.byref(cfg), _ptr(tokens), _ptr(targets), _ptr(params),
                               _ptr(workspace), _ptr(grads), int(accumulate), stream)
+
+
+# ---- tracing ----------------------------------------------------------------
+GPT_K_NAMES = ["gemm", "attn_fwd", "attn_bwd", "norm", "qkv", "loss", "sort", "scatter", "other"]
+
+
+class GptTraceStat(ctypes.Structure):
+    _fields_ = [("launches", ctypes.c_int32), ("kernels", ctypes.c_int32), ("ms", ctypes.c_double),
+                ("flops", ctypes.c_double), ("bytes", ctypes.c_double)]
+
+
+class Trace:
+    """Per-launch CUDA-event trace of the library's kernels (see gpt_trace_* in gpt.h)."""
+
+    def __init__(self, capacity: int):
+        L = lib()
+        L.gpt_trace_create.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]
+        L.gpt_trace_attach.argtypes = [ctypes.c_void_p]
+        L.gpt_trace_reset.argtypes = [ctypes.c_void_p]
+        L.gpt_trace_summary.argtypes = [ctypes.c_void_p, ctypes.POINTER(GptTraceStat),
+                                        ctypes.POINTER(ctypes.c_int32)]
+        L.gpt_trace_destroy.argtypes = [ctypes.c_void_p]
+        self._h = ctypes.c_void_p()
+        _check(L.gpt_trace_create(ctypes.byref(self._h), capacity), "gpt_trace_create")
+
+    def attach(self):
+        _check(lib().gpt_trace_attach(self._h), "gpt_trace_attach")
+
+    @staticmethod
+    def detach():
+        _check(lib().gpt_trace_attach(None), "gpt_trace_attach")
+
+    def reset(self):
+        _check(lib().gpt_trace_reset(self._h), "gpt_trace_reset")
+
+    def summary(self):
+        stats = (GptTraceStat * len(GPT_K_NAMES))()
+        dropped = ctypes.c_int32()
+        _check(lib().gpt_trace_summary(self._h, stats, ctypes.byref(dropped)), "gpt_trace_summary")
+        out = {n: dict(launches=s.launches, kernels=s.kernels, ms=s.ms, flops=s.flops,
+                       bytes=s.bytes) for n, s in zip(GPT_K_NAMES, stats)}
+        return out, dropped.value
+
+    def close(self):
+        if self._h:
+            lib().gpt_trace_destroy(self._h)
+            self._h = ctypes.c_void_p()

@@ -5,9 +5,11 @@
 
 #include <cmath>
 #include <cstdio>
+#include <algorithm>
 #include <cstring>
 
 #include "gpt_internal.h"
+#include "trace.h"
 
 namespace gpt {
 namespace {
@@ -89,6 +91,9 @@ bool make_layout(const gpt_config& c, Layout* L) {
   L->dO = b.take(N * d * esz);
   L->dqkv = b.take(N * 3 * d * esz);
   L->Dattn = b.take(B * H * T * 4);
+  // split-K partials of the weight-gradient GEMMs (up to 4 splits of the largest layer matrix)
+  L->splitk_floats = c.dtype == GPT_BF16 ? 4 * std::max(std::max(3 * d * d, F * d), d * d) : 0;
+  L->splitk = b.take(L->splitk_floats * 4);
   // deterministic embedding scatter
   L->sort_tiles = (N + 1023) / 1024;
   L->sort_perm = b.take(N * 4);
@@ -240,28 +245,89 @@ static int check_common(const gpt_config* c, const int32_t* tok, const int32_t* 
   return GPT_OK;
 }
 
-struct Bufs {
+
+
+static GemmArgs gemm_kk(const void* A, int64_t lda, const void* B, int64_t ldb, int M, int N,
+                        int K, Epilogue epi, void* out, int64_t ldo, int32_t* status) {
+  GemmArgs g{};
+  g.A = A; g.B = B; g.lda = lda; g.ldb = ldb;
+  g.a_mn_major = false; g.b_mn_major = false;
+  g.M = M; g.N = N; g.K = K; g.epi = epi; g.out = out; g.ldo = ldo;
+  g.status = status;
+  return g;
+}
+
+// Weight-gradient GEMMs get the workspace's split-K buffer (used when the tile
+// count alone would leave SMs idle).
+static GemmArgs with_splitk(GemmArgs g, const Layout& L, char* ws) {
+  g.splitk = reinterpret_cast<float*>(ws + L.splitk);
+  g.splitk_floats = L.splitk_floats;
+  return g;
+}
+
+// ---- traced launch wrappers: algorithmic FLOPs / HBM bytes per launch -------
+static int run_gemm(const gpt_config& c, const GemmArgs& g, cudaStream_t st) {
+  const double e = c.dtype == GPT_BF16 ? 2.0 : 4.0;
+  double bytes = (double(g.M) * g.K + double(g.N) * g.K) * e;
+  const double mn = double(g.M) * g.N;
+  switch (g.epi) {
+    case EPI_STORE: bytes += mn * e * (g.beta ? 2 : 1); break;
+    case EPI_RESID_F32: bytes += mn * 8; break;
+    case EPI_DRELU2: bytes += mn * e * 2; break;
+    case EPI_CE_FWD: bytes += double(g.M) * 12; break;
+    default: bytes += mn * e; break;
+  }
+  TraceScope ts(GPT_K_GEMM, gemm_kernel_count(c, g), 2.0 * double(g.M) * g.N * g.K, bytes, st);
+  return launch_gemm(c, g, st);
+}
+
+static double attn_pairs(const gpt_config& c) {  // (query, key) pairs with key <= query
+  return double(c.batch) * c.n_head * (double(c.seq_len) * (c.seq_len + 1) / 2);
+}
+
+struct Step {
+  const gpt_config* c;
   char* ws;
   const char* p;
   Layout L;
   int esz;
-  const gpt_config* c;
+  int N, d, F, V;
+  cudaStream_t st;
+  int32_t* status;
+  float* cos_t;
+  float* sin_t;
+  float* x;
+
+  Step(const gpt_config* cfg, void* workspace, const void* params, void* stream) : c(cfg) {
+    ws = static_cast<char*>(workspace);
+    p = static_cast<const char*>(params);
+    make_layout(*c, &L);
+    esz = L.esz;
+    N = int(L.N); d = c->d_model; F = c->d_ff; V = c->vocab;
+    st = static_cast<cudaStream_t>(stream);
+    status = reinterpret_cast<int32_t*>(ws + L.status);
+    cos_t = reinterpret_cast<float*>(ws + L.rope_cos);
+    sin_t = reinterpret_cast<float*>(ws + L.rope_sin);
+    x = reinterpret_cast<float*>(ws + L.x);
+  }
   char* layer(int l) const { return ws + L.layer_base + L.layer_stride * uint64_t(l); }
+  float* f(uint64_t off) const { return reinterpret_cast<float*>(ws + off); }
   const void* param(int t, int l) const {
     int64_t off, r, cc;
     gpt_param_offset(c, t, l, &off, &r, &cc);
     return p + off * esz;
   }
-};
+  double nd() const { return double(N) * d; }
 
-static GemmArgs gemm_kk(const void* A, int64_t lda, const void* B, int64_t ldb, int M, int N,
-                        int K, Epilogue epi, void* out, int64_t ldo) {
-  GemmArgs g{};
-  g.A = A; g.B = B; g.lda = lda; g.ldb = ldb;
-  g.a_mn_major = false; g.b_mn_major = false;
-  g.M = M; g.N = N; g.K = K; g.epi = epi; g.out = out; g.ldo = ldo;
-  return g;
-}
+  int rms_fwd(void* h, float* r) {
+    TraceScope ts(GPT_K_NORM, 1, 0, nd() * (4 + esz) + N * 4.0, st);
+    return launch_rms_fwd(*c, x, h, r, st);
+  }
+  int rms_bwd(const void* dh, const void* h, const float* r, int acc) {
+    TraceScope ts(GPT_K_NORM, 1, 0, nd() * (2 * esz + (acc ? 4 : 0) + 4 + esz) + N * 4.0, st);
+    return launch_rms_bwd(*c, dh, h, r, x, ws + L.dxs, acc, st);
+  }
+};
 
 int gpt_forward_loss(const gpt_config* c, const int32_t* tok, const int32_t* tgt,
                      const void* params, void* workspace, float* loss, float* token_loss,
@@ -269,69 +335,67 @@ int gpt_forward_loss(const gpt_config* c, const int32_t* tok, const int32_t* tgt
   int rc = check_common(c, tok, tgt, params, workspace);
   if (rc) return rc;
   if (!loss || !aligned(loss, 4) || (token_loss && !aligned(token_loss, 4))) return GPT_EINVAL;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  Bufs b{static_cast<char*>(workspace), static_cast<const char*>(params), {}, 0, c};
-  make_layout(*c, &b.L);
-  b.esz = b.L.esz;
-  const Layout& L = b.L;
-  const int N = int(L.N), d = c->d_model, F = c->d_ff, V = c->vocab;
-  char* ws = b.ws;
-  int32_t* status = reinterpret_cast<int32_t*>(ws + L.status);
-  float* cos_t = reinterpret_cast<float*>(ws + L.rope_cos);
-  float* sin_t = reinterpret_cast<float*>(ws + L.rope_sin);
-  float* x = reinterpret_cast<float*>(ws + L.x);
-
-  GPT_TRY(cuda_rc(cudaMemsetAsync(ws + L.status, 0, 256, st)));
-  GPT_TRY(launch_rope_table(*c, cos_t, sin_t, st));
+  Step S(c, workspace, params, stream);
+  const Layout& L = S.L;
+  const int N = S.N, d = S.d, F = S.F, V = S.V, esz = S.esz;
+  char* ws = S.ws;
+  cudaStream_t st = S.st;
   {
-    void* h0 = c->n_layer > 0 ? (void*)(b.layer(0) + L.lo.h1) : (void*)(ws + L.hf);
-    float* r0 = reinterpret_cast<float*>(c->n_layer > 0 ? b.layer(0) + L.lo.r1 : ws + L.rf);
-    GPT_TRY(launch_embed_norm(*c, tok, b.param(GPT_T_WTE, 0), x, h0, r0, status, st));
+    TraceScope ts(GPT_K_OTHER, 2, 0, c->seq_len * c->head_dim * 4.0, st);
+    GPT_TRY(cuda_rc(cudaMemsetAsync(ws + L.status, 0, 256, st)));
+    GPT_TRY(launch_rope_table(*c, S.cos_t, S.sin_t, st));
   }
+  {
+    void* h0 = c->n_layer > 0 ? (void*)(S.layer(0) + L.lo.h1) : (void*)(ws + L.hf);
+    float* r0 = reinterpret_cast<float*>(c->n_layer > 0 ? S.layer(0) + L.lo.r1 : ws + L.rf);
+    TraceScope ts(GPT_K_NORM, 1, 0, S.nd() * (esz + 4 + esz) + N * 8.0, st);
+    GPT_TRY(launch_embed_norm(*c, tok, S.param(GPT_T_WTE, 0), S.x, h0, r0, S.status, st));
+  }
+  const double attn_f = 4.0 * attn_pairs(*c) * c->head_dim;  // QK^T and PV, causal half
   for (int l = 0; l < c->n_layer; ++l) {
-    char* Lb = b.layer(l);
-    GemmArgs g = gemm_kk(Lb + L.lo.h1, d, b.param(GPT_T_WQKV, l), d, N, 3 * d, d, EPI_STORE,
-                         ws + L.qkv_raw, 3 * d);
-    g.status = status;
-    GPT_TRY(launch_gemm(*c, g, st));
-    GPT_TRY(launch_qkv_post(*c, ws + L.qkv_raw, cos_t, sin_t, Lb + L.lo.q, Lb + L.lo.k,
-                            Lb + L.lo.v, reinterpret_cast<float*>(Lb + L.lo.rq),
-                            reinterpret_cast<float*>(Lb + L.lo.rk), st));
-    GPT_TRY(launch_attn_fwd(*c, Lb + L.lo.q, Lb + L.lo.k, Lb + L.lo.v, Lb + L.lo.o,
-                            reinterpret_cast<float*>(Lb + L.lo.lse), st));
-    g = gemm_kk(Lb + L.lo.o, d, b.param(GPT_T_WO, l), d, N, d, d, EPI_RESID_F32, x, d);
-    g.status = status;
-    GPT_TRY(launch_gemm(*c, g, st));
-    GPT_TRY(launch_rms_fwd(*c, x, Lb + L.lo.h2, reinterpret_cast<float*>(Lb + L.lo.r2), st));
-    g = gemm_kk(Lb + L.lo.h2, d, b.param(GPT_T_WUP, l), d, N, F, d, EPI_RELU2, Lb + L.lo.a, F);
-    g.status = status;
-    GPT_TRY(launch_gemm(*c, g, st));
-    g = gemm_kk(Lb + L.lo.a, F, b.param(GPT_T_WDOWN, l), F, N, d, F, EPI_RESID_F32, x, d);
-    g.status = status;
-    GPT_TRY(launch_gemm(*c, g, st));
+    char* Lb = S.layer(l);
+    GPT_TRY(run_gemm(*c, gemm_kk(Lb + L.lo.h1, d, S.param(GPT_T_WQKV, l), d, N, 3 * d, d,
+                                 EPI_STORE, ws + L.qkv_raw, 3 * d, S.status), st));
+    {
+      TraceScope ts(GPT_K_QKV, 1, 0, S.nd() * 3 * esz * 2, st);
+      GPT_TRY(launch_qkv_post(*c, ws + L.qkv_raw, S.cos_t, S.sin_t, Lb + L.lo.q, Lb + L.lo.k,
+                              Lb + L.lo.v, reinterpret_cast<float*>(Lb + L.lo.rq),
+                              reinterpret_cast<float*>(Lb + L.lo.rk), st));
+    }
+    {
+      TraceScope ts(GPT_K_ATTN_FWD, 1, attn_f, S.nd() * esz * 4, st);
+      GPT_TRY(launch_attn_fwd(*c, Lb + L.lo.q, Lb + L.lo.k, Lb + L.lo.v, Lb + L.lo.o,
+                              reinterpret_cast<float*>(Lb + L.lo.lse), S.status, st));
+    }
+    GPT_TRY(run_gemm(*c, gemm_kk(Lb + L.lo.o, d, S.param(GPT_T_WO, l), d, N, d, d,
+                                 EPI_RESID_F32, S.x, d, S.status), st));
+    GPT_TRY(S.rms_fwd(Lb + L.lo.h2, reinterpret_cast<float*>(Lb + L.lo.r2)));
+    GPT_TRY(run_gemm(*c, gemm_kk(Lb + L.lo.h2, d, S.param(GPT_T_WUP, l), d, N, F, d,
+                                 EPI_RELU2, Lb + L.lo.a, F, S.status), st));
+    GPT_TRY(run_gemm(*c, gemm_kk(Lb + L.lo.a, F, S.param(GPT_T_WDOWN, l), F, N, d, F,
+                                 EPI_RESID_F32, S.x, d, S.status), st));
     const bool last = l + 1 == c->n_layer;
-    void* hn = last ? (void*)(ws + L.hf) : (void*)(b.layer(l + 1) + L.lo.h1);
-    float* rn = reinterpret_cast<float*>(last ? ws + L.rf : b.layer(l + 1) + L.lo.r1);
-    GPT_TRY(launch_rms_fwd(*c, x, hn, rn, st));
+    void* hn = last ? (void*)(ws + L.hf) : (void*)(S.layer(l + 1) + L.lo.h1);
+    float* rn = reinterpret_cast<float*>(last ? ws + L.rf : S.layer(l + 1) + L.lo.r1);
+    GPT_TRY(S.rms_fwd(hn, rn));
   }
   // lm_head GEMM with the cross-entropy statistics in its epilogue
-  GemmArgs g = gemm_kk(ws + L.hf, d, b.param(GPT_T_LM_HEAD, 0), d, N, V, d, EPI_CE_FWD,
-                       nullptr, 0);
+  GemmArgs g = gemm_kk(ws + L.hf, d, S.param(GPT_T_LM_HEAD, 0), d, N, V, d, EPI_CE_FWD,
+                       nullptr, 0, S.status);
   g.targets = tgt;
-  g.part_max = reinterpret_cast<float*>(ws + L.part_max);
-  g.part_sum = reinterpret_cast<float*>(ws + L.part_sum);
-  g.tgt_logit = reinterpret_cast<float*>(ws + L.tgt_logit);
+  g.part_max = S.f(L.part_max);
+  g.part_sum = S.f(L.part_sum);
+  g.tgt_logit = S.f(L.tgt_logit);
   g.n_valid = V;
-  g.status = status;
-  GPT_TRY(launch_gemm(*c, g, st));
+  GPT_TRY(run_gemm(*c, g, st));
   const int tile_n = gemm_ce_tile_n(*c);
-  GPT_TRY(launch_ce_merge(*c, reinterpret_cast<float*>(ws + L.part_max),
-                          reinterpret_cast<float*>(ws + L.part_sum), (V + tile_n - 1) / tile_n,
-                          reinterpret_cast<float*>(ws + L.tgt_logit), tgt,
-                          reinterpret_cast<float*>(ws + L.lse_z),
-                          reinterpret_cast<float*>(ws + L.tok_loss), status, st));
-  GPT_TRY(launch_loss_mean(*c, reinterpret_cast<float*>(ws + L.tok_loss), loss, token_loss,
-                           status, st));
+  const int n_part = (V + tile_n - 1) / tile_n;
+  {
+    TraceScope ts(GPT_K_LOSS, 2, 0, double(N) * (n_part * 8.0 + 24), st);
+    GPT_TRY(launch_ce_merge(*c, S.f(L.part_max), S.f(L.part_sum), n_part, S.f(L.tgt_logit), tgt,
+                            S.f(L.lse_z), S.f(L.tok_loss), S.status, st));
+    GPT_TRY(launch_loss_mean(*c, S.f(L.tok_loss), loss, token_loss, S.status, st));
+  }
   return GPT_OK;
 }
 
@@ -341,18 +405,12 @@ int gpt_backward(const gpt_config* c, const int32_t* tok, const int32_t* tgt,
   int rc = check_common(c, tok, tgt, params, workspace);
   if (rc) return rc;
   if (!grads || !aligned(grads, 256) || (accumulate != 0 && accumulate != 1)) return GPT_EINVAL;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  Bufs b{static_cast<char*>(workspace), static_cast<const char*>(params), {}, 0, c};
-  make_layout(*c, &b.L);
-  b.esz = b.L.esz;
-  const Layout& L = b.L;
-  const int N = int(L.N), d = c->d_model, F = c->d_ff, V = c->vocab;
-  const int esz = L.esz;
-  char* ws = b.ws;
-  int32_t* status = reinterpret_cast<int32_t*>(ws + L.status);
-  float* cos_t = reinterpret_cast<float*>(ws + L.rope_cos);
-  float* sin_t = reinterpret_cast<float*>(ws + L.rope_sin);
-  float* dx = reinterpret_cast<float*>(ws + L.x);
+  Step S(c, workspace, params, stream);
+  const Layout& L = S.L;
+  const int N = S.N, d = S.d, F = S.F, V = S.V, esz = S.esz;
+  char* ws = S.ws;
+  cudaStream_t st = S.st;
+  int32_t* status = S.status;
   char* gr = static_cast<char*>(grads);
   auto grad = [&](int t, int l) -> void* {
     int64_t off, r, cc;
@@ -360,73 +418,79 @@ int gpt_backward(const gpt_config* c, const int32_t* tok, const int32_t* tgt,
     return gr + off * esz;
   };
 
-  GPT_TRY(launch_sort_tokens(*c, L, tok, ws, st));
-
+  {
+    TraceScope ts(GPT_K_SORT, 8, 0, double(N) * 12 + double(V) * 16, st);
+    GPT_TRY(launch_sort_tokens(*c, L, tok, ws, st));
+  }
   // logits gradient G = (softmax(z) - onehot(target)) / N, recomputed from the saved lse
-  GemmArgs g = gemm_kk(ws + L.hf, d, b.param(GPT_T_LM_HEAD, 0), d, N, int(L.vpad), d,
-                       EPI_CE_BWD, ws + L.G, L.vpad);
+  GemmArgs g = gemm_kk(ws + L.hf, d, S.param(GPT_T_LM_HEAD, 0), d, N, int(L.vpad), d,
+                       EPI_CE_BWD, ws + L.G, L.vpad, status);
   g.targets = tgt;
-  g.lse = reinterpret_cast<float*>(ws + L.lse_z);
+  g.lse = S.f(L.lse_z);
   g.inv_n = 1.0f / float(N);
   g.n_valid = V;
-  g.status = status;
-  GPT_TRY(launch_gemm(*c, g, st));
-  // dhf = G Wlm
-  g = gemm_kk(ws + L.G, L.vpad, b.param(GPT_T_LM_HEAD, 0), d, N, d, V, EPI_STORE, ws + L.dh, d);
+  GPT_TRY(run_gemm(*c, g, st));
+  // dhf = G Wlm ; dWlm = G^T hf
+  g = gemm_kk(ws + L.G, L.vpad, S.param(GPT_T_LM_HEAD, 0), d, N, d, V, EPI_STORE, ws + L.dh, d,
+              status);
   g.b_mn_major = true;
-  g.status = status;
-  GPT_TRY(launch_gemm(*c, g, st));
-  // dWlm = G^T hf
-  g = gemm_kk(ws + L.G, L.vpad, ws + L.hf, d, V, d, N, EPI_STORE, grad(GPT_T_LM_HEAD, 0), d);
+  GPT_TRY(run_gemm(*c, g, st));
+  g = gemm_kk(ws + L.G, L.vpad, ws + L.hf, d, V, d, N, EPI_STORE, grad(GPT_T_LM_HEAD, 0), d,
+              status);
   g.a_mn_major = true; g.b_mn_major = true; g.beta = accumulate;
-  g.status = status;
-  GPT_TRY(launch_gemm(*c, g, st));
-  GPT_TRY(launch_rms_bwd(*c, ws + L.dh, ws + L.hf, reinterpret_cast<float*>(ws + L.rf), dx,
-                         ws + L.dxs, 0, st));
+  GPT_TRY(run_gemm(*c, g, st));
+  GPT_TRY(S.rms_bwd(ws + L.dh, ws + L.hf, S.f(L.rf), 0));
 
+  const double attn_b = 8.0 * attn_pairs(*c) * c->head_dim;  // dV, dP, dQ, dK, causal half
   for (int l = c->n_layer - 1; l >= 0; --l) {
-    char* Lb = b.layer(l);
+    char* Lb = S.layer(l);
     // MLP down: da = dx Wdown, du = da * 2 relu(u) (from the stored a = relu(u)^2)
-    g = gemm_kk(ws + L.dxs, d, b.param(GPT_T_WDOWN, l), F, N, F, d, EPI_DRELU2, ws + L.du, F);
-    g.b_mn_major = true; g.aux = Lb + L.lo.a; g.status = status;
-    GPT_TRY(launch_gemm(*c, g, st));
-    g = gemm_kk(ws + L.dxs, d, Lb + L.lo.a, F, d, F, N, EPI_STORE, grad(GPT_T_WDOWN, l), F);
-    g.a_mn_major = true; g.b_mn_major = true; g.beta = accumulate; g.status = status;
-    GPT_TRY(launch_gemm(*c, g, st));
+    g = gemm_kk(ws + L.dxs, d, S.param(GPT_T_WDOWN, l), F, N, F, d, EPI_DRELU2, ws + L.du, F,
+                status);
+    g.b_mn_major = true; g.aux = Lb + L.lo.a;
+    GPT_TRY(run_gemm(*c, g, st));
+    g = gemm_kk(ws + L.dxs, d, Lb + L.lo.a, F, d, F, N, EPI_STORE, grad(GPT_T_WDOWN, l), F,
+                status);
+    g.a_mn_major = true; g.b_mn_major = true; g.beta = accumulate;
+    GPT_TRY(run_gemm(*c, with_splitk(g, L, ws), st));
     // MLP up
-    g = gemm_kk(ws + L.du, F, b.param(GPT_T_WUP, l), d, N, d, F, EPI_STORE, ws + L.dh, d);
-    g.b_mn_major = true; g.status = status;
-    GPT_TRY(launch_gemm(*c, g, st));
-    g = gemm_kk(ws + L.du, F, Lb + L.lo.h2, d, F, d, N, EPI_STORE, grad(GPT_T_WUP, l), d);
-    g.a_mn_major = true; g.b_mn_major = true; g.beta = accumulate; g.status = status;
-    GPT_TRY(launch_gemm(*c, g, st));
-    GPT_TRY(launch_rms_bwd(*c, ws + L.dh, Lb + L.lo.h2, reinterpret_cast<float*>(Lb + L.lo.r2),
-                           dx, ws + L.dxs, 1, st));
+    g = gemm_kk(ws + L.du, F, S.param(GPT_T_WUP, l), d, N, d, F, EPI_STORE, ws + L.dh, d, status);
+    g.b_mn_major = true;
+    GPT_TRY(run_gemm(*c, g, st));
+    g = gemm_kk(ws + L.du, F, Lb + L.lo.h2, d, F, d, N, EPI_STORE, grad(GPT_T_WUP, l), d, status);
+    g.a_mn_major = true; g.b_mn_major = true; g.beta = accumulate;
+    GPT_TRY(run_gemm(*c, with_splitk(g, L, ws), st));
+    GPT_TRY(S.rms_bwd(ws + L.dh, Lb + L.lo.h2, reinterpret_cast<float*>(Lb + L.lo.r2), 1));
     // attention out-projection
-    g = gemm_kk(ws + L.dxs, d, b.param(GPT_T_WO, l), d, N, d, d, EPI_STORE, ws + L.dO, d);
-    g.b_mn_major = true; g.status = status;
-    GPT_TRY(launch_gemm(*c, g, st));
-    g = gemm_kk(ws + L.dxs, d, Lb + L.lo.o, d, d, d, N, EPI_STORE, grad(GPT_T_WO, l), d);
-    g.a_mn_major = true; g.b_mn_major = true; g.beta = accumulate; g.status = status;
-    GPT_TRY(launch_gemm(*c, g, st));
+    g = gemm_kk(ws + L.dxs, d, S.param(GPT_T_WO, l), d, N, d, d, EPI_STORE, ws + L.dO, d, status);
+    g.b_mn_major = true;
+    GPT_TRY(run_gemm(*c, g, st));
+    g = gemm_kk(ws + L.dxs, d, Lb + L.lo.o, d, d, d, N, EPI_STORE, grad(GPT_T_WO, l), d, status);
+    g.a_mn_major = true; g.b_mn_major = true; g.beta = accumulate;
+    GPT_TRY(run_gemm(*c, with_splitk(g, L, ws), st));
     // attention, then QK-norm and RoPE backward, into dqkv [N, 3d]
-    GPT_TRY(launch_attn_bwd(*c, Lb + L.lo.q, Lb + L.lo.k, Lb + L.lo.v, Lb + L.lo.o, ws + L.dO,
-                            reinterpret_cast<float*>(Lb + L.lo.lse),
-                            reinterpret_cast<float*>(Lb + L.lo.rq),
-                            reinterpret_cast<float*>(Lb + L.lo.rk), cos_t, sin_t,
-                            reinterpret_cast<float*>(ws + L.Dattn), ws + L.dqkv, st));
-    g = gemm_kk(ws + L.dqkv, 3 * d, b.param(GPT_T_WQKV, l), d, N, d, 3 * d, EPI_STORE,
-                ws + L.dh, d);
-    g.b_mn_major = true; g.status = status;
-    GPT_TRY(launch_gemm(*c, g, st));
+    {
+      TraceScope ts(GPT_K_ATTN_BWD, c->dtype == GPT_BF16 ? 3 : 2, attn_b, S.nd() * esz * 8, st);
+      GPT_TRY(launch_attn_bwd(*c, Lb + L.lo.q, Lb + L.lo.k, Lb + L.lo.v, Lb + L.lo.o, ws + L.dO,
+                              reinterpret_cast<float*>(Lb + L.lo.lse),
+                              reinterpret_cast<float*>(Lb + L.lo.rq),
+                              reinterpret_cast<float*>(Lb + L.lo.rk), S.cos_t, S.sin_t,
+                              S.f(L.Dattn), ws + L.dqkv, S.status, st));
+    }
+    g = gemm_kk(ws + L.dqkv, 3 * d, S.param(GPT_T_WQKV, l), d, N, d, 3 * d, EPI_STORE, ws + L.dh,
+                d, status);
+    g.b_mn_major = true;
+    GPT_TRY(run_gemm(*c, g, st));
     g = gemm_kk(ws + L.dqkv, 3 * d, Lb + L.lo.h1, d, 3 * d, d, N, EPI_STORE,
-                grad(GPT_T_WQKV, l), d);
-    g.a_mn_major = true; g.b_mn_major = true; g.beta = accumulate; g.status = status;
-    GPT_TRY(launch_gemm(*c, g, st));
-    GPT_TRY(launch_rms_bwd(*c, ws + L.dh, Lb + L.lo.h1, reinterpret_cast<float*>(Lb + L.lo.r1),
-                           dx, ws + L.dxs, 1, st));
+                grad(GPT_T_WQKV, l), d, status);
+    g.a_mn_major = true; g.b_mn_major = true; g.beta = accumulate;
+    GPT_TRY(run_gemm(*c, with_splitk(g, L, ws), st));
+    GPT_TRY(S.rms_bwd(ws + L.dh, Lb + L.lo.h1, reinterpret_cast<float*>(Lb + L.lo.r1), 1));
   }
-  GPT_TRY(launch_embed_scatter(*c, L, dx, ws, grad(GPT_T_WTE, 0), accumulate, st));
+  {
+    TraceScope ts(GPT_K_SCATTER, 6, 0, S.nd() * 4 + double(V) * d * esz, st);
+    GPT_TRY(launch_embed_scatter(*c, L, S.x, ws, grad(GPT_T_WTE, 0), accumulate, st));
+  }
   return GPT_OK;
 }
 

@@ -88,13 +88,17 @@ __device__ __forceinline__ void epi_chunk(const GemmArgs& g, int row, int col0, 
           *reinterpret_cast<float4*>(o + j) = x;
         }
       } else {
-        for (int j = 0; j < 32 && col0 + j < g.N; ++j) o[j] += v[j];
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (col0 + j < g.N) o[j] += v[j];
       }
       return;
     }
     case EPI_STORE_F32: {
       float* o = static_cast<float*>(g.out) + base;
-      for (int j = 0; j < 32 && col0 + j < g.N; ++j) o[j] = v[j];
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (col0 + j < g.N) o[j] = v[j];
       return;
     }
     default:
@@ -117,6 +121,7 @@ __device__ __forceinline__ void epi_chunk(const GemmArgs& g, int row, int col0, 
             r[j + 6] = v[j + 6] + d.x; r[j + 7] = v[j + 7] + d.y;
           }
         } else {
+#pragma unroll
           for (int j = 0; j < 32; ++j) r[j] = v[j] + (col0 + j < g.N ? __bfloat162float(o[j]) : 0.f);
         }
       } else {
@@ -145,6 +150,7 @@ __device__ __forceinline__ void epi_chunk(const GemmArgs& g, int row, int col0, 
           r[j + 6] = v[j + 6] * 2.f * sqrtf(p3.x); r[j + 7] = v[j + 7] * 2.f * sqrtf(p3.y);
         }
       } else {
+#pragma unroll
         for (int j = 0; j < 32; ++j)
           r[j] = col0 + j < g.N ? v[j] * 2.f * sqrtf(__bfloat162float(a[j])) : 0.f;
       }
@@ -174,14 +180,17 @@ __device__ __forceinline__ void epi_chunk(const GemmArgs& g, int row, int col0, 
       *reinterpret_cast<uint4*>(o + j) = u;
     }
   } else {
-    for (int j = 0; j < 32 && col0 + j < g.N; ++j) o[j] = __float2bfloat16_rn(r[j]);
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (col0 + j < g.N) o[j] = __float2bfloat16_rn(r[j]);
   }
 }
 
 template <bool AMN, bool BMN>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a,
-                   const __grid_constant__ CUtensorMap map_b, const __grid_constant__ GemmArgs g) {
+                   const __grid_constant__ CUtensorMap map_b, const __grid_constant__ GemmArgs g,
+                   int splits) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -193,6 +202,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int m_tiles = (g.M + BM - 1) / BM, n_tiles = (g.N + BN - 1) / BN;
   const int num_tiles = m_tiles * n_tiles;
   const int num_kb = (g.K + BK - 1) / BK;
+  // work unit = (tile, K split); unit u covers k-blocks [kb_lo(u), kb_hi(u))
+  const int num_units = num_tiles * splits;
+  const int kb_per = (num_kb + splits - 1) / splits;
   constexpr uint32_t idesc = tc::idesc_bf16_f32(BM, BN, AMN, BMN);
 
   if (threadIdx.x == 0) {
@@ -228,9 +240,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued_mask = 0, last_parity = 0;
-      for (int tile = blockIdx.x; tile < num_tiles && !*abort; tile += gridDim.x) {
+      for (int unit = blockIdx.x; unit < num_units && !*abort; unit += gridDim.x) {
+        const int tile = unit / splits, sp = unit % splits;
         const int mb = tile / n_tiles, nb = tile % n_tiles;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        const int kb_hi = min(num_kb, (sp + 1) * kb_per);
+        for (int kb = sp * kb_per; kb < kb_hi; ++kb) {
           if (!tc::mbar_wait_bounded(&tail->empty[stage], phase ^ 1, abort, kWaitLimitNs)) {
             record_status(g.status, GPT_ETIMEOUT, K_GEMM_TC, 1);
             *abort = 1;
@@ -272,7 +286,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       int local = 0;
       bool issued_any = false;
-      for (int tile = blockIdx.x; tile < num_tiles && !*abort; tile += gridDim.x, ++local) {
+      for (int unit = blockIdx.x; unit < num_units && !*abort; unit += gridDim.x, ++local) {
+        const int sp = unit % splits;
+        const int kb_lo = sp * kb_per, kb_hi = min(num_kb, (sp + 1) * kb_per);
         const int acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
         if (!tc::mbar_wait_bounded(&tail->tmem_empty[acc], acc_phase ^ 1, abort, kWaitLimitNs)) {
@@ -282,7 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc::tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb = kb_lo; kb < kb_hi; ++kb) {
           if (!tc::mbar_wait_bounded(&tail->full[stage], phase, abort, kWaitLimitNs)) {
             record_status(g.status, GPT_ETIMEOUT, K_GEMM_TC, 3);
             *abort = 1;
@@ -297,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     : tc::smem_desc_sw128(a_addr + k * 32, 16);
             const uint64_t db = BMN ? tc::smem_desc_sw128(b_addr + k * 2048, 8192)
                                     : tc::smem_desc_sw128(b_addr + k * 32, 16);
-            tc::mma_bf16_ss(d_tmem, da, db, idesc, (kb | k) != 0);
+            tc::mma_bf16_ss(d_tmem, da, db, idesc, (kb != kb_lo) || k != 0);
           }
           issued_any = true;
           tc::mma_commit(&tail->empty[stage]);
@@ -316,7 +332,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- epilogue (warps 2..5) ----------------
     const int quarter = warp & 3;  // TMEM lanes accessible to this warp
     int local = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+    for (int unit = blockIdx.x; unit < num_units; unit += gridDim.x, ++local) {
+      const int tile = unit / splits, sp = unit % splits;
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
       const bool ok = tc::mbar_wait_bounded(&tail->tmem_full[acc], acc_phase, abort, kWaitLimitNs);
@@ -344,10 +361,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::tmem_wait_ld();
         const int col0 = nb * BN + c * 32;
         if (row_ok && col0 < g.N) {
-          float v[32];
+          if (splits > 1) {
+            // fp32 partial of this K split; the reduce kernel applies the epilogue
+            float* dst = g.splitk + (int64_t(sp) * g.M + row) * g.N + col0;
+            if (col0 + 32 <= g.N) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = u2f(u[j]);
-          epi_chunk(g, row, col0, v, ce_max, ce_sum, ce_tgt, tgt, lse_row);
+              for (int j = 0; j < 32; j += 4)
+                *reinterpret_cast<float4*>(dst + j) =
+                    make_float4(u2f(u[j]), u2f(u[j + 1]), u2f(u[j + 2]), u2f(u[j + 3]));
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (col0 + j < g.N) dst[j] = u2f(u[j]);
+            }
+          } else {
+            float v[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = u2f(u[j]);
+            epi_chunk(g, row, col0, v, ce_max, ce_sum, ce_tgt, tgt, lse_row);
+          }
         }
       }
       if (row_ok && g.epi == EPI_CE_FWD) {
@@ -404,7 +436,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
 }
 
 template <bool AMN, bool BMN>
-int launch_tc(const GemmArgs& g, int grid, cudaStream_t st) {
+int launch_tc(const GemmArgs& g, int grid, int splits, cudaStream_t st) {
   CUtensorMap ma, mb;
   bool ok = AMN ? make_map(&ma, g.A, g.M, g.K, g.lda, 64, 64)
                 : make_map(&ma, g.A, g.K, g.M, g.lda, 64, BM);
@@ -415,11 +447,60 @@ int launch_tc(const GemmArgs& g, int grid, cudaStream_t st) {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes)) !=
       cudaSuccess)
     return 1;
-  kern<<<grid, kThreads, kSmemBytes, st>>>(ma, mb, g);
+  kern<<<grid, kThreads, kSmemBytes, st>>>(ma, mb, g, splits);
   return last_launch_rc();
 }
 
+// out[i] (+)= sum_s partial[s][i], s in order 0..splits-1, stored as bf16
+__global__ void splitk_reduce_kernel(const float* __restrict__ part, __nv_bfloat16* __restrict__ out,
+                                     int64_t n4, int splits, int beta) {
+  const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n4) return;
+  float4 a = reinterpret_cast<const float4*>(part)[i];
+  for (int s = 1; s < splits; ++s) {
+    float4 b = reinterpret_cast<const float4*>(part + int64_t(s) * n4 * 4)[i];
+    a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+  }
+  uint2* o = reinterpret_cast<uint2*>(out) + i;
+  if (beta) {
+    uint2 prev = *o;
+    float2 p0 = unpack_bf16(prev.x), p1 = unpack_bf16(prev.y);
+    a.x += p0.x; a.y += p0.y; a.z += p1.x; a.w += p1.y;
+  }
+  *o = make_uint2(pack_bf16(a.x, a.y), pack_bf16(a.z, a.w));
+}
+
+int num_sms() {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
 }  // namespace
+
+// K splits for a GEMM: only plain stores into a contiguous [M, N] output with a
+// split-K buffer, and only when the tile count alone would leave SMs idle; the
+// smallest split count that fills >= 90 % of the SM waves, keeping >= 8 k-blocks
+// per split and the partials within the buffer.
+int gemm_tc_splits(const GemmArgs& g) {
+  if (g.epi != EPI_STORE || !g.splitk || g.ldo != g.N || (g.N & 3)) return 1;
+  const int sms = num_sms();
+  const int tiles = ((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN);
+  const int num_kb = (g.K + BK - 1) / BK;
+  if (tiles >= 3 * sms) return 1;
+  int best = 1;
+  double best_eff = 0.0;
+  for (int s = 1; s <= 4; ++s) {
+    if (num_kb / s < 8 || int64_t(s) * g.M * g.N > g.splitk_floats) break;
+    const int units = tiles * s;
+    const int waves = (units + sms - 1) / sms;
+    const double eff = double(units) / (double(waves) * sms);
+    if (eff > best_eff + 1e-9) { best_eff = eff; best = s; }
+    if (eff >= 0.9) break;
+  }
+  return best;
+}
 
 int launch_gemm_tc(const GemmArgs& g_in, void* stream) {
   GemmArgs g = g_in;
@@ -427,14 +508,25 @@ int launch_gemm_tc(const GemmArgs& g_in, void* stream) {
   if (g.M <= 0 || g.N <= 0 || g.K <= 0) return 0;
   const int tiles = ((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN);
   if (g.epi == EPI_CE_FWD) g.n_part = (g.N + BN - 1) / BN;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int grid = tiles < sms ? tiles : sms;
-  if (!g.a_mn_major && !g.b_mn_major) return launch_tc<false, false>(g, grid, st);
-  if (!g.a_mn_major && g.b_mn_major) return launch_tc<false, true>(g, grid, st);
-  if (g.a_mn_major && g.b_mn_major) return launch_tc<true, true>(g, grid, st);
-  return launch_tc<true, false>(g, grid, st);
+  int splits = gemm_tc_splits(g);
+  if (splits > 1) {  // every split non-empty: ceil(num_kb / ceil(num_kb / splits)) splits
+    const int num_kb = (g.K + BK - 1) / BK;
+    const int kb_per = (num_kb + splits - 1) / splits;
+    splits = (num_kb + kb_per - 1) / kb_per;
+  }
+  const int sms = num_sms();
+  const int units = tiles * splits;
+  const int grid = units < sms ? units : sms;
+  int rc;
+  if (!g.a_mn_major && !g.b_mn_major) rc = launch_tc<false, false>(g, grid, splits, st);
+  else if (!g.a_mn_major && g.b_mn_major) rc = launch_tc<false, true>(g, grid, splits, st);
+  else if (g.a_mn_major && g.b_mn_major) rc = launch_tc<true, true>(g, grid, splits, st);
+  else rc = launch_tc<true, false>(g, grid, splits, st);
+  if (rc || splits == 1) return rc;
+  const int64_t n4 = int64_t(g.M) * g.N / 4;
+  splitk_reduce_kernel<<<int((n4 + 255) / 256), 256, 0, st>>>(
+      g.splitk, static_cast<__nv_bfloat16*>(g.out), n4, splits, g.beta);
+  return last_launch_rc();
 }
 
 int gemm_tc_tile_n() { return BN; }

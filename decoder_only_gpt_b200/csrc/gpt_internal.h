@@ -52,6 +52,9 @@ struct GemmArgs {
   float inv_n;
   int n_valid;              // columns >= n_valid are padding (EPI_CE_BWD writes 0)
   int32_t* status;          // device status word
+  // split-K (tensor-core GEMM, EPI_STORE only): fp32 partials [splits][M][N]
+  float* splitk;
+  int64_t splitk_floats;    // capacity of `splitk`
 };
 
 struct LayerOffsets {
@@ -71,6 +74,8 @@ struct Layout {
   uint64_t qkv_raw;
   uint64_t part_max, part_sum, tgt_logit, lse_z, tok_loss, loss_acc;
   uint64_t G, dh, du, dO, dqkv, Dattn;
+  uint64_t splitk;          // fp32 split-K partials
+  int64_t splitk_floats;
   uint64_t sort_perm, sort_offs, sort_count, sort_tilehist, scat_items, scat_item_offs,
       scat_partial;
   int64_t n_part_max;      // partial-stat columns reserved per row
@@ -97,16 +102,18 @@ int launch_ce_merge(const gpt_config& c, const float* part_max, const float* par
 int launch_loss_mean(const gpt_config& c, const float* tok_loss, float* loss,
                      float* user_tok_loss, int32_t* status, void* stream);
 int launch_attn_fwd(const gpt_config& c, const void* q, const void* k, const void* v, void* o,
-                    float* lse, void* stream);
+                    float* lse, int32_t* status, void* stream);
 int launch_attn_bwd(const gpt_config& c, const void* q, const void* k, const void* v,
                     const void* o, const void* dO, const float* lse, const float* rq,
                     const float* rk, const float* cos_t, const float* sin_t, float* Dbuf,
-                    void* dqkv, void* stream);
+                    void* dqkv, int32_t* status, void* stream);
 int launch_sort_tokens(const gpt_config& c, const Layout& L, const int32_t* tok, char* ws,
                        void* stream);
 int launch_embed_scatter(const gpt_config& c, const Layout& L, const float* dx0, char* ws,
                          void* dwte, int accumulate, void* stream);
 int launch_gemm(const gpt_config& c, const GemmArgs& g, void* stream);
+// Number of kernels launch_gemm enqueues for these arguments (2 with a split-K reduce).
+int gemm_kernel_count(const gpt_config& c, const GemmArgs& g);
 // Column width of the GEMM tile that produces the logits (partial-statistics granularity).
 int gemm_ce_tile_n(const gpt_config& c);
 

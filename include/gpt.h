@@ -172,6 +172,47 @@ const char* gpt_strerror(int code);
 /* Library version string. */
 const char* gpt_version(void);
 
+/* ---- tracing (optional; per-launch CUDA events) ------------------------------
+ * A trace records a CUDA event pair around every kernel launch that
+ * gpt_forward_loss / gpt_backward / gpt_train_step_host make from the calling
+ * host thread while the trace is attached, on the stream the kernels run on,
+ * tagged with the kernel class below and the launch's algorithmic FLOPs and
+ * HBM bytes (the minimum the operation must move).  The caller owns the trace;
+ * recording stops silently once `capacity` launches are held (the count of
+ * dropped launches is reported). */
+#define GPT_K_GEMM 0      /* tensor-core (bf16) or SIMT (fp32) GEMM           */
+#define GPT_K_ATTN_FWD 1  /* causal attention forward                         */
+#define GPT_K_ATTN_BWD 2  /* causal attention backward (+QK-norm/RoPE bwd)    */
+#define GPT_K_NORM 3      /* embedding gather + RMSNorm, RMSNorm fwd / bwd    */
+#define GPT_K_QKV 4       /* RoPE + QK-norm + head-major scatter of q, k, v   */
+#define GPT_K_LOSS 5      /* cross-entropy merge and loss mean                */
+#define GPT_K_SORT 6      /* stable counting sort of positions by token id    */
+#define GPT_K_SCATTER 7   /* embedding-gradient scatter-add                   */
+#define GPT_K_OTHER 8     /* RoPE table, status reset                          */
+#define GPT_K_COUNT 9
+
+typedef struct gpt_trace gpt_trace;
+
+typedef struct gpt_trace_stat {
+  int32_t launches;  /* launcher calls recorded                               */
+  int32_t kernels;   /* CUDA kernels (and memsets) those calls enqueued        */
+  double ms;         /* summed event-pair durations                           */
+  double flops;      /* summed algorithmic FLOPs                               */
+  double bytes;      /* summed algorithmic HBM bytes                           */
+} gpt_trace_stat;
+
+/* Create a trace with room for `capacity` launches (creates 2*capacity CUDA
+ * events on the current device). */
+int gpt_trace_create(gpt_trace** trace, int capacity);
+/* Attach `trace` to the calling host thread (NULL detaches). */
+int gpt_trace_attach(gpt_trace* trace);
+/* Forget every recorded launch (events are kept for reuse). */
+int gpt_trace_reset(gpt_trace* trace);
+/* Wait for the recorded events and fill stats[GPT_K_COUNT] (one per class);
+ * *dropped receives the number of launches not recorded for lack of room. */
+int gpt_trace_summary(gpt_trace* trace, gpt_trace_stat* stats, int32_t* dropped);
+int gpt_trace_destroy(gpt_trace* trace);
+
 #ifdef __cplusplus
 }
 #endif

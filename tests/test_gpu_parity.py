@@ -40,6 +40,9 @@ CASES = {
     # head_dim 128 with two heads, odd batch
     "hd128": ("d4", dict(n_layer=1, d_model=256, n_head=2, head_dim=128, d_ff=512, vocab=2048,
                          seq_len=192, batch=3)),
+    # head_dim 128 with a ragged sequence (150 = two 64-key steps + 22), vocab 700
+    "ragged_hd128": ("d4", dict(n_layer=2, d_model=256, n_head=2, head_dim=128, d_ff=512,
+                                vocab=700, seq_len=150, batch=2)),
     # fp32 ragged
     "tiny_ragged": ("tiny", dict(seq_len=37, batch=3, vocab=100, d_ff=96)),
 }
