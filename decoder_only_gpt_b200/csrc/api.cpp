@@ -76,7 +76,7 @@ bool make_layout(const gpt_config& c, Layout* L) {
   L->layer_base = b.take(L->layer_stride * uint64_t(c.n_layer));
   L->hf = b.take(N * d * esz);
   L->rf = b.take(N * 4);
-  L->qkv_raw = b.take(N * 3 * d * esz);
+  L->qkv_raw = b.take(c.dtype == GPT_F32 ? N * 3 * d * esz : 0);  // bf16: fused into the GEMM
   // cross-entropy partials: the narrowest GEMM tile used for the logits is 64 columns
   L->n_part_max = (V + 63) / 64;
   L->part_max = b.take(N * L->n_part_max * 4);
@@ -275,6 +275,7 @@ static int run_gemm(const gpt_config& c, const GemmArgs& g, cudaStream_t st) {
     case EPI_RESID_F32: bytes += mn * 8; break;
     case EPI_DRELU2: bytes += mn * e * 2; break;
     case EPI_CE_FWD: bytes += double(g.M) * 12; break;
+    case EPI_QKV: bytes += mn * e + double(g.M) * 2 * g.n_head * 4; break;
     default: bytes += mn * e; break;
   }
   TraceScope ts(GPT_K_GEMM, gemm_kernel_count(c, g), 2.0 * double(g.M) * g.N * g.K, bytes, st);
@@ -354,9 +355,20 @@ int gpt_forward_loss(const gpt_config* c, const int32_t* tok, const int32_t* tgt
   const double attn_f = 4.0 * attn_pairs(*c) * c->head_dim;  // QK^T and PV, causal half
   for (int l = 0; l < c->n_layer; ++l) {
     char* Lb = S.layer(l);
-    GPT_TRY(run_gemm(*c, gemm_kk(Lb + L.lo.h1, d, S.param(GPT_T_WQKV, l), d, N, 3 * d, d,
-                                 EPI_STORE, ws + L.qkv_raw, 3 * d, S.status), st));
-    {
+    if (c->dtype == GPT_BF16) {
+      // QKV projection with RoPE, QK-norm and the head-major scatter in its epilogue
+      GemmArgs g = gemm_kk(Lb + L.lo.h1, d, S.param(GPT_T_WQKV, l), d, N, 3 * d, d, EPI_QKV,
+                           nullptr, 3 * d, S.status);
+      g.q_out = Lb + L.lo.q; g.k_out = Lb + L.lo.k; g.v_out = Lb + L.lo.v;
+      g.rq = reinterpret_cast<float*>(Lb + L.lo.rq);
+      g.rk = reinterpret_cast<float*>(Lb + L.lo.rk);
+      g.rope_cos = S.cos_t; g.rope_sin = S.sin_t;
+      g.seq_len = c->seq_len; g.n_head = c->n_head; g.head_dim = c->head_dim;
+      g.qk_norm = c->qk_norm; g.norm_eps = c->norm_eps;
+      GPT_TRY(run_gemm(*c, g, st));
+    } else {
+      GPT_TRY(run_gemm(*c, gemm_kk(Lb + L.lo.h1, d, S.param(GPT_T_WQKV, l), d, N, 3 * d, d,
+                                   EPI_STORE, ws + L.qkv_raw, 3 * d, S.status), st));
       TraceScope ts(GPT_K_QKV, 1, 0, S.nd() * 3 * esz * 2, st);
       GPT_TRY(launch_qkv_post(*c, ws + L.qkv_raw, S.cos_t, S.sin_t, Lb + L.lo.q, Lb + L.lo.k,
                               Lb + L.lo.v, reinterpret_cast<float*>(Lb + L.lo.rq),

@@ -186,6 +186,86 @@ __device__ __forceinline__ void epi_chunk(const GemmArgs& g, int row, int col0, 
   }
 }
 
+// EPI_QKV: the tile's 256 columns hold whole heads (head_dim 64 or 128 divides
+// 256).  For each head of this row: v is copied to its head-major row; q and k
+// are rotated by RoPE (pairs (i, i + hd/2)), scaled by 1/rms of the rotated row
+// (the rotation keeps the norm, so the sum of squares is taken on the raw row)
+// and written head-major, with the 1/rms kept for the backward.
+__device__ __forceinline__ void epi_qkv_row(const GemmArgs& g, uint32_t taddr, int row, int nb,
+                                            bool row_ok) {
+  const int hd = g.head_dim, half = hd / 2, H = g.n_head, d = H * hd, T = g.seq_len;
+  const int b = row_ok ? row / T : 0, t = row_ok ? row % T : 0;
+  for (int seg = 0; seg < BN / hd; ++seg) {
+    const int c0 = nb * BN + seg * hd;
+    if (c0 >= g.N) break;  // uniform across the warp
+    const int part = c0 / d, h = (c0 % d) / hd;
+    const uint32_t tcol = taddr + seg * hd;
+    const int64_t dst = ((int64_t(b) * H + h) * T + t) * hd;
+    if (part == 2) {
+      __nv_bfloat16* vo = static_cast<__nv_bfloat16*>(g.v_out) + dst;
+      for (int c = 0; c < hd; c += 32) {
+        uint32_t u[32];
+        tc::tmem_ld_32x32b_x32(tcol + c, u);
+        tc::tmem_wait_ld();
+        if (!row_ok) continue;
+#pragma unroll
+        for (int i = 0; i < 32; i += 8)
+          *reinterpret_cast<uint4*>(vo + c + i) =
+              make_uint4(pack_bf16(u2f(u[i]), u2f(u[i + 1])), pack_bf16(u2f(u[i + 2]), u2f(u[i + 3])),
+                         pack_bf16(u2f(u[i + 4]), u2f(u[i + 5])), pack_bf16(u2f(u[i + 6]), u2f(u[i + 7])));
+      }
+      continue;
+    }
+    float ss = 0.f;
+    for (int c = 0; c < hd; c += 32) {
+      uint32_t u[32];
+      tc::tmem_ld_32x32b_x32(tcol + c, u);
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) ss = fmaf(u2f(u[i]), u2f(u[i]), ss);
+    }
+    const float r = g.qk_norm ? rsqrtf(ss / float(hd) + g.norm_eps) : 1.f;
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(part == 0 ? g.q_out : g.k_out) + dst;
+    const float* cr = g.rope_cos + int64_t(t) * half;
+    const float* sr = g.rope_sin + int64_t(t) * half;
+    for (int i0 = 0; i0 < half; i0 += 16) {
+      uint32_t ua[16], ub[16];
+      tc::tmem_ld_32x32b_x16(tcol + i0, ua);
+      tc::tmem_ld_32x32b_x16(tcol + half + i0, ub);
+      tc::tmem_wait_ld();
+      if (!row_ok) continue;
+      float cv[16], sv[16];
+#pragma unroll
+      for (int e = 0; e < 16; e += 4) {
+        const float4 c4 = *reinterpret_cast<const float4*>(cr + i0 + e);
+        const float4 s4 = *reinterpret_cast<const float4*>(sr + i0 + e);
+        cv[e] = c4.x; cv[e + 1] = c4.y; cv[e + 2] = c4.z; cv[e + 3] = c4.w;
+        sv[e] = s4.x; sv[e + 1] = s4.y; sv[e + 2] = s4.z; sv[e + 3] = s4.w;
+      }
+      uint32_t pa[8], pb[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float c0v = cv[2 * e], c1v = cv[2 * e + 1];
+        const float s0v = sv[2 * e], s1v = sv[2 * e + 1];
+        const float a0 = u2f(ua[2 * e]), a1 = u2f(ua[2 * e + 1]);
+        const float b0 = u2f(ub[2 * e]), b1 = u2f(ub[2 * e + 1]);
+        pa[e] = pack_bf16((a0 * c0v - b0 * s0v) * r, (a1 * c1v - b1 * s1v) * r);
+        pb[e] = pack_bf16((a0 * s0v + b0 * c0v) * r, (a1 * s1v + b1 * c1v) * r);
+      }
+      uint4* oa = reinterpret_cast<uint4*>(out + i0);
+      uint4* ob = reinterpret_cast<uint4*>(out + half + i0);
+      oa[0] = make_uint4(pa[0], pa[1], pa[2], pa[3]);
+      oa[1] = make_uint4(pa[4], pa[5], pa[6], pa[7]);
+      ob[0] = make_uint4(pb[0], pb[1], pb[2], pb[3]);
+      ob[1] = make_uint4(pb[4], pb[5], pb[6], pb[7]);
+    }
+    if (row_ok) {
+      const int64_t ri = (int64_t(b) * H + h) * T + t;
+      (part == 0 ? g.rq : g.rk)[ri] = r;
+    }
+  }
+}
+
 template <bool AMN, bool BMN>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a,
@@ -354,6 +434,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       float ce_max = -INFINITY, ce_sum = 0.f, ce_tgt = 0.f;
       const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + acc * BN;
+      if (g.epi == EPI_QKV) {
+        epi_qkv_row(g, taddr, row, nb, row_ok);
+        tc::tc_fence_before();
+        tc::mbar_arrive(&tail->tmem_empty[acc]);
+        continue;
+      }
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t u[32];

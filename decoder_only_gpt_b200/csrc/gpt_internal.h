@@ -27,6 +27,7 @@ enum Epilogue : int32_t {
   EPI_DRELU2,       // out_t = acc * 2*sqrt(aux_t)    (ReLU^2' from the stored activation)
   EPI_CE_FWD,       // per-row partial (max, sum exp) over the tile's columns + target logit
   EPI_CE_BWD,       // out_t = (exp(acc - lse[m]) - [n == tgt[m]]) * inv_n; 0 for n >= n_valid
+  EPI_QKV,          // [q|k|v] row: RoPE + per-head RMSNorm of q, k; head-major scatter of q, k, v
 };
 
 struct GemmArgs {
@@ -52,6 +53,16 @@ struct GemmArgs {
   float inv_n;
   int n_valid;              // columns >= n_valid are padding (EPI_CE_BWD writes 0)
   int32_t* status;          // device status word
+  // EPI_QKV (rows = tokens b*T + t, columns = [q | k | v] of n_head heads of head_dim)
+  void* q_out;
+  void* k_out;
+  void* v_out;              // [B, H, T, hd] each
+  float* rq;
+  float* rk;                // [B, H, T]: 1/rms of the rotated q, k rows
+  const float* rope_cos;
+  const float* rope_sin;    // [T, hd/2]
+  int seq_len, n_head, head_dim, qk_norm;
+  float norm_eps;
   // split-K (tensor-core GEMM, EPI_STORE only): fp32 partials [splits][M][N]
   float* splitk;
   int64_t splitk_floats;    // capacity of `splitk`

@@ -104,10 +104,60 @@ __global__ void rms_fwd_kernel(const float* __restrict__ x, T* __restrict__ h,
   if (lane == 0) r[row] = rr;
 }
 
+// bf16 output, d % 8 == 0 and d <= 8 * 32 * kMaxVec: 16-byte accesses, the row in registers.
+constexpr int kMaxVec = 8;  // 8-element groups per lane: d <= 2048
+
+__device__ __forceinline__ uint32_t pk_bf16(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float2 up_bf16(uint32_t u) {
+  return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u));
+}
+__device__ __forceinline__ void up8(const uint4& u, float (&f)[8]) {
+  float2 a = up_bf16(u.x), b = up_bf16(u.y), c = up_bf16(u.z), d = up_bf16(u.w);
+  f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y; f[4] = c.x; f[5] = c.y; f[6] = d.x; f[7] = d.y;
+}
+
+__global__ void rms_fwd_bf16_vec(const float* __restrict__ x, __nv_bfloat16* __restrict__ h,
+                                 float* __restrict__ r, int64_t N, int d, float eps) {
+  const int64_t row = int64_t(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (row >= N) return;
+  const int groups = d / 8;
+  const float4* xr = reinterpret_cast<const float4*>(x + row * d);
+  float4 va[kMaxVec], vb[kMaxVec];
+  float ss = 0.f;
+#pragma unroll
+  for (int k = 0; k < kMaxVec; ++k) {
+    const int gi = lane + 32 * k;
+    if (gi < groups) {
+      va[k] = xr[2 * gi];
+      vb[k] = xr[2 * gi + 1];
+      ss += va[k].x * va[k].x + va[k].y * va[k].y + va[k].z * va[k].z + va[k].w * va[k].w +
+            vb[k].x * vb[k].x + vb[k].y * vb[k].y + vb[k].z * vb[k].z + vb[k].w * vb[k].w;
+    }
+  }
+  ss = warp_sum(ss);
+  const float rr = rsqrtf(ss / float(d) + eps);
+  uint4* hr = reinterpret_cast<uint4*>(h + row * d);
+#pragma unroll
+  for (int k = 0; k < kMaxVec; ++k) {
+    const int gi = lane + 32 * k;
+    if (gi < groups)
+      hr[gi] = make_uint4(pk_bf16(va[k].x * rr, va[k].y * rr), pk_bf16(va[k].z * rr, va[k].w * rr),
+                          pk_bf16(vb[k].x * rr, vb[k].y * rr), pk_bf16(vb[k].z * rr, vb[k].w * rr));
+  }
+  if (lane == 0) r[row] = rr;
+}
+
 int launch_rms_fwd(const gpt_config& c, const float* x, void* h, float* r, void* stream) {
   int64_t N = int64_t(c.batch) * c.seq_len;
   dim3 grid(ceil_div(N, 8));
-  if (c.dtype == GPT_BF16)
+  if (c.dtype == GPT_BF16 && c.d_model % 8 == 0 && c.d_model <= 8 * 32 * kMaxVec)
+    rms_fwd_bf16_vec<<<grid, 256, 0, (cudaStream_t)stream>>>(x, (__nv_bfloat16*)h, r, N,
+                                                            c.d_model, c.norm_eps);
+  else if (c.dtype == GPT_BF16)
     rms_fwd_kernel<__nv_bfloat16><<<grid, 256, 0, (cudaStream_t)stream>>>(
         x, (__nv_bfloat16*)h, r, N, c.d_model, c.norm_eps);
   else
@@ -143,11 +193,66 @@ __global__ void rms_bwd_kernel(const T* __restrict__ dh, const T* __restrict__ h
   }
 }
 
+__global__ void rms_bwd_bf16_vec(const __nv_bfloat16* __restrict__ dh,
+                                 const __nv_bfloat16* __restrict__ h, const float* __restrict__ r,
+                                 float* __restrict__ dx, __nv_bfloat16* __restrict__ dxs,
+                                 int64_t N, int d, int accumulate) {
+  const int64_t row = int64_t(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (row >= N) return;
+  const int groups = d / 8;
+  const uint4* dr = reinterpret_cast<const uint4*>(dh + row * d);
+  const uint4* hr = reinterpret_cast<const uint4*>(h + row * d);
+  uint4 gd[kMaxVec], gh[kMaxVec];
+  float s = 0.f;
+#pragma unroll
+  for (int k = 0; k < kMaxVec; ++k) {
+    const int gi = lane + 32 * k;
+    if (gi < groups) {
+      gd[k] = dr[gi];
+      gh[k] = hr[gi];
+      float fa[8], fb[8];
+      up8(gd[k], fa);
+      up8(gh[k], fb);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s += fa[e] * fb[e];
+    }
+  }
+  s = warp_sum(s) / float(d);
+  const float rr = r[row];
+  float4* xr = reinterpret_cast<float4*>(dx + row * d);
+  uint4* sr = reinterpret_cast<uint4*>(dxs + row * d);
+#pragma unroll
+  for (int k = 0; k < kMaxVec; ++k) {
+    const int gi = lane + 32 * k;
+    if (gi < groups) {
+      float fa[8], fb[8], g[8];
+      up8(gd[k], fa);
+      up8(gh[k], fb);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) g[e] = rr * (fa[e] - fb[e] * s);
+      if (accumulate) {
+        const float4 p0 = xr[2 * gi], p1 = xr[2 * gi + 1];
+        g[0] += p0.x; g[1] += p0.y; g[2] += p0.z; g[3] += p0.w;
+        g[4] += p1.x; g[5] += p1.y; g[6] += p1.z; g[7] += p1.w;
+      }
+      xr[2 * gi] = make_float4(g[0], g[1], g[2], g[3]);
+      xr[2 * gi + 1] = make_float4(g[4], g[5], g[6], g[7]);
+      sr[gi] = make_uint4(pk_bf16(g[0], g[1]), pk_bf16(g[2], g[3]), pk_bf16(g[4], g[5]),
+                          pk_bf16(g[6], g[7]));
+    }
+  }
+}
+
 int launch_rms_bwd(const gpt_config& c, const void* dh, const void* h, const float* r,
                    float* dx, void* dxs, int accumulate, void* stream) {
   int64_t N = int64_t(c.batch) * c.seq_len;
   dim3 grid(ceil_div(N, 8));
-  if (c.dtype == GPT_BF16)
+  if (c.dtype == GPT_BF16 && c.d_model % 8 == 0 && c.d_model <= 8 * 32 * kMaxVec)
+    rms_bwd_bf16_vec<<<grid, 256, 0, (cudaStream_t)stream>>>(
+        (const __nv_bfloat16*)dh, (const __nv_bfloat16*)h, r, dx, (__nv_bfloat16*)dxs, N,
+        c.d_model, accumulate);
+  else if (c.dtype == GPT_BF16)
     rms_bwd_kernel<__nv_bfloat16><<<grid, 256, 0, (cudaStream_t)stream>>>(
         (const __nv_bfloat16*)dh, (const __nv_bfloat16*)h, r, dx, (__nv_bfloat16*)dxs, N,
         c.d_model, accumulate);
