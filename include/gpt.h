@@ -172,6 +172,31 @@ const char* gpt_strerror(int code);
 /* Library version string. */
 const char* gpt_version(void);
 
+/* Embedding-gradient scatter-add without any device allocation.  No passage of
+ * the pages corresponds to this call; it exists for callers that cannot
+ * allocate device memory when they need the gradient (their device memory
+ * all comes from a host framework's pool, or their memory budget is fixed up
+ * front) and so cannot provide a gpt_config workspace either.
+ *   tokens: device int32 [n_tokens];  dx0: device fp32 [n_tokens, d_model]
+ *   (the gradient w.r.t. the gathered embeddings);  dwte: device [vocab,
+ *   d_model], bf16 (dtype GPT_BF16) or fp32 (GPT_F32);  accumulate: 0 writes
+ *   dwte (rows no token hits become 0), 1 adds to it.
+ * Result: dwte[v] (+)= sum over positions n with tokens[n] == v of dx0[n],
+ * summed in the same fixed order as the wte gradient of gpt_backward, so the
+ * two agree bit for bit.  Tokens outside [0, vocab) count as id 0.
+ * Scratch: one 16 MiB array in device memory defined by the library, held by
+ * every GPU that loads the library until the process exits.  The first call
+ * on a device looks up that array's device address (cudaGetSymbolAddress) with
+ * the device current; make that first call before any stream capture.  All
+ * calls share the array, so calls that may overlap on the same GPU (for
+ * example on different streams) race: serialise them.  Sizes
+ * whose scratch exceeds 16 MiB (about n_tokens * (8 + 8 d_model / 64) +
+ * vocab * (4 n_tokens / 1024 + 28) bytes) return GPT_EUNSUPPORTED; NULL or
+ * non-16-byte-aligned pointers GPT_EINVAL; enqueue failures GPT_ECUDA. */
+int gpt_embedding_grad_noalloc(const int32_t* tokens, int64_t n_tokens, int32_t vocab,
+                               int32_t d_model, int32_t dtype, const float* dx0, void* dwte,
+                               int accumulate, void* stream);
+
 /* ---- tracing (optional; per-launch CUDA events) ------------------------------
  * A trace records a CUDA event pair around every kernel launch that
  * gpt_forward_loss / gpt_backward / gpt_train_step_host make from the calling

@@ -1,0 +1,109 @@
+"""gpt_embedding_grad_noalloc: the embedding-gradient scatter for callers that
+cannot allocate device memory, checked against the wte gradient that
+gpt_backward computes through its own workspace.
+
+The call uses a scratch array the library keeps in device memory, so its
+result must equal gpt_backward's bit for bit (same kernels, same fixed
+summation order) and, in any case, lie within the gradient tolerance of the
+other GPU tests (cosine >= 0.999, max-rel <= 3e-2).  It is called twice in a
+row on the same output buffer, pre-filled with different garbage each time,
+to show that the shared scratch carries nothing over between calls.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+
+import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def mods():
+    from decoder_only_gpt_b200 import build
+    build.build()
+    from decoder_only_gpt_b200 import binding, runtime
+    return binding, runtime
+
+
+def _entry(B):
+    f = B.lib().gpt_embedding_grad_noalloc
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    return f
+
+
+def _metrics(g, r):
+    g, r = g.ravel(), r.ravel()
+    cos = float(np.dot(g, r) / (np.linalg.norm(g) * np.linalg.norm(r)))
+    return cos, float(np.max(np.abs(g - r)) / np.max(np.abs(r)))
+
+
+CASES = {
+    # 300 tokens, vocab 1000: a ragged sort tile, many empty rows
+    "ragged": ("story", dict(n_layer=1, d_model=128, n_head=2, head_dim=64, d_ff=256, vocab=1000,
+                             seq_len=100, batch=3)),
+    # full depth-24 token / vocabulary / width sizes (one layer keeps it quick)
+    "d24_sizes": ("d24", dict(n_layer=1)),
+}
+
+
+@pytest.mark.parametrize("case", list(CASES))
+def test_noalloc_matches_backward_twice(mods, case):
+    import torch
+    B, R = mods
+    base, kw = CASES[case]
+    w = synth.workload(base, **kw)
+    cfg = B.config_from_workload(w)
+    st = R.TrainStep(cfg)
+    st.load_params(synth.make_params(w, as_bits=True))
+    tok, tgt = synth.make_tokens(w)
+    st.set_batch(tok, tgt)
+    st.step()
+    assert st.status() == B.GPT_OK
+    # after gpt_backward the residual region holds d loss / d x0 (fp32 [N, d])
+    off, nb = B.workspace_region(cfg, B.GPT_W_RESID)
+    dx0 = st.workspace[off:off + nb]
+    want_bits = B.unpack_flat(cfg, st.grads.cpu().numpy().view(np.uint16))["wte"].copy()
+    want = st.grads_f64()["wte"]
+
+    f = _entry(B)
+    N, V, d = w.batch * w.seq_len, w.vocab, w.d_model
+    out = torch.empty(V * d, dtype=torch.int16, device=st.device)
+    for garbage in (0x7FC0, 0x3F80):  # NaN, then 1.0: every row must be overwritten
+        out.fill_(garbage)
+        rc = f(st.tokens.data_ptr(), N, V, d, B.GPT_BF16, dx0.data_ptr(), out.data_ptr(), 0,
+               st.stream)
+        assert rc == B.GPT_OK, B.strerror(rc)
+        torch.cuda.synchronize()
+        got_bits = out.cpu().numpy().view(np.uint16).reshape(V, d)
+        got = (got_bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        cos, mr = _metrics(got, want)
+        assert cos >= 0.999 and mr <= 3e-2, (cos, mr)
+        assert np.array_equal(got_bits, want_bits)
+
+
+def test_noalloc_accumulate_and_limits(mods):
+    import torch
+    B, R = mods
+    f = _entry(B)
+    dev = torch.device("cuda")
+    N, V, d = 500, 300, 64
+    rng = np.random.default_rng(0)
+    tok = torch.from_numpy(rng.integers(0, V, N).astype(np.int32)).to(dev)
+    dx0 = torch.from_numpy(rng.standard_normal((N, d)).astype(np.float32)).to(dev)
+    out = torch.zeros(V * d, dtype=torch.float32, device=dev)
+    s = torch.cuda.current_stream().cuda_stream
+    assert f(tok.data_ptr(), N, V, d, B.GPT_F32, dx0.data_ptr(), out.data_ptr(), 0, s) == 0
+    assert f(tok.data_ptr(), N, V, d, B.GPT_F32, dx0.data_ptr(), out.data_ptr(), 1, s) == 0
+    torch.cuda.synchronize()
+    ref = np.zeros((V, d))
+    np.add.at(ref, tok.cpu().numpy(), dx0.cpu().numpy().astype(np.float64))
+    cos, mr = _metrics(out.cpu().numpy().reshape(V, d).astype(np.float64), 2 * ref)
+    assert cos >= 0.99999 and mr <= 1e-5, (cos, mr)
+    # scratch larger than the fixed array: rejected before any launch
+    assert f(tok.data_ptr(), 1 << 22, 1 << 20, 4096, B.GPT_F32, dx0.data_ptr(), out.data_ptr(),
+             0, s) == B.GPT_EUNSUPPORTED
+    assert f(None, N, V, d, B.GPT_F32, dx0.data_ptr(), out.data_ptr(), 0, s) == B.GPT_EINVAL
