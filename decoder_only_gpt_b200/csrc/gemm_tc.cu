@@ -1,19 +1,26 @@
 // bf16 GEMM on the sm_100a tensor cores: C[m,n] = sum_k A(m,k) B(n,k), fp32
 // accumulation in tensor memory, with the fused epilogues of the step.
 //
-// Design (one CTA per SM, persistent over output tiles):
-//   tile 128 x 256, K-block 64 (one 128-byte swizzle atom), 4-stage smem ring;
-//   warp 0      TMA producer: A and B tiles -> smem, mbarrier complete_tx;
-//   warp 1      one thread issues tcgen05.mma (M=128, N=256, K=16) into one of
-//               two 256-column fp32 accumulators in TMEM (512 columns), and
-//               tcgen05.commit frees smem stages / hands accumulators over;
-//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time (thread = row),
-//               apply the epilogue, store to global.  Double-buffered TMEM
-//               lets the epilogue of tile i overlap the MMAs of tile i+1.
-// Either operand may be K-major (forward: X W^T) or MN-major (dgrad reads W
-// as stored, wgrad reads dY and X as stored), selected per operand through
-// the TMA box shape, the smem descriptor and the instruction descriptor.
-// Every wait is bounded (GPT_ETIMEOUT recorded in the status word).
+// Design: clusters of two CTAs (one per SM), persistent over 256 x 256 output
+// tiles, K-block 64 (one 128-byte swizzle atom), 6-stage shared-memory ring:
+//   warp 0      TMA producer of each CTA: its 128 rows of A and its 128
+//               columns of B per stage; both CTAs' loads complete on the
+//               first CTA's stage barrier;
+//   warp 1      one thread of the first CTA issues tcgen05.mma.cta_group::2
+//               (M=256, N=256, K=16) reading both CTAs' shared memory into one
+//               of two 256-column fp32 accumulators (each CTA's TMEM holds its
+//               128 rows; 512 columns), and tcgen05.commit frees stages in both
+//               CTAs / hands the accumulator to both epilogues;
+//   warps 2..5  epilogue of each CTA: tcgen05.ld 32 columns at a time (thread
+//               = row), apply the epilogue, store to global.  Double-buffered
+//               TMEM lets the epilogue of tile i overlap the MMAs of tile i+1.
+// Each CTA loads only half of B, so a pair moves a third less operand data per
+// FLOP than two independent 128 x 256 tiles.  Either operand may be K-major
+// (forward: X W^T) or MN-major (dgrad reads W as stored, wgrad reads dY and X
+// as stored), selected per operand through the TMA box shape, the smem
+// descriptor and the instruction descriptor.  Weight-gradient GEMMs with too
+// few tiles to fill the GPU split K (fp32 partials, reduced in a fixed order).
+// No load is multicast.  Every wait is bounded (GPT_ETIMEOUT in the status word).
 #include <cudaTypedefs.h>
 
 #include "epilogue.cuh"
@@ -22,22 +29,11 @@
 namespace gpt {
 
 namespace {
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int BN = 256, BK = 64;
 constexpr int kThreads = 192;
-constexpr uint32_t A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
-struct __align__(8) SmemTail {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
-  uint64_t tmem_full[2];
-  uint64_t tmem_empty[2];
-  uint64_t mma_done;
-  uint32_t tmem_base;
-  int abort;
-};
-constexpr size_t kSmemBytes = 1024 /*align slack*/ + STAGES * (A_BYTES + B_BYTES) + sizeof(SmemTail);
 }  // namespace
 
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
@@ -266,43 +262,120 @@ __device__ __forceinline__ void epi_qkv_row(const GemmArgs& g, uint32_t taddr, i
   }
 }
 
+// Epilogue of one accumulator tile: rows row0 + 32*quarter + lane, columns
+// nb*BN .. nb*BN + BN (TMEM columns taddr ..), K split sp of `splits`.
+__device__ __forceinline__ void epilogue_tile(const GemmArgs& g, uint32_t taddr, int row0, int nb,
+                                              int sp, int splits, int quarter, int lane) {
+  const int row = row0 + quarter * 32 + lane;
+  const bool row_ok = row < g.M;
+  int tgt = -1;
+  float lse_row = 0.f;
+  if (row_ok && (g.epi == EPI_CE_FWD || g.epi == EPI_CE_BWD)) {
+    tgt = g.targets[row];
+    if (g.epi == EPI_CE_BWD) lse_row = g.lse[row];
+  }
+  float ce_max = -INFINITY, ce_sum = 0.f, ce_tgt = 0.f;
+  if (g.epi == EPI_QKV) {
+    epi_qkv_row(g, taddr, row, nb, row_ok);
+    return;
+  }
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    uint32_t u[32];
+    tc::tmem_ld_32x32b_x32(taddr + c * 32, u);
+    tc::tmem_wait_ld();
+    const int col0 = nb * BN + c * 32;
+    if (row_ok && col0 < g.N) {
+      if (splits > 1) {
+        // fp32 partial of this K split; the reduce kernel applies the epilogue
+        float* dst = g.splitk + (int64_t(sp) * g.M + row) * g.N + col0;
+        if (col0 + 32 <= g.N) {
+#pragma unroll
+          for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4*>(dst + j) =
+                make_float4(u2f(u[j]), u2f(u[j + 1]), u2f(u[j + 2]), u2f(u[j + 3]));
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (col0 + j < g.N) dst[j] = u2f(u[j]);
+        }
+      } else {
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = u2f(u[j]);
+        epi_chunk(g, row, col0, v, ce_max, ce_sum, ce_tgt, tgt, lse_row);
+      }
+    }
+  }
+  if (row_ok && g.epi == EPI_CE_FWD) {
+    g.part_max[int64_t(row) * g.n_part + nb] = ce_max;
+    g.part_sum[int64_t(row) * g.n_part + nb] = ce_sum;
+    if (tgt >= nb * BN && tgt < nb * BN + BN && tgt < g.n_valid) g.tgt_logit[row] = ce_tgt;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// CTA-pair variant: a cluster of two CTAs computes a 256 x 256 tile with
+// tcgen05.mma.cta_group::2 (M = 256 across the pair).  Each CTA loads its own
+// 128 rows of A and its own 128 columns of B (32 KB per stage, 6 stages); the
+// loads of both CTAs complete on the first CTA's stage barrier, whose MMA
+// thread then issues the pair MMA reading both CTAs' shared memory.  Each
+// CTA's TMEM receives its 128 output rows; the epilogue is the same as above.
+// No load is multicast.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr int P_BM = 256, P_STAGES = 6;
+constexpr uint32_t P_HALF = 128 * BK * 2;  // one CTA's A or B half of a stage: 16 KB
+struct __align__(8) PairTail {
+  uint64_t full[P_STAGES];
+  uint64_t empty[P_STAGES];
+  uint64_t tmem_full[2];
+  uint64_t tmem_empty[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort;
+};
+constexpr size_t kPairSmemBytes = 1024 + P_STAGES * 2 * P_HALF + sizeof(PairTail);
+}  // namespace
+
 template <bool AMN, bool BMN>
-__global__ void __launch_bounds__(kThreads, 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a,
-                   const __grid_constant__ CUtensorMap map_b, const __grid_constant__ GemmArgs g,
-                   int splits) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
+                     const __grid_constant__ CUtensorMap map_b, const __grid_constant__ GemmArgs g,
+                     int splits) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* smA = smem;
-  uint8_t* smB = smem + STAGES * A_BYTES;
-  SmemTail* tail = reinterpret_cast<SmemTail*>(smem + STAGES * (A_BYTES + B_BYTES));
+  uint8_t* smB = smem + P_STAGES * P_HALF;
+  PairTail* tail = reinterpret_cast<PairTail*>(smem + 2 * P_STAGES * P_HALF);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
-  const int m_tiles = (g.M + BM - 1) / BM, n_tiles = (g.N + BN - 1) / BN;
-  const int num_tiles = m_tiles * n_tiles;
+  const uint32_t rank = tc::cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+  const int m_tiles = (g.M + P_BM - 1) / P_BM, n_tiles = (g.N + BN - 1) / BN;
+  const int num_units = m_tiles * n_tiles * splits;
   const int num_kb = (g.K + BK - 1) / BK;
-  // work unit = (tile, K split); unit u covers k-blocks [kb_lo(u), kb_hi(u))
-  const int num_units = num_tiles * splits;
   const int kb_per = (num_kb + splits - 1) / splits;
-  constexpr uint32_t idesc = tc::idesc_bf16_f32(BM, BN, AMN, BMN);
+  constexpr uint32_t idesc = tc::idesc_bf16_f32(P_BM, BN, AMN, BMN);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < P_STAGES; ++s) {
       tc::mbar_init(&tail->full[s], 1);
       tc::mbar_init(&tail->empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       tc::mbar_init(&tail->tmem_full[a], 1);
-      tc::mbar_init(&tail->tmem_empty[a], 128);
+      tc::mbar_init(&tail->tmem_empty[a], 256);  // both CTAs' epilogue threads
     }
     tc::mbar_init(&tail->mma_done, 1);
     tail->abort = 0;
     tc::fence_barrier_init();
   }
   if (warp == 1) {
-    tc::tmem_alloc(&tail->tmem_base, TMEM_COLS);
-    tc::tmem_relinquish();
+    tc::tmem_alloc_pair(&tail->tmem_base, TMEM_COLS);
+    tc::tmem_relinquish_pair();
   }
   if (warp == 0 && lane == 0) {
     tc::tma_prefetch_desc(&map_a);
@@ -310,69 +383,59 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc::tc_fence_before();
   __syncthreads();
+  tc::cluster_sync();  // the peer's barriers exist before anything arrives on them
   tc::tc_fence_after();
   const uint32_t tmem_base = tail->tmem_base;
   volatile int* abort = &tail->abort;
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t issued_mask = 0, last_parity = 0;
-      for (int unit = blockIdx.x; unit < num_units && !*abort; unit += gridDim.x) {
+      for (int unit = pair; unit < num_units && !*abort; unit += num_pairs) {
         const int tile = unit / splits, sp = unit % splits;
         const int mb = tile / n_tiles, nb = tile % n_tiles;
+        const int m0 = mb * P_BM + int(rank) * 128, n0 = nb * BN + int(rank) * 128;
         const int kb_hi = min(num_kb, (sp + 1) * kb_per);
         for (int kb = sp * kb_per; kb < kb_hi; ++kb) {
           if (!tc::mbar_wait_bounded(&tail->empty[stage], phase ^ 1, abort, kWaitLimitNs)) {
-            record_status(g.status, GPT_ETIMEOUT, K_GEMM_TC, 1);
+            record_status(g.status, GPT_ETIMEOUT, K_GEMM_TC, 11);
             *abort = 1;
             break;
           }
-          tc::mbar_arrive_expect_tx(&tail->full[stage], A_BYTES + B_BYTES);
-          uint8_t* a_dst = smA + stage * A_BYTES;
-          uint8_t* b_dst = smB + stage * B_BYTES;
+          if (leader) tc::mbar_arrive_expect_tx(&tail->full[stage], 4 * P_HALF);
+          const uint32_t bar = tc::mapa_shared(tc::smem_u32(&tail->full[stage]), 0);
+          uint8_t* a_dst = smA + stage * P_HALF;
+          uint8_t* b_dst = smB + stage * P_HALF;
           if (AMN) {
-            tc::tma_load_2d(a_dst, &map_a, &tail->full[stage], mb * BM, kb * BK);
-            tc::tma_load_2d(a_dst + 8192, &map_a, &tail->full[stage], mb * BM + 64, kb * BK);
+            tc::tma_load_2d_pair(a_dst, &map_a, bar, m0, kb * BK);
+            tc::tma_load_2d_pair(a_dst + 8192, &map_a, bar, m0 + 64, kb * BK);
           } else {
-            tc::tma_load_2d(a_dst, &map_a, &tail->full[stage], kb * BK, mb * BM);
+            tc::tma_load_2d_pair(a_dst, &map_a, bar, kb * BK, m0);
           }
           if (BMN) {
-#pragma unroll
-            for (int j = 0; j < BN / 64; ++j)
-              tc::tma_load_2d(b_dst + j * 8192, &map_b, &tail->full[stage], nb * BN + 64 * j,
-                              kb * BK);
+            tc::tma_load_2d_pair(b_dst, &map_b, bar, n0, kb * BK);
+            tc::tma_load_2d_pair(b_dst + 8192, &map_b, bar, n0 + 64, kb * BK);
           } else {
-            tc::tma_load_2d(b_dst, &map_b, &tail->full[stage], kb * BK, nb * BN);
+            tc::tma_load_2d_pair(b_dst, &map_b, bar, kb * BK, n0);
           }
-          issued_mask |= 1u << stage;
-          last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          if (++stage == P_STAGES) { stage = 0; phase ^= 1; }
         }
-      }
-      if (*abort) {
-        // let every copy this thread started land before the CTA exits
-        for (int s = 0; s < STAGES; ++s)
-          if (issued_mask >> s & 1)
-            tc::mbar_wait_bounded(&tail->full[s], (last_parity >> s) & 1, nullptr, kWaitLimitNs);
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
       bool issued_any = false;
-      for (int unit = blockIdx.x; unit < num_units && !*abort; unit += gridDim.x, ++local) {
+      for (int unit = pair; unit < num_units && !*abort; unit += num_pairs, ++local) {
         const int sp = unit % splits;
         const int kb_lo = sp * kb_per, kb_hi = min(num_kb, (sp + 1) * kb_per);
         const int acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
         if (!tc::mbar_wait_bounded(&tail->tmem_empty[acc], acc_phase ^ 1, abort, kWaitLimitNs)) {
-          record_status(g.status, GPT_ETIMEOUT, K_GEMM_TC, 2);
+          record_status(g.status, GPT_ETIMEOUT, K_GEMM_TC, 12);
           *abort = 1;
           break;
         }
@@ -380,110 +443,66 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = kb_lo; kb < kb_hi; ++kb) {
           if (!tc::mbar_wait_bounded(&tail->full[stage], phase, abort, kWaitLimitNs)) {
-            record_status(g.status, GPT_ETIMEOUT, K_GEMM_TC, 3);
+            record_status(g.status, GPT_ETIMEOUT, K_GEMM_TC, 13);
             *abort = 1;
             break;
           }
           tc::tc_fence_after();
-          const uint32_t a_addr = tc::smem_u32(smA + stage * A_BYTES);
-          const uint32_t b_addr = tc::smem_u32(smB + stage * B_BYTES);
+          const uint32_t a_addr = tc::smem_u32(smA + stage * P_HALF);
+          const uint32_t b_addr = tc::smem_u32(smB + stage * P_HALF);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             const uint64_t da = AMN ? tc::smem_desc_sw128(a_addr + k * 2048, 8192)
                                     : tc::smem_desc_sw128(a_addr + k * 32, 16);
             const uint64_t db = BMN ? tc::smem_desc_sw128(b_addr + k * 2048, 8192)
                                     : tc::smem_desc_sw128(b_addr + k * 32, 16);
-            tc::mma_bf16_ss(d_tmem, da, db, idesc, (kb != kb_lo) || k != 0);
+            tc::mma_bf16_ss_pair(d_tmem, da, db, idesc, (kb != kb_lo) || k != 0);
           }
           issued_any = true;
-          tc::mma_commit(&tail->empty[stage]);
-          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          const uint32_t e = tc::smem_u32(&tail->empty[stage]);
+          tc::mma_commit_pair(e);
+          tc::mma_commit_pair(tc::mapa_shared(e, 1));
+          if (++stage == P_STAGES) { stage = 0; phase ^= 1; }
         }
         if (*abort) break;
-        tc::mma_commit(&tail->tmem_full[acc]);
+        const uint32_t f = tc::smem_u32(&tail->tmem_full[acc]);
+        tc::mma_commit_pair(f);
+        tc::mma_commit_pair(tc::mapa_shared(f, 1));
       }
-      // all MMAs of this CTA complete before TMEM is released
       if (issued_any) {
-        tc::mma_commit(&tail->mma_done);
+        tc::mma_commit_pair(tc::smem_u32(&tail->mma_done));
         tc::mbar_wait_bounded(&tail->mma_done, 0, nullptr, kWaitLimitNs);
       }
     }
   } else {
-    // ---------------- epilogue (warps 2..5) ----------------
-    const int quarter = warp & 3;  // TMEM lanes accessible to this warp
+    const int quarter = warp & 3;
     int local = 0;
-    for (int unit = blockIdx.x; unit < num_units; unit += gridDim.x, ++local) {
+    for (int unit = pair; unit < num_units; unit += num_pairs, ++local) {
       const int tile = unit / splits, sp = unit % splits;
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
       const bool ok = tc::mbar_wait_bounded(&tail->tmem_full[acc], acc_phase, abort, kWaitLimitNs);
       if (!__all_sync(0xffffffffu, ok)) {
-        if (lane == 0) record_status(g.status, GPT_ETIMEOUT, K_GEMM_TC, 4);
+        if (lane == 0) record_status(g.status, GPT_ETIMEOUT, K_GEMM_TC, 14);
         *abort = 1;
         break;
       }
       tc::tc_fence_after();
-      const int mb = tile / n_tiles, nb = tile % n_tiles;
-      const int row = mb * BM + quarter * 32 + lane;
-      const bool row_ok = row < g.M;
-      int tgt = -1;
-      float lse_row = 0.f;
-      if (row_ok && (g.epi == EPI_CE_FWD || g.epi == EPI_CE_BWD)) {
-        tgt = g.targets[row];
-        if (g.epi == EPI_CE_BWD) lse_row = g.lse[row];
-      }
-      float ce_max = -INFINITY, ce_sum = 0.f, ce_tgt = 0.f;
-      const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + acc * BN;
-      if (g.epi == EPI_QKV) {
-        epi_qkv_row(g, taddr, row, nb, row_ok);
-        tc::tc_fence_before();
-        tc::mbar_arrive(&tail->tmem_empty[acc]);
-        continue;
-      }
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t u[32];
-        tc::tmem_ld_32x32b_x32(taddr + c * 32, u);
-        tc::tmem_wait_ld();
-        const int col0 = nb * BN + c * 32;
-        if (row_ok && col0 < g.N) {
-          if (splits > 1) {
-            // fp32 partial of this K split; the reduce kernel applies the epilogue
-            float* dst = g.splitk + (int64_t(sp) * g.M + row) * g.N + col0;
-            if (col0 + 32 <= g.N) {
-#pragma unroll
-              for (int j = 0; j < 32; j += 4)
-                *reinterpret_cast<float4*>(dst + j) =
-                    make_float4(u2f(u[j]), u2f(u[j + 1]), u2f(u[j + 2]), u2f(u[j + 3]));
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (col0 + j < g.N) dst[j] = u2f(u[j]);
-            }
-          } else {
-            float v[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = u2f(u[j]);
-            epi_chunk(g, row, col0, v, ce_max, ce_sum, ce_tgt, tgt, lse_row);
-          }
-        }
-      }
-      if (row_ok && g.epi == EPI_CE_FWD) {
-        g.part_max[int64_t(row) * g.n_part + nb] = ce_max;
-        g.part_sum[int64_t(row) * g.n_part + nb] = ce_sum;
-        if (tgt >= nb * BN && tgt < nb * BN + BN && tgt < g.n_valid) g.tgt_logit[row] = ce_tgt;
-      }
+      epilogue_tile(g, tmem_base + (uint32_t(quarter * 32) << 16) + acc * BN,
+                    (tile / n_tiles) * P_BM + int(rank) * 128, tile % n_tiles, sp, splits, quarter,
+                    lane);
       tc::tc_fence_before();
-      tc::mbar_arrive(&tail->tmem_empty[acc]);
+      tc::mbar_arrive_cluster(tc::mapa_shared(tc::smem_u32(&tail->tmem_empty[acc]), 0));
     }
   }
 
   __syncwarp();
   tc::tc_fence_before();
   __syncthreads();
+  tc::cluster_sync();  // neither CTA leaves while the pair MMAs may read its shared memory
   if (warp == 1) {
     tc::tc_fence_after();
-    tc::tmem_dealloc(tmem_base, TMEM_COLS);
+    tc::tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
 }
 
@@ -522,18 +541,18 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
 }
 
 template <bool AMN, bool BMN>
-int launch_tc(const GemmArgs& g, int grid, int splits, cudaStream_t st) {
+int launch_pair(const GemmArgs& g, int grid, int splits, cudaStream_t st) {
   CUtensorMap ma, mb;
   bool ok = AMN ? make_map(&ma, g.A, g.M, g.K, g.lda, 64, 64)
-                : make_map(&ma, g.A, g.K, g.M, g.lda, 64, BM);
+                : make_map(&ma, g.A, g.K, g.M, g.lda, 64, 128);
   ok = ok && (BMN ? make_map(&mb, g.B, g.N, g.K, g.ldb, 64, 64)
-                  : make_map(&mb, g.B, g.K, g.N, g.ldb, 64, BN));
+                  : make_map(&mb, g.B, g.K, g.N, g.ldb, 64, 128));
   if (!ok) return 1;
-  auto kern = gemm_tc_kernel<AMN, BMN>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes)) !=
+  auto kern = gemm_pair_kernel<AMN, BMN>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kPairSmemBytes)) !=
       cudaSuccess)
     return 1;
-  kern<<<grid, kThreads, kSmemBytes, st>>>(ma, mb, g, splits);
+  kern<<<grid, kThreads, kPairSmemBytes, st>>>(ma, mb, g, splits);
   return last_launch_rc();
 }
 
@@ -566,24 +585,28 @@ int num_sms() {
 }  // namespace
 
 // K splits for a GEMM: only plain stores into a contiguous [M, N] output with a
-// split-K buffer, and only when the tile count alone would leave SMs idle; the
-// smallest split count that fills >= 90 % of the SM waves, keeping >= 8 k-blocks
-// per split and the partials within the buffer.
+// split-K buffer, and only when the pair-tile count alone would leave SM pairs
+// idle; the smallest split count that fills >= 90 % of the waves, keeping >= 8
+// k-blocks per split and the partials within the buffer.
 int gemm_tc_splits(const GemmArgs& g) {
   if (g.epi != EPI_STORE || !g.splitk || g.ldo != g.N || (g.N & 3)) return 1;
-  const int sms = num_sms();
-  const int tiles = ((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN);
+  const int pairs = num_sms() / 2;
+  const int tiles = ((g.M + P_BM - 1) / P_BM) * ((g.N + BN - 1) / BN);
   const int num_kb = (g.K + BK - 1) / BK;
-  if (tiles >= 3 * sms) return 1;
+  if (tiles >= 3 * pairs) return 1;
   int best = 1;
   double best_eff = 0.0;
   for (int s = 1; s <= 4; ++s) {
     if (num_kb / s < 8 || int64_t(s) * g.M * g.N > g.splitk_floats) break;
     const int units = tiles * s;
-    const int waves = (units + sms - 1) / sms;
-    const double eff = double(units) / (double(waves) * sms);
+    const int waves = (units + pairs - 1) / pairs;
+    const double eff = double(units) / (double(waves) * pairs);
     if (eff > best_eff + 1e-9) { best_eff = eff; best = s; }
     if (eff >= 0.9) break;
+  }
+  if (best > 1) {  // every split non-empty: ceil(num_kb / ceil(num_kb / best)) splits
+    const int kb_per = (num_kb + best - 1) / best;
+    best = (num_kb + kb_per - 1) / kb_per;
   }
   return best;
 }
@@ -592,22 +615,17 @@ int launch_gemm_tc(const GemmArgs& g_in, void* stream) {
   GemmArgs g = g_in;
   cudaStream_t st = (cudaStream_t)stream;
   if (g.M <= 0 || g.N <= 0 || g.K <= 0) return 0;
-  const int tiles = ((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN);
+  const int tiles = ((g.M + P_BM - 1) / P_BM) * ((g.N + BN - 1) / BN);
   if (g.epi == EPI_CE_FWD) g.n_part = (g.N + BN - 1) / BN;
-  int splits = gemm_tc_splits(g);
-  if (splits > 1) {  // every split non-empty: ceil(num_kb / ceil(num_kb / splits)) splits
-    const int num_kb = (g.K + BK - 1) / BK;
-    const int kb_per = (num_kb + splits - 1) / splits;
-    splits = (num_kb + kb_per - 1) / kb_per;
-  }
-  const int sms = num_sms();
+  const int splits = gemm_tc_splits(g);
+  const int pairs = num_sms() / 2;
   const int units = tiles * splits;
-  const int grid = units < sms ? units : sms;
+  const int grid = 2 * (units < pairs ? units : pairs);
   int rc;
-  if (!g.a_mn_major && !g.b_mn_major) rc = launch_tc<false, false>(g, grid, splits, st);
-  else if (!g.a_mn_major && g.b_mn_major) rc = launch_tc<false, true>(g, grid, splits, st);
-  else if (g.a_mn_major && g.b_mn_major) rc = launch_tc<true, true>(g, grid, splits, st);
-  else rc = launch_tc<true, false>(g, grid, splits, st);
+  if (!g.a_mn_major && !g.b_mn_major) rc = launch_pair<false, false>(g, grid, splits, st);
+  else if (!g.a_mn_major && g.b_mn_major) rc = launch_pair<false, true>(g, grid, splits, st);
+  else if (g.a_mn_major && g.b_mn_major) rc = launch_pair<true, true>(g, grid, splits, st);
+  else rc = launch_pair<true, false>(g, grid, splits, st);
   if (rc || splits == 1) return rc;
   const int64_t n4 = int64_t(g.M) * g.N / 4;
   splitk_reduce_kernel<<<int((n4 + 255) / 256), 256, 0, st>>>(
