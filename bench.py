@@ -159,6 +159,33 @@ def cpu_cores():
         return os.cpu_count() or 1
 
 
+def gemm_sites(records, w, steps):
+    """Per-call-site GEMM time from the launch-ordered trace: the step launches
+    forward [qkv, o, up, down] per layer then the lm_head statistics GEMM, and
+    backward [logit grad, dhf, dWlm] then per layer (last first) [down dgrad,
+    down wgrad, up dgrad, up wgrad, o dgrad, o wgrad, qkv dgrad, qkv wgrad]."""
+    L = w.n_layer
+    names = []
+    for _ in range(L):
+        names += ["qkv_fwd", "o_fwd", "up_fwd", "down_fwd"]
+    names += ["lm_fwd_ce", "lm_grad_logits", "lm_dgrad", "lm_wgrad"]
+    for _ in range(L):
+        names += ["down_dgrad", "down_wgrad", "up_dgrad", "up_wgrad", "o_dgrad", "o_wgrad",
+                  "qkv_dgrad", "qkv_wgrad"]
+    gemms = [r for r in records if r[0] == "gemm"]
+    if len(gemms) != len(names) * steps:
+        return None
+    acc = {}
+    for i, (_, _, ms, fl, _) in enumerate(gemms):
+        n = names[i % len(names)]
+        a = acc.setdefault(n, [0.0, 0.0])
+        a[0] += ms
+        a[1] += fl
+    return {n: {"ms_per_step": round(v[0] / steps, 3),
+                "tflops": round(v[1] / (v[0] / 1e3) / 1e12, 1) if v[0] else None}
+            for n, v in acc.items()}
+
+
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
@@ -178,6 +205,8 @@ def run_ours(args, rank, world, local_rank):
     w = synth.workload(args.workload)
     if args.batch:
         w = w.replace(batch=args.batch)
+    if args.layers is not None:
+        w = w.replace(n_layer=args.layers)
     wr = w.replace(seed=w.seed + 100 * rank)  # each replica its own batch
     cfg = B.config_from_workload(w)
     st = R.TrainStep(cfg, device=f"cuda:{local_rank}")
@@ -228,7 +257,9 @@ def run_ours(args, rank, world, local_rank):
     if code != B.GPT_OK:
         raise SystemExit(f"device status after timed steps: {B.strerror(code)}")
     stats, dropped = trace.summary()
+    records = trace.records(per_step * args.steps + 16)
     trace.close()
+    sites = gemm_sites(records, w, args.steps)
 
     # ---- end to end through the public host-buffer call ----
     ht = torch.from_numpy(tok.ravel().copy()).pin_memory()
@@ -309,6 +340,7 @@ def run_ours(args, rank, world, local_rank):
                      "peak_source": f"{peaks['source']} bf16_tflops_sustained",
                      "traffic": None},
         "kernel_breakdown": breakdown,
+        "gemm_sites": sites,
         "gpu_launches": kernels,
         "trace_dropped": dropped,
         "e2e": {"value": round(world * N * args.steps / (e2e_ms / 1e3), 1), "unit": "tokens/s",
@@ -367,6 +399,9 @@ def main():
     ap.add_argument("--workload", default=WORKLOAD, choices=list(synth.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip timing the CPU oracle sample")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="override the workload's layer count (profiling captures on a smaller "
+                         "case; the line then reports that model)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (profiling captures on a smaller "
                          "case; the line then reports that batch)")

@@ -209,6 +209,11 @@ class GptTraceStat(ctypes.Structure):
                 ("flops", ctypes.c_double), ("bytes", ctypes.c_double)]
 
 
+class GptTraceRecord(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("kernels", ctypes.c_int32), ("ms", ctypes.c_float),
+                ("flops", ctypes.c_double), ("bytes", ctypes.c_double)]
+
+
 class Trace:
     """Per-launch CUDA-event trace of the library's kernels (see gpt_trace_* in gpt.h)."""
 
@@ -240,6 +245,16 @@ class Trace:
         out = {n: dict(launches=s.launches, kernels=s.kernels, ms=s.ms, flops=s.flops,
                        bytes=s.bytes) for n, s in zip(GPT_K_NAMES, stats)}
         return out, dropped.value
+
+    def records(self, capacity: int):
+        """Per-launch records in launch order: list of (kind name, kernels, ms, flops, bytes)."""
+        L = lib()
+        L.gpt_trace_records.argtypes = [ctypes.c_void_p, ctypes.POINTER(GptTraceRecord),
+                                        ctypes.c_int, ctypes.POINTER(ctypes.c_int32)]
+        buf = (GptTraceRecord * capacity)()
+        n = ctypes.c_int32()
+        _check(L.gpt_trace_records(self._h, buf, capacity, ctypes.byref(n)), "gpt_trace_records")
+        return [(GPT_K_NAMES[r.kind], r.kernels, r.ms, r.flops, r.bytes) for r in buf[:n.value]]
 
     def close(self):
         if self._h:

@@ -11,8 +11,11 @@
 //               of two 256-column fp32 accumulators (each CTA's TMEM holds its
 //               128 rows; 512 columns), and tcgen05.commit frees stages in both
 //               CTAs / hands the accumulator to both epilogues;
-//   warps 2..5  epilogue of each CTA: tcgen05.ld 32 columns at a time (thread
-//               = row), apply the epilogue, store to global.  Double-buffered
+//   warps 2..9  epilogue of each CTA: two warps per TMEM lane quarter, each
+//               thread one row and 128 of the tile's 256 columns; tcgen05.ld
+//               32 columns at a time, apply the epilogue, store to global.  The
+//               operand bytes the epilogue reads (stored activation, fp32
+//               residual) are prefetched into L2 one tile ahead.  Double-buffered
 //               TMEM lets the epilogue of tile i overlap the MMAs of tile i+1.
 // Each CTA loads only half of B, so a pair moves a third less operand data per
 // FLOP than two independent 128 x 256 tiles.  Either operand may be K-major
@@ -30,13 +33,46 @@ namespace gpt {
 
 namespace {
 constexpr int BN = 256, BK = 64;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
+constexpr int EC = 128;          // columns of a tile handled by one epilogue thread
+static_assert((kThreads - 64) / 128 * EC == 256, "epilogue warps must cover the tile's columns");
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 }  // namespace
 
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
+
+__device__ __forceinline__ float sqrt_approx(float x) {
+  float y;
+  asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+// Ask L2 for the bytes this thread's epilogue will read for one tile row
+// (columns col0 .. col0 + EC): the stored activation (ReLU^2'), the fp32 residual
+// (residual add) or the gradient being accumulated.  Issued before the thread
+// waits for the tile's accumulator, so the reads hit L2 when the tile lands.
+__device__ __forceinline__ void epilogue_prefetch(const GemmArgs& g, int row, int col0, int splits) {
+  if (row >= g.M || splits > 1) return;
+  const int64_t base = int64_t(row) * g.ldo + col0;
+  const int cols = min(EC, g.N - col0);
+  if (cols <= 0) return;
+  if (g.epi == EPI_DRELU2) {
+    const char* p = reinterpret_cast<const char*>(static_cast<const __nv_bfloat16*>(g.aux) + base);
+    for (int b = 0; b < cols * 2; b += 128) prefetch_l2(p + b);
+  } else if (g.epi == EPI_RESID_F32) {
+    const char* p = reinterpret_cast<const char*>(static_cast<const float*>(g.out) + base);
+    for (int b = 0; b < cols * 4; b += 128) prefetch_l2(p + b);
+  } else if (g.epi == EPI_STORE && g.beta) {
+    const char* p = reinterpret_cast<const char*>(static_cast<const __nv_bfloat16*>(g.out) + base);
+    for (int b = 0; b < cols * 2; b += 128) prefetch_l2(p + b);
+  }
+}
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -140,15 +176,15 @@ __device__ __forceinline__ void epi_chunk(const GemmArgs& g, int row, int col0, 
           uint4 u = *reinterpret_cast<const uint4*>(a + j);
           float2 p0 = unpack_bf16(u.x), p1 = unpack_bf16(u.y), p2 = unpack_bf16(u.z),
                  p3 = unpack_bf16(u.w);
-          r[j] = v[j] * 2.f * sqrtf(p0.x); r[j + 1] = v[j + 1] * 2.f * sqrtf(p0.y);
-          r[j + 2] = v[j + 2] * 2.f * sqrtf(p1.x); r[j + 3] = v[j + 3] * 2.f * sqrtf(p1.y);
-          r[j + 4] = v[j + 4] * 2.f * sqrtf(p2.x); r[j + 5] = v[j + 5] * 2.f * sqrtf(p2.y);
-          r[j + 6] = v[j + 6] * 2.f * sqrtf(p3.x); r[j + 7] = v[j + 7] * 2.f * sqrtf(p3.y);
+          r[j] = v[j] * 2.f * sqrt_approx(p0.x); r[j + 1] = v[j + 1] * 2.f * sqrt_approx(p0.y);
+          r[j + 2] = v[j + 2] * 2.f * sqrt_approx(p1.x); r[j + 3] = v[j + 3] * 2.f * sqrt_approx(p1.y);
+          r[j + 4] = v[j + 4] * 2.f * sqrt_approx(p2.x); r[j + 5] = v[j + 5] * 2.f * sqrt_approx(p2.y);
+          r[j + 6] = v[j + 6] * 2.f * sqrt_approx(p3.x); r[j + 7] = v[j + 7] * 2.f * sqrt_approx(p3.y);
         }
       } else {
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-          r[j] = col0 + j < g.N ? v[j] * 2.f * sqrtf(__bfloat162float(a[j])) : 0.f;
+          r[j] = col0 + j < g.N ? v[j] * 2.f * sqrt_approx(__bfloat162float(a[j])) : 0.f;
       }
       break;
     }
@@ -182,17 +218,17 @@ __device__ __forceinline__ void epi_chunk(const GemmArgs& g, int row, int col0, 
   }
 }
 
-// EPI_QKV: the tile's 256 columns hold whole heads (head_dim 64 or 128 divides
-// 256).  For each head of this row: v is copied to its head-major row; q and k
+// EPI_QKV: a thread's 128 tile columns hold whole heads (head_dim 64 or 128
+// divides 128).  For each head of this row: v is copied to its head-major row; q and k
 // are rotated by RoPE (pairs (i, i + hd/2)), scaled by 1/rms of the rotated row
 // (the rotation keeps the norm, so the sum of squares is taken on the raw row)
 // and written head-major, with the 1/rms kept for the backward.
-__device__ __forceinline__ void epi_qkv_row(const GemmArgs& g, uint32_t taddr, int row, int nb,
-                                            bool row_ok) {
+__device__ __forceinline__ void epi_qkv_row(const GemmArgs& g, uint32_t taddr, int row,
+                                            int col_base, bool row_ok) {
   const int hd = g.head_dim, half = hd / 2, H = g.n_head, d = H * hd, T = g.seq_len;
   const int b = row_ok ? row / T : 0, t = row_ok ? row % T : 0;
-  for (int seg = 0; seg < BN / hd; ++seg) {
-    const int c0 = nb * BN + seg * hd;
+  for (int seg = 0; seg < EC / hd; ++seg) {
+    const int c0 = col_base + seg * hd;
     if (c0 >= g.N) break;  // uniform across the warp
     const int part = c0 / d, h = (c0 % d) / hd;
     const uint32_t tcol = taddr + seg * hd;
@@ -262,10 +298,12 @@ __device__ __forceinline__ void epi_qkv_row(const GemmArgs& g, uint32_t taddr, i
   }
 }
 
-// Epilogue of one accumulator tile: rows row0 + 32*quarter + lane, columns
-// nb*BN .. nb*BN + BN (TMEM columns taddr ..), K split sp of `splits`.
-__device__ __forceinline__ void epilogue_tile(const GemmArgs& g, uint32_t taddr, int row0, int nb,
-                                              int sp, int splits, int quarter, int lane) {
+// Epilogue of one accumulator tile for one thread: row row0 + 32*quarter +
+// lane, columns col_base .. col_base + EC (TMEM columns taddr ..), K split sp
+// of `splits`; `part` indexes this column block's cross-entropy partials.
+__device__ __forceinline__ void epilogue_tile(const GemmArgs& g, uint32_t taddr, int row0,
+                                              int col_base, int part, int sp, int splits,
+                                              int quarter, int lane) {
   const int row = row0 + quarter * 32 + lane;
   const bool row_ok = row < g.M;
   int tgt = -1;
@@ -276,15 +314,15 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& g, uint32_t taddr,
   }
   float ce_max = -INFINITY, ce_sum = 0.f, ce_tgt = 0.f;
   if (g.epi == EPI_QKV) {
-    epi_qkv_row(g, taddr, row, nb, row_ok);
+    epi_qkv_row(g, taddr, row, col_base, row_ok);
     return;
   }
 #pragma unroll 1
-  for (int c = 0; c < BN / 32; ++c) {
+  for (int c = 0; c < EC / 32; ++c) {
     uint32_t u[32];
     tc::tmem_ld_32x32b_x32(taddr + c * 32, u);
     tc::tmem_wait_ld();
-    const int col0 = nb * BN + c * 32;
+    const int col0 = col_base + c * 32;
     if (row_ok && col0 < g.N) {
       if (splits > 1) {
         // fp32 partial of this K split; the reduce kernel applies the epilogue
@@ -308,9 +346,9 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& g, uint32_t taddr,
     }
   }
   if (row_ok && g.epi == EPI_CE_FWD) {
-    g.part_max[int64_t(row) * g.n_part + nb] = ce_max;
-    g.part_sum[int64_t(row) * g.n_part + nb] = ce_sum;
-    if (tgt >= nb * BN && tgt < nb * BN + BN && tgt < g.n_valid) g.tgt_logit[row] = ce_tgt;
+    g.part_max[int64_t(row) * g.n_part + part] = ce_max;
+    g.part_sum[int64_t(row) * g.n_part + part] = ce_sum;
+    if (tgt >= col_base && tgt < col_base + EC && tgt < g.n_valid) g.tgt_logit[row] = ce_tgt;
   }
 }
 
@@ -367,7 +405,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       tc::mbar_init(&tail->tmem_full[a], 1);
-      tc::mbar_init(&tail->tmem_empty[a], 256);  // both CTAs' epilogue threads
+      tc::mbar_init(&tail->tmem_empty[a], 2 * (kThreads - 64));  // both CTAs' epilogue threads
     }
     tc::mbar_init(&tail->mma_done, 1);
     tail->abort = 0;
@@ -475,12 +513,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    const int quarter = warp & 3;
+    const int quarter = warp & 3;      // TMEM lanes 32*quarter .. +31
+    const int ch = (warp - 2) >> 2;    // columns ch*EC .. ch*EC + EC of each tile
+    const int my_row = int(rank) * 128 + quarter * 32 + lane;  // within a 256-row pair tile
+    if (pair < num_units)
+      epilogue_prefetch(g, (pair / splits / n_tiles) * P_BM + my_row,
+                        ((pair / splits) % n_tiles) * BN + ch * EC, splits);
     int local = 0;
     for (int unit = pair; unit < num_units; unit += num_pairs, ++local) {
       const int tile = unit / splits, sp = unit % splits;
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
+      // one tile ahead: the rows of the next unit
+      const int next = unit + num_pairs;
+      if (next < num_units)
+        epilogue_prefetch(g, (next / splits / n_tiles) * P_BM + my_row,
+                          ((next / splits) % n_tiles) * BN + ch * EC, splits);
       const bool ok = tc::mbar_wait_bounded(&tail->tmem_full[acc], acc_phase, abort, kWaitLimitNs);
       if (!__all_sync(0xffffffffu, ok)) {
         if (lane == 0) record_status(g.status, GPT_ETIMEOUT, K_GEMM_TC, 14);
@@ -488,9 +536,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         break;
       }
       tc::tc_fence_after();
-      epilogue_tile(g, tmem_base + (uint32_t(quarter * 32) << 16) + acc * BN,
-                    (tile / n_tiles) * P_BM + int(rank) * 128, tile % n_tiles, sp, splits, quarter,
-                    lane);
+      const int nb = tile % n_tiles;
+      epilogue_tile(g, tmem_base + (uint32_t(quarter * 32) << 16) + acc * BN + ch * EC,
+                    (tile / n_tiles) * P_BM + int(rank) * 128, nb * BN + ch * EC, nb * (BN / EC) + ch, sp,
+                    splits, quarter, lane);
       tc::tc_fence_before();
       tc::mbar_arrive_cluster(tc::mapa_shared(tc::smem_u32(&tail->tmem_empty[acc]), 0));
     }
@@ -616,7 +665,7 @@ int launch_gemm_tc(const GemmArgs& g_in, void* stream) {
   cudaStream_t st = (cudaStream_t)stream;
   if (g.M <= 0 || g.N <= 0 || g.K <= 0) return 0;
   const int tiles = ((g.M + P_BM - 1) / P_BM) * ((g.N + BN - 1) / BN);
-  if (g.epi == EPI_CE_FWD) g.n_part = (g.N + BN - 1) / BN;
+  if (g.epi == EPI_CE_FWD) g.n_part = (g.N + EC - 1) / EC;
   const int splits = gemm_tc_splits(g);
   const int pairs = num_sms() / 2;
   const int units = tiles * splits;
@@ -633,6 +682,6 @@ int launch_gemm_tc(const GemmArgs& g_in, void* stream) {
   return last_launch_rc();
 }
 
-int gemm_tc_tile_n() { return BN; }
+int gemm_tc_tile_n() { return EC; }
 
 }  // namespace gpt

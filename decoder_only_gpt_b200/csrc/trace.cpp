@@ -96,6 +96,20 @@ int gpt_trace_summary(gpt_trace* t, gpt_trace_stat* stats, int32_t* dropped) {
   return GPT_OK;
 }
 
+int gpt_trace_records(gpt_trace* t, gpt_trace_record* out, int capacity, int32_t* count) {
+  if (!t || (!out && capacity > 0) || !count) return GPT_EINVAL;
+  int n = 0;
+  for (int i = 0; i < t->used && n < capacity; ++i, ++n) {
+    if (cudaEventSynchronize(t->ev[2 * i + 1]) != cudaSuccess) return GPT_ECUDA;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, t->ev[2 * i], t->ev[2 * i + 1]) != cudaSuccess) return GPT_ECUDA;
+    const auto& r = t->rec[i];
+    out[n] = gpt_trace_record{r.cls, r.nk, ms, r.flops, r.bytes};
+  }
+  *count = n;
+  return GPT_OK;
+}
+
 int gpt_trace_destroy(gpt_trace* t) {
   if (!t) return GPT_EINVAL;
   if (gpt::t_trace == t) gpt::t_trace = nullptr;

@@ -236,6 +236,19 @@ int gpt_trace_reset(gpt_trace* trace);
 /* Wait for the recorded events and fill stats[GPT_K_COUNT] (one per class);
  * *dropped receives the number of launches not recorded for lack of room. */
 int gpt_trace_summary(gpt_trace* trace, gpt_trace_stat* stats, int32_t* dropped);
+
+/* One recorded launch, in launch order. */
+typedef struct gpt_trace_record {
+  int32_t kind;      /* GPT_K_* */
+  int32_t kernels;
+  float ms;
+  double flops;
+  double bytes;
+} gpt_trace_record;
+
+/* Wait for the recorded events and copy up to `capacity` records, in launch
+ * order, to `records`; *count receives the number copied. */
+int gpt_trace_records(gpt_trace* trace, gpt_trace_record* records, int capacity, int32_t* count);
 int gpt_trace_destroy(gpt_trace* trace);
 
 #ifdef __cplusplus
