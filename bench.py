@@ -186,6 +186,21 @@ def gemm_sites(records, w, steps):
             for n, v in acc.items()}
 
 
+def max_over_ranks(values, device):
+    """Element-wise maximum of per-rank timings over the process group (the
+    reported step time of a multi-GPU run is the slowest rank's)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def replica_throughput(tokens_per_step, steps, world, max_ms):
+    """Whole-job tokens/s of `world` replicas that each ran `steps` steps."""
+    return world * tokens_per_step * steps / (max_ms / 1e3)
+
+
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
@@ -282,16 +297,14 @@ def run_ours(args, rank, world, local_rank):
     e2e_ms = f0.elapsed_time(f1)
 
     if world > 1:
-        t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, e2e_ms = float(t[0]), float(t[1])
+        ms, e2e_ms = max_over_ranks([ms, e2e_ms], dev)
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
         return
 
     peaks = load_peaks()
-    tok_s = world * N * args.steps / (ms / 1e3)
+    tok_s = replica_throughput(N, args.steps, world, ms)
     fpt = flops_per_token(w)
     g = stats["gemm"]
     gemm_tf = g["flops"] / (g["ms"] / 1e3) / 1e12 if g["ms"] > 0 else 0.0
@@ -343,7 +356,7 @@ def run_ours(args, rank, world, local_rank):
         "gemm_sites": sites,
         "gpu_launches": kernels,
         "trace_dropped": dropped,
-        "e2e": {"value": round(world * N * args.steps / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+        "e2e": {"value": round(replica_throughput(N, args.steps, world, e2e_ms), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": 2 * N * 4, "d2h_bytes_per_step": 4},
         "clocks": clk,
         "cpu_baseline": cpu,

@@ -171,10 +171,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~uintptr_t(1023));
   FwdBars* bars = reinterpret_cast<FwdBars*>(smem + S::BAR_OFF);
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+  // (batch, head)-major order, longest causal rows first inside each head: the
+  // CTAs resident together share a few heads' K/V, which then stay in L2
   const int n_qt = (T + BQ - 1) / BQ;
-  const int BH = gridDim.x / n_qt;
-  const int qt = n_qt - 1 - int(blockIdx.x) / BH;
-  const int bh = int(blockIdx.x) % BH;
+  const int bh = int(blockIdx.x) / n_qt;
+  const int qt = n_qt - 1 - int(blockIdx.x) % n_qt;
   const int q0 = qt * BQ;
   const int n_kv = qt + 1;
   const int row_base = bh * T;
@@ -450,12 +451,13 @@ __global__ void attn_rowdot_kernel(const __nv_bfloat16* __restrict__ dO,
   }
 }
 
-constexpr int kRing = 3;  // slots of the per-step operand ring
+constexpr int kRing = 3;    // slots of the per-step operand ring (dK/dV kernel)
+constexpr int kRingQ = 4;   // slots of the K/V ring of the dQ kernel
 
 struct BwdBars {
   uint64_t fixed_full;
-  uint64_t ring_full[kRing];
-  uint64_t ring_empty[kRing];
+  uint64_t ring_full[kRingQ];
+  uint64_t ring_empty[kRingQ];
   uint64_t s_full[2];
   uint64_t ds_ready[2];
   uint64_t acc_full;
@@ -539,8 +541,8 @@ struct DqSmem {
   static constexpr uint32_t SMALL = kInner * HD * 2;
   static constexpr uint32_t DS = 128 * kInner * 2;
   static constexpr uint32_t Q_OFF = 0, DO_OFF = BIG, K_OFF = 2 * BIG;
-  static constexpr uint32_t V_OFF = K_OFF + kRing * SMALL;
-  static constexpr uint32_t DS_OFF = V_OFF + kRing * SMALL;
+  static constexpr uint32_t V_OFF = K_OFF + kRingQ * SMALL;
+  static constexpr uint32_t DS_OFF = V_OFF + kRingQ * SMALL;
   static constexpr uint32_t RED_OFF = DS_OFF + 2 * DS;
   static constexpr uint32_t BAR_OFF = RED_OFF + 2 * 128 * 4;
   static constexpr uint32_t BYTES = BAR_OFF + 256 + 1024;
@@ -569,9 +571,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   BwdBars* bars = reinterpret_cast<BwdBars*>(smem + S::BAR_OFF);
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int n_qt = (T + 127) / 128;
-  const int BH = gridDim.x / n_qt;
-  const int qt = n_qt - 1 - int(blockIdx.x) / BH;
-  const int bh = int(blockIdx.x) % BH;
+  const int bh = int(blockIdx.x) / n_qt;  // (batch, head)-major, as in the forward
+  const int qt = n_qt - 1 - int(blockIdx.x) % n_qt;
   const int b = bh / H, h = bh % H;
   const int q0 = qt * 128;
   const int n_steps = (min(q0 + 128, T) + kInner - 1) / kInner;
@@ -579,7 +580,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   ATTN_PROLOGUE(bars, {
     tc::mbar_init(&bars->fixed_full, 1);
-    for (int s = 0; s < kRing; ++s) {
+    for (int s = 0; s < kRingQ; ++s) {
       tc::mbar_init(&bars->ring_full[s], 1);
       tc::mbar_init(&bars->ring_empty[s], 1);
     }
@@ -605,8 +606,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         h * HD + c * 64, b * T + q0);
       }
       for (int j = 0; j < n_steps; ++j) {
-        const int st = j % kRing;
-        const uint32_t ph = (j / kRing) & 1;
+        const int st = j % kRingQ;
+        const uint32_t ph = (j / kRingQ) & 1;
         if (!tc::mbar_wait_bounded(&bars->ring_empty[st], ph ^ 1, abort, kWaitNs)) {
           record_status(status, GPT_ETIMEOUT, K_ATTN, 20);
           *abort = 1;
@@ -625,7 +626,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (*abort) {
         tc::mbar_wait_bounded(&bars->fixed_full, 0, nullptr, kWaitNs);
-        for (int s = 0; s < kRing; ++s)
+        for (int s = 0; s < kRingQ; ++s)
           if (issued >> s & 1) tc::mbar_wait_bounded(&bars->ring_full[s], (last_par >> s) & 1, nullptr, kWaitNs);
       }
     }
@@ -641,17 +642,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!tc::mbar_wait_bounded(&bars->ds_ready[j & 1], (j >> 1) & 1, abort, kWaitNs)) return false;
         tc::tc_fence_after();
         const uint32_t ds_addr = tc::smem_u32(smem + S::DS_OFF + (j & 1) * S::DS);
-        const uint32_t k_addr = tc::smem_u32(smem + S::K_OFF + (j % kRing) * S::SMALL);
+        const uint32_t k_addr = tc::smem_u32(smem + S::K_OFF + (j % kRingQ) * S::SMALL);
 #pragma unroll
         for (int k = 0; k < kInner / 16; ++k)
           tc::mma_bf16_ss(t_dq, tc::smem_desc_sw128(ds_addr + k * 32, 16),
                           tc::smem_desc_sw128(k_addr + k * 2048, kInner * 128), idesc_dq, (j | k) != 0);
-        tc::mma_commit(&bars->ring_empty[j % kRing]);
+        tc::mma_commit(&bars->ring_empty[j % kRingQ]);
         return true;
       };
       for (int j = 0; ok && j < n_steps; ++j) {
-        const int st = j % kRing;
-        if (!tc::mbar_wait_bounded(&bars->ring_full[st], (j / kRing) & 1, abort, kWaitNs)) { ok = false; break; }
+        const int st = j % kRingQ;
+        if (!tc::mbar_wait_bounded(&bars->ring_full[st], (j / kRingQ) & 1, abort, kWaitNs)) { ok = false; break; }
         tc::tc_fence_after();
         const uint32_t k_addr = tc::smem_u32(smem + S::K_OFF + st * S::SMALL);
         const uint32_t v_addr = tc::smem_u32(smem + S::V_OFF + st * S::SMALL);
@@ -778,9 +779,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   BwdBars* bars = reinterpret_cast<BwdBars*>(smem + S::BAR_OFF);
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int n_kt = (T + 127) / 128;
-  const int BH = gridDim.x / n_kt;
-  const int kt = int(blockIdx.x) / BH;  // key tile 0 has the most queries: first
-  const int bh = int(blockIdx.x) % BH;
+  const int bh = int(blockIdx.x) / n_kt;  // (batch, head)-major; key tile 0 (most queries) first
+  const int kt = int(blockIdx.x) % n_kt;
   const int b = bh / H, h = bh % H;
   const int k0 = kt * 128;
   const int i_begin = k0 / kInner;
