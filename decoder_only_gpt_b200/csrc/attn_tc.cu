@@ -94,6 +94,19 @@ bool tile_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+// [rows, cols] fp32 row-major (pitch ld elements), box 32 columns x box_rows rows
+bool tile_map_f32(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
+                  uint32_t box_rows) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 4};
+  cuuint32_t box[2] = {32, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 }  // namespace
 
 // Common prologue: barrier init by thread 0, TMEM allocation by warp 1.
@@ -234,50 +247,50 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    {  // the whole warp runs the MMA loop; elect.sync issues
       constexpr uint32_t idesc_s = tc::idesc_bf16_f32(BQ, BKV, false, false);
       constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(BQ, HD, false, true);
       const uint32_t q_addr = tc::smem_u32(smem + S::Q_OFF);
       const uint32_t p_addr = tc::smem_u32(smem + S::P_OFF);
-      bool ok = tc::mbar_wait_bounded(&bars->q_full, 0, abort, kWaitNs);
+      bool ok = tc::mbar_wait_warp(&bars->q_full, 0, abort, kWaitNs);
       bool issued_any = false;
       auto issue_pv = [&](int j) -> bool {
-        if (!tc::mbar_wait_bounded(&bars->p_ready, j & 1, abort, kWaitNs)) return false;
-        if (!tc::mbar_wait_bounded(&bars->v_full[j & 1], (j >> 1) & 1, abort, kWaitNs)) return false;
+        if (!tc::mbar_wait_warp(&bars->p_ready, j & 1, abort, kWaitNs)) return false;
+        if (!tc::mbar_wait_warp(&bars->v_full[j & 1], (j >> 1) & 1, abort, kWaitNs)) return false;
         tc::tc_fence_after();
         const uint32_t v_addr = tc::smem_u32(smem + S::V_OFF + (j & 1) * S::TILE);
 #pragma unroll
         for (int k = 0; k < BKV / 16; ++k)
-          tc::mma_bf16_ss(t_o, tc::smem_desc_sw128(p_addr + (k >> 2) * CH + (k & 3) * 32, 16),
+          tc::mma_bf16_ss_elect(t_o, tc::smem_desc_sw128(p_addr + (k >> 2) * CH + (k & 3) * 32, 16),
                           tc::smem_desc_sw128(v_addr + k * 2048, CH), idesc_pv, (j | k) != 0);
-        tc::mma_commit(&bars->pv_full);
-        tc::mma_commit(&bars->v_empty[j & 1]);
+        tc::mma_commit_elect(&bars->pv_full);
+        tc::mma_commit_elect(&bars->v_empty[j & 1]);
         return true;
       };
       for (int j = 0; ok && j < n_kv; ++j) {
         const int st = j & 1;
-        if (!tc::mbar_wait_bounded(&bars->k_full[st], (j >> 1) & 1, abort, kWaitNs)) { ok = false; break; }
+        if (!tc::mbar_wait_warp(&bars->k_full[st], (j >> 1) & 1, abort, kWaitNs)) { ok = false; break; }
         tc::tc_fence_after();
         const uint32_t k_addr = tc::smem_u32(smem + S::K_OFF + st * S::TILE);
 #pragma unroll
         for (int k = 0; k < HD / 16; ++k) {
           const uint32_t off = (k >> 2) * CH + (k & 3) * 32;
-          tc::mma_bf16_ss(tmem + st * 128, tc::smem_desc_sw128(q_addr + off, 16),
+          tc::mma_bf16_ss_elect(tmem + st * 128, tc::smem_desc_sw128(q_addr + off, 16),
                           tc::smem_desc_sw128(k_addr + off, 16), idesc_s, k != 0);
         }
         issued_any = true;
-        tc::mma_commit(&bars->s_full[st]);
-        tc::mma_commit(&bars->k_empty[st]);
+        tc::mma_commit_elect(&bars->s_full[st]);
+        tc::mma_commit_elect(&bars->k_empty[st]);
         if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
       }
       if (ok && n_kv >= 1) ok = issue_pv(n_kv - 1);
       if (!ok) {
-        record_status(status, GPT_ETIMEOUT, K_ATTN, 11);
+        if (lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 11);
         *abort = 1;
       }
       if (issued_any) {
-        tc::mma_commit(&bars->done);
-        tc::mbar_wait_bounded(&bars->done, 0, nullptr, kWaitNs);
+        tc::mma_commit_elect(&bars->done);
+        tc::mbar_wait_warp(&bars->done, 0, nullptr, kWaitNs);
       }
     }
   } else {
@@ -451,16 +464,19 @@ __global__ void attn_rowdot_kernel(const __nv_bfloat16* __restrict__ dO,
   }
 }
 
-constexpr int kRing = 3;    // slots of the per-step operand ring (dK/dV kernel)
+constexpr int kRing = 6;    // slots of the Q/dO ring of the dK/dV kernel
 constexpr int kRingQ = 4;   // slots of the K/V ring of the dQ kernel
+constexpr int kQ = 32;      // queries per step of the dK/dV kernel
+constexpr int kRingMax = kRing > kRingQ ? kRing : kRingQ;
 
 struct BwdBars {
   uint64_t fixed_full;
-  uint64_t ring_full[kRingQ];
-  uint64_t ring_empty[kRingQ];
+  uint64_t ring_full[kRingMax];
+  uint64_t ring_empty[kRingMax];
   uint64_t s_full[2];
   uint64_t ds_ready[2];
   uint64_t acc_full;
+  uint64_t epi_full;
   uint64_t done;
   uint32_t tmem_base;
   int abort;
@@ -468,22 +484,27 @@ struct BwdBars {
 
 // One row's gradient w.r.t. its normalised, rotated q or k (TMEM, fp32, HD
 // columns at `taddr`, times `scale`) back through RMSNorm (y: the normalised
-// row, rr: its 1/rms) and RoPE, written as bf16.  The row's two compute
-// threads split the rotation pairs: thread `half` takes pairs i in
+// row, rr: its 1/rms) and RoPE, written as bf16.  y, cos and sin come from
+// shared-memory tiles of the CTA's 128 rows, stored as TMA writes them with the
+// 128-byte swizzle: y [128 x HD] bf16 in 64-column chunks, cos / sin
+// [128 x HD/2] fp32 in 32-column chunks (16 KB per chunk).  The row's two
+// compute threads split the rotation pairs: thread `half` takes pairs i in
 // [half*HD/4, (half+1)*HD/4) and their partners i + HD/2; the mean(g y) of the
 // norm is summed across both through `red` (one compute_bar, reached on every
 // path).
+__device__ __forceinline__ uint32_t tile_unit(int r, int unit) {  // 16-byte unit of row r
+  return uint32_t(unit >> 3) * (128 * 128) + r * 128 + (((unit & 7) ^ (r & 7)) << 4);
+}
 template <int HD>
 __device__ __forceinline__ void norm_rope_bwd_half(uint32_t taddr, int half, int r, float scale,
-                                                   const __nv_bfloat16* __restrict__ y,
-                                                   float rr, int qk_norm,
-                                                   const float* __restrict__ cosr,
-                                                   const float* __restrict__ sinr,
+                                                   const uint8_t* y_tile, float rr, int qk_norm,
+                                                   const uint8_t* cos_tile, const uint8_t* sin_tile,
                                                    __nv_bfloat16* __restrict__ out, bool ok,
                                                    bool write, float* red) {
   constexpr int HALF = HD / 2, Q4 = HD / 4;
   const int i0 = half * Q4;
-  float ga[Q4], gb[Q4], ya[Q4], yb[Q4];
+  float ga[Q4], gb[Q4];
+  uint32_t wa[Q4 / 2], wb[Q4 / 2];  // y, kept as packed bf16 pairs
   float part = 0.f;
   if (ok) {
 #pragma unroll
@@ -496,20 +517,18 @@ __device__ __forceinline__ void norm_rope_bwd_half(uint32_t taddr, int half, int
     }
     if (write) {
 #pragma unroll
-      for (int c = 0; c < Q4; c += 8) {
-        const uint4 ua = *reinterpret_cast<const uint4*>(y + i0 + c);
-        const uint4 ub = *reinterpret_cast<const uint4*>(y + HALF + i0 + c);
-        const uint32_t wa[4] = {ua.x, ua.y, ua.z, ua.w}, wb[4] = {ub.x, ub.y, ub.z, ub.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wa[e]));
-          float2 fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wb[e]));
-          ya[c + 2 * e] = fa.x; ya[c + 2 * e + 1] = fa.y;
-          yb[c + 2 * e] = fb.x; yb[c + 2 * e + 1] = fb.y;
-        }
+      for (int c = 0; c < Q4 / 2; c += 4) {  // 8 bf16 per 16-byte unit
+        const uint4 ua = *reinterpret_cast<const uint4*>(y_tile + tile_unit(r, (i0 + 2 * c) / 8));
+        const uint4 ub = *reinterpret_cast<const uint4*>(y_tile + tile_unit(r, (HALF + i0 + 2 * c) / 8));
+        wa[c] = ua.x; wa[c + 1] = ua.y; wa[c + 2] = ua.z; wa[c + 3] = ua.w;
+        wb[c] = ub.x; wb[c + 1] = ub.y; wb[c + 2] = ub.z; wb[c + 3] = ub.w;
       }
 #pragma unroll
-      for (int i = 0; i < Q4; ++i) part += ga[i] * ya[i] + gb[i] * yb[i];
+      for (int i = 0; i < Q4 / 2; ++i) {
+        const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wa[i]));
+        const float2 fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wb[i]));
+        part += ga[2 * i] * fa.x + ga[2 * i + 1] * fa.y + gb[2 * i] * fb.x + gb[2 * i + 1] * fb.y;
+      }
     }
   }
   red[half * 128 + r] = part;
@@ -518,15 +537,22 @@ __device__ __forceinline__ void norm_rope_bwd_half(uint32_t taddr, int half, int
   if (!ok || !write) return;
   uint32_t pa[Q4 / 2], pb[Q4 / 2];
 #pragma unroll
-  for (int i = 0; i < Q4; i += 2) {
-    float a0 = ga[i], a1 = ga[i + 1], b0 = gb[i], b1 = gb[i + 1];
-    if (qk_norm) {
-      a0 = rr * (a0 - ya[i] * mean_gy); a1 = rr * (a1 - ya[i + 1] * mean_gy);
-      b0 = rr * (b0 - yb[i] * mean_gy); b1 = rr * (b1 - yb[i + 1] * mean_gy);
+  for (int i = 0; i < Q4; i += 4) {  // 4 fp32 per 16-byte unit
+    const float4 c4 = *reinterpret_cast<const float4*>(cos_tile + tile_unit(r, (i0 + i) / 4));
+    const float4 s4 = *reinterpret_cast<const float4*>(sin_tile + tile_unit(r, (i0 + i) / 4));
+    const float cc[4] = {c4.x, c4.y, c4.z, c4.w}, ss[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+    for (int e = 0; e < 4; e += 2) {
+      float a0 = ga[i + e], a1 = ga[i + e + 1], b0 = gb[i + e], b1 = gb[i + e + 1];
+      if (qk_norm) {
+        const float2 ya = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wa[(i + e) / 2]));
+        const float2 yb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wb[(i + e) / 2]));
+        a0 = rr * (a0 - ya.x * mean_gy); a1 = rr * (a1 - ya.y * mean_gy);
+        b0 = rr * (b0 - yb.x * mean_gy); b1 = rr * (b1 - yb.y * mean_gy);
+      }
+      pa[(i + e) / 2] = pack2(a0 * cc[e] + b0 * ss[e], a1 * cc[e + 1] + b1 * ss[e + 1]);
+      pb[(i + e) / 2] = pack2(-a0 * ss[e] + b0 * cc[e], -a1 * ss[e + 1] + b1 * cc[e + 1]);
     }
-    const float c0 = cosr[i0 + i], s0 = sinr[i0 + i], c1 = cosr[i0 + i + 1], s1 = sinr[i0 + i + 1];
-    pa[i / 2] = pack2(a0 * c0 + b0 * s0, a1 * c1 + b1 * s1);
-    pb[i / 2] = pack2(-a0 * s0 + b0 * c0, -a1 * s1 + b1 * c1);
   }
 #pragma unroll
   for (int i = 0; i < Q4 / 2; i += 4) {
@@ -535,31 +561,74 @@ __device__ __forceinline__ void norm_rope_bwd_half(uint32_t taddr, int half, int
   }
 }
 
+// The epilogue's inputs for 128 rows, loaded by TMA onto `bar`: the y rows
+// (bh*T + row0 ..) of a head-major [B*H*T, HD] tensor and the cos / sin table
+// rows (pos0 ..) of [T, HD/2] fp32.
+template <int HD>
+__device__ __forceinline__ void load_epilogue_tiles(uint8_t* y_dst, uint8_t* cos_dst, uint8_t* sin_dst,
+                                                    const CUtensorMap* map_y, const CUtensorMap* map_cos,
+                                                    const CUtensorMap* map_sin, uint64_t* bar,
+                                                    int y_row0, int pos0) {
+  constexpr int NCH = HD / 64;
+  tc::mbar_arrive_expect_tx(bar, 3u * 128 * HD * 2);
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) {
+    tc::tma_load_2d(y_dst + c * (128 * 128), map_y, bar, c * 64, y_row0);
+    tc::tma_load_2d(cos_dst + c * (128 * 128), map_cos, bar, c * 32, pos0);
+    tc::tma_load_2d(sin_dst + c * (128 * 128), map_sin, bar, c * 32, pos0);
+  }
+}
+
 template <int HD>
 struct DqSmem {
-  static constexpr uint32_t BIG = 128 * HD * 2;
   static constexpr uint32_t SMALL = kInner * HD * 2;
-  static constexpr uint32_t DS = 128 * kInner * 2;
-  static constexpr uint32_t Q_OFF = 0, DO_OFF = BIG, K_OFF = 2 * BIG;
+  static constexpr uint32_t EPI = 128 * HD * 2;  // one epilogue tile (y, cos or sin)
+  static constexpr uint32_t K_OFF = 0;
   static constexpr uint32_t V_OFF = K_OFF + kRingQ * SMALL;
-  static constexpr uint32_t DS_OFF = V_OFF + kRingQ * SMALL;
-  static constexpr uint32_t RED_OFF = DS_OFF + 2 * DS;
+  static constexpr uint32_t Y_OFF = V_OFF + kRingQ * SMALL;
+  static constexpr uint32_t COS_OFF = Y_OFF + EPI, SIN_OFF = COS_OFF + EPI;
+  static constexpr uint32_t RED_OFF = SIN_OFF + EPI;
   static constexpr uint32_t BAR_OFF = RED_OFF + 2 * 128 * 4;
   static constexpr uint32_t BYTES = BAR_OFF + 256 + 1024;
-  static_assert(K_OFF % 1024 == 0 && V_OFF % 1024 == 0 && DS_OFF % 1024 == 0, "");
+  static_assert(K_OFF % 1024 == 0 && V_OFF % 1024 == 0 && Y_OFF % 1024 == 0 && EPI % 1024 == 0, "");
+  static_assert(BYTES <= 232448, "");
 };
+
+// Half a bf16 row (HD/2 elements from `src`, zeros when !valid) into TMEM
+// columns taddr .. taddr + HD/4 of this thread's lane: the K-major layout of
+// an MMA A operand, two elements per column.
+template <int HD>
+__device__ __forceinline__ void stage_half_row(uint32_t taddr, const __nv_bfloat16* __restrict__ src,
+                                               bool valid) {
+  constexpr int W = HD / 4;
+  uint32_t w[W];
+#pragma unroll
+  for (int i = 0; i < W / 4; ++i) {
+    const uint4 u = valid ? reinterpret_cast<const uint4*>(src)[i] : make_uint4(0u, 0u, 0u, 0u);
+    w[4 * i] = u.x; w[4 * i + 1] = u.y; w[4 * i + 2] = u.z; w[4 * i + 3] = u.w;
+  }
+  if constexpr (W == 32) tc::tmem_st_32x32b_x32(taddr, w);
+  else tc::tmem_st_32x32b_x16(taddr, w);
+}
 
 }  // namespace
 
-// dQ for 128 queries of one (batch, head), looping over 64-key tiles.  Compute
-// thread (row, half) handles keys [32*half, 32*half + 32) of each tile.
+// dQ for 128 queries of one (batch, head), looping over 64-key tiles.  Q and dO
+// (fixed for the CTA) sit in TMEM as the A operands of S = Q K^T and
+// dP = dO V^T, so each MMA reads only its K or V slice from shared memory.
+// Compute thread (row, half) handles keys [32*half, 32*half + 32) of each tile
+// and writes its bf16 dS over its own S columns, the TMEM A operand of
+// dQ += dS K.  TMEM: S/dP pairs at columns 0 and 128 (64 + 64 each), dQ at
+// 256, Q at 384, dO at 448.
 template <int HD>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_dq_tc_kernel(const __grid_constant__ CUtensorMap map_q128,
-                      const __grid_constant__ CUtensorMap map_do128,
-                      const __grid_constant__ CUtensorMap map_k64,
+    attn_dq_tc_kernel(const __grid_constant__ CUtensorMap map_k64,
                       const __grid_constant__ CUtensorMap map_v64,
-                      const __nv_bfloat16* __restrict__ qn, const float* __restrict__ lse,
+                      const __grid_constant__ CUtensorMap map_y,
+                      const __grid_constant__ CUtensorMap map_cos,
+                      const __grid_constant__ CUtensorMap map_sin,
+                      const __nv_bfloat16* __restrict__ qn, const __nv_bfloat16* __restrict__ dO,
+                      const float* __restrict__ lse,
                       const float* __restrict__ D, const float* __restrict__ rq,
                       const float* __restrict__ cos_t, const float* __restrict__ sin_t,
                       __nv_bfloat16* __restrict__ dqkv, int H, int T, float scale,
@@ -577,9 +646,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int q0 = qt * 128;
   const int n_steps = (min(q0 + 128, T) + kInner - 1) / kInner;
   constexpr int NCH = HD / 64;
+  constexpr uint32_t Q_COL = 384, DO_COL = 448;
 
   ATTN_PROLOGUE(bars, {
-    tc::mbar_init(&bars->fixed_full, 1);
+    tc::mbar_init(&bars->fixed_full, 256);  // the compute threads' Q / dO stores
+    tc::mbar_init(&bars->epi_full, 1);
     for (int s = 0; s < kRingQ; ++s) {
       tc::mbar_init(&bars->ring_full[s], 1);
       tc::mbar_init(&bars->ring_empty[s], 1);
@@ -593,18 +664,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   })
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort = &bars->abort;
-  const uint32_t t_dq = tmem + 256;  // S/dP pairs at columns 0 and 128 (64 + 64 each)
+  const uint32_t t_dq = tmem + 256;
 
   if (warp == 0) {
     if (lane == 0) {
       uint32_t issued = 0, last_par = 0;
-      tc::mbar_arrive_expect_tx(&bars->fixed_full, 2 * S::BIG);
-#pragma unroll
-      for (int c = 0; c < NCH; ++c) {
-        tc::tma_load_2d(smem + S::Q_OFF + c * (128 * 128), &map_q128, &bars->fixed_full, c * 64, bh * T + q0);
-        tc::tma_load_2d(smem + S::DO_OFF + c * (128 * 128), &map_do128, &bars->fixed_full,
-                        h * HD + c * 64, b * T + q0);
-      }
       for (int j = 0; j < n_steps; ++j) {
         const int st = j % kRingQ;
         const uint32_t ph = (j / kRingQ) & 1;
@@ -621,70 +685,78 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::tma_load_2d(smem + S::V_OFF + st * S::SMALL + c * (kInner * 128), &map_v64,
                           &bars->ring_full[st], c * 64, bh * T + j * kInner);
         }
+        if (j == 0)
+          load_epilogue_tiles<HD>(smem + S::Y_OFF, smem + S::COS_OFF, smem + S::SIN_OFF, &map_y,
+                                  &map_cos, &map_sin, &bars->epi_full, bh * T + q0, q0);
         issued |= 1u << st;
         last_par = (last_par & ~(1u << st)) | (ph << st);
       }
       if (*abort) {
-        tc::mbar_wait_bounded(&bars->fixed_full, 0, nullptr, kWaitNs);
+        if (issued) tc::mbar_wait_bounded(&bars->epi_full, 0, nullptr, kWaitNs);
         for (int s = 0; s < kRingQ; ++s)
           if (issued >> s & 1) tc::mbar_wait_bounded(&bars->ring_full[s], (last_par >> s) & 1, nullptr, kWaitNs);
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    {  // the whole warp runs the MMA loop; elect.sync issues
       constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, kInner, false, false);
       constexpr uint32_t idesc_dq = tc::idesc_bf16_f32(128, HD, false, true);
-      const uint32_t q_addr = tc::smem_u32(smem + S::Q_OFF);
-      const uint32_t do_addr = tc::smem_u32(smem + S::DO_OFF);
-      bool ok = tc::mbar_wait_bounded(&bars->fixed_full, 0, abort, kWaitNs);
+      bool ok = tc::mbar_wait_warp(&bars->fixed_full, 0, abort, kWaitNs);
+      tc::tc_fence_after();
       bool issued_any = false;
       auto issue_dq = [&](int j) -> bool {
-        if (!tc::mbar_wait_bounded(&bars->ds_ready[j & 1], (j >> 1) & 1, abort, kWaitNs)) return false;
+        if (!tc::mbar_wait_warp(&bars->ds_ready[j & 1], (j >> 1) & 1, abort, kWaitNs)) return false;
         tc::tc_fence_after();
-        const uint32_t ds_addr = tc::smem_u32(smem + S::DS_OFF + (j & 1) * S::DS);
-        const uint32_t k_addr = tc::smem_u32(smem + S::K_OFF + (j % kRingQ) * S::SMALL);
+        const uint32_t ds_t = tmem + (j & 1) * 128;
+        const uint64_t kb = tc::smem_desc_sw128(tc::smem_u32(smem + S::K_OFF + (j % kRingQ) * S::SMALL),
+                                                kInner * 128);
 #pragma unroll
         for (int k = 0; k < kInner / 16; ++k)
-          tc::mma_bf16_ss(t_dq, tc::smem_desc_sw128(ds_addr + k * 32, 16),
-                          tc::smem_desc_sw128(k_addr + k * 2048, kInner * 128), idesc_dq, (j | k) != 0);
-        tc::mma_commit(&bars->ring_empty[j % kRingQ]);
+          tc::mma_bf16_ts_elect(t_dq, ds_t + 32 * (k >> 1) + 8 * (k & 1), tc::desc_advance(kb, k * 2048),
+                          idesc_dq, (j | k) != 0);
+        tc::mma_commit_elect(&bars->ring_empty[j % kRingQ]);
         return true;
       };
       for (int j = 0; ok && j < n_steps; ++j) {
         const int st = j % kRingQ;
-        if (!tc::mbar_wait_bounded(&bars->ring_full[st], (j / kRingQ) & 1, abort, kWaitNs)) { ok = false; break; }
+        if (!tc::mbar_wait_warp(&bars->ring_full[st], (j / kRingQ) & 1, abort, kWaitNs)) { ok = false; break; }
         tc::tc_fence_after();
-        const uint32_t k_addr = tc::smem_u32(smem + S::K_OFF + st * S::SMALL);
-        const uint32_t v_addr = tc::smem_u32(smem + S::V_OFF + st * S::SMALL);
+        const uint64_t kd = tc::smem_desc_sw128(tc::smem_u32(smem + S::K_OFF + st * S::SMALL), 16);
+        const uint64_t vd = tc::smem_desc_sw128(tc::smem_u32(smem + S::V_OFF + st * S::SMALL), 16);
         const uint32_t pair = tmem + (j & 1) * 128;
 #pragma unroll
         for (int k = 0; k < HD / 16; ++k) {
-          const uint32_t big = (k >> 2) * (128 * 128) + (k & 3) * 32;
           const uint32_t small = (k >> 2) * (kInner * 128) + (k & 3) * 32;
-          tc::mma_bf16_ss(pair, tc::smem_desc_sw128(q_addr + big, 16),
-                          tc::smem_desc_sw128(k_addr + small, 16), idesc_s, k != 0);
-          tc::mma_bf16_ss(pair + kInner, tc::smem_desc_sw128(do_addr + big, 16),
-                          tc::smem_desc_sw128(v_addr + small, 16), idesc_s, k != 0);
+          tc::mma_bf16_ts_elect(pair, tmem + Q_COL + 8 * k, tc::desc_advance(kd, small), idesc_s, k != 0);
+          tc::mma_bf16_ts_elect(pair + kInner, tmem + DO_COL + 8 * k, tc::desc_advance(vd, small), idesc_s, k != 0);
         }
         issued_any = true;
-        tc::mma_commit(&bars->s_full[j & 1]);
+        tc::mma_commit_elect(&bars->s_full[j & 1]);
         if (j >= 1 && !issue_dq(j - 1)) { ok = false; break; }
       }
       if (ok && n_steps >= 1) ok = issue_dq(n_steps - 1);
-      if (ok) tc::mma_commit(&bars->acc_full);
+      if (ok) tc::mma_commit_elect(&bars->acc_full);
       if (!ok) {
-        record_status(status, GPT_ETIMEOUT, K_ATTN, 21);
+        if (lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 21);
         *abort = 1;
       }
       if (issued_any) {
-        tc::mma_commit(&bars->done);
-        tc::mbar_wait_bounded(&bars->done, 0, nullptr, kWaitNs);
+        tc::mma_commit_elect(&bars->done);
+        tc::mbar_wait_warp(&bars->done, 0, nullptr, kWaitNs);
       }
     }
   } else {
     const Roles R = roles();
     const int q = q0 + R.r;
     const bool qv = q < T;
+    const int tq = qv ? q : 0;
+    stage_half_row<HD>(tmem + Q_COL + R.lane_off + R.half * (HD / 4),
+                       qn + (int64_t(bh) * T + tq) * HD + R.half * (HD / 2), qv);
+    stage_half_row<HD>(tmem + DO_COL + R.lane_off + R.half * (HD / 4),
+                       dO + (int64_t(b) * T + tq) * (int64_t(H) * HD) + h * HD + R.half * (HD / 2), qv);
+    tc::tmem_wait_st();
+    tc::tc_fence_before();
+    tc::mbar_arrive(&bars->fixed_full);
     const float lse2 = qv ? lse[int64_t(bh) * T + q] * kLog2e : 0.f;
     const float Dq = qv ? D[int64_t(bh) * T + q] : 0.f;
     bool ok = true;
@@ -694,34 +766,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) {
         tc::tc_fence_after();
         const int k0 = j * kInner + R.half * 32;
+        const uint32_t ts = tmem + sb * 128 + R.lane_off + R.half * 32;
         uint32_t us[32], up[32];
-        tc::tmem_ld_32x32b_x32(tmem + sb * 128 + R.lane_off + R.half * 32, us);
-        tc::tmem_ld_32x32b_x32(tmem + sb * 128 + kInner + R.lane_off + R.half * 32, up);
+        tc::tmem_ld_32x32b_x32(ts, us);
+        tc::tmem_ld_32x32b_x32(ts + kInner, up);
         tc::tmem_wait_ld();
         const bool need_mask = !qv || k0 + 32 > q || k0 + 32 > T;
-        uint8_t* rowp = smem + S::DS_OFF + sb * S::DS;
+        uint32_t pk[16];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          uint32_t pk[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int i = u * 8 + 2 * e;
-            float p0 = ex2(fmaf(__uint_as_float(us[i]), scale_log2, -lse2));
-            float p1 = ex2(fmaf(__uint_as_float(us[i + 1]), scale_log2, -lse2));
-            if (need_mask) {
-              if (k0 + i > q || k0 + i >= T || !qv) p0 = 0.f;
-              if (k0 + i + 1 > q || k0 + i + 1 >= T || !qv) p1 = 0.f;
-            }
-            pk[e] = pack2(p0 * (__uint_as_float(up[i]) - Dq), p1 * (__uint_as_float(up[i + 1]) - Dq));
+        for (int e = 0; e < 16; ++e) {
+          const int i = 2 * e;
+          float p0 = ex2(fmaf(__uint_as_float(us[i]), scale_log2, -lse2));
+          float p1 = ex2(fmaf(__uint_as_float(us[i + 1]), scale_log2, -lse2));
+          if (need_mask) {
+            if (k0 + i > q || k0 + i >= T || !qv) p0 = 0.f;
+            if (k0 + i + 1 > q || k0 + i + 1 >= T || !qv) p1 = 0.f;
           }
-          *reinterpret_cast<uint4*>(rowp + sw_off(R.r, R.half * 4 + u)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          pk[e] = pack2(p0 * (__uint_as_float(up[i]) - Dq), p1 * (__uint_as_float(up[i + 1]) - Dq));
         }
-        fence_async_smem();
+        tc::tmem_st_32x32b_x16(ts, pk);  // dS over this thread's own S columns
+        tc::tmem_wait_st();
         tc::tc_fence_before();
       }
       tc::mbar_arrive(&bars->ds_ready[sb]);
     }
     if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->acc_full, 0, abort, kWaitNs));
+    if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->epi_full, 0, abort, kWaitNs));
     if (!ok) {
       if (R.lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 22);
       *abort = 1;
@@ -729,10 +799,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tc_fence_after();
     }
     const int d = H * HD;
-    const int tq = qv ? q : 0;
-    norm_rope_bwd_half<HD>(t_dq + R.lane_off, R.half, R.r, scale, qn + (int64_t(bh) * T + tq) * HD,
-                           qv ? rq[int64_t(bh) * T + q] : 0.f, qk_norm, cos_t + tq * (HD / 2),
-                           sin_t + tq * (HD / 2), dqkv + (int64_t(b) * T + tq) * 3 * d + h * HD, ok,
+    norm_rope_bwd_half<HD>(t_dq + R.lane_off, R.half, R.r, scale, smem + S::Y_OFF,
+                           qv ? rq[int64_t(bh) * T + q] : 0.f, qk_norm, smem + S::COS_OFF,
+                           smem + S::SIN_OFF, dqkv + (int64_t(b) * T + tq) * 3 * d + h * HD, ok,
                            qv, reinterpret_cast<float*>(smem + S::RED_OFF));
   }
   ATTN_EPILOGUE(tmem)
@@ -741,33 +810,38 @@ __global__ void __launch_bounds__(kThreads, 1)
 namespace {
 template <int HD>
 struct DkvSmem {
-  static constexpr uint32_t BIG = 128 * HD * 2;
-  static constexpr uint32_t SMALL = kInner * HD * 2;
-  static constexpr uint32_t PT = 128 * kInner * 2;
-  static constexpr uint32_t K_OFF = 0, V_OFF = BIG, Q_OFF = 2 * BIG;
+  static constexpr uint32_t SMALL = kQ * HD * 2;
+  static constexpr uint32_t Q_OFF = 0;
+  static constexpr uint32_t EPI = 128 * HD * 2;  // one epilogue tile (y, cos or sin)
   static constexpr uint32_t DO_OFF = Q_OFF + kRing * SMALL;
-  // swizzled tiles first: each must start on a 1024-byte boundary
-  static constexpr uint32_t P_OFF = DO_OFF + kRing * SMALL;
-  static constexpr uint32_t DS_OFF = P_OFF + 2 * PT;
-  static constexpr uint32_t STAT_OFF = DS_OFF + 2 * PT;  // [ring][lse2 x 64 | D x 64]
-  static constexpr uint32_t RED_OFF = P_OFF;  // epilogue only, after the last P is consumed
-  static constexpr uint32_t BAR_OFF = STAT_OFF + kRing * 2 * kInner * 4;
-  static_assert(P_OFF % 1024 == 0 && DS_OFF % 1024 == 0 && DO_OFF % 1024 == 0, "");
+  static constexpr uint32_t Y_OFF = DO_OFF + kRing * SMALL;
+  static constexpr uint32_t COS_OFF = Y_OFF + EPI, SIN_OFF = COS_OFF + EPI;
+  static constexpr uint32_t STAT_OFF = SIN_OFF + EPI;  // [ring][lse2 x kQ | D x kQ]
+  static constexpr uint32_t RED_OFF = STAT_OFF + kRing * 2 * kQ * 4;
+  static constexpr uint32_t BAR_OFF = RED_OFF + 2 * 128 * 4;
+  static_assert(Q_OFF % 1024 == 0 && DO_OFF % 1024 == 0 && SMALL % 1024 == 0 && Y_OFF % 1024 == 0 &&
+                EPI % 1024 == 0, "");
   static constexpr uint32_t BYTES = BAR_OFF + 256 + 1024;
 };
 }  // namespace
 
-// dK, dV for 128 keys of one (batch, head), looping over 64-query tiles.
-// Compute thread (key row, half) handles queries [32*half, 32*half + 32) of
-// each tile; the producer warp stages lse and D of the tile's queries in
-// shared memory next to the Q / dO tiles.
+// dK, dV for 128 keys of one (batch, head), looping over 32-query tiles.  K and
+// V (fixed for the CTA) sit in TMEM as the A operands of S^T = K Q^T and
+// dP^T = V dO^T.  Compute thread (key row, half) handles queries
+// [16*half, 16*half + 16) of each tile and writes bf16 P^T and dS^T over its own
+// S^T and dP^T columns: the TMEM A operands of dV += P^T dO and dK += dS^T Q.
+// The producer warp stages lse and D of the tile's queries in shared memory
+// next to the Q / dO tiles.  TMEM: S^T/dP^T pairs at columns 0 and 64 (32 + 32
+// each), dV at 128, dK at 256, K at 384, V at 448.
 template <int HD>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_dkv_tc_kernel(const __grid_constant__ CUtensorMap map_k128,
-                       const __grid_constant__ CUtensorMap map_v128,
-                       const __grid_constant__ CUtensorMap map_q64,
-                       const __grid_constant__ CUtensorMap map_do64,
-                       const __nv_bfloat16* __restrict__ kn, const float* __restrict__ lse,
+    attn_dkv_tc_kernel(const __grid_constant__ CUtensorMap map_q32,
+                       const __grid_constant__ CUtensorMap map_do32,
+                       const __grid_constant__ CUtensorMap map_y,
+                       const __grid_constant__ CUtensorMap map_cos,
+                       const __grid_constant__ CUtensorMap map_sin,
+                       const __nv_bfloat16* __restrict__ kn, const __nv_bfloat16* __restrict__ vh,
+                       const float* __restrict__ lse,
                        const float* __restrict__ D, const float* __restrict__ rk,
                        const float* __restrict__ cos_t, const float* __restrict__ sin_t,
                        __nv_bfloat16* __restrict__ dqkv, int H, int T, float scale,
@@ -783,12 +857,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kt = int(blockIdx.x) % n_kt;
   const int b = bh / H, h = bh % H;
   const int k0 = kt * 128;
-  const int i_begin = k0 / kInner;
-  const int n_steps = (T + kInner - 1) / kInner - i_begin;
+  const int n_steps = (T - k0 + kQ - 1) / kQ;  // causal: queries k0 .. T-1
   constexpr int NCH = HD / 64;
+  constexpr uint32_t K_COL = 384, V_COL = 448;
 
   ATTN_PROLOGUE(bars, {
-    tc::mbar_init(&bars->fixed_full, 1);
+    tc::mbar_init(&bars->fixed_full, 256);  // the compute threads' K / V stores
+    tc::mbar_init(&bars->epi_full, 1);
     for (int s = 0; s < kRing; ++s) {
       tc::mbar_init(&bars->ring_full[s], 1 + 32);  // TMA bytes + the producer warp's stat stores
       tc::mbar_init(&bars->ring_empty[s], 1);
@@ -802,22 +877,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   })
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort = &bars->abort;
-  const uint32_t t_dv = tmem + 256, t_dk = tmem + 256 + HD;
+  const uint32_t t_dv = tmem + 128, t_dk = tmem + 256;
 
   if (warp == 0) {
     uint32_t issued = 0, last_par = 0;
-    if (lane == 0) {
-      tc::mbar_arrive_expect_tx(&bars->fixed_full, 2 * S::BIG);
-#pragma unroll
-      for (int c = 0; c < NCH; ++c) {
-        tc::tma_load_2d(smem + S::K_OFF + c * (128 * 128), &map_k128, &bars->fixed_full, c * 64, bh * T + k0);
-        tc::tma_load_2d(smem + S::V_OFF + c * (128 * 128), &map_v128, &bars->fixed_full, c * 64, bh * T + k0);
-      }
-    }
     for (int j = 0; j < n_steps; ++j) {
       const int st = j % kRing;
       const uint32_t ph = (j / kRing) & 1;
-      const int qs = (i_begin + j) * kInner;
+      const int qs = k0 + j * kQ;
       const bool ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->ring_empty[st], ph ^ 1, abort, kWaitNs));
       if (!ok) {
         if (lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 30);
@@ -828,89 +895,89 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mbar_arrive_expect_tx(&bars->ring_full[st], 2 * S::SMALL);
 #pragma unroll
         for (int c = 0; c < NCH; ++c) {
-          tc::tma_load_2d(smem + S::Q_OFF + st * S::SMALL + c * (kInner * 128), &map_q64,
+          tc::tma_load_2d(smem + S::Q_OFF + st * S::SMALL + c * (kQ * 128), &map_q32,
                           &bars->ring_full[st], c * 64, bh * T + qs);
-          tc::tma_load_2d(smem + S::DO_OFF + st * S::SMALL + c * (kInner * 128), &map_do64,
+          tc::tma_load_2d(smem + S::DO_OFF + st * S::SMALL + c * (kQ * 128), &map_do32,
                           &bars->ring_full[st], h * HD + c * 64, b * T + qs);
         }
+        if (j == 0)
+          load_epilogue_tiles<HD>(smem + S::Y_OFF, smem + S::COS_OFF, smem + S::SIN_OFF, &map_y,
+                                  &map_cos, &map_sin, &bars->epi_full, bh * T + k0, k0);
       }
-      float* stat = reinterpret_cast<float*>(smem + S::STAT_OFF) + st * 2 * kInner;
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int qi = lane * 2 + e;
-        const int qq = qs + qi;
-        stat[qi] = qq < T ? lse[int64_t(bh) * T + qq] * kLog2e : 0.f;
-        stat[kInner + qi] = qq < T ? D[int64_t(bh) * T + qq] : 0.f;
-      }
+      float* stat = reinterpret_cast<float*>(smem + S::STAT_OFF) + st * 2 * kQ;
+      const int qq = qs + lane;
+      stat[lane] = qq < T ? lse[int64_t(bh) * T + qq] * kLog2e : 0.f;
+      stat[kQ + lane] = qq < T ? D[int64_t(bh) * T + qq] : 0.f;
       tc::mbar_arrive(&bars->ring_full[st]);
       issued |= 1u << st;
       last_par = (last_par & ~(1u << st)) | (ph << st);
     }
     if (lane == 0 && *abort) {
-      tc::mbar_wait_bounded(&bars->fixed_full, 0, nullptr, kWaitNs);
+      if (issued) tc::mbar_wait_bounded(&bars->epi_full, 0, nullptr, kWaitNs);
       for (int s = 0; s < kRing; ++s)
         if (issued >> s & 1) tc::mbar_wait_bounded(&bars->ring_full[s], (last_par >> s) & 1, nullptr, kWaitNs);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, kInner, false, false);
+    {  // the whole warp runs the MMA loop; elect.sync issues
+      constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, kQ, false, false);
       constexpr uint32_t idesc_acc = tc::idesc_bf16_f32(128, HD, false, true);
-      const uint32_t k_addr = tc::smem_u32(smem + S::K_OFF);
-      const uint32_t v_addr = tc::smem_u32(smem + S::V_OFF);
-      bool ok = tc::mbar_wait_bounded(&bars->fixed_full, 0, abort, kWaitNs);
+      bool ok = tc::mbar_wait_warp(&bars->fixed_full, 0, abort, kWaitNs);
+      tc::tc_fence_after();
       bool issued_any = false;
       auto issue_acc = [&](int j) -> bool {
-        if (!tc::mbar_wait_bounded(&bars->ds_ready[j & 1], (j >> 1) & 1, abort, kWaitNs)) return false;
+        if (!tc::mbar_wait_warp(&bars->ds_ready[j & 1], (j >> 1) & 1, abort, kWaitNs)) return false;
         tc::tc_fence_after();
-        const uint32_t p_addr = tc::smem_u32(smem + S::P_OFF + (j & 1) * S::PT);
-        const uint32_t ds_addr = tc::smem_u32(smem + S::DS_OFF + (j & 1) * S::PT);
-        const uint32_t q_addr = tc::smem_u32(smem + S::Q_OFF + (j % kRing) * S::SMALL);
-        const uint32_t do_addr = tc::smem_u32(smem + S::DO_OFF + (j % kRing) * S::SMALL);
+        const uint32_t pt = tmem + (j & 1) * 64;  // P^T over S^T, dS^T over dP^T
+        const uint64_t qmn = tc::smem_desc_sw128(tc::smem_u32(smem + S::Q_OFF + (j % kRing) * S::SMALL), kQ * 128);
+        const uint64_t domn = tc::smem_desc_sw128(tc::smem_u32(smem + S::DO_OFF + (j % kRing) * S::SMALL), kQ * 128);
 #pragma unroll
-        for (int k = 0; k < kInner / 16; ++k) {
-          tc::mma_bf16_ss(t_dv, tc::smem_desc_sw128(p_addr + k * 32, 16),
-                          tc::smem_desc_sw128(do_addr + k * 2048, kInner * 128), idesc_acc, (j | k) != 0);
-          tc::mma_bf16_ss(t_dk, tc::smem_desc_sw128(ds_addr + k * 32, 16),
-                          tc::smem_desc_sw128(q_addr + k * 2048, kInner * 128), idesc_acc, (j | k) != 0);
+        for (int k = 0; k < kQ / 16; ++k) {
+          tc::mma_bf16_ts_elect(t_dv, pt + 16 * k, tc::desc_advance(domn, k * 2048), idesc_acc, (j | k) != 0);
+          tc::mma_bf16_ts_elect(t_dk, pt + 32 + 16 * k, tc::desc_advance(qmn, k * 2048), idesc_acc, (j | k) != 0);
         }
-        tc::mma_commit(&bars->ring_empty[j % kRing]);
+        tc::mma_commit_elect(&bars->ring_empty[j % kRing]);
         return true;
       };
       for (int j = 0; ok && j < n_steps; ++j) {
         const int st = j % kRing;
-        if (!tc::mbar_wait_bounded(&bars->ring_full[st], (j / kRing) & 1, abort, kWaitNs)) { ok = false; break; }
+        if (!tc::mbar_wait_warp(&bars->ring_full[st], (j / kRing) & 1, abort, kWaitNs)) { ok = false; break; }
         tc::tc_fence_after();
-        const uint32_t q_addr = tc::smem_u32(smem + S::Q_OFF + st * S::SMALL);
-        const uint32_t do_addr = tc::smem_u32(smem + S::DO_OFF + st * S::SMALL);
-        const uint32_t pair = tmem + (j & 1) * 128;
+        const uint64_t qd = tc::smem_desc_sw128(tc::smem_u32(smem + S::Q_OFF + st * S::SMALL), 16);
+        const uint64_t dod = tc::smem_desc_sw128(tc::smem_u32(smem + S::DO_OFF + st * S::SMALL), 16);
+        const uint32_t pair = tmem + (j & 1) * 64;
 #pragma unroll
         for (int k = 0; k < HD / 16; ++k) {
-          const uint32_t big = (k >> 2) * (128 * 128) + (k & 3) * 32;
-          const uint32_t small = (k >> 2) * (kInner * 128) + (k & 3) * 32;
-          tc::mma_bf16_ss(pair, tc::smem_desc_sw128(k_addr + big, 16),
-                          tc::smem_desc_sw128(q_addr + small, 16), idesc_s, k != 0);
-          tc::mma_bf16_ss(pair + kInner, tc::smem_desc_sw128(v_addr + big, 16),
-                          tc::smem_desc_sw128(do_addr + small, 16), idesc_s, k != 0);
+          const uint32_t small = (k >> 2) * (kQ * 128) + (k & 3) * 32;
+          tc::mma_bf16_ts_elect(pair, tmem + K_COL + 8 * k, tc::desc_advance(qd, small), idesc_s, k != 0);
+          tc::mma_bf16_ts_elect(pair + kQ, tmem + V_COL + 8 * k, tc::desc_advance(dod, small), idesc_s, k != 0);
         }
         issued_any = true;
-        tc::mma_commit(&bars->s_full[j & 1]);
+        tc::mma_commit_elect(&bars->s_full[j & 1]);
         if (j >= 1 && !issue_acc(j - 1)) { ok = false; break; }
       }
       if (ok && n_steps >= 1) ok = issue_acc(n_steps - 1);
-      if (ok) tc::mma_commit(&bars->acc_full);
+      if (ok) tc::mma_commit_elect(&bars->acc_full);
       if (!ok) {
-        record_status(status, GPT_ETIMEOUT, K_ATTN, 31);
+        if (lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 31);
         *abort = 1;
       }
       if (issued_any) {
-        tc::mma_commit(&bars->done);
-        tc::mbar_wait_bounded(&bars->done, 0, nullptr, kWaitNs);
+        tc::mma_commit_elect(&bars->done);
+        tc::mbar_wait_warp(&bars->done, 0, nullptr, kWaitNs);
       }
     }
   } else {
     const Roles R = roles();
     const int key = k0 + R.r;
     const bool kv = key < T;
+    const int tk = kv ? key : 0;
+    stage_half_row<HD>(tmem + K_COL + R.lane_off + R.half * (HD / 4),
+                       kn + (int64_t(bh) * T + tk) * HD + R.half * (HD / 2), kv);
+    stage_half_row<HD>(tmem + V_COL + R.lane_off + R.half * (HD / 4),
+                       vh + (int64_t(bh) * T + tk) * HD + R.half * (HD / 2), kv);
+    tc::tmem_wait_st();
+    tc::tc_fence_before();
+    tc::mbar_arrive(&bars->fixed_full);
     bool ok = true;
     for (int j = 0; j < n_steps; ++j) {
       const int sb = j & 1, st = j % kRing;
@@ -920,41 +987,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->ring_full[st], (j / kRing) & 1, abort, kWaitNs));
       if (ok) {
         tc::tc_fence_after();
-        const int qs = (i_begin + j) * kInner + R.half * 32;
-        const float* stat = reinterpret_cast<const float*>(smem + S::STAT_OFF) + st * 2 * kInner + R.half * 32;
-        uint32_t us[32], up[32];
-        tc::tmem_ld_32x32b_x32(tmem + sb * 128 + R.lane_off + R.half * 32, us);
-        tc::tmem_ld_32x32b_x32(tmem + sb * 128 + kInner + R.lane_off + R.half * 32, up);
-        tc::tmem_wait_ld();
-        const bool need_mask = !kv || qs < key || qs + 32 > T;
-        uint8_t* prow = smem + S::P_OFF + sb * S::PT;
-        uint8_t* drow = smem + S::DS_OFF + sb * S::PT;
+        const int qs = k0 + j * kQ + R.half * 16;
+        const float4* stat4 = reinterpret_cast<const float4*>(smem + S::STAT_OFF + (st * 2 * kQ + R.half * 16) * 4);
+        const uint32_t ts = tmem + sb * 64 + R.lane_off + R.half * 16;
+        uint32_t us[16], up[16];
+        tc::tmem_ld_32x32b_x16(ts, us);
+        tc::tmem_ld_32x32b_x16(ts + kQ, up);
+        float l2[16], dd[16];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          uint32_t pp[4], pd[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int i = u * 8 + 2 * e;
-            float p0 = ex2(fmaf(__uint_as_float(us[i]), scale_log2, -stat[i]));
-            float p1 = ex2(fmaf(__uint_as_float(us[i + 1]), scale_log2, -stat[i + 1]));
-            if (need_mask) {
-              if (qs + i < key || qs + i >= T || !kv) p0 = 0.f;
-              if (qs + i + 1 < key || qs + i + 1 >= T || !kv) p1 = 0.f;
-            }
-            pp[e] = pack2(p0, p1);
-            pd[e] = pack2(p0 * (__uint_as_float(up[i]) - stat[kInner + i]),
-                          p1 * (__uint_as_float(up[i + 1]) - stat[kInner + i + 1]));
-          }
-          const uint32_t off = sw_off(R.r, R.half * 4 + u);
-          *reinterpret_cast<uint4*>(prow + off) = make_uint4(pp[0], pp[1], pp[2], pp[3]);
-          *reinterpret_cast<uint4*>(drow + off) = make_uint4(pd[0], pd[1], pd[2], pd[3]);
+        for (int i = 0; i < 4; ++i) {
+          const float4 a = stat4[i], c = stat4[kQ / 4 + i];
+          l2[4 * i] = a.x; l2[4 * i + 1] = a.y; l2[4 * i + 2] = a.z; l2[4 * i + 3] = a.w;
+          dd[4 * i] = c.x; dd[4 * i + 1] = c.y; dd[4 * i + 2] = c.z; dd[4 * i + 3] = c.w;
         }
-        fence_async_smem();
+        tc::tmem_wait_ld();
+        const bool need_mask = !kv || qs < key || qs + 16 > T;
+        uint32_t pp[8], pd[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int i = 2 * e;
+          float p0 = ex2(fmaf(__uint_as_float(us[i]), scale_log2, -l2[i]));
+          float p1 = ex2(fmaf(__uint_as_float(us[i + 1]), scale_log2, -l2[i + 1]));
+          if (need_mask) {
+            if (qs + i < key || qs + i >= T || !kv) p0 = 0.f;
+            if (qs + i + 1 < key || qs + i + 1 >= T || !kv) p1 = 0.f;
+          }
+          pp[e] = pack2(p0, p1);
+          pd[e] = pack2(p0 * (__uint_as_float(up[i]) - dd[i]), p1 * (__uint_as_float(up[i + 1]) - dd[i + 1]));
+        }
+        tc::tmem_st_32x32b_x8(ts, pp);        // P^T over this thread's S^T columns
+        tc::tmem_st_32x32b_x8(ts + kQ, pd);   // dS^T over its dP^T columns
+        tc::tmem_wait_st();
         tc::tc_fence_before();
       }
       tc::mbar_arrive(&bars->ds_ready[sb]);
     }
     if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->acc_full, 0, abort, kWaitNs));
+    if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->epi_full, 0, abort, kWaitNs));
     if (!ok) {
       if (R.lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 32);
       *abort = 1;
@@ -962,7 +1031,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tc_fence_after();
     }
     const int d = H * HD;
-    const int tk = kv ? key : 0;
     __nv_bfloat16* row = dqkv + (int64_t(b) * T + tk) * 3 * d;
     if (ok) {  // dV: this thread's half of the columns
 #pragma unroll
@@ -978,9 +1046,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    norm_rope_bwd_half<HD>(t_dk + R.lane_off, R.half, R.r, scale, kn + (int64_t(bh) * T + tk) * HD,
-                           kv ? rk[int64_t(bh) * T + key] : 0.f, qk_norm, cos_t + tk * (HD / 2),
-                           sin_t + tk * (HD / 2), row + d + h * HD, ok, kv,
+    norm_rope_bwd_half<HD>(t_dk + R.lane_off, R.half, R.r, scale, smem + S::Y_OFF,
+                           kv ? rk[int64_t(bh) * T + key] : 0.f, qk_norm, smem + S::COS_OFF,
+                           smem + S::SIN_OFF, row + d + h * HD, ok, kv,
                            reinterpret_cast<float*>(smem + S::RED_OFF));
   }
   ATTN_EPILOGUE(tmem)
@@ -997,11 +1065,12 @@ int attn_bwd_tc_t(const gpt_config& c, const void* q, const void* k, const void*
   const int64_t N = int64_t(B) * T;
   attn_rowdot_kernel<<<ceil_div(N * H, 8), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(dO), static_cast<const __nv_bfloat16*>(o), Dbuf, N, H, T, HD);
-  CUtensorMap q128, do128, k64, v64, k128, v128, q64, do64;
-  bool ok = tile_map(&q128, q, rows, HD, HD, 128) && tile_map(&do128, dO, ntok, d, d, 128) &&
-            tile_map(&k64, k, rows, HD, HD, 64) && tile_map(&v64, v, rows, HD, HD, 64) &&
-            tile_map(&k128, k, rows, HD, HD, 128) && tile_map(&v128, v, rows, HD, HD, 128) &&
-            tile_map(&q64, q, rows, HD, HD, 64) && tile_map(&do64, dO, ntok, d, d, 64);
+  CUtensorMap k64, v64, q32, do32, yq, yk, mcos, msin;
+  bool ok = tile_map(&k64, k, rows, HD, HD, 64) && tile_map(&v64, v, rows, HD, HD, 64) &&
+            tile_map(&q32, q, rows, HD, HD, 32) && tile_map(&do32, dO, ntok, d, d, 32) &&
+            tile_map(&yq, q, rows, HD, HD, 128) && tile_map(&yk, k, rows, HD, HD, 128) &&
+            tile_map_f32(&mcos, cos_t, T, HD / 2, HD / 2, 128) &&
+            tile_map_f32(&msin, sin_t, T, HD / 2, HD / 2, 128);
   if (!ok) return 1;
   const float scale = 1.f / sqrtf(float(HD));
   const float scale_log2 = scale * kLog2e;
@@ -1010,7 +1079,8 @@ int attn_bwd_tc_t(const gpt_config& c, const void* q, const void* k, const void*
   const int smem_q = int(DqSmem<HD>::BYTES);
   if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_q) != cudaSuccess)
     return 1;
-  kq<<<nt * B * H, kThreads, smem_q, st>>>(q128, do128, k64, v64, static_cast<const __nv_bfloat16*>(q),
+  kq<<<nt * B * H, kThreads, smem_q, st>>>(k64, v64, yq, mcos, msin, static_cast<const __nv_bfloat16*>(q),
+                                           static_cast<const __nv_bfloat16*>(dO),
                                            lse, Dbuf, rq, cos_t, sin_t,
                                            static_cast<__nv_bfloat16*>(dqkv), H, T, scale,
                                            scale_log2, c.qk_norm, status);
@@ -1018,7 +1088,8 @@ int attn_bwd_tc_t(const gpt_config& c, const void* q, const void* k, const void*
   const int smem_k = int(DkvSmem<HD>::BYTES);
   if (cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_k) != cudaSuccess)
     return 1;
-  kk<<<nt * B * H, kThreads, smem_k, st>>>(k128, v128, q64, do64, static_cast<const __nv_bfloat16*>(k),
+  kk<<<nt * B * H, kThreads, smem_k, st>>>(q32, do32, yk, mcos, msin, static_cast<const __nv_bfloat16*>(k),
+                                           static_cast<const __nv_bfloat16*>(v),
                                            lse, Dbuf, rk, cos_t, sin_t,
                                            static_cast<__nv_bfloat16*>(dqkv), H, T, scale,
                                            scale_log2, c.qk_norm, status);

@@ -462,54 +462,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0 && leader) {
+    // the leader's whole warp runs the MMA loop; elect.sync issues
+    if (leader) {
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
-      bool issued_any = false;
-      for (int unit = pair; unit < num_units && !*abort; unit += num_pairs, ++local) {
+      bool issued_any = false, failed = false;
+      for (int unit = pair; unit < num_units; unit += num_pairs, ++local) {
+        if (__any_sync(0xffffffffu, *abort != 0)) break;
         const int sp = unit % splits;
         const int kb_lo = sp * kb_per, kb_hi = min(num_kb, (sp + 1) * kb_per);
         const int acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
-        if (!tc::mbar_wait_bounded(&tail->tmem_empty[acc], acc_phase ^ 1, abort, kWaitLimitNs)) {
-          record_status(g.status, GPT_ETIMEOUT, K_GEMM_TC, 12);
-          *abort = 1;
+        if (!tc::mbar_wait_warp(&tail->tmem_empty[acc], acc_phase ^ 1, abort, kWaitLimitNs)) {
+          if (lane == 0) record_status(g.status, GPT_ETIMEOUT, K_GEMM_TC, 12);
+          failed = true;
           break;
         }
         tc::tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = kb_lo; kb < kb_hi; ++kb) {
-          if (!tc::mbar_wait_bounded(&tail->full[stage], phase, abort, kWaitLimitNs)) {
-            record_status(g.status, GPT_ETIMEOUT, K_GEMM_TC, 13);
-            *abort = 1;
+          if (!tc::mbar_wait_warp(&tail->full[stage], phase, abort, kWaitLimitNs)) {
+            if (lane == 0) record_status(g.status, GPT_ETIMEOUT, K_GEMM_TC, 13);
+            failed = true;
             break;
           }
           tc::tc_fence_after();
-          const uint32_t a_addr = tc::smem_u32(smA + stage * P_HALF);
-          const uint32_t b_addr = tc::smem_u32(smB + stage * P_HALF);
+          const uint64_t da0 = tc::smem_desc_sw128(tc::smem_u32(smA + stage * P_HALF), AMN ? 8192 : 16);
+          const uint64_t db0 = tc::smem_desc_sw128(tc::smem_u32(smB + stage * P_HALF), BMN ? 8192 : 16);
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            const uint64_t da = AMN ? tc::smem_desc_sw128(a_addr + k * 2048, 8192)
-                                    : tc::smem_desc_sw128(a_addr + k * 32, 16);
-            const uint64_t db = BMN ? tc::smem_desc_sw128(b_addr + k * 2048, 8192)
-                                    : tc::smem_desc_sw128(b_addr + k * 32, 16);
-            tc::mma_bf16_ss_pair(d_tmem, da, db, idesc, (kb != kb_lo) || k != 0);
-          }
+          for (int k = 0; k < BK / 16; ++k)
+            tc::mma_bf16_ss_pair_elect(d_tmem, tc::desc_advance(da0, AMN ? k * 2048 : k * 32),
+                                       tc::desc_advance(db0, BMN ? k * 2048 : k * 32), idesc,
+                                       (kb != kb_lo) || k != 0);
           issued_any = true;
           const uint32_t e = tc::smem_u32(&tail->empty[stage]);
-          tc::mma_commit_pair(e);
-          tc::mma_commit_pair(tc::mapa_shared(e, 1));
+          tc::mma_commit_pair_elect(e);
+          tc::mma_commit_pair_elect(tc::mapa_shared(e, 1));
           if (++stage == P_STAGES) { stage = 0; phase ^= 1; }
         }
-        if (*abort) break;
+        if (failed) break;
         const uint32_t f = tc::smem_u32(&tail->tmem_full[acc]);
-        tc::mma_commit_pair(f);
-        tc::mma_commit_pair(tc::mapa_shared(f, 1));
+        tc::mma_commit_pair_elect(f);
+        tc::mma_commit_pair_elect(tc::mapa_shared(f, 1));
       }
+      if (failed && lane == 0) *abort = 1;
       if (issued_any) {
-        tc::mma_commit_pair(tc::smem_u32(&tail->mma_done));
-        tc::mbar_wait_bounded(&tail->mma_done, 0, nullptr, kWaitLimitNs);
+        tc::mma_commit_pair_elect(tc::smem_u32(&tail->mma_done));
+        tc::mbar_wait_warp(&tail->mma_done, 0, nullptr, kWaitLimitNs);
       }
     }
   } else {
