@@ -5,9 +5,11 @@
 // log-sum-exp of each query row's scaled scores s_ij = q_i . k_j / sqrt(hd)
 // over keys j <= i.
 //
-// Every kernel: warp 0 loads tiles with TMA (128-byte swizzle), one thread of
-// warp 1 issues tcgen05.mma into tensor memory, warps 2..9 (256 threads, two
-// per accumulator row: each TMEM lane quarter is read by two warps) do the
+// Every kernel: warp 0 loads tiles with TMA (128-byte swizzle), warps 1 and 10
+// issue tcgen05.mma into tensor memory (two independent MMA chains: one warp
+// issues an MMA only every ~90 cycles, slower than the tensor pipe runs the
+// small-N products of attention), warps 2..9 (256 threads, two per
+// accumulator row: each TMEM lane quarter is read by two warps) do the
 // element-wise work.  All mbarrier waits are bounded (GPT_ETIMEOUT in the
 // status word); the compute warps reach their named barriers the same number
 // of times on every path, so an expired wait cannot strand them.
@@ -20,7 +22,7 @@ namespace gpt {
 
 namespace {
 constexpr int BQ = 128, BKV = 128, kInner = 64;
-constexpr int kThreads = 320;   // warp 0 TMA, warp 1 MMA, warps 2..9 compute
+constexpr int kThreads = 352;   // warp 0 TMA, warps 1 and 10 MMA, warps 2..9 compute
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -163,9 +165,9 @@ struct FwdBars {
   uint64_t q_full;
   uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
   uint64_t s_full[2];
-  uint64_t p_ready;
+  uint64_t p_ready[2];  // per S buffer: the S and PV warps wait on it out of step
   uint64_t pv_full;
-  uint64_t done;
+  uint64_t done, done2;
   uint32_t tmem_base;
   int abort;
 };
@@ -202,9 +204,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_init(&bars->v_full[s], 1); tc::mbar_init(&bars->v_empty[s], 1);
       tc::mbar_init(&bars->s_full[s], 1);
     }
-    tc::mbar_init(&bars->p_ready, 256);
+    tc::mbar_init(&bars->p_ready[0], 256);
+    tc::mbar_init(&bars->p_ready[1], 256);
     tc::mbar_init(&bars->pv_full, 1);
     tc::mbar_init(&bars->done, 1);
+    tc::mbar_init(&bars->done2, 1);
   })
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort = &bars->abort;
@@ -247,51 +251,60 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    {  // the whole warp runs the MMA loop; elect.sync issues
-      constexpr uint32_t idesc_s = tc::idesc_bf16_f32(BQ, BKV, false, false);
-      constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(BQ, HD, false, true);
-      const uint32_t q_addr = tc::smem_u32(smem + S::Q_OFF);
-      const uint32_t p_addr = tc::smem_u32(smem + S::P_OFF);
-      bool ok = tc::mbar_wait_warp(&bars->q_full, 0, abort, kWaitNs);
-      bool issued_any = false;
-      auto issue_pv = [&](int j) -> bool {
-        if (!tc::mbar_wait_warp(&bars->p_ready, j & 1, abort, kWaitNs)) return false;
-        if (!tc::mbar_wait_warp(&bars->v_full[j & 1], (j >> 1) & 1, abort, kWaitNs)) return false;
-        tc::tc_fence_after();
-        const uint32_t v_addr = tc::smem_u32(smem + S::V_OFF + (j & 1) * S::TILE);
+    // S_j = Q K_j^T.  S_j reuses the TMEM buffer of S_{j-2}: the compute
+    // threads must have turned S_{j-2} into P_{j-2} first.
+    constexpr uint32_t idesc_s = tc::idesc_bf16_f32(BQ, BKV, false, false);
+    const uint64_t qd = tc::smem_desc_sw128(tc::smem_u32(smem + S::Q_OFF), 16);
+    bool ok = tc::mbar_wait_warp(&bars->q_full, 0, abort, kWaitNs);
+    bool issued_any = false;
+    for (int j = 0; ok && j < n_kv; ++j) {
+      const int st = j & 1;
+      if (j >= 2 && !tc::mbar_wait_warp(&bars->p_ready[st], ((j - 2) >> 1) & 1, abort, kWaitNs)) { ok = false; break; }
+      if (!tc::mbar_wait_warp(&bars->k_full[st], (j >> 1) & 1, abort, kWaitNs)) { ok = false; break; }
+      tc::tc_fence_after();
+      const uint64_t kd = tc::smem_desc_sw128(tc::smem_u32(smem + S::K_OFF + st * S::TILE), 16);
 #pragma unroll
-        for (int k = 0; k < BKV / 16; ++k)
-          tc::mma_bf16_ss_elect(t_o, tc::smem_desc_sw128(p_addr + (k >> 2) * CH + (k & 3) * 32, 16),
-                          tc::smem_desc_sw128(v_addr + k * 2048, CH), idesc_pv, (j | k) != 0);
-        tc::mma_commit_elect(&bars->pv_full);
-        tc::mma_commit_elect(&bars->v_empty[j & 1]);
-        return true;
-      };
-      for (int j = 0; ok && j < n_kv; ++j) {
-        const int st = j & 1;
-        if (!tc::mbar_wait_warp(&bars->k_full[st], (j >> 1) & 1, abort, kWaitNs)) { ok = false; break; }
-        tc::tc_fence_after();
-        const uint32_t k_addr = tc::smem_u32(smem + S::K_OFF + st * S::TILE);
+      for (int k = 0; k < HD / 16; ++k) {
+        const uint32_t off = (k >> 2) * CH + (k & 3) * 32;
+        tc::mma_bf16_ss_elect(tmem + st * 128, tc::desc_advance(qd, off), tc::desc_advance(kd, off), idesc_s, k != 0);
+      }
+      issued_any = true;
+      tc::mma_commit_elect(&bars->s_full[st]);
+      tc::mma_commit_elect(&bars->k_empty[st]);
+    }
+    if (!ok) {
+      if (lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 11);
+      *abort = 1;
+    }
+    if (issued_any) {
+      tc::mma_commit_elect(&bars->done);
+      tc::mbar_wait_warp(&bars->done, 0, nullptr, kWaitNs);
+    }
+  } else if (warp == 10) {
+    // O += P_j V_j once the compute threads have written P_j
+    constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(BQ, HD, false, true);
+    const uint64_t pd = tc::smem_desc_sw128(tc::smem_u32(smem + S::P_OFF), 16);
+    bool ok = true, issued_any = false;
+    for (int j = 0; ok && j < n_kv; ++j) {
+      if (!tc::mbar_wait_warp(&bars->p_ready[j & 1], (j >> 1) & 1, abort, kWaitNs)) { ok = false; break; }
+      if (!tc::mbar_wait_warp(&bars->v_full[j & 1], (j >> 1) & 1, abort, kWaitNs)) { ok = false; break; }
+      tc::tc_fence_after();
+      const uint64_t vd = tc::smem_desc_sw128(tc::smem_u32(smem + S::V_OFF + (j & 1) * S::TILE), CH);
 #pragma unroll
-        for (int k = 0; k < HD / 16; ++k) {
-          const uint32_t off = (k >> 2) * CH + (k & 3) * 32;
-          tc::mma_bf16_ss_elect(tmem + st * 128, tc::smem_desc_sw128(q_addr + off, 16),
-                          tc::smem_desc_sw128(k_addr + off, 16), idesc_s, k != 0);
-        }
-        issued_any = true;
-        tc::mma_commit_elect(&bars->s_full[st]);
-        tc::mma_commit_elect(&bars->k_empty[st]);
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
-      }
-      if (ok && n_kv >= 1) ok = issue_pv(n_kv - 1);
-      if (!ok) {
-        if (lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 11);
-        *abort = 1;
-      }
-      if (issued_any) {
-        tc::mma_commit_elect(&bars->done);
-        tc::mbar_wait_warp(&bars->done, 0, nullptr, kWaitNs);
-      }
+      for (int k = 0; k < BKV / 16; ++k)
+        tc::mma_bf16_ss_elect(t_o, tc::desc_advance(pd, (k >> 2) * CH + (k & 3) * 32), tc::desc_advance(vd, k * 2048),
+                              idesc_pv, (j | k) != 0);
+      issued_any = true;
+      tc::mma_commit_elect(&bars->pv_full);
+      tc::mma_commit_elect(&bars->v_empty[j & 1]);
+    }
+    if (!ok) {
+      if (lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 13);
+      *abort = 1;
+    }
+    if (issued_any) {
+      tc::mma_commit_elect(&bars->done2);
+      tc::mbar_wait_warp(&bars->done2, 0, nullptr, kWaitNs);
     }
   } else {
     const Roles R = roles();
@@ -327,14 +340,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       red[(st * 2 + R.half) * BQ + R.r] = mx;
       compute_bar();
       const float mx_all = fmaxf(red[(st * 2) * BQ + R.r], red[(st * 2 + 1) * BQ + R.r]) * scale_log2;
-      if (ok && j > 0) {
-        ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->pv_full, (j - 1) & 1, abort, kWaitNs));
-        if (ok) tc::tc_fence_after();
-      }
       if (ok) {
         const bool grow = mx_all > m_ref + 8.f;
         const float factor = grow ? ex2(m_ref - mx_all) : 1.f;
-        if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        if (grow) {
+          l_half *= factor;
+          m_ref = mx_all;
+        }
+        // P_j into registers first: this overlaps P_{j-1} V_{j-1}, which must
+        // finish before O is rescaled and before the P tile is rewritten
+        float lsum = 0.f;
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float p0 = ex2(fmaf(s[2 * i], scale_log2, -m_ref));
+          const float p1 = ex2(fmaf(s[2 * i + 1], scale_log2, -m_ref));
+          lsum += p0 + p1;
+          pk[i] = pack2(p0, p1);
+        }
+        l_half += lsum;
+        if (j > 0) {
+          ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->pv_full, (j - 1) & 1, abort, kWaitNs));
+          if (ok) tc::tc_fence_after();
+        }
+        if (ok) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<uint4*>(p_chunk + sw_off(R.r, u)) =
+                make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        }
+        if (ok && j > 0 && __any_sync(0xffffffffu, grow)) {
 #pragma unroll
           for (int c = 0; c < HD / 2; c += 16) {
             uint32_t u[16];
@@ -347,28 +382,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc::tmem_wait_st();
         }
-        if (grow) {
-          l_half *= factor;
-          m_ref = mx_all;
+        if (ok) {
+          fence_async_smem();
+          tc::tc_fence_before();
         }
-        float lsum = 0.f;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          uint32_t pk[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float p0 = ex2(fmaf(s[u * 8 + 2 * e], scale_log2, -m_ref));
-            const float p1 = ex2(fmaf(s[u * 8 + 2 * e + 1], scale_log2, -m_ref));
-            lsum += p0 + p1;
-            pk[e] = pack2(p0, p1);
-          }
-          *reinterpret_cast<uint4*>(p_chunk + sw_off(R.r, u)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        }
-        l_half += lsum;
-        fence_async_smem();
-        tc::tc_fence_before();
       }
-      tc::mbar_arrive(&bars->p_ready);
+      tc::mbar_arrive(&bars->p_ready[st]);
     }
     if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->pv_full, (n_kv - 1) & 1, abort, kWaitNs));
     sums[R.half * BQ + R.r] = l_half;
@@ -464,20 +483,20 @@ __global__ void attn_rowdot_kernel(const __nv_bfloat16* __restrict__ dO,
   }
 }
 
-constexpr int kRing = 6;    // slots of the Q/dO ring of the dK/dV kernel
-constexpr int kRingQ = 4;   // slots of the K/V ring of the dQ kernel
-constexpr int kQ = 32;      // queries per step of the dK/dV kernel
-constexpr int kRingMax = kRing > kRingQ ? kRing : kRingQ;
+constexpr int kRingKV = 3;  // slots of the Q/dO ring of the dK/dV kernel
+constexpr int kRingQ = 3;   // slots of the K/V ring of the dQ kernel
+constexpr int kRingMax = kRingKV > kRingQ ? kRingKV : kRingQ;
 
 struct BwdBars {
   uint64_t fixed_full;
   uint64_t ring_full[kRingMax];
   uint64_t ring_empty[kRingMax];
   uint64_t s_full[2];
+  uint64_t dp_full[2];
   uint64_t ds_ready[2];
   uint64_t acc_full;
   uint64_t epi_full;
-  uint64_t done;
+  uint64_t done, done2;
   uint32_t tmem_base;
   int abort;
 };
@@ -562,18 +581,18 @@ __device__ __forceinline__ void norm_rope_bwd_half(uint32_t taddr, int half, int
 }
 
 // The epilogue's inputs for 128 rows, loaded by TMA onto `bar`: the y rows
-// (bh*T + row0 ..) of a head-major [B*H*T, HD] tensor and the cos / sin table
-// rows (pos0 ..) of [T, HD/2] fp32.
+// (bh*T + row0 ..) of a head-major [B*H*T, HD] tensor (unless y_dst is null)
+// and the cos / sin table rows (pos0 ..) of [T, HD/2] fp32.
 template <int HD>
 __device__ __forceinline__ void load_epilogue_tiles(uint8_t* y_dst, uint8_t* cos_dst, uint8_t* sin_dst,
                                                     const CUtensorMap* map_y, const CUtensorMap* map_cos,
                                                     const CUtensorMap* map_sin, uint64_t* bar,
                                                     int y_row0, int pos0) {
   constexpr int NCH = HD / 64;
-  tc::mbar_arrive_expect_tx(bar, 3u * 128 * HD * 2);
+  tc::mbar_arrive_expect_tx(bar, (y_dst ? 3u : 2u) * 128 * HD * 2);
 #pragma unroll
   for (int c = 0; c < NCH; ++c) {
-    tc::tma_load_2d(y_dst + c * (128 * 128), map_y, bar, c * 64, y_row0);
+    if (y_dst) tc::tma_load_2d(y_dst + c * (128 * 128), map_y, bar, c * 64, y_row0);
     tc::tma_load_2d(cos_dst + c * (128 * 128), map_cos, bar, c * 32, pos0);
     tc::tma_load_2d(sin_dst + c * (128 * 128), map_sin, bar, c * 32, pos0);
   }
@@ -582,11 +601,12 @@ __device__ __forceinline__ void load_epilogue_tiles(uint8_t* y_dst, uint8_t* cos
 template <int HD>
 struct DqSmem {
   static constexpr uint32_t SMALL = kInner * HD * 2;
-  static constexpr uint32_t EPI = 128 * HD * 2;  // one epilogue tile (y, cos or sin)
-  static constexpr uint32_t K_OFF = 0;
+  static constexpr uint32_t EPI = 128 * HD * 2;  // the Q or dO tile; also a cos / sin tile
+  static constexpr uint32_t Q_OFF = 0, DO_OFF = EPI;
+  static constexpr uint32_t K_OFF = 2 * EPI;
   static constexpr uint32_t V_OFF = K_OFF + kRingQ * SMALL;
-  static constexpr uint32_t Y_OFF = V_OFF + kRingQ * SMALL;
-  static constexpr uint32_t COS_OFF = Y_OFF + EPI, SIN_OFF = COS_OFF + EPI;
+  static constexpr uint32_t Y_OFF = Q_OFF;  // the Q tile is the y of the norm backward
+  static constexpr uint32_t COS_OFF = V_OFF + kRingQ * SMALL, SIN_OFF = COS_OFF + EPI;
   static constexpr uint32_t RED_OFF = SIN_OFF + EPI;
   static constexpr uint32_t BAR_OFF = RED_OFF + 2 * 128 * 4;
   static constexpr uint32_t BYTES = BAR_OFF + 256 + 1024;
@@ -594,43 +614,25 @@ struct DqSmem {
   static_assert(BYTES <= 232448, "");
 };
 
-// Half a bf16 row (HD/2 elements from `src`, zeros when !valid) into TMEM
-// columns taddr .. taddr + HD/4 of this thread's lane: the K-major layout of
-// an MMA A operand, two elements per column.
-template <int HD>
-__device__ __forceinline__ void stage_half_row(uint32_t taddr, const __nv_bfloat16* __restrict__ src,
-                                               bool valid) {
-  constexpr int W = HD / 4;
-  uint32_t w[W];
-#pragma unroll
-  for (int i = 0; i < W / 4; ++i) {
-    const uint4 u = valid ? reinterpret_cast<const uint4*>(src)[i] : make_uint4(0u, 0u, 0u, 0u);
-    w[4 * i] = u.x; w[4 * i + 1] = u.y; w[4 * i + 2] = u.z; w[4 * i + 3] = u.w;
-  }
-  if constexpr (W == 32) tc::tmem_st_32x32b_x32(taddr, w);
-  else tc::tmem_st_32x32b_x16(taddr, w);
-}
-
 }  // namespace
 
-// dQ for 128 queries of one (batch, head), looping over 64-key tiles.  Q and dO
-// (fixed for the CTA) sit in TMEM as the A operands of S = Q K^T and
-// dP = dO V^T, so each MMA reads only its K or V slice from shared memory.
+// dQ for 128 queries of one (batch, head), looping over 64-key tiles.  Warp 1
+// issues S_j = Q K_j^T and dQ += dS_{j-1} K_{j-1}; warp 10 issues dP_j = dO V_j^T.
 // Compute thread (row, half) handles keys [32*half, 32*half + 32) of each tile
-// and writes its bf16 dS over its own S columns, the TMEM A operand of
-// dQ += dS K.  TMEM: S/dP pairs at columns 0 and 128 (64 + 64 each), dQ at
-// 256, Q at 384, dO at 448.
+// and writes its bf16 dS over its own S columns: the TMEM A operand of the dQ
+// product, which warp 1 issues before it next overwrites those columns.  TMEM:
+// S/dP pairs at columns 0 and 128 (64 + 64 each), dQ at 256.  The Q tile in
+// shared memory doubles as the y of the norm backward.
 template <int HD>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_dq_tc_kernel(const __grid_constant__ CUtensorMap map_k64,
+    attn_dq_tc_kernel(const __grid_constant__ CUtensorMap map_q128,
+                      const __grid_constant__ CUtensorMap map_do128,
+                      const __grid_constant__ CUtensorMap map_k64,
                       const __grid_constant__ CUtensorMap map_v64,
-                      const __grid_constant__ CUtensorMap map_y,
                       const __grid_constant__ CUtensorMap map_cos,
                       const __grid_constant__ CUtensorMap map_sin,
-                      const __nv_bfloat16* __restrict__ qn, const __nv_bfloat16* __restrict__ dO,
                       const float* __restrict__ lse,
                       const float* __restrict__ D, const float* __restrict__ rq,
-                      const float* __restrict__ cos_t, const float* __restrict__ sin_t,
                       __nv_bfloat16* __restrict__ dqkv, int H, int T, float scale,
                       float scale_log2, int qk_norm, int32_t* status) {
   using S = DqSmem<HD>;
@@ -646,21 +648,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int q0 = qt * 128;
   const int n_steps = (min(q0 + 128, T) + kInner - 1) / kInner;
   constexpr int NCH = HD / 64;
-  constexpr uint32_t Q_COL = 384, DO_COL = 448;
 
   ATTN_PROLOGUE(bars, {
-    tc::mbar_init(&bars->fixed_full, 256);  // the compute threads' Q / dO stores
+    tc::mbar_init(&bars->fixed_full, 1);
     tc::mbar_init(&bars->epi_full, 1);
     for (int s = 0; s < kRingQ; ++s) {
       tc::mbar_init(&bars->ring_full[s], 1);
-      tc::mbar_init(&bars->ring_empty[s], 1);
+      tc::mbar_init(&bars->ring_empty[s], 2);  // after S and dQ (warp 1) and dP (warp 10)
     }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&bars->s_full[s], 1);
+      tc::mbar_init(&bars->dp_full[s], 1);
       tc::mbar_init(&bars->ds_ready[s], 256);
     }
     tc::mbar_init(&bars->acc_full, 1);
     tc::mbar_init(&bars->done, 1);
+    tc::mbar_init(&bars->done2, 1);
   })
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort = &bars->abort;
@@ -669,6 +672,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       uint32_t issued = 0, last_par = 0;
+      tc::mbar_arrive_expect_tx(&bars->fixed_full, 2 * S::EPI);
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) {
+        tc::tma_load_2d(smem + S::Q_OFF + c * (128 * 128), &map_q128, &bars->fixed_full, c * 64, bh * T + q0);
+        tc::tma_load_2d(smem + S::DO_OFF + c * (128 * 128), &map_do128, &bars->fixed_full,
+                        h * HD + c * 64, b * T + q0);
+      }
       for (int j = 0; j < n_steps; ++j) {
         const int st = j % kRingQ;
         const uint32_t ph = (j / kRingQ) & 1;
@@ -686,83 +696,105 @@ __global__ void __launch_bounds__(kThreads, 1)
                           &bars->ring_full[st], c * 64, bh * T + j * kInner);
         }
         if (j == 0)
-          load_epilogue_tiles<HD>(smem + S::Y_OFF, smem + S::COS_OFF, smem + S::SIN_OFF, &map_y,
-                                  &map_cos, &map_sin, &bars->epi_full, bh * T + q0, q0);
+          load_epilogue_tiles<HD>(nullptr, smem + S::COS_OFF, smem + S::SIN_OFF, nullptr, &map_cos,
+                                  &map_sin, &bars->epi_full, 0, q0);
         issued |= 1u << st;
         last_par = (last_par & ~(1u << st)) | (ph << st);
       }
       if (*abort) {
+        tc::mbar_wait_bounded(&bars->fixed_full, 0, nullptr, kWaitNs);
         if (issued) tc::mbar_wait_bounded(&bars->epi_full, 0, nullptr, kWaitNs);
         for (int s = 0; s < kRingQ; ++s)
           if (issued >> s & 1) tc::mbar_wait_bounded(&bars->ring_full[s], (last_par >> s) & 1, nullptr, kWaitNs);
       }
     }
   } else if (warp == 1) {
-    {  // the whole warp runs the MMA loop; elect.sync issues
-      constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, kInner, false, false);
-      constexpr uint32_t idesc_dq = tc::idesc_bf16_f32(128, HD, false, true);
-      bool ok = tc::mbar_wait_warp(&bars->fixed_full, 0, abort, kWaitNs);
+    // S_j = Q K_j^T, then dQ += dS_{j-1} K_{j-1}.  S_j overwrites the dS_{j-2}
+    // that this warp's own dQ MMAs read (issued earlier: in order).
+    constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, kInner, false, false);
+    constexpr uint32_t idesc_dq = tc::idesc_bf16_f32(128, HD, false, true);
+    const uint64_t qd = tc::smem_desc_sw128(tc::smem_u32(smem + S::Q_OFF), 16);
+    bool ok = tc::mbar_wait_warp(&bars->fixed_full, 0, abort, kWaitNs);
+    bool issued_any = false;
+    auto issue_dq = [&](int j) -> bool {
+      if (!tc::mbar_wait_warp(&bars->ds_ready[j & 1], (j >> 1) & 1, abort, kWaitNs)) return false;
       tc::tc_fence_after();
-      bool issued_any = false;
-      auto issue_dq = [&](int j) -> bool {
-        if (!tc::mbar_wait_warp(&bars->ds_ready[j & 1], (j >> 1) & 1, abort, kWaitNs)) return false;
-        tc::tc_fence_after();
-        const uint32_t ds_t = tmem + (j & 1) * 128;
-        const uint64_t kb = tc::smem_desc_sw128(tc::smem_u32(smem + S::K_OFF + (j % kRingQ) * S::SMALL),
-                                                kInner * 128);
+      const uint32_t ds_t = tmem + (j & 1) * 128;
+      const uint64_t kb = tc::smem_desc_sw128(tc::smem_u32(smem + S::K_OFF + (j % kRingQ) * S::SMALL),
+                                              kInner * 128);
 #pragma unroll
-        for (int k = 0; k < kInner / 16; ++k)
-          tc::mma_bf16_ts_elect(t_dq, ds_t + 32 * (k >> 1) + 8 * (k & 1), tc::desc_advance(kb, k * 2048),
-                          idesc_dq, (j | k) != 0);
-        tc::mma_commit_elect(&bars->ring_empty[j % kRingQ]);
-        return true;
-      };
-      for (int j = 0; ok && j < n_steps; ++j) {
-        const int st = j % kRingQ;
-        if (!tc::mbar_wait_warp(&bars->ring_full[st], (j / kRingQ) & 1, abort, kWaitNs)) { ok = false; break; }
-        tc::tc_fence_after();
-        const uint64_t kd = tc::smem_desc_sw128(tc::smem_u32(smem + S::K_OFF + st * S::SMALL), 16);
-        const uint64_t vd = tc::smem_desc_sw128(tc::smem_u32(smem + S::V_OFF + st * S::SMALL), 16);
-        const uint32_t pair = tmem + (j & 1) * 128;
+      for (int k = 0; k < kInner / 16; ++k)
+        tc::mma_bf16_ts_elect(t_dq, ds_t + 32 * (k >> 1) + 8 * (k & 1), tc::desc_advance(kb, k * 2048),
+                              idesc_dq, (j | k) != 0);
+      tc::mma_commit_elect(&bars->ring_empty[j % kRingQ]);
+      return true;
+    };
+    for (int j = 0; ok && j < n_steps; ++j) {
+      const int st = j % kRingQ;
+      if (!tc::mbar_wait_warp(&bars->ring_full[st], (j / kRingQ) & 1, abort, kWaitNs)) { ok = false; break; }
+      tc::tc_fence_after();
+      const uint64_t kd = tc::smem_desc_sw128(tc::smem_u32(smem + S::K_OFF + st * S::SMALL), 16);
+      const uint32_t pair = tmem + (j & 1) * 128;
 #pragma unroll
-        for (int k = 0; k < HD / 16; ++k) {
-          const uint32_t small = (k >> 2) * (kInner * 128) + (k & 3) * 32;
-          tc::mma_bf16_ts_elect(pair, tmem + Q_COL + 8 * k, tc::desc_advance(kd, small), idesc_s, k != 0);
-          tc::mma_bf16_ts_elect(pair + kInner, tmem + DO_COL + 8 * k, tc::desc_advance(vd, small), idesc_s, k != 0);
-        }
-        issued_any = true;
-        tc::mma_commit_elect(&bars->s_full[j & 1]);
-        if (j >= 1 && !issue_dq(j - 1)) { ok = false; break; }
-      }
-      if (ok && n_steps >= 1) ok = issue_dq(n_steps - 1);
-      if (ok) tc::mma_commit_elect(&bars->acc_full);
-      if (!ok) {
-        if (lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 21);
-        *abort = 1;
-      }
-      if (issued_any) {
-        tc::mma_commit_elect(&bars->done);
-        tc::mbar_wait_warp(&bars->done, 0, nullptr, kWaitNs);
-      }
+      for (int k = 0; k < HD / 16; ++k)
+        tc::mma_bf16_ss_elect(pair, tc::desc_advance(qd, (k >> 2) * (128 * 128) + (k & 3) * 32),
+                              tc::desc_advance(kd, (k >> 2) * (kInner * 128) + (k & 3) * 32), idesc_s, k != 0);
+      issued_any = true;
+      tc::mma_commit_elect(&bars->s_full[j & 1]);
+      if (j >= 1 && !issue_dq(j - 1)) { ok = false; break; }
+    }
+    if (ok && n_steps >= 1) ok = issue_dq(n_steps - 1);
+    if (ok) tc::mma_commit_elect(&bars->acc_full);
+    if (!ok) {
+      if (lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 21);
+      *abort = 1;
+    }
+    if (issued_any) {
+      tc::mma_commit_elect(&bars->done);
+      tc::mbar_wait_warp(&bars->done, 0, nullptr, kWaitNs);
+    }
+  } else if (warp == 10) {
+    // dP_j = dO V_j^T into the dP half of the pair, once the compute threads
+    // are done with dP_{j-2}
+    constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, kInner, false, false);
+    const uint64_t dod = tc::smem_desc_sw128(tc::smem_u32(smem + S::DO_OFF), 16);
+    bool ok = tc::mbar_wait_warp(&bars->fixed_full, 0, abort, kWaitNs);
+    bool issued_any = false;
+    for (int j = 0; ok && j < n_steps; ++j) {
+      const int st = j % kRingQ;
+      if (j >= 2 && !tc::mbar_wait_warp(&bars->ds_ready[j & 1], ((j - 2) >> 1) & 1, abort, kWaitNs)) { ok = false; break; }
+      if (!tc::mbar_wait_warp(&bars->ring_full[st], (j / kRingQ) & 1, abort, kWaitNs)) { ok = false; break; }
+      tc::tc_fence_after();
+      const uint64_t vd = tc::smem_desc_sw128(tc::smem_u32(smem + S::V_OFF + st * S::SMALL), 16);
+      const uint32_t pair = tmem + (j & 1) * 128;
+#pragma unroll
+      for (int k = 0; k < HD / 16; ++k)
+        tc::mma_bf16_ss_elect(pair + kInner, tc::desc_advance(dod, (k >> 2) * (128 * 128) + (k & 3) * 32),
+                              tc::desc_advance(vd, (k >> 2) * (kInner * 128) + (k & 3) * 32), idesc_s, k != 0);
+      issued_any = true;
+      tc::mma_commit_elect(&bars->dp_full[j & 1]);
+      tc::mma_commit_elect(&bars->ring_empty[st]);
+    }
+    if (!ok) {
+      if (lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 23);
+      *abort = 1;
+    }
+    if (issued_any) {
+      tc::mma_commit_elect(&bars->done2);
+      tc::mbar_wait_warp(&bars->done2, 0, nullptr, kWaitNs);
     }
   } else {
     const Roles R = roles();
     const int q = q0 + R.r;
     const bool qv = q < T;
     const int tq = qv ? q : 0;
-    stage_half_row<HD>(tmem + Q_COL + R.lane_off + R.half * (HD / 4),
-                       qn + (int64_t(bh) * T + tq) * HD + R.half * (HD / 2), qv);
-    stage_half_row<HD>(tmem + DO_COL + R.lane_off + R.half * (HD / 4),
-                       dO + (int64_t(b) * T + tq) * (int64_t(H) * HD) + h * HD + R.half * (HD / 2), qv);
-    tc::tmem_wait_st();
-    tc::tc_fence_before();
-    tc::mbar_arrive(&bars->fixed_full);
     const float lse2 = qv ? lse[int64_t(bh) * T + q] * kLog2e : 0.f;
     const float Dq = qv ? D[int64_t(bh) * T + q] : 0.f;
     bool ok = true;
     for (int j = 0; j < n_steps; ++j) {
       const int sb = j & 1;
       if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->s_full[sb], (j >> 1) & 1, abort, kWaitNs));
+      if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->dp_full[sb], (j >> 1) & 1, abort, kWaitNs));
       if (ok) {
         tc::tc_fence_after();
         const int k0 = j * kInner + R.half * 32;
@@ -810,40 +842,43 @@ __global__ void __launch_bounds__(kThreads, 1)
 namespace {
 template <int HD>
 struct DkvSmem {
-  static constexpr uint32_t SMALL = kQ * HD * 2;
-  static constexpr uint32_t Q_OFF = 0;
-  static constexpr uint32_t EPI = 128 * HD * 2;  // one epilogue tile (y, cos or sin)
-  static constexpr uint32_t DO_OFF = Q_OFF + kRing * SMALL;
-  static constexpr uint32_t Y_OFF = DO_OFF + kRing * SMALL;
-  static constexpr uint32_t COS_OFF = Y_OFF + EPI, SIN_OFF = COS_OFF + EPI;
-  static constexpr uint32_t STAT_OFF = SIN_OFF + EPI;  // [ring][lse2 x kQ | D x kQ]
-  static constexpr uint32_t RED_OFF = STAT_OFF + kRing * 2 * kQ * 4;
-  static constexpr uint32_t BAR_OFF = RED_OFF + 2 * 128 * 4;
-  static_assert(Q_OFF % 1024 == 0 && DO_OFF % 1024 == 0 && SMALL % 1024 == 0 && Y_OFF % 1024 == 0 &&
-                EPI % 1024 == 0, "");
+  static constexpr uint32_t BIG = 128 * HD * 2;    // the K or V tile; also a cos / sin tile
+  static constexpr uint32_t SMALL = kInner * HD * 2;
+  static constexpr uint32_t K_OFF = 0, V_OFF = BIG;
+  static constexpr uint32_t Q_OFF = 2 * BIG;
+  static constexpr uint32_t DO_OFF = Q_OFF + kRingKV * SMALL;
+  static constexpr uint32_t COS_OFF = DO_OFF + kRingKV * SMALL, SIN_OFF = COS_OFF + BIG;
+  static constexpr uint32_t STAT_OFF = SIN_OFF + BIG;  // [ring][lse2 x 64 | D x 64]
+  static constexpr uint32_t RED_OFF = STAT_OFF;        // epilogue only, after the last step's stats
+  static constexpr uint32_t BAR_OFF = STAT_OFF + kRingKV * 2 * kInner * 4;
+  static_assert(V_OFF % 1024 == 0 && Q_OFF % 1024 == 0 && DO_OFF % 1024 == 0 && COS_OFF % 1024 == 0 &&
+                SMALL % 1024 == 0, "");
+  static_assert(kRingKV * 2 * kInner * 4 >= 2 * 128 * 4, "");
   static constexpr uint32_t BYTES = BAR_OFF + 256 + 1024;
+  static_assert(BYTES <= 232448, "");
 };
 }  // namespace
 
-// dK, dV for 128 keys of one (batch, head), looping over 32-query tiles.  K and
-// V (fixed for the CTA) sit in TMEM as the A operands of S^T = K Q^T and
-// dP^T = V dO^T.  Compute thread (key row, half) handles queries
-// [16*half, 16*half + 16) of each tile and writes bf16 P^T and dS^T over its own
-// S^T and dP^T columns: the TMEM A operands of dV += P^T dO and dK += dS^T Q.
-// The producer warp stages lse and D of the tile's queries in shared memory
-// next to the Q / dO tiles.  TMEM: S^T/dP^T pairs at columns 0 and 64 (32 + 32
-// each), dV at 128, dK at 256, K at 384, V at 448.
+// dK, dV for 128 keys of one (batch, head), looping over 64-query tiles.
+// Warp 1 issues S^T_j = K Q_j^T and dV += P^T_{j-1} dO_{j-1}; warp 10 issues
+// dP^T_j = V dO_j^T and dK += dS^T_{j-1} Q_{j-1}.  Compute thread (key row,
+// half) handles queries [32*half, 32*half + 32) of each tile and writes bf16
+// P^T over its S^T columns and dS^T over its dP^T columns: the TMEM A operands
+// of the dV and dK products, each read by the warp that next overwrites those
+// columns (so in issue order).  The producer warp stages lse and D of the
+// tile's queries in shared memory next to the Q / dO tiles.  TMEM: S^T/dP^T
+// pairs at columns 0 and 128 (64 + 64 each), dV at 256, dK at 384.  The K tile
+// in shared memory doubles as the y of the norm backward.
 template <int HD>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_dkv_tc_kernel(const __grid_constant__ CUtensorMap map_q32,
-                       const __grid_constant__ CUtensorMap map_do32,
-                       const __grid_constant__ CUtensorMap map_y,
+    attn_dkv_tc_kernel(const __grid_constant__ CUtensorMap map_k128,
+                       const __grid_constant__ CUtensorMap map_v128,
+                       const __grid_constant__ CUtensorMap map_q64,
+                       const __grid_constant__ CUtensorMap map_do64,
                        const __grid_constant__ CUtensorMap map_cos,
                        const __grid_constant__ CUtensorMap map_sin,
-                       const __nv_bfloat16* __restrict__ kn, const __nv_bfloat16* __restrict__ vh,
                        const float* __restrict__ lse,
                        const float* __restrict__ D, const float* __restrict__ rk,
-                       const float* __restrict__ cos_t, const float* __restrict__ sin_t,
                        __nv_bfloat16* __restrict__ dqkv, int H, int T, float scale,
                        float scale_log2, int qk_norm, int32_t* status) {
   using S = DkvSmem<HD>;
@@ -857,36 +892,45 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kt = int(blockIdx.x) % n_kt;
   const int b = bh / H, h = bh % H;
   const int k0 = kt * 128;
-  const int n_steps = (T - k0 + kQ - 1) / kQ;  // causal: queries k0 .. T-1
+  const int i_begin = k0 / kInner;
+  const int n_steps = (T + kInner - 1) / kInner - i_begin;  // causal: queries k0 .. T-1
   constexpr int NCH = HD / 64;
-  constexpr uint32_t K_COL = 384, V_COL = 448;
 
   ATTN_PROLOGUE(bars, {
-    tc::mbar_init(&bars->fixed_full, 256);  // the compute threads' K / V stores
+    tc::mbar_init(&bars->fixed_full, 1);
     tc::mbar_init(&bars->epi_full, 1);
-    for (int s = 0; s < kRing; ++s) {
+    for (int s = 0; s < kRingKV; ++s) {
       tc::mbar_init(&bars->ring_full[s], 1 + 32);  // TMA bytes + the producer warp's stat stores
-      tc::mbar_init(&bars->ring_empty[s], 1);
+      tc::mbar_init(&bars->ring_empty[s], 2);      // after dV (warp 1) and dK (warp 10)
     }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&bars->s_full[s], 1);
+      tc::mbar_init(&bars->dp_full[s], 1);
       tc::mbar_init(&bars->ds_ready[s], 256);
     }
-    tc::mbar_init(&bars->acc_full, 1);
+    tc::mbar_init(&bars->acc_full, 2);
     tc::mbar_init(&bars->done, 1);
+    tc::mbar_init(&bars->done2, 1);
   })
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort = &bars->abort;
-  const uint32_t t_dv = tmem + 128, t_dk = tmem + 256;
+  const uint32_t t_dv = tmem + 256, t_dk = tmem + 384;
 
   if (warp == 0) {
     uint32_t issued = 0, last_par = 0;
+    if (lane == 0) {
+      tc::mbar_arrive_expect_tx(&bars->fixed_full, 2 * S::BIG);
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) {
+        tc::tma_load_2d(smem + S::K_OFF + c * (128 * 128), &map_k128, &bars->fixed_full, c * 64, bh * T + k0);
+        tc::tma_load_2d(smem + S::V_OFF + c * (128 * 128), &map_v128, &bars->fixed_full, c * 64, bh * T + k0);
+      }
+    }
     for (int j = 0; j < n_steps; ++j) {
-      const int st = j % kRing;
-      const uint32_t ph = (j / kRing) & 1;
-      const int qs = k0 + j * kQ;
-      const bool ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->ring_empty[st], ph ^ 1, abort, kWaitNs));
-      if (!ok) {
+      const int st = j % kRingKV;
+      const uint32_t ph = (j / kRingKV) & 1;
+      const int qs = (i_begin + j) * kInner;
+      if (!tc::mbar_wait_warp(&bars->ring_empty[st], ph ^ 1, abort, kWaitNs)) {
         if (lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 30);
         *abort = 1;
         break;
@@ -895,128 +939,129 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mbar_arrive_expect_tx(&bars->ring_full[st], 2 * S::SMALL);
 #pragma unroll
         for (int c = 0; c < NCH; ++c) {
-          tc::tma_load_2d(smem + S::Q_OFF + st * S::SMALL + c * (kQ * 128), &map_q32,
+          tc::tma_load_2d(smem + S::Q_OFF + st * S::SMALL + c * (kInner * 128), &map_q64,
                           &bars->ring_full[st], c * 64, bh * T + qs);
-          tc::tma_load_2d(smem + S::DO_OFF + st * S::SMALL + c * (kQ * 128), &map_do32,
+          tc::tma_load_2d(smem + S::DO_OFF + st * S::SMALL + c * (kInner * 128), &map_do64,
                           &bars->ring_full[st], h * HD + c * 64, b * T + qs);
         }
         if (j == 0)
-          load_epilogue_tiles<HD>(smem + S::Y_OFF, smem + S::COS_OFF, smem + S::SIN_OFF, &map_y,
-                                  &map_cos, &map_sin, &bars->epi_full, bh * T + k0, k0);
+          load_epilogue_tiles<HD>(nullptr, smem + S::COS_OFF, smem + S::SIN_OFF, nullptr, &map_cos,
+                                  &map_sin, &bars->epi_full, 0, k0);
       }
-      float* stat = reinterpret_cast<float*>(smem + S::STAT_OFF) + st * 2 * kQ;
-      const int qq = qs + lane;
-      stat[lane] = qq < T ? lse[int64_t(bh) * T + qq] * kLog2e : 0.f;
-      stat[kQ + lane] = qq < T ? D[int64_t(bh) * T + qq] : 0.f;
+      float* stat = reinterpret_cast<float*>(smem + S::STAT_OFF) + st * 2 * kInner;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int qi = lane * 2 + e;
+        const int qq = qs + qi;
+        stat[qi] = qq < T ? lse[int64_t(bh) * T + qq] * kLog2e : 0.f;
+        stat[kInner + qi] = qq < T ? D[int64_t(bh) * T + qq] : 0.f;
+      }
       tc::mbar_arrive(&bars->ring_full[st]);
       issued |= 1u << st;
       last_par = (last_par & ~(1u << st)) | (ph << st);
     }
     if (lane == 0 && *abort) {
+      tc::mbar_wait_bounded(&bars->fixed_full, 0, nullptr, kWaitNs);
       if (issued) tc::mbar_wait_bounded(&bars->epi_full, 0, nullptr, kWaitNs);
-      for (int s = 0; s < kRing; ++s)
+      for (int s = 0; s < kRingKV; ++s)
         if (issued >> s & 1) tc::mbar_wait_bounded(&bars->ring_full[s], (last_par >> s) & 1, nullptr, kWaitNs);
     }
-  } else if (warp == 1) {
-    {  // the whole warp runs the MMA loop; elect.sync issues
-      constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, kQ, false, false);
-      constexpr uint32_t idesc_acc = tc::idesc_bf16_f32(128, HD, false, true);
-      bool ok = tc::mbar_wait_warp(&bars->fixed_full, 0, abort, kWaitNs);
+  } else if (warp == 1 || warp == 10) {
+    // warp 1: S^T = K Q^T and dV += P^T dO;  warp 10: dP^T = V dO^T and dK += dS^T Q
+    const bool is_s = warp == 1;
+    constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, kInner, false, false);
+    constexpr uint32_t idesc_acc = tc::idesc_bf16_f32(128, HD, false, true);
+    const uint64_t fd = tc::smem_desc_sw128(tc::smem_u32(smem + (is_s ? S::K_OFF : S::V_OFF)), 16);
+    const uint32_t col = is_s ? 0u : uint32_t(kInner);  // S^T or dP^T half of each pair
+    const uint32_t t_acc = is_s ? t_dv : t_dk;
+    uint64_t* prod_full = is_s ? bars->s_full : bars->dp_full;
+    bool ok = tc::mbar_wait_warp(&bars->fixed_full, 0, abort, kWaitNs);
+    bool issued_any = false;
+    auto issue_acc = [&](int j) -> bool {
+      if (!tc::mbar_wait_warp(&bars->ds_ready[j & 1], (j >> 1) & 1, abort, kWaitNs)) return false;
       tc::tc_fence_after();
-      bool issued_any = false;
-      auto issue_acc = [&](int j) -> bool {
-        if (!tc::mbar_wait_warp(&bars->ds_ready[j & 1], (j >> 1) & 1, abort, kWaitNs)) return false;
-        tc::tc_fence_after();
-        const uint32_t pt = tmem + (j & 1) * 64;  // P^T over S^T, dS^T over dP^T
-        const uint64_t qmn = tc::smem_desc_sw128(tc::smem_u32(smem + S::Q_OFF + (j % kRing) * S::SMALL), kQ * 128);
-        const uint64_t domn = tc::smem_desc_sw128(tc::smem_u32(smem + S::DO_OFF + (j % kRing) * S::SMALL), kQ * 128);
+      const uint32_t at = tmem + (j & 1) * 128 + col;  // P^T or dS^T, bf16 pairs
+      // dV takes dO, dK takes Q: the other ring tile
+      const uint64_t bmn = tc::smem_desc_sw128(
+          tc::smem_u32(smem + (is_s ? S::DO_OFF : S::Q_OFF) + (j % kRingKV) * S::SMALL), kInner * 128);
 #pragma unroll
-        for (int k = 0; k < kQ / 16; ++k) {
-          tc::mma_bf16_ts_elect(t_dv, pt + 16 * k, tc::desc_advance(domn, k * 2048), idesc_acc, (j | k) != 0);
-          tc::mma_bf16_ts_elect(t_dk, pt + 32 + 16 * k, tc::desc_advance(qmn, k * 2048), idesc_acc, (j | k) != 0);
-        }
-        tc::mma_commit_elect(&bars->ring_empty[j % kRing]);
-        return true;
-      };
-      for (int j = 0; ok && j < n_steps; ++j) {
-        const int st = j % kRing;
-        if (!tc::mbar_wait_warp(&bars->ring_full[st], (j / kRing) & 1, abort, kWaitNs)) { ok = false; break; }
-        tc::tc_fence_after();
-        const uint64_t qd = tc::smem_desc_sw128(tc::smem_u32(smem + S::Q_OFF + st * S::SMALL), 16);
-        const uint64_t dod = tc::smem_desc_sw128(tc::smem_u32(smem + S::DO_OFF + st * S::SMALL), 16);
-        const uint32_t pair = tmem + (j & 1) * 64;
+      for (int k = 0; k < kInner / 16; ++k)
+        tc::mma_bf16_ts_elect(t_acc, at + 32 * (k >> 1) + 8 * (k & 1), tc::desc_advance(bmn, k * 2048),
+                              idesc_acc, (j | k) != 0);
+      tc::mma_commit_elect(&bars->ring_empty[j % kRingKV]);
+      return true;
+    };
+    for (int j = 0; ok && j < n_steps; ++j) {
+      const int st = j % kRingKV;
+      if (!tc::mbar_wait_warp(&bars->ring_full[st], (j / kRingKV) & 1, abort, kWaitNs)) { ok = false; break; }
+      tc::tc_fence_after();
+      const uint64_t rd = tc::smem_desc_sw128(
+          tc::smem_u32(smem + (is_s ? S::Q_OFF : S::DO_OFF) + st * S::SMALL), 16);
+      const uint32_t pair = tmem + (j & 1) * 128 + col;
 #pragma unroll
-        for (int k = 0; k < HD / 16; ++k) {
-          const uint32_t small = (k >> 2) * (kQ * 128) + (k & 3) * 32;
-          tc::mma_bf16_ts_elect(pair, tmem + K_COL + 8 * k, tc::desc_advance(qd, small), idesc_s, k != 0);
-          tc::mma_bf16_ts_elect(pair + kQ, tmem + V_COL + 8 * k, tc::desc_advance(dod, small), idesc_s, k != 0);
-        }
-        issued_any = true;
-        tc::mma_commit_elect(&bars->s_full[j & 1]);
-        if (j >= 1 && !issue_acc(j - 1)) { ok = false; break; }
-      }
-      if (ok && n_steps >= 1) ok = issue_acc(n_steps - 1);
-      if (ok) tc::mma_commit_elect(&bars->acc_full);
-      if (!ok) {
-        if (lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 31);
-        *abort = 1;
-      }
-      if (issued_any) {
-        tc::mma_commit_elect(&bars->done);
-        tc::mbar_wait_warp(&bars->done, 0, nullptr, kWaitNs);
-      }
+      for (int k = 0; k < HD / 16; ++k)
+        tc::mma_bf16_ss_elect(pair, tc::desc_advance(fd, (k >> 2) * (128 * 128) + (k & 3) * 32),
+                              tc::desc_advance(rd, (k >> 2) * (kInner * 128) + (k & 3) * 32), idesc_s,
+                              k != 0);
+      issued_any = true;
+      tc::mma_commit_elect(&prod_full[j & 1]);
+      if (j >= 1 && !issue_acc(j - 1)) { ok = false; break; }
+    }
+    if (ok && n_steps >= 1) ok = issue_acc(n_steps - 1);
+    if (ok) tc::mma_commit_elect(&bars->acc_full);
+    if (!ok) {
+      if (lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, is_s ? 31 : 33);
+      *abort = 1;
+    }
+    if (issued_any) {
+      uint64_t* dn = is_s ? &bars->done : &bars->done2;
+      tc::mma_commit_elect(dn);
+      tc::mbar_wait_warp(dn, 0, nullptr, kWaitNs);
     }
   } else {
     const Roles R = roles();
     const int key = k0 + R.r;
     const bool kv = key < T;
     const int tk = kv ? key : 0;
-    stage_half_row<HD>(tmem + K_COL + R.lane_off + R.half * (HD / 4),
-                       kn + (int64_t(bh) * T + tk) * HD + R.half * (HD / 2), kv);
-    stage_half_row<HD>(tmem + V_COL + R.lane_off + R.half * (HD / 4),
-                       vh + (int64_t(bh) * T + tk) * HD + R.half * (HD / 2), kv);
-    tc::tmem_wait_st();
-    tc::tc_fence_before();
-    tc::mbar_arrive(&bars->fixed_full);
     bool ok = true;
     for (int j = 0; j < n_steps; ++j) {
-      const int sb = j & 1, st = j % kRing;
+      const int sb = j & 1, st = j % kRingKV;
       // the producer warp stored this step's stats before arriving on
       // ring_full[st]; waiting on that phase makes them visible here
       if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->s_full[sb], (j >> 1) & 1, abort, kWaitNs));
-      if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->ring_full[st], (j / kRing) & 1, abort, kWaitNs));
+      if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->dp_full[sb], (j >> 1) & 1, abort, kWaitNs));
+      if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->ring_full[st], (j / kRingKV) & 1, abort, kWaitNs));
       if (ok) {
         tc::tc_fence_after();
-        const int qs = k0 + j * kQ + R.half * 16;
-        const float4* stat4 = reinterpret_cast<const float4*>(smem + S::STAT_OFF + (st * 2 * kQ + R.half * 16) * 4);
-        const uint32_t ts = tmem + sb * 64 + R.lane_off + R.half * 16;
-        uint32_t us[16], up[16];
-        tc::tmem_ld_32x32b_x16(ts, us);
-        tc::tmem_ld_32x32b_x16(ts + kQ, up);
-        float l2[16], dd[16];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float4 a = stat4[i], c = stat4[kQ / 4 + i];
-          l2[4 * i] = a.x; l2[4 * i + 1] = a.y; l2[4 * i + 2] = a.z; l2[4 * i + 3] = a.w;
-          dd[4 * i] = c.x; dd[4 * i + 1] = c.y; dd[4 * i + 2] = c.z; dd[4 * i + 3] = c.w;
-        }
+        const int qs = (i_begin + j) * kInner + R.half * 32;
+        const float4* stat4 =
+            reinterpret_cast<const float4*>(smem + S::STAT_OFF + (st * 2 * kInner + R.half * 32) * 4);
+        const uint32_t ts = tmem + sb * 128 + R.lane_off + R.half * 32;
+        uint32_t us[32], up[32];
+        tc::tmem_ld_32x32b_x32(ts, us);
+        tc::tmem_ld_32x32b_x32(ts + kInner, up);
         tc::tmem_wait_ld();
-        const bool need_mask = !kv || qs < key || qs + 16 > T;
-        uint32_t pp[8], pd[8];
+        const bool need_mask = !kv || qs < key || qs + 32 > T;
+        uint32_t pp[16], pd[16];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int i = 2 * e;
-          float p0 = ex2(fmaf(__uint_as_float(us[i]), scale_log2, -l2[i]));
-          float p1 = ex2(fmaf(__uint_as_float(us[i + 1]), scale_log2, -l2[i + 1]));
-          if (need_mask) {
-            if (qs + i < key || qs + i >= T || !kv) p0 = 0.f;
-            if (qs + i + 1 < key || qs + i + 1 >= T || !kv) p1 = 0.f;
+        for (int g = 0; g < 8; ++g) {  // 4 queries per group
+          const float4 l4 = stat4[g], d4 = stat4[kInner / 4 + g];
+          const float l2[4] = {l4.x, l4.y, l4.z, l4.w}, dd[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+          for (int e = 0; e < 4; e += 2) {
+            const int i = 4 * g + e;
+            float p0 = ex2(fmaf(__uint_as_float(us[i]), scale_log2, -l2[e]));
+            float p1 = ex2(fmaf(__uint_as_float(us[i + 1]), scale_log2, -l2[e + 1]));
+            if (need_mask) {
+              if (qs + i < key || qs + i >= T || !kv) p0 = 0.f;
+              if (qs + i + 1 < key || qs + i + 1 >= T || !kv) p1 = 0.f;
+            }
+            pp[i / 2] = pack2(p0, p1);
+            pd[i / 2] = pack2(p0 * (__uint_as_float(up[i]) - dd[e]), p1 * (__uint_as_float(up[i + 1]) - dd[e + 1]));
           }
-          pp[e] = pack2(p0, p1);
-          pd[e] = pack2(p0 * (__uint_as_float(up[i]) - dd[i]), p1 * (__uint_as_float(up[i + 1]) - dd[i + 1]));
         }
-        tc::tmem_st_32x32b_x8(ts, pp);        // P^T over this thread's S^T columns
-        tc::tmem_st_32x32b_x8(ts + kQ, pd);   // dS^T over its dP^T columns
+        tc::tmem_st_32x32b_x16(ts, pp);           // P^T over this thread's S^T columns
+        tc::tmem_st_32x32b_x16(ts + kInner, pd);  // dS^T over its dP^T columns
         tc::tmem_wait_st();
         tc::tc_fence_before();
       }
@@ -1046,7 +1091,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    norm_rope_bwd_half<HD>(t_dk + R.lane_off, R.half, R.r, scale, smem + S::Y_OFF,
+    // the stats region is free once every step is done (acc_full): it holds red
+    norm_rope_bwd_half<HD>(t_dk + R.lane_off, R.half, R.r, scale, smem + S::K_OFF,
                            kv ? rk[int64_t(bh) * T + key] : 0.f, qk_norm, smem + S::COS_OFF,
                            smem + S::SIN_OFF, row + d + h * HD, ok, kv,
                            reinterpret_cast<float*>(smem + S::RED_OFF));
@@ -1065,10 +1111,11 @@ int attn_bwd_tc_t(const gpt_config& c, const void* q, const void* k, const void*
   const int64_t N = int64_t(B) * T;
   attn_rowdot_kernel<<<ceil_div(N * H, 8), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(dO), static_cast<const __nv_bfloat16*>(o), Dbuf, N, H, T, HD);
-  CUtensorMap k64, v64, q32, do32, yq, yk, mcos, msin;
+  CUtensorMap k64, v64, k128, v128, q64, do64, q128, do128, mcos, msin;
   bool ok = tile_map(&k64, k, rows, HD, HD, 64) && tile_map(&v64, v, rows, HD, HD, 64) &&
-            tile_map(&q32, q, rows, HD, HD, 32) && tile_map(&do32, dO, ntok, d, d, 32) &&
-            tile_map(&yq, q, rows, HD, HD, 128) && tile_map(&yk, k, rows, HD, HD, 128) &&
+            tile_map(&k128, k, rows, HD, HD, 128) && tile_map(&v128, v, rows, HD, HD, 128) &&
+            tile_map(&q64, q, rows, HD, HD, 64) && tile_map(&do64, dO, ntok, d, d, 64) &&
+            tile_map(&q128, q, rows, HD, HD, 128) && tile_map(&do128, dO, ntok, d, d, 128) &&
             tile_map_f32(&mcos, cos_t, T, HD / 2, HD / 2, 128) &&
             tile_map_f32(&msin, sin_t, T, HD / 2, HD / 2, 128);
   if (!ok) return 1;
@@ -1079,18 +1126,14 @@ int attn_bwd_tc_t(const gpt_config& c, const void* q, const void* k, const void*
   const int smem_q = int(DqSmem<HD>::BYTES);
   if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_q) != cudaSuccess)
     return 1;
-  kq<<<nt * B * H, kThreads, smem_q, st>>>(k64, v64, yq, mcos, msin, static_cast<const __nv_bfloat16*>(q),
-                                           static_cast<const __nv_bfloat16*>(dO),
-                                           lse, Dbuf, rq, cos_t, sin_t,
+  kq<<<nt * B * H, kThreads, smem_q, st>>>(q128, do128, k64, v64, mcos, msin, lse, Dbuf, rq,
                                            static_cast<__nv_bfloat16*>(dqkv), H, T, scale,
                                            scale_log2, c.qk_norm, status);
   auto kk = attn_dkv_tc_kernel<HD>;
   const int smem_k = int(DkvSmem<HD>::BYTES);
   if (cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_k) != cudaSuccess)
     return 1;
-  kk<<<nt * B * H, kThreads, smem_k, st>>>(q32, do32, yk, mcos, msin, static_cast<const __nv_bfloat16*>(k),
-                                           static_cast<const __nv_bfloat16*>(v),
-                                           lse, Dbuf, rk, cos_t, sin_t,
+  kk<<<nt * B * H, kThreads, smem_k, st>>>(k128, v128, q64, do64, mcos, msin, lse, Dbuf, rk,
                                            static_cast<__nv_bfloat16*>(dqkv), H, T, scale,
                                            scale_log2, c.qk_norm, status);
   return last_launch_rc();
