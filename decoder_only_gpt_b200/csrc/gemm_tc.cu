@@ -298,12 +298,136 @@ __device__ __forceinline__ void epi_qkv_row(const GemmArgs& g, uint32_t taddr, i
   }
 }
 
+// Staging tile of one epilogue warp: 32 rows x 32 fp32, its 16-byte units
+// XOR-swizzled by row so that both the row-wise writes and the column-wise
+// reads are free of bank conflicts.
+constexpr uint32_t kStageBytes = 32 * 32 * 4;
+__device__ __forceinline__ float4* stage_at(float* tile, int r, int u) {
+  return reinterpret_cast<float4*>(tile + r * 32 + ((u ^ (r & 7)) << 2));
+}
+
+// Partial-column fallback (col + 4 > N, or a row pitch that is not a multiple
+// of 4): the same element-wise epilogue, one element at a time.
+__device__ __noinline__ void epi4_scalar(const GemmArgs& g, int row, int col, float4 a, int sp,
+                                         int splits, int tgt, float lse_row) {
+  const int nc = min(4, g.N - col);
+  const float v[4] = {a.x, a.y, a.z, a.w};
+  for (int j = 0; j < nc; ++j) {
+    const int n = col + j;
+    if (splits > 1) {
+      g.splitk[(int64_t(sp) * g.M + row) * g.N + n] = v[j];
+      continue;
+    }
+    const int64_t e = int64_t(row) * g.ldo + n;
+    if (g.epi == EPI_RESID_F32) { static_cast<float*>(g.out)[e] += v[j]; continue; }
+    if (g.epi == EPI_STORE_F32) { static_cast<float*>(g.out)[e] = v[j]; continue; }
+    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(g.out);
+    float r = v[j];
+    if (g.epi == EPI_STORE && g.beta) r += __bfloat162float(o[e]);
+    if (g.epi == EPI_RELU2) { const float t = fmaxf(v[j], 0.f); r = t * t; }
+    if (g.epi == EPI_DRELU2) r = v[j] * 2.f * sqrt_approx(__bfloat162float(static_cast<const __nv_bfloat16*>(g.aux)[e]));
+    if (g.epi == EPI_CE_BWD) {
+      const float pr = __expf(v[j] - lse_row);
+      r = n < g.n_valid ? (pr - (n == tgt ? 1.f : 0.f)) * g.inv_n : 0.f;
+    }
+    o[e] = __float2bfloat16_rn(r);
+  }
+}
+
+// Element-wise epilogue of one 32-column chunk of a warp's 32 rows, from the
+// staging tile: lane (rsub, u4) handles columns col .. col + 4 of rows
+// 4i + rsub, i = 0..7, so each warp instruction covers 4 rows x 32 columns.
+// All of a lane's input loads are issued before any result is stored.
+// KIND: an Epilogue value, or -1 for the fp32 partial of a K split.
+template <int KIND>
+__device__ __forceinline__ void epi_chunk_coalesced(const GemmArgs& g, float* tile, int wrow0, int col,
+                                                    int rsub, int u4, int sp, int splits, int tgt,
+                                                    float lse_row) {
+  float4 a[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a[i] = *stage_at(tile, 4 * i + rsub, u4);
+  const bool col_ok = col < g.N;
+  const bool vec = col + 4 <= g.N && ((KIND == -1 ? g.N : g.ldo) & 3) == 0;
+  int t[8];
+  float ls[8];
+  if (KIND == EPI_CE_BWD) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      t[i] = __shfl_sync(0xffffffffu, tgt, 4 * i + rsub);
+      ls[i] = __shfl_sync(0xffffffffu, lse_row, 4 * i + rsub);
+    }
+  }
+  if (!col_ok) return;
+  if (!vec) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (wrow0 + 4 * i + rsub < g.M)
+        epi4_scalar(g, wrow0 + 4 * i + rsub, col, a[i], sp, splits, KIND == EPI_CE_BWD ? t[i] : -1,
+                    KIND == EPI_CE_BWD ? ls[i] : 0.f);
+    return;
+  }
+  bool ok[8];
+  int64_t e[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int row = wrow0 + 4 * i + rsub;
+    ok[i] = row < g.M;
+    e[i] = KIND == -1 ? (int64_t(sp) * g.M + row) * g.N + col : int64_t(row) * g.ldo + col;
+  }
+  if (KIND == -1 || KIND == EPI_STORE_F32 || KIND == EPI_RESID_F32) {
+    float* o = KIND == -1 ? g.splitk : static_cast<float*>(g.out);
+    if (KIND == EPI_RESID_F32) {
+      float4 x[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] = ok[i] ? *reinterpret_cast<const float4*>(o + e[i]) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        a[i].x += x[i].x; a[i].y += x[i].y; a[i].z += x[i].z; a[i].w += x[i].w;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (ok[i]) *reinterpret_cast<float4*>(o + e[i]) = a[i];
+    return;
+  }
+  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(g.out);
+  constexpr bool kIn = KIND == EPI_DRELU2 || KIND == EPI_STORE;
+  uint2 w[8];
+  if (kIn && (KIND == EPI_DRELU2 || g.beta)) {
+    const __nv_bfloat16* src = KIND == EPI_DRELU2 ? static_cast<const __nv_bfloat16*>(g.aux) : o;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = ok[i] ? *reinterpret_cast<const uint2*>(src + e[i]) : make_uint2(0u, 0u);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = make_uint2(0u, 0u);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float v[4] = {a[i].x, a[i].y, a[i].z, a[i].w};
+    const float2 i0 = unpack_bf16(w[i].x), i1 = unpack_bf16(w[i].y);
+    const float in[4] = {i0.x, i0.y, i1.x, i1.y};
+    float r[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (KIND == EPI_STORE) r[j] = v[j] + in[j];
+      else if (KIND == EPI_RELU2) { const float tt = fmaxf(v[j], 0.f); r[j] = tt * tt; }
+      else if (KIND == EPI_DRELU2) r[j] = v[j] * 2.f * sqrt_approx(in[j]);
+      else if (KIND == EPI_CE_BWD) {
+        const int n = col + j;
+        const float pr = __expf(v[j] - ls[i]);
+        r[j] = n < g.n_valid ? (pr - (n == t[i] ? 1.f : 0.f)) * g.inv_n : 0.f;
+      } else r[j] = v[j];
+    }
+    if (ok[i]) *reinterpret_cast<uint2*>(o + e[i]) = make_uint2(pack_bf16(r[0], r[1]), pack_bf16(r[2], r[3]));
+  }
+}
+
 // Epilogue of one accumulator tile for one thread: row row0 + 32*quarter +
 // lane, columns col_base .. col_base + EC (TMEM columns taddr ..), K split sp
 // of `splits`; `part` indexes this column block's cross-entropy partials.
 __device__ __forceinline__ void epilogue_tile(const GemmArgs& g, uint32_t taddr, int row0,
                                               int col_base, int part, int sp, int splits,
-                                              int quarter, int lane) {
+                                              int quarter, int lane, float* tile) {
   const int row = row0 + quarter * 32 + lane;
   const bool row_ok = row < g.M;
   int tgt = -1;
@@ -317,32 +441,50 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& g, uint32_t taddr,
     epi_qkv_row(g, taddr, row, col_base, row_ok);
     return;
   }
+  if ((g.epi == EPI_CE_FWD || g.epi == EPI_CE_BWD) && splits == 1) {
+    // per-row target and lse (or row reductions): each thread keeps its own row
 #pragma unroll 1
-  for (int c = 0; c < EC / 32; ++c) {
-    uint32_t u[32];
-    tc::tmem_ld_32x32b_x32(taddr + c * 32, u);
-    tc::tmem_wait_ld();
-    const int col0 = col_base + c * 32;
-    if (row_ok && col0 < g.N) {
-      if (splits > 1) {
-        // fp32 partial of this K split; the reduce kernel applies the epilogue
-        float* dst = g.splitk + (int64_t(sp) * g.M + row) * g.N + col0;
-        if (col0 + 32 <= g.N) {
-#pragma unroll
-          for (int j = 0; j < 32; j += 4)
-            *reinterpret_cast<float4*>(dst + j) =
-                make_float4(u2f(u[j]), u2f(u[j + 1]), u2f(u[j + 2]), u2f(u[j + 3]));
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (col0 + j < g.N) dst[j] = u2f(u[j]);
-        }
-      } else {
+    for (int c = 0; c < EC / 32; ++c) {
+      uint32_t u[32];
+      tc::tmem_ld_32x32b_x32(taddr + c * 32, u);
+      tc::tmem_wait_ld();
+      const int col0 = col_base + c * 32;
+      if (row_ok && col0 < g.N) {
         float v[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = u2f(u[j]);
         epi_chunk(g, row, col0, v, ce_max, ce_sum, ce_tgt, tgt, lse_row);
       }
+    }
+  } else {
+    // Everything that writes the output element by element: the warp's 32
+    // rows x 32 columns pass through its staging tile, then each lane handles
+    // 4 columns of a row so that a warp instruction covers 4 rows x 32
+    // consecutive columns.
+    const int wrow0 = row0 + quarter * 32;
+    const int rsub = lane >> 3, u4 = lane & 7;
+#pragma unroll 1
+    for (int c = 0; c < EC / 32; ++c) {
+      uint32_t u[32];
+      tc::tmem_ld_32x32b_x32(taddr + c * 32, u);
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        *stage_at(tile, lane, k) = make_float4(u2f(u[4 * k]), u2f(u[4 * k + 1]), u2f(u[4 * k + 2]), u2f(u[4 * k + 3]));
+      __syncwarp();
+      const int col = col_base + c * 32 + 4 * u4;
+      if (splits > 1) {
+        epi_chunk_coalesced<-1>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row);
+      } else {
+        switch (g.epi) {
+          case EPI_RESID_F32: epi_chunk_coalesced<EPI_RESID_F32>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row); break;
+          case EPI_STORE_F32: epi_chunk_coalesced<EPI_STORE_F32>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row); break;
+          case EPI_RELU2: epi_chunk_coalesced<EPI_RELU2>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row); break;
+          case EPI_DRELU2: epi_chunk_coalesced<EPI_DRELU2>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row); break;
+          default: epi_chunk_coalesced<EPI_STORE>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row); break;
+        }
+      }
+      __syncwarp();
     }
   }
   if (row_ok && g.epi == EPI_CE_FWD) {
@@ -373,7 +515,10 @@ struct __align__(8) PairTail {
   uint32_t tmem_base;
   int abort;
 };
-constexpr size_t kPairSmemBytes = 1024 + P_STAGES * 2 * P_HALF + sizeof(PairTail);
+constexpr size_t kPairTailBytes = (sizeof(PairTail) + 15) / 16 * 16;
+constexpr size_t kPairSmemBytes =
+    1024 + P_STAGES * 2 * P_HALF + kPairTailBytes + (kThreads - 64) / 32 * kStageBytes;
+static_assert(kPairSmemBytes <= 232448, "");
 }  // namespace
 
 template <bool AMN, bool BMN>
@@ -515,6 +660,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else {
     const int quarter = warp & 3;      // TMEM lanes 32*quarter .. +31
     const int ch = (warp - 2) >> 2;    // columns ch*EC .. ch*EC + EC of each tile
+    float* stage_tile = reinterpret_cast<float*>(smem + 2 * P_STAGES * P_HALF + kPairTailBytes +
+                                                 (warp - 2) * kStageBytes);
     const int my_row = int(rank) * 128 + quarter * 32 + lane;  // within a 256-row pair tile
     if (pair < num_units)
       epilogue_prefetch(g, (pair / splits / n_tiles) * P_BM + my_row,
@@ -539,7 +686,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int nb = tile % n_tiles;
       epilogue_tile(g, tmem_base + (uint32_t(quarter * 32) << 16) + acc * BN + ch * EC,
                     (tile / n_tiles) * P_BM + int(rank) * 128, nb * BN + ch * EC, nb * (BN / EC) + ch, sp,
-                    splits, quarter, lane);
+                    splits, quarter, lane, stage_tile);
       tc::tc_fence_before();
       tc::mbar_arrive_cluster(tc::mapa_shared(tc::smem_u32(&tail->tmem_empty[acc]), 0));
     }
