@@ -460,25 +460,32 @@ int launch_attn_fwd_tc(const gpt_config& c, const void* q, const void* k, const 
 // ===========================================================================
 namespace {
 
-// D_i = dO_i . o_i, one warp per (token, head)
+// D_i = dO_i . o_i: 8 elements (16 bytes of each operand) per thread, hd/8
+// consecutive threads per (token, head) row, reduced by shuffles in that group
 __global__ void attn_rowdot_kernel(const __nv_bfloat16* __restrict__ dO,
                                    const __nv_bfloat16* __restrict__ o, float* __restrict__ D,
                                    int64_t N, int H, int T, int hd) {
-  const int64_t w = int64_t(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
-  const int lane = threadIdx.x & 31;
-  if (w >= N * H) return;
-  const int64_t n = w / H;
-  const int h = int(w % H);
-  const __nv_bfloat162* a = reinterpret_cast<const __nv_bfloat162*>(dO + n * H * hd + h * hd);
-  const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(o + n * H * hd + h * hd);
+  const int G = hd / 8;  // 8 or 16: groups never straddle a warp
+  const int64_t gid = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t rowi = gid / G;  // token * H + head
+  const int part = int(gid % G);
+  const bool ok = rowi < N * H;
   float s = 0.f;
-  for (int i = lane; i < hd / 2; i += 32) {
-    float2 x = __bfloat1622float2(a[i]), y = __bfloat1622float2(b[i]);
-    s += x.x * y.x + x.y * y.y;
+  if (ok) {
+    const uint4 a = *reinterpret_cast<const uint4*>(dO + rowi * hd + part * 8);
+    const uint4 b = *reinterpret_cast<const uint4*>(o + rowi * hd + part * 8);
+    const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wa[e]));
+      const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wb[e]));
+      s += x.x * y.x + x.y * y.y;
+    }
   }
-  s = warp_sum(s);
-  if (lane == 0) {
-    const int64_t bb = n / T, t = n % T;
+  for (int off = G / 2; off >= 1; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  if (ok && part == 0) {
+    const int64_t n = rowi / H, bb = n / T, t = n % T;
+    const int h = int(rowi % H);
     D[(bb * H + h) * T + t] = s;
   }
 }
@@ -1109,7 +1116,7 @@ int attn_bwd_tc_t(const gpt_config& c, const void* q, const void* k, const void*
   const int H = c.n_head, T = c.seq_len, B = c.batch, d = H * HD;
   const uint64_t rows = uint64_t(B) * H * T, ntok = uint64_t(B) * T;
   const int64_t N = int64_t(B) * T;
-  attn_rowdot_kernel<<<ceil_div(N * H, 8), 256, 0, st>>>(
+  attn_rowdot_kernel<<<ceil_div(N * H * (HD / 8), 256), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(dO), static_cast<const __nv_bfloat16*>(o), Dbuf, N, H, T, HD);
   CUtensorMap k64, v64, k128, v128, q64, do64, q128, do128, mcos, msin;
   bool ok = tile_map(&k64, k, rows, HD, HD, 64) && tile_map(&v64, v, rows, HD, HD, 64) &&
