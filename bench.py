@@ -215,6 +215,44 @@ def roofline(sites, w, gemm_tf, peak_tf, peaks):
     return line
 
 
+def time_optimizer(B, st, stream, reps=3):
+    """Device time of gpt_optim_step on the step's own gradients (library
+    defaults: the two printed Newton-Schulz iterations), with the per-class
+    trace: the Newton-Schulz GEMMs and the element-wise AdamW / Muon passes."""
+    import torch
+    opt = B.optim_defaults()
+    st.init_optimizer()
+    st.optimizer_step(opt)  # warm-up
+    torch.cuda.synchronize()
+    trace = B.Trace(capacity=8192)
+    trace.attach()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(reps):
+        opt.step = 2 + i
+        st.optimizer_step(opt)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    B.Trace.detach()
+    stats, _ = trace.summary()
+    trace.close()
+    code = st.status()
+    if code != B.GPT_OK:
+        raise SystemExit(f"device status after optimizer steps: {B.strerror(code)}")
+    ms = e0.elapsed_time(e1) / reps
+    g, o = stats["gemm"], stats["other"]
+    line = {"ms_per_step": round(ms, 3), "ns_steps": int(opt.ns_steps),
+            "state_bytes": int(st.opt_state.numel()),
+            "newton_schulz_gemm": {"ms_per_step": round(g["ms"] / reps, 3),
+                                   "launches_per_step": g["launches"] // reps,
+                                   "tflops": round(g["flops"] / (g["ms"] / 1e3) / 1e12, 1) if g["ms"] else None},
+            "elementwise": {"ms_per_step": round(o["ms"] / reps, 3),
+                            "gbs": round(o["bytes"] / (o["ms"] / 1e3) / 1e9, 1) if o["ms"] else None}}
+    del st.opt_state
+    torch.cuda.empty_cache()
+    return line
+
+
 def max_over_ranks(values, device):
     """Element-wise maximum of per-rank timings over the process group (the
     reported step time of a multi-GPU run is the slowest rank's)."""
@@ -325,6 +363,12 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     e2e_ms = f0.elapsed_time(f1)
 
+    # ---- optimizer step (AdamW + Muon), timed on its own: not part of the
+    # fwd+bwd metric; single-GPU runs only ----
+    optim = None
+    if world == 1 and not args.no_optimizer and cfg.dtype == B.GPT_BF16:
+        optim = time_optimizer(B, st, stream)
+
     if world > 1:
         ms, e2e_ms = max_over_ranks([ms, e2e_ms], dev)
         dist.barrier()
@@ -386,6 +430,8 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk,
         "cpu_baseline": cpu,
     }
+    if optim is not None:
+        line["optimizer"] = optim
     print(json.dumps(line), flush=True)
 
 
@@ -435,6 +481,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD, choices=list(synth.WORKLOADS))
+    ap.add_argument("--no-optimizer", action="store_true",
+                    help="skip the separate timing of the optimizer step")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip timing the CPU oracle sample")
     ap.add_argument("--layers", type=int, default=None,

@@ -37,6 +37,27 @@ class GptConfig(ctypes.Structure):
     ]
 
 
+class GptOptim(ctypes.Structure):
+    """Mirror of gpt_optim (optimizer hyper-parameters of one step)."""
+    _fields_ = [("adam_lr", ctypes.c_float), ("adam_beta1", ctypes.c_float),
+                ("adam_beta2", ctypes.c_float), ("adam_eps", ctypes.c_float),
+                ("adam_weight_decay", ctypes.c_float), ("muon_lr", ctypes.c_float),
+                ("muon_momentum", ctypes.c_float), ("muon_nesterov", ctypes.c_int32),
+                ("ns_steps", ctypes.c_int32), ("ns_coeffs", (ctypes.c_float * 3) * 8),
+                ("step", ctypes.c_int64)]
+
+    def coeffs(self):
+        return [tuple(float(x) for x in self.ns_coeffs[i]) for i in range(self.ns_steps)]
+
+    def set_coeffs(self, triples):
+        if len(triples) > 8:
+            raise ValueError("at most 8 Newton-Schulz iterations")
+        self.ns_steps = len(triples)
+        for i, t in enumerate(triples):
+            for j in range(3):
+                self.ns_coeffs[i][j] = float(t[j])
+
+
 class GptError(RuntimeError):
     def __init__(self, code: int, what: str):
         self.code = code
@@ -67,9 +88,15 @@ def lib() -> ctypes.CDLL:
         L.gpt_strerror.argtypes = [I]
         L.gpt_strerror.restype = ctypes.c_char_p
         L.gpt_version.restype = ctypes.c_char_p
+        optp = ctypes.POINTER(GptOptim)
+        L.gpt_optim_defaults.argtypes = [optp]
+        L.gpt_optim_state_bytes.argtypes = [cfgp, ctypes.POINTER(ctypes.c_size_t)]
+        L.gpt_optim_init.argtypes = [cfgp, P, P, P]
+        L.gpt_optim_step.argtypes = [cfgp, optp, P, P, P, P, P]
         for f in ("gpt_config_init", "gpt_config_from_depth", "gpt_param_offset",
                   "gpt_workspace_region", "gpt_forward_loss", "gpt_backward",
-                  "gpt_train_step_host", "gpt_status"):
+                  "gpt_train_step_host", "gpt_status", "gpt_optim_defaults",
+                  "gpt_optim_state_bytes", "gpt_optim_init", "gpt_optim_step"):
             getattr(L, f).restype = I
         _lib = L
     return _lib
@@ -260,3 +287,29 @@ class Trace:
         if self._h:
             lib().gpt_trace_destroy(self._h)
             self._h = ctypes.c_void_p()
+
+
+# ---- optimizer step ---------------------------------------------------------
+def optim_defaults() -> GptOptim:
+    o = GptOptim()
+    _check(lib().gpt_optim_defaults(ctypes.byref(o)), "gpt_optim_defaults")
+    return o
+
+
+def optim_state_bytes(cfg: GptConfig) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().gpt_optim_state_bytes(ctypes.byref(cfg), ctypes.byref(n)), "gpt_optim_state_bytes")
+    return int(n.value)
+
+
+def optim_init(cfg, params, state, stream=None):
+    _check(lib().gpt_optim_init(ctypes.byref(cfg), _ptr(params), _ptr(state), stream), "gpt_optim_init")
+
+
+def raw_optim_step(cfg, opt, params, grads, state, workspace, stream=None) -> int:
+    return lib().gpt_optim_step(ctypes.byref(cfg), ctypes.byref(opt) if opt is not None else None,
+                                _ptr(params), _ptr(grads), _ptr(state), _ptr(workspace), stream)
+
+
+def optim_step(cfg, opt, params, grads, state, workspace, stream=None):
+    _check(raw_optim_step(cfg, opt, params, grads, state, workspace, stream), "gpt_optim_step")

@@ -1,6 +1,7 @@
 // libgpt C ABI: configuration, parameter / workspace layout and the step
 // orchestration (which kernel runs when, on which buffers).  Every numeric
 // step runs in the CUDA kernels of this directory; this file only enqueues.
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -104,6 +105,20 @@ bool make_layout(const gpt_config& c, Layout* L) {
   L->scat_items = b.take(L->scat_max_items * 8);
   L->scat_item_offs = b.take((V + 1) * 8);
   L->scat_partial = b.take((N / 64 + 1) * d * 4 * 2);
+  // optimizer scratch (bf16): two Newton-Schulz iterates of the largest block
+  // matrix, two Gram matrices of the smaller side (d for every block matrix),
+  // the sum-of-squares partials and the reciprocal norm
+  if (c.dtype == GPT_BF16) {
+    const int64_t mat = std::max(std::max(3 * d * d, F * d), d * d);
+    const int64_t gd = d;  // the smaller side of Wqkv, Wo, Wup and Wdown is at most d
+    L->opt_x0 = b.take(mat * 2);
+    L->opt_x1 = b.take(mat * 2);
+    L->opt_a = b.take(gd * gd * 2);
+    L->opt_b = b.take(gd * gd * 2);
+    L->opt_part = b.take((kOptNormBlocks + 1) * 4);
+  } else {
+    L->opt_x0 = L->opt_x1 = L->opt_a = L->opt_b = L->opt_part = 0;
+  }
   L->total = align_up(b.off, kAlign);
   return true;
 }
@@ -274,6 +289,7 @@ static int run_gemm(const gpt_config& c, const GemmArgs& g, cudaStream_t st) {
     case EPI_STORE: bytes += mn * e * (g.beta ? 2 : 1); break;
     case EPI_RESID_F32: bytes += mn * 8; break;
     case EPI_DRELU2: bytes += mn * e * 2; break;
+    case EPI_AXPBY: bytes += mn * e * 2; break;
     case EPI_CE_FWD: bytes += double(g.M) * 12; break;
     case EPI_QKV: bytes += mn * e + double(g.M) * 2 * g.n_head * 4; break;
     default: bytes += mn * e; break;
@@ -540,6 +556,158 @@ int gpt_status(const void* workspace, void* stream) {
   if (cudaMemcpy(&s, workspace, sizeof(s), cudaMemcpyDeviceToHost) != cudaSuccess)
     return GPT_ECUDA;
   return s.code;
+}
+
+
+// ---------------------------------------------------------------------------
+// optimizer step ("ChatGPT'nizi 50 Dolara Nasil Egitirsiniz?", section "2. Muon
+// Optimize Edici (nanochat/optim.py)"): AdamW for wte and lm_head, Muon for
+// the block matrices
+// ---------------------------------------------------------------------------
+int gpt_optim_defaults(gpt_optim* o) {
+  if (!o) return GPT_EINVAL;
+  *o = gpt_optim{};
+  // library defaults (the pages give no values): Adam's published
+  // suggestions, a common Muon setting, the two printed coefficient triples
+  o->adam_lr = 1e-3f;
+  o->adam_beta1 = 0.9f;
+  o->adam_beta2 = 0.999f;
+  o->adam_eps = 1e-8f;
+  o->adam_weight_decay = 0.f;
+  o->muon_lr = 0.02f;
+  o->muon_momentum = 0.95f;
+  o->muon_nesterov = 1;
+  o->ns_steps = 2;
+  const float printed[2][3] = {{8.156f, -22.483f, 15.879f}, {4.043f, -2.809f, 0.500f}};
+  for (int i = 0; i < 2; ++i)
+    for (int j = 0; j < 3; ++j) o->ns_coeffs[i][j] = printed[i][j];
+  o->step = 1;
+  return GPT_OK;
+}
+
+static int check_optim_cfg(const gpt_config* c) {
+  if (!c) return GPT_EINVAL;
+  gpt_config chk = *c;
+  int rc = gpt_config_init(&chk);
+  if (rc != GPT_OK) return rc;
+  if (chk.param_bytes != c->param_bytes || chk.workspace_bytes != c->workspace_bytes)
+    return GPT_EINVAL;
+  if (c->dtype != GPT_BF16) return GPT_EUNSUPPORTED;
+  return GPT_OK;
+}
+
+int gpt_optim_state_bytes(const gpt_config* c, size_t* bytes) {
+  if (!bytes) return GPT_EINVAL;
+  const int rc = check_optim_cfg(c);
+  if (rc != GPT_OK) return rc;
+  *bytes = size_t(3) * (c->param_bytes / 2) * 4;
+  return GPT_OK;
+}
+
+int gpt_optim_init(const gpt_config* c, const void* params, void* state, void* stream) {
+  const int rc = check_optim_cfg(c);
+  if (rc != GPT_OK) return rc;
+  if (!params || !state || !aligned(params, 256) || !aligned(state, 256)) return GPT_EINVAL;
+  const int64_t pe = int64_t(c->param_bytes / 2);
+  float* w = static_cast<float*>(state);
+  return launch_optim_init(params, w, w + pe, w + 2 * pe, pe, stream) ? GPT_ECUDA : GPT_OK;
+}
+
+int gpt_optim_step(const gpt_config* c, const gpt_optim* o, void* params, const void* grads,
+                   void* state, void* workspace, void* stream) {
+  int rc = check_optim_cfg(c);
+  if (rc != GPT_OK) return rc;
+  if (!o || !params || !grads || !state || !workspace) return GPT_EINVAL;
+  if (!aligned(params, 256) || !aligned(grads, 256) || !aligned(state, 256) || !aligned(workspace, 256))
+    return GPT_EINVAL;
+  if (o->ns_steps < 0 || o->ns_steps > 8 || o->step < 1) return GPT_EINVAL;
+  const float hp[] = {o->adam_lr, o->adam_beta1, o->adam_beta2, o->adam_eps, o->adam_weight_decay,
+                      o->muon_lr, o->muon_momentum};
+  for (float x : hp)
+    if (!std::isfinite(x)) return GPT_EINVAL;
+  for (int i = 0; i < o->ns_steps; ++i)
+    for (int j = 0; j < 3; ++j)
+      if (!std::isfinite(o->ns_coeffs[i][j])) return GPT_EINVAL;
+  if (!(o->adam_beta1 >= 0.f && o->adam_beta1 < 1.f && o->adam_beta2 >= 0.f && o->adam_beta2 < 1.f))
+    return GPT_EINVAL;
+  if (o->muon_nesterov != 0 && o->muon_nesterov != 1) return GPT_EINVAL;
+
+  cudaStream_t st = (cudaStream_t)stream;
+  Layout L;
+  make_layout(*c, &L);
+  char* ws = static_cast<char*>(workspace);
+  int32_t* status = reinterpret_cast<int32_t*>(ws + L.status);
+  const int64_t pe = int64_t(c->param_bytes / 2);
+  float* W = static_cast<float*>(state);
+  float* M = W + pe;
+  float* Vv = M + pe;
+  auto* P = static_cast<__nv_bfloat16*>(params);
+  auto* G = static_cast<const __nv_bfloat16*>(grads);
+
+  // AdamW: the embedding and lm_head
+  const double t = double(o->step);
+  const float bc1 = float(1.0 - std::pow(double(o->adam_beta1), t));
+  const float bc2 = float(1.0 - std::pow(double(o->adam_beta2), t));
+  for (int tensor : {GPT_T_WTE, GPT_T_LM_HEAD}) {
+    int64_t off, r, cc;
+    gpt_param_offset(c, tensor, 0, &off, &r, &cc);
+    const int64_t n = r * cc;
+    TraceScope ts(GPT_K_OTHER, 1, 0, double(n) * 30.0, st);
+    GPT_TRY(launch_adamw(P + off, G + off, W + off, M + off, Vv + off, n, o->adam_lr, o->adam_beta1,
+                         o->adam_beta2, o->adam_eps, o->adam_weight_decay, bc1, bc2, st));
+  }
+  // Muon: every block matrix
+  void* x0 = ws + L.opt_x0;
+  void* x1 = ws + L.opt_x1;
+  void* A = ws + L.opt_a;
+  void* Bm = ws + L.opt_b;
+  float* part = reinterpret_cast<float*>(ws + L.opt_part);
+  for (int l = 0; l < c->n_layer; ++l) {
+    for (int tensor : {GPT_T_WQKV, GPT_T_WO, GPT_T_WUP, GPT_T_WDOWN}) {
+      int64_t off, r, cc;
+      gpt_param_offset(c, tensor, l, &off, &r, &cc);
+      const int64_t n = r * cc;
+      {
+        TraceScope ts(GPT_K_OTHER, 3, 0, double(n) * 16.0, st);
+        GPT_TRY(launch_muon_prepare(G + off, M + off, n, o->muon_momentum, o->muon_nesterov, part, x0,
+                                    st));
+      }
+      // Newton-Schulz on X [r, cc]; the Gram matrix is gd x gd over the smaller side
+      const bool tall = r >= cc;
+      const int gd = int(tall ? cc : r);
+      void* X = x0;
+      void* Xn = x1;
+      for (int i = 0; i < o->ns_steps; ++i) {
+        const float a = o->ns_coeffs[i][0], b = o->ns_coeffs[i][1], cf = o->ns_coeffs[i][2];
+        // A = X^T X (tall) or X X^T (wide)
+        GemmArgs g1 = tall ? gemm_kk(X, cc, X, cc, gd, gd, int(r), EPI_STORE, A, gd, status)
+                           : gemm_kk(X, cc, X, cc, gd, gd, int(cc), EPI_STORE, A, gd, status);
+        g1.a_mn_major = tall;
+        g1.b_mn_major = tall;
+        GPT_TRY(run_gemm(*c, with_splitk(g1, L, ws), st));
+        // B = c A A + b A
+        GemmArgs g2 = gemm_kk(A, gd, A, gd, gd, gd, gd, EPI_AXPBY, Bm, gd, status);
+        g2.b_mn_major = true;
+        g2.aux = A;
+        g2.alpha = cf;
+        g2.beta_aux = b;
+        GPT_TRY(run_gemm(*c, g2, st));
+        // X' = X B + a X (tall) or B X + a X (wide)
+        GemmArgs g3 = tall ? gemm_kk(X, cc, Bm, gd, int(r), int(cc), gd, EPI_AXPBY, Xn, cc, status)
+                           : gemm_kk(Bm, gd, X, cc, int(r), int(cc), gd, EPI_AXPBY, Xn, cc, status);
+        g3.b_mn_major = true;
+        g3.aux = X;
+        g3.alpha = 1.f;
+        g3.beta_aux = a;
+        GPT_TRY(run_gemm(*c, g3, st));
+        std::swap(X, Xn);
+      }
+      const float step = o->muon_lr * std::sqrt(std::max(1.f, float(r) / float(cc)));
+      TraceScope ts(GPT_K_OTHER, 1, 0, double(n) * 12.0, st);
+      GPT_TRY(launch_muon_apply(X, W + off, P + off, n, step, st));
+    }
+  }
+  return GPT_OK;
 }
 
 }  // extern "C"

@@ -326,6 +326,8 @@ __device__ __noinline__ void epi4_scalar(const GemmArgs& g, int row, int col, fl
     if (g.epi == EPI_STORE && g.beta) r += __bfloat162float(o[e]);
     if (g.epi == EPI_RELU2) { const float t = fmaxf(v[j], 0.f); r = t * t; }
     if (g.epi == EPI_DRELU2) r = v[j] * 2.f * sqrt_approx(__bfloat162float(static_cast<const __nv_bfloat16*>(g.aux)[e]));
+    if (g.epi == EPI_AXPBY)
+      r = g.alpha * v[j] + g.beta_aux * __bfloat162float(static_cast<const __nv_bfloat16*>(g.aux)[e]);
     if (g.epi == EPI_CE_BWD) {
       const float pr = __expf(v[j] - lse_row);
       r = n < g.n_valid ? (pr - (n == tgt ? 1.f : 0.f)) * g.inv_n : 0.f;
@@ -391,10 +393,10 @@ __device__ __forceinline__ void epi_chunk_coalesced(const GemmArgs& g, float* ti
     return;
   }
   __nv_bfloat16* o = static_cast<__nv_bfloat16*>(g.out);
-  constexpr bool kIn = KIND == EPI_DRELU2 || KIND == EPI_STORE;
+  constexpr bool kIn = KIND == EPI_DRELU2 || KIND == EPI_STORE || KIND == EPI_AXPBY;
   uint2 w[8];
-  if (kIn && (KIND == EPI_DRELU2 || g.beta)) {
-    const __nv_bfloat16* src = KIND == EPI_DRELU2 ? static_cast<const __nv_bfloat16*>(g.aux) : o;
+  if (kIn && (KIND != EPI_STORE || g.beta)) {
+    const __nv_bfloat16* src = KIND == EPI_STORE ? o : static_cast<const __nv_bfloat16*>(g.aux);
 #pragma unroll
     for (int i = 0; i < 8; ++i) w[i] = ok[i] ? *reinterpret_cast<const uint2*>(src + e[i]) : make_uint2(0u, 0u);
   } else {
@@ -412,6 +414,7 @@ __device__ __forceinline__ void epi_chunk_coalesced(const GemmArgs& g, float* ti
       if (KIND == EPI_STORE) r[j] = v[j] + in[j];
       else if (KIND == EPI_RELU2) { const float tt = fmaxf(v[j], 0.f); r[j] = tt * tt; }
       else if (KIND == EPI_DRELU2) r[j] = v[j] * 2.f * sqrt_approx(in[j]);
+      else if (KIND == EPI_AXPBY) r[j] = g.alpha * v[j] + g.beta_aux * in[j];
       else if (KIND == EPI_CE_BWD) {
         const int n = col + j;
         const float pr = __expf(v[j] - ls[i]);
@@ -481,6 +484,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& g, uint32_t taddr,
           case EPI_STORE_F32: epi_chunk_coalesced<EPI_STORE_F32>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row); break;
           case EPI_RELU2: epi_chunk_coalesced<EPI_RELU2>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row); break;
           case EPI_DRELU2: epi_chunk_coalesced<EPI_DRELU2>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row); break;
+          case EPI_AXPBY: epi_chunk_coalesced<EPI_AXPBY>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row); break;
           default: epi_chunk_coalesced<EPI_STORE>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row); break;
         }
       }

@@ -28,6 +28,7 @@ enum Epilogue : int32_t {
   EPI_CE_FWD,       // per-row partial (max, sum exp) over the tile's columns + target logit
   EPI_CE_BWD,       // out_t = (exp(acc - lse[m]) - [n == tgt[m]]) * inv_n; 0 for n >= n_valid
   EPI_QKV,          // [q|k|v] row: RoPE + per-head RMSNorm of q, k; head-major scatter of q, k, v
+  EPI_AXPBY,        // out_t = alpha * acc + beta_aux * aux_t   (Newton-Schulz updates)
 };
 
 struct GemmArgs {
@@ -42,7 +43,8 @@ struct GemmArgs {
   void* out;
   int64_t ldo;
   int beta;                 // EPI_STORE: 1 = accumulate into out
-  const void* aux;          // EPI_DRELU2: stored activation a, leading dim ldo
+  const void* aux;          // EPI_DRELU2, EPI_AXPBY: second input, leading dim ldo
+  float alpha = 1.f, beta_aux = 0.f;  // EPI_AXPBY scales
   // cross-entropy epilogues
   const int32_t* targets;   // [M]
   float* part_max;          // [M, n_part]
@@ -92,10 +94,25 @@ struct Layout {
   int64_t n_part_max;      // partial-stat columns reserved per row
   int64_t sort_tiles;      // N / 1024 rounded up
   int64_t scat_max_items;  // upper bound of (row, chunk) work items of the scatter
+  // optimizer scratch (bf16 configs): Newton-Schulz iterates, Gram matrices,
+  // sum-of-squares partials
+  uint64_t opt_x0, opt_x1, opt_a, opt_b, opt_part;
   uint64_t total;
 };
 
 bool make_layout(const gpt_config& c, Layout* L);
+
+// ---- optimizer (csrc/optim.cu) ----
+constexpr int kOptNormBlocks = 296;  // fixed grid of the deterministic sum of squares
+int launch_optim_init(const void* params, float* master, float* m, float* v, int64_t n, void* stream);
+int launch_adamw(void* params, const void* grads, float* master, float* m, float* v, int64_t n,
+                 float lr, float b1, float b2, float eps, float wd, float bc1, float bc2, void* stream);
+// M = mu M + G; U = nesterov ? G + mu M : M; x = bf16(U / (||U||_F + 1e-7)).
+// partial: kOptNormBlocks + 1 floats of scratch.
+int launch_muon_prepare(const void* grads, float* mom, int64_t n, float mu, int nesterov,
+                        float* partial, void* x_out, void* stream);
+// master -= step * x; params = bf16(master)
+int launch_muon_apply(const void* x, float* master, void* params, int64_t n, float step, void* stream);
 
 // ---- launchers (all enqueue on `stream`, return cudaError_t as int) ------
 int launch_rope_table(const gpt_config& c, float* cos_t, float* sin_t, void* stream);

@@ -65,6 +65,23 @@ class TrainStep:
     def status(self) -> int:
         return B.status(self.workspace, self.stream)
 
+    # ---- optimizer ----------------------------------------------------------
+    def init_optimizer(self) -> None:
+        """Allocate the optimizer state and copy the parameters into its fp32 master."""
+        self.opt_state = torch.zeros(B.optim_state_bytes(self.cfg), dtype=torch.uint8,
+                                     device=self.device)
+        B.optim_init(self.cfg, self.params, self.opt_state, self.stream)
+
+    def optimizer_step(self, opt: B.GptOptim) -> None:
+        B.optim_step(self.cfg, opt, self.params, self.grads, self.opt_state, self.workspace,
+                     self.stream)
+
+    def optimizer_state(self):
+        """(master, m, v) as host float32 arrays in the parameter buffer's layout."""
+        st = self.opt_state.cpu().numpy().view(np.float32)
+        pe = self.cfg.param_bytes // 2
+        return st[:pe], st[pe:2 * pe], st[2 * pe:3 * pe]
+
     # ---- read-back --------------------------------------------------------
     def grads_f64(self) -> Dict[str, np.ndarray]:
         dt = B.elem_dtype(self.cfg)

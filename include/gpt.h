@@ -22,7 +22,8 @@
  *
  * Conventions for every call below:
  *  - All device buffers are owned by the caller; the library allocates no
- *    device memory and keeps no global mutable state.  Pointers marked
+ *    device memory and keeps no global mutable state (except the scratch
+ *    array of gpt_embedding_grad_noalloc, described there).  Pointers marked
  *    "device" must be device memory of the current CUDA device.
  *  - Device pointers must be 16-byte aligned (TMA); params/grads/workspace
  *    256-byte aligned.  A violation returns GPT_EINVAL before any launch.
@@ -196,6 +197,60 @@ const char* gpt_version(void);
 int gpt_embedding_grad_noalloc(const int32_t* tokens, int64_t n_tokens, int32_t vocab,
                                int32_t d_model, int32_t dtype, const float* dx0, void* dwte,
                                int accumulate, void* stream);
+
+/* ---- optimizer step ------------------------------------------------------------
+ * "ChatGPT'nizi 50 Dolara Nasil Egitirsiniz?" (dev.to), section "2. Muon
+ * Optimize Edici (nanochat/optim.py)": the embedding (wte) and lm_head are
+ * updated with AdamW, every 2-D block matrix (Wqkv, Wo, Wup, Wdown) with Muon,
+ * whose momentum is orthogonalised by the iteration
+ *     A = X^T X,  B = b A + c A A,  X <- a X + X B
+ * (the Gram matrix is taken over the smaller dimension: for a matrix with
+ * fewer rows than columns, A = X X^T and X <- a X + B X).
+ *
+ * State (caller-owned, device, fp32, gpt_optim_state_bytes): three arrays of
+ * the parameter buffer's element count, at the parameter buffer's element
+ * offsets: the fp32 master weights, then m (AdamW first moment; Muon momentum),
+ * then v (AdamW second moment; unused for Muon matrices).  The bf16 parameter
+ * buffer is the master rounded to nearest even after every step: the pages'
+ * layers cast a higher-precision weight to bf16 per call (section "3.
+ * Hassasiyet Yonetimi").
+ *
+ * Per step, with t = step (1-based):
+ *   AdamW:  m = b1 m + (1-b1) g;  v = b2 v + (1-b2) g^2;
+ *           w = w (1 - lr wd) - lr (m / (1-b1^t)) / (sqrt(v / (1-b2^t)) + eps)
+ *   Muon:   M = mu M + G;  U = G + mu M if nesterov else M;
+ *           X = U / (||U||_F + 1e-7), then ns_steps iterations with
+ *           (a, b, c) = ns_coeffs[i] in bf16 on the tensor cores;
+ *           w = w - lr sqrt(max(1, rows/cols)) X.
+ * bf16 configurations only (dtype GPT_F32 returns GPT_EUNSUPPORTED). */
+typedef struct {
+  float adam_lr, adam_beta1, adam_beta2, adam_eps, adam_weight_decay;
+  float muon_lr, muon_momentum;
+  int32_t muon_nesterov;   /* 1: orthogonalise G + mu M */
+  int32_t ns_steps;        /* 0 .. 8 */
+  float ns_coeffs[8][3];   /* (a, b, c) of iteration i */
+  int64_t step;            /* AdamW step count t >= 1 */
+} gpt_optim;
+
+/* Library defaults (the pages give no hyper-parameter values): AdamW lr 1e-3,
+ * betas (0.9, 0.999), eps 1e-8 (Adam's published suggestions), no weight
+ * decay; Muon lr 0.02, momentum 0.95, Nesterov; ns_steps 2 with the two
+ * coefficient triples the page prints, (8.156, -22.483, 15.879) and
+ * (4.043, -2.809, 0.5) (its list of five breaks off there: longer schedules
+ * are the caller's); step 1.  Returns GPT_EINVAL for a NULL pointer. */
+int gpt_optim_defaults(gpt_optim* opt);
+/* Bytes of the optimizer state for an initialised config (3 fp32 copies of
+ * the parameter buffer's elements). */
+int gpt_optim_state_bytes(const gpt_config* cfg, size_t* bytes);
+/* master = params (exact upcast), m = v = 0.  Async on `stream`. */
+int gpt_optim_init(const gpt_config* cfg, const void* params, void* state, void* stream);
+/* One optimizer step: updates state and params in place from grads (the
+ * gradient buffer gpt_backward writes).  Uses the workspace's optimizer
+ * scratch; async on `stream`, deterministic.  GPT_EINVAL for NULL or
+ * misaligned pointers, ns_steps outside 0..8, step < 1, betas outside [0, 1)
+ * or non-finite hyper-parameters. */
+int gpt_optim_step(const gpt_config* cfg, const gpt_optim* opt, void* params, const void* grads,
+                   void* state, void* workspace, void* stream);
 
 /* ---- tracing (optional; per-launch CUDA events) ------------------------------
  * A trace records a CUDA event pair around every kernel launch that

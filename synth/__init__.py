@@ -179,3 +179,10 @@ def make_params(w: Workload, as_bits: bool = False) -> Dict[str, np.ndarray]:
         else:
             raise ValueError(w.dtype)
     return params
+
+def random_bf16_bits(shape, seed: int, scale: float) -> np.ndarray:
+    """Seeded N(0, scale^2) values rounded to bf16 (uint16 bit patterns): the
+    synthetic gradients fed to the optimizer step."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    x = rng.standard_normal(shape, dtype=np.float32) * np.float32(scale)
+    return f64_to_bf16_bits(x)

@@ -156,3 +156,34 @@ def test_pack_unpack_roundtrip(B):
     back = B.unpack_flat(c, flat)
     for k in p:
         assert np.array_equal(back[k], p[k])
+
+
+# ---- optimizer step: argument checks (host side, no CUDA call is reached) ----
+def test_optim_defaults_and_state_bytes():
+    from decoder_only_gpt_b200 import binding as B
+    o = B.optim_defaults()
+    assert o.ns_steps == 2 and o.step == 1 and o.muon_nesterov == 1
+    assert o.coeffs() == [(np.float32(8.156), np.float32(-22.483), np.float32(15.879)),
+                          (np.float32(4.043), np.float32(-2.809), np.float32(0.5))]
+    cfg = B.config_from_workload(synth.workload("story"))
+    assert B.optim_state_bytes(cfg) == 3 * (cfg.param_bytes // 2) * 4
+
+
+def test_optim_rejects():
+    from decoder_only_gpt_b200 import binding as B
+    cfg = B.config_from_workload(synth.workload("story"))
+    o = B.optim_defaults()
+    fake = 1 << 40  # 256-aligned, never dereferenced: every case fails before any launch
+    assert B.raw_optim_step(cfg, None, fake, fake, fake, fake) == B.GPT_EINVAL
+    assert B.raw_optim_step(cfg, o, None, fake, fake, fake) == B.GPT_EINVAL
+    assert B.raw_optim_step(cfg, o, fake + 16, fake, fake, fake) == B.GPT_EINVAL
+    for field, bad in (("ns_steps", 9), ("ns_steps", -1), ("step", 0), ("adam_beta1", 1.0),
+                       ("adam_beta2", -0.5), ("muon_lr", float("nan")), ("muon_nesterov", 2)):
+        o2 = B.optim_defaults()
+        setattr(o2, field, bad)
+        assert B.raw_optim_step(cfg, o2, fake, fake, fake, fake) == B.GPT_EINVAL, field
+    o3 = B.optim_defaults()
+    o3.ns_coeffs[1][2] = float("inf")
+    assert B.raw_optim_step(cfg, o3, fake, fake, fake, fake) == B.GPT_EINVAL
+    tiny = B.config_from_workload(synth.workload("tiny"))  # fp32 storage
+    assert B.raw_optim_step(tiny, o, fake, fake, fake, fake) == B.GPT_EUNSUPPORTED
