@@ -93,10 +93,12 @@ def lib() -> ctypes.CDLL:
         L.gpt_optim_state_bytes.argtypes = [cfgp, ctypes.POINTER(ctypes.c_size_t)]
         L.gpt_optim_init.argtypes = [cfgp, P, P, P]
         L.gpt_optim_step.argtypes = [cfgp, optp, P, P, P, P, P]
+        L.gpt_wait_expiry_check.argtypes = [P, ctypes.c_int64, P]
         for f in ("gpt_config_init", "gpt_config_from_depth", "gpt_param_offset",
                   "gpt_workspace_region", "gpt_forward_loss", "gpt_backward",
                   "gpt_train_step_host", "gpt_status", "gpt_optim_defaults",
-                  "gpt_optim_state_bytes", "gpt_optim_init", "gpt_optim_step"):
+                  "gpt_optim_state_bytes", "gpt_optim_init", "gpt_optim_step",
+                  "gpt_wait_expiry_check"):
             getattr(L, f).restype = I
         _lib = L
     return _lib
@@ -313,3 +315,9 @@ def raw_optim_step(cfg, opt, params, grads, state, workspace, stream=None) -> in
 
 def optim_step(cfg, opt, params, grads, state, workspace, stream=None):
     _check(raw_optim_step(cfg, opt, params, grads, state, workspace, stream), "gpt_optim_step")
+
+
+def wait_expiry_check(workspace, limit_ns: int, stream=None) -> int:
+    """Launch the bounded-wait expiry check; returns the launch code (the
+    expiry itself is read with status())."""
+    return lib().gpt_wait_expiry_check(_ptr(workspace), int(limit_ns), stream)

@@ -558,6 +558,12 @@ int gpt_status(const void* workspace, void* stream) {
   return s.code;
 }
 
+int gpt_wait_expiry_check(void* workspace, int64_t limit_ns, void* stream) {
+  if (!workspace || !aligned(workspace, 256)) return GPT_EINVAL;
+  if (limit_ns < 1000 || limit_ns > 10000000000ll) return GPT_EINVAL;
+  return launch_wait_expiry(static_cast<int32_t*>(workspace), uint64_t(limit_ns), stream) ? GPT_ECUDA
+                                                                                         : GPT_OK;
+}
 
 // ---------------------------------------------------------------------------
 // optimizer step ("ChatGPT'nizi 50 Dolara Nasil Egitirsiniz?", section "2. Muon

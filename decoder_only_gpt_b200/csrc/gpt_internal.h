@@ -16,6 +16,7 @@ enum KernelId : int32_t {
   K_GEMM_TC = 3,
   K_ATTN = 4,
   K_LOSS = 5,
+  K_WAITCHECK = 6,
 };
 
 // Epilogues of the GEMM C[m,n] = sum_k A(m,k) B(n,k).
@@ -101,6 +102,9 @@ struct Layout {
 };
 
 bool make_layout(const gpt_config& c, Layout* L);
+
+// ---- bounded-wait expiry check (csrc/waitcheck.cu) ----
+int launch_wait_expiry(int32_t* status, uint64_t limit_ns, void* stream);
 
 // ---- optimizer (csrc/optim.cu) ----
 constexpr int kOptNormBlocks = 296;  // fixed grid of the deterministic sum of squares

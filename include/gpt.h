@@ -198,6 +198,16 @@ int gpt_embedding_grad_noalloc(const int32_t* tokens, int64_t n_tokens, int32_t 
                                int32_t d_model, int32_t dtype, const float* dx0, void* dwte,
                                int accumulate, void* stream);
 
+/* Failure-path check (no counterpart on the pages): launches one kernel whose
+ * single thread waits on a barrier that nothing arrives at, with the same
+ * bounded wait (%globaltimer limit) that every pipeline kernel uses, here
+ * limit_ns (1e3 .. 1e10) instead of 2 s.  When it expires the kernel records
+ * GPT_ETIMEOUT in the workspace's status word (read with gpt_status) and
+ * returns; nothing faults, traps or hangs, and the context stays usable.  The
+ * next gpt_forward_loss clears the status word.  GPT_EINVAL for a NULL or
+ * non-256-byte-aligned workspace or a limit out of range. */
+int gpt_wait_expiry_check(void* workspace, int64_t limit_ns, void* stream);
+
 /* ---- optimizer step ------------------------------------------------------------
  * "ChatGPT'nizi 50 Dolara Nasil Egitirsiniz?" (dev.to), section "2. Muon
  * Optimize Edici (nanochat/optim.py)": the embedding (wte) and lm_head are

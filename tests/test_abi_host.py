@@ -187,3 +187,12 @@ def test_optim_rejects():
     assert B.raw_optim_step(cfg, o3, fake, fake, fake, fake) == B.GPT_EINVAL
     tiny = B.config_from_workload(synth.workload("tiny"))  # fp32 storage
     assert B.raw_optim_step(tiny, o, fake, fake, fake, fake) == B.GPT_EUNSUPPORTED
+
+
+def test_wait_expiry_check_rejects():
+    from decoder_only_gpt_b200 import binding as B
+    fake = 1 << 40  # 256-aligned, never dereferenced: every case fails before any launch
+    assert B.wait_expiry_check(None, 20_000_000) == B.GPT_EINVAL
+    assert B.wait_expiry_check(fake + 16, 20_000_000) == B.GPT_EINVAL
+    assert B.wait_expiry_check(fake, 10) == B.GPT_EINVAL
+    assert B.wait_expiry_check(fake, 10**11) == B.GPT_EINVAL
