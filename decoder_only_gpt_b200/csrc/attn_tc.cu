@@ -35,6 +35,33 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
 }
+// Packed fp32 pairs (sm_100 f32x2 arithmetic: two IEEE fp32 operations per
+// instruction, results identical to the scalar ones).
+__device__ __forceinline__ uint64_t f2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float2 unf2(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -349,16 +376,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // P_j into registers first: this overlaps P_{j-1} V_{j-1}, which must
         // finish before O is rescaled and before the P tile is rewritten
-        float lsum = 0.f;
+        uint64_t lsum2 = f2(0.f, 0.f);
+        const uint64_t sc2 = f2(scale_log2, scale_log2), nm2 = f2(-m_ref, -m_ref);
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float p0 = ex2(fmaf(s[2 * i], scale_log2, -m_ref));
-          const float p1 = ex2(fmaf(s[2 * i + 1], scale_log2, -m_ref));
-          lsum += p0 + p1;
+          const float2 x = unf2(fma2(f2(s[2 * i], s[2 * i + 1]), sc2, nm2));
+          const float p0 = ex2(x.x), p1 = ex2(x.y);
+          lsum2 = add2(lsum2, f2(p0, p1));
           pk[i] = pack2(p0, p1);
         }
-        l_half += lsum;
+        const float2 ls = unf2(lsum2);
+        l_half += ls.x + ls.y;
         if (j > 0) {
           ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->pv_full, (j - 1) & 1, abort, kWaitNs));
           if (ok) tc::tc_fence_after();
@@ -812,16 +841,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::tmem_wait_ld();
         const bool need_mask = !qv || k0 + 32 > q || k0 + 32 > T;
         uint32_t pk[16];
+        const uint64_t sc2 = f2(scale_log2, scale_log2), nl2 = f2(-lse2, -lse2), nd2 = f2(-Dq, -Dq);
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int i = 2 * e;
-          float p0 = ex2(fmaf(__uint_as_float(us[i]), scale_log2, -lse2));
-          float p1 = ex2(fmaf(__uint_as_float(us[i + 1]), scale_log2, -lse2));
+          const float2 x = unf2(fma2(f2(__uint_as_float(us[i]), __uint_as_float(us[i + 1])), sc2, nl2));
+          float p0 = ex2(x.x), p1 = ex2(x.y);
           if (need_mask) {
             if (k0 + i > q || k0 + i >= T || !qv) p0 = 0.f;
             if (k0 + i + 1 > q || k0 + i + 1 >= T || !qv) p1 = 0.f;
           }
-          pk[e] = pack2(p0 * (__uint_as_float(up[i]) - Dq), p1 * (__uint_as_float(up[i + 1]) - Dq));
+          const float2 r =
+              unf2(mul2(f2(p0, p1), add2(f2(__uint_as_float(up[i]), __uint_as_float(up[i + 1])), nd2)));
+          pk[e] = pack2(r.x, r.y);
         }
         tc::tmem_st_32x32b_x16(ts, pk);  // dS over this thread's own S columns
         tc::tmem_wait_st();
@@ -1057,14 +1089,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; e += 2) {
             const int i = 4 * g + e;
-            float p0 = ex2(fmaf(__uint_as_float(us[i]), scale_log2, -l2[e]));
-            float p1 = ex2(fmaf(__uint_as_float(us[i + 1]), scale_log2, -l2[e + 1]));
+            const float2 x = unf2(fma2(f2(__uint_as_float(us[i]), __uint_as_float(us[i + 1])),
+                                       f2(scale_log2, scale_log2), f2(-l2[e], -l2[e + 1])));
+            float p0 = ex2(x.x), p1 = ex2(x.y);
             if (need_mask) {
               if (qs + i < key || qs + i >= T || !kv) p0 = 0.f;
               if (qs + i + 1 < key || qs + i + 1 >= T || !kv) p1 = 0.f;
             }
             pp[i / 2] = pack2(p0, p1);
-            pd[i / 2] = pack2(p0 * (__uint_as_float(up[i]) - dd[e]), p1 * (__uint_as_float(up[i + 1]) - dd[e + 1]));
+            const float2 r = unf2(mul2(f2(p0, p1), add2(f2(__uint_as_float(up[i]), __uint_as_float(up[i + 1])),
+                                                          f2(-dd[e], -dd[e + 1]))));
+            pd[i / 2] = pack2(r.x, r.y);
           }
         }
         tc::tmem_st_32x32b_x16(ts, pp);           // P^T over this thread's S^T columns
