@@ -190,7 +190,7 @@ def gemm_sites(records, w, steps):
 
 # DRAM bytes (read + write) of one up-projection forward launch at the bench
 # workload, from an ncu capture of the current CTA-pair GEMM kernel.
-UP_FWD_TRAFFIC_BYTES = 121_126_656 + 361_852_160
+UP_FWD_TRAFFIC_BYTES = 121_366_016 + 360_246_272
 
 
 def roofline(sites, w, gemm_tf, peak_tf, peaks):

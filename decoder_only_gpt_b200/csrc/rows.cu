@@ -193,6 +193,10 @@ __global__ void rms_bwd_kernel(const T* __restrict__ dh, const T* __restrict__ h
   }
 }
 
+// bf16, d % 8 == 0, d <= 8 * 32 * KV: all of a row's loads (dh, h and, when
+// accumulating, the fp32 dx) are issued before the row reduction, so their
+// latencies overlap; KV = the 8-element groups per lane, sized to d.
+template <int KV>
 __global__ void rms_bwd_bf16_vec(const __nv_bfloat16* __restrict__ dh,
                                  const __nv_bfloat16* __restrict__ h, const float* __restrict__ r,
                                  float* __restrict__ dx, __nv_bfloat16* __restrict__ dxs,
@@ -203,14 +207,26 @@ __global__ void rms_bwd_bf16_vec(const __nv_bfloat16* __restrict__ dh,
   const int groups = d / 8;
   const uint4* dr = reinterpret_cast<const uint4*>(dh + row * d);
   const uint4* hr = reinterpret_cast<const uint4*>(h + row * d);
-  uint4 gd[kMaxVec], gh[kMaxVec];
-  float s = 0.f;
+  float4* xr = reinterpret_cast<float4*>(dx + row * d);
+  uint4 gd[KV], gh[KV];
+  float4 p0[KV], p1[KV];
 #pragma unroll
-  for (int k = 0; k < kMaxVec; ++k) {
+  for (int k = 0; k < KV; ++k) {
     const int gi = lane + 32 * k;
     if (gi < groups) {
       gd[k] = dr[gi];
       gh[k] = hr[gi];
+      if (accumulate) {
+        p0[k] = xr[2 * gi];
+        p1[k] = xr[2 * gi + 1];
+      }
+    }
+  }
+  float s = 0.f;
+#pragma unroll
+  for (int k = 0; k < KV; ++k) {
+    const int gi = lane + 32 * k;
+    if (gi < groups) {
       float fa[8], fb[8];
       up8(gd[k], fa);
       up8(gh[k], fb);
@@ -220,10 +236,9 @@ __global__ void rms_bwd_bf16_vec(const __nv_bfloat16* __restrict__ dh,
   }
   s = warp_sum(s) / float(d);
   const float rr = r[row];
-  float4* xr = reinterpret_cast<float4*>(dx + row * d);
   uint4* sr = reinterpret_cast<uint4*>(dxs + row * d);
 #pragma unroll
-  for (int k = 0; k < kMaxVec; ++k) {
+  for (int k = 0; k < KV; ++k) {
     const int gi = lane + 32 * k;
     if (gi < groups) {
       float fa[8], fb[8], g[8];
@@ -232,9 +247,8 @@ __global__ void rms_bwd_bf16_vec(const __nv_bfloat16* __restrict__ dh,
 #pragma unroll
       for (int e = 0; e < 8; ++e) g[e] = rr * (fa[e] - fb[e] * s);
       if (accumulate) {
-        const float4 p0 = xr[2 * gi], p1 = xr[2 * gi + 1];
-        g[0] += p0.x; g[1] += p0.y; g[2] += p0.z; g[3] += p0.w;
-        g[4] += p1.x; g[5] += p1.y; g[6] += p1.z; g[7] += p1.w;
+        g[0] += p0[k].x; g[1] += p0[k].y; g[2] += p0[k].z; g[3] += p0[k].w;
+        g[4] += p1[k].x; g[5] += p1[k].y; g[6] += p1[k].z; g[7] += p1[k].w;
       }
       xr[2 * gi] = make_float4(g[0], g[1], g[2], g[3]);
       xr[2 * gi + 1] = make_float4(g[4], g[5], g[6], g[7]);
@@ -248,11 +262,23 @@ int launch_rms_bwd(const gpt_config& c, const void* dh, const void* h, const flo
                    float* dx, void* dxs, int accumulate, void* stream) {
   int64_t N = int64_t(c.batch) * c.seq_len;
   dim3 grid(ceil_div(N, 8));
-  if (c.dtype == GPT_BF16 && c.d_model % 8 == 0 && c.d_model <= 8 * 32 * kMaxVec)
-    rms_bwd_bf16_vec<<<grid, 256, 0, (cudaStream_t)stream>>>(
-        (const __nv_bfloat16*)dh, (const __nv_bfloat16*)h, r, dx, (__nv_bfloat16*)dxs, N,
-        c.d_model, accumulate);
-  else if (c.dtype == GPT_BF16)
+  if (c.dtype == GPT_BF16 && c.d_model % 8 == 0 && c.d_model <= 8 * 32 * kMaxVec) {
+    const int kv = (c.d_model / 8 + 31) / 32;  // 8-element groups per lane
+    auto args = [&](auto kern) {
+      kern<<<grid, 256, 0, (cudaStream_t)stream>>>((const __nv_bfloat16*)dh, (const __nv_bfloat16*)h, r,
+                                                   dx, (__nv_bfloat16*)dxs, N, c.d_model, accumulate);
+    };
+    switch (kv) {
+      case 1: args(rms_bwd_bf16_vec<1>); break;
+      case 2: args(rms_bwd_bf16_vec<2>); break;
+      case 3: args(rms_bwd_bf16_vec<3>); break;
+      case 4: args(rms_bwd_bf16_vec<4>); break;
+      case 5: args(rms_bwd_bf16_vec<5>); break;
+      case 6: args(rms_bwd_bf16_vec<6>); break;
+      case 7: args(rms_bwd_bf16_vec<7>); break;
+      default: args(rms_bwd_bf16_vec<8>); break;
+    }
+  } else if (c.dtype == GPT_BF16)
     rms_bwd_kernel<__nv_bfloat16><<<grid, 256, 0, (cudaStream_t)stream>>>(
         (const __nv_bfloat16*)dh, (const __nv_bfloat16*)h, r, dx, (__nv_bfloat16*)dxs, N,
         c.d_model, accumulate);
