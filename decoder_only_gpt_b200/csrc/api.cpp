@@ -74,7 +74,23 @@ bool make_layout(const gpt_config& c, Layout* L) {
   L->lo.r2 = lb.take(N * 4);
   L->lo.a = lb.take(N * F * esz);
   L->layer_stride = align_up(lb.off, kAlign);
-  L->layer_base = b.take(L->layer_stride * uint64_t(c.n_layer));
+  // optimizer scratch (bf16), in the same bytes as the saved activations (dead
+  // once gpt_backward has run): for every layer, two Newton-Schulz iterates of
+  // the largest block matrix and two Gram matrices of the smaller side (d for
+  // every block matrix), so that one kind of matrix is orthogonalised for all
+  // layers at once
+  uint64_t opt_bytes = 0;
+  if (c.dtype == GPT_BF16) {
+    const int64_t mat = std::max(std::max(3 * d * d, F * d), d * d);
+    const int64_t gd = d;
+    Bump ob;
+    L->opt_x0 = ob.take(mat * 2 * c.n_layer);
+    L->opt_x1 = ob.take(mat * 2 * c.n_layer);
+    L->opt_a = ob.take(gd * gd * 2 * c.n_layer);
+    L->opt_b = ob.take(gd * gd * 2 * c.n_layer);
+    opt_bytes = ob.off;
+  }
+  L->layer_base = b.take(std::max(L->layer_stride * uint64_t(c.n_layer), opt_bytes));
   L->hf = b.take(N * d * esz);
   L->rf = b.take(N * 4);
   L->qkv_raw = b.take(c.dtype == GPT_F32 ? N * 3 * d * esz : 0);  // bf16: fused into the GEMM
@@ -105,16 +121,12 @@ bool make_layout(const gpt_config& c, Layout* L) {
   L->scat_items = b.take(L->scat_max_items * 8);
   L->scat_item_offs = b.take((V + 1) * 8);
   L->scat_partial = b.take((N / 64 + 1) * d * 4 * 2);
-  // optimizer scratch (bf16): two Newton-Schulz iterates of the largest block
-  // matrix, two Gram matrices of the smaller side (d for every block matrix),
-  // the sum-of-squares partials and the reciprocal norm
+  // Muon's sum-of-squares partials and reciprocal norm
   if (c.dtype == GPT_BF16) {
-    const int64_t mat = std::max(std::max(3 * d * d, F * d), d * d);
-    const int64_t gd = d;  // the smaller side of Wqkv, Wo, Wup and Wdown is at most d
-    L->opt_x0 = b.take(mat * 2);
-    L->opt_x1 = b.take(mat * 2);
-    L->opt_a = b.take(gd * gd * 2);
-    L->opt_b = b.take(gd * gd * 2);
+    L->opt_x0 += L->layer_base;
+    L->opt_x1 += L->layer_base;
+    L->opt_a += L->layer_base;
+    L->opt_b += L->layer_base;
     L->opt_part = b.take((kOptNormBlocks + 1) * 4);
   } else {
     L->opt_x0 = L->opt_x1 = L->opt_a = L->opt_b = L->opt_part = 0;
@@ -294,7 +306,8 @@ static int run_gemm(const gpt_config& c, const GemmArgs& g, cudaStream_t st) {
     case EPI_QKV: bytes += mn * e + double(g.M) * 2 * g.n_head * 4; break;
     default: bytes += mn * e; break;
   }
-  TraceScope ts(GPT_K_GEMM, gemm_kernel_count(c, g), 2.0 * double(g.M) * g.N * g.K, bytes, st);
+  TraceScope ts(GPT_K_GEMM, gemm_kernel_count(c, g), 2.0 * double(g.M) * g.N * g.K * g.batch,
+                bytes * g.batch, st);
   return launch_gemm(c, g, st);
 }
 
@@ -662,55 +675,83 @@ int gpt_optim_step(const gpt_config* c, const gpt_optim* o, void* params, const 
     GPT_TRY(launch_adamw(P + off, G + off, W + off, M + off, Vv + off, n, o->adam_lr, o->adam_beta1,
                          o->adam_beta2, o->adam_eps, o->adam_weight_decay, bc1, bc2, st));
   }
-  // Muon: every block matrix
-  void* x0 = ws + L.opt_x0;
-  void* x1 = ws + L.opt_x1;
-  void* A = ws + L.opt_a;
-  void* Bm = ws + L.opt_b;
+  // Muon: every block matrix.  One kind of matrix (same shape in every layer)
+  // is orthogonalised for all layers together: the momentum pass writes each
+  // layer's X into a stacked [n_layer, rows, cols] buffer and every
+  // Newton-Schulz product is one batched GEMM over the layers.
+  char* x0 = ws + L.opt_x0;
+  char* x1 = ws + L.opt_x1;
+  char* A = ws + L.opt_a;
+  char* Bm = ws + L.opt_b;
   float* part = reinterpret_cast<float*>(ws + L.opt_part);
-  for (int l = 0; l < c->n_layer; ++l) {
-    for (int tensor : {GPT_T_WQKV, GPT_T_WO, GPT_T_WUP, GPT_T_WDOWN}) {
-      int64_t off, r, cc;
-      gpt_param_offset(c, tensor, l, &off, &r, &cc);
-      const int64_t n = r * cc;
-      {
-        TraceScope ts(GPT_K_OTHER, 3, 0, double(n) * 16.0, st);
-        GPT_TRY(launch_muon_prepare(G + off, M + off, n, o->muon_momentum, o->muon_nesterov, part, x0,
-                                    st));
-      }
-      // Newton-Schulz on X [r, cc]; the Gram matrix is gd x gd over the smaller side
-      const bool tall = r >= cc;
-      const int gd = int(tall ? cc : r);
-      void* X = x0;
-      void* Xn = x1;
-      for (int i = 0; i < o->ns_steps; ++i) {
-        const float a = o->ns_coeffs[i][0], b = o->ns_coeffs[i][1], cf = o->ns_coeffs[i][2];
-        // A = X^T X (tall) or X X^T (wide)
-        GemmArgs g1 = tall ? gemm_kk(X, cc, X, cc, gd, gd, int(r), EPI_STORE, A, gd, status)
-                           : gemm_kk(X, cc, X, cc, gd, gd, int(cc), EPI_STORE, A, gd, status);
-        g1.a_mn_major = tall;
-        g1.b_mn_major = tall;
-        GPT_TRY(run_gemm(*c, with_splitk(g1, L, ws), st));
-        // B = c A A + b A
-        GemmArgs g2 = gemm_kk(A, gd, A, gd, gd, gd, gd, EPI_AXPBY, Bm, gd, status);
-        g2.b_mn_major = true;
-        g2.aux = A;
-        g2.alpha = cf;
-        g2.beta_aux = b;
-        GPT_TRY(run_gemm(*c, g2, st));
-        // X' = X B + a X (tall) or B X + a X (wide)
-        GemmArgs g3 = tall ? gemm_kk(X, cc, Bm, gd, int(r), int(cc), gd, EPI_AXPBY, Xn, cc, status)
-                           : gemm_kk(Bm, gd, X, cc, int(r), int(cc), gd, EPI_AXPBY, Xn, cc, status);
-        g3.b_mn_major = true;
-        g3.aux = X;
-        g3.alpha = 1.f;
-        g3.beta_aux = a;
-        GPT_TRY(run_gemm(*c, g3, st));
-        std::swap(X, Xn);
-      }
-      const float step = o->muon_lr * std::sqrt(std::max(1.f, float(r) / float(cc)));
+  const int nl = c->n_layer;
+  // one batched product; per-layer launches when a K block would straddle two
+  // layers' rows (K not a multiple of the 64-wide K block)
+  auto batched = [&](GemmArgs g, int64_t a_bs, int64_t b_bs, int64_t o_bs, bool split) -> int {
+    if (g.K % 64 == 0) {
+      g.batch = nl;
+      g.a_bstride = a_bs;
+      g.b_bstride = b_bs;
+      g.o_bstride = o_bs;
+      return run_gemm(*c, g, st);
+    }
+    for (int l = 0; l < nl; ++l) {
+      GemmArgs gl = g;
+      gl.A = static_cast<const __nv_bfloat16*>(g.A) + l * a_bs * g.lda;
+      gl.B = static_cast<const __nv_bfloat16*>(g.B) + l * b_bs * g.ldb;
+      gl.out = static_cast<__nv_bfloat16*>(g.out) + l * o_bs * g.ldo;
+      if (g.aux) gl.aux = static_cast<const __nv_bfloat16*>(g.aux) + l * o_bs * g.ldo;
+      const int rc = run_gemm(*c, split ? with_splitk(gl, L, ws) : gl, st);
+      if (rc) return rc;
+    }
+    return 0;
+  };
+  for (int tensor : {GPT_T_WQKV, GPT_T_WO, GPT_T_WUP, GPT_T_WDOWN}) {
+    int64_t off0, r, cc;
+    gpt_param_offset(c, tensor, 0, &off0, &r, &cc);
+    const int64_t n = r * cc;
+    for (int l = 0; l < nl; ++l) {
+      int64_t off, rr, rc2;
+      gpt_param_offset(c, tensor, l, &off, &rr, &rc2);
+      TraceScope ts(GPT_K_OTHER, 3, 0, double(n) * 16.0, st);
+      GPT_TRY(launch_muon_prepare(G + off, M + off, n, o->muon_momentum, o->muon_nesterov, part,
+                                  x0 + l * n * 2, st));
+    }
+    // Newton-Schulz on each X [r, cc]; the Gram matrix is gd x gd over the smaller side
+    const bool tall = r >= cc;
+    const int gd = int(tall ? cc : r);
+    char* X = x0;
+    char* Xn = x1;
+    for (int i = 0; i < o->ns_steps; ++i) {
+      const float a = o->ns_coeffs[i][0], b = o->ns_coeffs[i][1], cf = o->ns_coeffs[i][2];
+      // A = X^T X (tall: both operands are X read MN-major) or X X^T (wide)
+      GemmArgs g1 = gemm_kk(X, cc, X, cc, gd, gd, int(tall ? r : cc), EPI_STORE, A, gd, status);
+      g1.a_mn_major = tall;
+      g1.b_mn_major = tall;
+      GPT_TRY(batched(g1, r, r, gd, true));
+      // B = c A A + b A
+      GemmArgs g2 = gemm_kk(A, gd, A, gd, gd, gd, gd, EPI_AXPBY, Bm, gd, status);
+      g2.b_mn_major = true;
+      g2.aux = A;
+      g2.alpha = cf;
+      g2.beta_aux = b;
+      GPT_TRY(batched(g2, gd, gd, gd, false));
+      // X' = X B + a X (tall) or B X + a X (wide)
+      GemmArgs g3 = tall ? gemm_kk(X, cc, Bm, gd, int(r), int(cc), gd, EPI_AXPBY, Xn, cc, status)
+                         : gemm_kk(Bm, gd, X, cc, int(r), int(cc), gd, EPI_AXPBY, Xn, cc, status);
+      g3.b_mn_major = true;
+      g3.aux = X;
+      g3.alpha = 1.f;
+      g3.beta_aux = a;
+      GPT_TRY(batched(g3, tall ? r : gd, tall ? gd : r, r, false));
+      std::swap(X, Xn);
+    }
+    const float step = o->muon_lr * std::sqrt(std::max(1.f, float(r) / float(cc)));
+    for (int l = 0; l < nl; ++l) {
+      int64_t off, rr, rc2;
+      gpt_param_offset(c, tensor, l, &off, &rr, &rc2);
       TraceScope ts(GPT_K_OTHER, 1, 0, double(n) * 12.0, st);
-      GPT_TRY(launch_muon_apply(X, W + off, P + off, n, step, st));
+      GPT_TRY(launch_muon_apply(X + l * n * 2, W + off, P + off, n, step, st));
     }
   }
   return GPT_OK;

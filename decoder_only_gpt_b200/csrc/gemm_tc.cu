@@ -309,7 +309,7 @@ __device__ __forceinline__ float4* stage_at(float* tile, int r, int u) {
 // Partial-column fallback (col + 4 > N, or a row pitch that is not a multiple
 // of 4): the same element-wise epilogue, one element at a time.
 __device__ __noinline__ void epi4_scalar(const GemmArgs& g, int row, int col, float4 a, int sp,
-                                         int splits, int tgt, float lse_row) {
+                                         int splits, int tgt, float lse_row, int64_t obase) {
   const int nc = min(4, g.N - col);
   const float v[4] = {a.x, a.y, a.z, a.w};
   for (int j = 0; j < nc; ++j) {
@@ -318,7 +318,7 @@ __device__ __noinline__ void epi4_scalar(const GemmArgs& g, int row, int col, fl
       g.splitk[(int64_t(sp) * g.M + row) * g.N + n] = v[j];
       continue;
     }
-    const int64_t e = int64_t(row) * g.ldo + n;
+    const int64_t e = obase + int64_t(row) * g.ldo + n;
     if (g.epi == EPI_RESID_F32) { static_cast<float*>(g.out)[e] += v[j]; continue; }
     if (g.epi == EPI_STORE_F32) { static_cast<float*>(g.out)[e] = v[j]; continue; }
     __nv_bfloat16* o = static_cast<__nv_bfloat16*>(g.out);
@@ -344,7 +344,7 @@ __device__ __noinline__ void epi4_scalar(const GemmArgs& g, int row, int col, fl
 template <int KIND>
 __device__ __forceinline__ void epi_chunk_coalesced(const GemmArgs& g, float* tile, int wrow0, int col,
                                                     int rsub, int u4, int sp, int splits, int tgt,
-                                                    float lse_row) {
+                                                    float lse_row, int64_t obase) {
   float4 a[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) a[i] = *stage_at(tile, 4 * i + rsub, u4);
@@ -365,7 +365,7 @@ __device__ __forceinline__ void epi_chunk_coalesced(const GemmArgs& g, float* ti
     for (int i = 0; i < 8; ++i)
       if (wrow0 + 4 * i + rsub < g.M)
         epi4_scalar(g, wrow0 + 4 * i + rsub, col, a[i], sp, splits, KIND == EPI_CE_BWD ? t[i] : -1,
-                    KIND == EPI_CE_BWD ? ls[i] : 0.f);
+                    KIND == EPI_CE_BWD ? ls[i] : 0.f, obase);
     return;
   }
   bool ok[8];
@@ -374,7 +374,7 @@ __device__ __forceinline__ void epi_chunk_coalesced(const GemmArgs& g, float* ti
   for (int i = 0; i < 8; ++i) {
     const int row = wrow0 + 4 * i + rsub;
     ok[i] = row < g.M;
-    e[i] = KIND == -1 ? (int64_t(sp) * g.M + row) * g.N + col : int64_t(row) * g.ldo + col;
+    e[i] = KIND == -1 ? (int64_t(sp) * g.M + row) * g.N + col : obase + int64_t(row) * g.ldo + col;
   }
   if (KIND == -1 || KIND == EPI_STORE_F32 || KIND == EPI_RESID_F32) {
     float* o = KIND == -1 ? g.splitk : static_cast<float*>(g.out);
@@ -430,7 +430,7 @@ __device__ __forceinline__ void epi_chunk_coalesced(const GemmArgs& g, float* ti
 // of `splits`; `part` indexes this column block's cross-entropy partials.
 __device__ __forceinline__ void epilogue_tile(const GemmArgs& g, uint32_t taddr, int row0,
                                               int col_base, int part, int sp, int splits,
-                                              int quarter, int lane, float* tile) {
+                                              int quarter, int lane, float* tile, int64_t obase) {
   const int row = row0 + quarter * 32 + lane;
   const bool row_ok = row < g.M;
   int tgt = -1;
@@ -477,15 +477,15 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& g, uint32_t taddr,
       __syncwarp();
       const int col = col_base + c * 32 + 4 * u4;
       if (splits > 1) {
-        epi_chunk_coalesced<-1>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row);
+        epi_chunk_coalesced<-1>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row, obase);
       } else {
         switch (g.epi) {
-          case EPI_RESID_F32: epi_chunk_coalesced<EPI_RESID_F32>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row); break;
-          case EPI_STORE_F32: epi_chunk_coalesced<EPI_STORE_F32>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row); break;
-          case EPI_RELU2: epi_chunk_coalesced<EPI_RELU2>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row); break;
-          case EPI_DRELU2: epi_chunk_coalesced<EPI_DRELU2>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row); break;
-          case EPI_AXPBY: epi_chunk_coalesced<EPI_AXPBY>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row); break;
-          default: epi_chunk_coalesced<EPI_STORE>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row); break;
+          case EPI_RESID_F32: epi_chunk_coalesced<EPI_RESID_F32>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row, obase); break;
+          case EPI_STORE_F32: epi_chunk_coalesced<EPI_STORE_F32>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row, obase); break;
+          case EPI_RELU2: epi_chunk_coalesced<EPI_RELU2>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row, obase); break;
+          case EPI_DRELU2: epi_chunk_coalesced<EPI_DRELU2>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row, obase); break;
+          case EPI_AXPBY: epi_chunk_coalesced<EPI_AXPBY>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row, obase); break;
+          default: epi_chunk_coalesced<EPI_STORE>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row, obase); break;
         }
       }
       __syncwarp();
@@ -542,7 +542,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
   const int m_tiles = (g.M + P_BM - 1) / P_BM, n_tiles = (g.N + BN - 1) / BN;
-  const int num_units = m_tiles * n_tiles * splits;
+  const int mn_tiles = m_tiles * n_tiles;  // per product; `g.batch` products
+  const int num_units = mn_tiles * g.batch * splits;
   const int num_kb = (g.K + BK - 1) / BK;
   const int kb_per = (num_kb + splits - 1) / splits;
   constexpr uint32_t idesc = tc::idesc_bf16_f32(P_BM, BN, AMN, BMN);
@@ -581,8 +582,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       for (int unit = pair; unit < num_units && !*abort; unit += num_pairs) {
         const int tile = unit / splits, sp = unit % splits;
-        const int mb = tile / n_tiles, nb = tile % n_tiles;
+        const int bi = tile / mn_tiles, mb = (tile % mn_tiles) / n_tiles, nb = tile % n_tiles;
         const int m0 = mb * P_BM + int(rank) * 128, n0 = nb * BN + int(rank) * 128;
+        const int ay = int(bi * g.a_bstride), by = int(bi * g.b_bstride);  // batch row offsets
         const int kb_hi = min(num_kb, (sp + 1) * kb_per);
         for (int kb = sp * kb_per; kb < kb_hi; ++kb) {
           if (!tc::mbar_wait_bounded(&tail->empty[stage], phase ^ 1, abort, kWaitLimitNs)) {
@@ -595,16 +597,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           uint8_t* a_dst = smA + stage * P_HALF;
           uint8_t* b_dst = smB + stage * P_HALF;
           if (AMN) {
-            tc::tma_load_2d_pair(a_dst, &map_a, bar, m0, kb * BK);
-            tc::tma_load_2d_pair(a_dst + 8192, &map_a, bar, m0 + 64, kb * BK);
+            tc::tma_load_2d_pair(a_dst, &map_a, bar, m0, ay + kb * BK);
+            tc::tma_load_2d_pair(a_dst + 8192, &map_a, bar, m0 + 64, ay + kb * BK);
           } else {
-            tc::tma_load_2d_pair(a_dst, &map_a, bar, kb * BK, m0);
+            tc::tma_load_2d_pair(a_dst, &map_a, bar, kb * BK, ay + m0);
           }
           if (BMN) {
-            tc::tma_load_2d_pair(b_dst, &map_b, bar, n0, kb * BK);
-            tc::tma_load_2d_pair(b_dst + 8192, &map_b, bar, n0 + 64, kb * BK);
+            tc::tma_load_2d_pair(b_dst, &map_b, bar, n0, by + kb * BK);
+            tc::tma_load_2d_pair(b_dst + 8192, &map_b, bar, n0 + 64, by + kb * BK);
           } else {
-            tc::tma_load_2d_pair(b_dst, &map_b, bar, kb * BK, n0);
+            tc::tma_load_2d_pair(b_dst, &map_b, bar, kb * BK, by + n0);
           }
           if (++stage == P_STAGES) { stage = 0; phase ^= 1; }
         }
@@ -667,7 +669,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     float* stage_tile = reinterpret_cast<float*>(smem + 2 * P_STAGES * P_HALF + kPairTailBytes +
                                                  (warp - 2) * kStageBytes);
     const int my_row = int(rank) * 128 + quarter * 32 + lane;  // within a 256-row pair tile
-    if (pair < num_units)
+    if (pair < num_units && g.batch == 1)
       epilogue_prefetch(g, (pair / splits / n_tiles) * P_BM + my_row,
                         ((pair / splits) % n_tiles) * BN + ch * EC, splits);
     int local = 0;
@@ -677,7 +679,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const uint32_t acc_phase = (local >> 1) & 1;
       // one tile ahead: the rows of the next unit
       const int next = unit + num_pairs;
-      if (next < num_units)
+      if (next < num_units && g.batch == 1)
         epilogue_prefetch(g, (next / splits / n_tiles) * P_BM + my_row,
                           ((next / splits) % n_tiles) * BN + ch * EC, splits);
       const bool ok = tc::mbar_wait_bounded(&tail->tmem_full[acc], acc_phase, abort, kWaitLimitNs);
@@ -687,10 +689,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         break;
       }
       tc::tc_fence_after();
-      const int nb = tile % n_tiles;
+      const int bi = tile / mn_tiles, nb = tile % n_tiles;
       epilogue_tile(g, tmem_base + (uint32_t(quarter * 32) << 16) + acc * BN + ch * EC,
-                    (tile / n_tiles) * P_BM + int(rank) * 128, nb * BN + ch * EC, nb * (BN / EC) + ch, sp,
-                    splits, quarter, lane, stage_tile);
+                    ((tile % mn_tiles) / n_tiles) * P_BM + int(rank) * 128, nb * BN + ch * EC,
+                    nb * (BN / EC) + ch, sp, splits, quarter, lane, stage_tile,
+                    int64_t(bi) * g.o_bstride * g.ldo);
       tc::tc_fence_before();
       tc::mbar_arrive_cluster(tc::mapa_shared(tc::smem_u32(&tail->tmem_empty[acc]), 0));
     }
@@ -743,10 +746,12 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
 template <bool AMN, bool BMN>
 int launch_pair(const GemmArgs& g, int grid, int splits, cudaStream_t st) {
   CUtensorMap ma, mb;
-  bool ok = AMN ? make_map(&ma, g.A, g.M, g.K, g.lda, 64, 64)
-                : make_map(&ma, g.A, g.K, g.M, g.lda, 64, 128);
-  ok = ok && (BMN ? make_map(&mb, g.B, g.N, g.K, g.ldb, 64, 64)
-                  : make_map(&mb, g.B, g.K, g.N, g.ldb, 64, 128));
+  // batched products: the maps span every product's rows of the stacked arrays
+  const uint64_t a_extra = uint64_t(g.batch - 1) * g.a_bstride, b_extra = uint64_t(g.batch - 1) * g.b_bstride;
+  bool ok = AMN ? make_map(&ma, g.A, g.M, g.K + a_extra, g.lda, 64, 64)
+                : make_map(&ma, g.A, g.K, g.M + a_extra, g.lda, 64, 128);
+  ok = ok && (BMN ? make_map(&mb, g.B, g.N, g.K + b_extra, g.ldb, 64, 64)
+                  : make_map(&mb, g.B, g.K, g.N + b_extra, g.ldb, 64, 128));
   if (!ok) return 1;
   auto kern = gemm_pair_kernel<AMN, BMN>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kPairSmemBytes)) !=
@@ -789,7 +794,7 @@ int num_sms() {
 // idle; the smallest split count that fills >= 90 % of the waves, keeping >= 8
 // k-blocks per split and the partials within the buffer.
 int gemm_tc_splits(const GemmArgs& g) {
-  if (g.epi != EPI_STORE || !g.splitk || g.ldo != g.N || (g.N & 3)) return 1;
+  if (g.epi != EPI_STORE || !g.splitk || g.ldo != g.N || (g.N & 3) || g.batch != 1) return 1;
   const int pairs = num_sms() / 2;
   const int tiles = ((g.M + P_BM - 1) / P_BM) * ((g.N + BN - 1) / BN);
   const int num_kb = (g.K + BK - 1) / BK;
@@ -814,8 +819,16 @@ int gemm_tc_splits(const GemmArgs& g) {
 int launch_gemm_tc(const GemmArgs& g_in, void* stream) {
   GemmArgs g = g_in;
   cudaStream_t st = (cudaStream_t)stream;
-  if (g.M <= 0 || g.N <= 0 || g.K <= 0) return 0;
-  const int tiles = ((g.M + P_BM - 1) / P_BM) * ((g.N + BN - 1) / BN);
+  if (g.M <= 0 || g.N <= 0 || g.K <= 0 || g.batch <= 0) return 0;
+  if (g.batch > 1) {
+    // a partial K block would read the next product's rows; the other
+    // epilogues are not batched
+    if (g.K % BK || !((g.epi == EPI_STORE && !g.beta) || g.epi == EPI_AXPBY)) return 1;
+    if (int64_t(g.batch) * std::max(g.a_bstride, g.b_bstride) + std::max(g.M, std::max(g.N, g.K)) >
+        (int64_t(1) << 31))
+      return 1;
+  }
+  const int tiles = ((g.M + P_BM - 1) / P_BM) * ((g.N + BN - 1) / BN) * g.batch;
   if (g.epi == EPI_CE_FWD) g.n_part = (g.N + EC - 1) / EC;
   const int splits = gemm_tc_splits(g);
   const int pairs = num_sms() / 2;

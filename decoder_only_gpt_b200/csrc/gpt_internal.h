@@ -66,6 +66,12 @@ struct GemmArgs {
   const float* rope_sin;    // [T, hd/2]
   int seq_len, n_head, head_dim, qk_norm;
   float norm_eps;
+  // batched products (tensor-core GEMM; EPI_STORE without beta or EPI_AXPBY,
+  // K a multiple of 64): product b reads A and B `a_bstride` / `b_bstride` rows
+  // further down their stored arrays and writes out (and reads aux) `o_bstride`
+  // rows further down
+  int batch = 1;
+  int64_t a_bstride = 0, b_bstride = 0, o_bstride = 0;
   // split-K (tensor-core GEMM, EPI_STORE only): fp32 partials [splits][M][N]
   float* splitk;
   int64_t splitk_floats;    // capacity of `splitk`

@@ -255,8 +255,11 @@ int gpt_optim_state_bytes(const gpt_config* cfg, size_t* bytes);
 /* master = params (exact upcast), m = v = 0.  Async on `stream`. */
 int gpt_optim_init(const gpt_config* cfg, const void* params, void* state, void* stream);
 /* One optimizer step: updates state and params in place from grads (the
- * gradient buffer gpt_backward writes).  Uses the workspace's optimizer
- * scratch; async on `stream`, deterministic.  GPT_EINVAL for NULL or
+ * gradient buffer gpt_backward writes).  Its scratch (every layer's
+ * Newton-Schulz iterates, stacked so that each product is one batched GEMM
+ * over the layers) overwrites the layers' saved activations in the workspace:
+ * a gpt_backward after it needs a new gpt_forward_loss first, as the new
+ * parameters do anyway.  Async on `stream`, deterministic.  GPT_EINVAL for NULL or
  * misaligned pointers, ns_steps outside 0..8, step < 1, betas outside [0, 1)
  * or non-finite hyper-parameters. */
 int gpt_optim_step(const gpt_config* cfg, const gpt_optim* opt, void* params, const void* grads,
