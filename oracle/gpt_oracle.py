@@ -10,9 +10,10 @@ What is computed, and where it comes from
 -----------------------------------------
 "ChatGPT'nizi 50 Dolara Nasil Egitirsiniz?" (dev.to), section "1. GPT Modeli
 (nanochat/gpt.py)", lists the model's ingredients: rotary embeddings, QK
-normalisation, untied embedding and output weights, the ReLU^2 activation
-(plus GQA, sliding windows and Flash Attention 3, which change nothing in
-exact arithmetic for the full-causal, n_kv = n_head shapes used here).
+normalisation, untied embedding and output weights, the ReLU^2 activation,
+grouped-query attention (GQA) and sliding-window attention (Flash Attention 3
+is how the page runs the attention, which changes nothing in exact
+arithmetic).
 Section "3. Hassasiyet Yonetimi (nanochat/common.py)" shows every linear layer
 as ``F.linear(x, W)`` with W stored [out, in] and no bias.  Section "5. Flash
 Dikkat Mekanizmasi Birlesimi" calls the attention with ``causal=True``.  The
@@ -30,12 +31,19 @@ Where the pages are silent the plainest reading is taken:
   applied after RoPE (a rotation keeps the norm, so the order does not change
   the result in exact arithmetic);
 * attention scale 1/sqrt(hd), no dropout, no soft-capping;
+* GQA: ``n_kv_head`` key/value heads shared by ``n_head / n_kv_head``
+  consecutive query heads (query head h reads key/value head
+  h // (n_head / n_kv_head)); 0 or n_head is ordinary multi-head attention;
+* sliding window: section "5. Flash Dikkat Mekanizmasi Birlesimi" passes a
+  ``window_size`` to the causal attention call; with ``window`` = W >= 1 query
+  i sees keys j with i - W < j <= i (its W most recent positions, itself
+  included), in every layer; 0 is the full causal window;
 * MLP u = h W_up^T, a = max(u, 0)^2, y = a W_down^T (not gated);
 * loss = mean over all B*T positions of logsumexp(z) - z[target].
 
 Layout conventions shared with the library's documented ABI (not its code):
-W_qkv is [3d, d] with the q rows first, then k, then v; inside each block head
-h owns rows [h*hd, (h+1)*hd).
+W_qkv is [(n_head + 2 n_kv_head) hd, d] with the q rows first, then k, then v
+([3d, d] without GQA); inside each block head h owns rows [h*hd, (h+1)*hd).
 
 The backward pass is derived by hand from the forward above; each step names
 the forward step it inverts.
@@ -56,6 +64,7 @@ __all__ = [
     "rope_tables",
     "rope",
     "rope_backward",
+    "attention_mask",
     "causal_attention",
     "causal_attention_backward",
     "cross_entropy",
@@ -79,13 +88,20 @@ class OracleConfig:
     norm_eps: float = 1e-6
     rope_base: float = 10000.0
     qk_norm: bool = True
+    n_kv_head: int = 0   # 0: n_head (multi-head attention)
+    window: int = 0      # 0: full causal window
+
+    @property
+    def kv_heads(self) -> int:
+        return self.n_kv_head or self.n_head
 
 
 def from_workload(w) -> OracleConfig:
     return OracleConfig(
         n_layer=w.n_layer, d_model=w.d_model, n_head=w.n_head, head_dim=w.head_dim,
         d_ff=w.d_ff, vocab=w.vocab, seq_len=w.seq_len, batch=w.batch,
-        norm_eps=w.norm_eps, rope_base=w.rope_base, qk_norm=w.qk_norm)
+        norm_eps=w.norm_eps, rope_base=w.rope_base, qk_norm=w.qk_norm,
+        n_kv_head=getattr(w, "n_kv_head", 0), window=getattr(w, "window", 0))
 
 
 # ---------------------------------------------------------------------------
@@ -139,26 +155,44 @@ def _heads_first(x: np.ndarray) -> np.ndarray:
     return np.ascontiguousarray(x.transpose(1, 0, 2))
 
 
-def _causal_probs(q: np.ndarray, k: np.ndarray):
+def attention_mask(T: int, window: int = 0) -> np.ndarray:
+    """[T, T] bool, True where query i may attend to key j: j <= i, and
+    i - j < window when a window is set (window >= 1)."""
+    i = np.arange(T)[:, None]
+    j = np.arange(T)[None, :]
+    visible = j <= i
+    if window > 0:
+        visible &= (i - j) < window
+    return visible
+
+
+def _per_query_head(x: np.ndarray, n_head: int) -> np.ndarray:
+    """[T, Hkv, hd] key/value heads -> [T, n_head, hd]: query head h uses
+    key/value head h // (n_head / Hkv)."""
+    return np.repeat(x, n_head // x.shape[1], axis=1)
+
+
+def _causal_probs(q: np.ndarray, k: np.ndarray, window: int):
     """Scores and probabilities for q, k [T, H, hd]; returns P [H, T, T] and lse [H, T]."""
     T, H, hd = q.shape
     s = (_heads_first(q) @ _heads_first(k).transpose(0, 2, 1)) / math.sqrt(hd)
-    future = np.triu(np.ones((T, T), dtype=bool), k=1)
-    s = np.where(future[None, :, :], -np.inf, s)
+    s = np.where(attention_mask(T, window)[None, :, :], s, -np.inf)
     m = np.max(s, axis=-1, keepdims=True)
     e = np.exp(s - m)
     tot = np.sum(e, axis=-1, keepdims=True)
     return e / tot, (m + np.log(tot))[..., 0]
 
 
-def causal_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray):
-    """softmax(q k^T / sqrt(hd) with j > i masked) v, per head.
+def causal_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, window: int = 0):
+    """softmax(q k^T / sqrt(hd), masked by ``attention_mask``) v, per query head.
 
-    q, k, v: [T, H, hd].  Returns o [T, H, hd], the probabilities P [H, T, T]
-    and the row log-sum-exp [H, T] of the scaled, masked scores.
+    q: [T, H, hd]; k, v: [T, Hkv, hd] with Hkv dividing H (GQA).  Returns
+    o [T, H, hd], the probabilities P [H, T, T] and the row log-sum-exp [H, T]
+    of the scaled, masked scores.
     """
-    p, lse = _causal_probs(q, k)
-    o = (p @ _heads_first(v)).transpose(1, 0, 2)
+    H = q.shape[1]
+    p, lse = _causal_probs(q, _per_query_head(k, H), window)
+    o = (p @ _heads_first(_per_query_head(v, H))).transpose(1, 0, 2)
     return o, p, lse
 
 
@@ -166,17 +200,22 @@ def causal_attention_backward(do, q, k, v, p):
     """Gradients of ``causal_attention`` w.r.t. q, k, v given dO and P.
 
     dV = P^T dO;  dP = dO V^T;  dS = P * (dP - rowsum(dP * P));
-    dQ = dS K / sqrt(hd);  dK = dS^T Q / sqrt(hd).
+    dQ = dS K / sqrt(hd);  dK = dS^T Q / sqrt(hd), per query head; a shared
+    key/value head (GQA) receives the sum over the query heads that read it.
+    The mask is already in P (masked entries are exactly 0).
     """
-    hd = q.shape[-1]
-    do_h, q_h, k_h, v_h = (_heads_first(t) for t in (do, q, k, v))
+    T, H, hd = q.shape
+    Hkv = k.shape[1]
+    do_h, q_h = _heads_first(do), _heads_first(q)
+    k_h, v_h = _heads_first(_per_query_head(k, H)), _heads_first(_per_query_head(v, H))
     dv = p.transpose(0, 2, 1) @ do_h
     dp = do_h @ v_h.transpose(0, 2, 1)
     ds = p * (dp - np.sum(dp * p, axis=-1, keepdims=True))
     dq = (ds @ k_h) / math.sqrt(hd)
     dk = (ds.transpose(0, 2, 1) @ q_h) / math.sqrt(hd)
     back = lambda t: t.transpose(1, 0, 2)
-    return back(dq), back(dk), back(dv)
+    group = lambda t: back(t).reshape(T, Hkv, H // Hkv, hd).sum(axis=2)
+    return back(dq), group(dk), group(dv)
 
 
 def cross_entropy(z: np.ndarray, y: np.ndarray):
@@ -206,7 +245,8 @@ def sequence_forward(cfg: OracleConfig, params: Dict[str, np.ndarray],
     (``token_loss``), the final logits' lse, and per-layer intermediates.
     """
     T = tok.shape[0]
-    d, H, hd = cfg.d_model, cfg.n_head, cfg.head_dim
+    d, H, hd, Hkv = cfg.d_model, cfg.n_head, cfg.head_dim, cfg.kv_heads
+    dkv = Hkv * hd
     eps = cfg.norm_eps
     cos, sin = rope_tables(T, hd, cfg.rope_base)
 
@@ -218,8 +258,8 @@ def sequence_forward(cfg: OracleConfig, params: Dict[str, np.ndarray],
         h, r1 = rms_norm(x, eps)                         # pre-attention norm
         qkv = h @ wqkv.T                                 # F.linear, no bias
         q = qkv[:, :d].reshape(T, H, hd)
-        k = qkv[:, d:2 * d].reshape(T, H, hd)
-        v = qkv[:, 2 * d:].reshape(T, H, hd)
+        k = qkv[:, d:d + dkv].reshape(T, Hkv, hd)
+        v = qkv[:, d + dkv:].reshape(T, Hkv, hd)
         q = rope(q, cos, sin)
         k = rope(k, cos, sin)
         if cfg.qk_norm:
@@ -227,7 +267,7 @@ def sequence_forward(cfg: OracleConfig, params: Dict[str, np.ndarray],
             kn, rk = rms_norm(k, eps)
         else:
             qn, rq, kn, rk = q, None, k, None
-        o, p, lse = causal_attention(qn, kn, v)
+        o, p, lse = causal_attention(qn, kn, v, cfg.window)
         o2 = o.reshape(T, d)
         x = x + o2 @ wo.T                                # attention residual
         h2, r2 = rms_norm(x, eps)                        # pre-MLP norm
@@ -251,7 +291,7 @@ def sequence_backward(cfg: OracleConfig, params: Dict[str, np.ndarray], cache: d
     """Accumulate d(scale * sum_t loss_t)/d(params) into ``grads``."""
     tok, tgt = cache["tok"], cache["tgt"]
     T = tok.shape[0]
-    d, H, hd = cfg.d_model, cfg.n_head, cfg.head_dim
+    d, H, hd, Hkv = cfg.d_model, cfg.n_head, cfg.head_dim, cfg.kv_heads
     cos, sin = cache["cos"], cache["sin"]
 
     g = cache["probs"].copy()                            # d loss / d z
@@ -274,7 +314,7 @@ def sequence_backward(cfg: OracleConfig, params: Dict[str, np.ndarray], cache: d
         # x_mid = x_in + o W_o^T
         grads[f"layers.{l}.wo"] += dx.T @ c["o"]
         do = (dx @ wo).reshape(T, H, hd)
-        _, p, _ = causal_attention(c["qn"], c["kn"], c["v"])
+        _, p, _ = causal_attention(c["qn"], c["kn"], c["v"], cfg.window)
         dqn, dkn, dv = causal_attention_backward(do, c["qn"], c["kn"], c["v"], p)
         if cfg.qk_norm:
             dq = rms_norm_backward(dqn, c["qn"], c["rq"])
@@ -283,7 +323,8 @@ def sequence_backward(cfg: OracleConfig, params: Dict[str, np.ndarray], cache: d
             dq, dk = dqn, dkn
         dq = rope_backward(dq, cos, sin)
         dk = rope_backward(dk, cos, sin)
-        dqkv = np.concatenate([dq.reshape(T, d), dk.reshape(T, d), dv.reshape(T, d)], axis=1)
+        dqkv = np.concatenate([dq.reshape(T, d), dk.reshape(T, Hkv * hd), dv.reshape(T, Hkv * hd)],
+                              axis=1)
         grads[f"layers.{l}.wqkv"] += dqkv.T @ c["h"]
         dh = dqkv @ wqkv
         dx = dx + rms_norm_backward(dh, c["h"], c["r1"])

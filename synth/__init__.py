@@ -58,6 +58,8 @@ class Workload:
     rope_base: float = 10000.0
     norm_eps: float = 1e-6
     qk_norm: bool = True
+    n_kv_head: int = 0  # key/value heads (GQA); 0 = n_head
+    window: int = 0     # sliding attention window in positions; 0 = full causal
 
     @property
     def n_tokens(self) -> int:
@@ -89,9 +91,10 @@ def workload(name: str, **overrides) -> Workload:
 def param_shapes(w: Workload) -> Iterator[Tuple[str, Tuple[int, int]]]:
     """Parameter names and [out, in] shapes, in generation order."""
     d, f, v = w.d_model, w.d_ff, w.vocab
+    qkv = d + 2 * (w.n_kv_head or w.n_head) * w.head_dim
     yield "wte", (v, d)
     for l in range(w.n_layer):
-        yield f"layers.{l}.wqkv", (3 * d, d)
+        yield f"layers.{l}.wqkv", (qkv, d)
         yield f"layers.{l}.wo", (d, d)
         yield f"layers.{l}.wup", (f, d)
         yield f"layers.{l}.wdown", (d, f)
