@@ -40,9 +40,16 @@ METRIC = "train tokens/sec (fwd+bwd) on 1 B200 for depth-12/24 GPT; MFU vs bf16 
 
 
 def flops_per_token(w) -> float:
-    """Algorithmic FLOPs per token, fwd+bwd = 3x fwd: 6*(12 L d^2 + V d) + 6 L T d (causal)."""
-    L, d, V, T = w.n_layer, w.d_model, w.vocab, w.seq_len
-    return 6.0 * (12 * L * d * d + V * d) + 6.0 * L * T * d
+    """Algorithmic FLOPs per token, fwd+bwd = 3x fwd: 6*(12 L d^2 + V d) + 6 L T d for the
+    plain model (causal: T/2 keys per query on average).  With grouped-query attention the
+    q/k/v projection has (d + 2 n_kv hd) d weights; with a sliding window W < T a query
+    sees (W T - W (W-1)/2) / T keys on average."""
+    L, d, V, T, F = w.n_layer, w.d_model, w.vocab, w.seq_len, w.d_ff
+    qkv = d + 2 * (w.n_kv_head or w.n_head) * w.head_dim
+    keys = T / 2
+    if w.window and w.window < T:
+        keys = (w.window * T - w.window * (w.window - 1) / 2) / T
+    return 6.0 * (L * (qkv * d + d * d + 2 * F * d) + V * d) + 12.0 * L * keys * d
 
 
 def load_peaks():
@@ -57,8 +64,13 @@ def load_peaks():
 
 
 def workload_desc(w):
+    extra = ""
+    if w.n_kv_head and w.n_kv_head != w.n_head:
+        extra += f", {w.n_kv_head} key/value heads"
+    if w.window:
+        extra += f", attention window {w.window}"
     return (f"{w.name}: {w.n_layer} layers, d_model {w.d_model}, {w.n_head}x{w.head_dim} heads, "
-            f"d_ff {w.d_ff}, vocab {w.vocab}, seq {w.seq_len}, batch {w.batch}")
+            f"d_ff {w.d_ff}, vocab {w.vocab}, seq {w.seq_len}, batch {w.batch}{extra}")
 
 
 # ---------------------------------------------------------------------------
@@ -289,6 +301,10 @@ def run_ours(args, rank, world, local_rank):
         w = w.replace(batch=args.batch)
     if args.layers is not None:
         w = w.replace(n_layer=args.layers)
+    if args.kv_heads:
+        w = w.replace(n_kv_head=args.kv_heads)
+    if args.window:
+        w = w.replace(window=args.window)
     wr = w.replace(seed=w.seed + 100 * rank)  # each replica its own batch
     cfg = B.config_from_workload(w)
     st = R.TrainStep(cfg, device=f"cuda:{local_rank}")
@@ -491,6 +507,11 @@ def main():
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (profiling captures on a smaller "
                          "case; the line then reports that batch)")
+    ap.add_argument("--kv-heads", type=int, default=0,
+                    help="grouped-query attention with this many key/value heads (a model "
+                         "variant; the line then reports it)")
+    ap.add_argument("--window", type=int, default=0,
+                    help="sliding attention window in positions (a model variant)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")

@@ -46,7 +46,7 @@ int cuda_rc(cudaError_t e) { return e == cudaSuccess ? GPT_OK : GPT_ECUDA; }
 bool make_layout(const gpt_config& c, Layout* L) {
   const int64_t N = int64_t(c.batch) * c.seq_len;
   const int64_t d = c.d_model, F = c.d_ff, V = c.vocab, H = c.n_head, T = c.seq_len,
-                B = c.batch, hd = c.head_dim;
+                B = c.batch, hd = c.head_dim, Hkv = c.n_kv_head, dkv = Hkv * hd, Q = qkv_cols(c);
   const int esz = c.dtype == GPT_BF16 ? 2 : 4;
   L->N = N;
   L->esz = esz;
@@ -64,10 +64,10 @@ bool make_layout(const gpt_config& c, Layout* L) {
   L->lo.h1 = lb.take(N * d * esz);
   L->lo.r1 = lb.take(N * 4);
   L->lo.q = lb.take(N * d * esz);
-  L->lo.k = lb.take(N * d * esz);
-  L->lo.v = lb.take(N * d * esz);
+  L->lo.k = lb.take(N * dkv * esz);
+  L->lo.v = lb.take(N * dkv * esz);
   L->lo.rq = lb.take(B * H * T * 4);
-  L->lo.rk = lb.take(B * H * T * 4);
+  L->lo.rk = lb.take(B * Hkv * T * 4);
   L->lo.o = lb.take(N * d * esz);
   L->lo.lse = lb.take(B * H * T * 4);
   L->lo.h2 = lb.take(N * d * esz);
@@ -81,8 +81,8 @@ bool make_layout(const gpt_config& c, Layout* L) {
   // layers at once
   uint64_t opt_bytes = 0;
   if (c.dtype == GPT_BF16) {
-    const int64_t mat = std::max(std::max(3 * d * d, F * d), d * d);
-    const int64_t gd = d;
+    const int64_t mat = std::max(std::max(Q * d, F * d), d * d);
+    const int64_t gd = d;  // Wqkv is [Q, d] with Q >= d, Wup [F, d], Wdown [d, F], Wo [d, d]
     Bump ob;
     L->opt_x0 = ob.take(mat * 2 * c.n_layer);
     L->opt_x1 = ob.take(mat * 2 * c.n_layer);
@@ -93,7 +93,7 @@ bool make_layout(const gpt_config& c, Layout* L) {
   L->layer_base = b.take(std::max(L->layer_stride * uint64_t(c.n_layer), opt_bytes));
   L->hf = b.take(N * d * esz);
   L->rf = b.take(N * 4);
-  L->qkv_raw = b.take(c.dtype == GPT_F32 ? N * 3 * d * esz : 0);  // bf16: fused into the GEMM
+  L->qkv_raw = b.take(c.dtype == GPT_F32 ? N * Q * esz : 0);  // bf16: fused into the GEMM
   // cross-entropy partials: the narrowest GEMM tile used for the logits is 64 columns
   L->n_part_max = (V + 63) / 64;
   L->part_max = b.take(N * L->n_part_max * 4);
@@ -106,10 +106,10 @@ bool make_layout(const gpt_config& c, Layout* L) {
   L->dh = b.take(N * d * esz);
   L->du = b.take(N * F * esz);
   L->dO = b.take(N * d * esz);
-  L->dqkv = b.take(N * 3 * d * esz);
+  L->dqkv = b.take(N * Q * esz);
   L->Dattn = b.take(B * H * T * 4);
   // split-K partials of the weight-gradient GEMMs (up to 4 splits of the largest layer matrix)
-  L->splitk_floats = c.dtype == GPT_BF16 ? 4 * std::max(std::max(3 * d * d, F * d), d * d) : 0;
+  L->splitk_floats = c.dtype == GPT_BF16 ? 4 * std::max(std::max(Q * d, F * d), d * d) : 0;
   L->splitk = b.take(L->splitk_floats * 4);
   // deterministic embedding scatter
   L->sort_tiles = (N + 1023) / 1024;
@@ -160,10 +160,12 @@ int gpt_config_init(gpt_config* c) {
   if (!c) return GPT_EINVAL;
   if (c->rope_base == 0.f) c->rope_base = 10000.f;
   if (c->norm_eps == 0.f) c->norm_eps = 1e-6f;
+  if (c->n_kv_head == 0) c->n_kv_head = c->n_head;
   if (c->n_layer < 0 || c->d_model <= 0 || c->n_head <= 0 || c->head_dim <= 0 ||
       c->d_ff <= 0 || c->vocab < 2 || c->seq_len <= 0 || c->batch <= 0)
     return GPT_EINVAL;
   if (int64_t(c->n_head) * c->head_dim != c->d_model) return GPT_EINVAL;
+  if (c->n_kv_head <= 0 || c->n_head % c->n_kv_head || c->attn_window < 0) return GPT_EINVAL;
   if (!(c->rope_base > 1.f) || !(c->norm_eps > 0.f) || !std::isfinite(c->rope_base) ||
       !std::isfinite(c->norm_eps))
     return GPT_EINVAL;
@@ -179,11 +181,11 @@ int gpt_config_init(gpt_config* c) {
   }
   const int64_t N = int64_t(c->batch) * c->seq_len;
   if (N > (int64_t(1) << 31) / 4 || int64_t(c->vocab) > (int64_t(1) << 24)) return GPT_EUNSUPPORTED;
-  const int64_t d = c->d_model, F = c->d_ff, V = c->vocab;
-  int64_t n = 2 * V * d + int64_t(c->n_layer) * (3 * d * d + d * d + 2 * F * d);
+  const int64_t d = c->d_model, F = c->d_ff, V = c->vocab, Q = qkv_cols(*c);
+  int64_t n = 2 * V * d + int64_t(c->n_layer) * (Q * d + d * d + 2 * F * d);
   c->n_params = n;
   int64_t elems = 2 * param_elems_aligned(V * d) +
-                  int64_t(c->n_layer) * (param_elems_aligned(3 * d * d) + param_elems_aligned(d * d) +
+                  int64_t(c->n_layer) * (param_elems_aligned(Q * d) + param_elems_aligned(d * d) +
                                          2 * param_elems_aligned(F * d));
   c->param_bytes = uint64_t(elems) * (c->dtype == GPT_BF16 ? 2 : 4);
   Layout L;
@@ -213,23 +215,23 @@ int gpt_config_from_depth(gpt_config* c, int depth, int seq_len, int batch, int 
 int gpt_param_offset(const gpt_config* c, int tensor, int layer, int64_t* off, int64_t* rows,
                      int64_t* cols) {
   if (!c || !off || !rows || !cols) return GPT_EINVAL;
-  const int64_t d = c->d_model, F = c->d_ff, V = c->vocab;
+  const int64_t d = c->d_model, F = c->d_ff, V = c->vocab, Q = qkv_cols(*c);
   const bool per_layer = tensor >= GPT_T_WQKV && tensor <= GPT_T_WDOWN;
   if (tensor < GPT_T_WTE || tensor > GPT_T_LM_HEAD) return GPT_EINVAL;
   if (per_layer && (layer < 0 || layer >= c->n_layer)) return GPT_EINVAL;
-  const int64_t lsz = param_elems_aligned(3 * d * d) + param_elems_aligned(d * d) +
+  const int64_t lsz = param_elems_aligned(Q * d) + param_elems_aligned(d * d) +
                       2 * param_elems_aligned(F * d);
   const int64_t base = param_elems_aligned(V * d);
   switch (tensor) {
     case GPT_T_WTE: *off = 0; *rows = V; *cols = d; break;
-    case GPT_T_WQKV: *off = base + layer * lsz; *rows = 3 * d; *cols = d; break;
+    case GPT_T_WQKV: *off = base + layer * lsz; *rows = Q; *cols = d; break;
     case GPT_T_WO:
-      *off = base + layer * lsz + param_elems_aligned(3 * d * d); *rows = d; *cols = d; break;
+      *off = base + layer * lsz + param_elems_aligned(Q * d); *rows = d; *cols = d; break;
     case GPT_T_WUP:
-      *off = base + layer * lsz + param_elems_aligned(3 * d * d) + param_elems_aligned(d * d);
+      *off = base + layer * lsz + param_elems_aligned(Q * d) + param_elems_aligned(d * d);
       *rows = F; *cols = d; break;
     case GPT_T_WDOWN:
-      *off = base + layer * lsz + param_elems_aligned(3 * d * d) + param_elems_aligned(d * d) +
+      *off = base + layer * lsz + param_elems_aligned(Q * d) + param_elems_aligned(d * d) +
              param_elems_aligned(F * d);
       *rows = d; *cols = F; break;
     case GPT_T_LM_HEAD: *off = base + int64_t(c->n_layer) * lsz; *rows = V; *cols = d; break;
@@ -303,7 +305,7 @@ static int run_gemm(const gpt_config& c, const GemmArgs& g, cudaStream_t st) {
     case EPI_DRELU2: bytes += mn * e * 2; break;
     case EPI_AXPBY: bytes += mn * e * 2; break;
     case EPI_CE_FWD: bytes += double(g.M) * 12; break;
-    case EPI_QKV: bytes += mn * e + double(g.M) * 2 * g.n_head * 4; break;
+    case EPI_QKV: bytes += mn * e + double(g.M) * (g.n_head + g.n_kv_head) * 4; break;
     default: bytes += mn * e; break;
   }
   TraceScope ts(GPT_K_GEMM, gemm_kernel_count(c, g), 2.0 * double(g.M) * g.N * g.K * g.batch,
@@ -311,8 +313,9 @@ static int run_gemm(const gpt_config& c, const GemmArgs& g, cudaStream_t st) {
   return launch_gemm(c, g, st);
 }
 
-static double attn_pairs(const gpt_config& c) {  // (query, key) pairs with key <= query
-  return double(c.batch) * c.n_head * (double(c.seq_len) * (c.seq_len + 1) / 2);
+static double attn_pairs(const gpt_config& c) {  // visible (query, key) pairs
+  const double T = c.seq_len, W = std::min<double>(window_span(c), T);
+  return double(c.batch) * c.n_head * (W * T - W * (W - 1) / 2);
 }
 
 struct Step {
@@ -381,24 +384,26 @@ int gpt_forward_loss(const gpt_config* c, const int32_t* tok, const int32_t* tgt
     TraceScope ts(GPT_K_NORM, 1, 0, S.nd() * (esz + 4 + esz) + N * 8.0, st);
     GPT_TRY(launch_embed_norm(*c, tok, S.param(GPT_T_WTE, 0), S.x, h0, r0, S.status, st));
   }
-  const double attn_f = 4.0 * attn_pairs(*c) * c->head_dim;  // QK^T and PV, causal half
+  const double attn_f = 4.0 * attn_pairs(*c) * c->head_dim;  // QK^T and PV, visible pairs
+  const int Qc = int(qkv_cols(*c));
   for (int l = 0; l < c->n_layer; ++l) {
     char* Lb = S.layer(l);
     if (c->dtype == GPT_BF16) {
       // QKV projection with RoPE, QK-norm and the head-major scatter in its epilogue
-      GemmArgs g = gemm_kk(Lb + L.lo.h1, d, S.param(GPT_T_WQKV, l), d, N, 3 * d, d, EPI_QKV,
-                           nullptr, 3 * d, S.status);
+      GemmArgs g = gemm_kk(Lb + L.lo.h1, d, S.param(GPT_T_WQKV, l), d, N, Qc, d, EPI_QKV,
+                           nullptr, Qc, S.status);
       g.q_out = Lb + L.lo.q; g.k_out = Lb + L.lo.k; g.v_out = Lb + L.lo.v;
       g.rq = reinterpret_cast<float*>(Lb + L.lo.rq);
       g.rk = reinterpret_cast<float*>(Lb + L.lo.rk);
       g.rope_cos = S.cos_t; g.rope_sin = S.sin_t;
       g.seq_len = c->seq_len; g.n_head = c->n_head; g.head_dim = c->head_dim;
+      g.n_kv_head = c->n_kv_head;
       g.qk_norm = c->qk_norm; g.norm_eps = c->norm_eps;
       GPT_TRY(run_gemm(*c, g, st));
     } else {
-      GPT_TRY(run_gemm(*c, gemm_kk(Lb + L.lo.h1, d, S.param(GPT_T_WQKV, l), d, N, 3 * d, d,
-                                   EPI_STORE, ws + L.qkv_raw, 3 * d, S.status), st));
-      TraceScope ts(GPT_K_QKV, 1, 0, S.nd() * 3 * esz * 2, st);
+      GPT_TRY(run_gemm(*c, gemm_kk(Lb + L.lo.h1, d, S.param(GPT_T_WQKV, l), d, N, Qc, d,
+                                   EPI_STORE, ws + L.qkv_raw, Qc, S.status), st));
+      TraceScope ts(GPT_K_QKV, 1, 0, double(N) * Qc * esz * 2, st);
       GPT_TRY(launch_qkv_post(*c, ws + L.qkv_raw, S.cos_t, S.sin_t, Lb + L.lo.q, Lb + L.lo.k,
                               Lb + L.lo.v, reinterpret_cast<float*>(Lb + L.lo.rq),
                               reinterpret_cast<float*>(Lb + L.lo.rk), st));
@@ -509,7 +514,7 @@ int gpt_backward(const gpt_config* c, const int32_t* tok, const int32_t* tgt,
     g = gemm_kk(ws + L.dxs, d, Lb + L.lo.o, d, d, d, N, EPI_STORE, grad(GPT_T_WO, l), d, status);
     g.a_mn_major = true; g.b_mn_major = true; g.beta = accumulate;
     GPT_TRY(run_gemm(*c, with_splitk(g, L, ws), st));
-    // attention, then QK-norm and RoPE backward, into dqkv [N, 3d]
+    // attention, then QK-norm and RoPE backward, into dqkv [N, Q] (Q = qkv columns)
     {
       TraceScope ts(GPT_K_ATTN_BWD, c->dtype == GPT_BF16 ? 3 : 2, attn_b, S.nd() * esz * 8, st);
       GPT_TRY(launch_attn_bwd(*c, Lb + L.lo.q, Lb + L.lo.k, Lb + L.lo.v, Lb + L.lo.o, ws + L.dO,
@@ -518,11 +523,12 @@ int gpt_backward(const gpt_config* c, const int32_t* tok, const int32_t* tgt,
                               reinterpret_cast<float*>(Lb + L.lo.rk), S.cos_t, S.sin_t,
                               S.f(L.Dattn), ws + L.dqkv, S.status, st));
     }
-    g = gemm_kk(ws + L.dqkv, 3 * d, S.param(GPT_T_WQKV, l), d, N, d, 3 * d, EPI_STORE, ws + L.dh,
+    const int Qc = int(qkv_cols(*c));
+    g = gemm_kk(ws + L.dqkv, Qc, S.param(GPT_T_WQKV, l), d, N, d, Qc, EPI_STORE, ws + L.dh,
                 d, status);
     g.b_mn_major = true;
     GPT_TRY(run_gemm(*c, g, st));
-    g = gemm_kk(ws + L.dqkv, 3 * d, Lb + L.lo.h1, d, 3 * d, d, N, EPI_STORE,
+    g = gemm_kk(ws + L.dqkv, Qc, Lb + L.lo.h1, d, Qc, d, N, EPI_STORE,
                 grad(GPT_T_WQKV, l), d, status);
     g.a_mn_major = true; g.b_mn_major = true; g.beta = accumulate;
     GPT_TRY(run_gemm(*c, with_splitk(g, L, ws), st));

@@ -1,9 +1,13 @@
 // Causal flash attention, forward and backward, on the sm_100a tensor cores.
 //
-// q, k, v: head-major [B*H*T, hd] bf16 (q and k already rotated and
-// normalised); o, dO: token-major [B*T, H*hd] bf16; lse: [B*H*T] fp32, the
-// log-sum-exp of each query row's scaled scores s_ij = q_i . k_j / sqrt(hd)
-// over keys j <= i.
+// q: head-major [B*H*T, hd] bf16, k, v: [B*Hkv*T, hd] (q and k already
+// rotated and normalised; query head h reads key/value head h / (H/Hkv),
+// grouped-query attention when Hkv < H); o, dO: token-major [B*T, H*hd] bf16;
+// lse: [B*H*T] fp32, the log-sum-exp of each query row's scaled scores
+// s_ij = q_i . k_j / sqrt(hd) over its visible keys i - W < j <= i (W, the
+// sliding window, longer than any sequence when unset).  Each kernel visits
+// only the key (or query) tiles that hold visible pairs and masks the rest
+// inside the boundary tiles.
 //
 // Every kernel: warp 0 loads tiles with TMA (128-byte swizzle), warps 1 and 10
 // issue tcgen05.mma into tensor memory (two independent MMA chains: one warp
@@ -205,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                        const __grid_constant__ CUtensorMap map_k,
                        const __grid_constant__ CUtensorMap map_v, __nv_bfloat16* __restrict__ o,
-                       float* __restrict__ lse, int H, int T, float scale_log2,
+                       float* __restrict__ lse, int H, int Hkv, int T, int W, float scale_log2,
                        int32_t* status) {
   using S = FwdSmem<HD>;
   extern __shared__ uint8_t smem_raw[];
@@ -219,8 +223,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int bh = int(blockIdx.x) / n_qt;
   const int qt = n_qt - 1 - int(blockIdx.x) % n_qt;
   const int q0 = qt * BQ;
-  const int n_kv = qt + 1;
+  const int j_lo = max(0, q0 - W + 1) / BKV;  // first key tile with a visible key
+  const int n_kv = qt - j_lo + 1;
   const int row_base = bh * T;
+  const int kv_row_base = ((bh / H) * Hkv + (bh % H) / (H / Hkv)) * T;
   constexpr uint32_t CH = BQ * 128;  // bytes of one 64-column chunk of a 128-row tile
   constexpr int NCH = HD / 64;
 
@@ -267,7 +273,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mbar_arrive_expect_tx(&full[st], S::TILE);
 #pragma unroll
         for (int c = 0; c < NCH; ++c)
-          tc::tma_load_2d(base + st * S::TILE + c * CH, map, &full[st], c * 64, row_base + j * BKV);
+          tc::tma_load_2d(base + st * S::TILE + c * CH, map, &full[st], c * 64,
+                          kv_row_base + (j_lo + j) * BKV);
         issued |= 1u << st;
         last_par = (last_par & ~(1u << st)) | (ph << st);
       }
@@ -336,6 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     const Roles R = roles();
     const int q = q0 + R.r;
+    const int lo_key = q - W + 1;  // the row's first visible key
     float* red = reinterpret_cast<float*>(smem + S::RED_OFF);
     float* sums = reinterpret_cast<float*>(smem + S::SUM_OFF);
     uint8_t* p_chunk = smem + S::P_OFF + R.half * CH;  // this thread's 64 keys
@@ -343,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
       const int st = j & 1;
-      const int k0 = j * BKV + R.half * 64;
+      const int k0 = (j_lo + j) * BKV + R.half * 64;
       if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->s_full[st], (j >> 1) & 1, abort, kWaitNs));
       float s[64];
       float mx = -INFINITY;
@@ -355,10 +363,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; ++i) { s[i] = __uint_as_float(ua[i]); s[32 + i] = __uint_as_float(ub[i]); }
-        if (j == qt || k0 + 64 > T) {
+        if (j_lo + j == qt || k0 + 64 > T || k0 < lo_key) {
 #pragma unroll
           for (int i = 0; i < 64; ++i)
-            if (k0 + i > q || k0 + i >= T) s[i] = -INFINITY;
+            if (k0 + i > q || k0 + i >= T || k0 + i < lo_key) s[i] = -INFINITY;
         }
 #pragma unroll
         for (int i = 0; i < 64; ++i) mx = fmaxf(mx, s[i]);
@@ -377,7 +385,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // P_j into registers first: this overlaps P_{j-1} V_{j-1}, which must
         // finish before O is rescaled and before the P tile is rewritten
         uint64_t lsum2 = f2(0.f, 0.f);
-        const uint64_t sc2 = f2(scale_log2, scale_log2), nm2 = f2(-m_ref, -m_ref);
+        // a row whose keys so far were all outside its window has no reference
+        // yet: its P is 0 (exp2(-inf - 0)), not NaN
+        const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
+        const uint64_t sc2 = f2(scale_log2, scale_log2), nm2 = f2(-m_use, -m_use);
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -453,9 +464,10 @@ template <int HD>
 int attn_fwd_tc_t(const gpt_config& c, const void* q, const void* k, const void* v, void* o,
                   float* lse, int32_t* status, cudaStream_t st) {
   const uint64_t rows = uint64_t(c.batch) * c.n_head * c.seq_len;
+  const uint64_t kv_rows = uint64_t(c.batch) * c.n_kv_head * c.seq_len;
   CUtensorMap mq, mk, mv;
-  if (!tile_map(&mq, q, rows, HD, HD, 128) || !tile_map(&mk, k, rows, HD, HD, 128) ||
-      !tile_map(&mv, v, rows, HD, HD, 128))
+  if (!tile_map(&mq, q, rows, HD, HD, 128) || !tile_map(&mk, k, kv_rows, HD, HD, 128) ||
+      !tile_map(&mv, v, kv_rows, HD, HD, 128))
     return 1;
   auto kern = attn_fwd_tc_kernel<HD>;
   const int smem = int(FwdSmem<HD>::BYTES);
@@ -463,8 +475,8 @@ int attn_fwd_tc_t(const gpt_config& c, const void* q, const void* k, const void*
     return 1;
   const int n_qt = (c.seq_len + BQ - 1) / BQ;
   kern<<<n_qt * c.batch * c.n_head, kThreads, smem, st>>>(
-      mq, mk, mv, static_cast<__nv_bfloat16*>(o), lse, c.n_head, c.seq_len,
-      kLog2e / sqrtf(float(HD)), status);
+      mq, mk, mv, static_cast<__nv_bfloat16*>(o), lse, c.n_head, c.n_kv_head, c.seq_len,
+      window_span(c), kLog2e / sqrtf(float(HD)), status);
   return last_launch_rc();
 }
 }  // namespace
@@ -669,8 +681,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap map_sin,
                       const float* __restrict__ lse,
                       const float* __restrict__ D, const float* __restrict__ rq,
-                      __nv_bfloat16* __restrict__ dqkv, int H, int T, float scale,
-                      float scale_log2, int qk_norm, int32_t* status) {
+                      __nv_bfloat16* __restrict__ dqkv, int64_t ldq, int H, int Hkv, int T,
+                      int W, float scale, float scale_log2, int qk_norm, int32_t* status) {
   using S = DqSmem<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -682,7 +694,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int qt = n_qt - 1 - int(blockIdx.x) % n_qt;
   const int b = bh / H, h = bh % H;
   const int q0 = qt * 128;
-  const int n_steps = (min(q0 + 128, T) + kInner - 1) / kInner;
+  const int s_lo = max(0, q0 - W + 1) / kInner;  // first key step with a visible key
+  const int n_steps = (min(q0 + 128, T) + kInner - 1) / kInner - s_lo;
+  const int kv_row_base = (b * Hkv + h / (H / Hkv)) * T;
   constexpr int NCH = HD / 64;
 
   ATTN_PROLOGUE(bars, {
@@ -727,9 +741,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < NCH; ++c) {
           tc::tma_load_2d(smem + S::K_OFF + st * S::SMALL + c * (kInner * 128), &map_k64,
-                          &bars->ring_full[st], c * 64, bh * T + j * kInner);
+                          &bars->ring_full[st], c * 64, kv_row_base + (s_lo + j) * kInner);
           tc::tma_load_2d(smem + S::V_OFF + st * S::SMALL + c * (kInner * 128), &map_v64,
-                          &bars->ring_full[st], c * 64, bh * T + j * kInner);
+                          &bars->ring_full[st], c * 64, kv_row_base + (s_lo + j) * kInner);
         }
         if (j == 0)
           load_epilogue_tiles<HD>(nullptr, smem + S::COS_OFF, smem + S::SIN_OFF, nullptr, &map_cos,
@@ -824,6 +838,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = q0 + R.r;
     const bool qv = q < T;
     const int tq = qv ? q : 0;
+    const int lo_key = q - W + 1;
     const float lse2 = qv ? lse[int64_t(bh) * T + q] * kLog2e : 0.f;
     const float Dq = qv ? D[int64_t(bh) * T + q] : 0.f;
     bool ok = true;
@@ -833,13 +848,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->dp_full[sb], (j >> 1) & 1, abort, kWaitNs));
       if (ok) {
         tc::tc_fence_after();
-        const int k0 = j * kInner + R.half * 32;
+        const int k0 = (s_lo + j) * kInner + R.half * 32;
         const uint32_t ts = tmem + sb * 128 + R.lane_off + R.half * 32;
         uint32_t us[32], up[32];
         tc::tmem_ld_32x32b_x32(ts, us);
         tc::tmem_ld_32x32b_x32(ts + kInner, up);
         tc::tmem_wait_ld();
-        const bool need_mask = !qv || k0 + 32 > q || k0 + 32 > T;
+        const bool need_mask = !qv || k0 + 32 > q || k0 + 32 > T || k0 < lo_key;
         uint32_t pk[16];
         const uint64_t sc2 = f2(scale_log2, scale_log2), nl2 = f2(-lse2, -lse2), nd2 = f2(-Dq, -Dq);
 #pragma unroll
@@ -848,8 +863,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float2 x = unf2(fma2(f2(__uint_as_float(us[i]), __uint_as_float(us[i + 1])), sc2, nl2));
           float p0 = ex2(x.x), p1 = ex2(x.y);
           if (need_mask) {
-            if (k0 + i > q || k0 + i >= T || !qv) p0 = 0.f;
-            if (k0 + i + 1 > q || k0 + i + 1 >= T || !qv) p1 = 0.f;
+            if (k0 + i > q || k0 + i >= T || !qv || k0 + i < lo_key) p0 = 0.f;
+            if (k0 + i + 1 > q || k0 + i + 1 >= T || !qv || k0 + i + 1 < lo_key) p1 = 0.f;
           }
           const float2 r =
               unf2(mul2(f2(p0, p1), add2(f2(__uint_as_float(up[i]), __uint_as_float(up[i + 1])), nd2)));
@@ -869,10 +884,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
       tc::tc_fence_after();
     }
-    const int d = H * HD;
     norm_rope_bwd_half<HD>(t_dq + R.lane_off, R.half, R.r, scale, smem + S::Y_OFF,
                            qv ? rq[int64_t(bh) * T + q] : 0.f, qk_norm, smem + S::COS_OFF,
-                           smem + S::SIN_OFF, dqkv + (int64_t(b) * T + tq) * 3 * d + h * HD, ok,
+                           smem + S::SIN_OFF, dqkv + (int64_t(b) * T + tq) * ldq + h * HD, ok,
                            qv, reinterpret_cast<float*>(smem + S::RED_OFF));
   }
   ATTN_EPILOGUE(tmem)
@@ -918,8 +932,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                        const __grid_constant__ CUtensorMap map_sin,
                        const float* __restrict__ lse,
                        const float* __restrict__ D, const float* __restrict__ rk,
-                       __nv_bfloat16* __restrict__ dqkv, int H, int T, float scale,
-                       float scale_log2, int qk_norm, int32_t* status) {
+                       __nv_bfloat16* __restrict__ dqkv, int64_t ldq, int H, int Hkv, int T,
+                       int W, float scale, float scale_log2, int qk_norm, int32_t* status) {
   using S = DkvSmem<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -927,12 +941,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   BwdBars* bars = reinterpret_cast<BwdBars*>(smem + S::BAR_OFF);
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int n_kt = (T + 127) / 128;
-  const int bh = int(blockIdx.x) / n_kt;  // (batch, head)-major; key tile 0 (most queries) first
+  const int bkv = int(blockIdx.x) / n_kt;  // (batch, kv head)-major; key tile 0 first
   const int kt = int(blockIdx.x) % n_kt;
-  const int b = bh / H, h = bh % H;
+  const int b = bkv / Hkv, hk = bkv % Hkv, rep = H / Hkv;
   const int k0 = kt * 128;
   const int i_begin = k0 / kInner;
-  const int n_steps = (T + kInner - 1) / kInner - i_begin;  // causal: queries k0 .. T-1
+  // queries k0 .. min(T, k0 + 127 + W) - 1 see some key of the tile; the steps
+  // run over them once per query head of the group (head hk*rep + j / n_h)
+  const int n_h = (min(T, k0 + 127 + W) + kInner - 1) / kInner - i_begin;
+  const int n_steps = rep * n_h;
   constexpr int NCH = HD / 64;
 
   ATTN_PROLOGUE(bars, {
@@ -961,14 +978,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_arrive_expect_tx(&bars->fixed_full, 2 * S::BIG);
 #pragma unroll
       for (int c = 0; c < NCH; ++c) {
-        tc::tma_load_2d(smem + S::K_OFF + c * (128 * 128), &map_k128, &bars->fixed_full, c * 64, bh * T + k0);
-        tc::tma_load_2d(smem + S::V_OFF + c * (128 * 128), &map_v128, &bars->fixed_full, c * 64, bh * T + k0);
+        tc::tma_load_2d(smem + S::K_OFF + c * (128 * 128), &map_k128, &bars->fixed_full, c * 64, bkv * T + k0);
+        tc::tma_load_2d(smem + S::V_OFF + c * (128 * 128), &map_v128, &bars->fixed_full, c * 64, bkv * T + k0);
       }
     }
     for (int j = 0; j < n_steps; ++j) {
       const int st = j % kRingKV;
       const uint32_t ph = (j / kRingKV) & 1;
-      const int qs = (i_begin + j) * kInner;
+      const int gi = j / n_h;
+      const int qs = (i_begin + j - gi * n_h) * kInner;
+      const int h = hk * rep + gi, bh = b * H + h;
       if (!tc::mbar_wait_warp(&bars->ring_empty[st], ph ^ 1, abort, kWaitNs)) {
         if (lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 30);
         *abort = 1;
@@ -1062,6 +1081,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int key = k0 + R.r;
     const bool kv = key < T;
     const int tk = kv ? key : 0;
+    const int end_q = key + W;  // the key's last visible query is end_q - 1
     bool ok = true;
     for (int j = 0; j < n_steps; ++j) {
       const int sb = j & 1, st = j % kRingKV;
@@ -1072,7 +1092,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->ring_full[st], (j / kRingKV) & 1, abort, kWaitNs));
       if (ok) {
         tc::tc_fence_after();
-        const int qs = (i_begin + j) * kInner + R.half * 32;
+        const int qs = (i_begin + j - (j / n_h) * n_h) * kInner + R.half * 32;
         const float4* stat4 =
             reinterpret_cast<const float4*>(smem + S::STAT_OFF + (st * 2 * kInner + R.half * 32) * 4);
         const uint32_t ts = tmem + sb * 128 + R.lane_off + R.half * 32;
@@ -1080,7 +1100,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::tmem_ld_32x32b_x32(ts, us);
         tc::tmem_ld_32x32b_x32(ts + kInner, up);
         tc::tmem_wait_ld();
-        const bool need_mask = !kv || qs < key || qs + 32 > T;
+        const bool need_mask = !kv || qs < key || qs + 32 > T || qs + 32 > end_q;
         uint32_t pp[16], pd[16];
 #pragma unroll
         for (int g = 0; g < 8; ++g) {  // 4 queries per group
@@ -1093,8 +1113,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                        f2(scale_log2, scale_log2), f2(-l2[e], -l2[e + 1])));
             float p0 = ex2(x.x), p1 = ex2(x.y);
             if (need_mask) {
-              if (qs + i < key || qs + i >= T || !kv) p0 = 0.f;
-              if (qs + i + 1 < key || qs + i + 1 >= T || !kv) p1 = 0.f;
+              if (qs + i < key || qs + i >= T || !kv || qs + i >= end_q) p0 = 0.f;
+              if (qs + i + 1 < key || qs + i + 1 >= T || !kv || qs + i + 1 >= end_q) p1 = 0.f;
             }
             pp[i / 2] = pack2(p0, p1);
             const float2 r = unf2(mul2(f2(p0, p1), add2(f2(__uint_as_float(up[i]), __uint_as_float(up[i + 1])),
@@ -1118,7 +1138,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tc_fence_after();
     }
     const int d = H * HD;
-    __nv_bfloat16* row = dqkv + (int64_t(b) * T + tk) * 3 * d;
+    __nv_bfloat16* row = dqkv + (int64_t(b) * T + tk) * ldq;
     if (ok) {  // dV: this thread's half of the columns
 #pragma unroll
       for (int c = 0; c < HD / 2; c += 32) {
@@ -1127,7 +1147,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (kv) {
 #pragma unroll
           for (int i = 0; i < 32; i += 8)
-            *reinterpret_cast<uint4*>(row + 2 * d + h * HD + R.half * (HD / 2) + c + i) =
+            *reinterpret_cast<uint4*>(row + d + (Hkv + hk) * HD + R.half * (HD / 2) + c + i) =
                 make_uint4(pack2(v[i], v[i + 1]), pack2(v[i + 2], v[i + 3]), pack2(v[i + 4], v[i + 5]),
                            pack2(v[i + 6], v[i + 7]));
         }
@@ -1135,8 +1155,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // the stats region is free once every step is done (acc_full): it holds red
     norm_rope_bwd_half<HD>(t_dk + R.lane_off, R.half, R.r, scale, smem + S::K_OFF,
-                           kv ? rk[int64_t(bh) * T + key] : 0.f, qk_norm, smem + S::COS_OFF,
-                           smem + S::SIN_OFF, row + d + h * HD, ok, kv,
+                           kv ? rk[int64_t(bkv) * T + key] : 0.f, qk_norm, smem + S::COS_OFF,
+                           smem + S::SIN_OFF, row + d + hk * HD, ok, kv,
                            reinterpret_cast<float*>(smem + S::RED_OFF));
   }
   ATTN_EPILOGUE(tmem)
@@ -1148,14 +1168,16 @@ int attn_bwd_tc_t(const gpt_config& c, const void* q, const void* k, const void*
                   const void* dO, const float* lse, const float* rq, const float* rk,
                   const float* cos_t, const float* sin_t, float* Dbuf, void* dqkv,
                   int32_t* status, cudaStream_t st) {
-  const int H = c.n_head, T = c.seq_len, B = c.batch, d = H * HD;
-  const uint64_t rows = uint64_t(B) * H * T, ntok = uint64_t(B) * T;
+  const int H = c.n_head, Hkv = c.n_kv_head, T = c.seq_len, B = c.batch, d = H * HD;
+  const int W = window_span(c);
+  const int64_t ldq = qkv_cols(c);
+  const uint64_t rows = uint64_t(B) * H * T, kv_rows = uint64_t(B) * Hkv * T, ntok = uint64_t(B) * T;
   const int64_t N = int64_t(B) * T;
   attn_rowdot_kernel<<<ceil_div(N * H * (HD / 8), 256), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(dO), static_cast<const __nv_bfloat16*>(o), Dbuf, N, H, T, HD);
   CUtensorMap k64, v64, k128, v128, q64, do64, q128, do128, mcos, msin;
-  bool ok = tile_map(&k64, k, rows, HD, HD, 64) && tile_map(&v64, v, rows, HD, HD, 64) &&
-            tile_map(&k128, k, rows, HD, HD, 128) && tile_map(&v128, v, rows, HD, HD, 128) &&
+  bool ok = tile_map(&k64, k, kv_rows, HD, HD, 64) && tile_map(&v64, v, kv_rows, HD, HD, 64) &&
+            tile_map(&k128, k, kv_rows, HD, HD, 128) && tile_map(&v128, v, kv_rows, HD, HD, 128) &&
             tile_map(&q64, q, rows, HD, HD, 64) && tile_map(&do64, dO, ntok, d, d, 64) &&
             tile_map(&q128, q, rows, HD, HD, 128) && tile_map(&do128, dO, ntok, d, d, 128) &&
             tile_map_f32(&mcos, cos_t, T, HD / 2, HD / 2, 128) &&
@@ -1169,15 +1191,15 @@ int attn_bwd_tc_t(const gpt_config& c, const void* q, const void* k, const void*
   if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_q) != cudaSuccess)
     return 1;
   kq<<<nt * B * H, kThreads, smem_q, st>>>(q128, do128, k64, v64, mcos, msin, lse, Dbuf, rq,
-                                           static_cast<__nv_bfloat16*>(dqkv), H, T, scale,
-                                           scale_log2, c.qk_norm, status);
+                                           static_cast<__nv_bfloat16*>(dqkv), ldq, H, Hkv, T, W,
+                                           scale, scale_log2, c.qk_norm, status);
   auto kk = attn_dkv_tc_kernel<HD>;
   const int smem_k = int(DkvSmem<HD>::BYTES);
   if (cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_k) != cudaSuccess)
     return 1;
-  kk<<<nt * B * H, kThreads, smem_k, st>>>(k128, v128, q64, do64, mcos, msin, lse, Dbuf, rk,
-                                           static_cast<__nv_bfloat16*>(dqkv), H, T, scale,
-                                           scale_log2, c.qk_norm, status);
+  kk<<<nt * B * Hkv, kThreads, smem_k, st>>>(k128, v128, q64, do64, mcos, msin, lse, Dbuf, rk,
+                                             static_cast<__nv_bfloat16*>(dqkv), ldq, H, Hkv, T, W,
+                                             scale, scale_log2, c.qk_norm, status);
   return last_launch_rc();
 }
 }  // namespace

@@ -225,14 +225,18 @@ __device__ __forceinline__ void epi_chunk(const GemmArgs& g, int row, int col0, 
 // and written head-major, with the 1/rms kept for the backward.
 __device__ __forceinline__ void epi_qkv_row(const GemmArgs& g, uint32_t taddr, int row,
                                             int col_base, bool row_ok) {
-  const int hd = g.head_dim, half = hd / 2, H = g.n_head, d = H * hd, T = g.seq_len;
+  const int hd = g.head_dim, half = hd / 2, H = g.n_head, Hkv = g.n_kv_head, T = g.seq_len;
   const int b = row_ok ? row / T : 0, t = row_ok ? row % T : 0;
   for (int seg = 0; seg < EC / hd; ++seg) {
     const int c0 = col_base + seg * hd;
     if (c0 >= g.N) break;  // uniform across the warp
-    const int part = c0 / d, h = (c0 % d) / hd;
+    // column head c0/hd: the n_head q heads, then n_kv_head k heads, then v heads
+    const int ch = c0 / hd;
+    const int part = ch < H ? 0 : (ch < H + Hkv ? 1 : 2);
+    const int h = part == 0 ? ch : (part == 1 ? ch - H : ch - H - Hkv);
+    const int nh = part == 0 ? H : Hkv;  // heads of this part's [B, nh, T, hd] output
     const uint32_t tcol = taddr + seg * hd;
-    const int64_t dst = ((int64_t(b) * H + h) * T + t) * hd;
+    const int64_t dst = ((int64_t(b) * nh + h) * T + t) * hd;
     if (part == 2) {
       __nv_bfloat16* vo = static_cast<__nv_bfloat16*>(g.v_out) + dst;
       for (int c = 0; c < hd; c += 32) {
@@ -292,7 +296,7 @@ __device__ __forceinline__ void epi_qkv_row(const GemmArgs& g, uint32_t taddr, i
       ob[1] = make_uint4(pb[4], pb[5], pb[6], pb[7]);
     }
     if (row_ok) {
-      const int64_t ri = (int64_t(b) * H + h) * T + t;
+      const int64_t ri = (int64_t(b) * nh + h) * T + t;
       (part == 0 ? g.rq : g.rk)[ri] = r;
     }
   }

@@ -9,6 +9,15 @@
 
 namespace gpt {
 
+// Columns of the [q | k | v] projection: n_head query heads and n_kv_head key
+// and value heads of head_dim each (gpt_config_init sets n_kv_head).
+inline int64_t qkv_cols(const gpt_config& c) {
+  return int64_t(c.n_head + 2 * c.n_kv_head) * c.head_dim;
+}
+// The sliding window as a key-distance bound: query i sees keys j with
+// i - j < window_span(c) (a span longer than any sequence when unset).
+inline int window_span(const gpt_config& c) { return c.attn_window > 0 ? c.attn_window : (1 << 30); }
+
 // Kernel ids recorded in gpt_device_status::where.
 enum KernelId : int32_t {
   K_EMBED = 1,
@@ -56,15 +65,17 @@ struct GemmArgs {
   float inv_n;
   int n_valid;              // columns >= n_valid are padding (EPI_CE_BWD writes 0)
   int32_t* status;          // device status word
-  // EPI_QKV (rows = tokens b*T + t, columns = [q | k | v] of n_head heads of head_dim)
-  void* q_out;
+  // EPI_QKV (rows = tokens b*T + t, columns = [q | k | v]: n_head q heads,
+  // then n_kv_head k heads and n_kv_head v heads, head_dim each)
+  void* q_out;              // [B, n_head, T, hd]
   void* k_out;
-  void* v_out;              // [B, H, T, hd] each
-  float* rq;
-  float* rk;                // [B, H, T]: 1/rms of the rotated q, k rows
+  void* v_out;              // [B, n_kv_head, T, hd] each
+  float* rq;                // [B, n_head, T]: 1/rms of the rotated q rows
+  float* rk;                // [B, n_kv_head, T]: the same for k
   const float* rope_cos;
   const float* rope_sin;    // [T, hd/2]
   int seq_len, n_head, head_dim, qk_norm;
+  int n_kv_head;
   float norm_eps;
   // batched products (tensor-core GEMM; EPI_STORE without beta or EPI_AXPBY,
   // K a multiple of 64): product b reads A and B `a_bstride` / `b_bstride` rows

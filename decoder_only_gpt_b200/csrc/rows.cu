@@ -289,14 +289,16 @@ int launch_rms_bwd(const gpt_config& c, const void* dh, const void* h, const flo
 }
 
 // ---------------------------------------------------------------------------
-// q, k <- rms_head(RoPE(q, k)); scatter q, k, v from [N, 3d] to [B, H, T, hd].
-// One warp per (token, head); lane handles rotation pairs (i, i + hd/2).
+// q, k <- rms_head(RoPE(q, k)); scatter q, k, v from [N, Q] rows (n_head q
+// heads, then Hkv k heads and Hkv v heads) to [B, heads, T, hd].  One warp per
+// (token, query head); the warps of heads below Hkv also handle that k and v
+// head.  A lane handles rotation pairs (i, i + hd/2).
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void qkv_post_kernel(const T* __restrict__ raw, const float* __restrict__ cos_t,
                                 const float* __restrict__ sin_t, T* __restrict__ q,
                                 T* __restrict__ k, T* __restrict__ v, float* __restrict__ rq,
-                                float* __restrict__ rk, int64_t N, int Tn, int H, int hd,
+                                float* __restrict__ rk, int64_t N, int Tn, int H, int Hkv, int hd,
                                 float eps, int qk_norm) {
   int64_t w = int64_t(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
   int lane = threadIdx.x & 31;
@@ -305,12 +307,13 @@ __global__ void qkv_post_kernel(const T* __restrict__ raw, const float* __restri
   int hh = int(w % H);
   int64_t b = n / Tn;
   int t = int(n % Tn);
-  const int d = H * hd, half = hd / 2;
-  const int64_t dst = ((b * H + hh) * Tn + t) * hd;
-  const int64_t ridx = (b * H + hh) * Tn + t;
-#pragma unroll
+  const int d = H * hd, half = hd / 2, Q = d + 2 * Hkv * hd;
   for (int part = 0; part < 2; ++part) {
-    const T* src = raw + n * 3 * d + part * d + hh * hd;
+    if (part == 1 && hh >= Hkv) break;
+    const int nh = part == 0 ? H : Hkv;
+    const int64_t dst = ((b * nh + hh) * Tn + t) * hd;
+    const int64_t ridx = (b * nh + hh) * Tn + t;
+    const T* src = raw + n * Q + (part == 0 ? 0 : d) + hh * hd;
     T* out = part == 0 ? q : k;
     float a0[4], b0[4];
     float ss = 0.f;
@@ -331,8 +334,10 @@ __global__ void qkv_post_kernel(const T* __restrict__ raw, const float* __restri
     }
     if (lane == 0) (part == 0 ? rq : rk)[ridx] = rr;
   }
-  const T* vs = raw + n * 3 * d + 2 * d + hh * hd;
-  for (int i = lane; i < hd; i += 32) v[dst + i] = vs[i];
+  if (hh >= Hkv) return;
+  const T* vs = raw + n * Q + d + Hkv * hd + hh * hd;
+  const int64_t vdst = ((b * Hkv + hh) * Tn + t) * hd;
+  for (int i = lane; i < hd; i += 32) v[vdst + i] = vs[i];
 }
 
 int launch_qkv_post(const gpt_config& c, const void* raw, const float* cos_t,
@@ -344,11 +349,12 @@ int launch_qkv_post(const gpt_config& c, const void* raw, const float* cos_t,
   if (c.dtype == GPT_BF16)
     qkv_post_kernel<__nv_bfloat16><<<grid, 256, 0, (cudaStream_t)stream>>>(
         (const __nv_bfloat16*)raw, cos_t, sin_t, (__nv_bfloat16*)q, (__nv_bfloat16*)k,
-        (__nv_bfloat16*)v, rq, rk, N, c.seq_len, c.n_head, c.head_dim, c.norm_eps, c.qk_norm);
+        (__nv_bfloat16*)v, rq, rk, N, c.seq_len, c.n_head, c.n_kv_head, c.head_dim, c.norm_eps,
+        c.qk_norm);
   else
     qkv_post_kernel<float><<<grid, 256, 0, (cudaStream_t)stream>>>(
         (const float*)raw, cos_t, sin_t, (float*)q, (float*)k, (float*)v, rq, rk, N,
-        c.seq_len, c.n_head, c.head_dim, c.norm_eps, c.qk_norm);
+        c.seq_len, c.n_head, c.n_kv_head, c.head_dim, c.norm_eps, c.qk_norm);
   return last_launch_rc();
 }
 

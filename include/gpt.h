@@ -6,7 +6,8 @@
  * Egitirsiniz?" (dev.to), section "1. GPT Modeli (nanochat/gpt.py)": rotary
  * position embeddings, QK normalisation, untied token embedding and lm_head,
  * ReLU^2 MLP, causal attention (section "5. Flash Dikkat Mekanizmasi
- * Birlesimi", causal=True), bias-free linear layers (section "3. Hassasiyet
+ * Birlesimi", causal=True, optionally with a sliding window), optionally
+ * grouped-query attention (the model list), bias-free linear layers (section "3. Hassasiyet
  * Yonetimi", F.linear(x, W) with W stored [out, in]).  Width, heads and MLP
  * size follow the depth dial of section "Felsefe: Her Seyi Kontrol Eden Tek
  * Bir Kadran" (d_model = 64 * depth, head_dim 128, d_ff = 4 * d_model).
@@ -16,6 +17,9 @@
  *   x = wte[tokens]
  *   per layer:  h = rms(x); [q|k|v] = h Wqkv^T; q,k <- rms_head(RoPE(q,k))
  *               x += causal_softmax(q k^T / sqrt(hd)) v  Wo^T
+ *               (k, v: n_kv_head heads, each shared by n_head/n_kv_head
+ *               consecutive query heads; keys restricted to the last
+ *               attn_window positions when that is set)
  *               h = rms(x); x += relu(h Wup^T)^2 Wdown^T
  *   z = rms(x) Wlm^T;  loss = mean_t (logsumexp(z_t) - z_t[target_t])
  * and the exact gradient of that loss w.r.t. every parameter.
@@ -59,8 +63,10 @@ extern "C" {
 
 /* ---- parameter tensors (for gpt_param_offset) -------------------------- */
 #define GPT_T_WTE 0     /* [vocab, d_model]          token embedding          */
-#define GPT_T_WQKV 1    /* [3*d_model, d_model]      q rows, then k, then v;  */
-                        /*   inside each block head h owns rows h*hd..h*hd+hd-1 */
+#define GPT_T_WQKV 1    /* [d_model + 2*n_kv_head*head_dim, d_model] (3*d_model
+                           without GQA): the n_head q heads' rows, then the
+                           n_kv_head k heads', then the v heads'; inside each
+                           block head h owns rows h*hd..h*hd+hd-1             */
 #define GPT_T_WO 2      /* [d_model, d_model]        attention out-projection */
 #define GPT_T_WUP 3     /* [d_ff, d_model]           MLP up                   */
 #define GPT_T_WDOWN 4   /* [d_model, d_ff]           MLP down                 */
@@ -97,6 +103,11 @@ typedef struct gpt_config {
   int32_t batch;    /* B >= 1                                            */
   int32_t dtype;    /* GPT_BF16 or GPT_F32                               */
   int32_t qk_norm;  /* 1: RMSNorm q and k per head after RoPE (default)  */
+  int32_t n_kv_head;   /* key/value heads (grouped-query attention): query
+                          head h reads key/value head h / (n_head/n_kv_head);
+                          divides n_head; 0 = n_head (set by gpt_config_init) */
+  int32_t attn_window; /* sliding window: query i attends to keys i-W < j <= i
+                          in every layer; 0 = the full causal window          */
   float rope_base;  /* 10000 by default                                  */
   float norm_eps;   /* 1e-6 by default                                   */
   /* derived by gpt_config_init */
@@ -106,9 +117,10 @@ typedef struct gpt_config {
 } gpt_config;
 
 /* Validate `cfg` and fill its derived fields.  Host only, no CUDA call.
- * Zero-valued rope_base / norm_eps are replaced by the defaults.
+ * Zero-valued rope_base / norm_eps / n_kv_head are replaced by the defaults.
  * GPT_EINVAL for a NULL or inconsistent config (d_model != n_head*head_dim,
- * non-positive sizes), GPT_EUNSUPPORTED for shapes the kernels do not cover
+ * non-positive sizes, n_kv_head not dividing n_head, attn_window < 0),
+ * GPT_EUNSUPPORTED for shapes the kernels do not cover
  * (bf16: d_model % 64, d_ff % 64, head_dim not 64/128; f32: odd head_dim or
  * head_dim > 128). */
 int gpt_config_init(gpt_config* cfg);

@@ -54,6 +54,7 @@ def test_config_derived_fields(B, name):
     c = B.config_from_workload(w)
     d, F, V, L = w.d_model, w.d_ff, w.vocab, w.n_layer
     assert c.n_params == 2 * V * d + L * (4 * d * d + 2 * F * d)
+    assert c.n_params == sum(r * cc for _, (r, cc) in synth.param_shapes(w))
     esz = 2 if w.dtype == "bf16" else 4
     assert c.param_bytes >= c.n_params * esz
     assert c.param_bytes - c.n_params * esz < (2 + 4 * L) * 128 * esz
@@ -75,6 +76,9 @@ def test_depth_dial(B):
     (dict(vocab=1), "EINVAL"),
     (dict(seq_len=0), "EINVAL"),
     (dict(batch=-1), "EINVAL"),
+    (dict(n_kv_head=3), "EINVAL"),              # does not divide n_head
+    (dict(n_kv_head=-2), "EINVAL"),
+    (dict(attn_window=-1), "EINVAL"),
 ])
 def test_config_rejects(B, kw, code):
     base = dict(n_layer=2, d_model=256, n_head=2, head_dim=128, d_ff=1024, vocab=4096,
@@ -92,9 +96,25 @@ def test_f32_config_rules(B):
     assert B.lib().gpt_config_init(ctypes.byref(bad)) == B.GPT_EUNSUPPORTED
 
 
-@pytest.mark.parametrize("name", ["tiny", "story", "d24"])
-def test_param_layout(B, name):
-    w = synth.workload(name)
+def test_gqa_and_window_config(B):
+    # n_kv_head 0 means n_head; the q/k/v projection shrinks with n_kv_head
+    c = B.make_config(2, 256, 4, 64, 1024, 4096, 128, 2)
+    assert c.n_kv_head == 4 and c.attn_window == 0
+    g = B.make_config(2, 256, 4, 64, 1024, 4096, 128, 2, n_kv_head=1, attn_window=48)
+    assert g.n_kv_head == 1 and g.attn_window == 48
+    d, F, V = 256, 1024, 4096
+    assert g.n_params == 2 * V * d + 2 * ((d + 2 * 64) * d + d * d + 2 * F * d)
+    assert B.param_offset(g, B.GPT_T_WQKV, 1)[1:] == (d + 2 * 64, d)
+    assert g.param_bytes < c.param_bytes and g.workspace_bytes < c.workspace_bytes
+    f = B.make_config(2, 64, 4, 16, 256, 256, 64, 4, dtype="f32", n_kv_head=2, attn_window=9)
+    assert f.n_kv_head == 2
+
+
+@pytest.mark.parametrize("name,kw", [("tiny", {}), ("story", {}), ("d24", {}),
+                                     ("story", dict(n_kv_head=2, window=100)),
+                                     ("tiny", dict(n_kv_head=1, window=3))])
+def test_param_layout(B, name, kw):
+    w = synth.workload(name, **kw)
     c = B.config_from_workload(w)
     esz = 2 if w.dtype == "bf16" else 4
     shapes = dict(synth.param_shapes(w))

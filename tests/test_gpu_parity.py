@@ -45,6 +45,21 @@ CASES = {
                                 vocab=700, seq_len=150, batch=2)),
     # fp32 ragged
     "tiny_ragged": ("tiny", dict(seq_len=37, batch=3, vocab=100, d_ff=96)),
+    # grouped-query attention and sliding windows: 2 query heads per key/value
+    # head with a window shorter than one 128-query tile (rows whose whole first
+    # key tile is outside the window)
+    "gqa_window": ("story", dict(n_layer=2, d_model=256, n_head=4, head_dim=64, n_kv_head=2,
+                                 window=100, d_ff=512, vocab=2048, seq_len=256, batch=2)),
+    # one key/value head (MQA), hd 128, window 70, ragged sequence of 300
+    "mqa_window_hd128": ("d4", dict(n_layer=2, d_model=256, n_head=2, head_dim=128, n_kv_head=1,
+                                    window=70, d_ff=512, vocab=1000, seq_len=300, batch=2)),
+    # a window spanning several key tiles that starts past the first one
+    "gqa_window_long": ("story", dict(n_layer=1, d_model=256, n_head=4, head_dim=64, n_kv_head=1,
+                                      window=200, d_ff=512, vocab=1024, seq_len=640, batch=1)),
+    # GQA alone, and the fp32 path with both
+    "gqa_full": ("story", dict(n_layer=2, d_model=256, n_head=4, head_dim=64, n_kv_head=2,
+                               d_ff=512, vocab=2048, seq_len=192, batch=2)),
+    "tiny_gqa_window": ("tiny", dict(n_kv_head=2, window=9, seq_len=37, batch=3, vocab=100)),
 }
 
 
@@ -194,6 +209,24 @@ def test_causality_on_gpu(B, R):
     lc = c.token_loss.cpu().numpy().reshape(w.batch, w.seq_len)
     assert np.array_equal(la[b, : t + 1].view(np.uint32), lc[b, : t + 1].view(np.uint32))
     assert not np.array_equal(la[b, t + 1:], lc[b, t + 1:])
+
+
+@pytest.mark.parametrize("case", ["gqa_window", "tiny_gqa_window"])
+def test_window_receptive_field_on_gpu(B, R, case):
+    # after L layers with window W a position sees the L(W-1) previous tokens:
+    # changing the token just beyond that reach leaves its loss bit-identical
+    w = workload_of(case)
+    tok, tgt = synth.make_tokens(w)
+    a, _ = run_gpu(B, R, w)
+    b, t = 1, w.seq_len - 3
+    reach = w.n_layer * (w.window - 1)
+    far = tok.copy()
+    far[b, t - reach - 1] = (far[b, t - reach - 1] + 5) % w.vocab
+    c, _ = run_gpu(B, R, w, tokens=far)
+    la = a.token_loss.cpu().numpy().reshape(w.batch, w.seq_len)
+    lc = c.token_loss.cpu().numpy().reshape(w.batch, w.seq_len)
+    assert la[b, t].view(np.uint32) == lc[b, t].view(np.uint32)
+    assert not np.array_equal(la[b], lc[b])
 
 
 def test_accumulate_doubles_gradient(B, R):
