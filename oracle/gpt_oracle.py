@@ -41,6 +41,24 @@ Where the pages are silent the plainest reading is taken:
 * MLP u = h W_up^T, a = max(u, 0)^2, y = a W_down^T (not gated);
 * loss = mean over all B*T positions of logsumexp(z) - z[target].
 
+FP8 forward (``fp8``; the page's training command line has an ``--fp8`` flag
+and names no scaling recipe).  Reading taken: the four block projections
+(W_qkv, W_o, W_up, W_down) multiply e4m3 operands in the forward; the
+embedding, lm_head and the whole backward stay as above.
+
+* quantizer input: the operand as the bf16 value the GPU stores (activations
+  rounded to bf16 here, weights are bf16 already) -- the same precision in
+  which the kernel takes its rounding decision;
+* scales: one per activation row (token), one per weight tensor, each the
+  largest power of two 2^k with amax * 2^k <= 448 (e4m3's largest finite
+  value; k = 0 for an all-zero row), so scaling and unscaling are exact;
+* code: round to the nearest e4m3 value (OCP E4M3: 4 exponent bits, bias 7,
+  3 mantissa bits, subnormals, no infinities), ties to the even code;
+* product: the dequantized operands multiplied exactly (fp64 here);
+* backward: the bf16 model's backward evaluated at the FP8 forward's
+  activations (dX = dY W and dW = dY^T X with the unquantized W and X), i.e.
+  the quantizer is taken as the identity (straight-through).
+
 Layout conventions shared with the library's documented ABI (not its code):
 W_qkv is [(n_head + 2 n_kv_head) hd, d] with the q rows first, then k, then v
 ([3d, d] without GQA); inside each block head h owns rows [h*hd, (h+1)*hd).
@@ -68,6 +86,9 @@ __all__ = [
     "causal_attention",
     "causal_attention_backward",
     "cross_entropy",
+    "e4m3_round",
+    "pow2_exponent",
+    "fp8_linear",
     "sequence_forward",
     "sequence_backward",
     "step",
@@ -90,6 +111,7 @@ class OracleConfig:
     qk_norm: bool = True
     n_kv_head: int = 0   # 0: n_head (multi-head attention)
     window: int = 0      # 0: full causal window
+    fp8: bool = False    # e4m3 operands in the block projections' forward
 
     @property
     def kv_heads(self) -> int:
@@ -101,7 +123,8 @@ def from_workload(w) -> OracleConfig:
         n_layer=w.n_layer, d_model=w.d_model, n_head=w.n_head, head_dim=w.head_dim,
         d_ff=w.d_ff, vocab=w.vocab, seq_len=w.seq_len, batch=w.batch,
         norm_eps=w.norm_eps, rope_base=w.rope_base, qk_norm=w.qk_norm,
-        n_kv_head=getattr(w, "n_kv_head", 0), window=getattr(w, "window", 0))
+        n_kv_head=getattr(w, "n_kv_head", 0), window=getattr(w, "window", 0),
+        fp8=bool(getattr(w, "fp8", False)))
 
 
 # ---------------------------------------------------------------------------
@@ -218,6 +241,67 @@ def causal_attention_backward(do, q, k, v, p):
     return back(dq), group(dk), group(dv)
 
 
+# ---------------------------------------------------------------------------
+# FP8 (e4m3) forward projections
+# ---------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+
+
+def _e4m3_table():
+    """Every finite non-negative e4m3 value (codes 0x00..0x7E) in increasing
+    order: exponent field e, mantissa m -> (m/8) 2^-6 if e == 0, else
+    (1 + m/8) 2^(e-7).  Code 0x7F is NaN."""
+    codes = np.arange(0x7F)
+    e, m = codes >> 3, codes & 7
+    vals = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    return vals, codes
+
+
+def e4m3_round(x: np.ndarray) -> np.ndarray:
+    """x rounded to the nearest e4m3 value, ties to the even code (|x| <= 448)."""
+    vals, codes = _e4m3_table()
+    a = np.abs(x)
+    hi_i = np.clip(np.searchsorted(vals, a), 1, len(vals) - 1)
+    lo, hi = vals[hi_i - 1], vals[hi_i]
+    up = (hi - a < a - lo) | ((hi - a == a - lo) & (codes[hi_i] % 2 == 0))
+    return np.sign(x) * np.where(up, hi, lo)
+
+
+def pow2_exponent(amax: np.ndarray) -> np.ndarray:
+    """The largest k with amax * 2^k <= 448 (0 where amax == 0), elementwise."""
+    amax = np.asarray(amax, dtype=np.float64)
+    safe = np.where(amax > 0, amax, 1.0)
+    _, e = np.frexp(E4M3_MAX / safe)       # 448/amax = f 2^e, f in [0.5, 1)
+    k = e.astype(np.int64) - 1
+    k = np.where(np.ldexp(safe, k) > E4M3_MAX, k - 1, k)     # exact fix-ups
+    k = np.where(np.ldexp(safe, k + 1) <= E4M3_MAX, k + 1, k)
+    return np.where(amax > 0, k, 0)
+
+
+def _round_bf16(x: np.ndarray) -> np.ndarray:
+    """Nearest bf16 value (ties to even), through the fp32 bit pattern."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    u = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
+    return u.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def fp8_linear(x: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """x W^T with both operands in e4m3: x [R, K] scaled per row, W [N, K]
+    (bf16 values) per tensor, by powers of two; the product is exact in fp64."""
+    xb = _round_bf16(x)
+    kx = pow2_exponent(np.max(np.abs(xb), axis=1))
+    kw = pow2_exponent(np.max(np.abs(w)))
+    xq = e4m3_round(np.ldexp(xb, kx[:, None]))
+    wq = e4m3_round(np.ldexp(w, kw))
+    return np.ldexp(xq, -kx[:, None]) @ np.ldexp(wq, -kw).T
+
+
+def _linear(cfg: "OracleConfig", x: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """One block projection, x W^T (F.linear without bias)."""
+    return fp8_linear(x, w) if cfg.fp8 else x @ w.T
+
+
 def cross_entropy(z: np.ndarray, y: np.ndarray):
     """Per-position loss logsumexp(z) - z[y] (max-shifted), plus lse and softmax."""
     m = np.max(z, axis=-1, keepdims=True)
@@ -256,7 +340,7 @@ def sequence_forward(cfg: OracleConfig, params: Dict[str, np.ndarray],
         wqkv, wo, wup, wdown = _layer_params(params, l)
         c = {"x_in": x}
         h, r1 = rms_norm(x, eps)                         # pre-attention norm
-        qkv = h @ wqkv.T                                 # F.linear, no bias
+        qkv = _linear(cfg, h, wqkv)                      # F.linear, no bias
         q = qkv[:, :d].reshape(T, H, hd)
         k = qkv[:, d:d + dkv].reshape(T, Hkv, hd)
         v = qkv[:, d + dkv:].reshape(T, Hkv, hd)
@@ -269,13 +353,14 @@ def sequence_forward(cfg: OracleConfig, params: Dict[str, np.ndarray],
             qn, rq, kn, rk = q, None, k, None
         o, p, lse = causal_attention(qn, kn, v, cfg.window)
         o2 = o.reshape(T, d)
-        x = x + o2 @ wo.T                                # attention residual
+        x = x + _linear(cfg, o2, wo)                     # attention residual
+        x_mid = x
         h2, r2 = rms_norm(x, eps)                        # pre-MLP norm
-        u = h2 @ wup.T
+        u = _linear(cfg, h2, wup)
         a = np.maximum(u, 0.0) ** 2                      # ReLU^2
-        x = x + a @ wdown.T                              # MLP residual
+        x = x + _linear(cfg, a, wdown)                   # MLP residual
         c.update(h=h, r1=r1, q=q, k=k, qn=qn, kn=kn, rq=rq, rk=rk, v=v, o=o2,
-                 lse=lse, x_mid=x - a @ wdown.T, h2=h2, r2=r2, u=u, a=a)
+                 lse=lse, x_mid=x_mid, h2=h2, r2=r2, u=u, a=a)
         layers.append(c)
 
     hf, rf = rms_norm(x, eps)                            # final norm

@@ -60,6 +60,7 @@ class Workload:
     qk_norm: bool = True
     n_kv_head: int = 0  # key/value heads (GQA); 0 = n_head
     window: int = 0     # sliding attention window in positions; 0 = full causal
+    fp8: bool = False   # e4m3 operands in the forward block projections
 
     @property
     def n_tokens(self) -> int:
