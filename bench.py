@@ -69,6 +69,8 @@ def workload_desc(w):
         extra += f", {w.n_kv_head} key/value heads"
     if w.window:
         extra += f", attention window {w.window}"
+    if w.fp8:
+        extra += ", e4m3 forward block projections"
     return (f"{w.name}: {w.n_layer} layers, d_model {w.d_model}, {w.n_head}x{w.head_dim} heads, "
             f"d_ff {w.d_ff}, vocab {w.vocab}, seq {w.seq_len}, batch {w.batch}{extra}")
 
@@ -216,12 +218,22 @@ def roofline(sites, w, gemm_tf, peak_tf, peaks):
             "peak": peak_tf, "unit": "TFLOP/s",
             "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel timed inside a long step)",
             "all_gemm_launches": {"achieved": round(gemm_tf, 1), "frac": round(gemm_tf / peak_tf, 4)}}
+    site_peak = peak_tf
+    if w.fp8:
+        # the site runs on e4m3 operands: the measured bf16 peak times the
+        # nominal e4m3 / bf16 dense ratio (4.5 / 2.25 PFLOP/s)
+        site_peak = 2.0 * peak_tf
+        line.update({"kernel": "gemm_pair_kernel (tcgen05 cta_group::2 GEMM, kind::f8f6f4 e4m3)",
+                     "peak": site_peak,
+                     "peak_source": f"{peaks['source']} bf16_tflops_sustained x 2 (nominal e4m3/bf16 ratio)",
+                     "all_gemm_launches": {"achieved": round(gemm_tf, 1), "mixed": "e4m3 forward, bf16 backward"}})
     if site and site["ms_per_launch"] > 0:
         tf = site["flops_per_launch"] / (site["ms_per_launch"] / 1e3) / 1e12
-        line.update({"achieved": round(tf, 1), "frac": round(tf / peak_tf, 4),
+        line.update({"achieved": round(tf, 1), "frac": round(tf / site_peak, 4),
                      "algorithmic_flops_per_launch": site["flops_per_launch"],
                      "traffic": UP_FWD_TRAFFIC_BYTES
-                     if (w.name, w.batch * w.seq_len, w.d_ff, w.d_model) == ("d24", 32768, 6144, 1536) else None})
+                     if (w.name, w.batch * w.seq_len, w.d_ff, w.d_model, w.fp8) == ("d24", 32768, 6144, 1536, False)
+                     else None})
     else:
         line.update({"achieved": round(gemm_tf, 1), "frac": round(gemm_tf / peak_tf, 4), "traffic": None})
     return line
@@ -305,6 +317,8 @@ def run_ours(args, rank, world, local_rank):
         w = w.replace(n_kv_head=args.kv_heads)
     if args.window:
         w = w.replace(window=args.window)
+    if args.fp8:
+        w = w.replace(fp8=True)
     wr = w.replace(seed=w.seed + 100 * rank)  # each replica its own batch
     cfg = B.config_from_workload(w)
     st = R.TrainStep(cfg, device=f"cuda:{local_rank}")
@@ -427,7 +441,7 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "bf16 + e4m3 forward block projections" if w.fp8 else "bf16",
         "data": "synthetic (Zipf(1.1) token ids, seeded N(0,0.02) bf16 weights)",
         "config": {"workload": workload_desc(w), "global_batch": w.batch * world,
                    "seq_len": w.seq_len, "tokens_per_step": N * world,
@@ -512,6 +526,8 @@ def main():
                          "variant; the line then reports it)")
     ap.add_argument("--window", type=int, default=0,
                     help="sliding attention window in positions (a model variant)")
+    ap.add_argument("--fp8", action="store_true",
+                    help="e4m3 operands in the forward block projections (a variant)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")

@@ -32,6 +32,7 @@ class GptConfig(ctypes.Structure):
         ("head_dim", ctypes.c_int32), ("d_ff", ctypes.c_int32), ("vocab", ctypes.c_int32),
         ("seq_len", ctypes.c_int32), ("batch", ctypes.c_int32), ("dtype", ctypes.c_int32),
         ("qk_norm", ctypes.c_int32), ("n_kv_head", ctypes.c_int32), ("attn_window", ctypes.c_int32),
+        ("fp8", ctypes.c_int32),
         ("rope_base", ctypes.c_float), ("norm_eps", ctypes.c_float),
         ("n_params", ctypes.c_int64), ("param_bytes", ctypes.c_uint64),
         ("workspace_bytes", ctypes.c_uint64),
@@ -116,10 +117,10 @@ def _check(rc: int, what: str) -> None:
 
 def make_config(n_layer, d_model, n_head, head_dim, d_ff, vocab, seq_len, batch,
                 dtype="bf16", qk_norm=True, rope_base=10000.0, norm_eps=1e-6,
-                n_kv_head=0, attn_window=0, check=True) -> GptConfig:
+                n_kv_head=0, attn_window=0, fp8=False, check=True) -> GptConfig:
     c = GptConfig(n_layer, d_model, n_head, head_dim, d_ff, vocab, seq_len, batch,
                   GPT_BF16 if dtype == "bf16" else GPT_F32, int(bool(qk_norm)),
-                  n_kv_head, attn_window, rope_base, norm_eps, 0, 0, 0)
+                  n_kv_head, attn_window, int(bool(fp8)), rope_base, norm_eps, 0, 0, 0)
     rc = lib().gpt_config_init(ctypes.byref(c))
     if check:
         _check(rc, "gpt_config_init")
@@ -130,7 +131,7 @@ def config_from_workload(w) -> GptConfig:
     """Config for a ``synth.Workload``-like object (shape fields + dtype)."""
     return make_config(w.n_layer, w.d_model, w.n_head, w.head_dim, w.d_ff, w.vocab, w.seq_len,
                        w.batch, w.dtype, w.qk_norm, w.rope_base, w.norm_eps,
-                       getattr(w, "n_kv_head", 0), getattr(w, "window", 0))
+                       getattr(w, "n_kv_head", 0), getattr(w, "window", 0), getattr(w, "fp8", False))
 
 
 def config_from_depth(depth: int, seq_len: int, batch: int, vocab: int) -> GptConfig:
@@ -232,7 +233,8 @@ def raw_backward(cfg, tokens, targets, params, workspace, grads, accumulate=0, s
 
 
 # ---- tracing ----------------------------------------------------------------
-GPT_K_NAMES = ["gemm", "attn_fwd", "attn_bwd", "norm", "qkv", "loss", "sort", "scatter", "other"]
+GPT_K_NAMES = ["gemm", "attn_fwd", "attn_bwd", "norm", "qkv", "loss", "sort", "scatter", "other",
+               "quant"]
 
 
 class GptTraceStat(ctypes.Structure):

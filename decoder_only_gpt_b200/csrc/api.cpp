@@ -121,6 +121,16 @@ bool make_layout(const gpt_config& c, Layout* L) {
   L->scat_items = b.take(L->scat_max_items * 8);
   L->scat_item_offs = b.take((V + 1) * 8);
   L->scat_partial = b.take((N / 64 + 1) * d * 4 * 2);
+  // e4m3 forward projections
+  if (c.fp8) {
+    L->w8 = b.take(uint64_t(c.param_bytes / 2));
+    L->w8_deq = b.take(4 * uint64_t(c.n_layer) * 4);
+    L->w8_amax = b.take(4 * uint64_t(c.n_layer) * 4);
+    L->a8 = b.take(N * std::max(d, F));
+    L->a8_deq = b.take(N * 4);
+  } else {
+    L->w8 = L->w8_deq = L->w8_amax = L->a8 = L->a8_deq = 0;
+  }
   // Muon's sum-of-squares partials and reciprocal norm
   if (c.dtype == GPT_BF16) {
     L->opt_x0 += L->layer_base;
@@ -166,6 +176,8 @@ int gpt_config_init(gpt_config* c) {
     return GPT_EINVAL;
   if (int64_t(c->n_head) * c->head_dim != c->d_model) return GPT_EINVAL;
   if (c->n_kv_head <= 0 || c->n_head % c->n_kv_head || c->attn_window < 0) return GPT_EINVAL;
+  if (c->fp8 != 0 && c->fp8 != 1) return GPT_EINVAL;
+  if (c->fp8 && c->dtype != GPT_BF16) return GPT_EUNSUPPORTED;
   if (!(c->rope_base > 1.f) || !(c->norm_eps > 0.f) || !std::isfinite(c->rope_base) ||
       !std::isfinite(c->norm_eps))
     return GPT_EINVAL;
@@ -297,7 +309,7 @@ static GemmArgs with_splitk(GemmArgs g, const Layout& L, char* ws) {
 // ---- traced launch wrappers: algorithmic FLOPs / HBM bytes per launch -------
 static int run_gemm(const gpt_config& c, const GemmArgs& g, cudaStream_t st) {
   const double e = c.dtype == GPT_BF16 ? 2.0 : 4.0;
-  double bytes = (double(g.M) * g.K + double(g.N) * g.K) * e;
+  double bytes = (double(g.M) * g.K + double(g.N) * g.K) * (g.fp8 ? 1.0 : e);
   const double mn = double(g.M) * g.N;
   switch (g.epi) {
     case EPI_STORE: bytes += mn * e * (g.beta ? 2 : 1); break;
@@ -352,6 +364,45 @@ struct Step {
   }
   double nd() const { return double(N) * d; }
 
+  // fp8 configs: e4m3 codes of every block matrix (per-tensor scales), once
+  // per forward, from the bf16 parameters
+  int quant_weights() {
+    for (int kind = 0; kind < 4; ++kind) {
+      const int tensor = GPT_T_WQKV + kind;
+      int64_t off0, r, cc, off1 = 0;
+      gpt_param_offset(c, tensor, 0, &off0, &r, &cc);
+      if (c->n_layer > 1) gpt_param_offset(c, tensor, 1, &off1, &r, &cc);
+      const int64_t stride = c->n_layer > 1 ? off1 - off0 : 0;
+      TraceScope ts(GPT_K_QUANT, 3, 0, double(c->n_layer) * r * cc * 5, st);
+      const int rc = launch_quant_tensors(p + off0 * esz, r * cc, stride, c->n_layer, ws + L.w8 + off0,
+                                          f(L.w8_deq) + kind * c->n_layer,
+                                          reinterpret_cast<unsigned*>(ws + L.w8_amax) + kind * c->n_layer,
+                                          st);
+      if (rc) return rc;
+    }
+    return 0;
+  }
+  // fp8 configs: one block projection of the bf16 activation `xact` [N, K]:
+  // quantize it per row into the scratch codes, then the e4m3 GEMM against the
+  // weight's codes; otherwise the bf16 GEMM as given
+  int projection(GemmArgs g, int tensor, int l) {
+    if (!c->fp8) return run_gemm(*c, g, st);
+    {
+      TraceScope ts(GPT_K_QUANT, 1, 0, double(N) * g.K * 3 + N * 4.0, st);
+      const int rc = launch_quant_rows(g.A, N, g.K, ws + L.a8, f(L.a8_deq), st);
+      if (rc) return rc;
+    }
+    int64_t off, r, cc;
+    gpt_param_offset(c, tensor, l, &off, &r, &cc);
+    g.A = ws + L.a8;
+    g.B = ws + L.w8 + off;
+    g.lda = g.ldb = g.K;
+    g.fp8 = true;
+    g.a_row_scale = f(L.a8_deq);
+    g.b_scale = f(L.w8_deq) + (tensor - GPT_T_WQKV) * c->n_layer + l;
+    return run_gemm(*c, g, st);
+  }
+
   int rms_fwd(void* h, float* r) {
     TraceScope ts(GPT_K_NORM, 1, 0, nd() * (4 + esz) + N * 4.0, st);
     return launch_rms_fwd(*c, x, h, r, st);
@@ -386,6 +437,7 @@ int gpt_forward_loss(const gpt_config* c, const int32_t* tok, const int32_t* tgt
   }
   const double attn_f = 4.0 * attn_pairs(*c) * c->head_dim;  // QK^T and PV, visible pairs
   const int Qc = int(qkv_cols(*c));
+  if (c->fp8 && c->n_layer > 0) GPT_TRY(S.quant_weights());
   for (int l = 0; l < c->n_layer; ++l) {
     char* Lb = S.layer(l);
     if (c->dtype == GPT_BF16) {
@@ -399,7 +451,7 @@ int gpt_forward_loss(const gpt_config* c, const int32_t* tok, const int32_t* tgt
       g.seq_len = c->seq_len; g.n_head = c->n_head; g.head_dim = c->head_dim;
       g.n_kv_head = c->n_kv_head;
       g.qk_norm = c->qk_norm; g.norm_eps = c->norm_eps;
-      GPT_TRY(run_gemm(*c, g, st));
+      GPT_TRY(S.projection(g, GPT_T_WQKV, l));
     } else {
       GPT_TRY(run_gemm(*c, gemm_kk(Lb + L.lo.h1, d, S.param(GPT_T_WQKV, l), d, N, Qc, d,
                                    EPI_STORE, ws + L.qkv_raw, Qc, S.status), st));
@@ -413,13 +465,13 @@ int gpt_forward_loss(const gpt_config* c, const int32_t* tok, const int32_t* tgt
       GPT_TRY(launch_attn_fwd(*c, Lb + L.lo.q, Lb + L.lo.k, Lb + L.lo.v, Lb + L.lo.o,
                               reinterpret_cast<float*>(Lb + L.lo.lse), S.status, st));
     }
-    GPT_TRY(run_gemm(*c, gemm_kk(Lb + L.lo.o, d, S.param(GPT_T_WO, l), d, N, d, d,
-                                 EPI_RESID_F32, S.x, d, S.status), st));
+    GPT_TRY(S.projection(gemm_kk(Lb + L.lo.o, d, S.param(GPT_T_WO, l), d, N, d, d,
+                                 EPI_RESID_F32, S.x, d, S.status), GPT_T_WO, l));
     GPT_TRY(S.rms_fwd(Lb + L.lo.h2, reinterpret_cast<float*>(Lb + L.lo.r2)));
-    GPT_TRY(run_gemm(*c, gemm_kk(Lb + L.lo.h2, d, S.param(GPT_T_WUP, l), d, N, F, d,
-                                 EPI_RELU2, Lb + L.lo.a, F, S.status), st));
-    GPT_TRY(run_gemm(*c, gemm_kk(Lb + L.lo.a, F, S.param(GPT_T_WDOWN, l), F, N, d, F,
-                                 EPI_RESID_F32, S.x, d, S.status), st));
+    GPT_TRY(S.projection(gemm_kk(Lb + L.lo.h2, d, S.param(GPT_T_WUP, l), d, N, F, d,
+                                 EPI_RELU2, Lb + L.lo.a, F, S.status), GPT_T_WUP, l));
+    GPT_TRY(S.projection(gemm_kk(Lb + L.lo.a, F, S.param(GPT_T_WDOWN, l), F, N, d, F,
+                                 EPI_RESID_F32, S.x, d, S.status), GPT_T_WDOWN, l));
     const bool last = l + 1 == c->n_layer;
     void* hn = last ? (void*)(ws + L.hf) : (void*)(S.layer(l + 1) + L.lo.h1);
     float* rn = reinterpret_cast<float*>(last ? ws + L.rf : S.layer(l + 1) + L.lo.r1);

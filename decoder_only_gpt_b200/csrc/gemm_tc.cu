@@ -223,8 +223,11 @@ __device__ __forceinline__ void epi_chunk(const GemmArgs& g, int row, int col0, 
 // are rotated by RoPE (pairs (i, i + hd/2)), scaled by 1/rms of the rotated row
 // (the rotation keeps the norm, so the sum of squares is taken on the raw row)
 // and written head-major, with the 1/rms kept for the backward.
+template <bool SCALED>
 __device__ __forceinline__ void epi_qkv_row(const GemmArgs& g, uint32_t taddr, int row,
-                                            int col_base, bool row_ok) {
+                                            int col_base, bool row_ok, float esc) {
+  // esc: the operands' dequantization factor of this row (8-bit operands only)
+  auto val = [&](uint32_t u) { return SCALED ? u2f(u) * esc : u2f(u); };
   const int hd = g.head_dim, half = hd / 2, H = g.n_head, Hkv = g.n_kv_head, T = g.seq_len;
   const int b = row_ok ? row / T : 0, t = row_ok ? row % T : 0;
   for (int seg = 0; seg < EC / hd; ++seg) {
@@ -247,8 +250,8 @@ __device__ __forceinline__ void epi_qkv_row(const GemmArgs& g, uint32_t taddr, i
 #pragma unroll
         for (int i = 0; i < 32; i += 8)
           *reinterpret_cast<uint4*>(vo + c + i) =
-              make_uint4(pack_bf16(u2f(u[i]), u2f(u[i + 1])), pack_bf16(u2f(u[i + 2]), u2f(u[i + 3])),
-                         pack_bf16(u2f(u[i + 4]), u2f(u[i + 5])), pack_bf16(u2f(u[i + 6]), u2f(u[i + 7])));
+              make_uint4(pack_bf16(val(u[i]), val(u[i + 1])), pack_bf16(val(u[i + 2]), val(u[i + 3])),
+                         pack_bf16(val(u[i + 4]), val(u[i + 5])), pack_bf16(val(u[i + 6]), val(u[i + 7])));
       }
       continue;
     }
@@ -258,7 +261,7 @@ __device__ __forceinline__ void epi_qkv_row(const GemmArgs& g, uint32_t taddr, i
       tc::tmem_ld_32x32b_x32(tcol + c, u);
       tc::tmem_wait_ld();
 #pragma unroll
-      for (int i = 0; i < 32; ++i) ss = fmaf(u2f(u[i]), u2f(u[i]), ss);
+      for (int i = 0; i < 32; ++i) ss = fmaf(val(u[i]), val(u[i]), ss);
     }
     const float r = g.qk_norm ? rsqrtf(ss / float(hd) + g.norm_eps) : 1.f;
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(part == 0 ? g.q_out : g.k_out) + dst;
@@ -283,8 +286,8 @@ __device__ __forceinline__ void epi_qkv_row(const GemmArgs& g, uint32_t taddr, i
       for (int e = 0; e < 8; ++e) {
         const float c0v = cv[2 * e], c1v = cv[2 * e + 1];
         const float s0v = sv[2 * e], s1v = sv[2 * e + 1];
-        const float a0 = u2f(ua[2 * e]), a1 = u2f(ua[2 * e + 1]);
-        const float b0 = u2f(ub[2 * e]), b1 = u2f(ub[2 * e + 1]);
+        const float a0 = val(ua[2 * e]), a1 = val(ua[2 * e + 1]);
+        const float b0 = val(ub[2 * e]), b1 = val(ub[2 * e + 1]);
         pa[e] = pack_bf16((a0 * c0v - b0 * s0v) * r, (a1 * c1v - b1 * s1v) * r);
         pb[e] = pack_bf16((a0 * s0v + b0 * c0v) * r, (a1 * s1v + b1 * c1v) * r);
       }
@@ -432,11 +435,16 @@ __device__ __forceinline__ void epi_chunk_coalesced(const GemmArgs& g, float* ti
 // Epilogue of one accumulator tile for one thread: row row0 + 32*quarter +
 // lane, columns col_base .. col_base + EC (TMEM columns taddr ..), K split sp
 // of `splits`; `part` indexes this column block's cross-entropy partials.
+template <bool SCALED>
 __device__ __forceinline__ void epilogue_tile(const GemmArgs& g, uint32_t taddr, int row0,
                                               int col_base, int part, int sp, int splits,
                                               int quarter, int lane, float* tile, int64_t obase) {
   const int row = row0 + quarter * 32 + lane;
   const bool row_ok = row < g.M;
+  // 8-bit operands: the accumulator times the row's and the weight's
+  // dequantization factors (powers of two)
+  float esc = 1.f;
+  if constexpr (SCALED) esc = (row_ok ? g.a_row_scale[row] : 0.f) * *g.b_scale;
   int tgt = -1;
   float lse_row = 0.f;
   if (row_ok && (g.epi == EPI_CE_FWD || g.epi == EPI_CE_BWD)) {
@@ -445,7 +453,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& g, uint32_t taddr,
   }
   float ce_max = -INFINITY, ce_sum = 0.f, ce_tgt = 0.f;
   if (g.epi == EPI_QKV) {
-    epi_qkv_row(g, taddr, row, col_base, row_ok);
+    epi_qkv_row<SCALED>(g, taddr, row, col_base, row_ok, esc);
     return;
   }
   if ((g.epi == EPI_CE_FWD || g.epi == EPI_CE_BWD) && splits == 1) {
@@ -476,8 +484,11 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& g, uint32_t taddr,
       tc::tmem_ld_32x32b_x32(taddr + c * 32, u);
       tc::tmem_wait_ld();
 #pragma unroll
-      for (int k = 0; k < 8; ++k)
-        *stage_at(tile, lane, k) = make_float4(u2f(u[4 * k]), u2f(u[4 * k + 1]), u2f(u[4 * k + 2]), u2f(u[4 * k + 3]));
+      for (int k = 0; k < 8; ++k) {
+        float4 v4 = make_float4(u2f(u[4 * k]), u2f(u[4 * k + 1]), u2f(u[4 * k + 2]), u2f(u[4 * k + 3]));
+        if constexpr (SCALED) { v4.x *= esc; v4.y *= esc; v4.z *= esc; v4.w *= esc; }
+        *stage_at(tile, lane, k) = v4;
+      }
       __syncwarp();
       const int col = col_base + c * 32 + 4 * u4;
       if (splits > 1) {
@@ -529,7 +540,7 @@ constexpr size_t kPairSmemBytes =
 static_assert(kPairSmemBytes <= 232448, "");
 }  // namespace
 
-template <bool AMN, bool BMN>
+template <bool AMN, bool BMN, bool F8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
                      const __grid_constant__ CUtensorMap map_b, const __grid_constant__ GemmArgs g,
@@ -548,9 +559,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int m_tiles = (g.M + P_BM - 1) / P_BM, n_tiles = (g.N + BN - 1) / BN;
   const int mn_tiles = m_tiles * n_tiles;  // per product; `g.batch` products
   const int num_units = mn_tiles * g.batch * splits;
-  const int num_kb = (g.K + BK - 1) / BK;
+  // a K-block is one 128-byte swizzle row of each operand: 64 bf16 or 128 e4m3
+  constexpr int BKE = F8 ? 2 * BK : BK;
+  static_assert(!F8 || (!AMN && !BMN), "8-bit operands are K-major");
+  const int num_kb = (g.K + BKE - 1) / BKE;
   const int kb_per = (num_kb + splits - 1) / splits;
-  constexpr uint32_t idesc = tc::idesc_bf16_f32(P_BM, BN, AMN, BMN);
+  constexpr uint32_t idesc =
+      F8 ? tc::idesc_e4m3_f32(P_BM, BN, AMN, BMN) : tc::idesc_bf16_f32(P_BM, BN, AMN, BMN);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < P_STAGES; ++s) {
@@ -601,16 +616,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           uint8_t* a_dst = smA + stage * P_HALF;
           uint8_t* b_dst = smB + stage * P_HALF;
           if (AMN) {
-            tc::tma_load_2d_pair(a_dst, &map_a, bar, m0, ay + kb * BK);
-            tc::tma_load_2d_pair(a_dst + 8192, &map_a, bar, m0 + 64, ay + kb * BK);
+            tc::tma_load_2d_pair(a_dst, &map_a, bar, m0, ay + kb * BKE);
+            tc::tma_load_2d_pair(a_dst + 8192, &map_a, bar, m0 + 64, ay + kb * BKE);
           } else {
-            tc::tma_load_2d_pair(a_dst, &map_a, bar, kb * BK, ay + m0);
+            tc::tma_load_2d_pair(a_dst, &map_a, bar, kb * BKE, ay + m0);
           }
           if (BMN) {
-            tc::tma_load_2d_pair(b_dst, &map_b, bar, n0, by + kb * BK);
-            tc::tma_load_2d_pair(b_dst + 8192, &map_b, bar, n0 + 64, by + kb * BK);
+            tc::tma_load_2d_pair(b_dst, &map_b, bar, n0, by + kb * BKE);
+            tc::tma_load_2d_pair(b_dst + 8192, &map_b, bar, n0 + 64, by + kb * BKE);
           } else {
-            tc::tma_load_2d_pair(b_dst, &map_b, bar, kb * BK, by + n0);
+            tc::tma_load_2d_pair(b_dst, &map_b, bar, kb * BKE, by + n0);
           }
           if (++stage == P_STAGES) { stage = 0; phase ^= 1; }
         }
@@ -646,10 +661,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint64_t da0 = tc::smem_desc_sw128(tc::smem_u32(smA + stage * P_HALF), AMN ? 8192 : 16);
           const uint64_t db0 = tc::smem_desc_sw128(tc::smem_u32(smB + stage * P_HALF), BMN ? 8192 : 16);
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
-            tc::mma_bf16_ss_pair_elect(d_tmem, tc::desc_advance(da0, AMN ? k * 2048 : k * 32),
-                                       tc::desc_advance(db0, BMN ? k * 2048 : k * 32), idesc,
-                                       (kb != kb_lo) || k != 0);
+          for (int k = 0; k < BK / 16; ++k) {  // 32 bytes of K per MMA, either type
+            if constexpr (F8)
+              tc::mma_f8_ss_pair_elect(d_tmem, tc::desc_advance(da0, k * 32), tc::desc_advance(db0, k * 32),
+                                       idesc, (kb != kb_lo) || k != 0);
+            else
+              tc::mma_bf16_ss_pair_elect(d_tmem, tc::desc_advance(da0, AMN ? k * 2048 : k * 32),
+                                         tc::desc_advance(db0, BMN ? k * 2048 : k * 32), idesc,
+                                         (kb != kb_lo) || k != 0);
+          }
           issued_any = true;
           const uint32_t e = tc::smem_u32(&tail->empty[stage]);
           tc::mma_commit_pair_elect(e);
@@ -694,7 +714,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       tc::tc_fence_after();
       const int bi = tile / mn_tiles, nb = tile % n_tiles;
-      epilogue_tile(g, tmem_base + (uint32_t(quarter * 32) << 16) + acc * BN + ch * EC,
+      epilogue_tile<F8>(g, tmem_base + (uint32_t(quarter * 32) << 16) + acc * BN + ch * EC,
                     ((tile % mn_tiles) / n_tiles) * P_BM + int(rank) * 128, nb * BN + ch * EC,
                     nb * (BN / EC) + ch, sp, splits, quarter, lane, stage_tile,
                     int64_t(bi) * g.o_bstride * g.ldo);
@@ -733,31 +753,35 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 
 // 2-D bf16 tensor [outer, inner] (inner contiguous, row pitch ld elements),
 // box [box_outer, box_inner], 128-byte swizzle, zero fill out of bounds.
+// [outer, inner] row-major, pitch ld elements; bf16, or one-byte elements
+// (e4m3 codes) when `bytes1`
 bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t ld,
-              uint32_t box_inner, uint32_t box_outer) {
+              uint32_t box_inner, uint32_t box_outer, bool bytes1 = false) {
   auto enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {ld * 2};
+  cuuint64_t strides[1] = {ld * (bytes1 ? 1 : 2)};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+  CUresult r = enc(m, bytes1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
-template <bool AMN, bool BMN>
+template <bool AMN, bool BMN, bool F8 = false>
 int launch_pair(const GemmArgs& g, int grid, int splits, cudaStream_t st) {
   CUtensorMap ma, mb;
   // batched products: the maps span every product's rows of the stacked arrays
   const uint64_t a_extra = uint64_t(g.batch - 1) * g.a_bstride, b_extra = uint64_t(g.batch - 1) * g.b_bstride;
+  constexpr uint32_t KB = F8 ? 128 : 64;  // K-block in elements: 128 bytes
   bool ok = AMN ? make_map(&ma, g.A, g.M, g.K + a_extra, g.lda, 64, 64)
-                : make_map(&ma, g.A, g.K, g.M + a_extra, g.lda, 64, 128);
+                : make_map(&ma, g.A, g.K, g.M + a_extra, g.lda, KB, 128, F8);
   ok = ok && (BMN ? make_map(&mb, g.B, g.N, g.K + b_extra, g.ldb, 64, 64)
-                  : make_map(&mb, g.B, g.K, g.N + b_extra, g.ldb, 64, 128));
+                  : make_map(&mb, g.B, g.K, g.N + b_extra, g.ldb, KB, 128, F8));
   if (!ok) return 1;
-  auto kern = gemm_pair_kernel<AMN, BMN>;
+  auto kern = gemm_pair_kernel<AMN, BMN, F8>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kPairSmemBytes)) !=
       cudaSuccess)
     return 1;
@@ -798,7 +822,7 @@ int num_sms() {
 // idle; the smallest split count that fills >= 90 % of the waves, keeping >= 8
 // k-blocks per split and the partials within the buffer.
 int gemm_tc_splits(const GemmArgs& g) {
-  if (g.epi != EPI_STORE || !g.splitk || g.ldo != g.N || (g.N & 3) || g.batch != 1) return 1;
+  if (g.epi != EPI_STORE || !g.splitk || g.ldo != g.N || (g.N & 3) || g.batch != 1 || g.fp8) return 1;
   const int pairs = num_sms() / 2;
   const int tiles = ((g.M + P_BM - 1) / P_BM) * ((g.N + BN - 1) / BN);
   const int num_kb = (g.K + BK - 1) / BK;
@@ -824,6 +848,16 @@ int launch_gemm_tc(const GemmArgs& g_in, void* stream) {
   GemmArgs g = g_in;
   cudaStream_t st = (cudaStream_t)stream;
   if (g.M <= 0 || g.N <= 0 || g.K <= 0 || g.batch <= 0) return 0;
+  if (g.fp8) {
+    // e4m3 operands: K-major A and B (16-byte aligned rows), one product, the
+    // dequantization factors given, no split; not the cross-entropy epilogues
+    if (g.a_mn_major || g.b_mn_major || g.batch != 1 || !g.a_row_scale || !g.b_scale ||
+        (g.lda | g.ldb) % 16 || g.epi == EPI_CE_FWD || g.epi == EPI_CE_BWD)
+      return 1;
+    const int tiles = ((g.M + P_BM - 1) / P_BM) * ((g.N + BN - 1) / BN);
+    const int pairs = num_sms() / 2;
+    return launch_pair<false, false, true>(g, 2 * (tiles < pairs ? tiles : pairs), 1, st);
+  }
   if (g.batch > 1) {
     // a partial K block would read the next product's rows; the other
     // epilogues are not batched

@@ -83,6 +83,12 @@ struct GemmArgs {
   // rows further down
   int batch = 1;
   int64_t a_bstride = 0, b_bstride = 0, o_bstride = 0;
+  // 8-bit operands (tensor-core GEMM, K-major A and B): A and B hold e4m3
+  // codes; the epilogue first multiplies the accumulator of row m by
+  // a_row_scale[m] * (*b_scale), the operands' dequantization factors
+  bool fp8 = false;
+  const float* a_row_scale = nullptr;
+  const float* b_scale = nullptr;
   // split-K (tensor-core GEMM, EPI_STORE only): fp32 partials [splits][M][N]
   float* splitk;
   int64_t splitk_floats;    // capacity of `splitk`
@@ -115,6 +121,11 @@ struct Layout {
   // optimizer scratch (bf16 configs): Newton-Schulz iterates, Gram matrices,
   // sum-of-squares partials
   uint64_t opt_x0, opt_x1, opt_a, opt_b, opt_part;
+  // e4m3 forward projections (fp8 configs): weight codes at the parameter
+  // buffer's element offsets (one byte each), their dequantization factors
+  // and amax bits [4 kinds][n_layer], one activation's codes [N, max(d, F)]
+  // and its per-row factors [N]
+  uint64_t w8, w8_deq, w8_amax, a8, a8_deq;
   uint64_t total;
 };
 
@@ -126,6 +137,9 @@ int launch_wait_expiry(int32_t* status, uint64_t limit_ns, void* stream);
 // ---- optimizer (csrc/optim.cu) ----
 constexpr int kOptNormBlocks = 296;  // fixed grid of the deterministic sum of squares
 int launch_optim_init(const void* params, float* master, float* m, float* v, int64_t n, void* stream);
+int launch_quant_rows(const void* x, int64_t rows, int cols, void* q, float* deq, void* stream);
+int launch_quant_tensors(const void* x, int64_t n, int64_t stride, int n_mat, void* q, float* deq,
+                         unsigned* amax_bits, void* stream);
 int launch_adamw(void* params, const void* grads, float* master, float* m, float* v, int64_t n,
                  float lr, float b1, float b2, float eps, float wd, float bc1, float bc2, void* stream);
 // M = mu M + G; U = nesterov ? G + mu M : M; x = bf16(U / (||U||_F + 1e-7)).

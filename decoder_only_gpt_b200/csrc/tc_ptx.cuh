@@ -289,6 +289,19 @@ __device__ __forceinline__ void mma_bf16_ss_pair_elect(uint32_t d_tmem, uint64_t
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// The same CTA-pair MMA on 8-bit floating-point operands (kind::f8f6f4: K = 32
+// per instruction, i.e. the same 32 bytes of each operand row as K = 16 bf16).
+__device__ __forceinline__ void mma_f8_ss_pair_elect(uint32_t d_tmem, uint64_t a_desc,
+                                                     uint64_t b_desc, uint32_t idesc,
+                                                     uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 __device__ __forceinline__ void mma_commit_pair_elect(uint32_t bar_cluster_addr) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"
@@ -324,6 +337,16 @@ __device__ __forceinline__ uint64_t desc_advance(uint64_t desc, uint32_t byte_of
 }
 
 // Instruction descriptor, kind::f16: bf16 x bf16 -> fp32, M x N tile.
+// kind::f8f6f4 with both operands e4m3 (format code 0), fp32 accumulation.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, bool a_mn, bool b_mn) {
+  return (1u << 4)                       // D format fp32
+         | (0u << 7)                     // A format e4m3
+         | (0u << 10)                    // B format e4m3
+         | (uint32_t(a_mn) << 15)
+         | (uint32_t(b_mn) << 16)
+         | (uint32_t(N >> 3) << 17)
+         | (uint32_t(M >> 4) << 24);
+}
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, bool b_mn) {
   return (1u << 4)                       // D format fp32
          | (1u << 7)                     // A format bf16

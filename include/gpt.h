@@ -108,6 +108,11 @@ typedef struct gpt_config {
                           divides n_head; 0 = n_head (set by gpt_config_init) */
   int32_t attn_window; /* sliding window: query i attends to keys i-W < j <= i
                           in every layer; 0 = the full causal window          */
+  int32_t fp8;         /* 1: the forward block projections (Wqkv, Wo, Wup,
+                          Wdown) multiply e4m3 operands -- activations scaled
+                          per row, weights per tensor, by powers of two -- and
+                          the backward stays bf16 (straight-through); bf16
+                          configs only                                        */
   float rope_base;  /* 10000 by default                                  */
   float norm_eps;   /* 1e-6 by default                                   */
   /* derived by gpt_config_init */
@@ -294,7 +299,8 @@ int gpt_optim_step(const gpt_config* cfg, const gpt_optim* opt, void* params, co
 #define GPT_K_SORT 6      /* stable counting sort of positions by token id    */
 #define GPT_K_SCATTER 7   /* embedding-gradient scatter-add                   */
 #define GPT_K_OTHER 8     /* RoPE table, status reset                          */
-#define GPT_K_COUNT 9
+#define GPT_K_QUANT 9     /* e4m3 quantization of projection operands (fp8)   */
+#define GPT_K_COUNT 10
 
 typedef struct gpt_trace gpt_trace;
 

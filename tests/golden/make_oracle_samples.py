@@ -6,7 +6,8 @@ Calls only ``oracle`` and ``synth``.  Stored: the loss, every per-position loss
 For ``wte`` half the coordinates are on rows that some token hits and half on
 rows that none hits (whose gradient must be exactly zero).
 
-Usage: python tests/golden/make_oracle_samples.py d12 [d24 ...]
+Usage: python tests/golden/make_oracle_samples.py d12 [d24 d24_kv4_w1024 ...]
+(a name is a workload, or one of VARIANTS: a workload with model overrides).
 """
 import os
 import sys
@@ -21,6 +22,19 @@ import oracle  # noqa: E402
 import synth  # noqa: E402
 
 SAMPLES_PER_TENSOR = 1024
+
+# block variants at full size: grouped-query attention with 4 key/value heads
+# and a 1024-position sliding window on the d24 model
+VARIANTS = {
+    "d24_kv4_w1024": ("d24", dict(n_kv_head=4, window=1024)),
+}
+
+
+def workload_of(name):
+    if name in VARIANTS:
+        base, kw = VARIANTS[name]
+        return synth.workload(base, **kw)
+    return synth.workload(name)
 
 
 def sample_coords(w, name, shape, tokens, rng):
@@ -38,7 +52,7 @@ def sample_coords(w, name, shape, tokens, rng):
 
 
 def main(name):
-    w = synth.workload(name)
+    w = workload_of(name)
     cfg = oracle.from_workload(w)
     tok, tgt = synth.make_tokens(w)
     params = synth.make_params(w)

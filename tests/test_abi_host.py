@@ -110,6 +110,19 @@ def test_gqa_and_window_config(B):
     assert f.n_kv_head == 2
 
 
+def test_fp8_config(B):
+    c = B.make_config(2, 256, 4, 64, 1024, 4096, 128, 2)
+    e = B.make_config(2, 256, 4, 64, 1024, 4096, 128, 2, fp8=True)
+    assert e.fp8 == 1 and e.param_bytes == c.param_bytes
+    # e4m3 weight codes (one byte per parameter) and one activation's codes
+    assert e.workspace_bytes >= c.workspace_bytes + c.param_bytes // 2 + 256 * 1024
+    bad = B.make_config(2, 64, 4, 16, 256, 256, 64, 4, dtype="f32", fp8=True, check=False)
+    assert B.lib().gpt_config_init(ctypes.byref(bad)) == B.GPT_EUNSUPPORTED
+    two = B.make_config(2, 256, 4, 64, 1024, 4096, 128, 2, check=False)
+    two.fp8 = 2
+    assert B.lib().gpt_config_init(ctypes.byref(two)) == B.GPT_EINVAL
+
+
 @pytest.mark.parametrize("name,kw", [("tiny", {}), ("story", {}), ("d24", {}),
                                      ("story", dict(n_kv_head=2, window=100)),
                                      ("tiny", dict(n_kv_head=1, window=3))])

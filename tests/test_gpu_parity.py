@@ -60,6 +60,14 @@ CASES = {
     "gqa_full": ("story", dict(n_layer=2, d_model=256, n_head=4, head_dim=64, n_kv_head=2,
                                d_ff=512, vocab=2048, seq_len=192, batch=2)),
     "tiny_gqa_window": ("tiny", dict(n_kv_head=2, window=9, seq_len=37, batch=3, vocab=100)),
+    # e4m3 forward projections against the oracle's e4m3 reading: the story
+    # model, ragged shapes (K = 320 ends in a partial 128-wide K block), and
+    # with GQA + window (the scaled QKV epilogue with fewer key/value heads)
+    "story_fp8": ("story", dict(fp8=True, batch=8)),
+    "ragged_fp8": ("story", dict(n_layer=2, d_model=128, n_head=2, head_dim=64, d_ff=320, vocab=1000,
+                                 seq_len=100, batch=3, fp8=True)),
+    "gqa_window_fp8": ("story", dict(n_layer=2, d_model=256, n_head=4, head_dim=64, n_kv_head=2,
+                                     window=100, d_ff=512, vocab=2048, seq_len=256, batch=2, fp8=True)),
 }
 
 
@@ -280,12 +288,23 @@ def _samples(name):
     return np.load(path)
 
 
-@pytest.mark.parametrize("name", ["d12", "d24"])
+def _sample_workload(name):
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("make_oracle_samples",
+                                                  os.path.join(GOLDEN, "make_oracle_samples.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod.workload_of(name)
+
+
+@pytest.mark.parametrize("name", ["d12", "d24", "d24_kv4_w1024"])
 def test_full_size_against_oracle_samples(B, R, name):
     """Full-size workloads in the benchmark's launch configuration: the loss, every
-    per-position loss, and gradient entries at the oracle's seeded coordinates."""
+    per-position loss, and gradient entries at the oracle's seeded coordinates
+    (d24_kv4_w1024: the d24 model with 4 key/value heads and a 1024-position
+    window, as ``bench.py --kv-heads 4 --window 1024`` runs it)."""
     s = _samples(name)
-    w = synth.workload(name)
+    w = _sample_workload(name)
     st, code = run_gpu(B, R, w)
     assert code == B.GPT_OK
     tol = TOL["bf16"]
