@@ -63,6 +63,23 @@ def load_peaks():
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
 
 
+def bench_workload(args):
+    """The workload both arms run: the named one with the command line's
+    model overrides (smaller profiling cases, the block and FP8 variants)."""
+    w = synth.workload(args.workload)
+    if args.batch:
+        w = w.replace(batch=args.batch)
+    if args.layers is not None:
+        w = w.replace(n_layer=args.layers)
+    if args.kv_heads:
+        w = w.replace(n_kv_head=args.kv_heads)
+    if args.window:
+        w = w.replace(window=args.window)
+    if args.fp8:
+        w = w.replace(fp8=True)
+    return w
+
+
 def workload_desc(w):
     extra = ""
     if w.n_kv_head and w.n_kv_head != w.n_head:
@@ -308,17 +325,7 @@ def run_ours(args, rank, world, local_rank):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
-    w = synth.workload(args.workload)
-    if args.batch:
-        w = w.replace(batch=args.batch)
-    if args.layers is not None:
-        w = w.replace(n_layer=args.layers)
-    if args.kv_heads:
-        w = w.replace(n_kv_head=args.kv_heads)
-    if args.window:
-        w = w.replace(window=args.window)
-    if args.fp8:
-        w = w.replace(fp8=True)
+    w = bench_workload(args)
     wr = w.replace(seed=w.seed + 100 * rank)  # each replica its own batch
     cfg = B.config_from_workload(w)
     st = R.TrainStep(cfg, device=f"cuda:{local_rank}")
@@ -471,7 +478,7 @@ def run_ours(args, rank, world, local_rank):
 def run_reference(args, rank):
     if rank != 0:
         return
-    w = synth.workload(args.workload)
+    w = bench_workload(args)
     setup = oracle_sample_setup(w, target_s=8.0)
     n = sample_tokens(setup)
     if args.warmup > 0:

@@ -23,10 +23,12 @@ import synth  # noqa: E402
 
 SAMPLES_PER_TENSOR = 1024
 
-# block variants at full size: grouped-query attention with 4 key/value heads
-# and a 1024-position sliding window on the d24 model
+# variants at full size: grouped-query attention with 4 key/value heads and a
+# 1024-position sliding window on the d24 model; the d24 model with e4m3
+# forward block projections
 VARIANTS = {
     "d24_kv4_w1024": ("d24", dict(n_kv_head=4, window=1024)),
+    "d24_fp8": ("d24", dict(fp8=True)),
 }
 
 
