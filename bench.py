@@ -220,8 +220,10 @@ def gemm_sites(records, w, steps):
 
 
 # DRAM bytes (read + write) of one up-projection forward launch at the bench
-# workload, from an ncu capture of the current CTA-pair GEMM kernel.
-UP_FWD_TRAFFIC_BYTES = 121_366_016 + 360_246_272
+# workload from an ncu capture, or None: the kernel has changed since the
+# last capture (batched products and the e4m3 instantiation were added), so
+# the counters no longer describe the code that runs.
+UP_FWD_TRAFFIC_BYTES = None
 
 
 def roofline(sites, w, gemm_tf, peak_tf, peaks):
@@ -250,7 +252,9 @@ def roofline(sites, w, gemm_tf, peak_tf, peaks):
                      "algorithmic_flops_per_launch": site["flops_per_launch"],
                      "traffic": UP_FWD_TRAFFIC_BYTES
                      if (w.name, w.batch * w.seq_len, w.d_ff, w.d_model, w.fp8) == ("d24", 32768, 6144, 1536, False)
-                     else None})
+                     else None,
+                     "traffic_note": "no ncu capture of the current kernel build (last capture: 481.6 MB per "
+                                     "launch on the build before batched products; profiles/gemm_up_fwd_d24.md)"})
     else:
         line.update({"achieved": round(gemm_tf, 1), "frac": round(gemm_tf / peak_tf, 4), "traffic": None})
     return line
