@@ -229,3 +229,32 @@ def test_wait_expiry_check_rejects():
     assert B.wait_expiry_check(fake + 16, 20_000_000) == B.GPT_EINVAL
     assert B.wait_expiry_check(fake, 10) == B.GPT_EINVAL
     assert B.wait_expiry_check(fake, 10**11) == B.GPT_EINVAL
+
+
+def test_struct_mirrors_match_the_header(B, tmp_path):
+    """The ctypes mirrors have the C layout: sizes and every field offset, as a
+    C compiler lays the header's structs out."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    mirrors = {"gpt_config": B.GptConfig, "gpt_optim": B.GptOptim,
+               "gpt_trace_stat": B.GptTraceStat, "gpt_trace_record": B.GptTraceRecord}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "gpt.h"', 'int main(void) {']
+    for cname, py in mirrors.items():
+        lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
+        for fname, _ in py._fields_:
+            lines.append(f'  printf("{cname} {fname} %zu\\n", offsetof({cname}, {fname}));')
+    lines += ['  return 0;', '}']
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)],
+                   check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
+    got = {tuple(l.split()[:2]): int(l.split()[2]) for l in out if l}
+    for cname, py in mirrors.items():
+        assert got[(cname, "size")] == ctypes.sizeof(py), cname
+        for fname, _ in py._fields_:
+            assert got[(cname, fname)] == getattr(py, fname).offset, (cname, fname)
