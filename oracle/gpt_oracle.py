@@ -88,7 +88,10 @@ __all__ = [
     "cross_entropy",
     "e4m3_round",
     "pow2_exponent",
+    "fp8_rows",
+    "fp8_tensor",
     "fp8_linear",
+    "fp8_weights",
     "sequence_forward",
     "sequence_backward",
     "step",
@@ -286,20 +289,43 @@ def _round_bf16(x: np.ndarray) -> np.ndarray:
     return u.astype(np.uint32).view(np.float32).astype(np.float64)
 
 
+def fp8_rows(x: np.ndarray) -> np.ndarray:
+    """The value an activation x [R, K] takes through e4m3: rounded to bf16,
+    scaled per row by a power of two, coded, unscaled."""
+    xb = _round_bf16(x)
+    kx = pow2_exponent(np.max(np.abs(xb), axis=1))
+    return np.ldexp(e4m3_round(np.ldexp(xb, kx[:, None])), -kx[:, None])
+
+
+def fp8_tensor(w: np.ndarray) -> np.ndarray:
+    """The value a weight W (bf16 values) takes through e4m3 with one
+    power-of-two scale for the whole tensor."""
+    kw = pow2_exponent(np.max(np.abs(w)))
+    return np.ldexp(e4m3_round(np.ldexp(w, kw)), -kw)
+
+
 def fp8_linear(x: np.ndarray, w: np.ndarray) -> np.ndarray:
     """x W^T with both operands in e4m3: x [R, K] scaled per row, W [N, K]
     (bf16 values) per tensor, by powers of two; the product is exact in fp64."""
-    xb = _round_bf16(x)
-    kx = pow2_exponent(np.max(np.abs(xb), axis=1))
-    kw = pow2_exponent(np.max(np.abs(w)))
-    xq = e4m3_round(np.ldexp(xb, kx[:, None]))
-    wq = e4m3_round(np.ldexp(w, kw))
-    return np.ldexp(xq, -kx[:, None]) @ np.ldexp(wq, -kw).T
+    return fp8_rows(x) @ fp8_tensor(w).T
 
 
-def _linear(cfg: "OracleConfig", x: np.ndarray, w: np.ndarray) -> np.ndarray:
-    """One block projection, x W^T (F.linear without bias)."""
-    return fp8_linear(x, w) if cfg.fp8 else x @ w.T
+def _linear(cfg: "OracleConfig", x: np.ndarray, w: np.ndarray,
+            w_fp8: Optional[np.ndarray] = None) -> np.ndarray:
+    """One block projection, x W^T (F.linear without bias); with fp8, the
+    e4m3 operands (w_fp8: W through e4m3, when already computed)."""
+    if not cfg.fp8:
+        return x @ w.T
+    return fp8_rows(x) @ (fp8_tensor(w) if w_fp8 is None else w_fp8).T
+
+
+def fp8_weights(cfg: "OracleConfig", params: Dict[str, np.ndarray]) -> Optional[Dict[str, np.ndarray]]:
+    """Every block matrix through e4m3 (fp8 configs; None otherwise): the
+    same for every sequence of a step, so computed once per step."""
+    if not cfg.fp8:
+        return None
+    names = [f"layers.{l}.{m}" for l in range(cfg.n_layer) for m in ("wqkv", "wo", "wup", "wdown")]
+    return {n: fp8_tensor(params[n]) for n in names}
 
 
 def cross_entropy(z: np.ndarray, y: np.ndarray):
@@ -322,7 +348,8 @@ def _layer_params(params, l):
 
 
 def sequence_forward(cfg: OracleConfig, params: Dict[str, np.ndarray],
-                     tok: np.ndarray, tgt: np.ndarray) -> dict:
+                     tok: np.ndarray, tgt: np.ndarray,
+                     w_fp8: Optional[Dict[str, np.ndarray]] = None) -> dict:
     """Forward pass of one sequence (tok, tgt: int [T]); returns a cache dict.
 
     The cache holds what the backward needs plus the per-position loss
@@ -332,6 +359,9 @@ def sequence_forward(cfg: OracleConfig, params: Dict[str, np.ndarray],
     d, H, hd, Hkv = cfg.d_model, cfg.n_head, cfg.head_dim, cfg.kv_heads
     dkv = Hkv * hd
     eps = cfg.norm_eps
+    if w_fp8 is None:
+        w_fp8 = fp8_weights(cfg, params)
+    wq = (lambda name: w_fp8[name]) if w_fp8 is not None else (lambda name: None)
     cos, sin = rope_tables(T, hd, cfg.rope_base)
 
     x = params["wte"][tok].astype(np.float64)           # token embedding gather
@@ -340,7 +370,7 @@ def sequence_forward(cfg: OracleConfig, params: Dict[str, np.ndarray],
         wqkv, wo, wup, wdown = _layer_params(params, l)
         c = {"x_in": x}
         h, r1 = rms_norm(x, eps)                         # pre-attention norm
-        qkv = _linear(cfg, h, wqkv)                      # F.linear, no bias
+        qkv = _linear(cfg, h, wqkv, wq(f"layers.{l}.wqkv"))  # F.linear, no bias
         q = qkv[:, :d].reshape(T, H, hd)
         k = qkv[:, d:d + dkv].reshape(T, Hkv, hd)
         v = qkv[:, d + dkv:].reshape(T, Hkv, hd)
@@ -353,12 +383,12 @@ def sequence_forward(cfg: OracleConfig, params: Dict[str, np.ndarray],
             qn, rq, kn, rk = q, None, k, None
         o, p, lse = causal_attention(qn, kn, v, cfg.window)
         o2 = o.reshape(T, d)
-        x = x + _linear(cfg, o2, wo)                     # attention residual
+        x = x + _linear(cfg, o2, wo, wq(f"layers.{l}.wo"))  # attention residual
         x_mid = x
         h2, r2 = rms_norm(x, eps)                        # pre-MLP norm
-        u = _linear(cfg, h2, wup)
+        u = _linear(cfg, h2, wup, wq(f"layers.{l}.wup"))
         a = np.maximum(u, 0.0) ** 2                      # ReLU^2
-        x = x + _linear(cfg, a, wdown)                   # MLP residual
+        x = x + _linear(cfg, a, wdown, wq(f"layers.{l}.wdown"))  # MLP residual
         c.update(h=h, r1=r1, q=q, k=k, qn=qn, kn=kn, rq=rq, rk=rk, v=v, o=o2,
                  lse=lse, x_mid=x_mid, h2=h2, r2=r2, u=u, a=a)
         layers.append(c)
@@ -443,13 +473,14 @@ def step(cfg: OracleConfig, params: Dict[str, np.ndarray], tokens: np.ndarray,
     B, T = tokens.shape
     denom = loss_denominator if loss_denominator is not None else B * T
     rows = list(range(B)) if rows is None else list(rows)
+    w_fp8 = fp8_weights(cfg, params)
     grads = None
     if backward:
         grads = {name: np.zeros_like(p, dtype=np.float64) for name, p in params.items()}
     token_loss = np.zeros((len(rows), T))
     caches = [] if keep_caches else None
     for i, b in enumerate(rows):
-        cache = sequence_forward(cfg, params, tokens[b], targets[b])
+        cache = sequence_forward(cfg, params, tokens[b], targets[b], w_fp8)
         token_loss[i] = cache["token_loss"]
         if backward:
             sequence_backward(cfg, params, cache, 1.0 / denom, grads)
