@@ -15,8 +15,12 @@ inline int64_t qkv_cols(const gpt_config& c) {
   return int64_t(c.n_head + 2 * c.n_kv_head) * c.head_dim;
 }
 // The sliding window as a key-distance bound: query i sees keys j with
-// i - j < window_span(c) (a span longer than any sequence when unset).
-inline int window_span(const gpt_config& c) { return c.attn_window > 0 ? c.attn_window : (1 << 30); }
+// i - j < window_span(c).  A window of T or more positions (or none) is the
+// full causal window, so the span is capped at T, which also keeps the
+// kernels' key and query bounds (position + span) far from int overflow.
+inline int window_span(const gpt_config& c) {
+  return c.attn_window > 0 && c.attn_window < c.seq_len ? c.attn_window : c.seq_len;
+}
 
 // Kernel ids recorded in gpt_device_status::where.
 enum KernelId : int32_t {
