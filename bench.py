@@ -157,7 +157,9 @@ def oracle_sample_setup(w, bits=None, target_s=10.0):
     import oracle
     if bits is None:
         bits = synth.make_params(w, as_bits=True)
-    params = {k: synth.bf16_bits_to_f64(v) for k, v in bits.items()}
+    # bf16 workloads: the stored bit patterns; fp32 workloads: the fp32 values
+    params = {k: synth.bf16_bits_to_f64(v) if w.dtype == "bf16" else np.asarray(v, dtype=np.float64)
+              for k, v in bits.items()}
     tok, tgt = synth.make_tokens(w)
 
     def setup(n):
