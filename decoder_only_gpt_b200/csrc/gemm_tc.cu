@@ -751,10 +751,9 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
-// 2-D bf16 tensor [outer, inner] (inner contiguous, row pitch ld elements),
-// box [box_outer, box_inner], 128-byte swizzle, zero fill out of bounds.
-// [outer, inner] row-major, pitch ld elements; bf16, or one-byte elements
-// (e4m3 codes) when `bytes1`
+// 2-D tensor [outer, inner] (inner contiguous, row pitch ld elements) of bf16,
+// or of one-byte elements (e4m3 codes) when `bytes1`; box [box_outer,
+// box_inner], 128-byte swizzle, zero fill out of bounds.
 bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t ld,
               uint32_t box_inner, uint32_t box_outer, bool bytes1 = false) {
   auto enc = get_encode();
