@@ -7,9 +7,10 @@ Facts fixed outside the oracle's code:
 * the power-of-two scale: amax * 2^k <= 448 < amax * 2^(k+1);
 * operands already on the scaled e4m3 grid pass through exactly;
 * the product's error stays inside the bound two e4m3 roundings allow;
-* the whole step against torch float64 autograd in which each block
-  projection quantizes through torch's float8 cast, bf16 cast and frexp, with
-  the straight-through backward written as its own autograd function.
+* the whole step (multi-head, and grouped-query with a window) against torch
+  float64 autograd in which each block projection quantizes through torch's
+  bf16 and float8 casts with a log2-derived exponent, the straight-through
+  backward written as its own autograd function.
 """
 import math
 
@@ -111,7 +112,11 @@ def _torch_fp8_step(w, params, tok, tgt):
 
     t = {k: torch.tensor(v, dtype=torch.float64, requires_grad=True) for k, v in params.items()}
     B, T = tok.shape
-    d, H, hd = w.d_model, w.n_head, w.head_dim
+    d, H, hd, Hkv = w.d_model, w.n_head, w.head_dim, w.n_kv_head or w.n_head
+    pos = torch.arange(T)
+    mask = pos[None, :] <= pos[:, None]
+    if w.window:
+        mask &= (pos[:, None] - pos[None, :]) < w.window
     i = torch.arange(hd // 2, dtype=torch.float64)
     ang = torch.arange(T, dtype=torch.float64)[:, None] * (w.rope_base ** (-2.0 * i / hd))[None]
     cos, sin = torch.cos(ang)[None, :, None, :], torch.sin(ang)[None, :, None, :]
@@ -126,12 +131,12 @@ def _torch_fp8_step(w, params, tok, tgt):
     x = t["wte"][torch.tensor(tok, dtype=torch.long)]
     for l in range(w.n_layer):
         qkv = Fp8Linear.apply(norm(x), t[f"layers.{l}.wqkv"])
-        qq, kk, vv = qkv.split(d, dim=-1)
+        qq, kk, vv = qkv.split([d, Hkv * hd, Hkv * hd], dim=-1)
         qq = norm(rot(qq.view(B, T, H, hd)))
-        kk = norm(rot(kk.view(B, T, H, hd)))
-        vv = vv.view(B, T, H, hd)
+        kk = norm(rot(kk.view(B, T, Hkv, hd)))
+        vv = vv.view(B, T, Hkv, hd)
         o = F.scaled_dot_product_attention(qq.transpose(1, 2), kk.transpose(1, 2), vv.transpose(1, 2),
-                                           is_causal=True)
+                                           attn_mask=mask, enable_gqa=True)
         x = x + Fp8Linear.apply(o.transpose(1, 2).reshape(B, T, d), t[f"layers.{l}.wo"])
         u = Fp8Linear.apply(norm(x), t[f"layers.{l}.wup"])
         x = x + Fp8Linear.apply(torch.relu(u).square(), t[f"layers.{l}.wdown"])
@@ -142,7 +147,8 @@ def _torch_fp8_step(w, params, tok, tgt):
 
 
 @pytest.mark.parametrize("kw", [dict(n_layer=2, seq_len=48, batch=2, vocab=512),
-                                dict(n_layer=1, seq_len=33, batch=3, vocab=300, d_ff=320)])
+                                dict(n_layer=1, seq_len=33, batch=3, vocab=300, d_ff=320),
+                                dict(n_layer=2, seq_len=40, batch=2, vocab=256, n_kv_head=2, window=9)])
 def test_fp8_step_matches_torch_casts_and_straight_through(kw):
     w = synth.workload("story", fp8=True, **kw)
     tok, tgt = synth.make_tokens(w)
