@@ -25,6 +25,13 @@ GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
 TOL = {
     "bf16": dict(loss=1e-3, cos=0.999, maxrel=3e-2, tok=2e-2),
+    # e4m3 forward projections at full d24 size: an e4m3 code turns the
+    # bf16-level difference between the GPU's and the oracle's quantizer
+    # inputs into a whole code step; the oracle with those inputs perturbed by
+    # 1e-3 relative noise moved per-position losses by up to 3.4e-2 and the
+    # embedding gradient to cosine 0.9985 / max-rel 3.9e-2 (d24, 2 sequences),
+    # so the bars are about twice that (the loss itself moved 1e-4)
+    "fp8_full": dict(loss=1e-3, cos=0.995, maxrel=8e-2, tok=8e-2),
     "f32": dict(loss=1e-5, cos=0.99999, maxrel=1e-3, tok=1e-4),
 }
 
@@ -297,17 +304,18 @@ def _sample_workload(name):
     return mod.workload_of(name)
 
 
-@pytest.mark.parametrize("name", ["d12", "d24", "d24_kv4_w1024"])
+@pytest.mark.parametrize("name", ["d12", "d24", "d24_kv4_w1024", "d24_fp8"])
 def test_full_size_against_oracle_samples(B, R, name):
     """Full-size workloads in the benchmark's launch configuration: the loss, every
     per-position loss, and gradient entries at the oracle's seeded coordinates
     (d24_kv4_w1024: the d24 model with 4 key/value heads and a 1024-position
-    window, as ``bench.py --kv-heads 4 --window 1024`` runs it)."""
+    window, as ``bench.py --kv-heads 4 --window 1024`` runs it; d24_fp8: e4m3
+    forward projections, as ``bench.py --fp8`` runs it, with the e4m3 bars)."""
     s = _samples(name)
     w = _sample_workload(name)
     st, code = run_gpu(B, R, w)
     assert code == B.GPT_OK
-    tol = TOL["bf16"]
+    tol = TOL["fp8_full"] if w.fp8 else TOL["bf16"]
     loss = float(st.loss.cpu()[0])
     assert abs(loss - float(s["loss"])) / float(s["loss"]) <= tol["loss"]
     tl = st.token_loss.cpu().numpy().astype(np.float64).reshape(w.batch, w.seq_len)
