@@ -5,7 +5,11 @@ One step = gpt_forward_loss + gpt_backward (every gradient written, no
 optimizer) on one synthetic batch of 16 x 2048 tokens (Zipf(1.1) ids, seeded
 N(0, 0.02) bf16 weights).  Inputs are resident in HBM when the timed region
 starts; the step touches tens of GB, far more than the 126 MB L2, so no L2
-flush is needed between steps.
+flush is needed between steps.  The headline region runs without the
+per-launch trace; a second pass with the trace attached gives the per-kernel
+breakdown.  Default runs also measure the depth-12 model (key "d12"), the
+other depth the metric names.  MFU is against the nominal dense bf16 peak
+(2.25 PFLOP/s), with the fraction of the measured sustained peak beside it.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -36,6 +40,7 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 WORKLOAD = "d24"
+SECOND_WORKLOAD = "d12"  # the metric names depth 12 and 24: d12 rides along in default runs
 METRIC = "train tokens/sec (fwd+bwd) on 1 B200 for depth-12/24 GPT; MFU vs bf16 peak"
 
 
@@ -221,18 +226,17 @@ def gemm_sites(records, w, steps):
             for n, v in acc.items()}
 
 
-# DRAM bytes (read + write) of one up-projection forward launch at the bench
-# workload from an ncu capture, or None: the kernel has changed since the
-# last capture (batched products and the e4m3 instantiation were added), so
-# the counters no longer describe the code that runs.
-UP_FWD_TRAFFIC_BYTES = None
+# DRAM bytes (read + write) of one launch of the dominant kernel's roofline
+# site, from an ncu capture of the current kernel build, keyed by (workload,
+# site, fp8); a site that has not been captured reports null.
+TRAFFIC_BYTES = {}
 
 
 def roofline(sites, w, gemm_tf, peak_tf, peaks):
     """Roofline of the dominant kernel, the tcgen05 CTA-pair GEMM: its
     up-projection forward launch (M = B*T, N = d_ff, K = d_model, ReLU^2
-    epilogue), timed live by the trace inside the step; the all-launch GEMM
-    figure rides along."""
+    epilogue), timed by the trace pass's CUDA events on the launching stream;
+    the all-launch GEMM figure rides along."""
     site = (sites or {}).get("up_fwd")
     line = {"bound": "tensor", "kernel": "gemm_pair_kernel (tcgen05 cta_group::2 GEMM)",
             "site": f"up-projection forward: M={w.batch * w.seq_len} N={w.d_ff} K={w.d_model}",
@@ -250,13 +254,13 @@ def roofline(sites, w, gemm_tf, peak_tf, peaks):
                      "all_gemm_launches": {"achieved": round(gemm_tf, 1), "mixed": "e4m3 forward, bf16 backward"}})
     if site and site["ms_per_launch"] > 0:
         tf = site["flops_per_launch"] / (site["ms_per_launch"] / 1e3) / 1e12
+        key = (w.name, w.batch * w.seq_len, w.d_ff, w.d_model, bool(w.fp8))
         line.update({"achieved": round(tf, 1), "frac": round(tf / site_peak, 4),
                      "algorithmic_flops_per_launch": site["flops_per_launch"],
-                     "traffic": UP_FWD_TRAFFIC_BYTES
-                     if (w.name, w.batch * w.seq_len, w.d_ff, w.d_model, w.fp8) == ("d24", 32768, 6144, 1536, False)
-                     else None,
-                     "traffic_note": "no ncu capture of the current kernel build (last capture: 481.6 MB per "
-                                     "launch on the build before batched products; profiles/gemm_up_fwd_d24.md)"})
+                     "algorithmic_bytes_per_launch": (1 if w.fp8 else 2) * (w.batch * w.seq_len * w.d_model
+                                                                           + w.d_ff * w.d_model)
+                                                     + 2 * w.batch * w.seq_len * w.d_ff,
+                     "traffic": TRAFFIC_BYTES.get(key)})
     else:
         line.update({"achieved": round(gemm_tf, 1), "frac": round(gemm_tf / peak_tf, 4), "traffic": None})
     return line
@@ -318,33 +322,24 @@ def replica_throughput(tokens_per_step, steps, world, max_ms):
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
-def run_ours(args, rank, world, local_rank):
+def measure(w, args, rank, world, dev, barrier, *, optimizer=False, e2e=True):
+    """Time one workload: an untraced timed region (the headline), then a
+    second pass with the per-launch trace attached (the per-kernel breakdown
+    and the roofline site), then the end-to-end host-buffer pass."""
     import torch
-    import torch.distributed as dist
 
     from decoder_only_gpt_b200 import binding as B
     from decoder_only_gpt_b200 import runtime as R
 
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
-
-    w = bench_workload(args)
     wr = w.replace(seed=w.seed + 100 * rank)  # each replica its own batch
     cfg = B.config_from_workload(w)
-    st = R.TrainStep(cfg, device=f"cuda:{local_rank}")
+    st = R.TrainStep(cfg, device=str(dev))
     bits = synth.make_params(w, as_bits=True)
     st.load_params(bits)
     tok, tgt = synth.make_tokens(wr)
     st.set_batch(tok, tgt)
     N = w.batch * w.seq_len
     stream = torch.cuda.current_stream(dev)
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
 
     for _ in range(args.warmup):
         st.step()
@@ -353,8 +348,6 @@ def run_ours(args, rank, world, local_rank):
     if code != B.GPT_OK:
         raise SystemExit(f"device status after warm-up: {B.strerror(code)}")
 
-    per_step = 600
-    trace = B.Trace(capacity=per_step * args.steps + 16)
     bus = None
     try:
         bus = torch.cuda.get_device_properties(dev).pci_bus_id
@@ -362,80 +355,145 @@ def run_ours(args, rank, world, local_rank):
         bus = None
     clocks = ClockSampler(bus if isinstance(bus, str) else None)
 
-    # ---- timed region (device time, CUDA events on the launching stream) ----
+    # ---- timed region (device time, CUDA events on the launching stream; no trace) ----
     barrier()
     torch.cuda.synchronize()
     clocks.start()
     time.sleep(0.3)
-    trace.attach()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
         st.step()
     e1.record(stream)
     torch.cuda.synchronize()
-    B.Trace.detach()
     barrier()
     clk = clocks.stop()
     ms = e0.elapsed_time(e1)
     code = st.status()
     if code != B.GPT_OK:
         raise SystemExit(f"device status after timed steps: {B.strerror(code)}")
+
+    # ---- the same steps again with every launch timed (breakdown only) ----
+    per_step = 600
+    trace = B.Trace(capacity=per_step * args.steps + 16)
+    barrier()
+    torch.cuda.synchronize()
+    trace.attach()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        st.step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    B.Trace.detach()
+    traced_ms = t0.elapsed_time(t1)
     stats, dropped = trace.summary()
     records = trace.records(per_step * args.steps + 16)
     trace.close()
     sites = gemm_sites(records, w, args.steps)
 
     # ---- end to end through the public host-buffer call ----
-    ht = torch.from_numpy(tok.ravel().copy()).pin_memory()
-    hy = torch.from_numpy(tgt.ravel().copy()).pin_memory()
-    hl = torch.zeros(1, dtype=torch.float32).pin_memory()
-    B.train_step_host(cfg, ht, hy, st.params, st.workspace, st.grads, hl, stream=stream.cuda_stream)
-    torch.cuda.synchronize()
-    barrier()
-    torch.cuda.synchronize()
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    for _ in range(args.steps):
-        B.train_step_host(cfg, ht, hy, st.params, st.workspace, st.grads, hl,
-                          stream=stream.cuda_stream)
-        stream.synchronize()  # the loss is read on the host every step
-        assert math.isfinite(float(hl[0]))
-    f1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    e2e_ms = f0.elapsed_time(f1)
+    e2e_ms = None
+    if e2e:
+        ht = torch.from_numpy(tok.ravel().copy()).pin_memory()
+        hy = torch.from_numpy(tgt.ravel().copy()).pin_memory()
+        hl = torch.zeros(1, dtype=torch.float32).pin_memory()
+        B.train_step_host(cfg, ht, hy, st.params, st.workspace, st.grads, hl, stream=stream.cuda_stream)
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.steps):
+            B.train_step_host(cfg, ht, hy, st.params, st.workspace, st.grads, hl,
+                              stream=stream.cuda_stream)
+            stream.synchronize()  # the loss is read on the host every step
+            assert math.isfinite(float(hl[0]))
+        f1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = f0.elapsed_time(f1)
 
     # ---- optimizer step (AdamW + Muon), timed on its own: not part of the
     # fwd+bwd metric; single-GPU runs only ----
     optim = None
-    if world == 1 and not args.no_optimizer and cfg.dtype == B.GPT_BF16:
+    if optimizer and world == 1 and cfg.dtype == B.GPT_BF16:
         optim = time_optimizer(B, st, stream)
 
-    if world > 1:
-        ms, e2e_ms = max_over_ranks([ms, e2e_ms], dev)
-        dist.barrier()
-        dist.destroy_process_group()
-    if rank != 0:
-        return
+    out = dict(w=w, N=N, ms=ms, traced_ms=traced_ms, e2e_ms=e2e_ms, stats=stats, dropped=dropped,
+               sites=sites, clk=clk, optim=optim, bits=bits)
+    del st
+    torch.cuda.empty_cache()
+    return out
 
-    peaks = load_peaks()
+
+def summarize(m, args, world, peaks):
+    """Throughput, MFU and the per-kernel breakdown of one measured workload."""
+    w, N, ms = m["w"], m["N"], m["ms"]
     tok_s = replica_throughput(N, args.steps, world, ms)
     fpt = flops_per_token(w)
+    stats = m["stats"]
     g = stats["gemm"]
     gemm_tf = g["flops"] / (g["ms"] / 1e3) / 1e12 if g["ms"] > 0 else 0.0
     peak_tf = peaks["bf16_tflops_sustained"]
-    kernels = sum(s["kernels"] for s in stats.values())
     breakdown = {k: {"ms_per_step": round(v["ms"] / args.steps, 3),
                      "launches_per_step": v["launches"] // max(args.steps, 1),
                      **({"tflops": round(v["flops"] / (v["ms"] / 1e3) / 1e12, 1)} if v["flops"] and v["ms"] else {}),
                      **({"gbs": round(v["bytes"] / (v["ms"] / 1e3) / 1e9, 1)} if not v["flops"] and v["ms"] else {})}
                  for k, v in stats.items() if v["launches"]}
+    kernels_per_step = sum(s["kernels"] for s in stats.values()) / max(args.steps, 1)
+    return dict(tok_s=tok_s, fpt=fpt, gemm_tf=gemm_tf, peak_tf=peak_tf, breakdown=breakdown,
+                kernels_per_step=kernels_per_step,
+                mfu=round(tok_s / world * fpt / NOMINAL_BF16_FLOPS, 4),
+                mfu_measured=round(tok_s / world * fpt / (peak_tf * 1e12), 4))
+
+
+# nominal dense bf16 tensor-core peak of one B200 (public datasheet figure)
+NOMINAL_BF16_FLOPS = 2.25e15
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    w = bench_workload(args)
+    main_m = measure(w, args, rank, world, dev, barrier, optimizer=not args.no_optimizer)
+    # the other depth the metric names, after the headline one (default runs)
+    second = None
+    if not args.no_second and args.workload == WORKLOAD and not (args.layers or args.batch or args.kv_heads
+                                                                  or args.window or args.fp8):
+        second = measure(synth.workload(SECOND_WORKLOAD), args, rank, world, dev, barrier, e2e=False)
+
+    ms, e2e_ms = main_m["ms"], main_m["e2e_ms"]
+    ms2 = second["ms"] if second else 0.0
+    if world > 1:
+        ms, e2e_ms, ms2 = max_over_ranks([ms, e2e_ms, ms2], dev)
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    main_m["ms"], main_m["e2e_ms"] = ms, e2e_ms
+    if second:
+        second["ms"] = ms2
+
+    peaks = load_peaks()
+    s = summarize(main_m, args, world, peaks)
+    N = main_m["N"]
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only) ----
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        setup = oracle_sample_setup(w, bits)
+        setup = oracle_sample_setup(w, main_m["bits"])
         n = sample_tokens(setup)
         secs = time_oracle(setup)
         cpu = {"value": round(n / secs, 3), "unit": "tokens/s",
@@ -445,7 +503,7 @@ def run_ours(args, rank, world, local_rank):
 
     line = {
         "metric": METRIC,
-        "value": round(tok_s, 1),
+        "value": round(s["tok_s"], 1),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -459,22 +517,34 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": workload_desc(w), "global_batch": w.batch * world,
                    "seq_len": w.seq_len, "tokens_per_step": N * world,
                    "parallelism": f"replicas only x{world}" if world > 1 else "single GPU",
-                   "l2": "no flush: every step moves tens of GB, far above the 126 MB L2"},
-        "mfu": round(tok_s / world * fpt / (peak_tf * 1e12), 4),
-        "mfu_vs_nominal_2250tf": round(tok_s / world * fpt / 2.25e15, 4),
-        "flops_per_token": fpt,
-        "roofline": roofline(sites, w, gemm_tf, peak_tf, peaks),
-        "kernel_breakdown": breakdown,
-        "gemm_sites": sites,
-        "gpu_launches": kernels,
-        "trace_dropped": dropped,
+                   "l2": "no flush: every step moves tens of GB, far above the 126 MB L2",
+                   "timing": "headline untraced; breakdown and roofline from a second, traced pass"},
+        "mfu": s["mfu"],
+        "mfu_peak": "nominal dense bf16 2.25 PFLOP/s",
+        "mfu_vs_measured_sustained": s["mfu_measured"],
+        "flops_per_token": s["fpt"],
+        "roofline": roofline(main_m["sites"], w, s["gemm_tf"], s["peak_tf"], peaks),
+        "kernel_breakdown": s["breakdown"],
+        "gemm_sites": main_m["sites"],
+        "traced_ms_per_step": round(main_m["traced_ms"] / args.steps, 3),
+        "gpu_launches": int(round(s["kernels_per_step"] * args.steps)),
+        "trace_dropped": main_m["dropped"],
         "e2e": {"value": round(replica_throughput(N, args.steps, world, e2e_ms), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": 2 * N * 4, "d2h_bytes_per_step": 4},
-        "clocks": clk,
+        "clocks": main_m["clk"],
         "cpu_baseline": cpu,
     }
-    if optim is not None:
-        line["optimizer"] = optim
+    if main_m["optim"] is not None:
+        line["optimizer"] = main_m["optim"]
+    if second:
+        s2 = summarize(second, args, world, peaks)
+        w2 = second["w"]
+        line[w2.name] = {"workload": workload_desc(w2), "value": round(s2["tok_s"], 1), "unit": "tokens/s",
+                         "ms_per_step": round(ms2 / args.steps, 3), "mfu": s2["mfu"],
+                         "mfu_vs_measured_sustained": s2["mfu_measured"], "flops_per_token": s2["fpt"],
+                         "kernel_breakdown": s2["breakdown"], "gemm_sites": second["sites"],
+                         "gpu_launches": int(round(s2["kernels_per_step"] * args.steps)),
+                         "clocks": second["clk"]}
     print(json.dumps(line), flush=True)
 
 
@@ -526,6 +596,8 @@ def main():
     ap.add_argument("--workload", default=WORKLOAD, choices=list(synth.WORKLOADS))
     ap.add_argument("--no-optimizer", action="store_true",
                     help="skip the separate timing of the optimizer step")
+    ap.add_argument("--no-second", action="store_true",
+                    help="skip the depth-12 measurement that default runs add")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip timing the CPU oracle sample")
     ap.add_argument("--layers", type=int, default=None,

@@ -167,296 +167,330 @@ bool tile_map_f32(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols
   }
 
 // ===========================================================================
-// Forward.  One CTA per (128-query tile, b*h), the longest causal rows first.
-// S_j = Q K_j^T into one of two TMEM score buffers; the compute threads (two
-// per row, 64 keys each) take the row max (exchanged through shared memory),
-// write P_j = 2^(s*log2e/sqrt(hd) - m) as bf16 into the swizzled P tile, and
-// O += P_j V_j accumulates in TMEM.  A row's O and running sum are rescaled
-// (tcgen05.ld/st, each thread its half of the columns) only when its max grows
-// by more than 2^8 over the reference they share, so the result is exact and
-// most tiles skip it.  K and V have separate 2-slot rings: K_{j+2} loads as soon
-// as S_j is done, V_{j+2} once P_j V_j is.
+// Forward.  One CTA per pair of consecutive 128-query tiles (A = 2p, B = 2p+1)
+// of one (batch, head), which share one stream of K and V tiles; pairs run
+// (batch, head)-major with the longest first inside each head, so the CTAs
+// resident together share a few heads' K/V in L2.
+//
+// Warps 0..3 own tile A's rows and warps 4..7 tile B's (one thread per query
+// row: TMEM lane quarter = warp % 4), warp 8 loads tiles with TMA, warp 9
+// issues S_X = Q_X K^T and O_X += P_X V, warps 10 and 11 only complete their
+// warpgroup.  TMEM: S_A at columns 0..127,
+// S_B at 128..255, O_A at 256, O_B at 384.  A row's thread reads its 128 scores,
+// writes P = 2^(s*log2e/sqrt(hd) - m) as packed bf16 over the first 64 columns
+// of its own S (the A operand of the PV product, read from TMEM), and so the
+// two tiles alternate on the tensor core: while one tile's exponentials run,
+// the other tile's products do.  S_X of the next key tile overwrites P_X; it
+// is issued after the PV product that reads P_X, by the same thread, so in
+// order.  A row
+// rescales its O and running sum (tcgen05.ld/st) only when its max grows by
+// more than 2^8 over the reference they share: exact, and rare after the
+// first tiles.  K_j and V_j take consecutive slots of one 4-slot ring.
 // ===========================================================================
 namespace {
+constexpr int kFwdRing = 4;
+constexpr int kFwdThreads = 384;  // warps 0..7 softmax, 8 TMA, 9 MMA, 10..11 idle
+// Register split between the warpgroups (setmaxnreg): the launch gives every
+// thread 168 (65,536 / 384 rounded down to the allocation granule of 8, and
+// 3 x 168 x 32 fits one sub-partition's 16K); warpgroup 2 (TMA, MMA) gives
+// registers back so that the two softmax warpgroups can each hold a row's 128
+// scores.  2 x 128 x 216 + 128 x 72 = 64,512 = 384 x 168: the raise never
+// waits for registers that are not there.
+constexpr int kFwdRegsSoftmax = 216, kFwdRegsOther = 72;
+static_assert(2 * 128 * kFwdRegsSoftmax + 128 * kFwdRegsOther <= kFwdThreads * 168, "");
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 template <int HD>
 struct FwdSmem {
-  static constexpr uint32_t TILE = BQ * HD * 2;
-  static constexpr uint32_t P_BYTES = BQ * BKV * 2;
-  static constexpr uint32_t Q_OFF = 0;
-  static constexpr uint32_t K_OFF = Q_OFF + TILE;
-  static constexpr uint32_t V_OFF = K_OFF + 2 * TILE;
-  static constexpr uint32_t P_OFF = V_OFF + 2 * TILE;
-  static constexpr uint32_t RED_OFF = P_OFF + P_BYTES;           // float [2 iter][2 half][128]
-  static constexpr uint32_t SUM_OFF = RED_OFF + 2 * 2 * BQ * 4;  // float [2 half][128]
-  static constexpr uint32_t BAR_OFF = SUM_OFF + 2 * BQ * 4;
+  static constexpr uint32_t TILE = 128 * HD * 2;  // a 128-row Q, K or V tile
+  static constexpr uint32_t QA_OFF = 0, QB_OFF = TILE;
+  static constexpr uint32_t RING_OFF = 2 * TILE;
+  static constexpr uint32_t BAR_OFF = RING_OFF + kFwdRing * TILE;
   static constexpr uint32_t BYTES = BAR_OFF + 256 + 1024;
-  static_assert(K_OFF % 1024 == 0 && V_OFF % 1024 == 0 && P_OFF % 1024 == 0, "");
+  static_assert(TILE % 1024 == 0 && BYTES <= 232448, "");
 };
 struct FwdBars {
   uint64_t q_full;
-  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
-  uint64_t s_full[2];
-  uint64_t p_ready[2];  // per S buffer: the S and PV warps wait on it out of step
-  uint64_t pv_full;
-  uint64_t done, done2;
+  uint64_t kv_full[kFwdRing], kv_empty[kFwdRing];
+  uint64_t s_full[2], p_ready[2], pv_done[2];
+  uint64_t done_s;
   uint32_t tmem_base;
   int abort;
 };
+
+// Key-tile range [lo, lo + n) of query tile qt (n = 0: the tile is past T).
+struct KeyRange {
+  int lo, n;
+};
+__device__ __forceinline__ KeyRange key_range(int qt, int T, int W) {
+  KeyRange r;
+  const int q0 = qt * 128;
+  r.lo = max(0, q0 - W + 1) / 128;
+  r.n = q0 < T ? qt - r.lo + 1 : 0;
+  return r;
+}
 }  // namespace
 
 template <int HD>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kFwdThreads, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                        const __grid_constant__ CUtensorMap map_k,
                        const __grid_constant__ CUtensorMap map_v, __nv_bfloat16* __restrict__ o,
                        float* __restrict__ lse, int H, int Hkv, int T, int W, float scale_log2,
                        int32_t* status) {
   using S = FwdSmem<HD>;
+  constexpr int NCH = HD / 64;
+  constexpr uint32_t CH = 128 * 128;  // bytes of one 64-column chunk of a 128-row tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   FwdBars* bars = reinterpret_cast<FwdBars*>(smem + S::BAR_OFF);
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
-  // (batch, head)-major order, longest causal rows first inside each head: the
-  // CTAs resident together share a few heads' K/V, which then stay in L2
-  const int n_qt = (T + BQ - 1) / BQ;
-  const int bh = int(blockIdx.x) / n_qt;
-  const int qt = n_qt - 1 - int(blockIdx.x) % n_qt;
-  const int q0 = qt * BQ;
-  const int j_lo = max(0, q0 - W + 1) / BKV;  // first key tile with a visible key
-  const int n_kv = qt - j_lo + 1;
+  const int n_qt = (T + 127) / 128, n_pairs = (n_qt + 1) / 2;
+  const int bh = int(blockIdx.x) / n_pairs;
+  const int pair = n_pairs - 1 - int(blockIdx.x) % n_pairs;
+  const KeyRange ra = key_range(2 * pair, T, W), rb = key_range(2 * pair + 1, T, W);
+  const int lo = ra.lo, n_kt = rb.n ? rb.lo + rb.n - ra.lo : ra.n;  // the shared stream
   const int row_base = bh * T;
   const int kv_row_base = ((bh / H) * Hkv + (bh % H) / (H / Hkv)) * T;
-  constexpr uint32_t CH = BQ * 128;  // bytes of one 64-column chunk of a 128-row tile
-  constexpr int NCH = HD / 64;
 
-  ATTN_PROLOGUE(bars, {
+  if (threadIdx.x == 0) {
     tc::mbar_init(&bars->q_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      tc::mbar_init(&bars->k_full[s], 1); tc::mbar_init(&bars->k_empty[s], 1);
-      tc::mbar_init(&bars->v_full[s], 1); tc::mbar_init(&bars->v_empty[s], 1);
-      tc::mbar_init(&bars->s_full[s], 1);
+    for (int s = 0; s < kFwdRing; ++s) {
+      tc::mbar_init(&bars->kv_full[s], 1);
+      tc::mbar_init(&bars->kv_empty[s], 1);
     }
-    tc::mbar_init(&bars->p_ready[0], 256);
-    tc::mbar_init(&bars->p_ready[1], 256);
-    tc::mbar_init(&bars->pv_full, 1);
-    tc::mbar_init(&bars->done, 1);
-    tc::mbar_init(&bars->done2, 1);
-  })
+    for (int x = 0; x < 2; ++x) {
+      tc::mbar_init(&bars->s_full[x], 1);
+      tc::mbar_init(&bars->p_ready[x], 128);
+      tc::mbar_init(&bars->pv_done[x], 1);
+    }
+    tc::mbar_init(&bars->done_s, 1);
+    bars->abort = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 9) {
+    tc::tmem_alloc(&bars->tmem_base, 512);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort = &bars->abort;
-  const uint32_t t_o = tmem + 256;  // S buffers at columns 0 and 128
-
-  if (warp == 0) {
-    // lane 0: Q then the K ring; lane 1: the V ring
-    if (lane < 2) {
-      const bool is_k = lane == 0;
-      uint64_t* full = is_k ? bars->k_full : bars->v_full;
-      uint64_t* empty = is_k ? bars->k_empty : bars->v_empty;
-      const CUtensorMap* map = is_k ? &map_k : &map_v;
-      uint8_t* base = smem + (is_k ? S::K_OFF : S::V_OFF);
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kFwdRegsOther));
+  }
+  if (warp == 8) {
+    if (lane == 0) {
       uint32_t issued = 0, last_par = 0;
-      if (is_k) {
-        tc::mbar_arrive_expect_tx(&bars->q_full, S::TILE);
+      tc::mbar_arrive_expect_tx(&bars->q_full, (rb.n ? 2 : 1) * S::TILE);
 #pragma unroll
-        for (int c = 0; c < NCH; ++c)
-          tc::tma_load_2d(smem + S::Q_OFF + c * CH, &map_q, &bars->q_full, c * 64, row_base + q0);
+      for (int c = 0; c < NCH; ++c) {
+        tc::tma_load_2d(smem + S::QA_OFF + c * CH, &map_q, &bars->q_full, c * 64, row_base + 2 * pair * 128);
+        if (rb.n)
+          tc::tma_load_2d(smem + S::QB_OFF + c * CH, &map_q, &bars->q_full, c * 64,
+                          row_base + (2 * pair + 1) * 128);
       }
-      for (int j = 0; j < n_kv; ++j) {
-        const int st = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        if (!tc::mbar_wait_bounded(&empty[st], ph ^ 1, abort, kWaitNs)) {
+      for (int u = 0; u < 2 * n_kt; ++u) {  // K_j, V_j, K_j+1, ...
+        const int st = u % kFwdRing;
+        const uint32_t ph = (u / kFwdRing) & 1;
+        if (!tc::mbar_wait_bounded(&bars->kv_empty[st], ph ^ 1, abort, kWaitNs)) {
           record_status(status, GPT_ETIMEOUT, K_ATTN, 10);
           *abort = 1;
           break;
         }
-        tc::mbar_arrive_expect_tx(&full[st], S::TILE);
+        tc::mbar_arrive_expect_tx(&bars->kv_full[st], S::TILE);
+        const CUtensorMap* map = (u & 1) ? &map_v : &map_k;
 #pragma unroll
         for (int c = 0; c < NCH; ++c)
-          tc::tma_load_2d(base + st * S::TILE + c * CH, map, &full[st], c * 64,
-                          kv_row_base + (j_lo + j) * BKV);
+          tc::tma_load_2d(smem + S::RING_OFF + st * S::TILE + c * CH, map, &bars->kv_full[st], c * 64,
+                          kv_row_base + (lo + u / 2) * 128);
         issued |= 1u << st;
         last_par = (last_par & ~(1u << st)) | (ph << st);
       }
       if (*abort) {
-        if (is_k) tc::mbar_wait_bounded(&bars->q_full, 0, nullptr, kWaitNs);
-        for (int s = 0; s < 2; ++s)
-          if (issued >> s & 1) tc::mbar_wait_bounded(&full[s], (last_par >> s) & 1, nullptr, kWaitNs);
+        tc::mbar_wait_bounded(&bars->q_full, 0, nullptr, kWaitNs);
+        for (int s = 0; s < kFwdRing; ++s)
+          if (issued >> s & 1) tc::mbar_wait_bounded(&bars->kv_full[s], (last_par >> s) & 1, nullptr, kWaitNs);
       }
     }
-  } else if (warp == 1) {
-    // S_j = Q K_j^T.  S_j reuses the TMEM buffer of S_{j-2}: the compute
-    // threads must have turned S_{j-2} into P_{j-2} first.
-    constexpr uint32_t idesc_s = tc::idesc_bf16_f32(BQ, BKV, false, false);
-    const uint64_t qd = tc::smem_desc_sw128(tc::smem_u32(smem + S::Q_OFF), 16);
+  } else if (warp == 9) {
+    // One warp issues every product, so they run in issue order: S_X of key
+    // tile j+1 (over P_X's columns) follows the O_X += P_X V_j that reads P_X.
+    // Per key tile: S_A, S_B, then O_A += P_A V once tile A's threads have
+    // written P_A (tile B's exponentials overlap it), then O_B += P_B V.
+    constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, 128, false, false);
+    constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(128, HD, false, true);
     bool ok = tc::mbar_wait_warp(&bars->q_full, 0, abort, kWaitNs);
     bool issued_any = false;
-    for (int j = 0; ok && j < n_kv; ++j) {
-      const int st = j & 1;
-      if (j >= 2 && !tc::mbar_wait_warp(&bars->p_ready[st], ((j - 2) >> 1) & 1, abort, kWaitNs)) { ok = false; break; }
-      if (!tc::mbar_wait_warp(&bars->k_full[st], (j >> 1) & 1, abort, kWaitNs)) { ok = false; break; }
+    for (int j = 0; ok && j < n_kt; ++j) {
+      const int uk = 2 * j, sk = uk % kFwdRing, uv = uk + 1, sv = uv % kFwdRing;
+      if (!tc::mbar_wait_warp(&bars->kv_full[sk], (uk / kFwdRing) & 1, abort, kWaitNs)) { ok = false; break; }
       tc::tc_fence_after();
-      const uint64_t kd = tc::smem_desc_sw128(tc::smem_u32(smem + S::K_OFF + st * S::TILE), 16);
+      const uint64_t kd = tc::smem_desc_sw128(tc::smem_u32(smem + S::RING_OFF + sk * S::TILE), 16);
 #pragma unroll
-      for (int k = 0; k < HD / 16; ++k) {
-        const uint32_t off = (k >> 2) * CH + (k & 3) * 32;
-        tc::mma_bf16_ss_elect(tmem + st * 128, tc::desc_advance(qd, off), tc::desc_advance(kd, off), idesc_s, k != 0);
+      for (int x = 0; x < 2; ++x) {
+        const KeyRange r = x ? rb : ra;
+        const int i = lo + j - r.lo;  // this tile's step
+        if (i < 0 || i >= r.n) continue;
+        const uint64_t qd = tc::smem_desc_sw128(tc::smem_u32(smem + (x ? S::QB_OFF : S::QA_OFF)), 16);
+#pragma unroll
+        for (int k = 0; k < HD / 16; ++k) {
+          const uint32_t off = (k >> 2) * CH + (k & 3) * 32;
+          tc::mma_bf16_ss_elect(tmem + x * 128, tc::desc_advance(qd, off), tc::desc_advance(kd, off), idesc_s,
+                                k != 0);
+        }
+        issued_any = true;
+        tc::mma_commit_elect(&bars->s_full[x]);
       }
-      issued_any = true;
-      tc::mma_commit_elect(&bars->s_full[st]);
-      tc::mma_commit_elect(&bars->k_empty[st]);
+      tc::mma_commit_elect(&bars->kv_empty[sk]);
+      if (!tc::mbar_wait_warp(&bars->kv_full[sv], (uv / kFwdRing) & 1, abort, kWaitNs)) { ok = false; break; }
+      const uint64_t vd = tc::smem_desc_sw128(tc::smem_u32(smem + S::RING_OFF + sv * S::TILE), CH);
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        const KeyRange r = x ? rb : ra;
+        const int i = lo + j - r.lo;
+        if (i < 0 || i >= r.n) continue;
+        if (!tc::mbar_wait_warp(&bars->p_ready[x], i & 1, abort, kWaitNs)) { ok = false; break; }
+        tc::tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 128 / 16; ++k)
+          tc::mma_bf16_ts_elect(tmem + 256 + x * 128, tmem + x * 128 + 8 * k, tc::desc_advance(vd, k * 2048),
+                                idesc_pv, (i | k) != 0);
+        tc::mma_commit_elect(&bars->pv_done[x]);
+      }
+      if (!ok) break;
+      tc::mma_commit_elect(&bars->kv_empty[sv]);
     }
     if (!ok) {
       if (lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 11);
       *abort = 1;
     }
     if (issued_any) {
-      tc::mma_commit_elect(&bars->done);
-      tc::mbar_wait_warp(&bars->done, 0, nullptr, kWaitNs);
+      tc::mma_commit_elect(&bars->done_s);
+      tc::mbar_wait_warp(&bars->done_s, 0, nullptr, kWaitNs);
     }
-  } else if (warp == 10) {
-    // O += P_j V_j once the compute threads have written P_j
-    constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(BQ, HD, false, true);
-    const uint64_t pd = tc::smem_desc_sw128(tc::smem_u32(smem + S::P_OFF), 16);
-    bool ok = true, issued_any = false;
-    for (int j = 0; ok && j < n_kv; ++j) {
-      if (!tc::mbar_wait_warp(&bars->p_ready[j & 1], (j >> 1) & 1, abort, kWaitNs)) { ok = false; break; }
-      if (!tc::mbar_wait_warp(&bars->v_full[j & 1], (j >> 1) & 1, abort, kWaitNs)) { ok = false; break; }
-      tc::tc_fence_after();
-      const uint64_t vd = tc::smem_desc_sw128(tc::smem_u32(smem + S::V_OFF + (j & 1) * S::TILE), CH);
-#pragma unroll
-      for (int k = 0; k < BKV / 16; ++k)
-        tc::mma_bf16_ss_elect(t_o, tc::desc_advance(pd, (k >> 2) * CH + (k & 3) * 32), tc::desc_advance(vd, k * 2048),
-                              idesc_pv, (j | k) != 0);
-      issued_any = true;
-      tc::mma_commit_elect(&bars->pv_full);
-      tc::mma_commit_elect(&bars->v_empty[j & 1]);
-    }
-    if (!ok) {
-      if (lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 13);
-      *abort = 1;
-    }
-    if (issued_any) {
-      tc::mma_commit_elect(&bars->done2);
-      tc::mbar_wait_warp(&bars->done2, 0, nullptr, kWaitNs);
-    }
-  } else {
-    const Roles R = roles();
-    const int q = q0 + R.r;
+  } else if (warp < 8) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kFwdRegsSoftmax));
+    // softmax: thread = one query row of tile x
+    const int x = warp >> 2;
+    const KeyRange r = x ? rb : ra;
+    const int row = (warp & 3) * 32 + lane;
+    const int q = (2 * pair + x) * 128 + row;
     const int lo_key = q - W + 1;  // the row's first visible key
-    float* red = reinterpret_cast<float*>(smem + S::RED_OFF);
-    float* sums = reinterpret_cast<float*>(smem + S::SUM_OFF);
-    uint8_t* p_chunk = smem + S::P_OFF + R.half * CH;  // this thread's 64 keys
-    float m_ref = -INFINITY, l_half = 0.f;
+    const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
+    const uint32_t t_s = tmem + x * 128 + lane_off, t_o = tmem + 256 + x * 128 + lane_off;
+    float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      const int st = j & 1;
-      const int k0 = (j_lo + j) * BKV + R.half * 64;
-      if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->s_full[st], (j >> 1) & 1, abort, kWaitNs));
-      float s[64];
-      float mx = -INFINITY;
-      if (ok) {
-        tc::tc_fence_after();
-        uint32_t ua[32], ub[32];
-        tc::tmem_ld_32x32b_x32(tmem + st * 128 + R.lane_off + R.half * 64, ua);
-        tc::tmem_ld_32x32b_x32(tmem + st * 128 + R.lane_off + R.half * 64 + 32, ub);
+    for (int i = 0; ok && i < r.n; ++i) {
+      const int k0 = (r.lo + i) * 128;
+      if (!tc::mbar_wait_warp(&bars->s_full[x], i & 1, abort, kWaitNs)) { ok = false; break; }
+      tc::tc_fence_after();
+      float s[128];
+      {
+        uint32_t u0[32], u1[32], u2[32], u3[32];
+        tc::tmem_ld_32x32b_x32(t_s, u0);
+        tc::tmem_ld_32x32b_x32(t_s + 32, u1);
+        tc::tmem_ld_32x32b_x32(t_s + 64, u2);
+        tc::tmem_ld_32x32b_x32(t_s + 96, u3);
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) { s[i] = __uint_as_float(ua[i]); s[32 + i] = __uint_as_float(ub[i]); }
-        if (j_lo + j == qt || k0 + 64 > T || k0 < lo_key) {
-#pragma unroll
-          for (int i = 0; i < 64; ++i)
-            if (k0 + i > q || k0 + i >= T || k0 + i < lo_key) s[i] = -INFINITY;
+        for (int e = 0; e < 32; ++e) {
+          s[e] = __uint_as_float(u0[e]);
+          s[32 + e] = __uint_as_float(u1[e]);
+          s[64 + e] = __uint_as_float(u2[e]);
+          s[96 + e] = __uint_as_float(u3[e]);
         }
-#pragma unroll
-        for (int i = 0; i < 64; ++i) mx = fmaxf(mx, s[i]);
       }
-      // row max over both halves (scores are unscaled here; the scale is positive)
-      red[(st * 2 + R.half) * BQ + R.r] = mx;
-      compute_bar();
-      const float mx_all = fmaxf(red[(st * 2) * BQ + R.r], red[(st * 2 + 1) * BQ + R.r]) * scale_log2;
-      if (ok) {
-        const bool grow = mx_all > m_ref + 8.f;
-        const float factor = grow ? ex2(m_ref - mx_all) : 1.f;
-        if (grow) {
-          l_half *= factor;
-          m_ref = mx_all;
-        }
-        // P_j into registers first: this overlaps P_{j-1} V_{j-1}, which must
-        // finish before O is rescaled and before the P tile is rewritten
-        uint64_t lsum2 = f2(0.f, 0.f);
-        // a row whose keys so far were all outside its window has no reference
-        // yet: its P is 0 (exp2(-inf - 0)), not NaN
-        const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
-        const uint64_t sc2 = f2(scale_log2, scale_log2), nm2 = f2(-m_use, -m_use);
+      if (k0 + 127 > q || k0 + 128 > T || k0 < lo_key) {
+#pragma unroll
+        for (int e = 0; e < 128; ++e)
+          if (k0 + e > q || k0 + e >= T || k0 + e < lo_key) s[e] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int e = 1; e < 127; e += 2) mx = fmax3(mx, s[e], s[e + 1]);
+      mx = fmaxf(mx, s[127]) * scale_log2;  // scores are unscaled; the scale is positive
+      const bool grow = mx > m_ref + 8.f;
+      const float factor = grow ? ex2(m_ref - mx) : 1.f;
+      if (grow) {
+        l *= factor;
+        m_ref = mx;
+      }
+      // a row whose keys so far were all outside its window has no reference
+      // yet: its P is 0 (exp2(-inf - 0)), not NaN
+      const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
+      const uint64_t sc2 = f2(scale_log2, scale_log2), nm2 = f2(-m_use, -m_use);
+      uint64_t lsum2 = f2(0.f, 0.f);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
         uint32_t pk[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float2 x = unf2(fma2(f2(s[2 * i], s[2 * i + 1]), sc2, nm2));
-          const float p0 = ex2(x.x), p1 = ex2(x.y);
+        for (int e = 0; e < 32; ++e) {
+          const float2 xx = unf2(fma2(f2(s[64 * h + 2 * e], s[64 * h + 2 * e + 1]), sc2, nm2));
+          const float p0 = ex2(xx.x), p1 = ex2(xx.y);
           lsum2 = add2(lsum2, f2(p0, p1));
-          pk[i] = pack2(p0, p1);
+          pk[e] = pack2(p0, p1);
         }
-        const float2 ls = unf2(lsum2);
-        l_half += ls.x + ls.y;
-        if (j > 0) {
-          ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->pv_full, (j - 1) & 1, abort, kWaitNs));
-          if (ok) tc::tc_fence_after();
-        }
-        if (ok) {
+        tc::tmem_st_32x32b_x32(t_s + 32 * h, pk);  // P over this row's first 64 S columns
+      }
+      const float2 ls = unf2(lsum2);
+      l += ls.x + ls.y;
+      if (i > 0 && __any_sync(0xffffffffu, grow)) {
+        // O holds P V up to step i-1 once that product is done
+        if (!tc::mbar_wait_warp(&bars->pv_done[x], (i - 1) & 1, abort, kWaitNs)) { ok = false; break; }
+        tc::tc_fence_after();
 #pragma unroll
-          for (int u = 0; u < 8; ++u)
-            *reinterpret_cast<uint4*>(p_chunk + sw_off(R.r, u)) =
-                make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-        }
-        if (ok && j > 0 && __any_sync(0xffffffffu, grow)) {
+        for (int c = 0; c < HD; c += 32) {
+          uint32_t u[32];
+          tc::tmem_ld_32x32b_x32(t_o + c, u);
+          tc::tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < HD / 2; c += 16) {
-            uint32_t u[16];
-            const uint32_t ta = t_o + R.lane_off + R.half * (HD / 2) + c;
-            tc::tmem_ld_32x32b_x16(ta, u);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * factor);
-            tc::tmem_st_32x32b_x16(ta, u);
-          }
-          tc::tmem_wait_st();
-        }
-        if (ok) {
-          fence_async_smem();
-          tc::tc_fence_before();
+          for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * factor);
+          tc::tmem_st_32x32b_x32(t_o + c, u);
         }
       }
-      tc::mbar_arrive(&bars->p_ready[st]);
+      tc::tmem_wait_st();
+      tc::tc_fence_before();
+      tc::mbar_arrive(&bars->p_ready[x]);
     }
-    if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->pv_full, (n_kv - 1) & 1, abort, kWaitNs));
-    sums[R.half * BQ + R.r] = l_half;
-    compute_bar();
-    const float l = sums[R.r] + sums[BQ + R.r];
+    if (ok && r.n > 0) ok = tc::mbar_wait_warp(&bars->pv_done[x], (r.n - 1) & 1, abort, kWaitNs);
     if (!ok) {
-      if (R.lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 12);
+      if (lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 12);
       *abort = 1;
-    } else {
+    } else if (r.n > 0) {
       tc::tc_fence_after();
       const int b = bh / H, h = bh % H;
       const float inv = 1.f / l;
-      __nv_bfloat16* dst = o + (int64_t(b) * T + q) * (int64_t(H) * HD) + h * HD + R.half * (HD / 2);
+      __nv_bfloat16* dst = o + (int64_t(b) * T + q) * (int64_t(H) * HD) + h * HD;
 #pragma unroll
-      for (int c = 0; c < HD / 2; c += 32) {
+      for (int c = 0; c < HD; c += 32) {
         float v[32];
-        tmem_ld<32>(t_o + R.lane_off + R.half * (HD / 2) + c, v);
+        tmem_ld<32>(t_o + c, v);
         if (q < T) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 8)
-            *reinterpret_cast<uint4*>(dst + c + i) =
-                make_uint4(pack2(v[i] * inv, v[i + 1] * inv), pack2(v[i + 2] * inv, v[i + 3] * inv),
-                           pack2(v[i + 4] * inv, v[i + 5] * inv), pack2(v[i + 6] * inv, v[i + 7] * inv));
+          for (int e = 0; e < 32; e += 8)
+            *reinterpret_cast<uint4*>(dst + c + e) =
+                make_uint4(pack2(v[e] * inv, v[e + 1] * inv), pack2(v[e + 2] * inv, v[e + 3] * inv),
+                           pack2(v[e + 4] * inv, v[e + 5] * inv), pack2(v[e + 6] * inv, v[e + 7] * inv));
         }
       }
-      if (q < T && R.half == 0) lse[int64_t(bh) * T + q] = (m_ref + __log2f(l)) * 0.69314718055994531f;
+      if (q < T) lse[int64_t(bh) * T + q] = (m_ref + __log2f(l)) * 0.69314718055994531f;
     }
   }
-  ATTN_EPILOGUE(tmem)
+  __syncwarp();
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 512);
+  }
 }
 
 namespace {
@@ -473,8 +507,8 @@ int attn_fwd_tc_t(const gpt_config& c, const void* q, const void* k, const void*
   const int smem = int(FwdSmem<HD>::BYTES);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return 1;
-  const int n_qt = (c.seq_len + BQ - 1) / BQ;
-  kern<<<n_qt * c.batch * c.n_head, kThreads, smem, st>>>(
+  const int n_pairs = ((c.seq_len + 127) / 128 + 1) / 2;
+  kern<<<n_pairs * c.batch * c.n_head, kFwdThreads, smem, st>>>(
       mq, mk, mv, static_cast<__nv_bfloat16*>(o), lse, c.n_head, c.n_kv_head, c.seq_len,
       window_span(c), kLog2e / sqrtf(float(HD)), status);
   return last_launch_rc();

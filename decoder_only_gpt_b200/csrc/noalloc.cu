@@ -10,8 +10,13 @@
 // They pass only the inputs and the output; the library supplies the scratch.
 //
 // The array is loaded on every GPU that loads this library and stays resident
-// until the process exits.  Its device address is looked up once per device,
-// on the first call made with that device current.
+// until the process exits.  Its device address belongs to a CUDA context, so
+// it is looked up on the first call made in each context (keyed by the
+// context's unique id, which a context created after cudaDeviceReset, or by
+// the driver API inside a host runtime, does not share with an earlier one).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "device_common.cuh"
@@ -21,12 +26,19 @@ namespace gpt {
 namespace {
 
 constexpr size_t kScratchBytes = size_t(16) << 20;  // 16 MiB
-constexpr int kMaxDevices = 64;
+constexpr int kMaxContexts = 64;
 
 __device__ __align__(256) unsigned char g_scatter_scratch[kScratchBytes];
 
+// device address of g_scatter_scratch per context (unique id), most recent
+// contexts kept when more than kMaxContexts have called
+struct ScratchAddr {
+  unsigned long long ctx_id;
+  void* addr;
+};
 std::mutex g_addr_mu;
-void* g_addr[kMaxDevices] = {};  // device address of g_scatter_scratch, per device
+ScratchAddr g_addr[kMaxContexts] = {};
+int g_addr_next = 0;
 
 uint64_t up256(uint64_t x) { return (x + 255) / 256 * 256; }
 
@@ -53,17 +65,51 @@ uint64_t scratch_layout(int64_t N, int64_t V, int64_t d, Layout* L) {
   return up256(off);
 }
 
-// Device address of the scratch array on the current device.
+// Unique id of the calling thread's current context (0 if it cannot be read).
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of the scratch array in the current context.  The first
+// call in a context looks it up (cudaGetSymbolAddress, with that context
+// current); later calls reuse it.  Without a readable context id the address
+// is looked up on every call.
 int scratch_address(char** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GPT_ECUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GPT_ECUDA;
+  const unsigned long long id = current_context_id();
   std::lock_guard<std::mutex> lock(g_addr_mu);
-  if (!g_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_scatter_scratch) != cudaSuccess || !p) return GPT_ECUDA;
-    g_addr[dev] = p;
+  if (id)
+    for (const ScratchAddr& a : g_addr)
+      if (a.ctx_id == id) {
+        *out = static_cast<char*>(a.addr);
+        return GPT_OK;
+      }
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_scatter_scratch) != cudaSuccess || !p) return GPT_ECUDA;
+  if (id) {
+    g_addr[g_addr_next] = {id, p};
+    g_addr_next = (g_addr_next + 1) % kMaxContexts;
   }
-  *out = static_cast<char*>(g_addr[dev]);
+  *out = static_cast<char*>(p);
   return GPT_OK;
 }
 

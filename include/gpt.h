@@ -201,11 +201,14 @@ const char* gpt_version(void);
  *   dwte (rows no token hits become 0), 1 adds to it.
  * Result: dwte[v] (+)= sum over positions n with tokens[n] == v of dx0[n],
  * summed in the same fixed order as the wte gradient of gpt_backward, so the
- * two agree bit for bit.  Tokens outside [0, vocab) count as id 0.
+ * two agree bit for bit.  This call does not check the ids: the caller must
+ * pass ids in [0, vocab) (gpt_forward_loss checks them, GPT_EDATA); an id
+ * outside that range is summed into row 0 without any error.
  * Scratch: one 16 MiB array in device memory defined by the library, held by
  * every GPU that loads the library until the process exits.  The first call
- * on a device looks up that array's device address (cudaGetSymbolAddress) with
- * the device current; make that first call before any stream capture.  All
+ * in each CUDA context (keyed by the context's unique id) looks up that
+ * array's device address (cudaGetSymbolAddress) with the context current;
+ * make that first call before any stream capture.  All
  * calls share the array, so calls that may overlap on the same GPU (for
  * example on different streams) race: serialise them.  Sizes
  * whose scratch exceeds 16 MiB (about n_tokens * (8 + 8 d_model / 64) +

@@ -276,6 +276,28 @@ def test_bad_ids_reported(B, R):
     assert st.status() == B.GPT_OK
 
 
+def test_nonfinite_loss_reported(B, R):
+    """An infinite weight in one lm_head row (injected through the parameter
+    buffer on the host: nothing faults) makes the loss non-finite, which the
+    step records as GPT_ENONFINITE; the next step on clean parameters clears it."""
+    w = workload_of("ragged")
+    cfg = B.config_from_workload(w)
+    st = R.TrainStep(cfg)
+    params = synth.make_params(w, as_bits=True)
+    bad = {k: v.copy() for k, v in params.items()}
+    bad["lm_head"][7, :] = 0x7F80  # +inf in bf16
+    st.load_params(bad)
+    tok, tgt = synth.make_tokens(w)
+    st.set_batch(tok, tgt)
+    st.step()
+    assert st.status() == B.GPT_ENONFINITE
+    assert not math.isfinite(float(st.loss.cpu()[0]))
+    st.load_params(params)
+    st.step()
+    assert st.status() == B.GPT_OK
+    assert math.isfinite(float(st.loss.cpu()[0]))
+
+
 def test_train_step_host_matches_device_path(B, R):
     import torch
     w = workload_of("ragged")

@@ -107,3 +107,62 @@ def test_noalloc_accumulate_and_limits(mods):
     assert f(tok.data_ptr(), 1 << 22, 1 << 20, 4096, B.GPT_F32, dx0.data_ptr(), out.data_ptr(),
              0, s) == B.GPT_EUNSUPPORTED
     assert f(None, N, V, d, B.GPT_F32, dx0.data_ptr(), out.data_ptr(), 0, s) == B.GPT_EINVAL
+
+
+def _scratch_bytes(N, V, d):
+    """Bytes of the shared scratch a call needs: the sort and scatter regions
+    at 256-byte aligned offsets (the layout of noalloc.cu, restated)."""
+    off = 0
+
+    def take(nbytes):
+        nonlocal off
+        off = (off + 255) // 256 * 256
+        off += nbytes
+
+    take(N * 4)
+    take((V + 1) * 4)
+    take((V + 1) * 4)
+    take((N + 1023) // 1024 * V * 4)
+    take((N // 64 + V + 1) * 8)
+    take((V + 1) * 8)
+    take((N // 64 + 1) * d * 4 * 2)
+    return (off + 255) // 256 * 256
+
+
+def test_noalloc_near_limit_then_smaller_call(mods):
+    """A call whose scratch nearly fills the array, then a much smaller one
+    (fewer sort tiles, smaller vocabulary): the second must not see the first
+    call's histograms, offsets or partial sums left in the shared array."""
+    import torch
+    B, _ = mods
+    f = _entry(B)
+    dev = torch.device("cuda")
+    s = torch.cuda.current_stream().cuda_stream
+    limit = 16 << 20
+    V, d = 8192, 128
+    N = 1024
+    while _scratch_bytes(N + 1024, V, d) <= limit:
+        N += 1024
+    assert _scratch_bytes(N, V, d) > limit - (64 << 10)  # within 64 KiB of the array's size
+    rng = np.random.default_rng(1)
+    for n, v in ((N, V), (700, 257)):
+        tok_h = rng.integers(0, v, n).astype(np.int32)
+        dx_h = rng.standard_normal((n, d)).astype(np.float32)
+        tok, dx0 = torch.from_numpy(tok_h).to(dev), torch.from_numpy(dx_h).to(dev)
+        out = torch.full((v * d,), float("nan"), dtype=torch.float32, device=dev)
+        rc = f(tok.data_ptr(), n, v, d, B.GPT_F32, dx0.data_ptr(), out.data_ptr(), 0, s)
+        assert rc == B.GPT_OK, B.strerror(rc)
+        torch.cuda.synchronize()
+        ref = np.zeros((v, d))
+        np.add.at(ref, tok_h, dx_h.astype(np.float64))
+        got = out.cpu().numpy().reshape(v, d).astype(np.float64)
+        cos, mr = _metrics(got, ref)
+        assert cos >= 0.99999 and mr <= 1e-5, (n, v, cos, mr)
+        assert np.all(got[np.bincount(tok_h, minlength=v) == 0] == 0)
+    # one sort tile more than fits: rejected before any launch
+    tok = torch.zeros(N + 1024, dtype=torch.int32, device=dev)
+    dx0 = torch.zeros((N + 1024) * d, dtype=torch.float32, device=dev)
+    out = torch.zeros(V * d, dtype=torch.float32, device=dev)
+    assert f(tok.data_ptr(), N + 1024, V, d, B.GPT_F32, dx0.data_ptr(), out.data_ptr(), 0,
+             s) == B.GPT_EUNSUPPORTED
+
