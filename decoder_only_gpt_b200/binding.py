@@ -46,7 +46,8 @@ class GptOptim(ctypes.Structure):
                 ("adam_weight_decay", ctypes.c_float), ("muon_lr", ctypes.c_float),
                 ("muon_momentum", ctypes.c_float), ("muon_nesterov", ctypes.c_int32),
                 ("ns_steps", ctypes.c_int32), ("ns_coeffs", (ctypes.c_float * 3) * 8),
-                ("step", ctypes.c_int64)]
+                ("step", ctypes.c_int64), ("normuon", ctypes.c_int32),
+                ("normuon_beta2", ctypes.c_float)]
 
     def coeffs(self):
         return [tuple(float(x) for x in self.ns_coeffs[i]) for i in range(self.ns_steps)]

@@ -138,8 +138,9 @@ bool make_layout(const gpt_config& c, Layout* L) {
     L->opt_a += L->layer_base;
     L->opt_b += L->layer_base;
     L->opt_part = b.take((kOptNormBlocks + 1) * 4);
+    L->opt_rows = b.take(2 * std::max(std::max(Q, F), d) * 4);
   } else {
-    L->opt_x0 = L->opt_x1 = L->opt_a = L->opt_b = L->opt_part = 0;
+    L->opt_x0 = L->opt_x1 = L->opt_a = L->opt_b = L->opt_part = L->opt_rows = 0;
   }
   L->total = align_up(b.off, kAlign);
   return true;
@@ -659,6 +660,8 @@ int gpt_optim_defaults(gpt_optim* o) {
   for (int i = 0; i < 2; ++i)
     for (int j = 0; j < 3; ++j) o->ns_coeffs[i][j] = printed[i][j];
   o->step = 1;
+  o->normuon = 0;
+  o->normuon_beta2 = 0.95f;
   return GPT_OK;
 }
 
@@ -708,6 +711,8 @@ int gpt_optim_step(const gpt_config* c, const gpt_optim* o, void* params, const 
   if (!(o->adam_beta1 >= 0.f && o->adam_beta1 < 1.f && o->adam_beta2 >= 0.f && o->adam_beta2 < 1.f))
     return GPT_EINVAL;
   if (o->muon_nesterov != 0 && o->muon_nesterov != 1) return GPT_EINVAL;
+  if (o->normuon != 0 && o->normuon != 1) return GPT_EINVAL;
+  if (o->normuon && !(o->normuon_beta2 >= 0.f && o->normuon_beta2 < 1.f)) return GPT_EINVAL;
 
   cudaStream_t st = (cudaStream_t)stream;
   Layout L;
@@ -805,11 +810,22 @@ int gpt_optim_step(const gpt_config* c, const gpt_optim* o, void* params, const 
       std::swap(X, Xn);
     }
     const float step = o->muon_lr * std::sqrt(std::max(1.f, float(r) / float(cc)));
+    float* vmean = reinterpret_cast<float*>(ws + L.opt_rows);
+    float* factor = vmean + std::max(std::max(qkv_cols(*c), int64_t(c->d_ff)), int64_t(c->d_model));
     for (int l = 0; l < nl; ++l) {
       int64_t off, rr, rc2;
       gpt_param_offset(c, tensor, l, &off, &rr, &rc2);
-      TraceScope ts(GPT_K_OTHER, 1, 0, double(n) * 12.0, st);
-      GPT_TRY(launch_muon_apply(X + l * n * 2, W + off, P + off, n, step, st));
+      if (o->normuon) {
+        // NorMuon: the per-row state lives in this matrix's (otherwise unused)
+        // second-moment slots of the state buffer
+        TraceScope ts(GPT_K_OTHER, 3, 0, double(n) * 2.0 + double(r) * 16.0, st);
+        GPT_TRY(launch_normuon(X + l * n * 2, Vv + off, int(r), int(cc), o->normuon_beta2, vmean, factor, st));
+        TraceScope ts2(GPT_K_OTHER, 1, 0, double(n) * 12.0, st);
+        GPT_TRY(launch_muon_apply_rows(X + l * n * 2, W + off, P + off, int(r), int(cc), step, factor, st));
+      } else {
+        TraceScope ts(GPT_K_OTHER, 1, 0, double(n) * 12.0, st);
+        GPT_TRY(launch_muon_apply(X + l * n * 2, W + off, P + off, n, step, st));
+      }
     }
   }
   return GPT_OK;

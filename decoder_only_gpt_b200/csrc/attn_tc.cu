@@ -19,6 +19,8 @@
 // of times on every path, so an expired wait cannot strand them.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+
 #include "device_common.cuh"
 #include "tc_ptx.cuh"
 
@@ -89,6 +91,22 @@ __device__ __forceinline__ Roles roles() {
   x.r = x.quarter * 32 + x.lane;     // accumulator row
   x.lane_off = uint32_t(x.quarter * 32) << 16;
   return x;
+}
+
+// Work item of CTA `b` in a launch over n_rows x n_ranks items (a row is a
+// (batch, head) and rank 0 its longest tile, the work shrinking with the
+// rank): rows go in groups of kGroupRows, and inside a group all rows' rank-0
+// items come first, then their rank-1 items, and so on.  The resident CTAs
+// then share a few rows' K/V in L2, and the short items of the last group
+// fill the tail instead of one row's long ones.
+constexpr int kGroupRows = 16;
+__device__ __forceinline__ void grouped_item(int b, int n_rows, int n_ranks, int& row, int& rank) {
+  const int grp = b / (kGroupRows * n_ranks);
+  const int base = grp * kGroupRows;
+  const int gs = min(kGroupRows, n_rows - base);
+  const int r = b - grp * kGroupRows * n_ranks;
+  rank = r / gs;
+  row = base + r % gs;
 }
 
 template <int N>
@@ -167,25 +185,26 @@ bool tile_map_f32(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols
   }
 
 // ===========================================================================
-// Forward.  One CTA per pair of consecutive 128-query tiles (A = 2p, B = 2p+1)
-// of one (batch, head), which share one stream of K and V tiles; pairs run
-// (batch, head)-major with the longest first inside each head, so the CTAs
-// resident together share a few heads' K/V in L2.
+// Forward.  A persistent grid (one CTA per SM) takes work items from a
+// counter: an item is a pair of consecutive 128-query tiles (A = 2p, B = 2p+1)
+// of one (batch, head), which share one stream of K and V tiles.  Items go in
+// groups of heads, the longest pairs first (grouped_item), so the resident
+// CTAs share a few heads' K/V in L2 and the short items fill the tail.
 //
 // Warps 0..3 own tile A's rows and warps 4..7 tile B's (one thread per query
-// row: TMEM lane quarter = warp % 4), warp 8 loads tiles with TMA, warp 9
-// issues S_X = Q_X K^T and O_X += P_X V, warps 10 and 11 only complete their
-// warpgroup.  TMEM: S_A at columns 0..127,
-// S_B at 128..255, O_A at 256, O_B at 384.  A row's thread reads its 128 scores,
-// writes P = 2^(s*log2e/sqrt(hd) - m) as packed bf16 over the first 64 columns
-// of its own S (the A operand of the PV product, read from TMEM), and so the
-// two tiles alternate on the tensor core: while one tile's exponentials run,
-// the other tile's products do.  S_X of the next key tile overwrites P_X; it
-// is issued after the PV product that reads P_X, by the same thread, so in
-// order.  A row
-// rescales its O and running sum (tcgen05.ld/st) only when its max grows by
-// more than 2^8 over the reference they share: exact, and rare after the
-// first tiles.  K_j and V_j take consecutive slots of one 4-slot ring.
+// row: TMEM lane quarter = warp % 4); warp 8 publishes the items and loads
+// tiles with TMA; warp 9 issues S_X = Q_X K^T and O_X += P_X V; warps 10 and
+// 11 only complete their warpgroup.  TMEM: S_A at columns 0..127, S_B at
+// 128..255, O_A at 256, O_B at 384.  A row's thread reads its 128 scores and
+// writes P = 2^(s*log2e/sqrt(hd) - m) as packed bf16 over the first 64
+// columns of its own S (the A operand of the PV product, read from TMEM), so
+// the two tiles alternate on the tensor core: while one tile's exponentials
+// run, the other tile's products do.  S_X of the next key tile overwrites
+// P_X; it is issued after the PV product that reads P_X, by the same thread,
+// so in order.  A row rescales its O and running sum (tcgen05.ld/st) only
+// when its max grows by more than 2^8 over the reference they share: exact,
+// and rare after the first tiles.  K_j and V_j take consecutive slots of one
+// 4-slot ring.
 // ===========================================================================
 namespace {
 constexpr int kFwdRing = 4;
@@ -194,9 +213,9 @@ constexpr int kFwdThreads = 384;  // warps 0..7 softmax, 8 TMA, 9 MMA, 10..11 id
 // thread 168 (65,536 / 384 rounded down to the allocation granule of 8, and
 // 3 x 168 x 32 fits one sub-partition's 16K); warpgroup 2 (TMA, MMA) gives
 // registers back so that the two softmax warpgroups can each hold a row's 128
-// scores.  2 x 128 x 216 + 128 x 72 = 64,512 = 384 x 168: the raise never
+// scores.  2 x 128 x 200 + 128 x 104 = 64,512 = 384 x 168: the raise never
 // waits for registers that are not there.
-constexpr int kFwdRegsSoftmax = 216, kFwdRegsOther = 72;
+constexpr int kFwdRegsSoftmax = 200, kFwdRegsOther = 104;
 static_assert(2 * 128 * kFwdRegsSoftmax + 128 * kFwdRegsOther <= kFwdThreads * 168, "");
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -215,12 +234,14 @@ struct FwdSmem {
   static_assert(TILE % 1024 == 0 && BYTES <= 232448, "");
 };
 struct FwdBars {
-  uint64_t q_full;
+  uint64_t q_full[2], q_empty[2];
   uint64_t kv_full[kFwdRing], kv_empty[kFwdRing];
   uint64_t s_full[2], p_ready[2], pv_done[2];
+  uint64_t item_full[2], item_empty[2];
   uint64_t done_s;
   uint32_t tmem_base;
   int abort;
+  int items[2];  // the published work items (-1: none left)
 };
 
 // Key-tile range [lo, lo + n) of query tile qt (n = 0: the tile is past T).
@@ -236,13 +257,29 @@ __device__ __forceinline__ KeyRange key_range(int qt, int T, int W) {
 }
 }  // namespace
 
+// Work counters of the persistent kernels, in the unused tail of the
+// workspace's 256-byte status region (which gpt_forward_loss zeroes): a pair
+// per kernel, [next item, CTAs finished].  The last CTA of a launch to finish
+// sets both back to zero, so every launch starts from zero without a memset.
+constexpr int kSchedFwd = 0;
+__host__ __device__ inline int32_t* sched_counters(int32_t* status, int which) {
+  return status + 32 + which;  // bytes 128.. of the status region
+}
+__device__ __forceinline__ void sched_finish(int32_t* sched) {
+  __threadfence();
+  if (atomicAdd(sched + 1, 1) == int(gridDim.x) - 1) {
+    atomicExch(sched, 0);
+    atomicExch(sched + 1, 0);
+  }
+}
+
 template <int HD>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                        const __grid_constant__ CUtensorMap map_k,
                        const __grid_constant__ CUtensorMap map_v, __nv_bfloat16* __restrict__ o,
                        float* __restrict__ lse, int H, int Hkv, int T, int W, float scale_log2,
-                       int32_t* status) {
+                       int n_rows, int32_t* status) {
   using S = FwdSmem<HD>;
   constexpr int NCH = HD / 64;
   constexpr uint32_t CH = 128 * 128;  // bytes of one 64-column chunk of a 128-row tile
@@ -252,23 +289,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   FwdBars* bars = reinterpret_cast<FwdBars*>(smem + S::BAR_OFF);
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int n_qt = (T + 127) / 128, n_pairs = (n_qt + 1) / 2;
-  const int bh = int(blockIdx.x) / n_pairs;
-  const int pair = n_pairs - 1 - int(blockIdx.x) % n_pairs;
-  const KeyRange ra = key_range(2 * pair, T, W), rb = key_range(2 * pair + 1, T, W);
-  const int lo = ra.lo, n_kt = rb.n ? rb.lo + rb.n - ra.lo : ra.n;  // the shared stream
-  const int row_base = bh * T;
-  const int kv_row_base = ((bh / H) * Hkv + (bh % H) / (H / Hkv)) * T;
+  const int n_items = n_rows * n_pairs;
+  int32_t* sched = sched_counters(status, kSchedFwd);
 
   if (threadIdx.x == 0) {
-    tc::mbar_init(&bars->q_full, 1);
-    for (int s = 0; s < kFwdRing; ++s) {
-      tc::mbar_init(&bars->kv_full[s], 1);
-      tc::mbar_init(&bars->kv_empty[s], 1);
-    }
     for (int x = 0; x < 2; ++x) {
+      tc::mbar_init(&bars->q_full[x], 1);
+      tc::mbar_init(&bars->q_empty[x], 1);
       tc::mbar_init(&bars->s_full[x], 1);
       tc::mbar_init(&bars->p_ready[x], 128);
       tc::mbar_init(&bars->pv_done[x], 1);
+      tc::mbar_init(&bars->item_full[x], 1);
+      tc::mbar_init(&bars->item_empty[x], 9);  // the MMA warp and the 8 softmax warps
+    }
+    for (int s = 0; s < kFwdRing; ++s) {
+      tc::mbar_init(&bars->kv_full[s], 1);
+      tc::mbar_init(&bars->kv_empty[s], 1);
     }
     tc::mbar_init(&bars->done_s, 1);
     bars->abort = 0;
@@ -283,90 +319,163 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   tc::tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort = &bars->abort;
+  volatile int* items = bars->items;
+  // the item's (batch, head) row, query-tile pair and both tiles' key ranges
+  auto decode = [=](int k, int& bh, int& pair, KeyRange& ra, KeyRange& rb) {
+    int rank;
+    grouped_item(k, n_rows, n_pairs, bh, rank);
+    pair = n_pairs - 1 - rank;
+    ra = key_range(2 * pair, T, W);
+    rb = key_range(2 * pair + 1, T, W);
+  };
   if (warp >= 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kFwdRegsOther));
   }
   if (warp == 8) {
+    // TMA producer and scheduler: publishes each work item (-1 at the end),
+    // then loads its Q tiles and its stream of K, V tiles
     if (lane == 0) {
-      uint32_t issued = 0, last_par = 0;
-      tc::mbar_arrive_expect_tx(&bars->q_full, (rb.n ? 2 : 1) * S::TILE);
+      uint32_t ring_issued = 0, ring_par = 0, q_issued = 0, q_par = 0;
+      int u = 0, qn[2] = {0, 0};
+      bool ok = true;
+      int k = int(blockIdx.x);
+      for (int seq = 0;; ++seq) {
+        const int s = seq & 1;
+        if (!tc::mbar_wait_bounded(&bars->item_empty[s], ((seq >> 1) & 1) ^ 1, abort, kWaitNs)) { ok = false; break; }
+        items[s] = k < n_items ? k : -1;
+        tc::mbar_arrive(&bars->item_full[s]);
+        if (k >= n_items) break;
+        int bh, pair;
+        KeyRange ra, rb;
+        decode(k, bh, pair, ra, rb);
+        const int n_kt = rb.n ? rb.lo + rb.n - ra.lo : ra.n;
+        const int kv_row_base = ((bh / H) * Hkv + (bh % H) / (H / Hkv)) * T;
+        for (int x = 0; ok && x < 2; ++x) {
+          if ((x ? rb : ra).n == 0) continue;
+          // the previous item's S products of this tile are done with Q_x
+          if (!tc::mbar_wait_bounded(&bars->q_empty[x], (qn[x] & 1) ^ 1, abort, kWaitNs)) { ok = false; break; }
+          tc::mbar_arrive_expect_tx(&bars->q_full[x], S::TILE);
 #pragma unroll
-      for (int c = 0; c < NCH; ++c) {
-        tc::tma_load_2d(smem + S::QA_OFF + c * CH, &map_q, &bars->q_full, c * 64, row_base + 2 * pair * 128);
-        if (rb.n)
-          tc::tma_load_2d(smem + S::QB_OFF + c * CH, &map_q, &bars->q_full, c * 64,
-                          row_base + (2 * pair + 1) * 128);
-      }
-      for (int u = 0; u < 2 * n_kt; ++u) {  // K_j, V_j, K_j+1, ...
-        const int st = u % kFwdRing;
-        const uint32_t ph = (u / kFwdRing) & 1;
-        if (!tc::mbar_wait_bounded(&bars->kv_empty[st], ph ^ 1, abort, kWaitNs)) {
-          record_status(status, GPT_ETIMEOUT, K_ATTN, 10);
-          *abort = 1;
-          break;
+          for (int c = 0; c < NCH; ++c)
+            tc::tma_load_2d(smem + (x ? S::QB_OFF : S::QA_OFF) + c * CH, &map_q, &bars->q_full[x], c * 64,
+                            bh * T + (2 * pair + x) * 128);
+          q_issued |= 1u << x;
+          q_par = (q_par & ~(1u << x)) | ((qn[x] & 1u) << x);
+          ++qn[x];
         }
-        tc::mbar_arrive_expect_tx(&bars->kv_full[st], S::TILE);
-        const CUtensorMap* map = (u & 1) ? &map_v : &map_k;
+        for (int v = 0; ok && v < 2 * n_kt; ++v, ++u) {  // K_j, V_j, K_j+1, ...
+          const int st = u % kFwdRing;
+          const uint32_t ph = (u / kFwdRing) & 1;
+          if (!tc::mbar_wait_bounded(&bars->kv_empty[st], ph ^ 1, abort, kWaitNs)) { ok = false; break; }
+          tc::mbar_arrive_expect_tx(&bars->kv_full[st], S::TILE);
+          const CUtensorMap* map = (v & 1) ? &map_v : &map_k;
 #pragma unroll
-        for (int c = 0; c < NCH; ++c)
-          tc::tma_load_2d(smem + S::RING_OFF + st * S::TILE + c * CH, map, &bars->kv_full[st], c * 64,
-                          kv_row_base + (lo + u / 2) * 128);
-        issued |= 1u << st;
-        last_par = (last_par & ~(1u << st)) | (ph << st);
+          for (int c = 0; c < NCH; ++c)
+            tc::tma_load_2d(smem + S::RING_OFF + st * S::TILE + c * CH, map, &bars->kv_full[st], c * 64,
+                            kv_row_base + (ra.lo + v / 2) * 128);
+          ring_issued |= 1u << st;
+          ring_par = (ring_par & ~(1u << st)) | (ph << st);
+        }
+        if (!ok) break;
+        k = atomicAdd(sched, 1) + int(gridDim.x);
       }
-      if (*abort) {
-        tc::mbar_wait_bounded(&bars->q_full, 0, nullptr, kWaitNs);
+      if (!ok) {
+        record_status(status, GPT_ETIMEOUT, K_ATTN, 10);
+        *abort = 1;
+        // wait for this warp's own copies in flight before the CTA exits
+        for (int x = 0; x < 2; ++x)
+          if (q_issued >> x & 1) tc::mbar_wait_bounded(&bars->q_full[x], (q_par >> x) & 1, nullptr, kWaitNs);
         for (int s = 0; s < kFwdRing; ++s)
-          if (issued >> s & 1) tc::mbar_wait_bounded(&bars->kv_full[s], (last_par >> s) & 1, nullptr, kWaitNs);
+          if (ring_issued >> s & 1) tc::mbar_wait_bounded(&bars->kv_full[s], (ring_par >> s) & 1, nullptr, kWaitNs);
       }
     }
   } else if (warp == 9) {
-    // One warp issues every product, so they run in issue order: S_X of key
-    // tile j+1 (over P_X's columns) follows the O_X += P_X V_j that reads P_X.
-    // Per key tile: S_A, S_B, then O_A += P_A V once tile A's threads have
-    // written P_A (tile B's exponentials overlap it), then O_B += P_B V.
+    // One warp issues every product, so they run in issue order.  Per key
+    // tile j: O_A += P_A V_j as soon as tile A's threads have written P_A,
+    // then at once S_A = Q_A K_{j+1}^T (over P_A's columns, after the product
+    // that reads them), then the same for tile B.  A tile's next scores are
+    // thus two products after its P, while the other tile's exponentials run.
     constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, 128, false, false);
     constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(128, HD, false, true);
-    bool ok = tc::mbar_wait_warp(&bars->q_full, 0, abort, kWaitNs);
-    bool issued_any = false;
-    for (int j = 0; ok && j < n_kt; ++j) {
-      const int uk = 2 * j, sk = uk % kFwdRing, uv = uk + 1, sv = uv % kFwdRing;
-      if (!tc::mbar_wait_warp(&bars->kv_full[sk], (uk / kFwdRing) & 1, abort, kWaitNs)) { ok = false; break; }
-      tc::tc_fence_after();
-      const uint64_t kd = tc::smem_desc_sw128(tc::smem_u32(smem + S::RING_OFF + sk * S::TILE), 16);
-#pragma unroll
-      for (int x = 0; x < 2; ++x) {
-        const KeyRange r = x ? rb : ra;
-        const int i = lo + j - r.lo;  // this tile's step
-        if (i < 0 || i >= r.n) continue;
-        const uint64_t qd = tc::smem_desc_sw128(tc::smem_u32(smem + (x ? S::QB_OFF : S::QA_OFF)), 16);
-#pragma unroll
-        for (int k = 0; k < HD / 16; ++k) {
-          const uint32_t off = (k >> 2) * CH + (k & 3) * 32;
-          tc::mma_bf16_ss_elect(tmem + x * 128, tc::desc_advance(qd, off), tc::desc_advance(kd, off), idesc_s,
-                                k != 0);
-        }
-        issued_any = true;
-        tc::mma_commit_elect(&bars->s_full[x]);
-      }
-      tc::mma_commit_elect(&bars->kv_empty[sk]);
-      if (!tc::mbar_wait_warp(&bars->kv_full[sv], (uv / kFwdRing) & 1, abort, kWaitNs)) { ok = false; break; }
-      const uint64_t vd = tc::smem_desc_sw128(tc::smem_u32(smem + S::RING_OFF + sv * S::TILE), CH);
-#pragma unroll
-      for (int x = 0; x < 2; ++x) {
+    const uint32_t ring0 = tc::smem_u32(smem + S::RING_OFF);
+    const uint32_t qa = tc::smem_u32(smem + S::QA_OFF), qb = tc::smem_u32(smem + S::QB_OFF);
+    bool ok = true, issued_any = false;
+    int u = 0, qn[2] = {0, 0}, cs[2] = {0, 0};  // ring items, Q fills, steps done per tile
+    for (int seq = 0; ok; ++seq) {
+      const int s = seq & 1;
+      if (!tc::mbar_wait_warp(&bars->item_full[s], (seq >> 1) & 1, abort, kWaitNs)) { ok = false; break; }
+      const int k = items[s];
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&bars->item_empty[s]);
+      if (k < 0) break;
+      int bh, pair;
+      KeyRange ra, rb;
+      decode(k, bh, pair, ra, rb);
+      const int lo = ra.lo, n_kt = rb.n ? rb.lo + rb.n - ra.lo : ra.n;
+      auto step_of = [=](int x, int j) {  // tile x's step at stream step j, or -1
         const KeyRange r = x ? rb : ra;
         const int i = lo + j - r.lo;
-        if (i < 0 || i >= r.n) continue;
-        if (!tc::mbar_wait_warp(&bars->p_ready[x], i & 1, abort, kWaitNs)) { ok = false; break; }
-        tc::tc_fence_after();
+        return i >= 0 && i < r.n ? i : -1;
+      };
+      // S_X = Q_X K^T, the K tile in ring slot `st`; Q_X freed after its last
+      auto issue_s = [&](int x, int st, bool last) {
+        const uint64_t kd = tc::smem_desc_sw128(ring0 + st * S::TILE, 16);
+        const uint64_t qd = tc::smem_desc_sw128(x ? qb : qa, 16);
 #pragma unroll
-        for (int k = 0; k < 128 / 16; ++k)
-          tc::mma_bf16_ts_elect(tmem + 256 + x * 128, tmem + x * 128 + 8 * k, tc::desc_advance(vd, k * 2048),
-                                idesc_pv, (i | k) != 0);
-        tc::mma_commit_elect(&bars->pv_done[x]);
-      }
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * CH + (kk & 3) * 32;
+          tc::mma_bf16_ss_elect(tmem + x * 128, tc::desc_advance(qd, off), tc::desc_advance(kd, off), idesc_s,
+                                kk != 0);
+        }
+        tc::mma_commit_elect(&bars->s_full[x]);
+        if (last) tc::mma_commit_elect(&bars->q_empty[x]);
+      };
+      for (int x = 0; ok && x < 2; ++x)
+        if ((x ? rb : ra).n && !tc::mbar_wait_warp(&bars->q_full[x], qn[x]++ & 1, abort, kWaitNs)) ok = false;
       if (!ok) break;
-      tc::mma_commit_elect(&bars->kv_empty[sv]);
+      {
+        const int st = u % kFwdRing;
+        if (!tc::mbar_wait_warp(&bars->kv_full[st], (u / kFwdRing) & 1, abort, kWaitNs)) { ok = false; break; }
+        tc::tc_fence_after();
+        for (int x = 0; x < 2; ++x)
+          if (step_of(x, 0) == 0) issue_s(x, st, (x ? rb : ra).n == 1);
+        issued_any = true;
+        tc::mma_commit_elect(&bars->kv_empty[st]);
+      }
+      for (int j = 0; ok && j < n_kt; ++j) {
+        const int uv = u + 2 * j + 1, sv = uv % kFwdRing;
+        const int uk = u + 2 * j + 2, sk = uk % kFwdRing;  // K of step j+1
+        if (!tc::mbar_wait_warp(&bars->kv_full[sv], (uv / kFwdRing) & 1, abort, kWaitNs)) { ok = false; break; }
+        const uint64_t vd = tc::smem_desc_sw128(ring0 + sv * S::TILE, CH);
+        bool k_waited = false;
+        for (int x = 0; ok && x < 2; ++x) {
+          const int i = step_of(x, j);
+          if (i >= 0) {
+            if (!tc::mbar_wait_warp(&bars->p_ready[x], (cs[x] + i) & 1, abort, kWaitNs)) { ok = false; break; }
+            tc::tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 128 / 16; ++kk)
+              tc::mma_bf16_ts_elect(tmem + 256 + x * 128, tmem + x * 128 + 8 * kk, tc::desc_advance(vd, kk * 2048),
+                                    idesc_pv, (i | kk) != 0);
+            tc::mma_commit_elect(&bars->pv_done[x]);
+          }
+          const int i1 = j + 1 < n_kt ? step_of(x, j + 1) : -1;
+          if (i1 >= 0) {
+            if (!k_waited) {
+              if (!tc::mbar_wait_warp(&bars->kv_full[sk], (uk / kFwdRing) & 1, abort, kWaitNs)) { ok = false; break; }
+              tc::tc_fence_after();
+              k_waited = true;
+            }
+            issue_s(x, sk, i1 == (x ? rb : ra).n - 1);
+          }
+        }
+        if (!ok) break;
+        tc::mma_commit_elect(&bars->kv_empty[sv]);
+        if (k_waited) tc::mma_commit_elect(&bars->kv_empty[sk]);
+      }
+      u += 2 * n_kt;
+      cs[0] += ra.n;
+      cs[1] += rb.n;
     }
     if (!ok) {
       if (lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 11);
@@ -380,108 +489,129 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kFwdRegsSoftmax));
     // softmax: thread = one query row of tile x
     const int x = warp >> 2;
-    const KeyRange r = x ? rb : ra;
     const int row = (warp & 3) * 32 + lane;
-    const int q = (2 * pair + x) * 128 + row;
-    const int lo_key = q - W + 1;  // the row's first visible key
     const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
     const uint32_t t_s = tmem + x * 128 + lane_off, t_o = tmem + 256 + x * 128 + lane_off;
-    float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int i = 0; ok && i < r.n; ++i) {
-      const int k0 = (r.lo + i) * 128;
-      if (!tc::mbar_wait_warp(&bars->s_full[x], i & 1, abort, kWaitNs)) { ok = false; break; }
-      tc::tc_fence_after();
-      float s[128];
-      {
-        uint32_t u0[32], u1[32], u2[32], u3[32];
-        tc::tmem_ld_32x32b_x32(t_s, u0);
-        tc::tmem_ld_32x32b_x32(t_s + 32, u1);
-        tc::tmem_ld_32x32b_x32(t_s + 64, u2);
-        tc::tmem_ld_32x32b_x32(t_s + 96, u3);
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          s[e] = __uint_as_float(u0[e]);
-          s[32 + e] = __uint_as_float(u1[e]);
-          s[64 + e] = __uint_as_float(u2[e]);
-          s[96 + e] = __uint_as_float(u3[e]);
-        }
-      }
-      if (k0 + 127 > q || k0 + 128 > T || k0 < lo_key) {
-#pragma unroll
-        for (int e = 0; e < 128; ++e)
-          if (k0 + e > q || k0 + e >= T || k0 + e < lo_key) s[e] = -INFINITY;
-      }
-      float mx = s[0];
-#pragma unroll
-      for (int e = 1; e < 127; e += 2) mx = fmax3(mx, s[e], s[e + 1]);
-      mx = fmaxf(mx, s[127]) * scale_log2;  // scores are unscaled; the scale is positive
-      const bool grow = mx > m_ref + 8.f;
-      const float factor = grow ? ex2(m_ref - mx) : 1.f;
-      if (grow) {
-        l *= factor;
-        m_ref = mx;
-      }
-      // a row whose keys so far were all outside its window has no reference
-      // yet: its P is 0 (exp2(-inf - 0)), not NaN
-      const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
-      const uint64_t sc2 = f2(scale_log2, scale_log2), nm2 = f2(-m_use, -m_use);
-      uint64_t lsum2 = f2(0.f, 0.f);
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float2 xx = unf2(fma2(f2(s[64 * h + 2 * e], s[64 * h + 2 * e + 1]), sc2, nm2));
-          const float p0 = ex2(xx.x), p1 = ex2(xx.y);
-          lsum2 = add2(lsum2, f2(p0, p1));
-          pk[e] = pack2(p0, p1);
-        }
-        tc::tmem_st_32x32b_x32(t_s + 32 * h, pk);  // P over this row's first 64 S columns
-      }
-      const float2 ls = unf2(lsum2);
-      l += ls.x + ls.y;
-      if (i > 0 && __any_sync(0xffffffffu, grow)) {
-        // O holds P V up to step i-1 once that product is done
-        if (!tc::mbar_wait_warp(&bars->pv_done[x], (i - 1) & 1, abort, kWaitNs)) { ok = false; break; }
+    int cs = 0;  // this tile's steps done over the previous items
+    for (int seq = 0; ok; ++seq) {
+      const int s = seq & 1;
+      if (!tc::mbar_wait_warp(&bars->item_full[s], (seq >> 1) & 1, abort, kWaitNs)) { ok = false; break; }
+      const int k = items[s];
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&bars->item_empty[s]);
+      if (k < 0) break;
+      int bh, pair;
+      KeyRange ra, rb;
+      decode(k, bh, pair, ra, rb);
+      const KeyRange r = x ? rb : ra;
+      const int q = (2 * pair + x) * 128 + row;
+      const int lo_key = q - W + 1;  // the row's first visible key
+      float m_ref = -INFINITY, l = 0.f;
+      for (int i = 0; ok && i < r.n; ++i) {
+        const int k0 = (r.lo + i) * 128;
+        if (!tc::mbar_wait_warp(&bars->s_full[x], (cs + i) & 1, abort, kWaitNs)) { ok = false; break; }
         tc::tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < HD; c += 32) {
-          uint32_t u[32];
-          tc::tmem_ld_32x32b_x32(t_o + c, u);
+        float sc[128];
+        {
+          uint32_t u0[32], u1[32], u2[32], u3[32];
+          tc::tmem_ld_32x32b_x32(t_s, u0);
+          tc::tmem_ld_32x32b_x32(t_s + 32, u1);
+          tc::tmem_ld_32x32b_x32(t_s + 64, u2);
+          tc::tmem_ld_32x32b_x32(t_s + 96, u3);
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * factor);
-          tc::tmem_st_32x32b_x32(t_o + c, u);
+          for (int e = 0; e < 32; ++e) {
+            sc[e] = __uint_as_float(u0[e]);
+            sc[32 + e] = __uint_as_float(u1[e]);
+            sc[64 + e] = __uint_as_float(u2[e]);
+            sc[96 + e] = __uint_as_float(u3[e]);
+          }
         }
+        if (k0 + 127 > q || k0 + 128 > T || k0 < lo_key) {
+#pragma unroll
+          for (int e = 0; e < 128; ++e)
+            if (k0 + e > q || k0 + e >= T || k0 + e < lo_key) sc[e] = -INFINITY;
+        }
+        float m4[4] = {sc[0], sc[1], sc[2], sc[3]};  // four independent chains
+#pragma unroll
+        for (int e = 4; e < 128; e += 8)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) m4[c] = fmax3(m4[c], sc[e + 2 * c], sc[e + 2 * c + 1]);
+        // scores are unscaled here; the scale is positive
+        float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * scale_log2;
+        const bool grow = mx > m_ref + 8.f;
+        const float factor = grow ? ex2(m_ref - mx) : 1.f;
+        if (grow) {
+          l *= factor;
+          m_ref = mx;
+        }
+        // a row whose keys so far were all outside its window has no reference
+        // yet: its P is 0 (exp2(-inf - 0)), not NaN
+        const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
+        const uint64_t sc2 = f2(scale_log2, scale_log2), nm2 = f2(-m_use, -m_use);
+        uint64_t lsum2[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float2 xx = unf2(fma2(f2(sc[64 * h + 2 * e], sc[64 * h + 2 * e + 1]), sc2, nm2));
+            const float p0 = ex2(xx.x), p1 = ex2(xx.y);
+            lsum2[e & 3] = add2(lsum2[e & 3], f2(p0, p1));
+            pk[e] = pack2(p0, p1);
+          }
+          tc::tmem_st_32x32b_x32(t_s + 32 * h, pk);  // P over this row's first 64 S columns
+        }
+        const float2 ls = unf2(add2(add2(lsum2[0], lsum2[1]), add2(lsum2[2], lsum2[3])));
+        l += ls.x + ls.y;
+        if (i > 0 && __any_sync(0xffffffffu, grow)) {
+          // O holds P V up to step i-1 once that product is done
+          if (!tc::mbar_wait_warp(&bars->pv_done[x], (cs + i - 1) & 1, abort, kWaitNs)) { ok = false; break; }
+          tc::tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < HD; c += 32) {
+            uint32_t uu[32];
+            tc::tmem_ld_32x32b_x32(t_o + c, uu);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) uu[e] = __float_as_uint(__uint_as_float(uu[e]) * factor);
+            tc::tmem_st_32x32b_x32(t_o + c, uu);
+          }
+        }
+        tc::tmem_wait_st();
+        tc::tc_fence_before();
+        tc::mbar_arrive(&bars->p_ready[x]);
       }
-      tc::tmem_wait_st();
-      tc::tc_fence_before();
-      tc::mbar_arrive(&bars->p_ready[x]);
+      if (!ok) break;
+      if (r.n > 0) {
+        if (!tc::mbar_wait_warp(&bars->pv_done[x], (cs + r.n - 1) & 1, abort, kWaitNs)) { ok = false; break; }
+        tc::tc_fence_after();
+        const int b = bh / H, h = bh % H;
+        const float inv = 1.f / l;
+        __nv_bfloat16* dst = o + (int64_t(b) * T + q) * (int64_t(H) * HD) + h * HD;
+#pragma unroll
+        for (int c = 0; c < HD; c += 32) {
+          float v[32];
+          tmem_ld<32>(t_o + c, v);
+          if (q < T) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 8)
+              *reinterpret_cast<uint4*>(dst + c + e) =
+                  make_uint4(pack2(v[e] * inv, v[e + 1] * inv), pack2(v[e + 2] * inv, v[e + 3] * inv),
+                             pack2(v[e + 4] * inv, v[e + 5] * inv), pack2(v[e + 6] * inv, v[e + 7] * inv));
+          }
+        }
+        if (q < T) lse[int64_t(bh) * T + q] = (m_ref + __log2f(l)) * 0.69314718055994531f;
+        // the next item's first O_x += P_x V overwrites these columns only
+        // after this warp's next p_ready arrival, which follows these reads
+        tc::tc_fence_before();
+      }
+      cs += r.n;
     }
-    if (ok && r.n > 0) ok = tc::mbar_wait_warp(&bars->pv_done[x], (r.n - 1) & 1, abort, kWaitNs);
     if (!ok) {
       if (lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 12);
       *abort = 1;
-    } else if (r.n > 0) {
-      tc::tc_fence_after();
-      const int b = bh / H, h = bh % H;
-      const float inv = 1.f / l;
-      __nv_bfloat16* dst = o + (int64_t(b) * T + q) * (int64_t(H) * HD) + h * HD;
-#pragma unroll
-      for (int c = 0; c < HD; c += 32) {
-        float v[32];
-        tmem_ld<32>(t_o + c, v);
-        if (q < T) {
-#pragma unroll
-          for (int e = 0; e < 32; e += 8)
-            *reinterpret_cast<uint4*>(dst + c + e) =
-                make_uint4(pack2(v[e] * inv, v[e + 1] * inv), pack2(v[e + 2] * inv, v[e + 3] * inv),
-                           pack2(v[e + 4] * inv, v[e + 5] * inv), pack2(v[e + 6] * inv, v[e + 7] * inv));
-        }
-      }
-      if (q < T) lse[int64_t(bh) * T + q] = (m_ref + __log2f(l)) * 0.69314718055994531f;
     }
   }
   __syncwarp();
@@ -491,6 +621,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, 512);
   }
+  if (threadIdx.x == 0) sched_finish(sched);
+}
+
+int num_sms() {
+  static int n[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!n[dev] && cudaDeviceGetAttribute(&n[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    n[dev] = 148;
+  return n[dev];
 }
 
 namespace {
@@ -507,10 +647,11 @@ int attn_fwd_tc_t(const gpt_config& c, const void* q, const void* k, const void*
   const int smem = int(FwdSmem<HD>::BYTES);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return 1;
-  const int n_pairs = ((c.seq_len + 127) / 128 + 1) / 2;
-  kern<<<n_pairs * c.batch * c.n_head, kFwdThreads, smem, st>>>(
+  const int n_rows = c.batch * c.n_head;
+  const int n_items = ((c.seq_len + 127) / 128 + 1) / 2 * n_rows;
+  kern<<<std::min(n_items, num_sms()), kFwdThreads, smem, st>>>(
       mq, mk, mv, static_cast<__nv_bfloat16*>(o), lse, c.n_head, c.n_kv_head, c.seq_len,
-      window_span(c), kLog2e / sqrtf(float(HD)), status);
+      window_span(c), kLog2e / sqrtf(float(HD)), n_rows, status);
   return last_launch_rc();
 }
 }  // namespace
@@ -724,8 +865,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   BwdBars* bars = reinterpret_cast<BwdBars*>(smem + S::BAR_OFF);
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int n_qt = (T + 127) / 128;
-  const int bh = int(blockIdx.x) / n_qt;  // (batch, head)-major, as in the forward
-  const int qt = n_qt - 1 - int(blockIdx.x) % n_qt;
+  int bh, rank;
+  grouped_item(int(blockIdx.x), int(gridDim.x) / n_qt, n_qt, bh, rank);  // longest first
+  const int qt = n_qt - 1 - rank;
   const int b = bh / H, h = bh % H;
   const int q0 = qt * 128;
   const int s_lo = max(0, q0 - W + 1) / kInner;  // first key step with a visible key
@@ -975,8 +1117,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   BwdBars* bars = reinterpret_cast<BwdBars*>(smem + S::BAR_OFF);
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int n_kt = (T + 127) / 128;
-  const int bkv = int(blockIdx.x) / n_kt;  // (batch, kv head)-major; key tile 0 first
-  const int kt = int(blockIdx.x) % n_kt;
+  int bkv, kt;  // key tile 0 (the most queries) first
+  grouped_item(int(blockIdx.x), int(gridDim.x) / n_kt, n_kt, bkv, kt);
   const int b = bkv / Hkv, hk = bkv % Hkv, rep = H / Hkv;
   const int k0 = kt * 128;
   const int i_begin = k0 / kInner;

@@ -125,6 +125,7 @@ struct Layout {
   // optimizer scratch (bf16 configs): Newton-Schulz iterates, Gram matrices,
   // sum-of-squares partials
   uint64_t opt_x0, opt_x1, opt_a, opt_b, opt_part;
+  uint64_t opt_rows;       // NorMuon per-row scratch: v_mean and factors [2][max rows]
   // e4m3 forward projections (fp8 configs): weight codes at the parameter
   // buffer's element offsets (one byte each), their dequantization factors
   // and amax bits [4 kinds][n_layer], one activation's codes [N, max(d, F)]
@@ -152,6 +153,14 @@ int launch_muon_prepare(const void* grads, float* mom, int64_t n, float mu, int 
                         float* partial, void* x_out, void* stream);
 // master -= step * x; params = bf16(master)
 int launch_muon_apply(const void* x, float* master, void* params, int64_t n, float step, void* stream);
+// NorMuon row factors of one update x [rows, cols]: buf (per-row state) is
+// updated; factor[r] = step_size[r] * v_norm / max(v_norm_new, 1e-10); vmean:
+// rows floats of scratch
+int launch_normuon(const void* x, float* buf, int rows, int cols, float beta2, float* vmean,
+                   float* factor, void* stream);
+// master -= step * factor[row] * x; params = bf16(master)
+int launch_muon_apply_rows(const void* x, float* master, void* params, int rows, int cols,
+                           float step, const float* factor, void* stream);
 
 // ---- launchers (all enqueue on `stream`, return cudaError_t as int) ------
 int launch_rope_table(const gpt_config& c, float* cos_t, float* sin_t, void* stream);

@@ -1,7 +1,8 @@
 // Element-wise parts of the optimizer step: AdamW for the embedding and
-// lm_head, and Muon's momentum, Frobenius normalisation and update for the
-// block matrices ("ChatGPT'nizi 50 Dolara Nasil Egitirsiniz?", section "2. Muon
-// Optimize Edici (nanochat/optim.py)").  The Newton-Schulz products between
+// lm_head, and Muon's momentum, Frobenius normalisation, NorMuon row rescale
+// and update for the block matrices ("ChatGPT'nizi 50 Dolara Nasil
+// Egitirsiniz?", section "2. Muon Optimize Edici (nanochat/optim.py)", and its
+// "NorMuon Varyans Azaltma" lines).  The Newton-Schulz products between
 // the normalisation and the update run on the tensor-core GEMM (EPI_AXPBY).
 //
 // All kernels are HBM-bound streams over 8-element groups (16-byte bf16 and
@@ -151,6 +152,76 @@ __global__ void muon_apply_kernel(const __nv_bfloat16* __restrict__ x, float* __
   }
 }
 
+// NorMuon, per row r of one orthogonalised update X [rows, cols] (bf16):
+// v_mean = mean_c X[r,c]^2; buf = beta2 buf + (1 - beta2) v_mean (the per-row
+// state); step = 1 / sqrt(max(buf, 1e-10)).  One warp per row, a fixed
+// lane-strided order.
+__global__ void normuon_rows_kernel(const __nv_bfloat16* __restrict__ x, float* __restrict__ buf,
+                                    int rows, int cols, float beta2, float* __restrict__ vmean,
+                                    float* __restrict__ step) {
+  const int r = int(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
+  if (r >= rows) return;
+  const __nv_bfloat16* row = x + int64_t(r) * cols;
+  float s = 0.f;
+  for (int c = threadIdx.x & 31; c < cols; c += 32) {
+    const float v = __bfloat162float(row[c]);
+    s += v * v;
+  }
+  s = warp_sum(s);
+  if ((threadIdx.x & 31) == 0) {
+    const float vm = s / float(cols);
+    const float b = beta2 * buf[r] + (1.f - beta2) * vm;
+    buf[r] = b;
+    vmean[r] = vm;
+    step[r] = 1.f / sqrtf(fmaxf(b, 1e-10f));
+  }
+}
+
+// The matrix-wide factor v_norm / max(v_norm_new, 1e-10) with v_norm^2 =
+// sum_r v_mean[r] and v_norm_new^2 = sum_r v_mean[r] step[r]^2 (one block, a
+// fixed summation order), folded into step[r] in place: the row factors.
+__global__ void normuon_scale_kernel(const float* __restrict__ vmean, float* __restrict__ step,
+                                     int rows) {
+  __shared__ float red[2][32];
+  float s1 = 0.f, s2 = 0.f;
+  for (int r = threadIdx.x; r < rows; r += blockDim.x) {
+    s1 += vmean[r];
+    s2 += vmean[r] * step[r] * step[r];
+  }
+  s1 = warp_sum(s1);
+  s2 = warp_sum(s2);
+  if ((threadIdx.x & 31) == 0) {
+    red[0][threadIdx.x / 32] = s1;
+    red[1][threadIdx.x / 32] = s2;
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const bool in = threadIdx.x < blockDim.x / 32;
+    s1 = warp_sum(in ? red[0][threadIdx.x] : 0.f);
+    s2 = warp_sum(in ? red[1][threadIdx.x] : 0.f);
+    if (threadIdx.x == 0) red[0][0] = sqrtf(s1) / fmaxf(sqrtf(s2), 1e-10f);
+  }
+  __syncthreads();
+  const float scale = red[0][0];
+  for (int r = threadIdx.x; r < rows; r += blockDim.x) step[r] *= scale;
+}
+
+// master -= step * factor[row] * x; params = bf16(master)
+__global__ void muon_apply_rows_kernel(const __nv_bfloat16* __restrict__ x, float* __restrict__ w,
+                                       __nv_bfloat16* __restrict__ p, int64_t n8, int cols,
+                                       float step, const float* __restrict__ factor) {
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    float xf[8], wf[8];
+    load8_bf16(x + 8 * i, xf);
+    load8_f32(w + 8 * i, wf);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) wf[e] -= step * factor[(8 * i + e) / cols] * xf[e];
+    store8_f32(w + 8 * i, wf);
+    store8_bf16(p + 8 * i, wf);
+  }
+}
+
 int stream_grid(int64_t n8) {
   const int64_t want = (n8 + 255) / 256;
   return int(want < 148 * 8 ? (want > 0 ? want : 1) : 148 * 8);
@@ -191,6 +262,25 @@ int launch_muon_apply(const void* x, float* master, void* params, int64_t n, flo
   if (n % 8) return 1;
   muon_apply_kernel<<<stream_grid(n / 8), 256, 0, (cudaStream_t)stream>>>(
       static_cast<const __nv_bfloat16*>(x), master, static_cast<__nv_bfloat16*>(params), n / 8, step);
+  return last_launch_rc();
+}
+
+int launch_normuon(const void* x, float* buf, int rows, int cols, float beta2, float* vmean,
+                   float* factor, void* stream) {
+  cudaStream_t st = (cudaStream_t)stream;
+  normuon_rows_kernel<<<(rows + 7) / 8, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), buf, rows,
+                                                      cols, beta2, vmean, factor);
+  normuon_scale_kernel<<<1, 1024, 0, st>>>(vmean, factor, rows);
+  return last_launch_rc();
+}
+
+int launch_muon_apply_rows(const void* x, float* master, void* params, int rows, int cols,
+                           float step, const float* factor, void* stream) {
+  const int64_t n = int64_t(rows) * cols;
+  if (n % 8) return 1;
+  muon_apply_rows_kernel<<<stream_grid(n / 8), 256, 0, (cudaStream_t)stream>>>(
+      static_cast<const __nv_bfloat16*>(x), master, static_cast<__nv_bfloat16*>(params), n / 8, cols,
+      step, factor);
   return last_launch_rc();
 }
 

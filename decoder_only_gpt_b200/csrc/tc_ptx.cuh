@@ -47,17 +47,35 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The same test, letting the thread sleep until the phase completes or
+// kSuspendNs nanoseconds pass: a waiting warp then takes no issue slots from
+// the warps that share its scheduler (the MMA issuer, the other tile's
+// softmax), which a hot polling loop would.
+constexpr uint32_t kSuspendNs = 20000;
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "n"(kSuspendNs)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait until the phase with the given parity has completed.  Gives up after
 // `limit_ns` nanoseconds (or early once *abort is set by another role, when
 // `abort` is not null), returning false; the caller then records
-// GPT_ETIMEOUT and unwinds.
+// GPT_ETIMEOUT and unwinds.  Between the checks of the limit and of *abort
+// the thread sleeps in try_wait (at most kSuspendNs at a time).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   volatile int* abort, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 0;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63) == 63) {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    if ((it & 7) == 7) {
       if (abort && *abort) return false;
       if (global_timer_ns() - t0 > limit_ns) return false;
     }

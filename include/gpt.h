@@ -252,6 +252,13 @@ int gpt_wait_expiry_check(void* workspace, int64_t limit_ns, void* stream);
  *           X = U / (||U||_F + 1e-7), then ns_steps iterations with
  *           (a, b, c) = ns_coeffs[i] in bf16 on the tensor cores;
  *           w = w - lr sqrt(max(1, rows/cols)) X.
+ *   NorMuon (normuon = 1; the section's "NorMuon Varyans Azaltma" lines,
+ *   whose undefined names are read after the published NorMuon method): per
+ *   row r of X, v_mean = mean_c X^2; the row's state buf = beta2 buf +
+ *   (1-beta2) v_mean (fp32, stored in the matrix's first `rows` v slots,
+ *   zero after gpt_optim_init); step_r = 1/sqrt(max(buf, 1e-10)); X row r is
+ *   scaled by step_r sqrt(sum v_mean) / max(sqrt(sum v_mean step^2), 1e-10)
+ *   (the Frobenius norm of X is kept) before the update above.
  * bf16 configurations only (dtype GPT_F32 returns GPT_EUNSUPPORTED). */
 typedef struct {
   float adam_lr, adam_beta1, adam_beta2, adam_eps, adam_weight_decay;
@@ -260,6 +267,8 @@ typedef struct {
   int32_t ns_steps;        /* 0 .. 8 */
   float ns_coeffs[8][3];   /* (a, b, c) of iteration i */
   int64_t step;            /* AdamW step count t >= 1 */
+  int32_t normuon;         /* 1: NorMuon row rescale of the orthogonalised update */
+  float normuon_beta2;     /* its second-moment decay, in [0, 1) */
 } gpt_optim;
 
 /* Library defaults (the pages give no hyper-parameter values): AdamW lr 1e-3,
@@ -267,7 +276,8 @@ typedef struct {
  * decay; Muon lr 0.02, momentum 0.95, Nesterov; ns_steps 2 with the two
  * coefficient triples the page prints, (8.156, -22.483, 15.879) and
  * (4.043, -2.809, 0.5) (its list of five breaks off there: longer schedules
- * are the caller's); step 1.  Returns GPT_EINVAL for a NULL pointer. */
+ * are the caller's); step 1; NorMuon off, its beta2 0.95 (the published
+ * method's value).  Returns GPT_EINVAL for a NULL pointer. */
 int gpt_optim_defaults(gpt_optim* opt);
 /* Bytes of the optimizer state for an initialised config (3 fp32 copies of
  * the parameter buffer's elements). */
@@ -281,7 +291,8 @@ int gpt_optim_init(const gpt_config* cfg, const void* params, void* state, void*
  * a gpt_backward after it needs a new gpt_forward_loss first, as the new
  * parameters do anyway.  Async on `stream`, deterministic.  GPT_EINVAL for NULL or
  * misaligned pointers, ns_steps outside 0..8, step < 1, betas outside [0, 1)
- * or non-finite hyper-parameters. */
+ * (NorMuon's included, when on), normuon not 0 or 1, or non-finite
+ * hyper-parameters. */
 int gpt_optim_step(const gpt_config* cfg, const gpt_optim* opt, void* params, const void* grads,
                    void* state, void* workspace, void* stream);
 

@@ -32,11 +32,27 @@ Readings where the pages are silent or the text breaks off
   the Gram matrix over the smaller dimension (for a wide X the same map is
   applied to X^T: A = X X^T, X <- a X + B X);  theta <- theta - lr s X_final
   with s = sqrt(max(1, rows / cols)); no weight decay on these matrices.
-* Coefficients are the caller's; the library's default schedule is the two
-  printed triples followed by the second one repeated (the page's list breaks
+* Coefficients are the caller's.  The library's default schedule is the two
+  printed triples only (ns_steps = 2); ``default_coeffs(n)`` here pads a
+  longer test schedule with the last printed triple (the page's list breaks
   off after two entries).
-* The NorMuon variance rescale is not built: its printed fragment uses names
-  it never defines (red_dim, v_norm_new, step_size).
+* NorMuon (same section, "NorMuon Varyans Azaltma"): the page prints the
+  rescale of the orthogonalised update g as four lines that use three names
+  it never defines (red_dim, step_size, v_norm_new).  Reading, after the
+  published NorMuon method (Li et al., 2025: one second-moment estimate per
+  output neuron of the orthogonalised update, the update normalised by it):
+    - red_dim is the column dimension: v_mean[r] = mean_c g[r, c]^2, one per
+      row (output neuron) of the [out, in] matrix;
+    - v_norm = sqrt(sum_r v_mean[r]), as printed;
+    - a per-row state buf (fp32, zero at init) follows the EMA
+      buf <- beta2 buf + (1 - beta2) v_mean, beta2 = 0.95 by default (the
+      published method's value); step_size[r] = 1 / sqrt(max(buf[r], 1e-10));
+    - v_norm_new is the same statistic of the rescaled update g * step_size:
+      sqrt(sum_r v_mean[r] step_size[r]^2);
+    - final_scale[r] = step_size[r] v_norm / max(v_norm_new, 1e-10) and
+      g <- g * final_scale, as printed: each row keeps its direction and the
+      update keeps its Frobenius norm, only its spread over the rows changes.
+  The Muon update then uses the rescaled g.
 """
 from __future__ import annotations
 
@@ -51,6 +67,7 @@ __all__ = [
     "adamw",
     "ns_iteration",
     "newton_schulz",
+    "normuon",
     "muon",
     "optimizer_step",
     "is_muon",
@@ -106,17 +123,36 @@ def newton_schulz(u: np.ndarray, coeffs: Sequence[Tuple[float, float, float]]) -
     return x
 
 
+def normuon(x: np.ndarray, buf: np.ndarray, beta2: float):
+    """The NorMuon rescale of an orthogonalised update x [rows, cols] with the
+    per-row second-moment state buf [rows] (reading in the module docstring).
+    Returns (x rescaled, new buf)."""
+    x = np.asarray(x, np.float64)
+    v_mean = np.mean(x * x, axis=1)                       # red_dim: the columns
+    v_norm = math.sqrt(float(np.sum(v_mean)))
+    buf = beta2 * np.asarray(buf, np.float64) + (1.0 - beta2) * v_mean
+    step_size = 1.0 / np.sqrt(np.maximum(buf, 1e-10))
+    v_norm_new = math.sqrt(float(np.sum(v_mean * step_size * step_size)))
+    final_scale = step_size * (v_norm / max(v_norm_new, 1e-10))
+    return x * final_scale[:, None], buf
+
+
 def muon(theta, g, mom, lr: float, mu: float, nesterov: bool,
-         coeffs: Sequence[Tuple[float, float, float]]):
-    """One Muon step on a [rows, cols] matrix.  Returns (theta, mom, x_final)."""
+         coeffs: Sequence[Tuple[float, float, float]], normuon_buf=None, normuon_beta2: float = 0.95):
+    """One Muon step on a [rows, cols] matrix.  With ``normuon_buf`` (the
+    per-row state) the orthogonalised update is NorMuon-rescaled first.
+    Returns (theta, mom, x_final, new normuon_buf or None)."""
     theta = np.asarray(theta, np.float64)
     g = np.asarray(g, np.float64)
     mom = mu * np.asarray(mom, np.float64) + g
     u = g + mu * mom if nesterov else mom
     x = newton_schulz(u, coeffs)
+    buf = None
+    if normuon_buf is not None:
+        x, buf = normuon(x, normuon_buf, normuon_beta2)
     rows, cols = theta.shape
     scale = math.sqrt(max(1.0, rows / cols))
-    return theta - lr * scale * x, mom, x
+    return theta - lr * scale * x, mom, x, buf
 
 
 def is_muon(name: str) -> bool:
@@ -127,15 +163,25 @@ def is_muon(name: str) -> bool:
 def optimizer_step(master: Dict[str, np.ndarray], grads: Dict[str, np.ndarray],
                    m: Dict[str, np.ndarray], v: Dict[str, np.ndarray], hp: dict):
     """One optimizer step over every tensor.  ``hp`` keys: adam_lr, beta1,
-    beta2, eps, weight_decay, muon_lr, momentum, nesterov, coeffs, step.
-    For Muon tensors ``m`` holds the momentum and ``v`` is unused.
+    beta2, eps, weight_decay, muon_lr, momentum, nesterov, coeffs, step, and
+    optionally normuon (bool) and normuon_beta2.  For Muon tensors ``m``
+    holds the momentum and ``v`` the NorMuon state in its first ``rows``
+    entries (flattened; the rest unused, as the library's state buffer).
     Returns new (master, m, v) dicts (float64)."""
     out_w, out_m, out_v = {}, {}, {}
     for name, w in master.items():
         if is_muon(name):
-            w2, mom, _ = muon(w, grads[name], m[name], hp["muon_lr"], hp["momentum"],
-                              bool(hp["nesterov"]), hp["coeffs"])
-            out_w[name], out_m[name], out_v[name] = w2, mom, np.asarray(v[name], np.float64)
+            vv = np.array(v[name], np.float64)
+            rows = w.shape[0]
+            buf = vv.ravel()[:rows] if hp.get("normuon") else None
+            w2, mom, _, buf = muon(w, grads[name], m[name], hp["muon_lr"], hp["momentum"],
+                                   bool(hp["nesterov"]), hp["coeffs"], buf,
+                                   hp.get("normuon_beta2", 0.95))
+            if buf is not None:
+                flat = vv.ravel()
+                flat[:rows] = buf
+                vv = flat.reshape(vv.shape)
+            out_w[name], out_m[name], out_v[name] = w2, mom, vv
         else:
             w2, m2, v2 = adamw(w, grads[name], m[name], v[name], hp["step"], hp["adam_lr"],
                                hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"])

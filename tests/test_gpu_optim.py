@@ -14,6 +14,11 @@ moments):
   <= 4.4e-2, so the bar is cosine >= 0.998, max-rel <= 0.1; with no iteration
   (normalisation only, one bf16 rounding) cosine >= 0.99999, max-rel <= 1e-2.
   The momentum buffer is fp32: max-rel <= 1e-6.
+* NorMuon (per-row rescale of the orthogonalised update, fp32 statistics of
+  the bf16 iterate): the update keeps the Muon bars of its schedule, since a
+  row factor is a smooth function of the row's mean square, whose relative
+  error averages the iterate's element errors down; its per-row state
+  max-rel <= 1e-2.
 * The bf16 parameters equal the fp32 master rounded to nearest even, bit for bit.
 """
 import numpy as np
@@ -56,7 +61,8 @@ def _hp(opt):
     return dict(adam_lr=f(opt.adam_lr), beta1=f(opt.adam_beta1), beta2=f(opt.adam_beta2),
                 eps=f(opt.adam_eps), weight_decay=f(opt.adam_weight_decay), muon_lr=f(opt.muon_lr),
                 momentum=f(opt.muon_momentum), nesterov=int(opt.muon_nesterov),
-                coeffs=opt.coeffs(), step=int(opt.step))
+                coeffs=opt.coeffs(), step=int(opt.step), normuon=bool(opt.normuon),
+                normuon_beta2=f(opt.normuon_beta2))
 
 
 def _grads(shapes, step, names):
@@ -112,6 +118,10 @@ def _check(res, names, muon_tol):
         assert c >= tol["cos"] and mr <= tol["maxrel"], (k, c, mr)
         if OO.is_muon(k):
             assert _maxrel(res["m1"][k], res["m_ref"][k]) <= 1e-6, k
+            rows = res["v_ref"][k].shape[0]
+            buf_ref = res["v_ref"][k].ravel()[:rows]
+            if np.any(buf_ref):  # NorMuon's per-row state (fp32 from the bf16 update)
+                assert _maxrel(res["v1"][k].ravel()[:rows], buf_ref) <= 1e-2, k
         else:
             assert _maxrel(res["m1"][k], res["m_ref"][k]) <= 1e-5, k
             assert _maxrel(res["v1"][k], res["v_ref"][k]) <= 1e-5, k
@@ -160,6 +170,21 @@ def test_ragged_shapes(B, R):
                        seq_len=64, batch=2)
     results, names = _run(B, R, w, [_opt(B)])
     _check(results[0], names, MUON[2])
+
+
+@pytest.mark.parametrize("shape", ["story", "ragged"])
+def test_normuon_two_steps(B, R, shape):
+    # the per-row state carries over from the first step into the second
+    if shape == "story":
+        w = synth.workload("story")
+    else:
+        w = synth.workload("story", n_layer=2, d_model=128, n_head=2, head_dim=64, d_ff=320,
+                           vocab=1000, seq_len=64, batch=2)
+    o1, o2 = _opt(B, normuon=1, normuon_beta2=0.9), _opt(B, normuon=1, normuon_beta2=0.9)
+    o2.step = 2
+    results, names = _run(B, R, w, [o1, o2])
+    for res in results:
+        _check(res, names, MUON[2])
 
 
 def test_deterministic(B, R):

@@ -11,9 +11,12 @@ Tolerances:
 * index work (gather, stable sort of positions by token id): bit-exact.
 * e4m3 forward projections (fp8 configs) against the oracle's e4m3 reading:
   the bf16 bars at the small shapes; at full d24 size loss 1e-3, per-position
-  losses and gradient max-rel 8e-2, gradient cosine 0.995 (derived in TOL
-  below from the quantizer's sensitivity to bf16-level input differences).
+  losses 6e-2 (an oracle-only emulation over all 32,768 positions, stored in
+  tests/golden/fp8_noise_d24.json), gradient max-rel 8e-2 and cosine 0.995
+  (derived in TOL below from the quantizer's sensitivity to bf16-level input
+  differences).
 """
+import json
 import math
 import os
 
@@ -27,15 +30,25 @@ pytestmark = pytest.mark.gpu
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
+def _fp8_token_bar():
+    """Per-position loss bar of the full-size FP8 check, sized by the oracle
+    alone (tests/golden/make_fp8_noise_bars.py): its forward over all 32,768
+    d24 positions with every quantizer input perturbed by 1e-3 relative noise
+    moved the per-position losses by at most 4.0e-2; the bar is 1.5 times that."""
+    with open(os.path.join(GOLDEN, "fp8_noise_d24.json")) as f:
+        return float(json.load(f)["token_bar"])
+
+
 TOL = {
     "bf16": dict(loss=1e-3, cos=0.999, maxrel=3e-2, tok=2e-2),
     # e4m3 forward projections at full d24 size: an e4m3 code turns the
     # bf16-level difference between the GPU's and the oracle's quantizer
-    # inputs into a whole code step; the oracle with those inputs perturbed by
-    # 1e-3 relative noise moved per-position losses by up to 3.4e-2 and the
-    # embedding gradient to cosine 0.9985 / max-rel 3.9e-2 (d24, 2 sequences),
-    # so the bars are about twice that (the loss itself moved 1e-4)
-    "fp8_full": dict(loss=1e-3, cos=0.995, maxrel=8e-2, tok=8e-2),
+    # inputs into a whole code step.  The oracle with those inputs perturbed by
+    # 1e-3 relative noise moved the embedding gradient to cosine 0.9985 /
+    # max-rel 3.9e-2 (d24, 2 sequences), so the gradient bars are about twice
+    # that; the per-position bar comes from the same emulation over every d24
+    # position (the loss itself moved 2e-5)
+    "fp8_full": dict(loss=1e-3, cos=0.995, maxrel=8e-2, tok=_fp8_token_bar()),
     "f32": dict(loss=1e-5, cos=0.99999, maxrel=1e-3, tok=1e-4),
 }
 

@@ -112,7 +112,7 @@ def test_momentum_geometric_sum():
     w = np.zeros_like(G)
     mu = 0.9
     for k in range(1, 6):
-        w, mom, _ = O.muon(w, G, mom, 0.0, mu, False, O.default_coeffs(5))
+        w, mom, _, _ = O.muon(w, G, mom, 0.0, mu, False, O.default_coeffs(5))
         np.testing.assert_allclose(mom, G * (1 - mu ** k) / (1 - mu), rtol=1e-14)
 
 
@@ -123,7 +123,7 @@ def test_muon_step_on_orthogonal_gradient():
     rng = _rng(6)
     Qm, _ = np.linalg.qr(rng.standard_normal((9, 4)))
     w0 = rng.standard_normal((9, 4))
-    w1, mom, x = O.muon(w0, Qm, np.zeros((9, 4)), 0.01, 0.95, False, [(1.5, -0.5, 0.0)] * 40)
+    w1, mom, x, _ = O.muon(w0, Qm, np.zeros((9, 4)), 0.01, 0.95, False, [(1.5, -0.5, 0.0)] * 40)
     np.testing.assert_allclose(x, Qm, atol=1e-10)
     np.testing.assert_allclose(w1, w0 - 0.01 * math.sqrt(9 / 4) * Qm, atol=1e-10)
 
@@ -134,8 +134,8 @@ def test_nesterov_direction():
     # large gradient makes the 1e-7 in the normalisation negligible)
     rng = _rng(7)
     G = 1e4 * rng.standard_normal((6, 6))
-    _, _, x1 = O.muon(np.zeros((6, 6)), G, np.zeros((6, 6)), 0.1, 0.9, True, O.default_coeffs(5))
-    _, _, x0 = O.muon(np.zeros((6, 6)), G, np.zeros((6, 6)), 0.1, 0.9, False, O.default_coeffs(5))
+    _, _, x1, _ = O.muon(np.zeros((6, 6)), G, np.zeros((6, 6)), 0.1, 0.9, True, O.default_coeffs(5))
+    _, _, x0, _ = O.muon(np.zeros((6, 6)), G, np.zeros((6, 6)), 0.1, 0.9, False, O.default_coeffs(5))
     np.testing.assert_allclose(x1, x0, atol=1e-12)
 
 
@@ -144,8 +144,8 @@ def test_nesterov_two_steps_closed_form():
     rng = _rng(9)
     G1, G2 = rng.standard_normal((5, 3)), rng.standard_normal((5, 3))
     mu, coeffs = 0.9, O.default_coeffs(5)
-    w, mom, _ = O.muon(np.zeros((5, 3)), G1, np.zeros((5, 3)), 0.0, mu, True, coeffs)
-    w, mom, x = O.muon(w, G2, mom, 0.0, mu, True, coeffs)
+    w, mom, _, _ = O.muon(np.zeros((5, 3)), G1, np.zeros((5, 3)), 0.0, mu, True, coeffs)
+    w, mom, x, _ = O.muon(w, G2, mom, 0.0, mu, True, coeffs)
     np.testing.assert_allclose(mom, mu * G1 + G2, rtol=1e-14)
     np.testing.assert_allclose(x, O.newton_schulz((1 + mu) * G2 + mu * mu * G1, coeffs), atol=1e-12)
 
@@ -163,7 +163,79 @@ def test_optimizer_step_routes_tensors():
         want, _, _ = O.adamw(master[k], grads[k], zeros[k], zeros[k], 1, 1e-3, 0.8, 0.95, 1e-10, 0.0)
         np.testing.assert_allclose(w[k], want)
         assert np.all(v[k] > 0)
-    want, _, _ = O.muon(master["layers.0.wo"], grads["layers.0.wo"], zeros["layers.0.wo"], 0.02, 0.95,
+    want, _, _, _ = O.muon(master["layers.0.wo"], grads["layers.0.wo"], zeros["layers.0.wo"], 0.02, 0.95,
                         True, O.default_coeffs(5))
     np.testing.assert_allclose(w["layers.0.wo"], want)
     assert np.all(v["layers.0.wo"] == 0)
+
+
+# ---- NorMuon rescale (reading of the fragment in "2. Muon Optimize Edici") --
+
+def test_normuon_hand_worked_2x3():
+    # x rows [1, 2, 2] and [0, 0, 1]: mean squares 3 and 1/3; beta2 = 0.5 from
+    # a zero state gives buf = (1.5, 1/6), step sizes 1/sqrt(1.5) and sqrt(6);
+    # v_norm = sqrt(10/3), v_norm_new = sqrt(3/1.5 + 6/3) = 2, so the rows are
+    # scaled by sqrt(10/3)/2 * (1/sqrt(1.5), sqrt(6)) = (sqrt(5)/3, sqrt(5)):
+    # both rows end with norm sqrt(5), and the total stays sqrt(10)
+    x = np.array([[1.0, 2.0, 2.0], [0.0, 0.0, 1.0]])
+    y, buf = O.normuon(x, np.zeros(2), 0.5)
+    np.testing.assert_allclose(buf, [1.5, 1.0 / 6.0], rtol=1e-15)
+    np.testing.assert_allclose(y, [[math.sqrt(5) / 3, 2 * math.sqrt(5) / 3, 2 * math.sqrt(5) / 3],
+                                   [0.0, 0.0, math.sqrt(5)]], rtol=1e-14)
+
+
+@pytest.mark.parametrize("shape", [(7, 5), (4, 11), (16, 16)])
+def test_normuon_keeps_frobenius_norm_and_row_directions(shape):
+    rng = _rng(21)
+    x = rng.standard_normal(shape) * rng.uniform(0.1, 3.0, (shape[0], 1))
+    buf0 = rng.uniform(0.0, 2.0, shape[0])
+    y, _ = O.normuon(x, buf0, 0.9)
+    assert abs(np.linalg.norm(y) / np.linalg.norm(x) - 1.0) < 1e-13
+    # each row is a positive multiple of the input row
+    ratio = np.sum(y * x, axis=1) / np.sum(x * x, axis=1)
+    assert np.all(ratio > 0)
+    np.testing.assert_allclose(y, ratio[:, None] * x, rtol=1e-12, atol=1e-15)
+
+
+def test_normuon_equal_rows_from_zero_state_is_identity():
+    # rows of equal mean square (an orthogonal matrix) from a zero state: every
+    # step size is the same, so the norm-preserving rescale changes nothing
+    rng = _rng(22)
+    q, _ = np.linalg.qr(rng.standard_normal((6, 6)))
+    y, buf = O.normuon(q, np.zeros(6), 0.95)
+    np.testing.assert_allclose(y, q, rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(buf, np.full(6, 0.05 / 6), rtol=1e-13)
+
+
+def test_normuon_state_is_a_geometric_average():
+    # the same update k times from a zero state: buf = (1 - beta2^k) mean_c x^2
+    rng = _rng(23)
+    x = rng.standard_normal((5, 4))
+    buf = np.zeros(5)
+    for k in range(1, 6):
+        _, buf = O.normuon(x, buf, 0.8)
+        np.testing.assert_allclose(buf, (1 - 0.8 ** k) * np.mean(x * x, axis=1), rtol=1e-14)
+
+
+def test_normuon_zero_row_stays_zero():
+    x = np.array([[0.0, 0.0, 0.0], [1.0, -1.0, 2.0]])
+    y, buf = O.normuon(x, np.zeros(2), 0.95)
+    assert np.all(np.isfinite(y)) and np.all(y[0] == 0)
+    np.testing.assert_allclose(np.linalg.norm(y), np.linalg.norm(x), rtol=1e-14)
+
+
+def test_optimizer_step_keeps_normuon_state_in_v():
+    rng = _rng(24)
+    master = {"layers.0.wup": rng.standard_normal((6, 4))}
+    grads = {"layers.0.wup": rng.standard_normal((6, 4))}
+    zeros = {"layers.0.wup": np.zeros((6, 4))}
+    hp = dict(adam_lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0, muon_lr=0.02,
+              momentum=0.95, nesterov=1, coeffs=O.default_coeffs(2), step=1, normuon=True,
+              normuon_beta2=0.9)
+    w, m, v = O.optimizer_step(master, grads, zeros, zeros, hp)
+    x = O.newton_schulz(grads["layers.0.wup"] * (1 + 0.95), O.default_coeffs(2))
+    y, buf = O.normuon(x, np.zeros(6), 0.9)
+    np.testing.assert_allclose(w["layers.0.wup"], master["layers.0.wup"] - 0.02 * math.sqrt(6 / 4) * y,
+                               rtol=1e-13)
+    np.testing.assert_allclose(v["layers.0.wup"].ravel()[:6], buf, rtol=1e-14)
+    assert np.all(v["layers.0.wup"].ravel()[6:] == 0)
