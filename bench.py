@@ -13,9 +13,11 @@ other depth the metric names.  MFU is against the nominal dense bf16 peak
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Multi-GPU runs (under torchrun) are replicas: every rank runs the whole step
-on its own batch; ranks meet only at the timing barriers, and the reported
-time is the maximum over ranks.  Rank 0 prints one JSON line.
+Multi-GPU runs (under torchrun) are replicas by default: every rank runs the
+whole step on its own batch; ranks meet only at the timing barriers, and the
+reported time is the maximum over ranks.  With --dp the ranks also sum their
+gradients (data-parallel training, NCCL all-reduce per layer bucket,
+overlapped with the backward).  Rank 0 prints one JSON line.
 
 --impl reference times the fp64 CPU oracle (the only reference there is) on
 the host cores, on a bounded sample of the same workload per step.
@@ -325,13 +327,15 @@ def replica_throughput(tokens_per_step, steps, world, max_ms):
 def measure(w, args, rank, world, dev, barrier, *, optimizer=False, e2e=True):
     """Time one workload: an untraced timed region (the headline), then a
     second pass with the per-launch trace attached (the per-kernel breakdown
-    and the roofline site), then the end-to-end host-buffer pass."""
+    and the roofline site), then the end-to-end host-buffer pass.  With
+    --dp (and several ranks) every step is a data-parallel step: the ranks'
+    gradients are summed over NCCL, overlapped with the backward."""
     import torch
 
     from decoder_only_gpt_b200 import binding as B
     from decoder_only_gpt_b200 import runtime as R
 
-    wr = w.replace(seed=w.seed + 100 * rank)  # each replica its own batch
+    wr = w.replace(seed=w.seed + 100 * rank)  # each rank its own batch
     cfg = B.config_from_workload(w)
     st = R.TrainStep(cfg, device=str(dev))
     bits = synth.make_params(w, as_bits=True)
@@ -340,9 +344,14 @@ def measure(w, args, rank, world, dev, barrier, *, optimizer=False, e2e=True):
     st.set_batch(tok, tgt)
     N = w.batch * w.seq_len
     stream = torch.cuda.current_stream(dev)
+    dps = None
+    if args.dp and world > 1:
+        from decoder_only_gpt_b200 import dp
+        dps = dp.DataParallelStep(st)
+    one_step = dps.run if dps is not None else st.step
 
     for _ in range(args.warmup):
-        st.step()
+        one_step()
     torch.cuda.synchronize()
     code = st.status()
     if code != B.GPT_OK:
@@ -363,7 +372,7 @@ def measure(w, args, rank, world, dev, barrier, *, optimizer=False, e2e=True):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
-        st.step()
+        one_step()
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -382,7 +391,7 @@ def measure(w, args, rank, world, dev, barrier, *, optimizer=False, e2e=True):
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for _ in range(args.steps):
-        st.step()
+        one_step()
     t1.record(stream)
     torch.cuda.synchronize()
     B.Trace.detach()
@@ -394,7 +403,28 @@ def measure(w, args, rank, world, dev, barrier, *, optimizer=False, e2e=True):
 
     # ---- end to end through the public host-buffer call ----
     e2e_ms = None
-    if e2e:
+    if e2e and dps is not None:
+        # the data-parallel step through its public call: this step's tokens
+        # and targets from pinned host memory, the global loss back to the host
+        ht = torch.from_numpy(tok.ravel().copy()).pin_memory()
+        hy = torch.from_numpy(tgt.ravel().copy()).pin_memory()
+        hl = torch.zeros(1, dtype=torch.float32).pin_memory()
+        barrier()
+        torch.cuda.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.steps):
+            st.tokens.copy_(ht, non_blocking=True)
+            st.targets.copy_(hy, non_blocking=True)
+            dps.run()
+            hl.copy_(dps.global_loss, non_blocking=True)
+            stream.synchronize()
+            assert math.isfinite(float(hl[0]))
+        f1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = f0.elapsed_time(f1)
+    elif e2e:
         ht = torch.from_numpy(tok.ravel().copy()).pin_memory()
         hy = torch.from_numpy(tgt.ravel().copy()).pin_memory()
         hl = torch.zeros(1, dtype=torch.float32).pin_memory()
@@ -516,7 +546,9 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic (Zipf(1.1) token ids, seeded N(0,0.02) bf16 weights)",
         "config": {"workload": workload_desc(w), "global_batch": w.batch * world,
                    "seq_len": w.seq_len, "tokens_per_step": N * world,
-                   "parallelism": f"replicas only x{world}" if world > 1 else "single GPU",
+                   "parallelism": (f"data parallel x{world} (gradients summed over NCCL, overlapped with "
+                                   "the backward)" if args.dp else f"replicas only x{world}")
+                                  if world > 1 else "single GPU",
                    "l2": "no flush: every step moves tens of GB, far above the 126 MB L2",
                    "timing": "headline untraced; breakdown and roofline from a second, traced pass"},
         "mfu": s["mfu"],
@@ -596,6 +628,9 @@ def main():
     ap.add_argument("--workload", default=WORKLOAD, choices=list(synth.WORKLOADS))
     ap.add_argument("--no-optimizer", action="store_true",
                     help="skip the separate timing of the optimizer step")
+    ap.add_argument("--dp", action="store_true",
+                    help="with several ranks: data-parallel steps (the ranks' gradients summed over "
+                         "NCCL, overlapped with the backward) instead of independent replicas")
     ap.add_argument("--no-second", action="store_true",
                     help="skip the depth-12 measurement that default runs add")
     ap.add_argument("--no-cpu-baseline", action="store_true",

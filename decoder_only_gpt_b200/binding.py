@@ -86,6 +86,8 @@ def lib() -> ctypes.CDLL:
         L.gpt_workspace_region.argtypes = [cfgp, I, I, ctypes.POINTER(U64), ctypes.POINTER(U64)]
         L.gpt_forward_loss.argtypes = [cfgp, P, P, P, P, P, P, P]
         L.gpt_backward.argtypes = [cfgp, P, P, P, P, P, I, P]
+        L.gpt_backward_ex.argtypes = [cfgp, P, P, P, P, P, I, ctypes.c_float,
+                                      ctypes.POINTER(ctypes.c_void_p), I, P]
         L.gpt_train_step_host.argtypes = [cfgp, P, P, P, P, P, I, P, P]
         L.gpt_status.argtypes = [P, P]
         L.gpt_strerror.argtypes = [I]
@@ -99,7 +101,7 @@ def lib() -> ctypes.CDLL:
         L.gpt_wait_expiry_check.argtypes = [P, ctypes.c_int64, P]
         for f in ("gpt_config_init", "gpt_config_from_depth", "gpt_param_offset",
                   "gpt_workspace_region", "gpt_forward_loss", "gpt_backward",
-                  "gpt_train_step_host", "gpt_status", "gpt_optim_defaults",
+                  "gpt_backward_ex", "gpt_train_step_host", "gpt_status", "gpt_optim_defaults",
                   "gpt_optim_state_bytes", "gpt_optim_init", "gpt_optim_step",
                   "gpt_wait_expiry_check"):
             getattr(L, f).restype = I
@@ -208,6 +210,24 @@ def backward(cfg, tokens, targets, params, workspace, grads, accumulate=False, s
     rc = lib().gpt_backward(ctypes.byref(cfg), _ptr(tokens), _ptr(targets), _ptr(params),
                             _ptr(workspace), _ptr(grads), int(bool(accumulate)), stream)
     _check(rc, "gpt_backward")
+
+
+def raw_backward_ex(cfg, tokens, targets, params, workspace, grads, accumulate=0, grad_scale=1.0,
+                    events=None, stream=None):
+    """gpt_backward_ex; `events` is a sequence of cudaEvent_t handles (ints) or None."""
+    arr, n = None, 0
+    if events is not None:
+        n = len(events)
+        arr = (ctypes.c_void_p * n)(*[ctypes.c_void_p(int(e)) for e in events])
+    return lib().gpt_backward_ex(ctypes.byref(cfg), _ptr(tokens), _ptr(targets), _ptr(params),
+                                 _ptr(workspace), _ptr(grads), int(accumulate), float(grad_scale),
+                                 arr, n, stream)
+
+
+def backward_ex(cfg, tokens, targets, params, workspace, grads, accumulate=False, grad_scale=1.0,
+                events=None, stream=None):
+    _check(raw_backward_ex(cfg, tokens, targets, params, workspace, grads, int(bool(accumulate)),
+                           grad_scale, events, stream), "gpt_backward_ex")
 
 
 def train_step_host(cfg, host_tokens, host_targets, params, workspace, grads, host_loss,

@@ -498,12 +498,22 @@ int gpt_forward_loss(const gpt_config* c, const int32_t* tok, const int32_t* tgt
   return GPT_OK;
 }
 
-int gpt_backward(const gpt_config* c, const int32_t* tok, const int32_t* tgt,
-                 const void* params, void* workspace, void* grads, int accumulate,
-                 void* stream) {
+// The backward with a gradient scale and optional per-bucket "gradient
+// final" events (gpt_backward_ex in gpt.h).
+static int backward_impl(const gpt_config* c, const int32_t* tok, const int32_t* tgt,
+                         const void* params, void* workspace, void* grads, int accumulate,
+                         float grad_scale, void* const* events, int n_events, void* stream) {
   int rc = check_common(c, tok, tgt, params, workspace);
   if (rc) return rc;
   if (!grads || !aligned(grads, 256) || (accumulate != 0 && accumulate != 1)) return GPT_EINVAL;
+  if (!std::isfinite(grad_scale) || !(grad_scale > 0.f)) return GPT_EINVAL;
+  if (events && n_events != c->n_layer + 2) return GPT_EINVAL;
+  for (int i = 0; events && i < n_events; ++i)
+    if (!events[i]) return GPT_EINVAL;
+  auto mark = [&](int i) -> int {  // the gradients of bucket i are final on `stream`
+    return events ? int(cudaEventRecord(static_cast<cudaEvent_t>(events[i]), (cudaStream_t)stream))
+                  : 0;
+  };
   Step S(c, workspace, params, stream);
   const Layout& L = S.L;
   const int N = S.N, d = S.d, F = S.F, V = S.V, esz = S.esz;
@@ -526,7 +536,7 @@ int gpt_backward(const gpt_config* c, const int32_t* tok, const int32_t* tgt,
                        EPI_CE_BWD, ws + L.G, L.vpad, status);
   g.targets = tgt;
   g.lse = S.f(L.lse_z);
-  g.inv_n = 1.0f / float(N);
+  g.inv_n = grad_scale / float(N);
   g.n_valid = V;
   GPT_TRY(run_gemm(*c, g, st));
   // dhf = G Wlm ; dWlm = G^T hf
@@ -538,6 +548,7 @@ int gpt_backward(const gpt_config* c, const int32_t* tok, const int32_t* tgt,
               status);
   g.a_mn_major = true; g.b_mn_major = true; g.beta = accumulate;
   GPT_TRY(run_gemm(*c, g, st));
+  GPT_TRY(cuda_rc(cudaError_t(mark(0))));
   GPT_TRY(S.rms_bwd(ws + L.dh, ws + L.hf, S.f(L.rf), 0));
 
   const double attn_b = 8.0 * attn_pairs(*c) * c->head_dim;  // dV, dP, dQ, dK, causal half
@@ -585,13 +596,28 @@ int gpt_backward(const gpt_config* c, const int32_t* tok, const int32_t* tgt,
                 grad(GPT_T_WQKV, l), d, status);
     g.a_mn_major = true; g.b_mn_major = true; g.beta = accumulate;
     GPT_TRY(run_gemm(*c, with_splitk(g, L, ws), st));
+    GPT_TRY(cuda_rc(cudaError_t(mark(1 + l))));  // every weight gradient of layer l is final
     GPT_TRY(S.rms_bwd(ws + L.dh, Lb + L.lo.h1, reinterpret_cast<float*>(Lb + L.lo.r1), 1));
   }
   {
     TraceScope ts(GPT_K_SCATTER, 6, 0, S.nd() * 4 + double(V) * d * esz, st);
     GPT_TRY(launch_embed_scatter(*c, L, S.x, ws, grad(GPT_T_WTE, 0), accumulate, st));
   }
+  GPT_TRY(cuda_rc(cudaError_t(mark(c->n_layer + 1))));
   return GPT_OK;
+}
+
+int gpt_backward(const gpt_config* c, const int32_t* tok, const int32_t* tgt,
+                 const void* params, void* workspace, void* grads, int accumulate,
+                 void* stream) {
+  return backward_impl(c, tok, tgt, params, workspace, grads, accumulate, 1.0f, nullptr, 0, stream);
+}
+
+int gpt_backward_ex(const gpt_config* c, const int32_t* tok, const int32_t* tgt,
+                    const void* params, void* workspace, void* grads, int accumulate,
+                    float grad_scale, void* const* grad_ready_events, int n_events, void* stream) {
+  return backward_impl(c, tok, tgt, params, workspace, grads, accumulate, grad_scale,
+                       grad_ready_events, n_events, stream);
 }
 
 int gpt_train_step_host(const gpt_config* c, const int32_t* host_tokens,

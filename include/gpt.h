@@ -170,6 +170,26 @@ int gpt_backward(const gpt_config* cfg, const int32_t* tokens, const int32_t* ta
                  const void* params, void* workspace, void* grads, int accumulate,
                  void* stream);
 
+/* gpt_backward for data-parallel training ("ChatGPT'nizi 50 Dolara Nasil
+ * Egitirsiniz?", section "Dagitilmis Egitim": the gradient exchange starts
+ * while the backward still runs).
+ *   grad_scale: every gradient is multiplied by it (> 0, finite).  With W
+ *     replicas on equal batches, 1/W makes the sum of their gradients the
+ *     gradient of the mean loss over all W*batch*seq_len positions.
+ *   grad_ready_events: NULL, or n_events = n_layer + 2 CUDA events
+ *     (cudaEvent_t, created by the caller on the current device), recorded on
+ *     `stream` when a bucket of the gradient buffer is final: [0] lm_head,
+ *     [1 + l] the four block matrices of layer l (recorded for l = n_layer-1
+ *     down to 0, in that order), [n_layer + 1] wte.  A collective on another
+ *     stream that waits for event i may then reduce that bucket while the
+ *     backward goes on.
+ * Everything else as gpt_backward (which is grad_scale 1, no events).
+ * GPT_EINVAL for a bad scale, n_events != n_layer + 2 with events, or a NULL
+ * event; GPT_ECUDA if an event record fails. */
+int gpt_backward_ex(const gpt_config* cfg, const int32_t* tokens, const int32_t* targets,
+                    const void* params, void* workspace, void* grads, int accumulate,
+                    float grad_scale, void* const* grad_ready_events, int n_events, void* stream);
+
 /* One whole training step from HOST token/target arrays (pinned memory gives
  * asynchronous copies): copies tokens/targets into the workspace's staging
  * area, runs gpt_forward_loss and gpt_backward, and copies the loss back to
