@@ -231,7 +231,10 @@ def gemm_sites(records, w, steps):
 # DRAM bytes (read + write) of one launch of the dominant kernel's roofline
 # site, from an ncu capture of the current kernel build, keyed by (workload,
 # site, fp8); a site that has not been captured reports null.
-TRAFFIC_BYTES = {}
+TRAFFIC_BYTES = {
+    ("d24", 32768, 6144, 1536, False): 121_360_896 + 362_861_824,  # ncu: 484.2 MB per launch
+    ("d24", 32768, 6144, 1536, True): 60_106_752 + 351_310_080,    # e4m3 operands: 411.4 MB
+}
 
 
 def roofline(sites, w, gemm_tf, peak_tf, peaks):

@@ -57,7 +57,11 @@ def test_roofline_uses_the_site_and_the_dtype_peak():
     assert r["unit"] == "TFLOP/s" and r["bound"] == "tensor" and "traffic" in r
     f = bench.roofline(sites, w.replace(fp8=True), 1300.0, 1400.0, peaks)
     assert f["peak"] == 2800.0 and f["frac"] == pytest.approx(1200.0 / 2800.0, rel=1e-3)
-    assert f["traffic"] is None
+    # DRAM traffic from the ncu captures of the d24 launches, below the
+    # algorithmic bytes (no re-reads); other shapes have none
+    assert r["traffic"] == 484_222_720 and r["traffic"] <= r["algorithmic_bytes_per_launch"]
+    assert f["traffic"] == 411_416_832 and f["traffic"] <= f["algorithmic_bytes_per_launch"]
+    assert bench.roofline(sites, synth.workload("d12"), 1300.0, 1400.0, peaks)["traffic"] is None
 
 
 def test_workload_builder_applies_overrides():
