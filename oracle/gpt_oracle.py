@@ -59,6 +59,25 @@ embedding, lm_head and the whole backward stay as above.
   activations (dX = dY W and dW = dY^T X with the unquantized W and X), i.e.
   the quantizer is taken as the identity (straight-through).
 
+Block variants (section "1. GPT Modeli": the "Deger Gommeleri (ResFormer)"
+and "Verimlilik Puf Noktalari" listings).  The page prints each as a line or
+two; the widths, the layers they act on and the initial values are not
+printed.  Readings taken (every scale and gate is a parameter, so its initial
+value is the caller's):
+
+* value embeddings (``ve_every`` = k >= 1): layers l with l % k == k - 1 own a
+  table VE_l [vocab, n_kv_head*hd]; with h the block's normalised input (the
+  attention's input), gate = 3 sigmoid(h[:, :C] W_g^T), W_g [n_kv_head, C],
+  C = ``ve_gate_channels``, and v <- v + gate (per key/value head) * VE_l[tok];
+* per-layer residual scaling (``resid_lambdas``): on entering layer l,
+  x <- lam[l, 0] x + lam[l, 1] x0, with x0 the stream entering layer 0;
+* smear (``smear``), once, right after the embedding gather e = wte[tok]:
+  g_t = smear_lambda sigmoid(e_t[:24] . w_smear), x_t = e_t + g_t e_{t-1}
+  (e_{-1} = 0: the first position of a sequence mixes nothing);
+* backout (``backout``): x_b is the stream entering layer n_layer // 2 (after
+  its residual scaling); after the last layer x <- x - backout_lambda x_b,
+  then the final norm.
+
 Layout conventions shared with the library's documented ABI (not its code):
 W_qkv is [(n_head + 2 n_kv_head) hd, d] with the q rows first, then k, then v
 ([3d, d] without GQA); inside each block head h owns rows [h*hd, (h+1)*hd).
@@ -115,10 +134,22 @@ class OracleConfig:
     n_kv_head: int = 0   # 0: n_head (multi-head attention)
     window: int = 0      # 0: full causal window
     fp8: bool = False    # e4m3 operands in the block projections' forward
+    ve_every: int = 0    # value embeddings on layers l % ve_every == ve_every - 1; 0: none
+    ve_gate_channels: int = 32
+    resid_lambdas: bool = False
+    smear: bool = False
+    backout: bool = False
 
     @property
     def kv_heads(self) -> int:
         return self.n_kv_head or self.n_head
+
+    def has_ve(self, l: int) -> bool:
+        return self.ve_every > 0 and l % self.ve_every == self.ve_every - 1
+
+    @property
+    def backout_layer(self) -> int:
+        return self.n_layer // 2
 
 
 def from_workload(w) -> OracleConfig:
@@ -127,7 +158,17 @@ def from_workload(w) -> OracleConfig:
         d_ff=w.d_ff, vocab=w.vocab, seq_len=w.seq_len, batch=w.batch,
         norm_eps=w.norm_eps, rope_base=w.rope_base, qk_norm=w.qk_norm,
         n_kv_head=getattr(w, "n_kv_head", 0), window=getattr(w, "window", 0),
-        fp8=bool(getattr(w, "fp8", False)))
+        fp8=bool(getattr(w, "fp8", False)), ve_every=getattr(w, "ve_every", 0),
+        ve_gate_channels=getattr(w, "ve_gate_channels", 32),
+        resid_lambdas=bool(getattr(w, "resid_lambdas", False)),
+        smear=bool(getattr(w, "smear", False)), backout=bool(getattr(w, "backout", False)))
+
+
+def _sigmoid(z: np.ndarray) -> np.ndarray:
+    return 1.0 / (1.0 + np.exp(-z))
+
+
+SMEAR_CHANNELS = 24  # the smear gate reads x[:, :, :24] ("Verimlilik Puf Noktalari")
 
 
 # ---------------------------------------------------------------------------
@@ -365,15 +406,39 @@ def sequence_forward(cfg: OracleConfig, params: Dict[str, np.ndarray],
     cos, sin = rope_tables(T, hd, cfg.rope_base)
 
     x = params["wte"][tok].astype(np.float64)           # token embedding gather
+    smear = None
+    if cfg.smear:                                        # mix in the previous token's embedding
+        e = x
+        u = e[:, :SMEAR_CHANNELS] @ params["smear_gate"][0]
+        sg = _sigmoid(u)
+        prev = np.zeros_like(e)
+        prev[1:] = e[:-1]
+        x = e + (params["scalars"][0, 0] * sg)[:, None] * prev
+        smear = dict(e=e, sg=sg, prev=prev)
+    x0 = x
+    x_b = None
     layers = []
     for l in range(cfg.n_layer):
         wqkv, wo, wup, wdown = _layer_params(params, l)
-        c = {"x_in": x}
+        c = {}
+        if cfg.resid_lambdas:                            # per-layer residual scaling
+            c["x_prev"] = x
+            x = params["lambdas"][l, 0] * x + params["lambdas"][l, 1] * x0
+        if cfg.backout and l == cfg.backout_layer:
+            x_b = x
+        c["x_in"] = x
         h, r1 = rms_norm(x, eps)                         # pre-attention norm
         qkv = _linear(cfg, h, wqkv, wq(f"layers.{l}.wqkv"))  # F.linear, no bias
         q = qkv[:, :d].reshape(T, H, hd)
         k = qkv[:, d:d + dkv].reshape(T, Hkv, hd)
         v = qkv[:, d + dkv:].reshape(T, Hkv, hd)
+        if cfg.has_ve(l):                                # value embedding, gated per kv head
+            C = cfg.ve_gate_channels
+            gz = h[:, :C] @ params[f"ve_gate.{l}"].T     # [T, Hkv]
+            gate = 3.0 * _sigmoid(gz)
+            ve = params[f"ve.{l}"][tok].reshape(T, Hkv, hd)
+            v = v + gate[:, :, None] * ve
+            c.update(ve_gz=gz, ve_rows=ve)
         q = rope(q, cos, sin)
         k = rope(k, cos, sin)
         if cfg.qk_norm:
@@ -393,12 +458,14 @@ def sequence_forward(cfg: OracleConfig, params: Dict[str, np.ndarray],
                  lse=lse, x_mid=x_mid, h2=h2, r2=r2, u=u, a=a)
         layers.append(c)
 
+    if cfg.backout:                                      # take out the middle layers' residual
+        x = x - params["scalars"][0, 1] * x_b
     hf, rf = rms_norm(x, eps)                            # final norm
     z = hf @ params["lm_head"].T                         # untied lm_head
     loss_t, lse_z, probs = cross_entropy(z, tgt)
     return {"tok": tok, "tgt": tgt, "layers": layers, "x_out": x, "hf": hf,
             "rf": rf, "z": z, "probs": probs, "lse_z": lse_z, "token_loss": loss_t,
-            "cos": cos, "sin": sin}
+            "cos": cos, "sin": sin, "x0": x0, "x_b": x_b, "smear": smear}
 
 
 def sequence_backward(cfg: OracleConfig, params: Dict[str, np.ndarray], cache: dict,
@@ -415,6 +482,10 @@ def sequence_backward(cfg: OracleConfig, params: Dict[str, np.ndarray], cache: d
     grads["lm_head"] += g.T @ cache["hf"]
     dhf = g @ params["lm_head"]
     dx = rms_norm_backward(dhf, cache["hf"], cache["rf"])
+    dx_final = dx                                        # backout: x_out = x_L - beta x_b
+    if cfg.backout:
+        grads["scalars"][0, 1] -= np.sum(dx_final * cache["x_b"])
+    dx0 = np.zeros_like(dx)                              # residual scaling's x0 term
 
     for l in reversed(range(cfg.n_layer)):
         wqkv, wo, wup, wdown = _layer_params(params, l)
@@ -431,6 +502,16 @@ def sequence_backward(cfg: OracleConfig, params: Dict[str, np.ndarray], cache: d
         do = (dx @ wo).reshape(T, H, hd)
         _, p, _ = causal_attention(c["qn"], c["kn"], c["v"], cfg.window)
         dqn, dkn, dv = causal_attention_backward(do, c["qn"], c["kn"], c["v"], p)
+        dh_ve = None
+        if cfg.has_ve(l):                                # v = v_proj + gate * VE[tok]
+            C = cfg.ve_gate_channels
+            sg = _sigmoid(c["ve_gz"])
+            gate = 3.0 * sg
+            np.add.at(grads[f"ve.{l}"], tok, (gate[:, :, None] * dv).reshape(T, Hkv * hd))
+            dgz = np.sum(dv * c["ve_rows"], axis=2) * 3.0 * sg * (1.0 - sg)   # [T, Hkv]
+            grads[f"ve_gate.{l}"] += dgz.T @ c["h"][:, :C]
+            dh_ve = np.zeros((T, d))
+            dh_ve[:, :C] = dgz @ params[f"ve_gate.{l}"]
         if cfg.qk_norm:
             dq = rms_norm_backward(dqn, c["qn"], c["rq"])
             dk = rms_norm_backward(dkn, c["kn"], c["rk"])
@@ -442,7 +523,30 @@ def sequence_backward(cfg: OracleConfig, params: Dict[str, np.ndarray], cache: d
                               axis=1)
         grads[f"layers.{l}.wqkv"] += dqkv.T @ c["h"]
         dh = dqkv @ wqkv
+        if dh_ve is not None:
+            dh = dh + dh_ve
         dx = dx + rms_norm_backward(dh, c["h"], c["r1"])
+        if cfg.backout and l == cfg.backout_layer:       # x_b is this layer's input
+            dx = dx - params["scalars"][0, 1] * dx_final
+        if cfg.resid_lambdas:                            # x_in = a x_prev + b x0
+            a, b = params["lambdas"][l, 0], params["lambdas"][l, 1]
+            grads["lambdas"][l, 0] += np.sum(dx * c["x_prev"])
+            grads["lambdas"][l, 1] += np.sum(dx * cache["x0"])
+            dx0 = dx0 + b * dx
+            dx = a * dx
+
+    dx = dx + dx0                                        # x0 is the stream entering layer 0
+    if cfg.smear:                                        # x = e + g * prev(e), g = beta sigmoid(u)
+        sm = cache["smear"]
+        lam = params["scalars"][0, 0]
+        dg = np.sum(dx * sm["prev"], axis=1)             # [T]
+        grads["scalars"][0, 0] += np.sum(dg * sm["sg"])
+        du = dg * lam * sm["sg"] * (1.0 - sm["sg"])
+        grads["smear_gate"][0] += du @ sm["e"][:, :SMEAR_CHANNELS]
+        de = dx.copy()
+        de[:-1] += (lam * sm["sg"][1:])[:, None] * dx[1:]   # e_t feeds x_{t+1} through prev
+        de[:, :SMEAR_CHANNELS] += du[:, None] * params["smear_gate"][0][None, :]
+        dx = de
 
     np.add.at(grads["wte"], tok, dx)                     # embedding scatter-add
 

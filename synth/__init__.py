@@ -61,6 +61,11 @@ class Workload:
     n_kv_head: int = 0  # key/value heads (GQA); 0 = n_head
     window: int = 0     # sliding attention window in positions; 0 = full causal
     fp8: bool = False   # e4m3 operands in the forward block projections
+    ve_every: int = 0   # value embeddings on layers l % ve_every == ve_every - 1; 0 = none
+    ve_gate_channels: int = 32
+    resid_lambdas: bool = False  # per-layer residual scaling x = a x + b x0
+    smear: bool = False          # previous-token embedding mixing after the gather
+    backout: bool = False        # subtract the middle layer's residual before the final norm
 
     @property
     def n_tokens(self) -> int:
@@ -100,6 +105,25 @@ def param_shapes(w: Workload) -> Iterator[Tuple[str, Tuple[int, int]]]:
         yield f"layers.{l}.wup", (f, d)
         yield f"layers.{l}.wdown", (d, f)
     yield "lm_head", (v, d)
+    # block-variant parameters, after the base model's (their draws come last)
+    kv = (w.n_kv_head or w.n_head) * w.head_dim
+    if w.ve_every:
+        for l in range(w.n_layer):
+            if l % w.ve_every == w.ve_every - 1:
+                yield f"ve.{l}", (v, kv)
+                yield f"ve_gate.{l}", (w.n_kv_head or w.n_head, w.ve_gate_channels)
+    if w.resid_lambdas:
+        yield "lambdas", (w.n_layer, 2)          # [resid, x0] per layer
+    if w.smear:
+        yield "smear_gate", (1, 24)
+    if w.smear or w.backout:
+        yield "scalars", (1, 2)                  # [smear lambda, backout lambda]
+
+
+# Draws of the block-variant parameters: (mean, scale) of a normal law per
+# kind; their initial values are the caller's, these only make every term of
+# the variants visible in the tests' gradients.
+_VARIANT_DRAWS = {"ve": (0.0, 0.3), "ve_gate": (0.0, 0.5), "smear_gate": (0.0, 10.0)}
 
 
 # ---------------------------------------------------------------------------
@@ -175,6 +199,14 @@ def make_params(w: Workload, as_bits: bool = False) -> Dict[str, np.ndarray]:
         x = rng.standard_normal(shape, dtype=np.float32) * np.float32(0.02)
         if name.endswith(".wo") or name.endswith(".wdown"):
             x = x * np.float32(out_scale)
+        kind = name.split(".")[0]
+        if kind in _VARIANT_DRAWS:
+            mean, scale = _VARIANT_DRAWS[kind]
+            x = x * np.float32(scale / 0.02) + np.float32(mean)
+        elif name == "lambdas":   # resid near 1, x0 near 0
+            x = x * np.float32(5.0) + np.array([1.0, 0.0], dtype=np.float32)
+        elif name == "scalars":   # smear and backout lambdas near 0.5 and 0.3
+            x = x * np.float32(5.0) + np.array([0.5, 0.3], dtype=np.float32)
         if w.dtype == "bf16":
             bits = f64_to_bf16_bits(x)
             params[name] = bits if as_bits else bf16_bits_to_f64(bits)
