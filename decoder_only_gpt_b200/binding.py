@@ -21,6 +21,7 @@ GPT_OK, GPT_EINVAL, GPT_EUNSUPPORTED, GPT_ECUDA, GPT_EDATA, GPT_ETIMEOUT, GPT_EN
     0, -1, -2, -3, -4, -5, -6)
 GPT_BF16, GPT_F32 = 0, 1
 GPT_T_WTE, GPT_T_WQKV, GPT_T_WO, GPT_T_WUP, GPT_T_WDOWN, GPT_T_LM_HEAD = range(6)
+GPT_T_VE, GPT_T_VE_GATE, GPT_T_LAMBDAS, GPT_T_SMEAR_GATE, GPT_T_SCALARS = range(6, 11)
 GPT_W_STATUS, GPT_W_RESID, GPT_W_LSE, GPT_W_SORT_PERM, GPT_W_SORT_OFFS, GPT_W_ATTN_LSE = range(6)
 
 _TENSOR_IDS = {"wqkv": GPT_T_WQKV, "wo": GPT_T_WO, "wup": GPT_T_WUP, "wdown": GPT_T_WDOWN}
@@ -32,7 +33,8 @@ class GptConfig(ctypes.Structure):
         ("head_dim", ctypes.c_int32), ("d_ff", ctypes.c_int32), ("vocab", ctypes.c_int32),
         ("seq_len", ctypes.c_int32), ("batch", ctypes.c_int32), ("dtype", ctypes.c_int32),
         ("qk_norm", ctypes.c_int32), ("n_kv_head", ctypes.c_int32), ("attn_window", ctypes.c_int32),
-        ("fp8", ctypes.c_int32),
+        ("fp8", ctypes.c_int32), ("ve_every", ctypes.c_int32), ("ve_gate_channels", ctypes.c_int32),
+        ("resid_lambdas", ctypes.c_int32), ("smear", ctypes.c_int32), ("backout", ctypes.c_int32),
         ("rope_base", ctypes.c_float), ("norm_eps", ctypes.c_float),
         ("n_params", ctypes.c_int64), ("param_bytes", ctypes.c_uint64),
         ("workspace_bytes", ctypes.c_uint64),
@@ -120,10 +122,13 @@ def _check(rc: int, what: str) -> None:
 
 def make_config(n_layer, d_model, n_head, head_dim, d_ff, vocab, seq_len, batch,
                 dtype="bf16", qk_norm=True, rope_base=10000.0, norm_eps=1e-6,
-                n_kv_head=0, attn_window=0, fp8=False, check=True) -> GptConfig:
+                n_kv_head=0, attn_window=0, fp8=False, check=True, ve_every=0, ve_gate_channels=0,
+                resid_lambdas=False, smear=False, backout=False) -> GptConfig:
     c = GptConfig(n_layer, d_model, n_head, head_dim, d_ff, vocab, seq_len, batch,
                   GPT_BF16 if dtype == "bf16" else GPT_F32, int(bool(qk_norm)),
-                  n_kv_head, attn_window, int(bool(fp8)), rope_base, norm_eps, 0, 0, 0)
+                  n_kv_head, attn_window, int(bool(fp8)), int(ve_every), int(ve_gate_channels),
+                  int(bool(resid_lambdas)), int(bool(smear)), int(bool(backout)),
+                  rope_base, norm_eps, 0, 0, 0)
     rc = lib().gpt_config_init(ctypes.byref(c))
     if check:
         _check(rc, "gpt_config_init")
@@ -134,7 +139,11 @@ def config_from_workload(w) -> GptConfig:
     """Config for a ``synth.Workload``-like object (shape fields + dtype)."""
     return make_config(w.n_layer, w.d_model, w.n_head, w.head_dim, w.d_ff, w.vocab, w.seq_len,
                        w.batch, w.dtype, w.qk_norm, w.rope_base, w.norm_eps,
-                       getattr(w, "n_kv_head", 0), getattr(w, "window", 0), getattr(w, "fp8", False))
+                       getattr(w, "n_kv_head", 0), getattr(w, "window", 0), getattr(w, "fp8", False),
+                       ve_every=getattr(w, "ve_every", 0),
+                       ve_gate_channels=getattr(w, "ve_gate_channels", 0) if getattr(w, "ve_every", 0) else 0,
+                       resid_lambdas=getattr(w, "resid_lambdas", False), smear=getattr(w, "smear", False),
+                       backout=getattr(w, "backout", False))
 
 
 def config_from_depth(depth: int, seq_len: int, batch: int, vocab: int) -> GptConfig:
@@ -165,6 +174,16 @@ def tensor_slots(cfg: GptConfig):
         for short, tid in _TENSOR_IDS.items():
             yield f"layers.{l}.{short}", tid, l
     yield "lm_head", GPT_T_LM_HEAD, 0
+    for l in range(cfg.n_layer):
+        if cfg.ve_every > 0 and l % cfg.ve_every == cfg.ve_every - 1:
+            yield f"ve.{l}", GPT_T_VE, l
+            yield f"ve_gate.{l}", GPT_T_VE_GATE, l
+    if cfg.resid_lambdas:
+        yield "lambdas", GPT_T_LAMBDAS, 0
+    if cfg.smear:
+        yield "smear_gate", GPT_T_SMEAR_GATE, 0
+    if cfg.smear or cfg.backout:
+        yield "scalars", GPT_T_SCALARS, 0
 
 
 def elem_dtype(cfg: GptConfig):

@@ -8,6 +8,7 @@
 #include <cstdio>
 #include <algorithm>
 #include <cstring>
+#include <vector>
 
 #include "gpt_internal.h"
 #include "trace.h"
@@ -31,6 +32,7 @@ struct Bump {
 
 int64_t param_elems_aligned(int64_t n) { return (n + 127) / 128 * 128; }
 
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 int cuda_rc(cudaError_t e) { return e == cudaSuccess ? GPT_OK : GPT_ECUDA; }
@@ -42,6 +44,43 @@ int cuda_rc(cudaError_t e) { return e == cudaSuccess ? GPT_OK : GPT_ECUDA; }
   } while (0)
 
 }  // namespace
+
+// Elements of the base model's parameters (wte, the layers, lm_head), aligned.
+int64_t base_param_elems(const gpt_config& c) {
+  const int64_t d = c.d_model, F = c.d_ff, V = c.vocab, Q = qkv_cols(c);
+  return 2 * param_elems_aligned(V * d) +
+         int64_t(c.n_layer) * (param_elems_aligned(Q * d) + param_elems_aligned(d * d) +
+                               2 * param_elems_aligned(F * d));
+}
+
+// Walk the block-variant tensors in their buffer order (after lm_head): for
+// each value-embedding layer its table and gate, then the residual scales,
+// the smear gate, the scalars.  Returns the aligned element count of all of
+// them; finds (tensor, layer)'s offset from the variants' start (at, rows,
+// cols; at stays -1 when absent) and adds the unaligned count to *count.
+int64_t variant_walk(const gpt_config& c, int tensor, int layer, int64_t* at, int64_t* rows,
+                     int64_t* cols, int64_t* count) {
+  int64_t off = 0;
+  auto take = [&](int t, int l, int64_t r, int64_t cc) {
+    if (t == tensor && (l == layer || (t != GPT_T_VE && t != GPT_T_VE_GATE))) {
+      *at = off;
+      *rows = r;
+      *cols = cc;
+    }
+    if (count) *count += r * cc;
+    off += param_elems_aligned(r * cc);
+  };
+  const int64_t kvd = int64_t(c.n_kv_head ? c.n_kv_head : c.n_head) * c.head_dim;
+  for (int l = 0; l < c.n_layer; ++l)
+    if (has_value_embed(c, l)) {
+      take(GPT_T_VE, l, c.vocab, kvd);
+      take(GPT_T_VE_GATE, l, c.n_kv_head ? c.n_kv_head : c.n_head, c.ve_gate_channels);
+    }
+  if (c.resid_lambdas) take(GPT_T_LAMBDAS, 0, c.n_layer, 2);
+  if (c.smear) take(GPT_T_SMEAR_GATE, 0, 1, kSmearChannels);
+  if (c.smear || c.backout) take(GPT_T_SCALARS, 0, 1, 2);
+  return off;
+}
 
 bool make_layout(const gpt_config& c, Layout* L) {
   const int64_t N = int64_t(c.batch) * c.seq_len;
@@ -131,6 +170,24 @@ bool make_layout(const gpt_config& c, Layout* L) {
   } else {
     L->w8 = L->w8_deq = L->w8_amax = L->a8 = L->a8_deq = 0;
   }
+  // block variants
+  {
+    const int64_t nd4 = N * d * 4, Hkv = c.n_kv_head ? c.n_kv_head : c.n_head;
+    bool any_ve = false;
+    for (int l = 0; l < c.n_layer; ++l) any_ve |= has_value_embed(c, l);
+    L->emb = c.smear ? b.take(nd4) : 0;
+    L->sm_sg = c.smear ? b.take(N * 4) : 0;
+    L->sm_dg = c.smear ? b.take(N * 4) : 0;
+    L->sm_du = c.smear ? b.take(N * 4) : 0;
+    L->x0 = c.resid_lambdas ? b.take(nd4) : 0;
+    L->xprev = c.resid_lambdas ? b.take(nd4 * c.n_layer) : 0;
+    L->dx0 = c.resid_lambdas ? b.take(nd4) : 0;
+    L->xb = c.backout ? b.take(nd4) : 0;
+    L->dxf = c.backout ? b.take(nd4) : 0;
+    L->ve_rows = any_ve ? b.take(N * Hkv * c.head_dim * 4) : 0;
+    L->ve_dgz = any_ve ? b.take(N * Hkv * 4) : 0;
+    L->vred = has_variants(c) ? b.take(int64_t(variant_red_floats()) * 4) : 0;
+  }
   // Muon's sum-of-squares partials and reciprocal norm
   if (c.dtype == GPT_BF16) {
     L->opt_x0 += L->layer_base;
@@ -192,14 +249,20 @@ int gpt_config_init(gpt_config* c) {
   } else {
     return GPT_EINVAL;
   }
+  if (c->ve_every < 0 || (c->resid_lambdas != 0 && c->resid_lambdas != 1) ||
+      (c->smear != 0 && c->smear != 1) || (c->backout != 0 && c->backout != 1))
+    return GPT_EINVAL;
+  if (c->ve_every > 0 && c->ve_gate_channels == 0) c->ve_gate_channels = std::min(32, c->d_model);
+  if (c->ve_every > 0 && (c->ve_gate_channels < 1 || c->ve_gate_channels > c->d_model)) return GPT_EINVAL;
+  if (c->smear && c->d_model < kSmearChannels) return GPT_EUNSUPPORTED;
+  if (c->backout && c->n_layer < 1) return GPT_EINVAL;
   const int64_t N = int64_t(c->batch) * c->seq_len;
   if (N > (int64_t(1) << 31) / 4 || int64_t(c->vocab) > (int64_t(1) << 24)) return GPT_EUNSUPPORTED;
   const int64_t d = c->d_model, F = c->d_ff, V = c->vocab, Q = qkv_cols(*c);
   int64_t n = 2 * V * d + int64_t(c->n_layer) * (Q * d + d * d + 2 * F * d);
-  c->n_params = n;
-  int64_t elems = 2 * param_elems_aligned(V * d) +
-                  int64_t(c->n_layer) * (param_elems_aligned(Q * d) + param_elems_aligned(d * d) +
-                                         2 * param_elems_aligned(F * d));
+  int64_t vn = 0;
+  const int64_t elems = base_param_elems(*c) + variant_walk(*c, -1, -1, nullptr, nullptr, nullptr, &vn);
+  c->n_params = n + vn;
   c->param_bytes = uint64_t(elems) * (c->dtype == GPT_BF16 ? 2 : 4);
   Layout L;
   make_layout(*c, &L);
@@ -228,6 +291,17 @@ int gpt_config_from_depth(gpt_config* c, int depth, int seq_len, int batch, int 
 int gpt_param_offset(const gpt_config* c, int tensor, int layer, int64_t* off, int64_t* rows,
                      int64_t* cols) {
   if (!c || !off || !rows || !cols) return GPT_EINVAL;
+  if (tensor >= GPT_T_VE && tensor <= GPT_T_SCALARS) {
+    *off = -1;
+    const int64_t o = base_param_elems(*c) + 0;
+    int64_t r = 0, cc = 0, at = -1;
+    variant_walk(*c, tensor, layer, &at, &r, &cc, nullptr);
+    if (at < 0) return GPT_EINVAL;  // not present in this config (or no such layer)
+    *off = o + at;
+    *rows = r;
+    *cols = cc;
+    return GPT_OK;
+  }
   const int64_t d = c->d_model, F = c->d_ff, V = c->vocab, Q = qkv_cols(*c);
   const bool per_layer = tensor >= GPT_T_WQKV && tensor <= GPT_T_WDOWN;
   if (tensor < GPT_T_WTE || tensor > GPT_T_LM_HEAD) return GPT_EINVAL;
@@ -436,11 +510,37 @@ int gpt_forward_loss(const gpt_config* c, const int32_t* tok, const int32_t* tgt
     TraceScope ts(GPT_K_NORM, 1, 0, S.nd() * (esz + 4 + esz) + N * 8.0, st);
     GPT_TRY(launch_embed_norm(*c, tok, S.param(GPT_T_WTE, 0), S.x, h0, r0, S.status, st));
   }
+  const uint64_t nd4 = uint64_t(N) * d * 4;
+  if (c->smear) {  // x = e + s sigmoid(e[:24] . w) e_prev, from a copy of the gathered e
+    TraceScope ts(GPT_K_OTHER, 2, 0, S.nd() * 16.0, st);
+    GPT_TRY(cuda_rc(cudaMemcpyAsync(ws + L.emb, S.x, nd4, cudaMemcpyDeviceToDevice, st)));
+    GPT_TRY(launch_smear_fwd(*c, S.f(L.emb), S.param(GPT_T_SMEAR_GATE, 0), S.param(GPT_T_SCALARS, 0), S.x,
+                             S.f(L.sm_sg), st));
+    if (c->n_layer == 0) GPT_TRY(S.rms_fwd(ws + L.hf, S.f(L.rf)));
+  }
+  if (c->resid_lambdas) {  // x0: the stream entering layer 0
+    TraceScope ts(GPT_K_OTHER, 1, 0, S.nd() * 8.0, st);
+    GPT_TRY(cuda_rc(cudaMemcpyAsync(ws + L.x0, S.x, nd4, cudaMemcpyDeviceToDevice, st)));
+  }
   const double attn_f = 4.0 * attn_pairs(*c) * c->head_dim;  // QK^T and PV, visible pairs
   const int Qc = int(qkv_cols(*c));
   if (c->fp8 && c->n_layer > 0) GPT_TRY(S.quant_weights());
   for (int l = 0; l < c->n_layer; ++l) {
     char* Lb = S.layer(l);
+    {  // block variants at the layer's entry: residual scaling, the backout point
+      bool renorm = l == 0 && c->smear;
+      if (c->resid_lambdas) {
+        TraceScope ts(GPT_K_OTHER, 1, 0, S.nd() * 16.0, st);
+        const char* lam = static_cast<const char*>(S.param(GPT_T_LAMBDAS, 0)) + int64_t(l) * 2 * esz;
+        GPT_TRY(launch_lambda_mix(*c, S.x, S.f(L.x0), S.f(L.xprev + uint64_t(l) * nd4), lam, st));
+        renorm = true;
+      }
+      if (c->backout && l == backout_layer(*c)) {
+        TraceScope ts(GPT_K_OTHER, 1, 0, S.nd() * 8.0, st);
+        GPT_TRY(cuda_rc(cudaMemcpyAsync(ws + L.xb, S.x, nd4, cudaMemcpyDeviceToDevice, st)));
+      }
+      if (renorm) GPT_TRY(S.rms_fwd(Lb + L.lo.h1, reinterpret_cast<float*>(Lb + L.lo.r1)));
+    }
     if (c->dtype == GPT_BF16) {
       // QKV projection with RoPE, QK-norm and the head-major scatter in its epilogue
       GemmArgs g = gemm_kk(Lb + L.lo.h1, d, S.param(GPT_T_WQKV, l), d, N, Qc, d, EPI_QKV,
@@ -461,6 +561,11 @@ int gpt_forward_loss(const gpt_config* c, const int32_t* tok, const int32_t* tgt
                               Lb + L.lo.v, reinterpret_cast<float*>(Lb + L.lo.rq),
                               reinterpret_cast<float*>(Lb + L.lo.rk), st));
     }
+    if (has_value_embed(*c, l)) {  // v += 3 sigmoid(h[:, :C] Wg^T) VE[tok], per kv head
+      TraceScope ts(GPT_K_OTHER, 1, 0, double(N) * c->n_kv_head * c->head_dim * esz * 3, st);
+      GPT_TRY(launch_ve_fwd(*c, Lb + L.lo.h1, S.param(GPT_T_VE_GATE, l), S.param(GPT_T_VE, l), tok,
+                            Lb + L.lo.v, st));
+    }
     {
       TraceScope ts(GPT_K_ATTN_FWD, 1, attn_f, S.nd() * esz * 4, st);
       GPT_TRY(launch_attn_fwd(*c, Lb + L.lo.q, Lb + L.lo.k, Lb + L.lo.v, Lb + L.lo.o,
@@ -474,6 +579,12 @@ int gpt_forward_loss(const gpt_config* c, const int32_t* tok, const int32_t* tgt
     GPT_TRY(S.projection(gemm_kk(Lb + L.lo.a, F, S.param(GPT_T_WDOWN, l), F, N, d, F,
                                  EPI_RESID_F32, S.x, d, S.status), GPT_T_WDOWN, l));
     const bool last = l + 1 == c->n_layer;
+    if (last && c->backout) {  // x -= backout_lambda x_b before the final norm
+      TraceScope ts(GPT_K_OTHER, 1, 0, S.nd() * 12.0, st);
+      GPT_TRY(launch_axpy(*c, S.x, S.f(L.xb), static_cast<const char*>(S.param(GPT_T_SCALARS, 0)) + esz,
+                          -1.f, st));
+    }
+    if (!last && c->resid_lambdas) continue;  // the next layer's entry scales x, then normalises it
     void* hn = last ? (void*)(ws + L.hf) : (void*)(S.layer(l + 1) + L.lo.h1);
     float* rn = reinterpret_cast<float*>(last ? ws + L.rf : S.layer(l + 1) + L.lo.r1);
     GPT_TRY(S.rms_fwd(hn, rn));
@@ -550,6 +661,14 @@ static int backward_impl(const gpt_config* c, const int32_t* tok, const int32_t*
   GPT_TRY(run_gemm(*c, g, st));
   GPT_TRY(cuda_rc(cudaError_t(mark(0))));
   GPT_TRY(S.rms_bwd(ws + L.dh, ws + L.hf, S.f(L.rf), 0));
+  const uint64_t nd4 = uint64_t(N) * d * 4;
+  char* gvar_scalars = (c->smear || c->backout) ? static_cast<char*>(grad(GPT_T_SCALARS, 0)) : nullptr;
+  if (c->backout) {  // x_out = x_L - beta x_b: d beta = -sum(dx_out x_b); keep dx_out
+    TraceScope ts(GPT_K_OTHER, 3, 0, S.nd() * 16.0, st);
+    GPT_TRY(cuda_rc(cudaMemcpyAsync(ws + L.dxf, S.x, nd4, cudaMemcpyDeviceToDevice, st)));
+    GPT_TRY(launch_dot(*c, S.f(L.dxf), S.f(L.xb), -1.f, S.f(L.vred), gvar_scalars + esz, accumulate, st));
+  }
+  if (c->resid_lambdas) GPT_TRY(cuda_rc(cudaMemsetAsync(ws + L.dx0, 0, nd4, st)));
 
   const double attn_b = 8.0 * attn_pairs(*c) * c->head_dim;  // dV, dP, dQ, dK, causal half
   for (int l = c->n_layer - 1; l >= 0; --l) {
@@ -587,21 +706,57 @@ static int backward_impl(const gpt_config* c, const int32_t* tok, const int32_t*
                               reinterpret_cast<float*>(Lb + L.lo.rk), S.cos_t, S.sin_t,
                               S.f(L.Dattn), ws + L.dqkv, S.status, st));
     }
+    const bool ve = has_value_embed(*c, l);
+    if (ve) {  // the value embedding's table and gate gradients from dv
+      TraceScope ts(GPT_K_OTHER, 2, 0, double(N) * c->n_kv_head * c->head_dim * (esz * 2 + 4), st);
+      GPT_TRY(launch_ve_bwd(*c, ws + L.dqkv, Lb + L.lo.h1, S.param(GPT_T_VE_GATE, l), S.param(GPT_T_VE, l),
+                            tok, S.f(L.ve_rows), S.f(L.ve_dgz), grad(GPT_T_VE_GATE, l), accumulate, st));
+      gpt_config cv = *c;
+      cv.d_model = c->n_kv_head * c->head_dim;
+      TraceScope ts2(GPT_K_SCATTER, 5, 0, double(N) * cv.d_model * 4 + double(V) * cv.d_model * esz, st);
+      GPT_TRY(launch_embed_scatter(cv, L, S.f(L.ve_rows), ws, grad(GPT_T_VE, l), accumulate, st));
+    }
     const int Qc = int(qkv_cols(*c));
     g = gemm_kk(ws + L.dqkv, Qc, S.param(GPT_T_WQKV, l), d, N, d, Qc, EPI_STORE, ws + L.dh,
                 d, status);
     g.b_mn_major = true;
     GPT_TRY(run_gemm(*c, g, st));
+    if (ve) {  // the gate's input h[:, :C]
+      TraceScope ts(GPT_K_OTHER, 1, 0, double(N) * c->ve_gate_channels * esz * 2, st);
+      GPT_TRY(launch_ve_dh(*c, ws + L.dh, S.f(L.ve_dgz), S.param(GPT_T_VE_GATE, l), st));
+    }
     g = gemm_kk(ws + L.dqkv, Qc, Lb + L.lo.h1, d, Qc, d, N, EPI_STORE,
                 grad(GPT_T_WQKV, l), d, status);
     g.a_mn_major = true; g.b_mn_major = true; g.beta = accumulate;
     GPT_TRY(run_gemm(*c, with_splitk(g, L, ws), st));
     GPT_TRY(cuda_rc(cudaError_t(mark(1 + l))));  // every weight gradient of layer l is final
     GPT_TRY(S.rms_bwd(ws + L.dh, Lb + L.lo.h1, reinterpret_cast<float*>(Lb + L.lo.r1), 1));
+    const bool bo = c->backout && l == backout_layer(*c);
+    if (bo || c->resid_lambdas) {  // the layer's entry: backout point, residual scaling
+      TraceScope ts(GPT_K_OTHER, c->resid_lambdas ? 2 : 1, 0, S.nd() * (c->resid_lambdas ? 26.0 : 14.0), st);
+      const char* lam =
+          c->resid_lambdas ? static_cast<const char*>(S.param(GPT_T_LAMBDAS, 0)) + int64_t(l) * 2 * esz : nullptr;
+      char* dlam = c->resid_lambdas ? static_cast<char*>(grad(GPT_T_LAMBDAS, 0)) + int64_t(l) * 2 * esz : nullptr;
+      GPT_TRY(launch_resid_bwd(*c, S.x, ws + L.dxs, bo ? S.f(L.dxf) : nullptr,
+                               bo ? S.param(GPT_T_SCALARS, 0) : nullptr,
+                               c->resid_lambdas ? S.f(L.xprev + uint64_t(l) * nd4) : nullptr,
+                               c->resid_lambdas ? S.f(L.x0) : nullptr, c->resid_lambdas ? S.f(L.dx0) : nullptr,
+                               lam, S.f(L.vred), dlam, accumulate, st));
+    }
+  }
+  if (c->resid_lambdas) {  // x0 is the stream entering layer 0
+    TraceScope ts(GPT_K_OTHER, 1, 0, S.nd() * 12.0, st);
+    GPT_TRY(launch_axpy(*c, S.x, S.f(L.dx0), nullptr, 1.f, st));
+  }
+  if (c->smear) {  // back through x = e + s sigmoid(e[:24] . w) e_prev, into L.emb
+    TraceScope ts(GPT_K_OTHER, 4, 0, S.nd() * 16.0, st);
+    GPT_TRY(launch_smear_bwd(*c, S.x, S.f(L.emb), S.f(L.sm_sg), S.f(L.sm_dg), S.f(L.sm_du),
+                             S.param(GPT_T_SMEAR_GATE, 0), S.param(GPT_T_SCALARS, 0),
+                             grad(GPT_T_SMEAR_GATE, 0), gvar_scalars, accumulate, st));
   }
   {
     TraceScope ts(GPT_K_SCATTER, 6, 0, S.nd() * 4 + double(V) * d * esz, st);
-    GPT_TRY(launch_embed_scatter(*c, L, S.x, ws, grad(GPT_T_WTE, 0), accumulate, st));
+    GPT_TRY(launch_embed_scatter(*c, L, c->smear ? S.f(L.emb) : S.x, ws, grad(GPT_T_WTE, 0), accumulate, st));
   }
   GPT_TRY(cuda_rc(cudaError_t(mark(c->n_layer + 1))));
   return GPT_OK;
@@ -756,10 +911,22 @@ int gpt_optim_step(const gpt_config* c, const gpt_optim* o, void* params, const 
   const double t = double(o->step);
   const float bc1 = float(1.0 - std::pow(double(o->adam_beta1), t));
   const float bc2 = float(1.0 - std::pow(double(o->adam_beta2), t));
-  for (int tensor : {GPT_T_WTE, GPT_T_LM_HEAD}) {
+  // AdamW: the embedding, lm_head and every block-variant parameter (value
+  // embeddings and their gates, scales), each over its aligned span (the
+  // padding's gradient and state are zero and stay zero)
+  std::vector<std::pair<int, int>> adam = {{GPT_T_WTE, 0}, {GPT_T_LM_HEAD, 0}};
+  for (int l = 0; l < c->n_layer; ++l)
+    if (has_value_embed(*c, l)) {
+      adam.push_back({GPT_T_VE, l});
+      adam.push_back({GPT_T_VE_GATE, l});
+    }
+  if (c->resid_lambdas) adam.push_back({GPT_T_LAMBDAS, 0});
+  if (c->smear) adam.push_back({GPT_T_SMEAR_GATE, 0});
+  if (c->smear || c->backout) adam.push_back({GPT_T_SCALARS, 0});
+  for (auto [tensor, layer] : adam) {
     int64_t off, r, cc;
-    gpt_param_offset(c, tensor, 0, &off, &r, &cc);
-    const int64_t n = r * cc;
+    gpt_param_offset(c, tensor, layer, &off, &r, &cc);
+    const int64_t n = param_elems_aligned(r * cc);
     TraceScope ts(GPT_K_OTHER, 1, 0, double(n) * 30.0, st);
     GPT_TRY(launch_adamw(P + off, G + off, W + off, M + off, Vv + off, n, o->adam_lr, o->adam_beta1,
                          o->adam_beta2, o->adam_eps, o->adam_weight_decay, bc1, bc2, st));

@@ -22,6 +22,19 @@ inline int window_span(const gpt_config& c) {
   return c.attn_window > 0 && c.attn_window < c.seq_len ? c.attn_window : c.seq_len;
 }
 
+// Block variants.  Value embeddings on layers l % ve_every == ve_every - 1.
+inline bool has_value_embed(const gpt_config& c, int l) {
+  return c.ve_every > 0 && l % c.ve_every == c.ve_every - 1;
+}
+inline int backout_layer(const gpt_config& c) { return c.n_layer / 2; }
+constexpr int kSmearChannels = 24;  // the smear gate reads x[:, :, :24]
+inline bool has_variants(const gpt_config& c) {
+  return c.ve_every > 0 || c.resid_lambdas || c.smear || c.backout;
+}
+int64_t base_param_elems(const gpt_config& c);
+int64_t variant_walk(const gpt_config& c, int tensor, int layer, int64_t* at, int64_t* rows,
+                     int64_t* cols, int64_t* count);
+
 // Kernel ids recorded in gpt_device_status::where.
 enum KernelId : int32_t {
   K_EMBED = 1,
@@ -131,6 +144,11 @@ struct Layout {
   // and amax bits [4 kinds][n_layer], one activation's codes [N, max(d, F)]
   // and its per-row factors [N]
   uint64_t w8, w8_deq, w8_amax, a8, a8_deq;
+  // block variants: smear (embedding, gate values, step-1 results), residual
+  // scaling (x0, every layer's pre-scaling stream, the x0 gradient), backout
+  // (x_b, the final stream gradient), value embeddings (table-gradient rows,
+  // gate gradients), reduction partials
+  uint64_t emb, sm_sg, sm_dg, sm_du, x0, xprev, dx0, xb, dxf, ve_rows, ve_dgz, vred;
   uint64_t total;
 };
 
@@ -187,6 +205,27 @@ int launch_sort_tokens(const gpt_config& c, const Layout& L, const int32_t* tok,
                        void* stream);
 int launch_embed_scatter(const gpt_config& c, const Layout& L, const float* dx0, char* ws,
                          void* dwte, int accumulate, void* stream);
+// ---- block variants (csrc/variants.cu) ----
+int launch_smear_fwd(const gpt_config& c, const float* e, const void* w, const void* scalars, float* x,
+                     float* sg, void* stream);
+int launch_lambda_mix(const gpt_config& c, float* x, const float* x0, float* xprev, const void* lam,
+                      void* stream);
+int launch_axpy(const gpt_config& c, float* y, const float* x, const void* s, float mul, void* stream);
+int launch_ve_fwd(const gpt_config& c, const void* h, const void* wg, const void* ve, const int32_t* tok,
+                  void* v, void* stream);
+int launch_ve_bwd(const gpt_config& c, const void* dqkv, const void* h, const void* wg, const void* ve,
+                  const int32_t* tok, float* rows, float* dgz, void* d_wg, int accumulate, void* stream);
+int launch_ve_dh(const gpt_config& c, void* dh, const float* dgz, const void* wg, void* stream);
+int launch_resid_bwd(const gpt_config& c, float* dx, void* dxs, const float* dxf, const void* scalars,
+                     const float* xprev, const float* x0, float* dx0, const void* lam, float* partial,
+                     void* d_lam, int accumulate, void* stream);
+int launch_dot(const gpt_config& c, const float* x, const float* y, float scale, float* partial,
+               void* out, int accumulate, void* stream);
+int launch_smear_bwd(const gpt_config& c, const float* dx, float* e, const float* sg, float* dg,
+                     float* du, const void* w, const void* scalars, void* d_w, void* d_scalars,
+                     int accumulate, void* stream);
+int variant_red_floats();
+
 int launch_gemm(const gpt_config& c, const GemmArgs& g, void* stream);
 // Number of kernels launch_gemm enqueues for these arguments (2 with a split-K reduce).
 int gemm_kernel_count(const gpt_config& c, const GemmArgs& g);

@@ -71,6 +71,14 @@ extern "C" {
 #define GPT_T_WUP 3     /* [d_ff, d_model]           MLP up                   */
 #define GPT_T_WDOWN 4   /* [d_model, d_ff]           MLP down                 */
 #define GPT_T_LM_HEAD 5 /* [vocab, d_model]          untied output head       */
+/* Block-variant parameters (present only when their config field is on; they
+ * follow lm_head in the flat buffer, in this order): */
+#define GPT_T_VE 6         /* [vocab, n_kv_head*head_dim] value embedding of layer l
+                              (layers l with l % ve_every == ve_every - 1)       */
+#define GPT_T_VE_GATE 7    /* [n_kv_head, ve_gate_channels] its gate             */
+#define GPT_T_LAMBDAS 8    /* [n_layer, 2]: (resid, x0) scale of each layer      */
+#define GPT_T_SMEAR_GATE 9 /* [1, 24]: smear gate on the embedding's 24 channels */
+#define GPT_T_SCALARS 10   /* [1, 2]: (smear scale, backout scale)               */
 
 /* ---- workspace regions (for gpt_workspace_region, diagnostics/tests) ---- */
 #define GPT_W_STATUS 0     /* gpt_device_status struct                                 */
@@ -113,6 +121,22 @@ typedef struct gpt_config {
                           per row, weights per tensor, by powers of two -- and
                           the backward stays bf16 (straight-through); bf16
                           configs only                                        */
+  /* Block variants ("ChatGPT'nizi 50 Dolara Nasil Egitirsiniz?", section
+   * "1. GPT Modeli": the value-embedding and efficiency-trick listings); each
+   * one's parameters are inputs like every other weight (GPT_T_VE ..
+   * GPT_T_SCALARS), so their initial values are the caller's: */
+  int32_t ve_every;    /* k >= 1: layers l with l % k == k - 1 add a gated value
+                          embedding to v, v += 3 sigmoid(h[:, :C] Wg^T) VE[token]
+                          per key/value head (h: the block's normalised input);
+                          0 = none                                             */
+  int32_t ve_gate_channels; /* C, 1 .. d_model; 0 = 32 (capped at d_model)     */
+  int32_t resid_lambdas;    /* 1: x = lam[l,0] x + lam[l,1] x0 on entering layer l
+                               (x0: the stream entering layer 0)               */
+  int32_t smear;       /* 1: after the gather, x_t = e_t + s sigmoid(e_t[:24] . w)
+                          e_{t-1} (s = scalars[0]; nothing at a sequence start);
+                          d_model >= 24                                        */
+  int32_t backout;     /* 1: x = x - scalars[1] x_b before the final norm, x_b the
+                          stream entering layer n_layer / 2                    */
   float rope_base;  /* 10000 by default                                  */
   float norm_eps;   /* 1e-6 by default                                   */
   /* derived by gpt_config_init */

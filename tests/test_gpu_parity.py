@@ -92,6 +92,19 @@ CASES = {
                                  seq_len=100, batch=3, fp8=True)),
     "gqa_window_fp8": ("story", dict(n_layer=2, d_model=256, n_head=4, head_dim=64, n_kv_head=2,
                                      window=100, d_ff=512, vocab=2048, seq_len=256, batch=2, fp8=True)),
+    # block variants (value embeddings with their gate, residual scaling,
+    # smear, backout): the fp32 path, the bf16 path with GQA (two key/value
+    # heads, a 16-channel gate), and ragged shapes with value embeddings on
+    # every other layer and a window
+    "tiny_variants": ("tiny", dict(ve_every=1, resid_lambdas=True, smear=True, backout=True,
+                                   seq_len=37, batch=3, vocab=100)),
+    "story_variants": ("story", dict(n_layer=3, n_kv_head=2, ve_every=1, ve_gate_channels=16,
+                                     resid_lambdas=True, smear=True, backout=True, batch=4)),
+    "ragged_variants": ("story", dict(n_layer=4, d_model=128, n_head=2, head_dim=64, d_ff=320,
+                                      vocab=1000, seq_len=100, batch=3, ve_every=2,
+                                      resid_lambdas=True, smear=True, backout=True, window=60)),
+    "hd128_ve_only": ("d4", dict(n_layer=2, d_model=256, n_head=2, head_dim=128, d_ff=512,
+                                 vocab=2048, seq_len=192, batch=2, ve_every=1)),
 }
 
 
@@ -176,7 +189,7 @@ def test_step_matches_oracle(B, R, case):
     check_against_oracle(st, w, oracle_result(case))
 
 
-@pytest.mark.parametrize("case", ["story", "tiny"])
+@pytest.mark.parametrize("case", ["story", "tiny", "story_variants"])
 def test_bitwise_deterministic(B, R, case):
     w = workload_of(case)
     a, _ = run_gpu(B, R, w)
@@ -229,12 +242,13 @@ def test_untouched_embedding_rows_are_zero(B, R):
     assert miss.size > 0 and np.all(g[miss] == 0.0)
 
 
-def test_causality_on_gpu(B, R):
-    w = workload_of("story")
+@pytest.mark.parametrize("case", ["story", "story_variants"])
+def test_causality_on_gpu(B, R, case):
+    w = workload_of(case)
     tok, tgt = synth.make_tokens(w)
     a, _ = run_gpu(B, R, w)
     tok2 = tok.copy()
-    b, t = 5, 100
+    b, t = min(5, w.batch - 1), 100
     tok2[b, t + 1:] = (tok2[b, t + 1:] + 7) % w.vocab
     c, _ = run_gpu(B, R, w, tokens=tok2)
     la = a.token_loss.cpu().numpy().reshape(w.batch, w.seq_len)
