@@ -84,6 +84,8 @@ def bench_workload(args):
         w = w.replace(window=args.window)
     if args.fp8:
         w = w.replace(fp8=True)
+    if getattr(args, "variants", False):
+        w = w.replace(ve_every=2, resid_lambdas=True, smear=True, backout=True)
     return w
 
 
@@ -95,6 +97,11 @@ def workload_desc(w):
         extra += f", attention window {w.window}"
     if w.fp8:
         extra += ", e4m3 forward block projections"
+    if w.ve_every or w.resid_lambdas or w.smear or w.backout:
+        parts = ([f"value embeddings every {w.ve_every} layers"] if w.ve_every else []) + \
+                (["residual scaling"] if w.resid_lambdas else []) + (["smear"] if w.smear else []) + \
+                (["backout"] if w.backout else [])
+        extra += ", " + ", ".join(parts)
     return (f"{w.name}: {w.n_layer} layers, d_model {w.d_model}, {w.n_head}x{w.head_dim} heads, "
             f"d_ff {w.d_ff}, vocab {w.vocab}, seq {w.seq_len}, batch {w.batch}{extra}")
 
@@ -504,7 +511,8 @@ def run_ours(args, rank, world, local_rank):
     # the other depth the metric names, after the headline one (default runs)
     second = None
     if not args.no_second and args.workload == WORKLOAD and not (args.layers or args.batch or args.kv_heads
-                                                                  or args.window or args.fp8):
+                                                                  or args.window or args.fp8
+                                                                  or args.variants):
         second = measure(synth.workload(SECOND_WORKLOAD), args, rank, world, dev, barrier, e2e=False)
 
     ms, e2e_ms = main_m["ms"], main_m["e2e_ms"]
@@ -651,6 +659,9 @@ def main():
                     help="sliding attention window in positions (a model variant)")
     ap.add_argument("--fp8", action="store_true",
                     help="e4m3 operands in the forward block projections (a variant)")
+    ap.add_argument("--variants", action="store_true",
+                    help="block variants: value embeddings on every other layer, residual "
+                         "scaling, smear and backout (a model variant)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")

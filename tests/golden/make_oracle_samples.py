@@ -29,6 +29,9 @@ SAMPLES_PER_TENSOR = 1024
 VARIANTS = {
     "d24_kv4_w1024": ("d24", dict(n_kv_head=4, window=1024)),
     "d24_fp8": ("d24", dict(fp8=True)),
+    # the block variants at full size: value embeddings on every other layer,
+    # residual scaling, smear and backout
+    "d24_variants": ("d24", dict(ve_every=2, resid_lambdas=True, smear=True, backout=True)),
 }
 
 

@@ -357,13 +357,15 @@ def _sample_workload(name):
     return mod.workload_of(name)
 
 
-@pytest.mark.parametrize("name", ["d12", "d24", "d24_kv4_w1024", "d24_fp8"])
+@pytest.mark.parametrize("name", ["d12", "d24", "d24_kv4_w1024", "d24_fp8", "d24_variants"])
 def test_full_size_against_oracle_samples(B, R, name):
     """Full-size workloads in the benchmark's launch configuration: the loss, every
     per-position loss, and gradient entries at the oracle's seeded coordinates
     (d24_kv4_w1024: the d24 model with 4 key/value heads and a 1024-position
     window, as ``bench.py --kv-heads 4 --window 1024`` runs it; d24_fp8: e4m3
-    forward projections, as ``bench.py --fp8`` runs it, with the e4m3 bars)."""
+    forward projections, as ``bench.py --fp8`` runs it, with the e4m3 bars;
+    d24_variants: value embeddings on every other layer, residual scaling,
+    smear and backout, as ``bench.py --variants`` runs it)."""
     s = _samples(name)
     w = _sample_workload(name)
     st, code = run_gpu(B, R, w)
