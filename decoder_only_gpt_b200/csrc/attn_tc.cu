@@ -27,7 +27,6 @@
 namespace gpt {
 
 namespace {
-constexpr int BQ = 128, BKV = 128, kInner = 64;
 constexpr int kThreads = 352;   // warp 0 TMA, warps 1 and 10 MMA, warps 2..9 compute
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -68,15 +67,8 @@ __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
-__device__ __forceinline__ void fence_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 // barrier among the 256 compute threads (warps 2..9)
 __device__ __forceinline__ void compute_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
-
-// byte offset of 16-byte unit `u` (8 bf16) of row r of a [rows x 64] bf16 tile
-// stored with the 128-byte swizzle (the layout TMA writes and the MMA reads)
-__device__ __forceinline__ uint32_t sw_off(int r, int u) { return r * 128 + ((u ^ (r & 7)) << 4); }
 
 struct Roles {
   int warp, lane, quarter, half, r;
@@ -706,23 +698,14 @@ __global__ void attn_rowdot_kernel(const __nv_bfloat16* __restrict__ dO,
   }
 }
 
-constexpr int kRingKV = 3;  // slots of the Q/dO ring of the dK/dV kernel
-constexpr int kRingQ = 3;   // slots of the K/V ring of the dQ kernel
-constexpr int kRingMax = kRingKV > kRingQ ? kRingKV : kRingQ;
-
-struct BwdBars {
-  uint64_t fixed_full;
-  uint64_t ring_full[kRingMax];
-  uint64_t ring_empty[kRingMax];
-  uint64_t s_full[2];
-  uint64_t dp_full[2];
-  uint64_t ds_ready[2];
-  uint64_t acc_full;
-  uint64_t epi_full;
-  uint64_t done, done2;
-  uint32_t tmem_base;
-  int abort;
-};
+// slots of the dK/dV kernel's Q and dO rings (a Q tile is read by S^T_j and,
+// after the threads have formed dS^T_j, by dK_j)
+constexpr int kDkvRingQ = 3, kDkvRingDO = 2;
+constexpr int kDkvThreads = 384;  // as kThreads, plus warp 11 staging lse and D
+// slots of the dQ kernel's K and V rings: a K tile is read by S_j early in its
+// step and by the dQ product at the end of it, so it stays resident about two
+// steps and needs a third slot to be prefetched in time; V only feeds dP_j
+constexpr int kDqRingK = 3, kDqRingV = 2;
 
 // One row's gradient w.r.t. its normalised, rotated q or k (TMEM, fp32, HD
 // columns at `taddr`, times `scale`) back through RMSNorm (y: the normalised
@@ -736,6 +719,18 @@ struct BwdBars {
 // path).
 __device__ __forceinline__ uint32_t tile_unit(int r, int unit) {  // 16-byte unit of row r
   return uint32_t(unit >> 3) * (128 * 128) + r * 128 + (((unit & 7) ^ (r & 7)) << 4);
+}
+// The RoPE table rows pos0 .. pos0 + 127 ([T, HD/2] fp32 each) as two tiles of
+// 128 * HD * 2 bytes (the size of a bf16 [128 x HD] ring slot), loaded onto `bar`
+template <int HD>
+__device__ __forceinline__ void load_rope_tiles(uint8_t* cos_dst, uint8_t* sin_dst, const CUtensorMap* map_cos,
+                                                const CUtensorMap* map_sin, uint64_t* bar, int pos0) {
+  tc::mbar_arrive_expect_tx(bar, 2u * 128 * HD * 2);
+#pragma unroll
+  for (int c = 0; c < HD / 64; ++c) {
+    tc::tma_load_2d(cos_dst + c * (128 * 128), map_cos, bar, c * 32, pos0);
+    tc::tma_load_2d(sin_dst + c * (128 * 128), map_sin, bar, c * 32, pos0);
+  }
 }
 template <int HD>
 __device__ __forceinline__ void norm_rope_bwd_half(uint32_t taddr, int half, int r, float scale,
@@ -803,55 +798,105 @@ __device__ __forceinline__ void norm_rope_bwd_half(uint32_t taddr, int half, int
   }
 }
 
-// The epilogue's inputs for 128 rows, loaded by TMA onto `bar`: the y rows
-// (bh*T + row0 ..) of a head-major [B*H*T, HD] tensor (unless y_dst is null)
-// and the cos / sin table rows (pos0 ..) of [T, HD/2] fp32.
-template <int HD>
-__device__ __forceinline__ void load_epilogue_tiles(uint8_t* y_dst, uint8_t* cos_dst, uint8_t* sin_dst,
-                                                    const CUtensorMap* map_y, const CUtensorMap* map_cos,
-                                                    const CUtensorMap* map_sin, uint64_t* bar,
-                                                    int y_row0, int pos0) {
-  constexpr int NCH = HD / 64;
-  tc::mbar_arrive_expect_tx(bar, (y_dst ? 3u : 2u) * 128 * HD * 2);
+
+}  // namespace
+
+namespace {
+// dS = P (dP - D) for 32 keys k0 .. k0 + 31 of one query row, with P =
+// 2^(s * scale_log2 - lse2) from the S columns `us` and dP from `up`, as 16
+// packed bf16 pairs.  MASK: P = 0 outside the row's visible keys [k_lo, k_hi).
+template <bool MASK>
+__device__ __forceinline__ void ds_row32(const uint32_t (&us)[32], const uint32_t (&up)[32], uint32_t* pk,
+                                         uint64_t sc2, uint64_t nl2, uint64_t nd2, int k0, int k_lo, int k_hi) {
 #pragma unroll
-  for (int c = 0; c < NCH; ++c) {
-    if (y_dst) tc::tma_load_2d(y_dst + c * (128 * 128), map_y, bar, c * 64, y_row0);
-    tc::tma_load_2d(cos_dst + c * (128 * 128), map_cos, bar, c * 32, pos0);
-    tc::tma_load_2d(sin_dst + c * (128 * 128), map_sin, bar, c * 32, pos0);
+  for (int e = 0; e < 16; ++e) {
+    const int i = 2 * e;
+    const float2 x = unf2(fma2(f2(__uint_as_float(us[i]), __uint_as_float(us[i + 1])), sc2, nl2));
+    float p0 = ex2(x.x), p1 = ex2(x.y);
+    if (MASK) {
+      if (k0 + i < k_lo || k0 + i >= k_hi) p0 = 0.f;
+      if (k0 + i + 1 < k_lo || k0 + i + 1 >= k_hi) p1 = 0.f;
+    }
+    const float2 r =
+        unf2(mul2(f2(p0, p1), add2(f2(__uint_as_float(up[i]), __uint_as_float(up[i + 1])), nd2)));
+    pk[e] = pack2(r.x, r.y);
+  }
+}
+// P^T for 64 queries q0 .. q0 + 63 of one key row: p = 2^(s * scale_log2 -
+// lse2_q) from the S^T columns us0 | us1 and the staged lse2 (`l2`), kept in
+// fp32 and as 32 packed bf16 pairs.  MASK: P = 0 outside the key's visible
+// queries [q_lo, q_hi).
+template <bool MASK>
+__device__ __forceinline__ void p_col64(const uint32_t (&us0)[32], const uint32_t (&us1)[32], const float* l2s,
+                                        float (&p)[64], uint32_t (&pk)[32], float scale_log2, int q0, int q_lo,
+                                        int q_hi) {
+#pragma unroll
+  for (int g = 0; g < 16; ++g) {  // 4 queries per group
+    const float4 l4 = *reinterpret_cast<const float4*>(l2s + 4 * g);
+    const float l2[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+    for (int e = 0; e < 4; e += 2) {
+      const int i = 4 * g + e;
+      const uint32_t a = i < 32 ? us0[i] : us1[i - 32], c = i < 32 ? us0[i + 1] : us1[i - 31];
+      const float2 x = unf2(fma2(f2(__uint_as_float(a), __uint_as_float(c)), f2(scale_log2, scale_log2),
+                                 f2(-l2[e], -l2[e + 1])));
+      float p0 = ex2(x.x), p1 = ex2(x.y);
+      if (MASK) {
+        if (q0 + i < q_lo || q0 + i >= q_hi) p0 = 0.f;
+        if (q0 + i + 1 < q_lo || q0 + i + 1 >= q_hi) p1 = 0.f;
+      }
+      p[i] = p0;
+      p[i + 1] = p1;
+      pk[i / 2] = pack2(p0, p1);
+    }
   }
 }
 
 template <int HD>
 struct DqSmem {
-  static constexpr uint32_t SMALL = kInner * HD * 2;
-  static constexpr uint32_t EPI = 128 * HD * 2;  // the Q or dO tile; also a cos / sin tile
-  static constexpr uint32_t Q_OFF = 0, DO_OFF = EPI;
-  static constexpr uint32_t K_OFF = 2 * EPI;
-  static constexpr uint32_t V_OFF = K_OFF + kRingQ * SMALL;
-  static constexpr uint32_t Y_OFF = Q_OFF;  // the Q tile is the y of the norm backward
-  static constexpr uint32_t COS_OFF = V_OFF + kRingQ * SMALL, SIN_OFF = COS_OFF + EPI;
-  static constexpr uint32_t RED_OFF = SIN_OFF + EPI;
-  static constexpr uint32_t BAR_OFF = RED_OFF + 2 * 128 * 4;
+  static constexpr uint32_t TILE = 128 * HD * 2;  // a 128-row Q, dO, K or V tile
+  static constexpr uint32_t Q_OFF = 0, DO_OFF = TILE;
+  static constexpr uint32_t K_OFF = 2 * TILE;                   // K ring
+  static constexpr uint32_t V_OFF = K_OFF + kDqRingK * TILE;    // V ring
+  static constexpr uint32_t Y_OFF = Q_OFF;   // the Q tile is the y of the norm backward
+  static constexpr uint32_t RED_OFF = K_OFF;  // epilogue only, once no product reads K
+  // the RoPE tiles of the epilogue, loaded into the V ring once the last dP is done
+  static constexpr uint32_t COS_OFF = V_OFF, SIN_OFF = V_OFF + TILE;
+  static constexpr uint32_t BAR_OFF = V_OFF + kDqRingV * TILE;
   static constexpr uint32_t BYTES = BAR_OFF + 256 + 1024;
-  static_assert(K_OFF % 1024 == 0 && V_OFF % 1024 == 0 && Y_OFF % 1024 == 0 && EPI % 1024 == 0, "");
-  static_assert(BYTES <= 232448, "");
+  static_assert(TILE % 1024 == 0 && BYTES <= 232448, "");
 };
-
+struct DqBars {
+  uint64_t fixed_full;
+  uint64_t k_full[kDqRingK], k_empty[kDqRingK], v_full[kDqRingV], v_empty[kDqRingV];
+  uint64_t s_full[2], ds_ready[2];
+  uint64_t dp_full, dp_free;
+  uint64_t acc_full, epi_full, done, done2;
+  uint32_t tmem_base;
+  int abort;
+};
 }  // namespace
 
-// dQ for 128 queries of one (batch, head), looping over 64-key tiles.  Warp 1
-// issues S_j = Q K_j^T and dQ += dS_{j-1} K_{j-1}; warp 10 issues dP_j = dO V_j^T.
-// Compute thread (row, half) handles keys [32*half, 32*half + 32) of each tile
-// and writes its bf16 dS over its own S columns: the TMEM A operand of the dQ
-// product, which warp 1 issues before it next overwrites those columns.  TMEM:
-// S/dP pairs at columns 0 and 128 (64 + 64 each), dQ at 256.  The Q tile in
-// shared memory doubles as the y of the norm backward.
+// dQ for 128 queries of one (batch, head), looping over 128-key tiles (all
+// products M = 128, N = 128: a single issuing warp keeps up with each).  Warp
+// 1 issues S_j = Q K_j^T into one of two TMEM S buffers, then dQ += dS_{j-1}
+// K_{j-1}; warp 10 issues dP_j = dO V_j^T into the one dP buffer as soon as
+// the compute threads have loaded dP_{j-1}.  So S_{j+1} and dP_{j+1} run on
+// the tensor core while the threads turn step j into dS.  Compute thread
+// (row, half) handles keys [64*half, 64*half + 64) of each tile, in two
+// 32-key chunks, and writes bf16 dS into the first 32 of its own 64 S columns:
+// the TMEM A operand of the dQ product (its 16-key step k starts at column
+// 64*(k/4) + 8*(k%4)), which warp 1 issues before it next overwrites them.
+// TMEM: S at columns 0 and 128, dP at 256, dQ at 384.  K and V have separate
+// rings (a K tile is also the dQ product's B operand, so it has three slots);
+// the Q tile in shared memory doubles as the y of the norm backward, and the
+// RoPE tables of its 128 positions are loaded into the V ring after the last dP.
 template <int HD>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_dq_tc_kernel(const __grid_constant__ CUtensorMap map_q128,
                       const __grid_constant__ CUtensorMap map_do128,
-                      const __grid_constant__ CUtensorMap map_k64,
-                      const __grid_constant__ CUtensorMap map_v64,
+                      const __grid_constant__ CUtensorMap map_k128,
+                      const __grid_constant__ CUtensorMap map_v128,
                       const __grid_constant__ CUtensorMap map_cos,
                       const __grid_constant__ CUtensorMap map_sin,
                       const float* __restrict__ lse,
@@ -859,10 +904,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                       __nv_bfloat16* __restrict__ dqkv, int64_t ldq, int H, int Hkv, int T,
                       int W, float scale, float scale_log2, int qk_norm, int32_t* status) {
   using S = DqSmem<HD>;
+  constexpr int NCH = HD / 64;
+  constexpr uint32_t CH = 128 * 128;  // bytes of one 64-column chunk of a 128-row tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  BwdBars* bars = reinterpret_cast<BwdBars*>(smem + S::BAR_OFF);
+  DqBars* bars = reinterpret_cast<DqBars*>(smem + S::BAR_OFF);
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int n_qt = (T + 127) / 128;
   int bh, rank;
@@ -870,74 +917,95 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int qt = n_qt - 1 - rank;
   const int b = bh / H, h = bh % H;
   const int q0 = qt * 128;
-  const int s_lo = max(0, q0 - W + 1) / kInner;  // first key step with a visible key
-  const int n_steps = (min(q0 + 128, T) + kInner - 1) / kInner - s_lo;
+  const int s_lo = max(0, q0 - W + 1) / 128;  // first key tile with a visible key
+  const int n_steps = qt - s_lo + 1;
   const int kv_row_base = (b * Hkv + h / (H / Hkv)) * T;
-  constexpr int NCH = HD / 64;
 
   ATTN_PROLOGUE(bars, {
     tc::mbar_init(&bars->fixed_full, 1);
-    tc::mbar_init(&bars->epi_full, 1);
-    for (int s = 0; s < kRingQ; ++s) {
-      tc::mbar_init(&bars->ring_full[s], 1);
-      tc::mbar_init(&bars->ring_empty[s], 2);  // after S and dQ (warp 1) and dP (warp 10)
+    for (int s = 0; s < kDqRingK; ++s) {
+      tc::mbar_init(&bars->k_full[s], 1);
+      tc::mbar_init(&bars->k_empty[s], 1);
+    }
+    for (int s = 0; s < kDqRingV; ++s) {
+      tc::mbar_init(&bars->v_full[s], 1);
+      tc::mbar_init(&bars->v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&bars->s_full[s], 1);
-      tc::mbar_init(&bars->dp_full[s], 1);
       tc::mbar_init(&bars->ds_ready[s], 256);
     }
+    tc::mbar_init(&bars->dp_full, 1);
+    tc::mbar_init(&bars->dp_free, 256);
     tc::mbar_init(&bars->acc_full, 1);
+    tc::mbar_init(&bars->epi_full, 1);
     tc::mbar_init(&bars->done, 1);
     tc::mbar_init(&bars->done2, 1);
   })
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort = &bars->abort;
-  const uint32_t t_dq = tmem + 256;
+  const uint32_t t_dp = tmem + 256, t_dq = tmem + 384;
 
   if (warp == 0) {
-    if (lane == 0) {
+    // lane 0: Q, dO, then the K ring; lane 1: the V ring
+    if (lane < 2) {
+      const bool is_k = lane == 0;
+      uint64_t* full = is_k ? bars->k_full : bars->v_full;
+      uint64_t* empty = is_k ? bars->k_empty : bars->v_empty;
+      const CUtensorMap* map = is_k ? &map_k128 : &map_v128;
+      uint8_t* base = smem + (is_k ? S::K_OFF : S::V_OFF);
+      const int ring = is_k ? kDqRingK : kDqRingV;
       uint32_t issued = 0, last_par = 0;
-      tc::mbar_arrive_expect_tx(&bars->fixed_full, 2 * S::EPI);
+      if (is_k) {
+        tc::mbar_arrive_expect_tx(&bars->fixed_full, 2 * S::TILE);
 #pragma unroll
-      for (int c = 0; c < NCH; ++c) {
-        tc::tma_load_2d(smem + S::Q_OFF + c * (128 * 128), &map_q128, &bars->fixed_full, c * 64, bh * T + q0);
-        tc::tma_load_2d(smem + S::DO_OFF + c * (128 * 128), &map_do128, &bars->fixed_full,
-                        h * HD + c * 64, b * T + q0);
+        for (int c = 0; c < NCH; ++c) {
+          tc::tma_load_2d(smem + S::Q_OFF + c * CH, &map_q128, &bars->fixed_full, c * 64, bh * T + q0);
+          tc::tma_load_2d(smem + S::DO_OFF + c * CH, &map_do128, &bars->fixed_full, h * HD + c * 64,
+                          b * T + q0);
+        }
       }
       for (int j = 0; j < n_steps; ++j) {
-        const int st = j % kRingQ;
-        const uint32_t ph = (j / kRingQ) & 1;
-        if (!tc::mbar_wait_bounded(&bars->ring_empty[st], ph ^ 1, abort, kWaitNs)) {
+        const int st = j % ring;
+        const uint32_t ph = (j / ring) & 1;
+        if (!tc::mbar_wait_bounded(&empty[st], ph ^ 1, abort, kWaitNs)) {
           record_status(status, GPT_ETIMEOUT, K_ATTN, 20);
           *abort = 1;
           break;
         }
-        tc::mbar_arrive_expect_tx(&bars->ring_full[st], 2 * S::SMALL);
+        tc::mbar_arrive_expect_tx(&full[st], S::TILE);
 #pragma unroll
-        for (int c = 0; c < NCH; ++c) {
-          tc::tma_load_2d(smem + S::K_OFF + st * S::SMALL + c * (kInner * 128), &map_k64,
-                          &bars->ring_full[st], c * 64, kv_row_base + (s_lo + j) * kInner);
-          tc::tma_load_2d(smem + S::V_OFF + st * S::SMALL + c * (kInner * 128), &map_v64,
-                          &bars->ring_full[st], c * 64, kv_row_base + (s_lo + j) * kInner);
-        }
-        if (j == 0)
-          load_epilogue_tiles<HD>(nullptr, smem + S::COS_OFF, smem + S::SIN_OFF, nullptr, &map_cos,
-                                  &map_sin, &bars->epi_full, 0, q0);
+        for (int c = 0; c < NCH; ++c)
+          tc::tma_load_2d(base + st * S::TILE + c * CH, map, &full[st], c * 64,
+                          kv_row_base + (s_lo + j) * 128);
         issued |= 1u << st;
         last_par = (last_par & ~(1u << st)) | (ph << st);
       }
+      // the V ring is free once every dP is done: the epilogue's RoPE tiles go there
+      bool epi = false;
+      if (!is_k && !*abort) {
+        bool freed = true;
+        for (int s = 0; s < ring; ++s)
+          if (issued >> s & 1) freed = freed && tc::mbar_wait_bounded(&empty[s], (last_par >> s) & 1, abort, kWaitNs);
+        if (freed) {
+          load_rope_tiles<HD>(smem + S::COS_OFF, smem + S::SIN_OFF, &map_cos, &map_sin, &bars->epi_full, q0);
+          epi = true;
+        } else {
+          record_status(status, GPT_ETIMEOUT, K_ATTN, 24);
+          *abort = 1;
+        }
+      }
       if (*abort) {
-        tc::mbar_wait_bounded(&bars->fixed_full, 0, nullptr, kWaitNs);
-        if (issued) tc::mbar_wait_bounded(&bars->epi_full, 0, nullptr, kWaitNs);
-        for (int s = 0; s < kRingQ; ++s)
-          if (issued >> s & 1) tc::mbar_wait_bounded(&bars->ring_full[s], (last_par >> s) & 1, nullptr, kWaitNs);
+        if (is_k) tc::mbar_wait_bounded(&bars->fixed_full, 0, nullptr, kWaitNs);
+        if (epi) tc::mbar_wait_bounded(&bars->epi_full, 0, nullptr, kWaitNs);
+        for (int s = 0; s < ring; ++s)
+          if (issued >> s & 1) tc::mbar_wait_bounded(&full[s], (last_par >> s) & 1, nullptr, kWaitNs);
       }
     }
   } else if (warp == 1) {
     // S_j = Q K_j^T, then dQ += dS_{j-1} K_{j-1}.  S_j overwrites the dS_{j-2}
-    // that this warp's own dQ MMAs read (issued earlier: in order).
-    constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, kInner, false, false);
+    // that this warp's own dQ product read (issued earlier: in order).
+    constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, 128, false, false);
     constexpr uint32_t idesc_dq = tc::idesc_bf16_f32(128, HD, false, true);
     const uint64_t qd = tc::smem_desc_sw128(tc::smem_u32(smem + S::Q_OFF), 16);
     bool ok = tc::mbar_wait_warp(&bars->fixed_full, 0, abort, kWaitNs);
@@ -946,25 +1014,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!tc::mbar_wait_warp(&bars->ds_ready[j & 1], (j >> 1) & 1, abort, kWaitNs)) return false;
       tc::tc_fence_after();
       const uint32_t ds_t = tmem + (j & 1) * 128;
-      const uint64_t kb = tc::smem_desc_sw128(tc::smem_u32(smem + S::K_OFF + (j % kRingQ) * S::SMALL),
-                                              kInner * 128);
+      const uint64_t kb = tc::smem_desc_sw128(tc::smem_u32(smem + S::K_OFF + (j % kDqRingK) * S::TILE), CH);
 #pragma unroll
-      for (int k = 0; k < kInner / 16; ++k)
-        tc::mma_bf16_ts_elect(t_dq, ds_t + 32 * (k >> 1) + 8 * (k & 1), tc::desc_advance(kb, k * 2048),
+      for (int k = 0; k < 128 / 16; ++k)
+        tc::mma_bf16_ts_elect(t_dq, ds_t + 64 * (k >> 2) + 8 * (k & 3), tc::desc_advance(kb, k * 2048),
                               idesc_dq, (j | k) != 0);
-      tc::mma_commit_elect(&bars->ring_empty[j % kRingQ]);
+      tc::mma_commit_elect(&bars->k_empty[j % kDqRingK]);
       return true;
     };
     for (int j = 0; ok && j < n_steps; ++j) {
-      const int st = j % kRingQ;
-      if (!tc::mbar_wait_warp(&bars->ring_full[st], (j / kRingQ) & 1, abort, kWaitNs)) { ok = false; break; }
+      const int st = j % kDqRingK;
+      if (!tc::mbar_wait_warp(&bars->k_full[st], (j / kDqRingK) & 1, abort, kWaitNs)) { ok = false; break; }
       tc::tc_fence_after();
-      const uint64_t kd = tc::smem_desc_sw128(tc::smem_u32(smem + S::K_OFF + st * S::SMALL), 16);
-      const uint32_t pair = tmem + (j & 1) * 128;
+      const uint64_t kd = tc::smem_desc_sw128(tc::smem_u32(smem + S::K_OFF + st * S::TILE), 16);
 #pragma unroll
-      for (int k = 0; k < HD / 16; ++k)
-        tc::mma_bf16_ss_elect(pair, tc::desc_advance(qd, (k >> 2) * (128 * 128) + (k & 3) * 32),
-                              tc::desc_advance(kd, (k >> 2) * (kInner * 128) + (k & 3) * 32), idesc_s, k != 0);
+      for (int k = 0; k < HD / 16; ++k) {
+        const uint32_t off = (k >> 2) * CH + (k & 3) * 32;
+        tc::mma_bf16_ss_elect(tmem + (j & 1) * 128, tc::desc_advance(qd, off), tc::desc_advance(kd, off),
+                              idesc_s, k != 0);
+      }
       issued_any = true;
       tc::mma_commit_elect(&bars->s_full[j & 1]);
       if (j >= 1 && !issue_dq(j - 1)) { ok = false; break; }
@@ -980,26 +1048,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_wait_warp(&bars->done, 0, nullptr, kWaitNs);
     }
   } else if (warp == 10) {
-    // dP_j = dO V_j^T into the dP half of the pair, once the compute threads
-    // are done with dP_{j-2}
-    constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, kInner, false, false);
+    // dP_j = dO V_j^T into the dP buffer, once the compute threads have loaded dP_{j-1}
+    constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, 128, false, false);
     const uint64_t dod = tc::smem_desc_sw128(tc::smem_u32(smem + S::DO_OFF), 16);
     bool ok = tc::mbar_wait_warp(&bars->fixed_full, 0, abort, kWaitNs);
     bool issued_any = false;
     for (int j = 0; ok && j < n_steps; ++j) {
-      const int st = j % kRingQ;
-      if (j >= 2 && !tc::mbar_wait_warp(&bars->ds_ready[j & 1], ((j - 2) >> 1) & 1, abort, kWaitNs)) { ok = false; break; }
-      if (!tc::mbar_wait_warp(&bars->ring_full[st], (j / kRingQ) & 1, abort, kWaitNs)) { ok = false; break; }
+      const int st = j % kDqRingV;
+      if (j >= 1 && !tc::mbar_wait_warp(&bars->dp_free, (j - 1) & 1, abort, kWaitNs)) { ok = false; break; }
+      if (!tc::mbar_wait_warp(&bars->v_full[st], (j / kDqRingV) & 1, abort, kWaitNs)) { ok = false; break; }
       tc::tc_fence_after();
-      const uint64_t vd = tc::smem_desc_sw128(tc::smem_u32(smem + S::V_OFF + st * S::SMALL), 16);
-      const uint32_t pair = tmem + (j & 1) * 128;
+      const uint64_t vd = tc::smem_desc_sw128(tc::smem_u32(smem + S::V_OFF + st * S::TILE), 16);
 #pragma unroll
-      for (int k = 0; k < HD / 16; ++k)
-        tc::mma_bf16_ss_elect(pair + kInner, tc::desc_advance(dod, (k >> 2) * (128 * 128) + (k & 3) * 32),
-                              tc::desc_advance(vd, (k >> 2) * (kInner * 128) + (k & 3) * 32), idesc_s, k != 0);
+      for (int k = 0; k < HD / 16; ++k) {
+        const uint32_t off = (k >> 2) * CH + (k & 3) * 32;
+        tc::mma_bf16_ss_elect(t_dp, tc::desc_advance(dod, off), tc::desc_advance(vd, off), idesc_s, k != 0);
+      }
       issued_any = true;
-      tc::mma_commit_elect(&bars->dp_full[j & 1]);
-      tc::mma_commit_elect(&bars->ring_empty[st]);
+      tc::mma_commit_elect(&bars->dp_full);
+      tc::mma_commit_elect(&bars->v_empty[st]);
     }
     if (!ok) {
       if (lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 23);
@@ -1014,39 +1081,46 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = q0 + R.r;
     const bool qv = q < T;
     const int tq = qv ? q : 0;
-    const int lo_key = q - W + 1;
+    // the query's visible keys [k_lo, k_hi): none for a row past T
+    const int k_lo = q - W + 1, k_hi = qv ? q + 1 : k_lo;
     const float lse2 = qv ? lse[int64_t(bh) * T + q] * kLog2e : 0.f;
     const float Dq = qv ? D[int64_t(bh) * T + q] : 0.f;
     bool ok = true;
     for (int j = 0; j < n_steps; ++j) {
       const int sb = j & 1;
       if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->s_full[sb], (j >> 1) & 1, abort, kWaitNs));
-      if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->dp_full[sb], (j >> 1) & 1, abort, kWaitNs));
+      if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->dp_full, j & 1, abort, kWaitNs));
+      // dP first, so that dP_{j+1} may start as early as possible; S in two
+      // 32-column chunks (fewer live registers)
+      uint32_t up0[32], up1[32], us[32], pk[32];
+      const uint32_t ts = tmem + sb * 128 + R.lane_off + R.half * 64;
+      const uint32_t tp = t_dp + R.lane_off + R.half * 64;
       if (ok) {
         tc::tc_fence_after();
-        const int k0 = (s_lo + j) * kInner + R.half * 32;
-        const uint32_t ts = tmem + sb * 128 + R.lane_off + R.half * 32;
-        uint32_t us[32], up[32];
+        tc::tmem_ld_32x32b_x32(tp, up0);
+        tc::tmem_ld_32x32b_x32(tp + 32, up1);
         tc::tmem_ld_32x32b_x32(ts, us);
-        tc::tmem_ld_32x32b_x32(ts + kInner, up);
         tc::tmem_wait_ld();
-        const bool need_mask = !qv || k0 + 32 > q || k0 + 32 > T || k0 < lo_key;
-        uint32_t pk[16];
+        tc::tc_fence_before();
+      }
+      tc::mbar_arrive(&bars->dp_free);  // dP_{j+1} may overwrite the dP columns
+      if (ok) {
+        const int kb = (s_lo + j) * 128 + R.half * 64;
+        const bool need_mask = kb < k_lo || kb + 64 > k_hi;
         const uint64_t sc2 = f2(scale_log2, scale_log2), nl2 = f2(-lse2, -lse2), nd2 = f2(-Dq, -Dq);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int i = 2 * e;
-          const float2 x = unf2(fma2(f2(__uint_as_float(us[i]), __uint_as_float(us[i + 1])), sc2, nl2));
-          float p0 = ex2(x.x), p1 = ex2(x.y);
-          if (need_mask) {
-            if (k0 + i > q || k0 + i >= T || !qv || k0 + i < lo_key) p0 = 0.f;
-            if (k0 + i + 1 > q || k0 + i + 1 >= T || !qv || k0 + i + 1 < lo_key) p1 = 0.f;
+        for (int c = 0; c < 2; ++c) {
+          if (c == 1) {
+            tc::tmem_ld_32x32b_x32(ts + 32, us);
+            tc::tmem_wait_ld();
           }
-          const float2 r =
-              unf2(mul2(f2(p0, p1), add2(f2(__uint_as_float(up[i]), __uint_as_float(up[i + 1])), nd2)));
-          pk[e] = pack2(r.x, r.y);
+          if (need_mask)
+            ds_row32<true>(us, c ? up1 : up0, pk + 16 * c, sc2, nl2, nd2, kb + 32 * c, k_lo, k_hi);
+          else
+            ds_row32<false>(us, c ? up1 : up0, pk + 16 * c, sc2, nl2, nd2, kb + 32 * c, k_lo, k_hi);
         }
-        tc::tmem_st_32x32b_x16(ts, pk);  // dS over this thread's own S columns
+        tc::tc_fence_before();  // the chunk-1 load precedes the dS store over the same columns
+        tc::tmem_st_32x32b_x32(ts, pk);  // dS over the first 32 of this thread's 64 S columns
         tc::tmem_wait_st();
         tc::tc_fence_before();
       }
@@ -1061,9 +1135,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tc_fence_after();
     }
     norm_rope_bwd_half<HD>(t_dq + R.lane_off, R.half, R.r, scale, smem + S::Y_OFF,
-                           qv ? rq[int64_t(bh) * T + q] : 0.f, qk_norm, smem + S::COS_OFF,
-                           smem + S::SIN_OFF, dqkv + (int64_t(b) * T + tq) * ldq + h * HD, ok,
-                           qv, reinterpret_cast<float*>(smem + S::RED_OFF));
+                           qv ? rq[int64_t(bh) * T + q] : 0.f, qk_norm, smem + S::COS_OFF, smem + S::SIN_OFF,
+                           dqkv + (int64_t(b) * T + tq) * ldq + h * HD, ok, qv,
+                           reinterpret_cast<float*>(smem + S::RED_OFF));
   }
   ATTN_EPILOGUE(tmem)
 }
@@ -1071,39 +1145,54 @@ __global__ void __launch_bounds__(kThreads, 1)
 namespace {
 template <int HD>
 struct DkvSmem {
-  static constexpr uint32_t BIG = 128 * HD * 2;    // the K or V tile; also a cos / sin tile
-  static constexpr uint32_t SMALL = kInner * HD * 2;
-  static constexpr uint32_t K_OFF = 0, V_OFF = BIG;
-  static constexpr uint32_t Q_OFF = 2 * BIG;
-  static constexpr uint32_t DO_OFF = Q_OFF + kRingKV * SMALL;
-  static constexpr uint32_t COS_OFF = DO_OFF + kRingKV * SMALL, SIN_OFF = COS_OFF + BIG;
-  static constexpr uint32_t STAT_OFF = SIN_OFF + BIG;  // [ring][lse2 x 64 | D x 64]
-  static constexpr uint32_t RED_OFF = STAT_OFF;        // epilogue only, after the last step's stats
-  static constexpr uint32_t BAR_OFF = STAT_OFF + kRingKV * 2 * kInner * 4;
-  static_assert(V_OFF % 1024 == 0 && Q_OFF % 1024 == 0 && DO_OFF % 1024 == 0 && COS_OFF % 1024 == 0 &&
-                SMALL % 1024 == 0, "");
-  static_assert(kRingKV * 2 * kInner * 4 >= 2 * 128 * 4, "");
+  static constexpr uint32_t TILE = 128 * HD * 2;  // a 128-row K, V, Q or dO tile
+  static constexpr uint32_t K_OFF = 0, V_OFF = TILE;
+  static constexpr uint32_t Q_OFF = 2 * TILE;                    // Q ring
+  static constexpr uint32_t DO_OFF = Q_OFF + kDkvRingQ * TILE;   // dO ring
+  static constexpr uint32_t STAT_OFF = DO_OFF + kDkvRingDO * TILE;  // lse2 x 128 | D x 128
+  // the RoPE tiles of the epilogue, loaded into the dO ring once the last dV is done
+  static constexpr uint32_t COS_OFF = DO_OFF, SIN_OFF = DO_OFF + TILE;
+  static constexpr uint32_t RED_OFF = STAT_OFF;  // epilogue only, after the last step's stats
+  static constexpr uint32_t BAR_OFF = STAT_OFF + 2 * 128 * 4;
   static constexpr uint32_t BYTES = BAR_OFF + 256 + 1024;
-  static_assert(BYTES <= 232448, "");
+  static_assert(TILE % 1024 == 0 && BYTES <= 232448, "");
+};
+struct DkvBars {
+  uint64_t fixed_full;
+  uint64_t q_full[kDkvRingQ], q_empty[kDkvRingQ], do_full[kDkvRingDO], do_empty[kDkvRingDO];
+  uint64_t stat_full, stat_empty;
+  uint64_t s_full, dp_full, p_ready, ds_ready;
+  uint64_t acc_full, epi_full, done, done2;
+  uint32_t tmem_base;
+  int abort;
 };
 }  // namespace
 
-// dK, dV for 128 keys of one (batch, head), looping over 64-query tiles.
-// Warp 1 issues S^T_j = K Q_j^T and dV += P^T_{j-1} dO_{j-1}; warp 10 issues
-// dP^T_j = V dO_j^T and dK += dS^T_{j-1} Q_{j-1}.  Compute thread (key row,
-// half) handles queries [32*half, 32*half + 32) of each tile and writes bf16
-// P^T over its S^T columns and dS^T over its dP^T columns: the TMEM A operands
-// of the dV and dK products, each read by the warp that next overwrites those
-// columns (so in issue order).  The producer warp stages lse and D of the
-// tile's queries in shared memory next to the Q / dO tiles.  TMEM: S^T/dP^T
-// pairs at columns 0 and 128 (64 + 64 each), dV at 256, dK at 384.  The K tile
-// in shared memory doubles as the y of the norm backward.
+// dK, dV for 128 keys of one (batch, kv head), looping over 128-query tiles
+// of every query head of its group (all products M = 128, N = 128).  Warp 1
+// issues S^T_j = K Q_j^T, then dV += P^T_j dO_j once the threads have written
+// P^T_j; warp 10 issues dP^T_j = V dO_j^T, then dK += dS^T_j Q_j once they
+// have written dS^T_j.  Compute thread (key row, half) handles queries
+// [64*half, 64*half + 64) of each tile: it writes bf16 P^T over the first 32
+// of its 64 S^T columns and bf16 dS^T over the first 32 of its dP^T columns
+// (the TMEM A operands of the dV and dK products; 16-query step k at column
+// 64*(k/4) + 8*(k%4)).  The next S^T (dP^T) is issued by the same warp after
+// the dV (dK) product that reads those columns, so in order.  While the
+// threads turn S^T_j into P^T_j the tensor core runs dK_{j-1} and dP^T_j;
+// while they form dS^T_j it runs dV_j and S^T_{j+1}.  Warp 0 loads K and V
+// once and runs the Q and dO rings (a Q tile is read by S^T_j and, a step
+// later, by dK_j, so its ring has a third slot); warp 11 stages lse and D of
+// each step's queries in shared memory, loading the next step's while the
+// threads use the current one.  TMEM: S^T at column 0, dP^T at 128, dV at
+// 256, dK at 384.  The K tile in shared memory doubles as the y of the norm
+// backward; the RoPE tables of its 128 positions are loaded into the dO ring
+// after the last dV.
 template <int HD>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kDkvThreads, 1)
     attn_dkv_tc_kernel(const __grid_constant__ CUtensorMap map_k128,
                        const __grid_constant__ CUtensorMap map_v128,
-                       const __grid_constant__ CUtensorMap map_q64,
-                       const __grid_constant__ CUtensorMap map_do64,
+                       const __grid_constant__ CUtensorMap map_q128,
+                       const __grid_constant__ CUtensorMap map_do128,
                        const __grid_constant__ CUtensorMap map_cos,
                        const __grid_constant__ CUtensorMap map_sin,
                        const float* __restrict__ lse,
@@ -1111,137 +1200,174 @@ __global__ void __launch_bounds__(kThreads, 1)
                        __nv_bfloat16* __restrict__ dqkv, int64_t ldq, int H, int Hkv, int T,
                        int W, float scale, float scale_log2, int qk_norm, int32_t* status) {
   using S = DkvSmem<HD>;
+  constexpr int NCH = HD / 64;
+  constexpr uint32_t CH = 128 * 128;  // bytes of one 64-column chunk of a 128-row tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  BwdBars* bars = reinterpret_cast<BwdBars*>(smem + S::BAR_OFF);
+  DkvBars* bars = reinterpret_cast<DkvBars*>(smem + S::BAR_OFF);
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int n_kt = (T + 127) / 128;
   int bkv, kt;  // key tile 0 (the most queries) first
   grouped_item(int(blockIdx.x), int(gridDim.x) / n_kt, n_kt, bkv, kt);
   const int b = bkv / Hkv, hk = bkv % Hkv, rep = H / Hkv;
   const int k0 = kt * 128;
-  const int i_begin = k0 / kInner;
   // queries k0 .. min(T, k0 + 127 + W) - 1 see some key of the tile; the steps
-  // run over them once per query head of the group (head hk*rep + j / n_h)
-  const int n_h = (min(T, k0 + 127 + W) + kInner - 1) / kInner - i_begin;
+  // run over their 128-query tiles once per query head of the group (head
+  // hk*rep + j / n_h)
+  const int n_h = (min(T, k0 + 127 + W) + 127) / 128 - kt;
   const int n_steps = rep * n_h;
-  constexpr int NCH = HD / 64;
 
   ATTN_PROLOGUE(bars, {
     tc::mbar_init(&bars->fixed_full, 1);
-    tc::mbar_init(&bars->epi_full, 1);
-    for (int s = 0; s < kRingKV; ++s) {
-      tc::mbar_init(&bars->ring_full[s], 1 + 32);  // TMA bytes + the producer warp's stat stores
-      tc::mbar_init(&bars->ring_empty[s], 2);      // after dV (warp 1) and dK (warp 10)
+    for (int s = 0; s < kDkvRingQ; ++s) {
+      tc::mbar_init(&bars->q_full[s], 1);
+      tc::mbar_init(&bars->q_empty[s], 2);  // after S^T and dV (warp 1) and dK (warp 10)
     }
-    for (int s = 0; s < 2; ++s) {
-      tc::mbar_init(&bars->s_full[s], 1);
-      tc::mbar_init(&bars->dp_full[s], 1);
-      tc::mbar_init(&bars->ds_ready[s], 256);
+    for (int s = 0; s < kDkvRingDO; ++s) {
+      tc::mbar_init(&bars->do_full[s], 1);
+      tc::mbar_init(&bars->do_empty[s], 2);
     }
+    tc::mbar_init(&bars->stat_full, 32);
+    tc::mbar_init(&bars->stat_empty, 256);
+    tc::mbar_init(&bars->s_full, 1);
+    tc::mbar_init(&bars->dp_full, 1);
+    tc::mbar_init(&bars->p_ready, 256);
+    tc::mbar_init(&bars->ds_ready, 256);
     tc::mbar_init(&bars->acc_full, 2);
+    tc::mbar_init(&bars->epi_full, 1);
     tc::mbar_init(&bars->done, 1);
     tc::mbar_init(&bars->done2, 1);
   })
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort = &bars->abort;
-  const uint32_t t_dv = tmem + 256, t_dk = tmem + 384;
+  const uint32_t t_dp = tmem + 128, t_dv = tmem + 256, t_dk = tmem + 384;
 
   if (warp == 0) {
-    uint32_t issued = 0, last_par = 0;
-    if (lane == 0) {
-      tc::mbar_arrive_expect_tx(&bars->fixed_full, 2 * S::BIG);
+    // lane 0: K and V, then the Q ring; lane 1: the dO ring
+    if (lane < 2) {
+      const bool is_q = lane == 0;
+      uint64_t* full = is_q ? bars->q_full : bars->do_full;
+      uint64_t* empty = is_q ? bars->q_empty : bars->do_empty;
+      uint8_t* base = smem + (is_q ? S::Q_OFF : S::DO_OFF);
+      const int ring = is_q ? kDkvRingQ : kDkvRingDO;
+      uint32_t issued = 0, last_par = 0;
+      if (is_q) {
+        tc::mbar_arrive_expect_tx(&bars->fixed_full, 2 * S::TILE);
 #pragma unroll
-      for (int c = 0; c < NCH; ++c) {
-        tc::tma_load_2d(smem + S::K_OFF + c * (128 * 128), &map_k128, &bars->fixed_full, c * 64, bkv * T + k0);
-        tc::tma_load_2d(smem + S::V_OFF + c * (128 * 128), &map_v128, &bars->fixed_full, c * 64, bkv * T + k0);
+        for (int c = 0; c < NCH; ++c) {
+          tc::tma_load_2d(smem + S::K_OFF + c * CH, &map_k128, &bars->fixed_full, c * 64, bkv * T + k0);
+          tc::tma_load_2d(smem + S::V_OFF + c * CH, &map_v128, &bars->fixed_full, c * 64, bkv * T + k0);
+        }
+      }
+      for (int j = 0; j < n_steps; ++j) {
+        const int st = j % ring;
+        const uint32_t ph = (j / ring) & 1;
+        const int gi = j / n_h;
+        const int qs = (kt + j - gi * n_h) * 128;
+        const int h = hk * rep + gi;
+        if (!tc::mbar_wait_bounded(&empty[st], ph ^ 1, abort, kWaitNs)) {
+          record_status(status, GPT_ETIMEOUT, K_ATTN, 30);
+          *abort = 1;
+          break;
+        }
+        tc::mbar_arrive_expect_tx(&full[st], S::TILE);
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+          if (is_q)
+            tc::tma_load_2d(base + st * S::TILE + c * CH, &map_q128, &full[st], c * 64, (b * H + h) * T + qs);
+          else
+            tc::tma_load_2d(base + st * S::TILE + c * CH, &map_do128, &full[st], h * HD + c * 64, b * T + qs);
+        }
+        issued |= 1u << st;
+        last_par = (last_par & ~(1u << st)) | (ph << st);
+      }
+      // the dO ring is free once every dV and dP^T is done: the epilogue's RoPE tiles go there
+      bool epi = false;
+      if (!is_q && !*abort) {
+        bool freed = true;
+        for (int s = 0; s < ring; ++s)
+          if (issued >> s & 1) freed = freed && tc::mbar_wait_bounded(&empty[s], (last_par >> s) & 1, abort, kWaitNs);
+        if (freed) {
+          load_rope_tiles<HD>(smem + S::COS_OFF, smem + S::SIN_OFF, &map_cos, &map_sin, &bars->epi_full, k0);
+          epi = true;
+        } else {
+          record_status(status, GPT_ETIMEOUT, K_ATTN, 35);
+          *abort = 1;
+        }
+      }
+      if (*abort) {
+        if (is_q) tc::mbar_wait_bounded(&bars->fixed_full, 0, nullptr, kWaitNs);
+        if (epi) tc::mbar_wait_bounded(&bars->epi_full, 0, nullptr, kWaitNs);
+        for (int s = 0; s < ring; ++s)
+          if (issued >> s & 1) tc::mbar_wait_bounded(&full[s], (last_par >> s) & 1, nullptr, kWaitNs);
       }
     }
+  } else if (warp == 11) {
+    // lse2 and D of step j's queries (4 per lane), loaded before the wait for
+    // the threads to be done with step j-1's
+    float* stat = reinterpret_cast<float*>(smem + S::STAT_OFF);
     for (int j = 0; j < n_steps; ++j) {
-      const int st = j % kRingKV;
-      const uint32_t ph = (j / kRingKV) & 1;
       const int gi = j / n_h;
-      const int qs = (i_begin + j - gi * n_h) * kInner;
-      const int h = hk * rep + gi, bh = b * H + h;
-      if (!tc::mbar_wait_warp(&bars->ring_empty[st], ph ^ 1, abort, kWaitNs)) {
-        if (lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 30);
+      const int qs = (kt + j - gi * n_h) * 128;
+      const int bh = b * H + hk * rep + gi;
+      float l4[4], d4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int qq = qs + lane * 4 + e;
+        l4[e] = qq < T ? lse[int64_t(bh) * T + qq] * kLog2e : 0.f;
+        d4[e] = qq < T ? D[int64_t(bh) * T + qq] : 0.f;
+      }
+      if (!tc::mbar_wait_warp(&bars->stat_empty, (j & 1) ^ 1, abort, kWaitNs)) {
+        if (lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 34);
         *abort = 1;
         break;
       }
-      if (lane == 0) {
-        tc::mbar_arrive_expect_tx(&bars->ring_full[st], 2 * S::SMALL);
-#pragma unroll
-        for (int c = 0; c < NCH; ++c) {
-          tc::tma_load_2d(smem + S::Q_OFF + st * S::SMALL + c * (kInner * 128), &map_q64,
-                          &bars->ring_full[st], c * 64, bh * T + qs);
-          tc::tma_load_2d(smem + S::DO_OFF + st * S::SMALL + c * (kInner * 128), &map_do64,
-                          &bars->ring_full[st], h * HD + c * 64, b * T + qs);
-        }
-        if (j == 0)
-          load_epilogue_tiles<HD>(nullptr, smem + S::COS_OFF, smem + S::SIN_OFF, nullptr, &map_cos,
-                                  &map_sin, &bars->epi_full, 0, k0);
-      }
-      float* stat = reinterpret_cast<float*>(smem + S::STAT_OFF) + st * 2 * kInner;
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int qi = lane * 2 + e;
-        const int qq = qs + qi;
-        stat[qi] = qq < T ? lse[int64_t(bh) * T + qq] * kLog2e : 0.f;
-        stat[kInner + qi] = qq < T ? D[int64_t(bh) * T + qq] : 0.f;
-      }
-      tc::mbar_arrive(&bars->ring_full[st]);
-      issued |= 1u << st;
-      last_par = (last_par & ~(1u << st)) | (ph << st);
-    }
-    if (lane == 0 && *abort) {
-      tc::mbar_wait_bounded(&bars->fixed_full, 0, nullptr, kWaitNs);
-      if (issued) tc::mbar_wait_bounded(&bars->epi_full, 0, nullptr, kWaitNs);
-      for (int s = 0; s < kRingKV; ++s)
-        if (issued >> s & 1) tc::mbar_wait_bounded(&bars->ring_full[s], (last_par >> s) & 1, nullptr, kWaitNs);
+      *reinterpret_cast<float4*>(stat + lane * 4) = make_float4(l4[0], l4[1], l4[2], l4[3]);
+      *reinterpret_cast<float4*>(stat + 128 + lane * 4) = make_float4(d4[0], d4[1], d4[2], d4[3]);
+      tc::mbar_arrive(&bars->stat_full);
     }
   } else if (warp == 1 || warp == 10) {
-    // warp 1: S^T = K Q^T and dV += P^T dO;  warp 10: dP^T = V dO^T and dK += dS^T Q
+    // warp 1: S^T = K Q^T, then dV += P^T dO;  warp 10: dP^T = V dO^T, then dK += dS^T Q
     const bool is_s = warp == 1;
-    constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, kInner, false, false);
+    constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, 128, false, false);
     constexpr uint32_t idesc_acc = tc::idesc_bf16_f32(128, HD, false, true);
     const uint64_t fd = tc::smem_desc_sw128(tc::smem_u32(smem + (is_s ? S::K_OFF : S::V_OFF)), 16);
-    const uint32_t col = is_s ? 0u : uint32_t(kInner);  // S^T or dP^T half of each pair
+    const uint32_t t_prod = is_s ? tmem : t_dp;  // S^T or dP^T; then P^T or dS^T over it
     const uint32_t t_acc = is_s ? t_dv : t_dk;
-    uint64_t* prod_full = is_s ? bars->s_full : bars->dp_full;
+    uint64_t* prod_full = is_s ? &bars->s_full : &bars->dp_full;
+    uint64_t* a_ready = is_s ? &bars->p_ready : &bars->ds_ready;
     bool ok = tc::mbar_wait_warp(&bars->fixed_full, 0, abort, kWaitNs);
     bool issued_any = false;
-    auto issue_acc = [&](int j) -> bool {
-      if (!tc::mbar_wait_warp(&bars->ds_ready[j & 1], (j >> 1) & 1, abort, kWaitNs)) return false;
-      tc::tc_fence_after();
-      const uint32_t at = tmem + (j & 1) * 128 + col;  // P^T or dS^T, bf16 pairs
-      // dV takes dO, dK takes Q: the other ring tile
-      const uint64_t bmn = tc::smem_desc_sw128(
-          tc::smem_u32(smem + (is_s ? S::DO_OFF : S::Q_OFF) + (j % kRingKV) * S::SMALL), kInner * 128);
-#pragma unroll
-      for (int k = 0; k < kInner / 16; ++k)
-        tc::mma_bf16_ts_elect(t_acc, at + 32 * (k >> 1) + 8 * (k & 1), tc::desc_advance(bmn, k * 2048),
-                              idesc_acc, (j | k) != 0);
-      tc::mma_commit_elect(&bars->ring_empty[j % kRingKV]);
-      return true;
-    };
     for (int j = 0; ok && j < n_steps; ++j) {
-      const int st = j % kRingKV;
-      if (!tc::mbar_wait_warp(&bars->ring_full[st], (j / kRingKV) & 1, abort, kWaitNs)) { ok = false; break; }
+      const int sq = j % kDkvRingQ, sd = j % kDkvRingDO;
+      uint64_t* own_full = is_s ? &bars->q_full[sq] : &bars->do_full[sd];  // S^T reads Q, dP^T reads dO
+      const uint32_t own_par = is_s ? (j / kDkvRingQ) & 1 : (j / kDkvRingDO) & 1;
+      uint64_t* oth_full = is_s ? &bars->do_full[sd] : &bars->q_full[sq];  // dV reads dO, dK reads Q
+      const uint32_t oth_par = is_s ? (j / kDkvRingDO) & 1 : (j / kDkvRingQ) & 1;
+      uint8_t* own = smem + (is_s ? S::Q_OFF + sq * S::TILE : S::DO_OFF + sd * S::TILE);
+      uint8_t* oth = smem + (is_s ? S::DO_OFF + sd * S::TILE : S::Q_OFF + sq * S::TILE);
+      if (!tc::mbar_wait_warp(own_full, own_par, abort, kWaitNs)) { ok = false; break; }
       tc::tc_fence_after();
-      const uint64_t rd = tc::smem_desc_sw128(
-          tc::smem_u32(smem + (is_s ? S::Q_OFF : S::DO_OFF) + st * S::SMALL), 16);
-      const uint32_t pair = tmem + (j & 1) * 128 + col;
+      const uint64_t rd = tc::smem_desc_sw128(tc::smem_u32(own), 16);
 #pragma unroll
-      for (int k = 0; k < HD / 16; ++k)
-        tc::mma_bf16_ss_elect(pair, tc::desc_advance(fd, (k >> 2) * (128 * 128) + (k & 3) * 32),
-                              tc::desc_advance(rd, (k >> 2) * (kInner * 128) + (k & 3) * 32), idesc_s,
-                              k != 0);
+      for (int k = 0; k < HD / 16; ++k) {
+        const uint32_t off = (k >> 2) * CH + (k & 3) * 32;
+        tc::mma_bf16_ss_elect(t_prod, tc::desc_advance(fd, off), tc::desc_advance(rd, off), idesc_s, k != 0);
+      }
       issued_any = true;
-      tc::mma_commit_elect(&prod_full[j & 1]);
-      if (j >= 1 && !issue_acc(j - 1)) { ok = false; break; }
+      tc::mma_commit_elect(prod_full);
+      if (!tc::mbar_wait_warp(a_ready, j & 1, abort, kWaitNs)) { ok = false; break; }
+      if (!tc::mbar_wait_warp(oth_full, oth_par, abort, kWaitNs)) { ok = false; break; }
+      tc::tc_fence_after();
+      const uint64_t bmn = tc::smem_desc_sw128(tc::smem_u32(oth), CH);
+#pragma unroll
+      for (int k = 0; k < 128 / 16; ++k)
+        tc::mma_bf16_ts_elect(t_acc, t_prod + 64 * (k >> 2) + 8 * (k & 3), tc::desc_advance(bmn, k * 2048),
+                              idesc_acc, (j | k) != 0);
+      tc::mma_commit_elect(&bars->q_empty[sq]);
+      tc::mma_commit_elect(&bars->do_empty[sd]);
     }
-    if (ok && n_steps >= 1) ok = issue_acc(n_steps - 1);
     if (ok) tc::mma_commit_elect(&bars->acc_full);
     if (!ok) {
       if (lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, is_s ? 31 : 33);
@@ -1257,56 +1383,65 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int key = k0 + R.r;
     const bool kv = key < T;
     const int tk = kv ? key : 0;
-    const int end_q = key + W;  // the key's last visible query is end_q - 1
+    // the key's visible queries [q_lo, q_hi): none for a row past T
+    const int q_lo = key, q_hi = kv ? min(T, key + W) : key;
+    const uint32_t ts = tmem + R.lane_off + R.half * 64;
+    const uint32_t tp = t_dp + R.lane_off + R.half * 64;
+    const float* stat = reinterpret_cast<const float*>(smem + S::STAT_OFF) + R.half * 64;
     bool ok = true;
     for (int j = 0; j < n_steps; ++j) {
-      const int sb = j & 1, st = j % kRingKV;
-      // the producer warp stored this step's stats before arriving on
-      // ring_full[st]; waiting on that phase makes them visible here
-      if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->s_full[sb], (j >> 1) & 1, abort, kWaitNs));
-      if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->dp_full[sb], (j >> 1) & 1, abort, kWaitNs));
-      if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->ring_full[st], (j / kRingKV) & 1, abort, kWaitNs));
+      const int qs = (kt + j - (j / n_h) * n_h) * 128 + R.half * 64;
+      if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->stat_full, j & 1, abort, kWaitNs));
+      if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->s_full, j & 1, abort, kWaitNs));
+      const bool need_mask = qs < q_lo || qs + 64 > q_hi;
+      float p[64];
       if (ok) {
         tc::tc_fence_after();
-        const int qs = (i_begin + j - (j / n_h) * n_h) * kInner + R.half * 32;
-        const float4* stat4 =
-            reinterpret_cast<const float4*>(smem + S::STAT_OFF + (st * 2 * kInner + R.half * 32) * 4);
-        const uint32_t ts = tmem + sb * 128 + R.lane_off + R.half * 32;
-        uint32_t us[32], up[32];
-        tc::tmem_ld_32x32b_x32(ts, us);
-        tc::tmem_ld_32x32b_x32(ts + kInner, up);
+        uint32_t us0[32], us1[32];
+        tc::tmem_ld_32x32b_x32(ts, us0);
+        tc::tmem_ld_32x32b_x32(ts + 32, us1);
         tc::tmem_wait_ld();
-        const bool need_mask = !kv || qs < key || qs + 32 > T || qs + 32 > end_q;
-        uint32_t pp[16], pd[16];
-#pragma unroll
-        for (int g = 0; g < 8; ++g) {  // 4 queries per group
-          const float4 l4 = stat4[g], d4 = stat4[kInner / 4 + g];
-          const float l2[4] = {l4.x, l4.y, l4.z, l4.w}, dd[4] = {d4.x, d4.y, d4.z, d4.w};
-#pragma unroll
-          for (int e = 0; e < 4; e += 2) {
-            const int i = 4 * g + e;
-            const float2 x = unf2(fma2(f2(__uint_as_float(us[i]), __uint_as_float(us[i + 1])),
-                                       f2(scale_log2, scale_log2), f2(-l2[e], -l2[e + 1])));
-            float p0 = ex2(x.x), p1 = ex2(x.y);
-            if (need_mask) {
-              if (qs + i < key || qs + i >= T || !kv || qs + i >= end_q) p0 = 0.f;
-              if (qs + i + 1 < key || qs + i + 1 >= T || !kv || qs + i + 1 >= end_q) p1 = 0.f;
-            }
-            pp[i / 2] = pack2(p0, p1);
-            const float2 r = unf2(mul2(f2(p0, p1), add2(f2(__uint_as_float(up[i]), __uint_as_float(up[i + 1])),
-                                                          f2(-dd[e], -dd[e + 1]))));
-            pd[i / 2] = pack2(r.x, r.y);
-          }
-        }
-        tc::tmem_st_32x32b_x16(ts, pp);           // P^T over this thread's S^T columns
-        tc::tmem_st_32x32b_x16(ts + kInner, pd);  // dS^T over its dP^T columns
+        uint32_t pk[32];
+        if (need_mask)
+          p_col64<true>(us0, us1, stat, p, pk, scale_log2, qs, q_lo, q_hi);
+        else
+          p_col64<false>(us0, us1, stat, p, pk, scale_log2, qs, q_lo, q_hi);
+        tc::tmem_st_32x32b_x32(ts, pk);  // P^T over the first 32 of this thread's S^T columns
         tc::tmem_wait_st();
         tc::tc_fence_before();
       }
-      tc::mbar_arrive(&bars->ds_ready[sb]);
+      tc::mbar_arrive(&bars->p_ready);
+      if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->dp_full, j & 1, abort, kWaitNs));
+      if (ok) {
+        tc::tc_fence_after();
+        uint32_t pd[32];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t up[32];
+          tc::tmem_ld_32x32b_x32(tp + 32 * c, up);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int g = 0; g < 8; ++g) {
+            const float4 d4 = *reinterpret_cast<const float4*>(stat + 128 + 32 * c + 4 * g);
+            const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+            for (int e = 0; e < 4; e += 2) {
+              const int i = 4 * g + e;
+              const float2 r = unf2(mul2(f2(p[32 * c + i], p[32 * c + i + 1]),
+                                         add2(f2(__uint_as_float(up[i]), __uint_as_float(up[i + 1])),
+                                              f2(-dd[e], -dd[e + 1]))));
+              pd[16 * c + i / 2] = pack2(r.x, r.y);
+            }
+          }
+        }
+        tc::tmem_st_32x32b_x32(tp, pd);  // dS^T over the first 32 of this thread's dP^T columns
+        tc::tmem_wait_st();
+        tc::tc_fence_before();
+      }
+      tc::mbar_arrive(&bars->stat_empty);  // this step's lse and D are no longer read
+      tc::mbar_arrive(&bars->ds_ready);
     }
     if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->acc_full, 0, abort, kWaitNs));
-    if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->epi_full, 0, abort, kWaitNs));
     if (!ok) {
       if (R.lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 32);
       *abort = 1;
@@ -1328,6 +1463,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                            pack2(v[i + 6], v[i + 7]));
         }
       }
+    }
+    if (ok && !__all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->epi_full, 0, abort, kWaitNs))) {
+      if (R.lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 36);
+      *abort = 1;
+      ok = false;
     }
     // the stats region is free once every step is done (acc_full): it holds red
     norm_rope_bwd_half<HD>(t_dk + R.lane_off, R.half, R.r, scale, smem + S::K_OFF,
@@ -1351,13 +1491,11 @@ int attn_bwd_tc_t(const gpt_config& c, const void* q, const void* k, const void*
   const int64_t N = int64_t(B) * T;
   attn_rowdot_kernel<<<ceil_div(N * H * (HD / 8), 256), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(dO), static_cast<const __nv_bfloat16*>(o), Dbuf, N, H, T, HD);
-  CUtensorMap k64, v64, k128, v128, q64, do64, q128, do128, mcos, msin;
-  bool ok = tile_map(&k64, k, kv_rows, HD, HD, 64) && tile_map(&v64, v, kv_rows, HD, HD, 64) &&
-            tile_map(&k128, k, kv_rows, HD, HD, 128) && tile_map(&v128, v, kv_rows, HD, HD, 128) &&
-            tile_map(&q64, q, rows, HD, HD, 64) && tile_map(&do64, dO, ntok, d, d, 64) &&
-            tile_map(&q128, q, rows, HD, HD, 128) && tile_map(&do128, dO, ntok, d, d, 128) &&
-            tile_map_f32(&mcos, cos_t, T, HD / 2, HD / 2, 128) &&
-            tile_map_f32(&msin, sin_t, T, HD / 2, HD / 2, 128);
+  CUtensorMap k128, v128, q128, do128, mcos, msin;
+  const bool ok = tile_map(&k128, k, kv_rows, HD, HD, 128) && tile_map(&v128, v, kv_rows, HD, HD, 128) &&
+                  tile_map(&q128, q, rows, HD, HD, 128) && tile_map(&do128, dO, ntok, d, d, 128) &&
+                  tile_map_f32(&mcos, cos_t, T, HD / 2, HD / 2, 128) &&
+                  tile_map_f32(&msin, sin_t, T, HD / 2, HD / 2, 128);
   if (!ok) return 1;
   const float scale = 1.f / sqrtf(float(HD));
   const float scale_log2 = scale * kLog2e;
@@ -1366,14 +1504,14 @@ int attn_bwd_tc_t(const gpt_config& c, const void* q, const void* k, const void*
   const int smem_q = int(DqSmem<HD>::BYTES);
   if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_q) != cudaSuccess)
     return 1;
-  kq<<<nt * B * H, kThreads, smem_q, st>>>(q128, do128, k64, v64, mcos, msin, lse, Dbuf, rq,
+  kq<<<nt * B * H, kThreads, smem_q, st>>>(q128, do128, k128, v128, mcos, msin, lse, Dbuf, rq,
                                            static_cast<__nv_bfloat16*>(dqkv), ldq, H, Hkv, T, W,
                                            scale, scale_log2, c.qk_norm, status);
   auto kk = attn_dkv_tc_kernel<HD>;
   const int smem_k = int(DkvSmem<HD>::BYTES);
   if (cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_k) != cudaSuccess)
     return 1;
-  kk<<<nt * B * Hkv, kThreads, smem_k, st>>>(k128, v128, q64, do64, mcos, msin, lse, Dbuf, rk,
+  kk<<<nt * B * Hkv, kDkvThreads, smem_k, st>>>(k128, v128, q128, do128, mcos, msin, lse, Dbuf, rk,
                                              static_cast<__nv_bfloat16*>(dqkv), ldq, H, Hkv, T, W,
                                              scale, scale_log2, c.qk_norm, status);
   return last_launch_rc();
