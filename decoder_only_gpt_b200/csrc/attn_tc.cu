@@ -137,6 +137,20 @@ bool tile_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+// The [B, T, ld] bf16 rows of the q|k|v gradient as a 3-D map with boxes of 64
+// columns x 128 positions x 1 sequence: a box past position T - 1 is clipped
+// at the end of its own sequence.
+bool seq_map(CUtensorMap* m, const void* base, uint64_t B, uint64_t T, uint64_t ld) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {ld, T, B};
+  cuuint64_t strides[2] = {ld * 2, T * ld * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 // [rows, cols] fp32 row-major (pitch ld elements), box 32 columns x box_rows rows
 bool tile_map_f32(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
                   uint32_t box_rows) {
@@ -701,7 +715,6 @@ __global__ void attn_rowdot_kernel(const __nv_bfloat16* __restrict__ dO,
 // slots of the dK/dV kernel's Q and dO rings (a Q tile is read by S^T_j and,
 // after the threads have formed dS^T_j, by dK_j)
 constexpr int kDkvRingQ = 3, kDkvRingDO = 2;
-constexpr int kDkvThreads = 384;  // as kThreads, plus warp 11 staging lse and D
 // slots of the dQ kernel's K and V rings: a K tile is read by S_j early in its
 // step and by the dQ product at the end of it, so it stays resident about two
 // steps and needs a third slot to be prefetched in time; V only feeds dP_j
@@ -709,10 +722,11 @@ constexpr int kDqRingK = 3, kDqRingV = 2;
 
 // One row's gradient w.r.t. its normalised, rotated q or k (TMEM, fp32, HD
 // columns at `taddr`, times `scale`) back through RMSNorm (y: the normalised
-// row, rr: its 1/rms) and RoPE, written as bf16.  y, cos and sin come from
-// shared-memory tiles of the CTA's 128 rows, stored as TMA writes them with the
-// 128-byte swizzle: y [128 x HD] bf16 in 64-column chunks, cos / sin
-// [128 x HD/2] fp32 in 32-column chunks (16 KB per chunk).  The row's two
+// row, rr: its 1/rms) and RoPE, written as bf16 into row r of the shared-memory
+// tile `out_tile` (for a TMA store).  y, cos and sin come from shared-memory
+// tiles of the CTA's 128 rows.  All tiles are stored as TMA writes and reads
+// them, with the 128-byte swizzle: y and out [128 x HD] bf16 in 64-column
+// chunks, cos / sin [128 x HD/2] fp32 in 32-column chunks (16 KB per chunk).  The row's two
 // compute threads split the rotation pairs: thread `half` takes pairs i in
 // [half*HD/4, (half+1)*HD/4) and their partners i + HD/2; the mean(g y) of the
 // norm is summed across both through `red` (one compute_bar, reached on every
@@ -736,8 +750,7 @@ template <int HD>
 __device__ __forceinline__ void norm_rope_bwd_half(uint32_t taddr, int half, int r, float scale,
                                                    const uint8_t* y_tile, float rr, int qk_norm,
                                                    const uint8_t* cos_tile, const uint8_t* sin_tile,
-                                                   __nv_bfloat16* __restrict__ out, bool ok,
-                                                   bool write, float* red) {
+                                                   uint8_t* out_tile, bool ok, bool write, float* red) {
   constexpr int HALF = HD / 2, Q4 = HD / 4;
   const int i0 = half * Q4;
   float ga[Q4], gb[Q4];
@@ -792,9 +805,28 @@ __device__ __forceinline__ void norm_rope_bwd_half(uint32_t taddr, int half, int
     }
   }
 #pragma unroll
-  for (int i = 0; i < Q4 / 2; i += 4) {
-    *reinterpret_cast<uint4*>(out + i0 + 2 * i) = make_uint4(pa[i], pa[i + 1], pa[i + 2], pa[i + 3]);
-    *reinterpret_cast<uint4*>(out + HALF + i0 + 2 * i) = make_uint4(pb[i], pb[i + 1], pb[i + 2], pb[i + 3]);
+  for (int i = 0; i < Q4 / 2; i += 4) {  // 8 bf16 per 16-byte unit
+    *reinterpret_cast<uint4*>(out_tile + tile_unit(r, (i0 + 2 * i) / 8)) =
+        make_uint4(pa[i], pa[i + 1], pa[i + 2], pa[i + 3]);
+    *reinterpret_cast<uint4*>(out_tile + tile_unit(r, (HALF + i0 + 2 * i) / 8)) =
+        make_uint4(pb[i], pb[i + 1], pb[i + 2], pb[i + 3]);
+  }
+}
+
+// After every compute thread has written its rows of the output tiles: fence,
+// barrier, and one thread stores `n` tiles of [128 x HD] with TMA at columns
+// col[t] of positions pos0 .. pos0 + 127 of sequence b (clipped at T).
+template <int HD>
+__device__ __forceinline__ void store_tiles(const CUtensorMap* map, uint8_t* const* tiles, const int* col, int n,
+                                            int pos0, int b, bool ok) {
+  tc::fence_proxy_async_smem();
+  compute_bar();
+  if (ok && threadIdx.x == 64) {
+    for (int t = 0; t < n; ++t)
+#pragma unroll
+      for (int c = 0; c < HD / 64; ++c) tc::tma_store_3d(map, tiles[t] + c * (128 * 128), col[t] + c * 64, pos0, b);
+    tc::bulk_commit();
+    tc::bulk_wait_read();  // the tiles' shared memory is released when the CTA ends
   }
 }
 
@@ -822,24 +854,21 @@ __device__ __forceinline__ void ds_row32(const uint32_t (&us)[32], const uint32_
     pk[e] = pack2(r.x, r.y);
   }
 }
-// P^T for 64 queries q0 .. q0 + 63 of one key row: p = 2^(s * scale_log2 -
-// lse2_q) from the S^T columns us0 | us1 and the staged lse2 (`l2`), kept in
-// fp32 and as 32 packed bf16 pairs.  MASK: P = 0 outside the key's visible
-// queries [q_lo, q_hi).
+// P^T for 32 queries q0 .. q0 + 31 of one key row: p = 2^(s * scale_log2 -
+// lse2_q) from the S^T columns `us` and the staged -lse2 (`nl2s`), kept in fp32
+// and as 16 packed bf16 pairs.  MASK: P = 0 outside the key's visible queries
+// [q_lo, q_hi).
 template <bool MASK>
-__device__ __forceinline__ void p_col64(const uint32_t (&us0)[32], const uint32_t (&us1)[32], const float* l2s,
-                                        float (&p)[64], uint32_t (&pk)[32], float scale_log2, int q0, int q_lo,
-                                        int q_hi) {
+__device__ __forceinline__ void p_col32(const uint32_t (&us)[32], const float* nl2s, float* p, uint32_t (&pk)[16],
+                                        float scale_log2, int q0, int q_lo, int q_hi) {
 #pragma unroll
-  for (int g = 0; g < 16; ++g) {  // 4 queries per group
-    const float4 l4 = *reinterpret_cast<const float4*>(l2s + 4 * g);
-    const float l2[4] = {l4.x, l4.y, l4.z, l4.w};
+  for (int g = 0; g < 8; ++g) {  // 4 queries per group
+    const float4 l4 = *reinterpret_cast<const float4*>(nl2s + 4 * g);
 #pragma unroll
     for (int e = 0; e < 4; e += 2) {
       const int i = 4 * g + e;
-      const uint32_t a = i < 32 ? us0[i] : us1[i - 32], c = i < 32 ? us0[i + 1] : us1[i - 31];
-      const float2 x = unf2(fma2(f2(__uint_as_float(a), __uint_as_float(c)), f2(scale_log2, scale_log2),
-                                 f2(-l2[e], -l2[e + 1])));
+      const float2 x = unf2(fma2(f2(__uint_as_float(us[i]), __uint_as_float(us[i + 1])),
+                                 f2(scale_log2, scale_log2), e ? f2(l4.z, l4.w) : f2(l4.x, l4.y)));
       float p0 = ex2(x.x), p1 = ex2(x.y);
       if (MASK) {
         if (q0 + i < q_lo || q0 + i >= q_hi) p0 = 0.f;
@@ -859,7 +888,8 @@ struct DqSmem {
   static constexpr uint32_t K_OFF = 2 * TILE;                   // K ring
   static constexpr uint32_t V_OFF = K_OFF + kDqRingK * TILE;    // V ring
   static constexpr uint32_t Y_OFF = Q_OFF;   // the Q tile is the y of the norm backward
-  static constexpr uint32_t RED_OFF = K_OFF;  // epilogue only, once no product reads K
+  // epilogue only, once no product reads K: the norm reduction and the dQ tile
+  static constexpr uint32_t RED_OFF = K_OFF, OUT_OFF = K_OFF + TILE;
   // the RoPE tiles of the epilogue, loaded into the V ring once the last dP is done
   static constexpr uint32_t COS_OFF = V_OFF, SIN_OFF = V_OFF + TILE;
   static constexpr uint32_t BAR_OFF = V_OFF + kDqRingV * TILE;
@@ -899,9 +929,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap map_v128,
                       const __grid_constant__ CUtensorMap map_cos,
                       const __grid_constant__ CUtensorMap map_sin,
+                      const __grid_constant__ CUtensorMap map_out,
                       const float* __restrict__ lse,
-                      const float* __restrict__ D, const float* __restrict__ rq,
-                      __nv_bfloat16* __restrict__ dqkv, int64_t ldq, int H, int Hkv, int T,
+                      const float* __restrict__ D, const float* __restrict__ rq, int H, int Hkv, int T,
                       int W, float scale, float scale_log2, int qk_norm, int32_t* status) {
   using S = DqSmem<HD>;
   constexpr int NCH = HD / 64;
@@ -1008,10 +1038,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, 128, false, false);
     constexpr uint32_t idesc_dq = tc::idesc_bf16_f32(128, HD, false, true);
     const uint64_t qd = tc::smem_desc_sw128(tc::smem_u32(smem + S::Q_OFF), 16);
-    bool ok = tc::mbar_wait_warp(&bars->fixed_full, 0, abort, kWaitNs);
+    bool ok = tc::mbar_spin_warp(&bars->fixed_full, 0, abort, kWaitNs);
     bool issued_any = false;
     auto issue_dq = [&](int j) -> bool {
-      if (!tc::mbar_wait_warp(&bars->ds_ready[j & 1], (j >> 1) & 1, abort, kWaitNs)) return false;
+      if (!tc::mbar_spin_warp(&bars->ds_ready[j & 1], (j >> 1) & 1, abort, kWaitNs)) return false;
       tc::tc_fence_after();
       const uint32_t ds_t = tmem + (j & 1) * 128;
       const uint64_t kb = tc::smem_desc_sw128(tc::smem_u32(smem + S::K_OFF + (j % kDqRingK) * S::TILE), CH);
@@ -1024,7 +1054,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     for (int j = 0; ok && j < n_steps; ++j) {
       const int st = j % kDqRingK;
-      if (!tc::mbar_wait_warp(&bars->k_full[st], (j / kDqRingK) & 1, abort, kWaitNs)) { ok = false; break; }
+      if (!tc::mbar_spin_warp(&bars->k_full[st], (j / kDqRingK) & 1, abort, kWaitNs)) { ok = false; break; }
       tc::tc_fence_after();
       const uint64_t kd = tc::smem_desc_sw128(tc::smem_u32(smem + S::K_OFF + st * S::TILE), 16);
 #pragma unroll
@@ -1051,12 +1081,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // dP_j = dO V_j^T into the dP buffer, once the compute threads have loaded dP_{j-1}
     constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, 128, false, false);
     const uint64_t dod = tc::smem_desc_sw128(tc::smem_u32(smem + S::DO_OFF), 16);
-    bool ok = tc::mbar_wait_warp(&bars->fixed_full, 0, abort, kWaitNs);
+    bool ok = tc::mbar_spin_warp(&bars->fixed_full, 0, abort, kWaitNs);
     bool issued_any = false;
     for (int j = 0; ok && j < n_steps; ++j) {
       const int st = j % kDqRingV;
-      if (j >= 1 && !tc::mbar_wait_warp(&bars->dp_free, (j - 1) & 1, abort, kWaitNs)) { ok = false; break; }
-      if (!tc::mbar_wait_warp(&bars->v_full[st], (j / kDqRingV) & 1, abort, kWaitNs)) { ok = false; break; }
+      if (j >= 1 && !tc::mbar_spin_warp(&bars->dp_free, (j - 1) & 1, abort, kWaitNs)) { ok = false; break; }
+      if (!tc::mbar_spin_warp(&bars->v_full[st], (j / kDqRingV) & 1, abort, kWaitNs)) { ok = false; break; }
       tc::tc_fence_after();
       const uint64_t vd = tc::smem_desc_sw128(tc::smem_u32(smem + S::V_OFF + st * S::TILE), 16);
 #pragma unroll
@@ -1080,7 +1110,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const Roles R = roles();
     const int q = q0 + R.r;
     const bool qv = q < T;
-    const int tq = qv ? q : 0;
     // the query's visible keys [k_lo, k_hi): none for a row past T
     const int k_lo = q - W + 1, k_hi = qv ? q + 1 : k_lo;
     const float lse2 = qv ? lse[int64_t(bh) * T + q] * kLog2e : 0.f;
@@ -1088,8 +1117,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int j = 0; j < n_steps; ++j) {
       const int sb = j & 1;
-      if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->s_full[sb], (j >> 1) & 1, abort, kWaitNs));
-      if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->dp_full, j & 1, abort, kWaitNs));
+      if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_spin(&bars->s_full[sb], (j >> 1) & 1, abort, kWaitNs));
+      if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_spin(&bars->dp_full, j & 1, abort, kWaitNs));
       // dP first, so that dP_{j+1} may start as early as possible; S in two
       // 32-column chunks (fewer live registers)
       uint32_t up0[32], up1[32], us[32], pk[32];
@@ -1126,8 +1155,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc::mbar_arrive(&bars->ds_ready[sb]);
     }
-    if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->acc_full, 0, abort, kWaitNs));
-    if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->epi_full, 0, abort, kWaitNs));
+    if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_spin(&bars->acc_full, 0, abort, kWaitNs));
+    if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_spin(&bars->epi_full, 0, abort, kWaitNs));
     if (!ok) {
       if (R.lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 22);
       *abort = 1;
@@ -1136,8 +1165,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     norm_rope_bwd_half<HD>(t_dq + R.lane_off, R.half, R.r, scale, smem + S::Y_OFF,
                            qv ? rq[int64_t(bh) * T + q] : 0.f, qk_norm, smem + S::COS_OFF, smem + S::SIN_OFF,
-                           dqkv + (int64_t(b) * T + tq) * ldq + h * HD, ok, qv,
-                           reinterpret_cast<float*>(smem + S::RED_OFF));
+                           smem + S::OUT_OFF, ok, qv, reinterpret_cast<float*>(smem + S::RED_OFF));
+    uint8_t* const tiles[1] = {smem + S::OUT_OFF};
+    const int cols[1] = {h * HD};
+    store_tiles<HD>(&map_out, tiles, cols, 1, q0, b, ok);
   }
   ATTN_EPILOGUE(tmem)
 }
@@ -1149,10 +1180,12 @@ struct DkvSmem {
   static constexpr uint32_t K_OFF = 0, V_OFF = TILE;
   static constexpr uint32_t Q_OFF = 2 * TILE;                    // Q ring
   static constexpr uint32_t DO_OFF = Q_OFF + kDkvRingQ * TILE;   // dO ring
-  static constexpr uint32_t STAT_OFF = DO_OFF + kDkvRingDO * TILE;  // lse2 x 128 | D x 128
+  static constexpr uint32_t STAT_OFF = DO_OFF + kDkvRingDO * TILE;  // -lse2 x 128 | -D x 128
   // the RoPE tiles of the epilogue, loaded into the dO ring once the last dV is done
   static constexpr uint32_t COS_OFF = DO_OFF, SIN_OFF = DO_OFF + TILE;
   static constexpr uint32_t RED_OFF = STAT_OFF;  // epilogue only, after the last step's stats
+  // epilogue only, once no product reads the Q ring: the dV and dK tiles
+  static constexpr uint32_t DV_OFF = Q_OFF, DK_OFF = Q_OFF + TILE;
   static constexpr uint32_t BAR_OFF = STAT_OFF + 2 * 128 * 4;
   static constexpr uint32_t BYTES = BAR_OFF + 256 + 1024;
   static_assert(TILE % 1024 == 0 && BYTES <= 232448, "");
@@ -1162,42 +1195,39 @@ struct DkvBars {
   uint64_t q_full[kDkvRingQ], q_empty[kDkvRingQ], do_full[kDkvRingDO], do_empty[kDkvRingDO];
   uint64_t stat_full, stat_empty;
   uint64_t s_full, dp_full, p_ready, ds_ready;
-  uint64_t acc_full, epi_full, done, done2;
+  uint64_t acc_full, epi_full, done;
   uint32_t tmem_base;
   int abort;
 };
 }  // namespace
 
 // dK, dV for 128 keys of one (batch, kv head), looping over 128-query tiles
-// of every query head of its group (all products M = 128, N = 128).  Warp 1
-// issues S^T_j = K Q_j^T, then dV += P^T_j dO_j once the threads have written
-// P^T_j; warp 10 issues dP^T_j = V dO_j^T, then dK += dS^T_j Q_j once they
-// have written dS^T_j.  Compute thread (key row, half) handles queries
-// [64*half, 64*half + 64) of each tile: it writes bf16 P^T over the first 32
-// of its 64 S^T columns and bf16 dS^T over the first 32 of its dP^T columns
-// (the TMEM A operands of the dV and dK products; 16-query step k at column
-// 64*(k/4) + 8*(k%4)).  The next S^T (dP^T) is issued by the same warp after
-// the dV (dK) product that reads those columns, so in order.  While the
-// threads turn S^T_j into P^T_j the tensor core runs dK_{j-1} and dP^T_j;
-// while they form dS^T_j it runs dV_j and S^T_{j+1}.  Warp 0 loads K and V
-// once and runs the Q and dO rings (a Q tile is read by S^T_j and, a step
-// later, by dK_j, so its ring has a third slot); warp 11 stages lse and D of
-// each step's queries in shared memory, loading the next step's while the
+// of every query head of its group (all products M = 128, N = 128): S^T_j =
+// K Q_j^T, dP^T_j = V dO_j^T, dV += P^T_j dO_j, dK += dS^T_j Q_j, all issued by
+// warp 1.  Compute thread (key row, half) handles queries [64*half, 64*half +
+// 64) of each tile: it writes bf16 P^T over the first 32 of its 64 S^T columns
+// and bf16 dS^T over the first 32 of its dP^T columns (the TMEM A operands of
+// the dV and dK products; 16-query step k at column 64*(k/4) + 8*(k%4)).
+// While the threads turn S^T_j into P^T_j the tensor core runs dK_{j-1} and
+// dP^T_j; while they form dS^T_j it runs dV_j and S^T_{j+1}.  Warp 0 loads K
+// and V once and runs the Q and dO rings (a Q tile is read by S^T_j and, a
+// step later, by dK_j, so its ring has a third slot); warp 10 stages lse and D
+// of each step's queries in shared memory, loading the next step's while the
 // threads use the current one.  TMEM: S^T at column 0, dP^T at 128, dV at
 // 256, dK at 384.  The K tile in shared memory doubles as the y of the norm
 // backward; the RoPE tables of its 128 positions are loaded into the dO ring
 // after the last dV.
 template <int HD>
-__global__ void __launch_bounds__(kDkvThreads, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     attn_dkv_tc_kernel(const __grid_constant__ CUtensorMap map_k128,
                        const __grid_constant__ CUtensorMap map_v128,
                        const __grid_constant__ CUtensorMap map_q128,
                        const __grid_constant__ CUtensorMap map_do128,
                        const __grid_constant__ CUtensorMap map_cos,
                        const __grid_constant__ CUtensorMap map_sin,
+                       const __grid_constant__ CUtensorMap map_out,
                        const float* __restrict__ lse,
-                       const float* __restrict__ D, const float* __restrict__ rk,
-                       __nv_bfloat16* __restrict__ dqkv, int64_t ldq, int H, int Hkv, int T,
+                       const float* __restrict__ D, const float* __restrict__ rk, int H, int Hkv, int T,
                        int W, float scale, float scale_log2, int qk_norm, int32_t* status) {
   using S = DkvSmem<HD>;
   constexpr int NCH = HD / 64;
@@ -1222,11 +1252,11 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
     tc::mbar_init(&bars->fixed_full, 1);
     for (int s = 0; s < kDkvRingQ; ++s) {
       tc::mbar_init(&bars->q_full[s], 1);
-      tc::mbar_init(&bars->q_empty[s], 2);  // after S^T and dV (warp 1) and dK (warp 10)
+      tc::mbar_init(&bars->q_empty[s], 1);
     }
     for (int s = 0; s < kDkvRingDO; ++s) {
       tc::mbar_init(&bars->do_full[s], 1);
-      tc::mbar_init(&bars->do_empty[s], 2);
+      tc::mbar_init(&bars->do_empty[s], 1);
     }
     tc::mbar_init(&bars->stat_full, 32);
     tc::mbar_init(&bars->stat_empty, 256);
@@ -1234,10 +1264,9 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
     tc::mbar_init(&bars->dp_full, 1);
     tc::mbar_init(&bars->p_ready, 256);
     tc::mbar_init(&bars->ds_ready, 256);
-    tc::mbar_init(&bars->acc_full, 2);
+    tc::mbar_init(&bars->acc_full, 1);
     tc::mbar_init(&bars->epi_full, 1);
     tc::mbar_init(&bars->done, 1);
-    tc::mbar_init(&bars->done2, 1);
   })
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort = &bars->abort;
@@ -1303,8 +1332,8 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
           if (issued >> s & 1) tc::mbar_wait_bounded(&full[s], (last_par >> s) & 1, nullptr, kWaitNs);
       }
     }
-  } else if (warp == 11) {
-    // lse2 and D of step j's queries (4 per lane), loaded before the wait for
+  } else if (warp == 10) {
+    // -lse2 and -D of step j's queries (4 per lane), loaded before the wait for
     // the threads to be done with step j-1's
     float* stat = reinterpret_cast<float*>(smem + S::STAT_OFF);
     for (int j = 0; j < n_steps; ++j) {
@@ -1315,8 +1344,8 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int qq = qs + lane * 4 + e;
-        l4[e] = qq < T ? lse[int64_t(bh) * T + qq] * kLog2e : 0.f;
-        d4[e] = qq < T ? D[int64_t(bh) * T + qq] : 0.f;
+        l4[e] = qq < T ? -lse[int64_t(bh) * T + qq] * kLog2e : 0.f;  // staged negated
+        d4[e] = qq < T ? -D[int64_t(bh) * T + qq] : 0.f;
       }
       if (!tc::mbar_wait_warp(&bars->stat_empty, (j & 1) ^ 1, abort, kWaitNs)) {
         if (lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 34);
@@ -1327,62 +1356,87 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
       *reinterpret_cast<float4*>(stat + 128 + lane * 4) = make_float4(d4[0], d4[1], d4[2], d4[3]);
       tc::mbar_arrive(&bars->stat_full);
     }
-  } else if (warp == 1 || warp == 10) {
-    // warp 1: S^T = K Q^T, then dV += P^T dO;  warp 10: dP^T = V dO^T, then dK += dS^T Q
-    const bool is_s = warp == 1;
+  } else if (warp == 1) {
+    // The products in the order the step needs them: S^T_0 and dP^T_0 first;
+    // then per step dV_j (once P^T_j is written), S^T_{j+1} (over P^T_j's
+    // columns, so after dV_j), dK_j (once dS^T_j is written) and dP^T_{j+1}
+    // (over dS^T_j's columns, so after dK_j).  One issuing thread keeps that
+    // order on the tensor core: S^T_{j+1}, which the threads wait for next,
+    // never queues behind dK_j.
     constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, 128, false, false);
     constexpr uint32_t idesc_acc = tc::idesc_bf16_f32(128, HD, false, true);
-    const uint64_t fd = tc::smem_desc_sw128(tc::smem_u32(smem + (is_s ? S::K_OFF : S::V_OFF)), 16);
-    const uint32_t t_prod = is_s ? tmem : t_dp;  // S^T or dP^T; then P^T or dS^T over it
-    const uint32_t t_acc = is_s ? t_dv : t_dk;
-    uint64_t* prod_full = is_s ? &bars->s_full : &bars->dp_full;
-    uint64_t* a_ready = is_s ? &bars->p_ready : &bars->ds_ready;
-    bool ok = tc::mbar_wait_warp(&bars->fixed_full, 0, abort, kWaitNs);
-    bool issued_any = false;
-    for (int j = 0; ok && j < n_steps; ++j) {
-      const int sq = j % kDkvRingQ, sd = j % kDkvRingDO;
-      uint64_t* own_full = is_s ? &bars->q_full[sq] : &bars->do_full[sd];  // S^T reads Q, dP^T reads dO
-      const uint32_t own_par = is_s ? (j / kDkvRingQ) & 1 : (j / kDkvRingDO) & 1;
-      uint64_t* oth_full = is_s ? &bars->do_full[sd] : &bars->q_full[sq];  // dV reads dO, dK reads Q
-      const uint32_t oth_par = is_s ? (j / kDkvRingDO) & 1 : (j / kDkvRingQ) & 1;
-      uint8_t* own = smem + (is_s ? S::Q_OFF + sq * S::TILE : S::DO_OFF + sd * S::TILE);
-      uint8_t* oth = smem + (is_s ? S::DO_OFF + sd * S::TILE : S::Q_OFF + sq * S::TILE);
-      if (!tc::mbar_wait_warp(own_full, own_par, abort, kWaitNs)) { ok = false; break; }
-      tc::tc_fence_after();
-      const uint64_t rd = tc::smem_desc_sw128(tc::smem_u32(own), 16);
+    const uint64_t kd = tc::smem_desc_sw128(tc::smem_u32(smem + S::K_OFF), 16);
+    const uint64_t vd = tc::smem_desc_sw128(tc::smem_u32(smem + S::V_OFF), 16);
+    // X^T = F Y^T over HD (F: the fixed K or V tile, Y: a ring tile), into `t`
+    auto issue_prod = [&](uint32_t t, uint64_t fd, const uint8_t* y) {
+      const uint64_t rd = tc::smem_desc_sw128(tc::smem_u32(y), 16);
 #pragma unroll
       for (int k = 0; k < HD / 16; ++k) {
         const uint32_t off = (k >> 2) * CH + (k & 3) * 32;
-        tc::mma_bf16_ss_elect(t_prod, tc::desc_advance(fd, off), tc::desc_advance(rd, off), idesc_s, k != 0);
+        tc::mma_bf16_ss_elect(t, tc::desc_advance(fd, off), tc::desc_advance(rd, off), idesc_s, k != 0);
       }
-      issued_any = true;
-      tc::mma_commit_elect(prod_full);
-      if (!tc::mbar_wait_warp(a_ready, j & 1, abort, kWaitNs)) { ok = false; break; }
-      if (!tc::mbar_wait_warp(oth_full, oth_par, abort, kWaitNs)) { ok = false; break; }
-      tc::tc_fence_after();
-      const uint64_t bmn = tc::smem_desc_sw128(tc::smem_u32(oth), CH);
+    };
+    // acc += A^T B over the tile's 128 queries (A: bf16 pairs over `t`'s columns, B: a ring tile)
+    auto issue_acc = [&](uint32_t acc, uint32_t t, const uint8_t* bt, bool first) {
+      const uint64_t bmn = tc::smem_desc_sw128(tc::smem_u32(bt), CH);
 #pragma unroll
       for (int k = 0; k < 128 / 16; ++k)
-        tc::mma_bf16_ts_elect(t_acc, t_prod + 64 * (k >> 2) + 8 * (k & 3), tc::desc_advance(bmn, k * 2048),
-                              idesc_acc, (j | k) != 0);
-      tc::mma_commit_elect(&bars->q_empty[sq]);
-      tc::mma_commit_elect(&bars->do_empty[sd]);
+        tc::mma_bf16_ts_elect(acc, t + 64 * (k >> 2) + 8 * (k & 3), tc::desc_advance(bmn, k * 2048), idesc_acc,
+                              !(first && k == 0));
+    };
+    auto q_tile = [&](int j) { return smem + S::Q_OFF + (j % kDkvRingQ) * S::TILE; };
+    auto do_tile = [&](int j) { return smem + S::DO_OFF + (j % kDkvRingDO) * S::TILE; };
+    auto q_ready = [&](int j) { return tc::mbar_spin_warp(&bars->q_full[j % kDkvRingQ], (j / kDkvRingQ) & 1, abort, kWaitNs); };
+    auto do_ready = [&](int j) { return tc::mbar_spin_warp(&bars->do_full[j % kDkvRingDO], (j / kDkvRingDO) & 1, abort, kWaitNs); };
+    bool ok = tc::mbar_spin_warp(&bars->fixed_full, 0, abort, kWaitNs) && q_ready(0);
+    bool issued_any = false;
+    if (ok) {
+      tc::tc_fence_after();
+      issue_prod(tmem, kd, q_tile(0));
+      tc::mma_commit_elect(&bars->s_full);
+      issued_any = true;
+      ok = do_ready(0);
+    }
+    if (ok) {
+      tc::tc_fence_after();
+      issue_prod(t_dp, vd, do_tile(0));
+      tc::mma_commit_elect(&bars->dp_full);
+    }
+    for (int j = 0; ok && j < n_steps; ++j) {
+      if (!tc::mbar_spin_warp(&bars->p_ready, j & 1, abort, kWaitNs)) { ok = false; break; }
+      tc::tc_fence_after();
+      issue_acc(t_dv, tmem, do_tile(j), j == 0);           // dV += P^T_j dO_j
+      tc::mma_commit_elect(&bars->do_empty[j % kDkvRingDO]);  // dP^T_j and dV_j read dO_j
+      if (j + 1 < n_steps) {
+        if (!q_ready(j + 1)) { ok = false; break; }
+        tc::tc_fence_after();
+        issue_prod(tmem, kd, q_tile(j + 1));  // S^T_{j+1}
+        tc::mma_commit_elect(&bars->s_full);
+      }
+      if (!tc::mbar_spin_warp(&bars->ds_ready, j & 1, abort, kWaitNs)) { ok = false; break; }
+      tc::tc_fence_after();
+      issue_acc(t_dk, t_dp, q_tile(j), j == 0);            // dK += dS^T_j Q_j
+      tc::mma_commit_elect(&bars->q_empty[j % kDkvRingQ]);  // S^T_j and dK_j read Q_j
+      if (j + 1 < n_steps) {
+        if (!do_ready(j + 1)) { ok = false; break; }
+        tc::tc_fence_after();
+        issue_prod(t_dp, vd, do_tile(j + 1));  // dP^T_{j+1}
+        tc::mma_commit_elect(&bars->dp_full);
+      }
     }
     if (ok) tc::mma_commit_elect(&bars->acc_full);
     if (!ok) {
-      if (lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, is_s ? 31 : 33);
+      if (lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 31);
       *abort = 1;
     }
     if (issued_any) {
-      uint64_t* dn = is_s ? &bars->done : &bars->done2;
-      tc::mma_commit_elect(dn);
-      tc::mbar_wait_warp(dn, 0, nullptr, kWaitNs);
+      tc::mma_commit_elect(&bars->done);
+      tc::mbar_wait_warp(&bars->done, 0, nullptr, kWaitNs);
     }
   } else {
     const Roles R = roles();
     const int key = k0 + R.r;
     const bool kv = key < T;
-    const int tk = kv ? key : 0;
     // the key's visible queries [q_lo, q_hi): none for a row past T
     const int q_lo = key, q_hi = kv ? min(T, key + W) : key;
     const uint32_t ts = tmem + R.lane_off + R.half * 64;
@@ -1391,8 +1445,8 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
     bool ok = true;
     for (int j = 0; j < n_steps; ++j) {
       const int qs = (kt + j - (j / n_h) * n_h) * 128 + R.half * 64;
-      if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->stat_full, j & 1, abort, kWaitNs));
-      if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->s_full, j & 1, abort, kWaitNs));
+      if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_spin(&bars->stat_full, j & 1, abort, kWaitNs));
+      if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_spin(&bars->s_full, j & 1, abort, kWaitNs));
       const bool need_mask = qs < q_lo || qs + 64 > q_hi;
       float p[64];
       if (ok) {
@@ -1401,47 +1455,51 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
         tc::tmem_ld_32x32b_x32(ts, us0);
         tc::tmem_ld_32x32b_x32(ts + 32, us1);
         tc::tmem_wait_ld();
-        uint32_t pk[32];
-        if (need_mask)
-          p_col64<true>(us0, us1, stat, p, pk, scale_log2, qs, q_lo, q_hi);
-        else
-          p_col64<false>(us0, us1, stat, p, pk, scale_log2, qs, q_lo, q_hi);
-        tc::tmem_st_32x32b_x32(ts, pk);  // P^T over the first 32 of this thread's S^T columns
+        // P^T over the first 32 of this thread's S^T columns (all 64 S^T values are in registers)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t pk[16];
+          if (need_mask)
+            p_col32<true>(c ? us1 : us0, stat + 32 * c, p + 32 * c, pk, scale_log2, qs + 32 * c, q_lo, q_hi);
+          else
+            p_col32<false>(c ? us1 : us0, stat + 32 * c, p + 32 * c, pk, scale_log2, qs + 32 * c, q_lo, q_hi);
+          tc::tmem_st_32x32b_x16(ts + 16 * c, pk);
+        }
         tc::tmem_wait_st();
         tc::tc_fence_before();
       }
       tc::mbar_arrive(&bars->p_ready);
-      if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->dp_full, j & 1, abort, kWaitNs));
+      if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_spin(&bars->dp_full, j & 1, abort, kWaitNs));
       if (ok) {
         tc::tc_fence_after();
-        uint32_t pd[32];
+        // dS^T over the first 32 of this thread's dP^T columns: 16 of them per
+        // 32 queries, each written after those columns' dP values were loaded
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-          uint32_t up[32];
+          uint32_t up[32], pd[16];
           tc::tmem_ld_32x32b_x32(tp + 32 * c, up);
           tc::tmem_wait_ld();
 #pragma unroll
           for (int g = 0; g < 8; ++g) {
             const float4 d4 = *reinterpret_cast<const float4*>(stat + 128 + 32 * c + 4 * g);
-            const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
             for (int e = 0; e < 4; e += 2) {
               const int i = 4 * g + e;
               const float2 r = unf2(mul2(f2(p[32 * c + i], p[32 * c + i + 1]),
                                          add2(f2(__uint_as_float(up[i]), __uint_as_float(up[i + 1])),
-                                              f2(-dd[e], -dd[e + 1]))));
-              pd[16 * c + i / 2] = pack2(r.x, r.y);
+                                              e ? f2(d4.z, d4.w) : f2(d4.x, d4.y))));
+              pd[i / 2] = pack2(r.x, r.y);
             }
           }
+          tc::tmem_st_32x32b_x16(tp + 16 * c, pd);
         }
-        tc::tmem_st_32x32b_x32(tp, pd);  // dS^T over the first 32 of this thread's dP^T columns
         tc::tmem_wait_st();
         tc::tc_fence_before();
       }
       tc::mbar_arrive(&bars->stat_empty);  // this step's lse and D are no longer read
       tc::mbar_arrive(&bars->ds_ready);
     }
-    if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->acc_full, 0, abort, kWaitNs));
+    if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_spin(&bars->acc_full, 0, abort, kWaitNs));
     if (!ok) {
       if (R.lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 32);
       *abort = 1;
@@ -1449,22 +1507,19 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
       tc::tc_fence_after();
     }
     const int d = H * HD;
-    __nv_bfloat16* row = dqkv + (int64_t(b) * T + tk) * ldq;
-    if (ok) {  // dV: this thread's half of the columns
+    if (ok) {  // dV: this thread's half of the columns, into the dV tile
 #pragma unroll
       for (int c = 0; c < HD / 2; c += 32) {
         float v[32];
         tmem_ld<32>(t_dv + R.lane_off + R.half * (HD / 2) + c, v);
-        if (kv) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 8)
-            *reinterpret_cast<uint4*>(row + d + (Hkv + hk) * HD + R.half * (HD / 2) + c + i) =
-                make_uint4(pack2(v[i], v[i + 1]), pack2(v[i + 2], v[i + 3]), pack2(v[i + 4], v[i + 5]),
-                           pack2(v[i + 6], v[i + 7]));
-        }
+        for (int i = 0; i < 32; i += 8)
+          *reinterpret_cast<uint4*>(smem + S::DV_OFF + tile_unit(R.r, (R.half * (HD / 2) + c + i) / 8)) =
+              make_uint4(pack2(v[i], v[i + 1]), pack2(v[i + 2], v[i + 3]), pack2(v[i + 4], v[i + 5]),
+                         pack2(v[i + 6], v[i + 7]));
       }
     }
-    if (ok && !__all_sync(0xffffffffu, tc::mbar_wait_bounded(&bars->epi_full, 0, abort, kWaitNs))) {
+    if (ok && !__all_sync(0xffffffffu, tc::mbar_wait_spin(&bars->epi_full, 0, abort, kWaitNs))) {
       if (R.lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 36);
       *abort = 1;
       ok = false;
@@ -1472,8 +1527,11 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
     // the stats region is free once every step is done (acc_full): it holds red
     norm_rope_bwd_half<HD>(t_dk + R.lane_off, R.half, R.r, scale, smem + S::K_OFF,
                            kv ? rk[int64_t(bkv) * T + key] : 0.f, qk_norm, smem + S::COS_OFF,
-                           smem + S::SIN_OFF, row + d + hk * HD, ok, kv,
+                           smem + S::SIN_OFF, smem + S::DK_OFF, ok, kv,
                            reinterpret_cast<float*>(smem + S::RED_OFF));
+    uint8_t* const tiles[2] = {smem + S::DV_OFF, smem + S::DK_OFF};
+    const int cols[2] = {d + (Hkv + hk) * HD, d + hk * HD};
+    store_tiles<HD>(&map_out, tiles, cols, 2, k0, b, ok);
   }
   ATTN_EPILOGUE(tmem)
 }
@@ -1491,11 +1549,11 @@ int attn_bwd_tc_t(const gpt_config& c, const void* q, const void* k, const void*
   const int64_t N = int64_t(B) * T;
   attn_rowdot_kernel<<<ceil_div(N * H * (HD / 8), 256), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(dO), static_cast<const __nv_bfloat16*>(o), Dbuf, N, H, T, HD);
-  CUtensorMap k128, v128, q128, do128, mcos, msin;
+  CUtensorMap k128, v128, q128, do128, mcos, msin, mout;
   const bool ok = tile_map(&k128, k, kv_rows, HD, HD, 128) && tile_map(&v128, v, kv_rows, HD, HD, 128) &&
                   tile_map(&q128, q, rows, HD, HD, 128) && tile_map(&do128, dO, ntok, d, d, 128) &&
                   tile_map_f32(&mcos, cos_t, T, HD / 2, HD / 2, 128) &&
-                  tile_map_f32(&msin, sin_t, T, HD / 2, HD / 2, 128);
+                  tile_map_f32(&msin, sin_t, T, HD / 2, HD / 2, 128) && seq_map(&mout, dqkv, B, T, ldq);
   if (!ok) return 1;
   const float scale = 1.f / sqrtf(float(HD));
   const float scale_log2 = scale * kLog2e;
@@ -1504,16 +1562,14 @@ int attn_bwd_tc_t(const gpt_config& c, const void* q, const void* k, const void*
   const int smem_q = int(DqSmem<HD>::BYTES);
   if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_q) != cudaSuccess)
     return 1;
-  kq<<<nt * B * H, kThreads, smem_q, st>>>(q128, do128, k128, v128, mcos, msin, lse, Dbuf, rq,
-                                           static_cast<__nv_bfloat16*>(dqkv), ldq, H, Hkv, T, W,
-                                           scale, scale_log2, c.qk_norm, status);
+  kq<<<nt * B * H, kThreads, smem_q, st>>>(q128, do128, k128, v128, mcos, msin, mout, lse, Dbuf, rq, H,
+                                           Hkv, T, W, scale, scale_log2, c.qk_norm, status);
   auto kk = attn_dkv_tc_kernel<HD>;
   const int smem_k = int(DkvSmem<HD>::BYTES);
   if (cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_k) != cudaSuccess)
     return 1;
-  kk<<<nt * B * Hkv, kDkvThreads, smem_k, st>>>(k128, v128, q128, do128, mcos, msin, lse, Dbuf, rk,
-                                             static_cast<__nv_bfloat16*>(dqkv), ldq, H, Hkv, T, W,
-                                             scale, scale_log2, c.qk_norm, status);
+  kk<<<nt * B * Hkv, kThreads, smem_k, st>>>(k128, v128, q128, do128, mcos, msin, mout, lse, Dbuf, rk, H,
+                                                Hkv, T, W, scale, scale_log2, c.qk_norm, status);
   return last_launch_rc();
 }
 }  // namespace

@@ -64,6 +64,38 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
   return ok != 0;
 }
 
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// As mbar_wait_bounded, but polling with test_wait instead of sleeping in
+// try_wait: a thread suspended in try_wait was measured to resume on the order
+// of a thousand cycles after the phase completed, which a wait on the critical
+// path of a pipeline (an MMA issuer waiting for its operands, the threads
+// waiting for an MMA result) cannot afford.  The poll takes issue slots, so it
+// is for waits that are short or that no other warp of the scheduler needs.
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                               uint64_t limit_ns) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((it & 63) == 63) {
+      if (abort && *abort) return false;
+      if (global_timer_ns() - t0 > limit_ns) return false;
+    }
+  }
+}
+
 // Wait until the phase with the given parity has completed.  Gives up after
 // `limit_ns` nanoseconds (or early once *abort is set by another role, when
 // `abort` is not null), returning false; the caller then records
@@ -83,6 +115,23 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
 }
 
 // ---- TMA --------------------------------------------------------------------
+// Generic-proxy shared-memory writes made visible to the async proxy (a TMA
+// store that reads them); each writing thread fences before the barrier that
+// precedes the store.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Tiled store of a shared-memory box to global coordinates (x, y, z) of a 3-D
+// tensor map; boxes past the tensor's bounds are clipped.  Completion is
+// tracked by bulk groups: commit, then wait before the source is reused.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// every committed group has finished reading its shared-memory source
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -332,6 +381,10 @@ __device__ __forceinline__ void mma_commit_pair_elect(uint32_t bar_cluster_addr)
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort,
                                                uint64_t limit_ns) {
   return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, abort, limit_ns));
+}
+__device__ __forceinline__ bool mbar_spin_warp(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                               uint64_t limit_ns) {
+  return __all_sync(0xffffffffu, mbar_wait_spin(bar, parity, abort, limit_ns));
 }
 
 // Shared-memory matrix descriptor (tcgen05 format), 128-byte swizzle.
