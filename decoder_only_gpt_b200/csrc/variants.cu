@@ -16,9 +16,26 @@
 namespace gpt {
 namespace {
 
-constexpr int kRedBlocks = 296;  // fixed grid of the deterministic flat dot products
+// fixed grid of the deterministic flat dot products: 8 blocks of 256 threads
+// per SM, enough warps in flight to keep HBM busy
+constexpr int kRedBlocks = 148 * 8;
 
 __device__ __forceinline__ float sigmoidf_(float z) { return 1.f / (1.f + __expf(-z)); }
+
+// four consecutive elements of T, as one 8- (bf16) or 16-byte (fp32) access
+__device__ __forceinline__ float4 load4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+__device__ __forceinline__ void store4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+__device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
+  const __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+  *reinterpret_cast<uint2*>(p) =
+      make_uint2(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b));
+}
 
 template <typename T>
 __device__ __forceinline__ void store_acc(T* out, float v, int accumulate) {
@@ -94,7 +111,14 @@ __global__ void ve_fwd_kernel(const T* __restrict__ h, const T* __restrict__ wg,
   const T* row = ve + int64_t(id) * Hkv * hd + hk * hd;
   const int64_t b = t / Tlen, tt = t % Tlen;
   T* vr = v + ((b * Hkv + hk) * Tlen + tt) * hd;
-  for (int i = lane; i < hd; i += 32) vr[i] = from_f<T>(to_f(vr[i]) + gate * to_f(row[i]));
+  if ((hd & 3) == 0) {
+    for (int i = 4 * lane; i < hd; i += 128) {
+      const float4 a = load4(vr + i), e = load4(row + i);
+      store4(vr + i, make_float4(a.x + gate * e.x, a.y + gate * e.y, a.z + gate * e.z, a.w + gate * e.w));
+    }
+  } else {
+    for (int i = lane; i < hd; i += 32) vr[i] = from_f<T>(to_f(vr[i]) + gate * to_f(row[i]));
+  }
 }
 
 // Value embedding, backward: warp per (token, key/value head).  dv is the v
@@ -121,10 +145,18 @@ __global__ void ve_bwd_kernel(const T* __restrict__ dqkv, int64_t ldq, int64_t v
   const T* dv = dqkv + t * ldq + v_col0 + hk * hd;
   float* out = rows + (t * Hkv + hk) * hd;
   float s = 0.f;
-  for (int i = lane; i < hd; i += 32) {
-    const float g = to_f(dv[i]);
-    s += g * to_f(row[i]);
-    out[i] = gate * g;
+  if ((hd & 3) == 0 && (ldq & 3) == 0 && (v_col0 & 3) == 0) {
+    for (int i = 4 * lane; i < hd; i += 128) {
+      const float4 g = load4(dv + i), e = load4(row + i);
+      s += g.x * e.x + g.y * e.y + g.z * e.z + g.w * e.w;
+      store4(out + i, make_float4(gate * g.x, gate * g.y, gate * g.z, gate * g.w));
+    }
+  } else {
+    for (int i = lane; i < hd; i += 32) {
+      const float g = to_f(dv[i]);
+      s += g * to_f(row[i]);
+      out[i] = gate * g;
+    }
   }
   s = warp_sum(s);
   if (lane == 0) dgz[item] = s * 3.f * sg * (1.f - sg);
@@ -224,8 +256,7 @@ __global__ void resid_bwd_kernel(float* __restrict__ dx, T* __restrict__ dxs, co
       g.x *= a; g.y *= a; g.z *= a; g.w *= a;
     }
     reinterpret_cast<float4*>(dx)[i] = g;
-    T* o = dxs + 4 * i;
-    o[0] = from_f<T>(g.x); o[1] = from_f<T>(g.y); o[2] = from_f<T>(g.z); o[3] = from_f<T>(g.w);
+    store4(dxs + 4 * i, g);
   }
   if (!lam) return;
   __shared__ float red[2][32];
