@@ -41,10 +41,11 @@ Where the pages are silent the plainest reading is taken:
 * MLP u = h W_up^T, a = max(u, 0)^2, y = a W_down^T (not gated);
 * loss = mean over all B*T positions of logsumexp(z) - z[target].
 
-FP8 forward (``fp8``; the page's training command line has an ``--fp8`` flag
-and names no scaling recipe).  Reading taken: the four block projections
-(W_qkv, W_o, W_up, W_down) multiply e4m3 operands in the forward; the
-embedding, lm_head and the whole backward stay as above.
+FP8 (``fp8``; the page's training command line has an ``--fp8`` flag and
+names no scaling recipe).  Reading taken: the four block projections (W_qkv,
+W_o, W_up, W_down) multiply e4m3 operands in the forward and in their data
+gradients dX = dY W; the embedding, lm_head and every weight gradient stay as
+above.
 
 * quantizer input: the operand as the bf16 value the GPU stores (activations
   rounded to bf16 here, weights are bf16 already) -- the same precision in
@@ -55,9 +56,12 @@ embedding, lm_head and the whole backward stay as above.
 * code: round to the nearest e4m3 value (OCP E4M3: 4 exponent bits, bias 7,
   3 mantissa bits, subnormals, no infinities), ties to the even code;
 * product: the dequantized operands multiplied exactly (fp64 here);
-* backward: the bf16 model's backward evaluated at the FP8 forward's
-  activations (dX = dY W and dW = dY^T X with the unquantized W and X), i.e.
-  the quantizer is taken as the identity (straight-through).
+* data gradient: dX = dY W with dY through e4m3 exactly as an activation
+  (rounded to bf16, one power-of-two scale per row, i.e. per token) and W
+  through the forward's per-tensor codes;
+* weight gradient: dW = dY^T X with the unquantized dY and X (the bf16
+  model's, at the FP8 forward's activations), i.e. the quantizer taken as the
+  identity there (straight-through).
 
 Block variants (section "1. GPT Modeli": the "Deger Gommeleri (ResFormer)"
 and "Verimlilik Puf Noktalari" listings).  The page prints each as a line or
@@ -360,6 +364,14 @@ def _linear(cfg: "OracleConfig", x: np.ndarray, w: np.ndarray,
     return fp8_rows(x) @ (fp8_tensor(w) if w_fp8 is None else w_fp8).T
 
 
+def _dgrad(dy: np.ndarray, w: np.ndarray, w_fp8: Optional[np.ndarray]) -> np.ndarray:
+    """The data gradient of one block projection y = x W^T: dy W, or with
+    fp8 (w_fp8: W through e4m3) dy through e4m3 per row times w_fp8."""
+    if w_fp8 is None:
+        return dy @ w
+    return fp8_rows(dy) @ w_fp8
+
+
 def fp8_weights(cfg: "OracleConfig", params: Dict[str, np.ndarray]) -> Optional[Dict[str, np.ndarray]]:
     """Every block matrix through e4m3 (fp8 configs; None otherwise): the
     same for every sequence of a step, so computed once per step."""
@@ -469,8 +481,10 @@ def sequence_forward(cfg: OracleConfig, params: Dict[str, np.ndarray],
 
 
 def sequence_backward(cfg: OracleConfig, params: Dict[str, np.ndarray], cache: dict,
-                      scale: float, grads: Dict[str, np.ndarray]) -> None:
-    """Accumulate d(scale * sum_t loss_t)/d(params) into ``grads``."""
+                      scale: float, grads: Dict[str, np.ndarray],
+                      w_fp8: Optional[Dict[str, np.ndarray]] = None) -> None:
+    """Accumulate d(scale * sum_t loss_t)/d(params) into ``grads``; with fp8,
+    ``w_fp8`` holds the block matrices through e4m3 (``fp8_weights``)."""
     tok, tgt = cache["tok"], cache["tgt"]
     T = tok.shape[0]
     d, H, hd, Hkv = cfg.d_model, cfg.n_head, cfg.head_dim, cfg.kv_heads
@@ -487,19 +501,22 @@ def sequence_backward(cfg: OracleConfig, params: Dict[str, np.ndarray], cache: d
         grads["scalars"][0, 1] -= np.sum(dx_final * cache["x_b"])
     dx0 = np.zeros_like(dx)                              # residual scaling's x0 term
 
+    if cfg.fp8 and w_fp8 is None:
+        w_fp8 = fp8_weights(cfg, params)
+    wq = (lambda name: w_fp8[name]) if cfg.fp8 else (lambda name: None)
     for l in reversed(range(cfg.n_layer)):
         wqkv, wo, wup, wdown = _layer_params(params, l)
         c = cache["layers"][l]
         # x_out = x_mid + a W_down^T
         grads[f"layers.{l}.wdown"] += dx.T @ c["a"]
-        da = dx @ wdown
+        da = _dgrad(dx, wdown, wq(f"layers.{l}.wdown"))
         du = da * 2.0 * np.maximum(c["u"], 0.0)
         grads[f"layers.{l}.wup"] += du.T @ c["h2"]
-        dh2 = du @ wup
+        dh2 = _dgrad(du, wup, wq(f"layers.{l}.wup"))
         dx = dx + rms_norm_backward(dh2, c["h2"], c["r2"])
         # x_mid = x_in + o W_o^T
         grads[f"layers.{l}.wo"] += dx.T @ c["o"]
-        do = (dx @ wo).reshape(T, H, hd)
+        do = _dgrad(dx, wo, wq(f"layers.{l}.wo")).reshape(T, H, hd)
         _, p, _ = causal_attention(c["qn"], c["kn"], c["v"], cfg.window)
         dqn, dkn, dv = causal_attention_backward(do, c["qn"], c["kn"], c["v"], p)
         dh_ve = None
@@ -522,7 +539,7 @@ def sequence_backward(cfg: OracleConfig, params: Dict[str, np.ndarray], cache: d
         dqkv = np.concatenate([dq.reshape(T, d), dk.reshape(T, Hkv * hd), dv.reshape(T, Hkv * hd)],
                               axis=1)
         grads[f"layers.{l}.wqkv"] += dqkv.T @ c["h"]
-        dh = dqkv @ wqkv
+        dh = _dgrad(dqkv, wqkv, wq(f"layers.{l}.wqkv"))
         if dh_ve is not None:
             dh = dh + dh_ve
         dx = dx + rms_norm_backward(dh, c["h"], c["r1"])
@@ -587,7 +604,7 @@ def step(cfg: OracleConfig, params: Dict[str, np.ndarray], tokens: np.ndarray,
         cache = sequence_forward(cfg, params, tokens[b], targets[b], w_fp8)
         token_loss[i] = cache["token_loss"]
         if backward:
-            sequence_backward(cfg, params, cache, 1.0 / denom, grads)
+            sequence_backward(cfg, params, cache, 1.0 / denom, grads, w_fp8)
         if keep_caches:
             caches.append(cache)
     loss = float(np.sum(token_loss) / denom)

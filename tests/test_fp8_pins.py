@@ -1,4 +1,4 @@
-"""Pins for the oracle's FP8 (e4m3) forward projections.
+"""Pins for the oracle's FP8 (e4m3) block projections: forward and data gradient.
 
 Facts fixed outside the oracle's code:
 
@@ -7,10 +7,13 @@ Facts fixed outside the oracle's code:
 * the power-of-two scale: amax * 2^k <= 448 < amax * 2^(k+1);
 * operands already on the scaled e4m3 grid pass through exactly;
 * the product's error stays inside the bound two e4m3 roundings allow;
+* the data gradient dY W with dY through e4m3 per row: exact for operands on
+  the grid, inside the two-rounding bound otherwise;
 * the whole step (multi-head, and grouped-query with a window) against torch
   float64 autograd in which each block projection quantizes through torch's
-  bf16 and float8 casts with a log2-derived exponent, the straight-through
-  backward written as its own autograd function.
+  bf16 and float8 casts with a log2-derived exponent, its backward written as
+  its own autograd function (dY through the same casts for dX = dY W, the
+  unquantized dY and X for dW).
 """
 import math
 
@@ -84,6 +87,35 @@ def test_fp8_linear_error_bound():
     assert np.abs(got - exact).max() > 0
 
 
+def test_fp8_dgrad_exact_on_grid():
+    rng = np.random.default_rng(15)
+    vals, _ = go._e4m3_table()
+    grid = np.concatenate([vals, -vals])
+    dy = rng.choice(grid, (7, 24))
+    dy[:, 3] = -448.0                                 # row amax 448 * 2^-11 after scaling
+    dy = dy * 2.0 ** -11
+    w = rng.choice(grid, (24, 40))
+    w[5, 1] = 448.0
+    w = w * 2.0 ** 2
+    assert np.array_equal(go._dgrad(dy, w, go.fp8_tensor(w)), dy @ w)
+    assert np.array_equal(go._dgrad(dy, w, None), dy @ w)
+
+
+def test_fp8_dgrad_error_bound():
+    rng = np.random.default_rng(17)
+    dy = go._round_bf16(rng.standard_normal((12, 200)) * 1e-4)
+    w = go._round_bf16(rng.standard_normal((200, 96)) * 0.02)
+    got = go._dgrad(dy, w, go.fp8_tensor(w))
+    exact = dy @ w
+    ky = go.pow2_exponent(np.abs(dy).max(1))[:, None]
+    kw = go.pow2_exponent(np.abs(w).max())
+    ey = np.maximum(np.abs(dy) * 2.0 ** -4, np.ldexp(2.0 ** -10, -ky))
+    ew = np.maximum(np.abs(w) * 2.0 ** -4, np.ldexp(2.0 ** -10, -kw))
+    bound = np.abs(dy) @ ew + ey @ np.abs(w) + ey @ ew
+    assert np.all(np.abs(got - exact) <= bound * (1 + 1e-12))
+    assert np.abs(got - exact).max() > 0
+
+
 def _torch_fp8_step(w, params, tok, tgt):
     import torch.nn.functional as F
 
@@ -100,15 +132,16 @@ def _torch_fp8_step(w, params, tok, tgt):
     class Fp8Linear(torch.autograd.Function):
         @staticmethod
         def forward(ctx, x, W):
-            ctx.save_for_backward(x, W)
             xq = q(x.reshape(-1, x.shape[-1])).reshape(x.shape)
             wq = q(W.reshape(1, -1)).reshape(W.shape)          # one scale per tensor
+            ctx.save_for_backward(x, wq)
             return xq @ wq.T
 
         @staticmethod
         def backward(ctx, g):
-            x, W = ctx.saved_tensors
-            return g @ W, (g.reshape(-1, g.shape[-1]).T @ x.reshape(-1, x.shape[-1]))
+            x, wq = ctx.saved_tensors
+            gq = q(g.reshape(-1, g.shape[-1])).reshape(g.shape)  # one scale per token
+            return gq @ wq, (g.reshape(-1, g.shape[-1]).T @ x.reshape(-1, x.shape[-1]))
 
     t = {k: torch.tensor(v, dtype=torch.float64, requires_grad=True) for k, v in params.items()}
     B, T = tok.shape
