@@ -165,10 +165,11 @@ bool make_layout(const gpt_config& c, Layout* L) {
     L->w8 = b.take(uint64_t(c.param_bytes / 2));
     L->w8_deq = b.take(4 * uint64_t(c.n_layer) * 4);
     L->w8_amax = b.take(4 * uint64_t(c.n_layer) * 4);
-    L->a8 = b.take(N * std::max(d, F));
+    L->w8t = b.take(uint64_t(c.param_bytes / 2));
+    L->a8 = b.take(N * std::max(std::max(d, F), int64_t(qkv_cols(c))));
     L->a8_deq = b.take(N * 4);
   } else {
-    L->w8 = L->w8_deq = L->w8_amax = L->a8 = L->a8_deq = 0;
+    L->w8 = L->w8_deq = L->w8_amax = L->w8t = L->a8 = L->a8_deq = 0;
   }
   // block variants
   {
@@ -457,6 +458,44 @@ struct Step {
     }
     return 0;
   }
+  // fp8 configs: the codes of every block matrix's transpose, for the data
+  // gradients, with the scales the forward's quant_weights found
+  int quant_weights_t() {
+    for (int kind = 0; kind < 4; ++kind) {
+      const int tensor = GPT_T_WQKV + kind;
+      int64_t off0, r, cc, off1 = 0;
+      gpt_param_offset(c, tensor, 0, &off0, &r, &cc);
+      if (c->n_layer > 1) gpt_param_offset(c, tensor, 1, &off1, &r, &cc);
+      const int64_t stride = c->n_layer > 1 ? off1 - off0 : 0;
+      TraceScope ts(GPT_K_QUANT, 1, 0, double(c->n_layer) * r * cc * 3, st);
+      const int rc = launch_quant_tensors_t(p + off0 * esz, int(r), int(cc), stride, c->n_layer, 
+                                            reinterpret_cast<unsigned*>(ws + L.w8_amax) + kind * c->n_layer,
+                                            ws + L.w8t + off0, st);
+      if (rc) return rc;
+    }
+    return 0;
+  }
+  // the data gradient dX = dY W of block matrix `tensor` of layer l, given as
+  // the bf16 GEMM (A = dY [N, K] K-major, B = W as the MN-major [K, N]); fp8
+  // configs quantize dY per row and multiply it with the codes of W^T
+  int dgrad(GemmArgs g, int tensor, int l) {
+    if (!c->fp8) return run_gemm(*c, g, st);
+    {
+      TraceScope ts(GPT_K_QUANT, 1, 0, double(N) * g.K * 3 + N * 4.0, st);
+      const int rc = launch_quant_rows(g.A, N, g.K, ws + L.a8, f(L.a8_deq), st);
+      if (rc) return rc;
+    }
+    int64_t off, r, cc;
+    gpt_param_offset(c, tensor, l, &off, &r, &cc);
+    g.A = ws + L.a8;
+    g.B = ws + L.w8t + off;
+    g.lda = g.ldb = g.K;
+    g.b_mn_major = false;
+    g.fp8 = true;
+    g.a_row_scale = f(L.a8_deq);
+    g.b_scale = f(L.w8_deq) + (tensor - GPT_T_WQKV) * c->n_layer + l;
+    return run_gemm(*c, g, st);
+  }
   // fp8 configs: one block projection of the bf16 activation `xact` [N, K]:
   // quantize it per row into the scratch codes, then the e4m3 GEMM against the
   // weight's codes; otherwise the bf16 GEMM as given
@@ -642,6 +681,7 @@ static int backward_impl(const gpt_config* c, const int32_t* tok, const int32_t*
     TraceScope ts(GPT_K_SORT, 8, 0, double(N) * 12 + double(V) * 16, st);
     GPT_TRY(launch_sort_tokens(*c, L, tok, ws, st));
   }
+  if (c->fp8 && c->n_layer > 0) GPT_TRY(S.quant_weights_t());
   // logits gradient G = (softmax(z) - onehot(target)) / N, recomputed from the saved lse
   GemmArgs g = gemm_kk(ws + L.hf, d, S.param(GPT_T_LM_HEAD, 0), d, N, int(L.vpad), d,
                        EPI_CE_BWD, ws + L.G, L.vpad, status);
@@ -677,7 +717,7 @@ static int backward_impl(const gpt_config* c, const int32_t* tok, const int32_t*
     g = gemm_kk(ws + L.dxs, d, S.param(GPT_T_WDOWN, l), F, N, F, d, EPI_DRELU2, ws + L.du, F,
                 status);
     g.b_mn_major = true; g.aux = Lb + L.lo.a;
-    GPT_TRY(run_gemm(*c, g, st));
+    GPT_TRY(S.dgrad(g, GPT_T_WDOWN, l));
     g = gemm_kk(ws + L.dxs, d, Lb + L.lo.a, F, d, F, N, EPI_STORE, grad(GPT_T_WDOWN, l), F,
                 status);
     g.a_mn_major = true; g.b_mn_major = true; g.beta = accumulate;
@@ -685,7 +725,7 @@ static int backward_impl(const gpt_config* c, const int32_t* tok, const int32_t*
     // MLP up
     g = gemm_kk(ws + L.du, F, S.param(GPT_T_WUP, l), d, N, d, F, EPI_STORE, ws + L.dh, d, status);
     g.b_mn_major = true;
-    GPT_TRY(run_gemm(*c, g, st));
+    GPT_TRY(S.dgrad(g, GPT_T_WUP, l));
     g = gemm_kk(ws + L.du, F, Lb + L.lo.h2, d, F, d, N, EPI_STORE, grad(GPT_T_WUP, l), d, status);
     g.a_mn_major = true; g.b_mn_major = true; g.beta = accumulate;
     GPT_TRY(run_gemm(*c, with_splitk(g, L, ws), st));
@@ -693,7 +733,7 @@ static int backward_impl(const gpt_config* c, const int32_t* tok, const int32_t*
     // attention out-projection
     g = gemm_kk(ws + L.dxs, d, S.param(GPT_T_WO, l), d, N, d, d, EPI_STORE, ws + L.dO, d, status);
     g.b_mn_major = true;
-    GPT_TRY(run_gemm(*c, g, st));
+    GPT_TRY(S.dgrad(g, GPT_T_WO, l));
     g = gemm_kk(ws + L.dxs, d, Lb + L.lo.o, d, d, d, N, EPI_STORE, grad(GPT_T_WO, l), d, status);
     g.a_mn_major = true; g.b_mn_major = true; g.beta = accumulate;
     GPT_TRY(run_gemm(*c, with_splitk(g, L, ws), st));
@@ -720,7 +760,7 @@ static int backward_impl(const gpt_config* c, const int32_t* tok, const int32_t*
     g = gemm_kk(ws + L.dqkv, Qc, S.param(GPT_T_WQKV, l), d, N, d, Qc, EPI_STORE, ws + L.dh,
                 d, status);
     g.b_mn_major = true;
-    GPT_TRY(run_gemm(*c, g, st));
+    GPT_TRY(S.dgrad(g, GPT_T_WQKV, l));
     if (ve) {  // the gate's input h[:, :C]
       TraceScope ts(GPT_K_OTHER, 1, 0, double(N) * c->ve_gate_channels * esz * 2, st);
       GPT_TRY(launch_ve_dh(*c, ws + L.dh, S.f(L.ve_dgz), S.param(GPT_T_VE_GATE, l), st));

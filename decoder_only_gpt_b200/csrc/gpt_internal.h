@@ -139,11 +139,12 @@ struct Layout {
   // sum-of-squares partials
   uint64_t opt_x0, opt_x1, opt_a, opt_b, opt_part;
   uint64_t opt_rows;       // NorMuon per-row scratch: v_mean and factors [2][max rows]
-  // e4m3 forward projections (fp8 configs): weight codes at the parameter
+  // e4m3 block projections (fp8 configs): weight codes at the parameter
   // buffer's element offsets (one byte each), their dequantization factors
-  // and amax bits [4 kinds][n_layer], one activation's codes [N, max(d, F)]
-  // and its per-row factors [N]
-  uint64_t w8, w8_deq, w8_amax, a8, a8_deq;
+  // and amax bits [4 kinds][n_layer], the codes of each W^T at the same
+  // offsets (for the data gradients), one activation's or output gradient's
+  // codes [N, max(d, F, q|k|v columns)] and its per-row factors [N]
+  uint64_t w8, w8_deq, w8_amax, w8t, a8, a8_deq;
   // block variants: smear (embedding, gate values, step-1 results), residual
   // scaling (x0, every layer's pre-scaling stream, the x0 gradient), backout
   // (x_b, the final stream gradient), value embeddings (table-gradient rows,
@@ -163,6 +164,10 @@ int launch_optim_init(const void* params, float* master, float* m, float* v, int
 int launch_quant_rows(const void* x, int64_t rows, int cols, void* q, float* deq, void* stream);
 int launch_quant_tensors(const void* x, int64_t n, int64_t stride, int n_mat, void* q, float* deq,
                          unsigned* amax_bits, void* stream);
+// codes of each W^T ([cols, rows]; rows, cols multiples of 64) with the scale
+// of the amax bits launch_quant_tensors left for the same matrices
+int launch_quant_tensors_t(const void* x, int rows, int cols, int64_t stride, int n_mat,
+                           const unsigned* amax_bits, void* q, void* stream);
 int launch_adamw(void* params, const void* grads, float* master, float* m, float* v, int64_t n,
                  float lr, float b1, float b2, float eps, float wd, float bc1, float bc2, void* stream);
 // M = mu M + G; U = nesterov ? G + mu M : M; x = bf16(U / (||U||_F + 1e-7)).

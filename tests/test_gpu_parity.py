@@ -9,8 +9,10 @@ Tolerances:
 * fp32 storage (tiny model): loss 1e-5 relative, cosine >= 0.99999,
   max-rel <= 1e-3 (fp32 accumulation over at most a few thousand terms).
 * index work (gather, stable sort of positions by token id): bit-exact.
-* e4m3 forward projections (fp8 configs) against the oracle's e4m3 reading:
-  the bf16 bars at the small shapes; at full d24 size loss 1e-3, per-position
+* e4m3 block projections (fp8 configs: forward and data gradients) against
+  the oracle's e4m3 reading: at the small shapes the bf16 bars widened to
+  what an oracle-only emulation of bf16-level quantizer-input differences
+  shows (tests/golden/fp8_noise_small.json); at full d24 size loss 1e-3, per-position
   losses 6e-2 (an oracle-only emulation over all 32,768 positions, stored in
   tests/golden/fp8_noise_d24.json), gradient max-rel 8e-2 and cosine 0.995
   (derived in TOL below from the quantizer's sensitivity to bf16-level input
@@ -39,8 +41,22 @@ def _fp8_token_bar():
         return float(json.load(f)["token_bar"])
 
 
+def _fp8_small_bars(bf16):
+    """Bars of the small FP8 shapes: the bf16 bars, widened where the oracle
+    alone shows more spread (tests/golden/make_fp8_small_bars.py: every input
+    of its row quantizer -- forward activations and the output gradients of
+    the e4m3 data-gradient products -- perturbed by 1e-3 relative noise, the
+    worst change over the three shapes and three seeds, times two)."""
+    with open(os.path.join(GOLDEN, "fp8_noise_small.json")) as f:
+        b = json.load(f)["bars"]
+    return dict(loss=max(bf16["loss"], b["loss"]), cos=min(bf16["cos"], b["cos"]),
+                maxrel=max(bf16["maxrel"], b["maxrel"]), tok=max(bf16["tok"], b["tok"]))
+
+
+_BF16 = dict(loss=1e-3, cos=0.999, maxrel=3e-2, tok=2e-2)
 TOL = {
-    "bf16": dict(loss=1e-3, cos=0.999, maxrel=3e-2, tok=2e-2),
+    "bf16": _BF16,
+    "fp8_small": _fp8_small_bars(_BF16),
     # e4m3 forward projections at full d24 size: an e4m3 code turns the
     # bf16-level difference between the GPU's and the oracle's quantizer
     # inputs into a whole code step.  The oracle with those inputs perturbed by
@@ -166,7 +182,7 @@ def grad_metrics(g, r):
 
 
 def check_against_oracle(st, w, res):
-    tol = TOL[w.dtype]
+    tol = TOL["fp8_small"] if w.fp8 else TOL[w.dtype]
     loss = float(st.loss.cpu().numpy()[0])
     assert abs(loss - res.loss) / abs(res.loss) <= tol["loss"], (loss, res.loss)
     tl = st.token_loss.cpu().numpy().astype(np.float64).reshape(w.batch, w.seq_len)
