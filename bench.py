@@ -367,6 +367,19 @@ def measure(w, args, rank, world, dev, barrier, *, optimizer=False, e2e=True):
     if code != B.GPT_OK:
         raise SystemExit(f"device status after warm-up: {B.strerror(code)}")
 
+    # the headline replays the step as one CUDA graph (the runtime's capture);
+    # the data-parallel step (NCCL on a second stream) runs eagerly
+    timed_step = one_step
+    if not args.no_graph and dps is None:
+        st.capture()
+        for _ in range(2):
+            st.replay()
+        torch.cuda.synchronize()
+        code = st.status()
+        if code != B.GPT_OK:
+            raise SystemExit(f"device status after graph warm-up: {B.strerror(code)}")
+        timed_step = st.replay
+
     bus = None
     try:
         bus = torch.cuda.get_device_properties(dev).pci_bus_id
@@ -382,7 +395,7 @@ def measure(w, args, rank, world, dev, barrier, *, optimizer=False, e2e=True):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
-        one_step()
+        timed_step()
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -391,6 +404,17 @@ def measure(w, args, rank, world, dev, barrier, *, optimizer=False, e2e=True):
     code = st.status()
     if code != B.GPT_OK:
         raise SystemExit(f"device status after timed steps: {B.strerror(code)}")
+    eager_ms = None
+    if timed_step is not one_step:  # the same steps launched one by one, for comparison
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            one_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        eager_ms = e0.elapsed_time(e1)
 
     # ---- the same steps again with every launch timed (breakdown only) ----
     per_step = 600
@@ -460,7 +484,8 @@ def measure(w, args, rank, world, dev, barrier, *, optimizer=False, e2e=True):
     if optimizer and world == 1 and cfg.dtype == B.GPT_BF16:
         optim = time_optimizer(B, st, stream)
 
-    out = dict(w=w, N=N, ms=ms, traced_ms=traced_ms, e2e_ms=e2e_ms, stats=stats, dropped=dropped,
+    out = dict(w=w, N=N, ms=ms, eager_ms=eager_ms, traced_ms=traced_ms, e2e_ms=e2e_ms, stats=stats,
+               dropped=dropped,
                sites=sites, clk=clk, optim=optim, bits=bits)
     del st
     torch.cuda.empty_cache()
@@ -553,7 +578,7 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16 + e4m3 forward block projections" if w.fp8 else "bf16",
+        "dtype": "bf16 + e4m3 block projections (forward and data gradients)" if w.fp8 else "bf16",
         "data": "synthetic (Zipf(1.1) token ids, seeded N(0,0.02) bf16 weights)",
         "config": {"workload": workload_desc(w), "global_batch": w.batch * world,
                    "seq_len": w.seq_len, "tokens_per_step": N * world,
@@ -561,7 +586,10 @@ def run_ours(args, rank, world, local_rank):
                                    "the backward)" if args.dp else f"replicas only x{world}")
                                   if world > 1 else "single GPU",
                    "l2": "no flush: every step moves tens of GB, far above the 126 MB L2",
-                   "timing": "headline untraced; breakdown and roofline from a second, traced pass"},
+                   "timing": ("headline untraced, the step replayed as one CUDA graph "
+                              "(eager_ms_per_step: the same steps launched one by one); "
+                              if main_m["eager_ms"] is not None else "headline untraced; ")
+                             + "breakdown and roofline from a second, traced pass of eager launches"},
         "mfu": s["mfu"],
         "mfu_peak": "nominal dense bf16 2.25 PFLOP/s",
         "mfu_vs_measured_sustained": s["mfu_measured"],
@@ -569,6 +597,8 @@ def run_ours(args, rank, world, local_rank):
         "roofline": roofline(main_m["sites"], w, s["gemm_tf"], s["peak_tf"], peaks),
         "kernel_breakdown": s["breakdown"],
         "gemm_sites": main_m["sites"],
+        "eager_ms_per_step": (round(main_m["eager_ms"] / args.steps, 3)
+                              if main_m["eager_ms"] is not None else None),
         "traced_ms_per_step": round(main_m["traced_ms"] / args.steps, 3),
         "gpu_launches": int(round(s["kernels_per_step"] * args.steps)),
         "trace_dropped": main_m["dropped"],
@@ -646,6 +676,8 @@ def main():
                     help="skip the depth-12 measurement that default runs add")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip timing the CPU oracle sample")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time eager launches instead of the step replayed as one CUDA graph")
     ap.add_argument("--layers", type=int, default=None,
                     help="override the workload's layer count (profiling captures on a smaller "
                          "case; the line then reports that model)")

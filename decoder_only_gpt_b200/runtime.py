@@ -62,6 +62,26 @@ class TrainStep:
         self.forward()
         self.backward()
 
+    # ---- the step as a CUDA graph --------------------------------------------
+    def capture(self) -> None:
+        """Record one forward + backward into a CUDA graph.  Every call of the
+        step is stream-ordered device work (kernels, async copies and memsets;
+        no host synchronisation, no allocation), so the whole step captures;
+        ``replay`` then launches it as one graph, without the per-launch host
+        work and gaps.  The graph reads the buffers in place: new tokens
+        (``set_batch``) and parameters take effect on the next replay."""
+        side = torch.cuda.Stream(self.device)
+        side.wait_stream(torch.cuda.current_stream(self.device))
+        with torch.cuda.stream(side):  # one eager step on the capture stream first
+            self.step()
+        torch.cuda.current_stream(self.device).wait_stream(side)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, stream=side):
+            self.step()
+
+    def replay(self) -> None:
+        self.graph.replay()
+
     def status(self) -> int:
         return B.status(self.workspace, self.stream)
 
