@@ -96,6 +96,8 @@ bool make_layout(const gpt_config& c, Layout* L) {
   L->tgt_stage = b.take(N * 4);
   L->rope_cos = b.take(T * (hd / 2) * 4);
   L->rope_sin = b.take(T * (hd / 2) * 4);
+  L->rope_cos_tr = b.take(T * (hd / 2) * 4);
+  L->rope_sin_tr = b.take(T * (hd / 2) * 4);
   L->x = b.take(N * d * 4);
   L->dxs = b.take(N * d * esz);
   // one layer's saved activations
@@ -541,7 +543,8 @@ int gpt_forward_loss(const gpt_config* c, const int32_t* tok, const int32_t* tgt
   {
     TraceScope ts(GPT_K_OTHER, 2, 0, c->seq_len * c->head_dim * 4.0, st);
     GPT_TRY(cuda_rc(cudaMemsetAsync(ws + L.status, 0, 256, st)));
-    GPT_TRY(launch_rope_table(*c, S.cos_t, S.sin_t, st));
+    GPT_TRY(launch_rope_table(*c, S.cos_t, S.sin_t, reinterpret_cast<float*>(ws + L.rope_cos_tr),
+                              reinterpret_cast<float*>(ws + L.rope_sin_tr), st));
   }
   {
     void* h0 = c->n_layer > 0 ? (void*)(S.layer(0) + L.lo.h1) : (void*)(ws + L.hf);
@@ -587,7 +590,8 @@ int gpt_forward_loss(const gpt_config* c, const int32_t* tok, const int32_t* tgt
       g.q_out = Lb + L.lo.q; g.k_out = Lb + L.lo.k; g.v_out = Lb + L.lo.v;
       g.rq = reinterpret_cast<float*>(Lb + L.lo.rq);
       g.rk = reinterpret_cast<float*>(Lb + L.lo.rk);
-      g.rope_cos = S.cos_t; g.rope_sin = S.sin_t;
+      g.rope_cos = reinterpret_cast<const float*>(ws + L.rope_cos_tr);
+      g.rope_sin = reinterpret_cast<const float*>(ws + L.rope_sin_tr);
       g.seq_len = c->seq_len; g.n_head = c->n_head; g.head_dim = c->head_dim;
       g.n_kv_head = c->n_kv_head;
       g.qk_norm = c->qk_norm; g.norm_eps = c->norm_eps;

@@ -265,8 +265,10 @@ __device__ __forceinline__ void epi_qkv_row(const GemmArgs& g, uint32_t taddr, i
     }
     const float r = g.qk_norm ? rsqrtf(ss / float(hd) + g.norm_eps) : 1.f;
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(part == 0 ? g.q_out : g.k_out) + dst;
-    const float* cr = g.rope_cos + int64_t(t) * half;
-    const float* sr = g.rope_sin + int64_t(t) * half;
+    // pair-major tables: the warp's lanes hold consecutive positions, so each
+    // load instruction reads one contiguous 128-byte line
+    const float* cr = g.rope_cos + t;
+    const float* sr = g.rope_sin + t;
     for (int i0 = 0; i0 < half; i0 += 16) {
       uint32_t ua[16], ub[16];
       tc::tmem_ld_32x32b_x16(tcol + i0, ua);
@@ -275,11 +277,9 @@ __device__ __forceinline__ void epi_qkv_row(const GemmArgs& g, uint32_t taddr, i
       if (!row_ok) continue;
       float cv[16], sv[16];
 #pragma unroll
-      for (int e = 0; e < 16; e += 4) {
-        const float4 c4 = *reinterpret_cast<const float4*>(cr + i0 + e);
-        const float4 s4 = *reinterpret_cast<const float4*>(sr + i0 + e);
-        cv[e] = c4.x; cv[e + 1] = c4.y; cv[e + 2] = c4.z; cv[e + 3] = c4.w;
-        sv[e] = s4.x; sv[e + 1] = s4.y; sv[e + 2] = s4.z; sv[e + 3] = s4.w;
+      for (int e = 0; e < 16; ++e) {
+        cv[e] = __ldg(cr + int64_t(i0 + e) * T);
+        sv[e] = __ldg(sr + int64_t(i0 + e) * T);
       }
       uint32_t pa[8], pb[8];
 #pragma unroll

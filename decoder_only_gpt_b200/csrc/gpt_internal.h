@@ -90,7 +90,7 @@ struct GemmArgs {
   float* rq;                // [B, n_head, T]: 1/rms of the rotated q rows
   float* rk;                // [B, n_kv_head, T]: the same for k
   const float* rope_cos;
-  const float* rope_sin;    // [T, hd/2]
+  const float* rope_sin;    // [hd/2, T]: position-contiguous, one table row per pair index
   int seq_len, n_head, head_dim, qk_norm;
   int n_kv_head;
   float norm_eps;
@@ -120,7 +120,8 @@ struct Layout {
   int64_t N;               // batch * seq_len
   int64_t vpad;            // vocab rounded up to 256 (row stride of the logit-gradient buffer)
   int esz;                 // bytes per stored activation element (2 bf16, 4 f32)
-  uint64_t status, tok_stage, tgt_stage, rope_cos, rope_sin;
+  // RoPE tables [T, hd/2] and the same transposed, [hd/2, T]
+  uint64_t status, tok_stage, tgt_stage, rope_cos, rope_sin, rope_cos_tr, rope_sin_tr;
   uint64_t x, dxs;
   uint64_t layer_base, layer_stride;
   LayerOffsets lo;         // offsets relative to the layer's base
@@ -186,7 +187,8 @@ int launch_muon_apply_rows(const void* x, float* master, void* params, int rows,
                            float step, const float* factor, void* stream);
 
 // ---- launchers (all enqueue on `stream`, return cudaError_t as int) ------
-int launch_rope_table(const gpt_config& c, float* cos_t, float* sin_t, void* stream);
+int launch_rope_table(const gpt_config& c, float* cos_t, float* sin_t, float* cos_tr, float* sin_tr,
+                      void* stream);
 int launch_embed_norm(const gpt_config& c, const int32_t* tok, const void* wte, float* x,
                       void* h, float* r, int32_t* status, void* stream);
 int launch_rms_fwd(const gpt_config& c, const float* x, void* h, float* r, void* stream);

@@ -12,10 +12,12 @@
 namespace gpt {
 
 // ---------------------------------------------------------------------------
-// RoPE table: angle(t, i) = t * base^(-2i/hd), evaluated in fp64, stored fp32.
+// RoPE table: angle(t, i) = t * base^(-2i/hd), evaluated in fp64, stored fp32,
+// both position-major [T, hd/2] and pair-major [hd/2, T] (the QKV epilogue's
+// threads hold consecutive positions, so a pair-major row is one coalesced load)
 // ---------------------------------------------------------------------------
-__global__ void rope_table_kernel(float* cos_t, float* sin_t, int T, int half, double base,
-                                  int hd) {
+__global__ void rope_table_kernel(float* cos_t, float* sin_t, float* cos_tr, float* sin_tr, int T, int half,
+                                  double base, int hd) {
   int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= T * half) return;
   int t = idx / half, i = idx % half;
@@ -24,12 +26,15 @@ __global__ void rope_table_kernel(float* cos_t, float* sin_t, int T, int half, d
   sincos(double(t) * theta, &s, &c);
   cos_t[idx] = float(c);
   sin_t[idx] = float(s);
+  cos_tr[int64_t(i) * T + t] = float(c);
+  sin_tr[int64_t(i) * T + t] = float(s);
 }
 
-int launch_rope_table(const gpt_config& c, float* cos_t, float* sin_t, void* stream) {
+int launch_rope_table(const gpt_config& c, float* cos_t, float* sin_t, float* cos_tr, float* sin_tr,
+                      void* stream) {
   int half = c.head_dim / 2, n = c.seq_len * half;
   rope_table_kernel<<<ceil_div(n, 256), 256, 0, (cudaStream_t)stream>>>(
-      cos_t, sin_t, c.seq_len, half, double(c.rope_base), c.head_dim);
+      cos_t, sin_t, cos_tr, sin_tr, c.seq_len, half, double(c.rope_base), c.head_dim);
   return last_launch_rc();
 }
 
