@@ -218,6 +218,14 @@ __device__ __forceinline__ void epi_chunk(const GemmArgs& g, int row, int col0, 
   }
 }
 
+// Staging tile of one epilogue warp: 32 rows x 32 fp32, its 16-byte units
+// XOR-swizzled by row so that both the row-wise writes and the column-wise
+// reads are free of bank conflicts.
+constexpr uint32_t kStageBytes = 32 * 32 * 4;
+__device__ __forceinline__ float4* stage_at(float* tile, int r, int u) {
+  return reinterpret_cast<float4*>(tile + r * 32 + ((u ^ (r & 7)) << 2));
+}
+
 // EPI_QKV: a thread's 128 tile columns hold whole heads (head_dim 64 or 128
 // divides 128).  For each head of this row: v is copied to its head-major row; q and k
 // are rotated by RoPE (pairs (i, i + hd/2)), scaled by 1/rms of the rotated row
@@ -225,7 +233,7 @@ __device__ __forceinline__ void epi_chunk(const GemmArgs& g, int row, int col0, 
 // and written head-major, with the 1/rms kept for the backward.
 template <bool SCALED>
 __device__ __forceinline__ void epi_qkv_row(const GemmArgs& g, uint32_t taddr, int row,
-                                            int col_base, bool row_ok, float esc) {
+                                            int col_base, bool row_ok, float esc, float* tile) {
   // esc: the operands' dequantization factor of this row (8-bit operands only)
   auto val = [&](uint32_t u) { return SCALED ? u2f(u) * esc : u2f(u); };
   const int hd = g.head_dim, half = hd / 2, H = g.n_head, Hkv = g.n_kv_head, T = g.seq_len;
@@ -269,12 +277,12 @@ __device__ __forceinline__ void epi_qkv_row(const GemmArgs& g, uint32_t taddr, i
     // load instruction reads one contiguous 128-byte line
     const float* cr = g.rope_cos + t;
     const float* sr = g.rope_sin + t;
+    const int lane = threadIdx.x & 31;
     for (int i0 = 0; i0 < half; i0 += 16) {
       uint32_t ua[16], ub[16];
       tc::tmem_ld_32x32b_x16(tcol + i0, ua);
       tc::tmem_ld_32x32b_x16(tcol + half + i0, ub);
       tc::tmem_wait_ld();
-      if (!row_ok) continue;
       float cv[16], sv[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
@@ -291,12 +299,26 @@ __device__ __forceinline__ void epi_qkv_row(const GemmArgs& g, uint32_t taddr, i
         pa[e] = pack_bf16((a0 * c0v - b0 * s0v) * r, (a1 * c1v - b1 * s1v) * r);
         pb[e] = pack_bf16((a0 * s0v + b0 * c0v) * r, (a1 * s1v + b1 * c1v) * r);
       }
-      uint4* oa = reinterpret_cast<uint4*>(out + i0);
-      uint4* ob = reinterpret_cast<uint4*>(out + half + i0);
-      oa[0] = make_uint4(pa[0], pa[1], pa[2], pa[3]);
-      oa[1] = make_uint4(pa[4], pa[5], pa[6], pa[7]);
-      ob[0] = make_uint4(pb[0], pb[1], pb[2], pb[3]);
-      ob[1] = make_uint4(pb[4], pb[5], pb[6], pb[7]);
+      // through the warp's staging tile, so that each store instruction
+      // writes 8 rows x 64 contiguous bytes (whole 32-byte sectors) instead of
+      // 32 rows x 16 bytes: row r's 32 outputs go to units 0..3 of tile row r,
+      // then lane (row 8k + lane/4, unit lane%4) stores one unit
+      __syncwarp();
+      *reinterpret_cast<uint4*>(stage_at(tile, lane, 0)) = make_uint4(pa[0], pa[1], pa[2], pa[3]);
+      *reinterpret_cast<uint4*>(stage_at(tile, lane, 1)) = make_uint4(pa[4], pa[5], pa[6], pa[7]);
+      *reinterpret_cast<uint4*>(stage_at(tile, lane, 2)) = make_uint4(pb[0], pb[1], pb[2], pb[3]);
+      *reinterpret_cast<uint4*>(stage_at(tile, lane, 3)) = make_uint4(pb[4], pb[5], pb[6], pb[7]);
+      __syncwarp();
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int rr = 8 * k + (lane >> 2), u = lane & 3;
+        const uint64_t orow = __shfl_sync(0xffffffffu, reinterpret_cast<uint64_t>(out), rr);
+        const bool rok = __shfl_sync(0xffffffffu, int(row_ok), rr) != 0;
+        const uint4 v = *reinterpret_cast<const uint4*>(stage_at(tile, rr, u));
+        if (rok)
+          *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(orow) + (u < 2 ? i0 : half + i0) +
+                                    8 * (u & 1)) = v;
+      }
     }
     if (row_ok) {
       const int64_t ri = (int64_t(b) * nh + h) * T + t;
@@ -305,13 +327,6 @@ __device__ __forceinline__ void epi_qkv_row(const GemmArgs& g, uint32_t taddr, i
   }
 }
 
-// Staging tile of one epilogue warp: 32 rows x 32 fp32, its 16-byte units
-// XOR-swizzled by row so that both the row-wise writes and the column-wise
-// reads are free of bank conflicts.
-constexpr uint32_t kStageBytes = 32 * 32 * 4;
-__device__ __forceinline__ float4* stage_at(float* tile, int r, int u) {
-  return reinterpret_cast<float4*>(tile + r * 32 + ((u ^ (r & 7)) << 2));
-}
 
 // Partial-column fallback (col + 4 > N, or a row pitch that is not a multiple
 // of 4): the same element-wise epilogue, one element at a time.
@@ -453,7 +468,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& g, uint32_t taddr,
   }
   float ce_max = -INFINITY, ce_sum = 0.f, ce_tgt = 0.f;
   if (g.epi == EPI_QKV) {
-    epi_qkv_row<SCALED>(g, taddr, row, col_base, row_ok, esc);
+    epi_qkv_row<SCALED>(g, taddr, row, col_base, row_ok, esc, tile);
     return;
   }
   if ((g.epi == EPI_CE_FWD || g.epi == EPI_CE_BWD) && splits == 1) {
