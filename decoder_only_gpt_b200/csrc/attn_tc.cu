@@ -1194,7 +1194,7 @@ struct DkvBars {
   uint64_t fixed_full;
   uint64_t q_full[kDkvRingQ], q_empty[kDkvRingQ], do_full[kDkvRingDO], do_empty[kDkvRingDO];
   uint64_t stat_full, stat_empty;
-  uint64_t s_full, dp_full, p_ready, ds_ready;
+  uint64_t s_full, dp_full, p_ready[2], ds_ready;  // p_ready[c]: P^T of query chunk c written
   uint64_t acc_full, epi_full, done;
   uint32_t tmem_base;
   int abort;
@@ -1262,7 +1262,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::mbar_init(&bars->stat_empty, 256);
     tc::mbar_init(&bars->s_full, 1);
     tc::mbar_init(&bars->dp_full, 1);
-    tc::mbar_init(&bars->p_ready, 256);
+    tc::mbar_init(&bars->p_ready[0], 256);
+    tc::mbar_init(&bars->p_ready[1], 256);
     tc::mbar_init(&bars->ds_ready, 256);
     tc::mbar_init(&bars->acc_full, 1);
     tc::mbar_init(&bars->epi_full, 1);
@@ -1376,14 +1377,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mma_bf16_ss_elect(t, tc::desc_advance(fd, off), tc::desc_advance(rd, off), idesc_s, k != 0);
       }
     };
-    // acc += A^T B over the tile's 128 queries (A: bf16 pairs over `t`'s columns, B: a ring tile)
-    auto issue_acc = [&](uint32_t acc, uint32_t t, const uint8_t* bt, bool first) {
+    // acc += A^T B over 16-query steps k of the tile's 128 queries (A: bf16
+    // pairs over `t`'s columns, B: a ring tile); `kmask` selects the steps
+    auto issue_acc = [&](uint32_t acc, uint32_t t, const uint8_t* bt, bool first, uint32_t kmask) {
       const uint64_t bmn = tc::smem_desc_sw128(tc::smem_u32(bt), CH);
 #pragma unroll
       for (int k = 0; k < 128 / 16; ++k)
-        tc::mma_bf16_ts_elect(acc, t + 64 * (k >> 2) + 8 * (k & 3), tc::desc_advance(bmn, k * 2048), idesc_acc,
-                              !(first && k == 0));
+        if (kmask >> k & 1)
+          tc::mma_bf16_ts_elect(acc, t + 64 * (k >> 2) + 8 * (k & 3), tc::desc_advance(bmn, k * 2048),
+                                idesc_acc, !(first && k == 0));
     };
+    // the threads' first 32-query chunk covers steps 0, 1 (half 0) and 4, 5 (half 1)
+    constexpr uint32_t kChunk0 = 0x33u, kChunk1 = 0xCCu;
     auto q_tile = [&](int j) { return smem + S::Q_OFF + (j % kDkvRingQ) * S::TILE; };
     auto do_tile = [&](int j) { return smem + S::DO_OFF + (j % kDkvRingDO) * S::TILE; };
     auto q_ready = [&](int j) { return tc::mbar_spin_warp(&bars->q_full[j % kDkvRingQ], (j / kDkvRingQ) & 1, abort, kWaitNs); };
@@ -1403,9 +1408,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mma_commit_elect(&bars->dp_full);
     }
     for (int j = 0; ok && j < n_steps; ++j) {
-      if (!tc::mbar_spin_warp(&bars->p_ready, j & 1, abort, kWaitNs)) { ok = false; break; }
+      // dV += P^T_j dO_j, the first chunk's steps as soon as the threads have
+      // written them, while they form the second
+      if (!tc::mbar_spin_warp(&bars->p_ready[0], j & 1, abort, kWaitNs)) { ok = false; break; }
       tc::tc_fence_after();
-      issue_acc(t_dv, tmem, do_tile(j), j == 0);           // dV += P^T_j dO_j
+      issue_acc(t_dv, tmem, do_tile(j), j == 0, kChunk0);
+      if (!tc::mbar_spin_warp(&bars->p_ready[1], j & 1, abort, kWaitNs)) { ok = false; break; }
+      tc::tc_fence_after();
+      issue_acc(t_dv, tmem, do_tile(j), false, kChunk1);
       tc::mma_commit_elect(&bars->do_empty[j % kDkvRingDO]);  // dP^T_j and dV_j read dO_j
       if (j + 1 < n_steps) {
         if (!q_ready(j + 1)) { ok = false; break; }
@@ -1415,7 +1425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!tc::mbar_spin_warp(&bars->ds_ready, j & 1, abort, kWaitNs)) { ok = false; break; }
       tc::tc_fence_after();
-      issue_acc(t_dk, t_dp, q_tile(j), j == 0);            // dK += dS^T_j Q_j
+      issue_acc(t_dk, t_dp, q_tile(j), j == 0, 0xFFu);     // dK += dS^T_j Q_j
       tc::mma_commit_elect(&bars->q_empty[j % kDkvRingQ]);  // S^T_j and dK_j read Q_j
       if (j + 1 < n_steps) {
         if (!do_ready(j + 1)) { ok = false; break; }
@@ -1455,7 +1465,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::tmem_ld_32x32b_x32(ts, us0);
         tc::tmem_ld_32x32b_x32(ts + 32, us1);
         tc::tmem_wait_ld();
-        // P^T over the first 32 of this thread's S^T columns (all 64 S^T values are in registers)
+        // P^T over the first 32 of this thread's S^T columns (all 64 S^T values
+        // are in registers), one 32-query chunk at a time, each announced
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint32_t pk[16];
@@ -1464,11 +1475,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           else
             p_col32<false>(c ? us1 : us0, stat + 32 * c, p + 32 * c, pk, scale_log2, qs + 32 * c, q_lo, q_hi);
           tc::tmem_st_32x32b_x16(ts + 16 * c, pk);
+          tc::tmem_wait_st();
+          tc::tc_fence_before();
+          tc::mbar_arrive(&bars->p_ready[c]);
         }
-        tc::tmem_wait_st();
-        tc::tc_fence_before();
+      } else {
+        tc::mbar_arrive(&bars->p_ready[0]);
+        tc::mbar_arrive(&bars->p_ready[1]);
       }
-      tc::mbar_arrive(&bars->p_ready);
       if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_spin(&bars->dp_full, j & 1, abort, kWaitNs));
       if (ok) {
         tc::tc_fence_after();
