@@ -198,9 +198,10 @@ __global__ void rms_bwd_kernel(const T* __restrict__ dh, const T* __restrict__ h
   }
 }
 
-// bf16, d % 8 == 0, d <= 8 * 32 * KV: all of a row's loads (dh, h and, when
-// accumulating, the fp32 dx) are issued before the row reduction, so their
-// latencies overlap; KV = the 8-element groups per lane, sized to d.
+// bf16, d % 8 == 0, d <= 8 * 32 * KV: a row's dh and h loads are issued
+// before the row reduction, so their latencies overlap; the fp32 dx it
+// accumulates into is read after it (fewer live registers, more warps per SM
+// to cover the latency); KV = the 8-element groups per lane, sized to d.
 template <int KV>
 __global__ void rms_bwd_bf16_vec(const __nv_bfloat16* __restrict__ dh,
                                  const __nv_bfloat16* __restrict__ h, const float* __restrict__ r,
@@ -214,17 +215,12 @@ __global__ void rms_bwd_bf16_vec(const __nv_bfloat16* __restrict__ dh,
   const uint4* hr = reinterpret_cast<const uint4*>(h + row * d);
   float4* xr = reinterpret_cast<float4*>(dx + row * d);
   uint4 gd[KV], gh[KV];
-  float4 p0[KV], p1[KV];
 #pragma unroll
   for (int k = 0; k < KV; ++k) {
     const int gi = lane + 32 * k;
     if (gi < groups) {
       gd[k] = dr[gi];
       gh[k] = hr[gi];
-      if (accumulate) {
-        p0[k] = xr[2 * gi];
-        p1[k] = xr[2 * gi + 1];
-      }
     }
   }
   float s = 0.f;
@@ -252,8 +248,9 @@ __global__ void rms_bwd_bf16_vec(const __nv_bfloat16* __restrict__ dh,
 #pragma unroll
       for (int e = 0; e < 8; ++e) g[e] = rr * (fa[e] - fb[e] * s);
       if (accumulate) {
-        g[0] += p0[k].x; g[1] += p0[k].y; g[2] += p0[k].z; g[3] += p0[k].w;
-        g[4] += p1[k].x; g[5] += p1[k].y; g[6] += p1[k].z; g[7] += p1[k].w;
+        const float4 p0 = xr[2 * gi], p1 = xr[2 * gi + 1];
+        g[0] += p0.x; g[1] += p0.y; g[2] += p0.z; g[3] += p0.w;
+        g[4] += p1.x; g[5] += p1.y; g[6] += p1.z; g[7] += p1.w;
       }
       xr[2 * gi] = make_float4(g[0], g[1], g[2], g[3]);
       xr[2 * gi + 1] = make_float4(g[4], g[5], g[6], g[7]);
