@@ -239,7 +239,7 @@ def gemm_sites(records, w, steps):
 # site, from an ncu capture of the current kernel build, keyed by (workload,
 # site, fp8); a site that has not been captured reports null.
 TRAFFIC_BYTES = {
-    ("d24", 32768, 6144, 1536, False): 121_360_896 + 362_861_824,  # ncu: 484.2 MB per launch
+    ("d24", 32768, 6144, 1536, False): 120_946_432 + 361_932_032,  # ncu: 482.9 MB per launch
     ("d24", 32768, 6144, 1536, True): 60_106_752 + 351_310_080,    # e4m3 operands: 411.4 MB
 }
 
@@ -263,7 +263,7 @@ def roofline(sites, w, gemm_tf, peak_tf, peaks):
         line.update({"kernel": "gemm_pair_kernel (tcgen05 cta_group::2 GEMM, kind::f8f6f4 e4m3)",
                      "peak": site_peak,
                      "peak_source": f"{peaks['source']} bf16_tflops_sustained x 2 (nominal e4m3/bf16 ratio)",
-                     "all_gemm_launches": {"achieved": round(gemm_tf, 1), "mixed": "e4m3 forward, bf16 backward"}})
+                     "all_gemm_launches": {"achieved": round(gemm_tf, 1), "mixed": "e4m3 forward and data gradients, bf16 weight gradients"}})
     if site and site["ms_per_launch"] > 0:
         tf = site["flops_per_launch"] / (site["ms_per_launch"] / 1e3) / 1e12
         key = (w.name, w.batch * w.seq_len, w.d_ff, w.d_model, bool(w.fp8))
