@@ -143,6 +143,10 @@ bool make_layout(const gpt_config& c, Layout* L) {
   L->lse_z = b.take(N * 4);
   L->tok_loss = b.take(N * 4);
   L->loss_acc = b.take(256);
+  // the MLP norm's backward, folded into the down- and up-projection data
+  // gradients (bf16): one fp32 row partial per output column block of >= 64
+  L->n_npart = (F + 63) / 64;
+  L->npart = b.take(c.dtype == GPT_BF16 ? N * L->n_npart * 4 : 0);
   L->G = b.take(N * L->vpad * esz);
   L->dh = b.take(N * d * esz);
   L->du = b.take(N * F * esz);
@@ -392,7 +396,8 @@ static int run_gemm(const gpt_config& c, const GemmArgs& g, cudaStream_t st) {
   switch (g.epi) {
     case EPI_STORE: bytes += mn * e * (g.beta ? 2 : 1); break;
     case EPI_RESID_F32: bytes += mn * 8; break;
-    case EPI_DRELU2: bytes += mn * e * 2; break;
+    case EPI_DRELU2: bytes += mn * e * 2 + (g.norm_part_out ? double(g.M) * g.n_npart * 4 : 0.0); break;
+    case EPI_NORM_BWD: bytes += mn * (2 * e + 8) + double(g.M) * (g.n_npart + 1) * 4; break;
     case EPI_AXPBY: bytes += mn * e * 2; break;
     case EPI_CE_FWD: bytes += double(g.M) * 12; break;
     case EPI_QKV: bytes += mn * e + double(g.M) * (g.n_head + g.n_kv_head) * 4; break;
@@ -715,25 +720,42 @@ static int backward_impl(const gpt_config* c, const int32_t* tok, const int32_t*
   if (c->resid_lambdas) GPT_TRY(cuda_rc(cudaMemsetAsync(ws + L.dx0, 0, nd4, st)));
 
   const double attn_b = 8.0 * attn_pairs(*c) * c->head_dim;  // dV, dP, dQ, dK, causal half
+  // bf16 steps fold the MLP norm's backward into the two MLP data-gradient
+  // GEMMs.  With h = h2 the norm's output, u = h Wup^T, a = relu(u)^2 and
+  // dh = du Wup, the row sum that the RMSNorm backward needs is
+  //   sum_j dh_j h_j = sum_f du_f u_f = 2 sum_f da_f a_f
+  // (du = da * 2 relu(u) is 0 where u <= 0, and relu(u) u = a elsewhere):
+  // the down-projection dgrad's epilogue has da and a in hand and writes
+  // per-row partials of it; the up-projection dgrad's epilogue sums them and
+  // applies dx += r (dh - h s), s = (2/d) sum, writing the bf16 copy of dx.
+  const bool fold = c->dtype == GPT_BF16 && !c->fp8;
+  const int n_np = (F + gemm_ce_tile_n(*c) - 1) / gemm_ce_tile_n(*c);
   for (int l = c->n_layer - 1; l >= 0; --l) {
     char* Lb = S.layer(l);
     // MLP down: da = dx Wdown, du = da * 2 relu(u) (from the stored a = relu(u)^2)
     g = gemm_kk(ws + L.dxs, d, S.param(GPT_T_WDOWN, l), F, N, F, d, EPI_DRELU2, ws + L.du, F,
                 status);
     g.b_mn_major = true; g.aux = Lb + L.lo.a;
+    if (fold) { g.norm_part_out = S.f(L.npart); g.n_npart = n_np; }
     GPT_TRY(S.dgrad(g, GPT_T_WDOWN, l));
     g = gemm_kk(ws + L.dxs, d, Lb + L.lo.a, F, d, F, N, EPI_STORE, grad(GPT_T_WDOWN, l), F,
                 status);
     g.a_mn_major = true; g.b_mn_major = true; g.beta = accumulate;
     GPT_TRY(run_gemm(*c, with_splitk(g, L, ws), st));
-    // MLP up
-    g = gemm_kk(ws + L.du, F, S.param(GPT_T_WUP, l), d, N, d, F, EPI_STORE, ws + L.dh, d, status);
+    // MLP up (with the norm's backward when folded)
+    float* r2 = reinterpret_cast<float*>(Lb + L.lo.r2);
+    g = gemm_kk(ws + L.du, F, S.param(GPT_T_WUP, l), d, N, d, F, fold ? EPI_NORM_BWD : EPI_STORE,
+                fold ? static_cast<void*>(S.x) : ws + L.dh, d, status);
     g.b_mn_major = true;
+    if (fold) {
+      g.aux = Lb + L.lo.h2; g.out2 = ws + L.dxs; g.norm_part = S.f(L.npart); g.norm_r = r2;
+      g.n_npart = n_np; g.norm_scale = 2.f / float(d);
+    }
     GPT_TRY(S.dgrad(g, GPT_T_WUP, l));
     g = gemm_kk(ws + L.du, F, Lb + L.lo.h2, d, F, d, N, EPI_STORE, grad(GPT_T_WUP, l), d, status);
     g.a_mn_major = true; g.b_mn_major = true; g.beta = accumulate;
     GPT_TRY(run_gemm(*c, with_splitk(g, L, ws), st));
-    GPT_TRY(S.rms_bwd(ws + L.dh, Lb + L.lo.h2, reinterpret_cast<float*>(Lb + L.lo.r2), 1));
+    if (!fold) GPT_TRY(S.rms_bwd(ws + L.dh, Lb + L.lo.h2, r2, 1));
     // attention out-projection
     g = gemm_kk(ws + L.dxs, d, S.param(GPT_T_WO, l), d, N, d, d, EPI_STORE, ws + L.dO, d, status);
     g.b_mn_major = true;

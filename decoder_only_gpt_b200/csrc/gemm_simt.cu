@@ -105,6 +105,8 @@ static int launch_simt(GemmArgs g, cudaStream_t st) {
 }
 
 int launch_gemm_simt_f32(const GemmArgs& g, void* stream) {
+  // the folded RMSNorm backward is a tensor-core epilogue only
+  if (g.epi == EPI_NORM_BWD || g.norm_part_out) return 1;
   return launch_simt<float>(g, (cudaStream_t)stream);
 }
 

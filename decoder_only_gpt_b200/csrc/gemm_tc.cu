@@ -65,9 +65,13 @@ __device__ __forceinline__ void epilogue_prefetch(const GemmArgs& g, int row, in
   if (g.epi == EPI_DRELU2) {
     const char* p = reinterpret_cast<const char*>(static_cast<const __nv_bfloat16*>(g.aux) + base);
     for (int b = 0; b < cols * 2; b += 128) prefetch_l2(p + b);
-  } else if (g.epi == EPI_RESID_F32) {
+  } else if (g.epi == EPI_RESID_F32 || g.epi == EPI_NORM_BWD) {
     const char* p = reinterpret_cast<const char*>(static_cast<const float*>(g.out) + base);
     for (int b = 0; b < cols * 4; b += 128) prefetch_l2(p + b);
+    if (g.epi == EPI_NORM_BWD) {
+      const char* h = reinterpret_cast<const char*>(static_cast<const __nv_bfloat16*>(g.aux) + base);
+      for (int b = 0; b < cols * 2; b += 128) prefetch_l2(h + b);
+    }
   } else if (g.epi == EPI_STORE && g.beta) {
     const char* p = reinterpret_cast<const char*>(static_cast<const __nv_bfloat16*>(g.out) + base);
     for (int b = 0; b < cols * 2; b += 128) prefetch_l2(p + b);
@@ -220,8 +224,9 @@ __device__ __forceinline__ void epi_chunk(const GemmArgs& g, int row, int col0, 
 
 // Staging tile of one epilogue warp: 32 rows x 32 fp32, its 16-byte units
 // XOR-swizzled by row so that both the row-wise writes and the column-wise
-// reads are free of bank conflicts.
-constexpr uint32_t kStageBytes = 32 * 32 * 4;
+// reads are free of bank conflicts; then one fp32 per row (kStageRowSlot).
+constexpr uint32_t kStageBytes = 32 * 32 * 4 + 32 * 4;
+constexpr int kStageRowSlot = 32 * 32;
 __device__ __forceinline__ float4* stage_at(float* tile, int r, int u) {
   return reinterpret_cast<float4*>(tile + r * 32 + ((u ^ (r & 7)) << 2));
 }
@@ -329,11 +334,16 @@ __device__ __forceinline__ void epi_qkv_row(const GemmArgs& g, uint32_t taddr, i
 
 
 // Partial-column fallback (col + 4 > N, or a row pitch that is not a multiple
-// of 4): the same element-wise epilogue, one element at a time.
-__device__ __noinline__ void epi4_scalar(const GemmArgs& g, int row, int col, float4 a, int sp,
-                                         int splits, int tgt, float lse_row, int64_t obase) {
+// of 4): the same element-wise epilogue, one element at a time.  rs: the
+// row's r s (EPI_NORM_BWD, whose staged accumulator is already r acc).
+// Returns the row partial sum of acc * aux over these columns (EPI_DRELU2),
+// else 0.
+__device__ __noinline__ float epi4_scalar(const GemmArgs& g, int row, int col, float4 a, int sp,
+                                          int splits, int tgt, float lse_row, int64_t obase,
+                                          float rs) {
   const int nc = min(4, g.N - col);
   const float v[4] = {a.x, a.y, a.z, a.w};
+  float part = 0.f;
   for (int j = 0; j < nc; ++j) {
     const int n = col + j;
     if (splits > 1) {
@@ -343,11 +353,23 @@ __device__ __noinline__ void epi4_scalar(const GemmArgs& g, int row, int col, fl
     const int64_t e = obase + int64_t(row) * g.ldo + n;
     if (g.epi == EPI_RESID_F32) { static_cast<float*>(g.out)[e] += v[j]; continue; }
     if (g.epi == EPI_STORE_F32) { static_cast<float*>(g.out)[e] = v[j]; continue; }
+    if (g.epi == EPI_NORM_BWD) {
+      float* x = static_cast<float*>(g.out);
+      const float h = __bfloat162float(static_cast<const __nv_bfloat16*>(g.aux)[e]);
+      const float gv = v[j] - h * rs + x[e];
+      x[e] = gv;
+      static_cast<__nv_bfloat16*>(g.out2)[e] = __float2bfloat16_rn(gv);
+      continue;
+    }
     __nv_bfloat16* o = static_cast<__nv_bfloat16*>(g.out);
     float r = v[j];
     if (g.epi == EPI_STORE && g.beta) r += __bfloat162float(o[e]);
     if (g.epi == EPI_RELU2) { const float t = fmaxf(v[j], 0.f); r = t * t; }
-    if (g.epi == EPI_DRELU2) r = v[j] * 2.f * sqrt_approx(__bfloat162float(static_cast<const __nv_bfloat16*>(g.aux)[e]));
+    if (g.epi == EPI_DRELU2) {
+      const float in = __bfloat162float(static_cast<const __nv_bfloat16*>(g.aux)[e]);
+      part = fmaf(v[j], in, part);
+      r = v[j] * 2.f * sqrt_approx(in);
+    }
     if (g.epi == EPI_AXPBY)
       r = g.alpha * v[j] + g.beta_aux * __bfloat162float(static_cast<const __nv_bfloat16*>(g.aux)[e]);
     if (g.epi == EPI_CE_BWD) {
@@ -356,7 +378,14 @@ __device__ __noinline__ void epi4_scalar(const GemmArgs& g, int row, int col, fl
     }
     o[e] = __float2bfloat16_rn(r);
   }
+  return part;
 }
+
+// The lane's partials of acc * aux for its rows 4i + rsub (EPI_DRELU2 with
+// norm_part_out).
+struct NormRows {
+  float part[8];
+};
 
 // Element-wise epilogue of one 32-column chunk of a warp's 32 rows, from the
 // staging tile: lane (rsub, u4) handles columns col .. col + 4 of rows
@@ -366,7 +395,7 @@ __device__ __noinline__ void epi4_scalar(const GemmArgs& g, int row, int col, fl
 template <int KIND>
 __device__ __forceinline__ void epi_chunk_coalesced(const GemmArgs& g, float* tile, int wrow0, int col,
                                                     int rsub, int u4, int sp, int splits, int tgt,
-                                                    float lse_row, int64_t obase) {
+                                                    float lse_row, int64_t obase, NormRows& nrm) {
   float4 a[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) a[i] = *stage_at(tile, 4 * i + rsub, u4);
@@ -386,8 +415,9 @@ __device__ __forceinline__ void epi_chunk_coalesced(const GemmArgs& g, float* ti
 #pragma unroll
     for (int i = 0; i < 8; ++i)
       if (wrow0 + 4 * i + rsub < g.M)
-        epi4_scalar(g, wrow0 + 4 * i + rsub, col, a[i], sp, splits, KIND == EPI_CE_BWD ? t[i] : -1,
-                    KIND == EPI_CE_BWD ? ls[i] : 0.f, obase);
+        nrm.part[i] += epi4_scalar(g, wrow0 + 4 * i + rsub, col, a[i], sp, splits,
+                                   KIND == EPI_CE_BWD ? t[i] : -1, KIND == EPI_CE_BWD ? ls[i] : 0.f,
+                                   obase, KIND == EPI_NORM_BWD ? tile[kStageRowSlot + 4 * i + rsub] : 0.f);
     return;
   }
   bool ok[8];
@@ -414,6 +444,41 @@ __device__ __forceinline__ void epi_chunk_coalesced(const GemmArgs& g, float* ti
       if (ok[i]) *reinterpret_cast<float4*>(o + e[i]) = a[i];
     return;
   }
+  if (KIND == EPI_NORM_BWD) {
+    // x <- x + r acc - (r s) h (the staged values are r acc; r s per row in
+    // the staging tile's row slots), and its bf16 copy
+    float* xo = static_cast<float*>(g.out);
+    const __nv_bfloat16* hs = static_cast<const __nv_bfloat16*>(g.aux);
+    __nv_bfloat16* o2 = static_cast<__nv_bfloat16*>(g.out2);
+    // two halves of 4 rows: every load of a half issued before its stores
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      float4 x[4];
+      uint2 hw[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int i = 4 * half + q;
+        x[q] = ok[i] ? *reinterpret_cast<const float4*>(xo + e[i]) : make_float4(0.f, 0.f, 0.f, 0.f);
+        hw[q] = ok[i] ? *reinterpret_cast<const uint2*>(hs + e[i]) : make_uint2(0u, 0u);
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int i = 4 * half + q;
+        const float rs = tile[kStageRowSlot + 4 * i + rsub];
+        const float2 h0 = unpack_bf16(hw[q].x), h1 = unpack_bf16(hw[q].y);
+        float4 r;
+        r.x = fmaf(-rs, h0.x, a[i].x) + x[q].x;
+        r.y = fmaf(-rs, h0.y, a[i].y) + x[q].y;
+        r.z = fmaf(-rs, h1.x, a[i].z) + x[q].z;
+        r.w = fmaf(-rs, h1.y, a[i].w) + x[q].w;
+        if (ok[i]) {
+          *reinterpret_cast<float4*>(xo + e[i]) = r;
+          *reinterpret_cast<uint2*>(o2 + e[i]) = make_uint2(pack_bf16(r.x, r.y), pack_bf16(r.z, r.w));
+        }
+      }
+    }
+    return;
+  }
   __nv_bfloat16* o = static_cast<__nv_bfloat16*>(g.out);
   constexpr bool kIn = KIND == EPI_DRELU2 || KIND == EPI_STORE || KIND == EPI_AXPBY;
   uint2 w[8];
@@ -431,6 +496,8 @@ __device__ __forceinline__ void epi_chunk_coalesced(const GemmArgs& g, float* ti
     const float2 i0 = unpack_bf16(w[i].x), i1 = unpack_bf16(w[i].y);
     const float in[4] = {i0.x, i0.y, i1.x, i1.y};
     float r[4];
+    if (KIND == EPI_DRELU2 && ok[i])
+      nrm.part[i] = fmaf(v[0], in[0], fmaf(v[1], in[1], fmaf(v[2], in[2], fmaf(v[3], in[3], nrm.part[i]))));
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       if (KIND == EPI_STORE) r[j] = v[j] + in[j];
@@ -444,6 +511,70 @@ __device__ __forceinline__ void epi_chunk_coalesced(const GemmArgs& g, float* ti
       } else r[j] = v[j];
     }
     if (ok[i]) *reinterpret_cast<uint2*>(o + e[i]) = make_uint2(pack_bf16(r[0], r[1]), pack_bf16(r[2], r[3]));
+  }
+}
+
+// The element-wise epilogues of one thread's EC columns (KIND: an Epilogue
+// value, or -1 for the fp32 partials of a K split).  The warp's 32 rows x 32
+// columns pass through its staging tile, then each lane handles 4 columns of
+// a row so that a warp instruction covers 4 rows x 32 consecutive columns.
+// EPI_NORM_BWD: the thread stages r acc for its row and leaves r s in its
+// row slot of the staging tile.  EPI_DRELU2 with norm_part_out: each chunk's lane partials reduced
+// over the row's 8 lanes, lane u4 keeping row 4 u4 + rsub's running sum.
+template <int KIND, bool SCALED>
+__device__ __forceinline__ void epi_tile_coalesced(const GemmArgs& g, uint32_t taddr, int row, bool row_ok,
+                                                   int wrow0, int col_base, int part, int sp, int splits,
+                                                   int lane, float* tile, int64_t obase, float esc) {
+  const int rsub = lane >> 3, u4 = lane & 7;
+  float r_row = 1.f;
+  if (KIND == EPI_NORM_BWD) {
+    // s = scale * (the row's partials, summed in order)
+    float s_row = 0.f;
+    r_row = 0.f;
+    if (row_ok) {
+      const float* pp = g.norm_part + int64_t(row) * g.n_npart;
+#pragma unroll 4
+      for (int p = 0; p < g.n_npart; ++p) s_row += pp[p];
+      s_row *= g.norm_scale;
+      r_row = g.norm_r[row];
+    }
+    tile[kStageRowSlot + lane] = r_row * s_row;  // read after the first chunk's __syncwarp
+  }
+  const bool want_part = KIND == EPI_DRELU2 && g.norm_part_out != nullptr;
+  float psum = 0.f;
+#pragma unroll 1
+  for (int c = 0; c < EC / 32; ++c) {
+    uint32_t u[32];
+    tc::tmem_ld_32x32b_x32(taddr + c * 32, u);
+    tc::tmem_wait_ld();
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      float4 v4 = make_float4(u2f(u[4 * k]), u2f(u[4 * k + 1]), u2f(u[4 * k + 2]), u2f(u[4 * k + 3]));
+      if constexpr (SCALED) { v4.x *= esc; v4.y *= esc; v4.z *= esc; v4.w *= esc; }
+      if constexpr (KIND == EPI_NORM_BWD) { v4.x *= r_row; v4.y *= r_row; v4.z *= r_row; v4.w *= r_row; }
+      *stage_at(tile, lane, k) = v4;
+    }
+    __syncwarp();
+    NormRows nrm;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) nrm.part[i] = 0.f;
+    epi_chunk_coalesced<KIND>(g, tile, wrow0, col_base + c * 32 + 4 * u4, rsub, u4, sp, splits, -1, 0.f,
+                              obase, nrm);
+    if (want_part) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float p = nrm.part[i];
+        p += __shfl_xor_sync(0xffffffffu, p, 1);
+        p += __shfl_xor_sync(0xffffffffu, p, 2);
+        p += __shfl_xor_sync(0xffffffffu, p, 4);
+        if (u4 == i) psum += p;
+      }
+    }
+    __syncwarp();
+  }
+  if (want_part && part < g.n_npart) {
+    const int r = wrow0 + 4 * u4 + rsub;
+    if (r < g.M) g.norm_part_out[int64_t(r) * g.n_npart + part] = psum;
   }
 }
 
@@ -487,38 +618,16 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& g, uint32_t taddr,
       }
     }
   } else {
-    // Everything that writes the output element by element: the warp's 32
-    // rows x 32 columns pass through its staging tile, then each lane handles
-    // 4 columns of a row so that a warp instruction covers 4 rows x 32
-    // consecutive columns.
     const int wrow0 = row0 + quarter * 32;
-    const int rsub = lane >> 3, u4 = lane & 7;
-#pragma unroll 1
-    for (int c = 0; c < EC / 32; ++c) {
-      uint32_t u[32];
-      tc::tmem_ld_32x32b_x32(taddr + c * 32, u);
-      tc::tmem_wait_ld();
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        float4 v4 = make_float4(u2f(u[4 * k]), u2f(u[4 * k + 1]), u2f(u[4 * k + 2]), u2f(u[4 * k + 3]));
-        if constexpr (SCALED) { v4.x *= esc; v4.y *= esc; v4.z *= esc; v4.w *= esc; }
-        *stage_at(tile, lane, k) = v4;
-      }
-      __syncwarp();
-      const int col = col_base + c * 32 + 4 * u4;
-      if (splits > 1) {
-        epi_chunk_coalesced<-1>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row, obase);
-      } else {
-        switch (g.epi) {
-          case EPI_RESID_F32: epi_chunk_coalesced<EPI_RESID_F32>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row, obase); break;
-          case EPI_STORE_F32: epi_chunk_coalesced<EPI_STORE_F32>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row, obase); break;
-          case EPI_RELU2: epi_chunk_coalesced<EPI_RELU2>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row, obase); break;
-          case EPI_DRELU2: epi_chunk_coalesced<EPI_DRELU2>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row, obase); break;
-          case EPI_AXPBY: epi_chunk_coalesced<EPI_AXPBY>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row, obase); break;
-          default: epi_chunk_coalesced<EPI_STORE>(g, tile, wrow0, col, rsub, u4, sp, splits, tgt, lse_row, obase); break;
-        }
-      }
-      __syncwarp();
+    switch (splits > 1 ? -1 : int(g.epi)) {
+      case -1: epi_tile_coalesced<-1, SCALED>(g, taddr, row, row_ok, wrow0, col_base, part, sp, splits, lane, tile, obase, esc); break;
+      case EPI_RESID_F32: epi_tile_coalesced<EPI_RESID_F32, SCALED>(g, taddr, row, row_ok, wrow0, col_base, part, sp, splits, lane, tile, obase, esc); break;
+      case EPI_STORE_F32: epi_tile_coalesced<EPI_STORE_F32, SCALED>(g, taddr, row, row_ok, wrow0, col_base, part, sp, splits, lane, tile, obase, esc); break;
+      case EPI_RELU2: epi_tile_coalesced<EPI_RELU2, SCALED>(g, taddr, row, row_ok, wrow0, col_base, part, sp, splits, lane, tile, obase, esc); break;
+      case EPI_DRELU2: epi_tile_coalesced<EPI_DRELU2, SCALED>(g, taddr, row, row_ok, wrow0, col_base, part, sp, splits, lane, tile, obase, esc); break;
+      case EPI_AXPBY: epi_tile_coalesced<EPI_AXPBY, SCALED>(g, taddr, row, row_ok, wrow0, col_base, part, sp, splits, lane, tile, obase, esc); break;
+      case EPI_NORM_BWD: epi_tile_coalesced<EPI_NORM_BWD, SCALED>(g, taddr, row, row_ok, wrow0, col_base, part, sp, splits, lane, tile, obase, esc); break;
+      default: epi_tile_coalesced<EPI_STORE, SCALED>(g, taddr, row, row_ok, wrow0, col_base, part, sp, splits, lane, tile, obase, esc); break;
     }
   }
   if (row_ok && g.epi == EPI_CE_FWD) {
@@ -862,6 +971,9 @@ int launch_gemm_tc(const GemmArgs& g_in, void* stream) {
   GemmArgs g = g_in;
   cudaStream_t st = (cudaStream_t)stream;
   if (g.M <= 0 || g.N <= 0 || g.K <= 0 || g.batch <= 0) return 0;
+  if (g.epi == EPI_NORM_BWD && (!g.aux || !g.out2 || !g.norm_part || !g.norm_r || g.n_npart <= 0))
+    return 1;
+  if (g.norm_part_out && (g.epi != EPI_DRELU2 || g.n_npart < (g.N + EC - 1) / EC)) return 1;
   if (g.fp8) {
     // e4m3 operands: K-major A and B (16-byte aligned rows), one product, the
     // dequantization factors given, no split; not the cross-entropy epilogues

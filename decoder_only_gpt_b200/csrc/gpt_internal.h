@@ -56,6 +56,8 @@ enum Epilogue : int32_t {
   EPI_CE_BWD,       // out_t = (exp(acc - lse[m]) - [n == tgt[m]]) * inv_n; 0 for n >= n_valid
   EPI_QKV,          // [q|k|v] row: RoPE + per-head RMSNorm of q, k; head-major scatter of q, k, v
   EPI_AXPBY,        // out_t = alpha * acc + beta_aux * aux_t   (Newton-Schulz updates)
+  EPI_NORM_BWD,     // RMSNorm backward of the GEMM's output row (see norm_* below):
+                    // out_f32 += r[m] (acc - aux_t * s[m]); out2_t = bf16(out_f32)
 };
 
 struct GemmArgs {
@@ -106,6 +108,20 @@ struct GemmArgs {
   bool fp8 = false;
   const float* a_row_scale = nullptr;
   const float* b_scale = nullptr;
+  // RMSNorm backward folded into GEMM epilogues (tensor-core GEMM, bf16).
+  // EPI_DRELU2 with norm_part_out: also writes, per row m and 128-column
+  // block p of the output, norm_part_out[m * n_npart + p] = sum of acc * aux
+  // over the block's columns (the accumulator before the ReLU^2' factor).
+  // EPI_NORM_BWD: s[m] = norm_scale * sum_p norm_part[m * n_npart + p],
+  // r[m] = norm_r[m]; out is the fp32 gradient it accumulates into, out2
+  // (bf16, leading dim ldo) receives its rounded copy, aux holds the norm's
+  // output h.
+  float* norm_part_out = nullptr;
+  const float* norm_part = nullptr;
+  const float* norm_r = nullptr;
+  void* out2 = nullptr;
+  int n_npart = 0;
+  float norm_scale = 0.f;
   // split-K (tensor-core GEMM, EPI_STORE only): fp32 partials [splits][M][N]
   float* splitk;
   int64_t splitk_floats;    // capacity of `splitk`
@@ -128,6 +144,8 @@ struct Layout {
   uint64_t hf, rf;
   uint64_t qkv_raw;
   uint64_t part_max, part_sum, tgt_logit, lse_z, tok_loss, loss_acc;
+  uint64_t npart;          // [N, n_npart] fp32: the MLP norm's folded-backward row partials
+  int64_t n_npart;
   uint64_t G, dh, du, dO, dqkv, Dattn;
   uint64_t splitk;          // fp32 split-K partials
   int64_t splitk_floats;
