@@ -143,9 +143,10 @@ bool make_layout(const gpt_config& c, Layout* L) {
   L->lse_z = b.take(N * 4);
   L->tok_loss = b.take(N * 4);
   L->loss_acc = b.take(256);
-  // the MLP norm's backward, folded into the down- and up-projection data
-  // gradients (bf16): one fp32 row partial per output column block of >= 64
-  L->n_npart = (F + 63) / 64;
+  // the block norms' backward, folded into the data-gradient GEMMs (bf16): one
+  // fp32 row partial per down-projection dgrad column block of >= 64, or per
+  // attention head (q, k and v heads)
+  L->n_npart = std::max((F + 63) / 64, H + 2 * Hkv);
   L->npart = b.take(c.dtype == GPT_BF16 ? N * L->n_npart * 4 : 0);
   L->G = b.take(N * L->vpad * esz);
   L->dh = b.take(N * d * esz);
@@ -763,16 +764,23 @@ static int backward_impl(const gpt_config* c, const int32_t* tok, const int32_t*
     g = gemm_kk(ws + L.dxs, d, Lb + L.lo.o, d, d, d, N, EPI_STORE, grad(GPT_T_WO, l), d, status);
     g.a_mn_major = true; g.b_mn_major = true; g.beta = accumulate;
     GPT_TRY(run_gemm(*c, with_splitk(g, L, ws), st));
-    // attention, then QK-norm and RoPE backward, into dqkv [N, Q] (Q = qkv columns)
+    // attention, then QK-norm and RoPE backward, into dqkv [N, Q] (Q = qkv columns);
+    // folded: the attention kernels also write the input norm's row partials
+    // (sum_j dh_j h_j = sum_c dqkv_c qkv_c with qkv = h Wqkv^T the raw
+    // projection, per head), and the QKV dgrad's epilogue applies the norm's
+    // backward.  Not with a value embedding in this layer: its v is not the
+    // projection's, and its gate adds to dh after the GEMM.
+    const bool ve = has_value_embed(*c, l);
+    const bool fold_attn = fold && !ve;
     {
       TraceScope ts(GPT_K_ATTN_BWD, c->dtype == GPT_BF16 ? 3 : 2, attn_b, S.nd() * esz * 8, st);
       GPT_TRY(launch_attn_bwd(*c, Lb + L.lo.q, Lb + L.lo.k, Lb + L.lo.v, Lb + L.lo.o, ws + L.dO,
                               reinterpret_cast<float*>(Lb + L.lo.lse),
                               reinterpret_cast<float*>(Lb + L.lo.rq),
                               reinterpret_cast<float*>(Lb + L.lo.rk), S.cos_t, S.sin_t,
-                              S.f(L.Dattn), ws + L.dqkv, S.status, st));
+                              S.f(L.Dattn), ws + L.dqkv, fold_attn ? S.f(L.npart) : nullptr,
+                              S.status, st));
     }
-    const bool ve = has_value_embed(*c, l);
     if (ve) {  // the value embedding's table and gate gradients from dv
       TraceScope ts(GPT_K_OTHER, 2, 0, double(N) * c->n_kv_head * c->head_dim * (esz * 2 + 4), st);
       GPT_TRY(launch_ve_bwd(*c, ws + L.dqkv, Lb + L.lo.h1, S.param(GPT_T_VE_GATE, l), S.param(GPT_T_VE, l),
@@ -783,9 +791,15 @@ static int backward_impl(const gpt_config* c, const int32_t* tok, const int32_t*
       GPT_TRY(launch_embed_scatter(cv, L, S.f(L.ve_rows), ws, grad(GPT_T_VE, l), accumulate, st));
     }
     const int Qc = int(qkv_cols(*c));
-    g = gemm_kk(ws + L.dqkv, Qc, S.param(GPT_T_WQKV, l), d, N, d, Qc, EPI_STORE, ws + L.dh,
+    float* r1 = reinterpret_cast<float*>(Lb + L.lo.r1);
+    g = gemm_kk(ws + L.dqkv, Qc, S.param(GPT_T_WQKV, l), d, N, d, Qc,
+                fold_attn ? EPI_NORM_BWD : EPI_STORE, fold_attn ? static_cast<void*>(S.x) : ws + L.dh,
                 d, status);
     g.b_mn_major = true;
+    if (fold_attn) {
+      g.aux = Lb + L.lo.h1; g.out2 = ws + L.dxs; g.norm_part = S.f(L.npart); g.norm_r = r1;
+      g.n_npart = c->n_head + 2 * c->n_kv_head; g.norm_scale = 1.f / float(d);
+    }
     GPT_TRY(S.dgrad(g, GPT_T_WQKV, l));
     if (ve) {  // the gate's input h[:, :C]
       TraceScope ts(GPT_K_OTHER, 1, 0, double(N) * c->ve_gate_channels * esz * 2, st);
@@ -796,7 +810,7 @@ static int backward_impl(const gpt_config* c, const int32_t* tok, const int32_t*
     g.a_mn_major = true; g.b_mn_major = true; g.beta = accumulate;
     GPT_TRY(run_gemm(*c, with_splitk(g, L, ws), st));
     GPT_TRY(cuda_rc(cudaError_t(mark(1 + l))));  // every weight gradient of layer l is final
-    GPT_TRY(S.rms_bwd(ws + L.dh, Lb + L.lo.h1, reinterpret_cast<float*>(Lb + L.lo.r1), 1));
+    if (!fold_attn) GPT_TRY(S.rms_bwd(ws + L.dh, Lb + L.lo.h1, r1, 1));
     const bool bo = c->backout && l == backout_layer(*c);
     if (bo || c->resid_lambdas) {  // the layer's entry: backout point, residual scaling
       TraceScope ts(GPT_K_OTHER, c->resid_lambdas ? 2 : 1, 0, S.nd() * (c->resid_lambdas ? 26.0 : 14.0), st);

@@ -746,8 +746,20 @@ __device__ __forceinline__ void load_rope_tiles(uint8_t* cos_dst, uint8_t* sin_d
     tc::tma_load_2d(sin_dst + c * (128 * 128), map_sin, bar, c * 32, pos0);
   }
 }
+// One head's share of the row sum sum_c dqkv_c * qkv_c that the backward of
+// the norm in front of the QKV projection needs (qkv = the projection's raw
+// output).  RoPE is a rotation, so the share of q (or k) is g . x with x the
+// rotated raw head and g the gradient reaching it; without QK-norm x is the
+// stored head y and the share is g . y = gy.  With QK-norm (y = x r,
+// r = 1 / sqrt(mean(x^2) + eps)), g = r (dy - y mean(dy y)) gives
+// g . x = sum(dy y) (1 - mean(y^2)) = gy eps r^2: the norm's gradient is
+// almost orthogonal to its input.
+__device__ __forceinline__ float norm_row_part(float gy, float rr, int qk_norm, float eps) {
+  return qk_norm ? gy * eps * rr * rr : gy;
+}
+
 template <int HD>
-__device__ __forceinline__ void norm_rope_bwd_half(uint32_t taddr, int half, int r, float scale,
+__device__ __forceinline__ float norm_rope_bwd_half(uint32_t taddr, int half, int r, float scale,
                                                    const uint8_t* y_tile, float rr, int qk_norm,
                                                    const uint8_t* cos_tile, const uint8_t* sin_tile,
                                                    uint8_t* out_tile, bool ok, bool write, float* red) {
@@ -783,8 +795,9 @@ __device__ __forceinline__ void norm_rope_bwd_half(uint32_t taddr, int half, int
   }
   red[half * 128 + r] = part;
   compute_bar();
-  const float mean_gy = (red[r] + red[128 + r]) / float(HD);
-  if (!ok || !write) return;
+  const float sum_gy = red[r] + red[128 + r];
+  const float mean_gy = sum_gy / float(HD);
+  if (!ok || !write) return sum_gy;
   uint32_t pa[Q4 / 2], pb[Q4 / 2];
 #pragma unroll
   for (int i = 0; i < Q4; i += 4) {  // 4 fp32 per 16-byte unit
@@ -811,6 +824,7 @@ __device__ __forceinline__ void norm_rope_bwd_half(uint32_t taddr, int half, int
     *reinterpret_cast<uint4*>(out_tile + tile_unit(r, (HALF + i0 + 2 * i) / 8)) =
         make_uint4(pb[i], pb[i + 1], pb[i + 2], pb[i + 3]);
   }
+  return sum_gy;
 }
 
 // After every compute thread has written its rows of the output tiles: fence,
@@ -932,7 +946,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap map_out,
                       const float* __restrict__ lse,
                       const float* __restrict__ D, const float* __restrict__ rq, int H, int Hkv, int T,
-                      int W, float scale, float scale_log2, int qk_norm, int32_t* status) {
+                      int W, float scale, float scale_log2, int qk_norm, float eps,
+                      float* __restrict__ npart, int np_stride, int32_t* status) {
   using S = DqSmem<HD>;
   constexpr int NCH = HD / 64;
   constexpr uint32_t CH = 128 * 128;  // bytes of one 64-column chunk of a 128-row tile
@@ -1163,9 +1178,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
       tc::tc_fence_after();
     }
-    norm_rope_bwd_half<HD>(t_dq + R.lane_off, R.half, R.r, scale, smem + S::Y_OFF,
-                           qv ? rq[int64_t(bh) * T + q] : 0.f, qk_norm, smem + S::COS_OFF, smem + S::SIN_OFF,
-                           smem + S::OUT_OFF, ok, qv, reinterpret_cast<float*>(smem + S::RED_OFF));
+    const float rrq = qv ? rq[int64_t(bh) * T + q] : 0.f;
+    const float gy = norm_rope_bwd_half<HD>(t_dq + R.lane_off, R.half, R.r, scale, smem + S::Y_OFF, rrq,
+                                            qk_norm, smem + S::COS_OFF, smem + S::SIN_OFF,
+                                            smem + S::OUT_OFF, ok, qv,
+                                            reinterpret_cast<float*>(smem + S::RED_OFF));
+    if (npart && ok && qv && R.half == 0)  // this head's share of the input norm's row sum
+      npart[(int64_t(b) * T + q) * np_stride + h] = norm_row_part(gy, rrq, qk_norm, eps);
     uint8_t* const tiles[1] = {smem + S::OUT_OFF};
     const int cols[1] = {h * HD};
     store_tiles<HD>(&map_out, tiles, cols, 1, q0, b, ok);
@@ -1186,6 +1205,8 @@ struct DkvSmem {
   static constexpr uint32_t RED_OFF = STAT_OFF;  // epilogue only, after the last step's stats
   // epilogue only, once no product reads the Q ring: the dV and dK tiles
   static constexpr uint32_t DV_OFF = Q_OFF, DK_OFF = Q_OFF + TILE;
+  static constexpr uint32_t VRED_OFF = Q_OFF + 2 * TILE;  // epilogue only: 2 x 128 floats
+  static_assert(kDkvRingQ >= 3, "the epilogue's dv . v exchange uses the third Q slot");
   static constexpr uint32_t BAR_OFF = STAT_OFF + 2 * 128 * 4;
   static constexpr uint32_t BYTES = BAR_OFF + 256 + 1024;
   static_assert(TILE % 1024 == 0 && BYTES <= 232448, "");
@@ -1228,7 +1249,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                        const __grid_constant__ CUtensorMap map_out,
                        const float* __restrict__ lse,
                        const float* __restrict__ D, const float* __restrict__ rk, int H, int Hkv, int T,
-                       int W, float scale, float scale_log2, int qk_norm, int32_t* status) {
+                       int W, float scale, float scale_log2, int qk_norm, float eps,
+                       float* __restrict__ npart, int np_stride, int32_t* status) {
   using S = DkvSmem<HD>;
   constexpr int NCH = HD / 64;
   constexpr uint32_t CH = 128 * 128;  // bytes of one 64-column chunk of a 128-row tile
@@ -1521,28 +1543,50 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tc_fence_after();
     }
     const int d = H * HD;
+    float vdot = 0.f;  // this half's sum dv . v (the input norm's row sum, when asked for)
     if (ok) {  // dV: this thread's half of the columns, into the dV tile
 #pragma unroll
       for (int c = 0; c < HD / 2; c += 32) {
         float v[32];
         tmem_ld<32>(t_dv + R.lane_off + R.half * (HD / 2) + c, v);
 #pragma unroll
-        for (int i = 0; i < 32; i += 8)
-          *reinterpret_cast<uint4*>(smem + S::DV_OFF + tile_unit(R.r, (R.half * (HD / 2) + c + i) / 8)) =
+        for (int i = 0; i < 32; i += 8) {
+          const int unit = (R.half * (HD / 2) + c + i) / 8;
+          *reinterpret_cast<uint4*>(smem + S::DV_OFF + tile_unit(R.r, unit)) =
               make_uint4(pack2(v[i], v[i + 1]), pack2(v[i + 2], v[i + 3]), pack2(v[i + 4], v[i + 5]),
                          pack2(v[i + 6], v[i + 7]));
+          if (npart) {
+            const uint4 w = *reinterpret_cast<const uint4*>(smem + S::V_OFF + tile_unit(R.r, unit));
+            const uint32_t wu[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wu[e]));
+              vdot = fmaf(v[i + 2 * e], f.x, fmaf(v[i + 2 * e + 1], f.y, vdot));
+            }
+          }
+        }
       }
     }
+    // the two halves' dv . v meet in the Q ring's third slot (free in the
+    // epilogue), ordered by the norm backward's barrier below
+    float* vred = reinterpret_cast<float*>(smem + S::VRED_OFF);
+    vred[R.half * 128 + R.r] = vdot;
     if (ok && !__all_sync(0xffffffffu, tc::mbar_wait_spin(&bars->epi_full, 0, abort, kWaitNs))) {
       if (R.lane == 0) record_status(status, GPT_ETIMEOUT, K_ATTN, 36);
       *abort = 1;
       ok = false;
     }
     // the stats region is free once every step is done (acc_full): it holds red
-    norm_rope_bwd_half<HD>(t_dk + R.lane_off, R.half, R.r, scale, smem + S::K_OFF,
-                           kv ? rk[int64_t(bkv) * T + key] : 0.f, qk_norm, smem + S::COS_OFF,
-                           smem + S::SIN_OFF, smem + S::DK_OFF, ok, kv,
-                           reinterpret_cast<float*>(smem + S::RED_OFF));
+    const float rrk = kv ? rk[int64_t(bkv) * T + key] : 0.f;
+    const float gy = norm_rope_bwd_half<HD>(t_dk + R.lane_off, R.half, R.r, scale, smem + S::K_OFF, rrk,
+                                            qk_norm, smem + S::COS_OFF, smem + S::SIN_OFF,
+                                            smem + S::DK_OFF, ok, kv,
+                                            reinterpret_cast<float*>(smem + S::RED_OFF));
+    if (npart && ok && kv && R.half == 0) {  // this k head's and v head's shares
+      float* pr = npart + (int64_t(b) * T + key) * np_stride + H;
+      pr[hk] = norm_row_part(gy, rrk, qk_norm, eps);
+      pr[Hkv + hk] = vred[R.r] + vred[128 + R.r];
+    }
     uint8_t* const tiles[2] = {smem + S::DV_OFF, smem + S::DK_OFF};
     const int cols[2] = {d + (Hkv + hk) * HD, d + hk * HD};
     store_tiles<HD>(&map_out, tiles, cols, 2, k0, b, ok);
@@ -1554,9 +1598,10 @@ namespace {
 template <int HD>
 int attn_bwd_tc_t(const gpt_config& c, const void* q, const void* k, const void* v, const void* o,
                   const void* dO, const float* lse, const float* rq, const float* rk,
-                  const float* cos_t, const float* sin_t, float* Dbuf, void* dqkv,
+                  const float* cos_t, const float* sin_t, float* Dbuf, void* dqkv, float* npart,
                   int32_t* status, cudaStream_t st) {
   const int H = c.n_head, Hkv = c.n_kv_head, T = c.seq_len, B = c.batch, d = H * HD;
+  const int np_stride = H + 2 * Hkv;
   const int W = window_span(c);
   const int64_t ldq = qkv_cols(c);
   const uint64_t rows = uint64_t(B) * H * T, kv_rows = uint64_t(B) * Hkv * T, ntok = uint64_t(B) * T;
@@ -1577,13 +1622,15 @@ int attn_bwd_tc_t(const gpt_config& c, const void* q, const void* k, const void*
   if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_q) != cudaSuccess)
     return 1;
   kq<<<nt * B * H, kThreads, smem_q, st>>>(q128, do128, k128, v128, mcos, msin, mout, lse, Dbuf, rq, H,
-                                           Hkv, T, W, scale, scale_log2, c.qk_norm, status);
+                                           Hkv, T, W, scale, scale_log2, c.qk_norm, c.norm_eps, npart,
+                                           np_stride, status);
   auto kk = attn_dkv_tc_kernel<HD>;
   const int smem_k = int(DkvSmem<HD>::BYTES);
   if (cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_k) != cudaSuccess)
     return 1;
   kk<<<nt * B * Hkv, kThreads, smem_k, st>>>(k128, v128, q128, do128, mcos, msin, mout, lse, Dbuf, rk, H,
-                                                Hkv, T, W, scale, scale_log2, c.qk_norm, status);
+                                                Hkv, T, W, scale, scale_log2, c.qk_norm, c.norm_eps, npart,
+                                                np_stride, status);
   return last_launch_rc();
 }
 }  // namespace
@@ -1591,11 +1638,11 @@ int attn_bwd_tc_t(const gpt_config& c, const void* q, const void* k, const void*
 int launch_attn_bwd_tc(const gpt_config& c, const void* q, const void* k, const void* v,
                        const void* o, const void* dO, const float* lse, const float* rq,
                        const float* rk, const float* cos_t, const float* sin_t, float* Dbuf,
-                       void* dqkv, int32_t* status, void* stream) {
+                       void* dqkv, float* norm_part, int32_t* status, void* stream) {
   cudaStream_t st = (cudaStream_t)stream;
   return c.head_dim == 128
-             ? attn_bwd_tc_t<128>(c, q, k, v, o, dO, lse, rq, rk, cos_t, sin_t, Dbuf, dqkv, status, st)
-             : attn_bwd_tc_t<64>(c, q, k, v, o, dO, lse, rq, rk, cos_t, sin_t, Dbuf, dqkv, status, st);
+             ? attn_bwd_tc_t<128>(c, q, k, v, o, dO, lse, rq, rk, cos_t, sin_t, Dbuf, dqkv, norm_part, status, st)
+             : attn_bwd_tc_t<64>(c, q, k, v, o, dO, lse, rq, rk, cos_t, sin_t, Dbuf, dqkv, norm_part, status, st);
 }
 
 }  // namespace gpt

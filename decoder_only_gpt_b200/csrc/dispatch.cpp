@@ -21,7 +21,7 @@ int launch_attn_bwd_simt(const gpt_config& c, const void* q, const void* k, cons
 int launch_attn_bwd_tc(const gpt_config& c, const void* q, const void* k, const void* v,
                        const void* o, const void* dO, const float* lse, const float* rq,
                        const float* rk, const float* cos_t, const float* sin_t, float* Dbuf,
-                       void* dqkv, int32_t* status, void* stream);
+                       void* dqkv, float* norm_part, int32_t* status, void* stream);
 
 int launch_gemm(const gpt_config& c, const GemmArgs& g, void* stream) {
   return c.dtype == GPT_BF16 ? launch_gemm_tc(g, stream) : launch_gemm_simt_f32(g, stream);
@@ -44,10 +44,11 @@ int launch_attn_fwd(const gpt_config& c, const void* q, const void* k, const voi
 int launch_attn_bwd(const gpt_config& c, const void* q, const void* k, const void* v,
                     const void* o, const void* dO, const float* lse, const float* rq,
                     const float* rk, const float* cos_t, const float* sin_t, float* Dbuf,
-                    void* dqkv, int32_t* status, void* stream) {
+                    void* dqkv, float* norm_part, int32_t* status, void* stream) {
+  if (c.dtype != GPT_BF16 && norm_part) return 1;  // the row partials are a tensor-core output
   return c.dtype == GPT_BF16
-             ? launch_attn_bwd_tc(c, q, k, v, o, dO, lse, rq, rk, cos_t, sin_t, Dbuf, dqkv, status,
-                                  stream)
+             ? launch_attn_bwd_tc(c, q, k, v, o, dO, lse, rq, rk, cos_t, sin_t, Dbuf, dqkv, norm_part,
+                                  status, stream)
              : launch_attn_bwd_simt(c, q, k, v, o, dO, lse, rq, rk, cos_t, sin_t, Dbuf, dqkv,
                                     stream);
 }

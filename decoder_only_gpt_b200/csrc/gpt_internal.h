@@ -144,7 +144,7 @@ struct Layout {
   uint64_t hf, rf;
   uint64_t qkv_raw;
   uint64_t part_max, part_sum, tgt_logit, lse_z, tok_loss, loss_acc;
-  uint64_t npart;          // [N, n_npart] fp32: the MLP norm's folded-backward row partials
+  uint64_t npart;          // [N, n_npart] fp32: the folded norm backwards' row partials
   int64_t n_npart;
   uint64_t G, dh, du, dO, dqkv, Dattn;
   uint64_t splitk;          // fp32 split-K partials
@@ -222,10 +222,13 @@ int launch_loss_mean(const gpt_config& c, const float* tok_loss, float* loss,
                      float* user_tok_loss, int32_t* status, void* stream);
 int launch_attn_fwd(const gpt_config& c, const void* q, const void* k, const void* v, void* o,
                     float* lse, int32_t* status, void* stream);
+// norm_part (bf16 only, or null): per token b*T + t, row stride H + 2*Hkv,
+// each q head's, then k head's, then v head's share of sum_c dqkv_c * qkv_c,
+// qkv the QKV projection's raw output (for the backward of the norm before it)
 int launch_attn_bwd(const gpt_config& c, const void* q, const void* k, const void* v,
                     const void* o, const void* dO, const float* lse, const float* rq,
                     const float* rk, const float* cos_t, const float* sin_t, float* Dbuf,
-                    void* dqkv, int32_t* status, void* stream);
+                    void* dqkv, float* norm_part, int32_t* status, void* stream);
 int launch_sort_tokens(const gpt_config& c, const Layout& L, const int32_t* tok, char* ws,
                        void* stream);
 int launch_embed_scatter(const gpt_config& c, const Layout& L, const float* dx0, char* ws,
