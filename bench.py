@@ -239,7 +239,7 @@ def gemm_sites(records, w, steps):
 # site, from an ncu capture of the current kernel build, keyed by (workload,
 # site, fp8); a site that has not been captured reports null.
 TRAFFIC_BYTES = {
-    ("d24", 32768, 6144, 1536, False): 120_946_432 + 361_932_032,  # ncu: 482.9 MB per launch
+    ("d24", 32768, 6144, 1536, False): 121_198_336 + 361_594_624,  # ncu: 482.8 MB per launch
     ("d24", 32768, 6144, 1536, True): 60_106_752 + 351_310_080,    # e4m3 operands: 411.4 MB
 }
 
