@@ -240,7 +240,7 @@ def gemm_sites(records, w, steps):
 # site, fp8); a site that has not been captured reports null.
 TRAFFIC_BYTES = {
     ("d24", 32768, 6144, 1536, False): 121_198_336 + 361_594_624,  # ncu: 482.8 MB per launch
-    ("d24", 32768, 6144, 1536, True): 60_106_752 + 351_310_080,    # e4m3 operands: 411.4 MB
+    ("d24", 32768, 6144, 1536, True): 60_164_608 + 351_863_808,    # e4m3 operands: 412.0 MB
 }
 
 
@@ -274,7 +274,7 @@ def roofline(sites, w, gemm_tf, peak_tf, peaks):
                                                      + 2 * w.batch * w.seq_len * w.d_ff,
                      "traffic": TRAFFIC_BYTES.get(key)})
     else:
-        line.update({"achieved": round(gemm_tf, 1), "frac": round(gemm_tf / peak_tf, 4), "traffic": None})
+        line.update({"achieved": round(gemm_tf, 1), "frac": round(gemm_tf / site_peak, 4), "traffic": None})
     return line
 
 
@@ -417,7 +417,7 @@ def measure(w, args, rank, world, dev, barrier, *, optimizer=False, e2e=True):
         eager_ms = e0.elapsed_time(e1)
 
     # ---- the same steps again with every launch timed (breakdown only) ----
-    per_step = 600
+    per_step = 1200  # trace records per step: ~500 launches, ~650 with the FP8 quantizers
     trace = B.Trace(capacity=per_step * args.steps + 16)
     barrier()
     torch.cuda.synchronize()

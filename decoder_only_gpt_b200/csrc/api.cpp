@@ -773,7 +773,7 @@ static int backward_impl(const gpt_config* c, const int32_t* tok, const int32_t*
     const bool ve = has_value_embed(*c, l);
     const bool fold_attn = fold && !ve;
     {
-      TraceScope ts(GPT_K_ATTN_BWD, c->dtype == GPT_BF16 ? 3 : 2, attn_b, S.nd() * esz * 8, st);
+      TraceScope ts(GPT_K_ATTN_BWD, 2, attn_b, S.nd() * esz * 8, st);
       GPT_TRY(launch_attn_bwd(*c, Lb + L.lo.q, Lb + L.lo.k, Lb + L.lo.v, Lb + L.lo.o, ws + L.dO,
                               reinterpret_cast<float*>(Lb + L.lo.lse),
                               reinterpret_cast<float*>(Lb + L.lo.rq),

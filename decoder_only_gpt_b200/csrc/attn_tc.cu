@@ -675,42 +675,14 @@ int launch_attn_fwd_tc(const gpt_config& c, const void* q, const void* k, const 
 //   dQ_i  = sum_j dS_ij k_j / sqrt(hd)      (attn_dq_tc: CTA = 128 queries)
 //   dK_j  = sum_i dS_ij q_i / sqrt(hd)      (attn_dkv_tc: CTA = 128 keys)
 //   dV_j  = sum_i P_ij dO_i
-// Each kernel owns its outputs, so no sum needs atomics (deterministic).  The
+// The dQ kernel forms D_i (its dO tile is in shared memory) and writes it for
+// the dK/dV kernel, which runs after it on the same stream.  Each kernel owns
+// its outputs, so no sum needs atomics (deterministic).  The
 // gradients of q and k then go back through the per-head RMSNorm,
 // dx = r (g - y mean(g y)), and the transposed RoPE rotation, and land in the
 // [q | k | v] gradient rows [B*T, 3*H*hd].
 // ===========================================================================
 namespace {
-
-// D_i = dO_i . o_i: 8 elements (16 bytes of each operand) per thread, hd/8
-// consecutive threads per (token, head) row, reduced by shuffles in that group
-__global__ void attn_rowdot_kernel(const __nv_bfloat16* __restrict__ dO,
-                                   const __nv_bfloat16* __restrict__ o, float* __restrict__ D,
-                                   int64_t N, int H, int T, int hd) {
-  const int G = hd / 8;  // 8 or 16: groups never straddle a warp
-  const int64_t gid = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t rowi = gid / G;  // token * H + head
-  const int part = int(gid % G);
-  const bool ok = rowi < N * H;
-  float s = 0.f;
-  if (ok) {
-    const uint4 a = *reinterpret_cast<const uint4*>(dO + rowi * hd + part * 8);
-    const uint4 b = *reinterpret_cast<const uint4*>(o + rowi * hd + part * 8);
-    const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wa[e]));
-      const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wb[e]));
-      s += x.x * y.x + x.y * y.y;
-    }
-  }
-  for (int off = G / 2; off >= 1; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  if (ok && part == 0) {
-    const int64_t n = rowi / H, bb = n / T, t = n % T;
-    const int h = int(rowi % H);
-    D[(bb * H + h) * T + t] = s;
-  }
-}
 
 // slots of the dK/dV kernel's Q and dO rings (a Q tile is read by S^T_j and,
 // after the threads have formed dS^T_j, by dK_j)
@@ -907,7 +879,8 @@ struct DqSmem {
   // the RoPE tiles of the epilogue, loaded into the V ring once the last dP is done
   static constexpr uint32_t COS_OFF = V_OFF, SIN_OFF = V_OFF + TILE;
   static constexpr uint32_t BAR_OFF = V_OFF + kDqRingV * TILE;
-  static constexpr uint32_t BYTES = BAR_OFF + 256 + 1024;
+  static constexpr uint32_t DRED_OFF = BAR_OFF + 256;  // the halves of D: 2 x 128 floats
+  static constexpr uint32_t BYTES = DRED_OFF + 1024 + 1024;
   static_assert(TILE % 1024 == 0 && BYTES <= 232448, "");
 };
 struct DqBars {
@@ -944,8 +917,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap map_cos,
                       const __grid_constant__ CUtensorMap map_sin,
                       const __grid_constant__ CUtensorMap map_out,
-                      const float* __restrict__ lse,
-                      const float* __restrict__ D, const float* __restrict__ rq, int H, int Hkv, int T,
+                      const __nv_bfloat16* __restrict__ o, const float* __restrict__ lse,
+                      float* __restrict__ D, const float* __restrict__ rq, int H, int Hkv, int T,
                       int W, float scale, float scale_log2, int qk_norm, float eps,
                       float* __restrict__ npart, int np_stride, int32_t* status) {
   using S = DqSmem<HD>;
@@ -1128,8 +1101,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the query's visible keys [k_lo, k_hi): none for a row past T
     const int k_lo = q - W + 1, k_hi = qv ? q + 1 : k_lo;
     const float lse2 = qv ? lse[int64_t(bh) * T + q] * kLog2e : 0.f;
-    const float Dq = qv ? D[int64_t(bh) * T + q] : 0.f;
-    bool ok = true;
+    // D = rowsum(dO o) of this query: each half of the row's columns from the
+    // dO tile in shared memory and o in global memory, the halves added in
+    // shared memory; written out for the dK/dV kernel
+    bool ok = __all_sync(0xffffffffu, tc::mbar_wait_spin(&bars->fixed_full, 0, abort, kWaitNs));
+    float dpart = 0.f;
+    if (ok && qv) {
+      const uint4* orow = reinterpret_cast<const uint4*>(o + (int64_t(b) * T + q) * (int64_t(H) * HD) + h * HD +
+                                                         R.half * (HD / 2));
+#pragma unroll
+      for (int u = 0; u < HD / 16; ++u) {
+        const uint4 a = *reinterpret_cast<const uint4*>(smem + S::DO_OFF + tile_unit(R.r, R.half * (HD / 16) + u));
+        const uint4 c = __ldg(orow + u);
+        const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wc[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wa[e]));
+          const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wc[e]));
+          dpart = fmaf(x.x, y.x, fmaf(x.y, y.y, dpart));
+        }
+      }
+    }
+    float* dred = reinterpret_cast<float*>(smem + S::DRED_OFF);
+    dred[R.half * 128 + R.r] = dpart;
+    compute_bar();
+    const float Dq = dred[R.r] + dred[128 + R.r];
+    if (ok && qv && R.half == 0) D[int64_t(bh) * T + q] = Dq;
+    if (!ok && R.lane == 0) {
+      record_status(status, GPT_ETIMEOUT, K_ATTN, 25);
+      *abort = 1;
+    }
     for (int j = 0; j < n_steps; ++j) {
       const int sb = j & 1;
       if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait_spin(&bars->s_full[sb], (j >> 1) & 1, abort, kWaitNs));
@@ -1605,9 +1606,6 @@ int attn_bwd_tc_t(const gpt_config& c, const void* q, const void* k, const void*
   const int W = window_span(c);
   const int64_t ldq = qkv_cols(c);
   const uint64_t rows = uint64_t(B) * H * T, kv_rows = uint64_t(B) * Hkv * T, ntok = uint64_t(B) * T;
-  const int64_t N = int64_t(B) * T;
-  attn_rowdot_kernel<<<ceil_div(N * H * (HD / 8), 256), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(dO), static_cast<const __nv_bfloat16*>(o), Dbuf, N, H, T, HD);
   CUtensorMap k128, v128, q128, do128, mcos, msin, mout;
   const bool ok = tile_map(&k128, k, kv_rows, HD, HD, 128) && tile_map(&v128, v, kv_rows, HD, HD, 128) &&
                   tile_map(&q128, q, rows, HD, HD, 128) && tile_map(&do128, dO, ntok, d, d, 128) &&
@@ -1621,7 +1619,8 @@ int attn_bwd_tc_t(const gpt_config& c, const void* q, const void* k, const void*
   const int smem_q = int(DqSmem<HD>::BYTES);
   if (cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_q) != cudaSuccess)
     return 1;
-  kq<<<nt * B * H, kThreads, smem_q, st>>>(q128, do128, k128, v128, mcos, msin, mout, lse, Dbuf, rq, H,
+  kq<<<nt * B * H, kThreads, smem_q, st>>>(q128, do128, k128, v128, mcos, msin, mout,
+                                           static_cast<const __nv_bfloat16*>(o), lse, Dbuf, rq, H,
                                            Hkv, T, W, scale, scale_log2, c.qk_norm, c.norm_eps, npart,
                                            np_stride, status);
   auto kk = attn_dkv_tc_kernel<HD>;

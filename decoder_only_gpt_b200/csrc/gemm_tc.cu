@@ -52,6 +52,9 @@ __device__ __forceinline__ float sqrt_approx(float x) {
 __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
 
 // Ask L2 for the bytes this thread's epilogue will read for one tile row
 // (columns col0 .. col0 + EC): the stored activation (ReLU^2'), the fp32 residual
@@ -542,8 +545,16 @@ __device__ __forceinline__ void epi_tile_coalesced(const GemmArgs& g, uint32_t t
   }
   const bool want_part = KIND == EPI_DRELU2 && g.norm_part_out != nullptr;
   float psum = 0.f;
+  // EPI_DRELU2: the stored activation of chunk c + 1 is prefetched into L1
+  // while chunk c is processed (lane l: row l's 64 bytes of the chunk), so
+  // the chunk's loads hit L1 instead of waiting on L2
+  const __nv_bfloat16* l1_row =
+      KIND == EPI_DRELU2 && row_ok ? static_cast<const __nv_bfloat16*>(g.aux) + obase + int64_t(row) * g.ldo
+                                   : nullptr;
+  if (l1_row && col_base < g.N) prefetch_l1(l1_row + col_base);
 #pragma unroll 1
   for (int c = 0; c < EC / 32; ++c) {
+    if (l1_row && c + 1 < EC / 32 && col_base + (c + 1) * 32 < g.N) prefetch_l1(l1_row + col_base + (c + 1) * 32);
     uint32_t u[32];
     tc::tmem_ld_32x32b_x32(taddr + c * 32, u);
     tc::tmem_wait_ld();
