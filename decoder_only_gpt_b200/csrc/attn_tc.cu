@@ -1102,17 +1102,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int k_lo = q - W + 1, k_hi = qv ? q + 1 : k_lo;
     const float lse2 = qv ? lse[int64_t(bh) * T + q] * kLog2e : 0.f;
     // D = rowsum(dO o) of this query: each half of the row's columns from the
-    // dO tile in shared memory and o in global memory, the halves added in
-    // shared memory; written out for the dK/dV kernel
-    bool ok = __all_sync(0xffffffffu, tc::mbar_wait_spin(&bars->fixed_full, 0, abort, kWaitNs));
-    float dpart = 0.f;
-    if (ok && qv) {
+    // dO tile in shared memory and o in global memory (loaded while the tile
+    // is on its way), the halves added in shared memory; written out for the
+    // dK/dV kernel
+    uint4 ov[HD / 16];
+    if (qv) {
       const uint4* orow = reinterpret_cast<const uint4*>(o + (int64_t(b) * T + q) * (int64_t(H) * HD) + h * HD +
                                                          R.half * (HD / 2));
 #pragma unroll
+      for (int u = 0; u < HD / 16; ++u) ov[u] = __ldg(orow + u);
+    }
+    bool ok = __all_sync(0xffffffffu, tc::mbar_wait_spin(&bars->fixed_full, 0, abort, kWaitNs));
+    float dpart = 0.f;
+    if (ok && qv) {
+#pragma unroll
       for (int u = 0; u < HD / 16; ++u) {
         const uint4 a = *reinterpret_cast<const uint4*>(smem + S::DO_OFF + tile_unit(R.r, R.half * (HD / 16) + u));
-        const uint4 c = __ldg(orow + u);
+        const uint4 c = ov[u];
         const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wc[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
