@@ -522,8 +522,9 @@ __device__ __forceinline__ void epi_chunk_coalesced(const GemmArgs& g, float* ti
 // columns pass through its staging tile, then each lane handles 4 columns of
 // a row so that a warp instruction covers 4 rows x 32 consecutive columns.
 // EPI_NORM_BWD: the thread stages r acc for its row and leaves r s in its
-// row slot of the staging tile.  EPI_DRELU2 with norm_part_out: each chunk's lane partials reduced
-// over the row's 8 lanes, lane u4 keeping row 4 u4 + rsub's running sum.
+// row slot of the staging tile.  EPI_DRELU2 with norm_part_out: each chunk's
+// lane partials reduced over the row's 8 lanes, lane u4 keeping row
+// 4 u4 + rsub's running sum.
 template <int KIND, bool SCALED>
 __device__ __forceinline__ void epi_tile_coalesced(const GemmArgs& g, uint32_t taddr, int row, bool row_ok,
                                                    int wrow0, int col_base, int part, int sp, int splits,
@@ -554,7 +555,8 @@ __device__ __forceinline__ void epi_tile_coalesced(const GemmArgs& g, uint32_t t
   if (l1_row && col_base < g.N) prefetch_l1(l1_row + col_base);
 #pragma unroll 1
   for (int c = 0; c < EC / 32; ++c) {
-    if (l1_row && c + 1 < EC / 32 && col_base + (c + 1) * 32 < g.N) prefetch_l1(l1_row + col_base + (c + 1) * 32);
+    if (l1_row && c + 1 < EC / 32 && col_base + (c + 1) * 32 < g.N)
+      prefetch_l1(l1_row + col_base + (c + 1) * 32);
     uint32_t u[32];
     tc::tmem_ld_32x32b_x32(taddr + c * 32, u);
     tc::tmem_wait_ld();
